@@ -1,0 +1,146 @@
+"""Float64 CPU oracle for the differential-attention forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the package's smoke check and the
+benchmark's CPU-baseline leg may import this module.  It shares no code with
+the CUDA path (different language, different build, no common helpers) and the
+CUDA path never calls it.
+
+The arithmetic lives in ``diffattn_oracle.c`` (plain loops, float64, no tiling,
+no online softmax); this module only marshals NumPy arrays.  What it computes:
+
+    Y = Norm( softmax(s Q1 K1^T) V - lambda * softmax(s Q2 K2^T) V )
+
+per batch, signal head and query row, with causal masking (diagonal included),
+the noise map of signal head h taken from noise head h // g, and Norm the
+per-head RMS normalisation with gain (Motif 2.6B explainer, section
+"Differential attention" and figure 1; Motif 3 summary, section 2.2).
+
+Pins (tests/test_oracle_pins.py): lambda = 0 against torch's scaled-dot-product
+attention plus torch's rms_norm; map 2 against the same library routine; the
+Q2=Q1, K2=K1 reduction; softmax rows summing to one; causal independence;
+SciPy-softmax brute force for N <= 8; the row-0 closed form; exact scale
+invariance; the grouped head map against repeat_interleave; decode against the
+last prefill row; a hand-derived golden example.  Parity unpinned: the choice of
+RMS normalisation for the pages' "GroupNorm" and the grouped V layout are
+readings of the pages, not facts the pages fix.
+"""
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+
+def load(path):
+    """Load an oracle shared library from ``path`` and declare its signatures."""
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    ip = ctypes.POINTER(ctypes.c_int64)
+    i64 = ctypes.c_int64
+    lib.diffattn_oracle_prefill.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, i64,
+                                            i64, i64, dp, dp, ctypes.c_double,
+                                            ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                            ip, i64, dp]
+    lib.diffattn_oracle_prefill.restype = ctypes.c_int
+    lib.diffattn_oracle_decode.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, i64,
+                                           ip, dp, dp, ctypes.c_double, ctypes.c_double,
+                                           ctypes.c_int, dp]
+    lib.diffattn_oracle_decode.restype = ctypes.c_int
+    lib.diffattn_oracle_softmax_row.argtypes = [dp, dp, i64, i64, ctypes.c_double, dp]
+    lib.diffattn_oracle_softmax_row.restype = None
+    lib.diffattn_oracle_threads.argtypes = []
+    lib.diffattn_oracle_threads.restype = ctypes.c_int
+    return lib
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        _LIB = load(_build.build())
+    return _LIB
+
+
+def _f64(x):
+    """Widen to a contiguous float64 NumPy array (torch tensors accepted)."""
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _dp(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def threads() -> int:
+    """OpenMP threads the oracle runs on."""
+    return int(_lib().diffattn_oracle_threads())
+
+
+def softmax_row(q, k, scale):
+    """Normalised softmax weights of one query row q [d] against keys k [n, d]."""
+    q, k = _f64(q), _f64(k)
+    out = np.empty(k.shape[0], dtype=np.float64)
+    _lib().diffattn_oracle_softmax_row(_dp(q), _dp(k), k.shape[0], k.shape[1], float(scale),
+                                       _dp(out))
+    return out
+
+
+def prefill(q1, q2, k1, k2, v, lam, gain=None, *, scale, eps, causal=True, apply_norm=True,
+            rows=None):
+    """Prefill oracle.
+
+    q1, k1: [B, N, H, d]; q2, k2: [B, N, H_N, d]; v: [B, N, H_V, dv];
+    lam: [H]; gain: [H, dv] or None.  Returns float64 [B, N, H, dv].
+    rows: None (all rows) or an int array [R, 3] of (b, i, h); then only those
+    rows are computed and the rest of the result is NaN.
+    """
+    q1, q2, k1, k2, v = map(_f64, (q1, q2, k1, k2, v))
+    lam, gain = _f64(lam), _f64(gain)
+    B, N, H, d = q1.shape
+    H_N, H_V, dv = q2.shape[2], v.shape[2], v.shape[3]
+    assert k1.shape == q1.shape and k2.shape == q2.shape and v.shape[:2] == (B, N)
+    assert lam.shape == (H,) and (gain is None or gain.shape == (H, dv))
+    out = np.full((B, N, H, dv), np.nan, dtype=np.float64)
+    rp, nrows = None, 0
+    if rows is not None:
+        rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
+        rp, nrows = rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), rows.shape[0]
+    rc = _lib().diffattn_oracle_prefill(_dp(q1), _dp(q2), _dp(k1), _dp(k2), _dp(v), B, N, H,
+                                        H_N, H_V, d, dv, _dp(lam), _dp(gain), float(scale),
+                                        float(eps), int(bool(causal)), int(bool(apply_norm)),
+                                        rp, nrows, _dp(out))
+    if rc != 0:
+        raise ValueError("oracle prefill: invalid arguments")
+    return out
+
+
+def decode(q1, q2, k1, k2, v, lam, gain=None, *, kv_len=None, scale, eps, apply_norm=True):
+    """Single-query decode oracle.
+
+    q1, q2: [B, H, d]; k1, k2: [B, H, L, d]; v: [B, H, L, dv]; kv_len: [B] or
+    None; lam [H]; gain [H, dv] or None.  Returns float64 [B, H, dv].
+    """
+    q1, q2, k1, k2, v = map(_f64, (q1, q2, k1, k2, v))
+    lam, gain = _f64(lam), _f64(gain)
+    B, H, L, d = k1.shape
+    dv = v.shape[3]
+    kl = None
+    if kv_len is not None:
+        if hasattr(kv_len, "detach"):
+            kv_len = kv_len.detach().cpu().numpy()
+        kl = np.ascontiguousarray(np.asarray(kv_len, dtype=np.int64))
+        assert kl.shape == (B,)
+    out = np.empty((B, H, dv), dtype=np.float64)
+    rc = _lib().diffattn_oracle_decode(
+        _dp(q1), _dp(q2), _dp(k1), _dp(k2), _dp(v), B, H, L, d, dv,
+        kl.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)) if kl is not None else None,
+        _dp(lam), _dp(gain), float(scale), float(eps), int(bool(apply_norm)), _dp(out))
+    if rc != 0:
+        raise ValueError("oracle decode: invalid arguments")
+    return out

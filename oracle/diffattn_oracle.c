@@ -1,0 +1,194 @@
+/*
+ * diffattn_oracle.c -- plain float64 CPU oracle for the differential-attention
+ * forward pass (prefill, grouped prefill, single-query decode).
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file exists so that tests, the package's
+ * smoke check and the benchmark's CPU-baseline leg have an obviously correct
+ * result to compare against.  It shares no code, header, table or helper with
+ * the CUDA path, and the CUDA path never calls it.
+ *
+ * What it computes (one output row = one batch b, one signal head h, one query
+ * position i), step by step, with no tiling, no online softmax and no fusion:
+ *
+ *   1. Key range J.  Causal prefill: keys 0..i (the diagonal is included, so
+ *      no row is empty).  Non-causal prefill: keys 0..N-1.  Decode: the query
+ *      sits at position kv_len-1 and sees keys 0..kv_len-1.
+ *      (Motif 2.6B is a decoder-only Transformer: edgentiq Motif-2.6B blog;
+ *      Motif 3 summary, section 2.1 "full causal-attention layer".)
+ *   2. For each map t in {1,2}: z_j = s * <q_t, k_t[j]>, m = max_j z_j,
+ *      w_j = exp(z_j - m), l = sum_j w_j, A_t[c] = sum_j w_j v[j][c] / l.
+ *      This is softmax(Q_t K_t^T) V written out row by row
+ *      (Motif 2.6B explainer, section "Differential attention", the formula
+ *      attn = [softmax(Q1 K1^T) - lambda softmax(Q2 K2^T)] V; both maps use
+ *      the same V).  The scale s is a parameter (the pages print none).
+ *   3. D[c] = A_1[c] - lambda_h * A_2[c]   (same formula, the subtraction).
+ *      Grouped form: the noise map of signal head h is that of noise head
+ *      n(h) = h / g, i.e. Repeat_g interleaves the noise heads (Motif 3
+ *      summary, section 2.2, eq. "grouped differential output"
+ *      D_t = H_S,t - lambda_t (.) Repeat_g(H_N,t)).  The V head of signal head
+ *      h is v(h) = h / (H / H_V).
+ *   4. Norm after the subtraction (Motif 2.6B explainer, figure 1 caption and
+ *      the paragraph on the GroupNorm that "keeps the ... scores stable"),
+ *      read as one RMS group per head and token over its dv channels:
+ *      Y[c] = D[c] / sqrt(mean_c D[c]^2 + eps) * gain[h][c].
+ *      With apply_norm == 0 the pre-norm D is returned.
+ *
+ * Every input is float64 (the exact bf16 / fp32 values widened by the caller)
+ * and every intermediate is float64.  Built with -ffp-contract=off so that the
+ * compiler does not fuse multiplies and adds behind the reader's back.
+ *
+ * Layouts (all contiguous, row-major, element counts not bytes):
+ *   prefill: q1,k1 [B][N][H][d]; q2,k2 [B][N][H_N][d]; v [B][N][H_V][dv];
+ *            out [B][N][H][dv]; lambda [H]; gain [H][dv] or NULL (= 1).
+ *   decode:  q1,q2 [B][H][d]; k1,k2 [B][H][L][d]; v [B][H][L][dv];
+ *            kv_len [B] or NULL (= L); out [B][H][dv].
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Softmax weights of one query row against nkeys keys (step 2 above, before
+ * the product with V).  w receives exp(z_j - m); the return value is l.       */
+static double softmax_weights(const double *q, const double *k, int64_t k_row_stride,
+                              int64_t nkeys, int64_t d, double scale, double *w)
+{
+    double m = -INFINITY;
+    for (int64_t j = 0; j < nkeys; ++j) {
+        const double *kj = k + j * k_row_stride;
+        double dot = 0.0;
+        for (int64_t c = 0; c < d; ++c) dot += q[c] * kj[c];
+        w[j] = scale * dot;
+        if (w[j] > m) m = w[j];
+    }
+    double l = 0.0;
+    for (int64_t j = 0; j < nkeys; ++j) {
+        w[j] = exp(w[j] - m);
+        l += w[j];
+    }
+    return l;
+}
+
+/* One output row: steps 2-4 above.  a1, a2 are scratch of length dv; w1, w2 of
+ * length nkeys.                                                               */
+static void diff_row(const double *q1, const double *k1, int64_t k1_rs,
+                     const double *q2, const double *k2, int64_t k2_rs,
+                     const double *v, int64_t v_rs,
+                     int64_t nkeys, int64_t d, int64_t dv, double scale,
+                     double lambda, const double *gain, double eps, int apply_norm,
+                     double *w1, double *w2, double *a1, double *a2, double *out)
+{
+    double l1 = softmax_weights(q1, k1, k1_rs, nkeys, d, scale, w1);
+    double l2 = softmax_weights(q2, k2, k2_rs, nkeys, d, scale, w2);
+    for (int64_t c = 0; c < dv; ++c) { a1[c] = 0.0; a2[c] = 0.0; }
+    for (int64_t j = 0; j < nkeys; ++j) {
+        const double *vj = v + j * v_rs;
+        for (int64_t c = 0; c < dv; ++c) {
+            a1[c] += w1[j] * vj[c];
+            a2[c] += w2[j] * vj[c];
+        }
+    }
+    for (int64_t c = 0; c < dv; ++c) out[c] = a1[c] / l1 - lambda * (a2[c] / l2);
+    if (!apply_norm) return;
+    double ss = 0.0;
+    for (int64_t c = 0; c < dv; ++c) ss += out[c] * out[c];
+    double r = 1.0 / sqrt(ss / (double)dv + eps);
+    for (int64_t c = 0; c < dv; ++c) out[c] = out[c] * r * (gain ? gain[c] : 1.0);
+}
+
+/* Number of OpenMP threads the oracle will use (reported beside its timings). */
+int diffattn_oracle_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Softmax weights w_j / l of one query row (one map), for the "each row sums
+ * to 1" check.  q [d]; k [nkeys][d]; out [nkeys].                             */
+void diffattn_oracle_softmax_row(const double *q, const double *k, int64_t nkeys, int64_t d,
+                                 double scale, double *out)
+{
+    double l = softmax_weights(q, k, d, nkeys, d, scale, out);
+    for (int64_t j = 0; j < nkeys; ++j) out[j] /= l;
+}
+
+/* Prefill (and grouped prefill).  rows: NULL for every (b, i, h), otherwise
+ * nrows triples (b, i, h) whose outputs are written; other rows of out are not
+ * touched.  Returns 0, or -1 on an invalid argument.                          */
+int diffattn_oracle_prefill(const double *q1, const double *q2, const double *k1,
+                            const double *k2, const double *v,
+                            int64_t B, int64_t N, int64_t H, int64_t H_N, int64_t H_V,
+                            int64_t d, int64_t dv,
+                            const double *lambda, const double *gain,
+                            double scale, double eps, int causal, int apply_norm,
+                            const int64_t *rows, int64_t nrows, double *out)
+{
+    if (B < 0 || N < 0 || H <= 0 || H_N <= 0 || H_V <= 0 || d <= 0 || dv <= 0) return -1;
+    if (H % H_N != 0 || H % H_V != 0) return -1;
+    const int64_t g = H / H_N;       /* signal heads per noise head */
+    const int64_t gv = H / H_V;      /* signal heads per V head */
+    const int64_t total = rows ? nrows : B * N * H;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *w1 = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+        double *w2 = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
+        double *a1 = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *a2 = (double *)malloc(sizeof(double) * (size_t)dv);
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t r = 0; r < total; ++r) {
+            int64_t b, i, h;
+            if (rows) { b = rows[3 * r]; i = rows[3 * r + 1]; h = rows[3 * r + 2]; }
+            else { b = r / (N * H); i = (r / H) % N; h = r % H; }
+            if (b < 0 || b >= B || i < 0 || i >= N || h < 0 || h >= H) { bad = 1; continue; }
+            const int64_t n = h / g, hv = h / gv;
+            const int64_t nkeys = causal ? i + 1 : N;
+            const double *q1r = q1 + ((b * N + i) * H + h) * d;
+            const double *q2r = q2 + ((b * N + i) * H_N + n) * d;
+            const double *k1b = k1 + ((b * N) * H + h) * d;
+            const double *k2b = k2 + ((b * N) * H_N + n) * d;
+            const double *vb = v + ((b * N) * H_V + hv) * dv;
+            diff_row(q1r, k1b, H * d, q2r, k2b, H_N * d, vb, H_V * dv, nkeys, d, dv, scale,
+                     lambda[h], gain ? gain + h * dv : NULL, eps, apply_norm, w1, w2, a1, a2,
+                     out + ((b * N + i) * H + h) * dv);
+        }
+        free(w1); free(w2); free(a1); free(a2);
+    }
+    return bad ? -1 : 0;
+}
+
+/* Single-query decode.  kv_len: NULL (every sequence has L keys) or [B] with
+ * 1 <= kv_len[b] <= L.  Returns 0, or -1 on an invalid argument.              */
+int diffattn_oracle_decode(const double *q1, const double *q2, const double *k1,
+                           const double *k2, const double *v,
+                           int64_t B, int64_t H, int64_t L, int64_t d, int64_t dv,
+                           const int64_t *kv_len, const double *lambda, const double *gain,
+                           double scale, double eps, int apply_norm, double *out)
+{
+    if (B < 0 || H <= 0 || L <= 0 || d <= 0 || dv <= 0) return -1;
+    for (int64_t b = 0; b < B; ++b)
+        if (kv_len && (kv_len[b] < 1 || kv_len[b] > L)) return -1;
+#pragma omp parallel
+    {
+        double *w1 = (double *)malloc(sizeof(double) * (size_t)L);
+        double *w2 = (double *)malloc(sizeof(double) * (size_t)L);
+        double *a1 = (double *)malloc(sizeof(double) * (size_t)dv);
+        double *a2 = (double *)malloc(sizeof(double) * (size_t)dv);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < B * H; ++r) {
+            const int64_t b = r / H, h = r % H;
+            const int64_t nkeys = kv_len ? kv_len[b] : L;
+            diff_row(q1 + r * d, k1 + r * L * d, d, q2 + r * d, k2 + r * L * d, d,
+                     v + r * L * dv, dv, nkeys, d, dv, scale, lambda[h],
+                     gain ? gain + h * dv : NULL, eps, apply_norm, w1, w2, a1, a2, out + r * dv);
+        }
+        free(w1); free(w2); free(a1); free(a2);
+    }
+    return 0;
+}

@@ -1,0 +1,21 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+@pytest.fixture(scope="session")
+def cuda_ok():
+    import torch
+    # GPU tests fail rather than skip without a device: a silent skip would
+    # read as a pass.
+    assert torch.cuda.is_available(), "gpu-marked test needs a CUDA device"
+    return True
