@@ -1,0 +1,440 @@
+"""Benchmark of the differential-attention forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one causal prefill of the Motif-2.6B-shaped workload (batch 4,
+sequence 4096, 16 heads, Q/K head dim 64, V head dim 128, bf16) through the C
+ABI: the fp16 V staging kernel plus the warp-specialised tcgen05 prefill
+kernel.  Rank 0 prints one JSON line:
+
+* value        prefill TFLOP/s over all ranks (768 FLOP per causal
+               query/key pair per head), inputs resident in HBM;
+* e2e          the same metric with pinned-host inputs copied in and the output
+               copied out inside the timed region;
+* roofline     the prefill kernel alone, timed with CUDA events recorded
+               around its launch, against the measured dense-bf16 peak;
+* cpu_baseline the float64 oracle on a bounded sample of the same workload
+               (rank 0, one GPU only);
+* extra        the other workloads at one pass each: long context (1 x 16384),
+               grouped (24 signal / 8 noise heads), decode (batch 64, 8192
+               cached keys; GB/s against the measured HBM copy bandwidth).
+
+With more than one GPU (torchrun) every rank runs its own batch of the same
+shape (weak scaling; the path has no exchange step) and the time is the max
+over ranks.  `--impl reference` times the oracle itself on the host cores.
+"""
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from differential_attention_07_b200 import inputs  # noqa: E402
+
+FLOP_PER_PAIR = 768  # 2*64 + 2*64 (two QK^T) + 2*128 + 2*128 (two P.V)
+
+
+def causal_pairs(N):
+    return N * (N + 1) // 2
+
+
+def prefill_flops(w):
+    """Algorithmic FLOP of one prefill call (causal pairs only)."""
+    pairs = causal_pairs(w.N) if w.causal else w.N * w.N
+    return FLOP_PER_PAIR * pairs * w.B * w.H
+
+
+def decode_bytes(w):
+    """Algorithmic HBM bytes of one decode call: K1 + K2 + V read once."""
+    return w.B * w.H * w.N * (64 + 64 + 128) * 2
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return dict(hbm_gbs=j["hbm_gbs"], bf16_tflops=j["bf16_tflops"],
+                    bf16_tflops_sustained=j.get("bf16_tflops_sustained"), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                source="fallback")
+
+
+# ------------------------------------------------------------------ distributed
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def max_over_ranks(x, device):
+    """Max of a float over ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def aggregate_throughput(units_per_rank, elapsed_s_local, device, world):
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    t = max_over_ranks(elapsed_s_local, device)
+    return units_per_rank * world / t, t
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r.split(",") for r in (getattr(self, "out", "") or "").strip().splitlines()]
+        rows = [[c.strip() for c in r] for r in rows if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
+        mx = max((float(r[2]) for r in rows if r[2].replace(".", "").isdigit()), default=None)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ timing helpers
+def time_loop(fn, steps, warmup, device, stream=None):
+    """Device time (s) of `steps` calls of fn after `warmup` calls; barrier and
+    synchronize on both sides; events on the launching stream."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    s = stream or torch.cuda.current_stream(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        fn()
+    e1.record(s)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    return e0.elapsed_time(e1) / 1e3
+
+
+def kernel_time(call, steps, ops):
+    """Average duration (s) of the main kernel of `call`, from events the
+    library records around that launch, over `steps` calls."""
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for e in starts + stops:
+        e.record()  # torch creates the CUDA event on first record
+    torch.cuda.synchronize()
+    for a, b in zip(starts, stops):
+        ops.set_profile_events(a, b)
+        call()
+    ops.set_profile_events(None, None)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in zip(starts, stops)) / steps / 1e3
+
+
+# ------------------------------------------------------------------ CPU baseline
+def cpu_baseline(w, budget_s=12.0, seed_rows=0):
+    """The float64 oracle on a bounded, row-sampled piece of workload `w`:
+    returns (throughput in the workload's unit, description, threads)."""
+    import oracle
+    x = inputs.workload_inputs(w)
+    if w.kind == "decode":
+        nseq = 1
+        t0 = time.perf_counter()
+        while True:
+            sub = {k: (v[:nseq] if k not in ("lam", "gain") else v) for k, v in x.items()}
+            t0 = time.perf_counter()
+            oracle.decode(sub["q1"], sub["q2"], sub["k1"], sub["k2"], sub["v"], sub["lam"],
+                          sub["gain"], scale=w.scale, eps=w.eps)
+            dt = time.perf_counter() - t0
+            if dt > budget_s / 4 or nseq >= w.B:
+                break
+            nseq = min(w.B, nseq * 4)
+        byts = nseq * w.H * w.N * 256 * 2
+        return byts / dt / 1e9, f"{nseq} of {w.B} sequences x {w.H} heads x {w.N} keys", oracle.threads()
+    # prefill: sample rows uniformly over (b, i, h); work of a row = (i+1) pairs
+    nrows = 64
+    while True:
+        rows = inputs.sample_rows(w.B, w.N, w.H, nrows, seed=w.seed + 7 + seed_rows)
+        t0 = time.perf_counter()
+        oracle.prefill(x["q1"], x["q2"], x["k1"], x["k2"], x["v"], x["lam"], x["gain"],
+                       scale=w.scale, eps=w.eps, causal=w.causal, rows=rows)
+        dt = time.perf_counter() - t0
+        if dt > budget_s / 4 or nrows >= 1 << 16:
+            break
+        nrows *= 4
+    pairs = int((rows[:, 1] + 1).sum()) if w.causal else nrows * w.N
+    flops = pairs * FLOP_PER_PAIR
+    return flops / dt / 1e12, f"{nrows} sampled query rows of {w.name} ({pairs} causal pairs)", oracle.threads()
+
+
+# ------------------------------------------------------------------ GPU arm
+def to_dev(x, device):
+    return {k: v.to(device, non_blocking=True) for k, v in x.items()}
+
+
+def run_prefill_workload(w, steps, warmup, device, ops, rank=0):
+    x = inputs.workload_inputs(inputs.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}))
+    d = to_dev(x, device)
+    grouped = w.kind == "grouped"
+    f = ops.diffattn_grouped_fwd if grouped else ops.diffattn_fwd
+    out = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=device)
+    ws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H, w.H_V), dtype=torch.uint8, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def call():
+        f(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"], scale=w.scale, eps=w.eps,
+          causal=w.causal, out=out, workspace=ws, dev_status=status)
+
+    call()
+    launches = ops.last_launch_count()
+    t = time_loop(call, steps, warmup, device)
+    tk = kernel_time(call, max(3, min(steps, 20)), ops)
+    torch.cuda.synchronize(device)
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()} in {w.name}")
+    return dict(step_s=t / steps, kernel_s=tk, launches=launches, x=x, d=d, call=call, out=out,
+                ws=ws, f=f)
+
+
+def run_decode_workload(w, steps, warmup, device, ops):
+    x = inputs.workload_inputs(w)
+    d = to_dev(x, device)
+    out = torch.empty(w.B, w.H, w.dv, dtype=torch.bfloat16, device=device)
+    ws = torch.empty(ops.decode_workspace_size(w.B, w.H, w.N), dtype=torch.uint8, device=device)
+
+    def call():
+        ops.diffattn_decode(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"],
+                            scale=w.scale, eps=w.eps, out=out, workspace=ws)
+
+    call()
+    launches = ops.last_launch_count()
+    t = time_loop(call, steps, warmup, device)
+    tk = kernel_time(call, max(3, min(steps, 20)), ops)
+    return dict(step_s=t / steps, kernel_s=tk, launches=launches)
+
+
+def e2e_prefill(w, steps, warmup, device, ops, x):
+    """Same metric through the public call with pinned-host inputs: H2D copies
+    of every input, the call, D2H copy of the output, all inside the timing."""
+    host = {k: v.pin_memory() for k, v in x.items()}
+    dev = {k: torch.empty_like(v, device=device) for k, v in x.items()}
+    out = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=device)
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    ws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H, w.H_V), dtype=torch.uint8, device=device)
+    f = ops.diffattn_grouped_fwd if w.kind == "grouped" else ops.diffattn_fwd
+
+    def step():
+        for k in dev:
+            dev[k].copy_(host[k], non_blocking=True)
+        f(dev["q1"], dev["q2"], dev["k1"], dev["k2"], dev["v"], dev["lam"], dev["gain"],
+          scale=w.scale, eps=w.eps, causal=w.causal, out=out, workspace=ws)
+        out_host.copy_(out, non_blocking=True)
+
+    t = time_loop(step, steps, warmup, device)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    return t / steps, h2d, d2h
+
+
+def gpu_arm(args):
+    world, rank, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    init_dist(world, "nccl")
+    from differential_attention_07_b200 import build, ops
+    if rank == 0:
+        build.build()
+    barrier(device)
+    peaks = measured_peaks()
+    w = inputs.WORKLOADS[args.workload]
+    units = prefill_flops(w)
+
+    with ClockSampler(local) as clk:
+        r = run_prefill_workload(w, args.steps, args.warmup, device, ops, rank)
+    value, t_max = aggregate_throughput(units * args.steps, r["step_s"] * args.steps, device, world)
+    value /= 1e12
+    e2e_s, h2d, d2h = e2e_prefill(w, max(3, args.steps // 4), 2, device, ops, r["x"])
+    e2e_value, _ = aggregate_throughput(units, e2e_s, device, world)
+
+    achieved = units / r["kernel_s"] / 1e12
+    result = {
+        "metric": "diff-attn fwd TFLOP/s (bf16 causal)",
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(t_max / args.steps * 1e3, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name}: B{w.B} N{w.N} H{w.H} d64 dv128 causal prefill",
+                   "global_batch": w.B * world, "seq_len": w.N, "heads": w.H,
+                   "parallelism": f"dp{world} (independent batches)",
+                   "l2": "inputs 201 MB per rank, larger than the 126 MB L2; no flush"},
+        "e2e": {"value": round(e2e_value / 1e12, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / peaks["bf16_tflops"], 4),
+                     "peak_source": peaks["source"] + " bf16 burst (MEASURED_PEAKS.json)",
+                     "kernel": "prefill_kernel", "traffic": None},
+        "gpu_launches": r["launches"] * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_extra:
+        extra = {}
+        for name in ("lc16k", "grouped"):
+            wx = inputs.WORKLOADS[name]
+            rx = run_prefill_workload(wx, max(3, args.steps // 5), 2, device, ops)
+            fx = prefill_flops(wx)
+            extra[name] = {"tflops": round(fx / rx["step_s"] / 1e12, 2),
+                           "kernel_tflops": round(fx / rx["kernel_s"] / 1e12, 2),
+                           "frac_of_peak": round(fx / rx["kernel_s"] / 1e12 / peaks["bf16_tflops"], 4),
+                           "ms": round(rx["step_s"] * 1e3, 4)}
+            del rx
+        wd = inputs.WORKLOADS["decode"]
+        rd = run_decode_workload(wd, max(5, args.steps), 3, device, ops)
+        bd = decode_bytes(wd)
+        extra["decode"] = {"gbs": round(bd / rd["step_s"] / 1e9, 1),
+                           "split_kernel_gbs": round(bd / rd["kernel_s"] / 1e9, 1),
+                           "roofline": {"bound": "hbm", "achieved": round(bd / rd["step_s"] / 1e9, 1),
+                                        "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                        "frac": round(bd / rd["step_s"] / 1e9 / peaks["hbm_gbs"], 4)},
+                           "us": round(rd["step_s"] * 1e6, 2), "launches": rd["launches"]}
+        result["extra"] = extra
+    if world == 1 and rank == 0 and not args.no_cpu:
+        v, sample, cores = cpu_baseline(w, budget_s=args.cpu_budget)
+        result["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": cores,
+                                  "kind": "oracle", "sample": sample}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+
+
+def reference_arm(args):
+    """The oracle as it stands, timed on the host cores (rank 0 only)."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    w = inputs.WORKLOADS[args.workload]
+    import oracle
+    x = inputs.workload_inputs(w)
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    rows = None
+    nrows = 16
+    while True:  # size one step's row sample to about per_step seconds
+        rows = inputs.sample_rows(w.B, w.N, w.H, nrows, seed=w.seed + 99)
+        t0 = time.perf_counter()
+        oracle.prefill(x["q1"], x["q2"], x["k1"], x["k2"], x["v"], x["lam"], x["gain"],
+                       scale=w.scale, eps=w.eps, causal=w.causal, rows=rows)
+        if time.perf_counter() - t0 > per_step / 4 or nrows >= 1 << 16:
+            break
+        nrows *= 2
+    nrows = int(nrows * min(4.0, per_step / max(1e-3, time.perf_counter() - t0)))
+    total_flops, total_t = 0, 0.0
+    for s in range(args.warmup + args.steps):
+        rows = inputs.sample_rows(w.B, w.N, w.H, nrows, seed=w.seed + 100 + s)
+        t0 = time.perf_counter()
+        oracle.prefill(x["q1"], x["q2"], x["k1"], x["k2"], x["v"], x["lam"], x["gain"],
+                       scale=w.scale, eps=w.eps, causal=w.causal, rows=rows)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            total_t += dt
+            total_flops += int((rows[:, 1] + 1).sum()) * FLOP_PER_PAIR
+    value = total_flops / total_t / 1e12
+    sample = f"{nrows} sampled query rows per step of {w.name}"
+    print(json.dumps({
+        "impl": "reference", "metric": "diff-attn fwd TFLOP/s (bf16 causal)",
+        "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_t / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{w.name}: B{w.B} N{w.N} H{w.H} d64 dv128 causal prefill",
+                   "global_batch": w.B, "seq_len": w.N, "heads": w.H},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="motif4k", choices=["motif4k", "lc16k", "grouped"])
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        gpu_arm(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,330 @@
+// api.cu -- the C ABI of libdiffattn: argument validation, TMA tensor-map
+// encoding, workspace layout and kernel launches.  Nothing here allocates
+// device memory or synchronises a stream.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "diffattn.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local int32_t g_last_launches = 0;
+thread_local da::ProfileEvents g_events;
+
+constexpr uint32_t kDefaultTimeoutMs = 2000;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool stride8(int64_t s) { return s % 8 == 0; }
+
+// cuTensorMapEncodeTiled, fetched once from the driver through the runtime
+// (so the library does not link libcuda directly).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 4-D map over a [B, N, heads, inner] tensor (element strides sb, sn, sh;
+// inner contiguous), box {64, 128, 1, 1}, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int64_t inner,
+              int64_t N, int64_t heads, int64_t B, int64_t sb, int64_t sn, int64_t sh)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)inner, (cuuint64_t)N, (cuuint64_t)heads,
+                                (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)(sn * 2), (cuuint64_t)(sh * 2),
+                                   (cuuint64_t)(sb * 2)};
+    const cuuint32_t box[4] = {64, 128, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, dt, 4, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+diffattn_status validate_fwd(const diffattn_fwd_args *a, int grouped)
+{
+    if (!a) return DIFFATTN_ERR_INVALID_ARG;
+    if (a->B < 0 || a->N < 0 || a->H <= 0) return DIFFATTN_ERR_INVALID_ARG;
+    const int64_t HN = a->H_N ? a->H_N : a->H, HV = a->H_V ? a->H_V : a->H;
+    if (HN <= 0 || HV <= 0 || a->H_N < 0 || a->H_V < 0) return DIFFATTN_ERR_INVALID_ARG;
+    if (!grouped && (HN != a->H || HV != a->H)) return DIFFATTN_ERR_INVALID_ARG;
+    if (a->H % HN != 0 || a->H % HV != 0) return DIFFATTN_ERR_INVALID_ARG;
+    if (a->d != 64 || a->dv != 128) return DIFFATTN_ERR_UNSUPPORTED;
+    if (a->flags & ~(DIFFATTN_FLAG_CAUSAL | DIFFATTN_FLAG_APPLY_NORM)) return DIFFATTN_ERR_INVALID_ARG;
+    if (!(a->scale > 0.0f) || !std::isfinite(a->scale)) return DIFFATTN_ERR_INVALID_ARG;
+    if (!(a->eps >= 0.0f) || !std::isfinite(a->eps)) return DIFFATTN_ERR_INVALID_ARG;
+    // Index arithmetic inside the kernels is 32-bit for counts.
+    if (a->N > (1 << 24) || a->B > (1 << 16) || a->H > 4096) return DIFFATTN_ERR_UNSUPPORTED;
+    if ((a->B * a->H * ((a->N + 127) / 128)) > INT32_MAX) return DIFFATTN_ERR_UNSUPPORTED;
+    if (a->B == 0 || a->N == 0) return DIFFATTN_OK;  // nothing to compute
+    const void *ptrs[6] = {a->q1, a->q2, a->k1, a->k2, a->v, a->out};
+    for (const void *p : ptrs)
+        if (!p) return DIFFATTN_ERR_INVALID_ARG;
+    if (!a->lambda) return DIFFATTN_ERR_INVALID_ARG;
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return DIFFATTN_ERR_ALIGNMENT;
+    const int64_t *strides[6] = {a->q1_stride, a->q2_stride, a->k1_stride, a->k2_stride,
+                                 a->v_stride, a->out_stride};
+    for (const int64_t *s : strides)
+        for (int i = 0; i < 3; ++i) {
+            if (s[i] < 0) return DIFFATTN_ERR_INVALID_ARG;
+            if (!stride8(s[i])) return DIFFATTN_ERR_ALIGNMENT;
+        }
+    return DIFFATTN_OK;
+}
+
+diffattn_status validate_decode(const diffattn_decode_args *a)
+{
+    if (!a) return DIFFATTN_ERR_INVALID_ARG;
+    if (a->B < 0 || a->H <= 0 || a->L <= 0) return DIFFATTN_ERR_INVALID_ARG;
+    if (a->d != 64 || a->dv != 128) return DIFFATTN_ERR_UNSUPPORTED;
+    if (a->flags & ~(DIFFATTN_FLAG_CAUSAL | DIFFATTN_FLAG_APPLY_NORM)) return DIFFATTN_ERR_INVALID_ARG;
+    if (a->num_splits < 0) return DIFFATTN_ERR_INVALID_ARG;
+    if (!(a->scale > 0.0f) || !std::isfinite(a->scale)) return DIFFATTN_ERR_INVALID_ARG;
+    if (!(a->eps >= 0.0f) || !std::isfinite(a->eps)) return DIFFATTN_ERR_INVALID_ARG;
+    if (a->L > (1 << 26) || a->B > (1 << 16) || a->H > 4096) return DIFFATTN_ERR_UNSUPPORTED;
+    if (a->B == 0) return DIFFATTN_OK;
+    const void *ptrs[6] = {a->q1, a->q2, a->k1, a->k2, a->v, a->out};
+    for (const void *p : ptrs)
+        if (!p) return DIFFATTN_ERR_INVALID_ARG;
+    if (!a->lambda) return DIFFATTN_ERR_INVALID_ARG;
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return DIFFATTN_ERR_ALIGNMENT;
+    const int64_t s2[4] = {a->q1_stride[0], a->q1_stride[1], a->q2_stride[0], a->q2_stride[1]};
+    for (int64_t s : s2) {
+        if (s < 0) return DIFFATTN_ERR_INVALID_ARG;
+        if (!stride8(s)) return DIFFATTN_ERR_ALIGNMENT;
+    }
+    const int64_t *s3[3] = {a->k1_stride, a->k2_stride, a->v_stride};
+    for (const int64_t *s : s3)
+        for (int i = 0; i < 3; ++i) {
+            if (s[i] < 0) return DIFFATTN_ERR_INVALID_ARG;
+            if (!stride8(s[i])) return DIFFATTN_ERR_ALIGNMENT;
+        }
+    if (a->out_stride[0] < 0 || a->out_stride[1] < 0) return DIFFATTN_ERR_INVALID_ARG;
+    return DIFFATTN_OK;
+}
+
+int decode_splits(int64_t B, int64_t H, int64_t L, int32_t requested)
+{
+    const int64_t min_splits = (L + da::kDecodeMaxChunk - 1) / da::kDecodeMaxChunk;
+    int64_t s = requested > 0 ? requested : 0;
+    if (s == 0) {
+        // Enough CTAs for about four per SM on 148 SMs, chunks of >= 256 keys.
+        const int64_t bh = B * H > 0 ? B * H : 1;
+        s = (4 * 148 + bh - 1) / bh;
+        const int64_t max_by_len = (L + 255) / 256;
+        if (s > max_by_len) s = max_by_len;
+    }
+    if (s < min_splits) s = min_splits;
+    if (s > L) s = L;
+    if (s < 1) s = 1;
+    // Chunk rounded up to 64 keys; drop splits that would be empty.
+    const int64_t chunk = ((L + s - 1) / s + 63) / 64 * 64;
+    s = (L + chunk - 1) / chunk;
+    return (int)s;
+}
+
+int decode_chunk(int64_t L, int splits) { return (int)(((L + splits - 1) / splits + 63) / 64 * 64); }
+
+diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, void *stream,
+                        int grouped)
+{
+    g_last_launches = 0;
+    diffattn_status st = validate_fwd(a, grouped);
+    if (st != DIFFATTN_OK) return st;
+    if (a->B == 0 || a->N == 0) return DIFFATTN_OK;
+    const size_t need = diffattn_fwd_workspace_size(a);
+    if (!ws || ws_bytes < need) return DIFFATTN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return DIFFATTN_ERR_ALIGNMENT;
+    const int64_t HN = a->H_N ? a->H_N : a->H, HV = a->H_V ? a->H_V : a->H;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    CUtensorMap mq1, mq2, mk1, mk2, mv;
+    const bool ok =
+        make_map(&mq1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->q1, 64, a->N, a->H, a->B,
+                 a->q1_stride[0], a->q1_stride[1], a->q1_stride[2]) &&
+        make_map(&mq2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->q2, 64, a->N, HN, a->B,
+                 a->q2_stride[0], a->q2_stride[1], a->q2_stride[2]) &&
+        make_map(&mk1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->k1, 64, a->N, a->H, a->B,
+                 a->k1_stride[0], a->k1_stride[1], a->k1_stride[2]) &&
+        make_map(&mk2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->k2, 64, a->N, HN, a->B,
+                 a->k2_stride[0], a->k2_stride[1], a->k2_stride[2]) &&
+        make_map(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws, 128, a->N, HV, a->B, a->N * HV * 128,
+                 HV * 128, 128);
+    if (!ok) return DIFFATTN_ERR_CUDA;
+
+    int launches = 0;
+    cudaError_t e = da::launch_v_to_f16(a->v, a->v_stride[0], a->v_stride[1], a->v_stride[2], ws,
+                                        (int)a->B, (int)a->N, (int)HV, a->dev_status, s, &launches);
+    if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
+
+    da::PrefillParams p{};
+    p.B = (int)a->B;
+    p.N = (int)a->N;
+    p.H = (int)a->H;
+    p.H_N = (int)HN;
+    p.H_V = (int)HV;
+    p.num_qt = (int)((a->N + 127) / 128);
+    int G = (2 * 148) / p.num_qt;
+    if (G < 1) G = 1;
+    if (G > p.B * p.H) G = p.B * p.H;
+    p.heads_per_group = G;
+    p.scale_log2 = a->scale * 1.4426950408889634f;
+    p.eps = a->eps;
+    p.causal = (a->flags & DIFFATTN_FLAG_CAUSAL) ? 1 : 0;
+    p.apply_norm = (a->flags & DIFFATTN_FLAG_APPLY_NORM) ? 1 : 0;
+    p.lambda = a->lambda;
+    p.gain = a->gain;
+    p.out = a->out;
+    p.out_sb = a->out_stride[0];
+    p.out_sn = a->out_stride[1];
+    p.out_sh = a->out_stride[2];
+    p.dev_status = a->dev_status;
+    p.timeout_ns = (uint64_t)(a->timeout_ms ? a->timeout_ms : kDefaultTimeoutMs) * 1000000ull;
+    e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, p, s, &launches, g_events);
+    if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
+    g_last_launches = launches;
+    return DIFFATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+diffattn_status diffattn_fwd_validate(const diffattn_fwd_args *args, int grouped)
+{
+    return validate_fwd(args, grouped);
+}
+
+size_t diffattn_fwd_workspace_size(const diffattn_fwd_args *a)
+{
+    if (!a || a->B <= 0 || a->N <= 0) return 0;
+    const int64_t HV = a->H_V ? a->H_V : a->H;
+    return align256((size_t)a->B * a->N * HV * 128 * 2);
+}
+
+diffattn_status diffattn_fwd(const diffattn_fwd_args *args, void *workspace, size_t ws_bytes,
+                             void *stream)
+{
+    return run_fwd(args, workspace, ws_bytes, stream, 0);
+}
+
+diffattn_status diffattn_grouped_fwd(const diffattn_fwd_args *args, void *workspace,
+                                     size_t ws_bytes, void *stream)
+{
+    return run_fwd(args, workspace, ws_bytes, stream, 1);
+}
+
+diffattn_status diffattn_decode_validate(const diffattn_decode_args *args)
+{
+    return validate_decode(args);
+}
+
+int32_t diffattn_decode_num_splits(int64_t B, int64_t H, int64_t L, int32_t num_splits)
+{
+    if (B < 0 || H <= 0 || L <= 0 || num_splits < 0) return 0;
+    return decode_splits(B, H, L, num_splits);
+}
+
+size_t diffattn_decode_workspace_size(int64_t B, int64_t H, int64_t L, int32_t num_splits)
+{
+    if (B <= 0 || H <= 0 || L <= 0 || num_splits < 0) return 0;
+    const int s = decode_splits(B, H, L, num_splits);
+    return align256((size_t)B * H * s * da::kDecodePartialFloats * sizeof(float));
+}
+
+diffattn_status diffattn_decode(const diffattn_decode_args *a, void *workspace, size_t ws_bytes,
+                                void *stream)
+{
+    g_last_launches = 0;
+    diffattn_status st = validate_decode(a);
+    if (st != DIFFATTN_OK) return st;
+    if (a->B == 0) return DIFFATTN_OK;
+    const size_t need = diffattn_decode_workspace_size(a->B, a->H, a->L, a->num_splits);
+    if (!workspace || ws_bytes < need) return DIFFATTN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return DIFFATTN_ERR_ALIGNMENT;
+    da::DecodeParams p{};
+    p.B = (int)a->B;
+    p.H = (int)a->H;
+    p.L = (int)a->L;
+    p.splits = decode_splits(a->B, a->H, a->L, a->num_splits);
+    p.chunk = decode_chunk(a->L, p.splits);
+    p.scale_log2 = a->scale * 1.4426950408889634f;
+    p.eps = a->eps;
+    p.apply_norm = (a->flags & DIFFATTN_FLAG_APPLY_NORM) ? 1 : 0;
+    p.q1 = a->q1;
+    p.q2 = a->q2;
+    p.k1 = a->k1;
+    p.k2 = a->k2;
+    p.v = a->v;
+    p.q1_sb = a->q1_stride[0];
+    p.q1_sh = a->q1_stride[1];
+    p.q2_sb = a->q2_stride[0];
+    p.q2_sh = a->q2_stride[1];
+    p.k1_sb = a->k1_stride[0];
+    p.k1_sh = a->k1_stride[1];
+    p.k1_sl = a->k1_stride[2];
+    p.k2_sb = a->k2_stride[0];
+    p.k2_sh = a->k2_stride[1];
+    p.k2_sl = a->k2_stride[2];
+    p.v_sb = a->v_stride[0];
+    p.v_sh = a->v_stride[1];
+    p.v_sl = a->v_stride[2];
+    p.out = a->out;
+    p.out_sb = a->out_stride[0];
+    p.out_sh = a->out_stride[1];
+    p.kv_len = a->kv_len;
+    p.lambda = a->lambda;
+    p.gain = a->gain;
+    p.partials = static_cast<float *>(workspace);
+    p.dev_status = a->dev_status;
+    int launches = 0;
+    cudaError_t e = da::launch_decode(p, static_cast<cudaStream_t>(stream), &launches, g_events);
+    if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
+    g_last_launches = launches;
+    return DIFFATTN_OK;
+}
+
+const char *diffattn_status_str(diffattn_status s)
+{
+    switch (s) {
+    case DIFFATTN_OK: return "ok";
+    case DIFFATTN_ERR_INVALID_ARG: return "invalid argument";
+    case DIFFATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case DIFFATTN_ERR_ALIGNMENT: return "misaligned pointer or stride";
+    case DIFFATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case DIFFATTN_ERR_CUDA: return "CUDA error";
+    case DIFFATTN_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+int32_t diffattn_last_launch_count(void) { return g_last_launches; }
+
+void diffattn_set_profile_events(void *start, void *stop)
+{
+    g_events.start = static_cast<cudaEvent_t>(start);
+    g_events.stop = static_cast<cudaEvent_t>(stop);
+}
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// kernels.h -- host-side launch interface between the C ABI (api.cu) and the
+// kernel translation units.  Internal to libdiffattn.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace da {
+
+// Events to record around the main kernel of a call (benchmark timing hook);
+// both null when unused.
+struct ProfileEvents {
+    cudaEvent_t start = nullptr, stop = nullptr;
+};
+
+// Everything the prefill kernel needs besides its five tensor maps.
+struct PrefillParams {
+    int B, N, H, H_N, H_V;
+    int num_qt;           // query tiles per (b, h): ceil(N / 128)
+    int heads_per_group;  // (b, h) pairs scheduled together for L2 reuse of K/V
+    float scale_log2;     // softmax scale * log2(e)
+    float eps;
+    int causal, apply_norm;
+    const float *lambda;
+    const float *gain;    // [H, 128] or nullptr
+    void *out;            // bf16
+    int64_t out_sb, out_sn, out_sh;
+    int32_t *dev_status;
+    uint64_t timeout_ns;
+};
+
+// Tensor maps: Q1/K1 over [B, N, H, 64] bf16, Q2/K2 over [B, N, H_N, 64]
+// bf16, V over the fp16 copy [B, N, H_V, 128]; all with 128-byte swizzle and
+// {64, 128, 1, 1} boxes.
+cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const CUtensorMap &k1,
+                           const CUtensorMap &k2, const CUtensorMap &v16, const PrefillParams &p,
+                           cudaStream_t stream, int *launches, const ProfileEvents &ev);
+
+// bf16 V [B, N, H_V, 128] (strided) -> contiguous fp16 copy in `dst`.
+cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, void *dst, int B,
+                            int N, int H_V, int32_t *dev_status, cudaStream_t stream,
+                            int *launches);
+
+struct DecodeParams {
+    int B, H, L;
+    int splits, chunk;    // keys per split (multiple of 64)
+    float scale_log2, eps;
+    int apply_norm;
+    const void *q1, *q2, *k1, *k2, *v;
+    int64_t q1_sb, q1_sh, q2_sb, q2_sh;
+    int64_t k1_sb, k1_sh, k1_sl, k2_sb, k2_sh, k2_sl, v_sb, v_sh, v_sl;
+    void *out;
+    int64_t out_sb, out_sh;
+    const int32_t *kv_len;
+    const float *lambda, *gain;
+    float *partials;      // [B*H][splits][4 + 2*128] fp32
+    int32_t *dev_status;
+};
+
+// Floats of one split's partial state: m1, l1, m2, l2, acc1[128], acc2[128].
+constexpr int kDecodePartialFloats = 4 + 2 * 128;
+constexpr int kDecodeMaxChunk = 2048;
+
+cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream, int *launches,
+                          const ProfileEvents &ev);
+
+}  // namespace da

@@ -1,0 +1,478 @@
+// prefill_sm100.cu -- causal differential-attention prefill on sm_100a.
+//
+// Computes, per (b, h) and 128-row query tile, the two softmax maps of
+// differential attention (Motif 2.6B explainer, section "Differential
+// attention": attn = [softmax(Q1 K1^T) - lambda softmax(Q2 K2^T)] V) with an
+// online softmax for each map, and finishes with the subtraction and the norm
+// after it (same page, figure 1: GroupNorm after the subtraction, read as a
+// per-head RMS norm with gain).
+//
+// One CTA per (b, h, query tile), 384 threads, one CTA per SM:
+//   warp 0        TMA producer: Q1/Q2 once, then K1/K2/V per 128-key tile
+//                 into a 3-stage ring (64 KB per stage).
+//   warp 1        MMA issuer (one thread): S1 = Q1 K1^T and S2 = Q2 K2^T
+//                 (bf16, fp32 accumulate in TMEM), then O1 += P1 V and
+//                 O2 += P2 V with P read from TMEM and V (fp16) from the same
+//                 shared-memory tile for both maps.
+//   warps 4-7     softmax of map 1 (one thread per query row) and the
+//                 epilogue: D = O1/l1 - lambda O2/l2, RMS norm, gain, bf16.
+//   warps 8-11    softmax of map 2.
+// TMEM (512 columns): O1 [0,128) O2 [128,256) S1/P1 [256,384) S2/P2 [384,512).
+// P (fp16, two per column) overwrites the first 64 columns of its S.
+//
+// The MMA issue order S1_0 S2_0 | PV1_0 S1_1 PV2_0 S2_1 | PV1_1 S1_2 ... makes
+// every "S_t ready" commit also certify that the previous P_t.V product has
+// finished, so the softmax thread may rescale O_t and overwrite P_t as soon as
+// it sees S_t.  The softmax keeps a stale row maximum until the new one
+// exceeds it by more than 2^8 (P stays <= 256, exact enough in fp16), so O is
+// rescaled only when the maximum really moves.
+//
+// Every wait is bounded (PrefillParams::timeout_ns); on expiry the CTA raises
+// an abort flag, reports DIFFATTN_ERR_TIMEOUT, drains its own TMA loads and
+// MMAs, frees TMEM and exits without storing.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace da {
+namespace {
+
+constexpr int BM = 128;   // query rows per tile (MMA M)
+constexpr int BN = 128;   // keys per KV tile (MMA N of S, K of P.V)
+constexpr int HD = 64;    // Q/K head dim
+constexpr int HDV = 128;  // V head dim (MMA N of P.V)
+constexpr int STAGES = 3;
+constexpr int NTHREADS = 384;
+
+constexpr uint32_t Q_BYTES = BM * HD * 2;           // 16 KB
+constexpr uint32_t K_BYTES = BN * HD * 2;           // 16 KB
+constexpr uint32_t VHALF_BYTES = BN * 64 * 2;       // 16 KB: 64 of the 128 V columns
+constexpr uint32_t V_BYTES = 2 * VHALF_BYTES;       // 32 KB
+constexpr uint32_t STAGE_BYTES = 2 * K_BYTES + V_BYTES;
+
+constexpr uint32_t OFF_Q1 = 0;
+constexpr uint32_t OFF_Q2 = Q_BYTES;
+constexpr uint32_t OFF_STAGE0 = 2 * Q_BYTES;
+constexpr uint32_t OFF_BARS = OFF_STAGE0 + STAGES * STAGE_BYTES;
+// barriers: q, full[S], empty[S], s1, s2, p1, p2, o
+constexpr int NBARS = 1 + 2 * STAGES + 5;
+constexpr uint32_t OFF_TMEM_PTR = OFF_BARS + NBARS * 8;
+constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
+constexpr uint32_t OFF_L2 = OFF_ABORT + 12;  // 16-byte aligned
+constexpr uint32_t SMEM_USED = OFF_L2 + BM * 4;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
+
+constexpr uint32_t TM_O1 = 0, TM_O2 = 128, TM_S1 = 256, TM_S2 = 384;
+constexpr uint32_t TMEM_COLS = 512;
+
+// P.V MMAs read a stale-max P of at most 2^RESCALE_THRESHOLD.
+constexpr float RESCALE_THRESHOLD = 8.0f;
+
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(OFF_STAGE0 % 1024 == 0 && STAGE_BYTES % 1024 == 0, "SW128 atoms need 1 KB alignment");
+
+struct Work {
+    int b, h, qt;
+};
+
+// Map the linear CTA index to (b, h, query tile).  (b, h) pairs are taken in
+// groups of heads_per_group so that the CTAs running at the same time share
+// K/V tiles in L2; inside a group the longest (latest) query tiles go first.
+__device__ __forceinline__ Work work_of(int idx, const PrefillParams &p)
+{
+    const int BH = p.B * p.H, G = p.heads_per_group, nq = p.num_qt;
+    const int full = BH / G, per_group = G * nq;
+    int bh, qt;
+    if (idx < full * per_group) {
+        const int g = idx / per_group, r = idx - g * per_group;
+        qt = nq - 1 - r / G;
+        bh = g * G + r % G;
+    } else {
+        const int r = idx - full * per_group, tail = BH - full * G;
+        qt = nq - 1 - r / tail;
+        bh = full * G + r % tail;
+    }
+    return Work{bh / p.H, bh % p.H, qt};
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
+{
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ uint32_t pack_bf162(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Softmax of one map for one KV tile, for the query row this thread owns.
+// Reads S (fp32) from TMEM, updates the running max / sum, rescales the O row
+// when the max moved, writes P (fp16) over the first 64 S columns.
+__device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, int j, int limit,
+                                             float scale_log2, float &m_run, float &l_run)
+{
+    uint32_t v[4][32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, v[c]);
+    tmem_wait_ld();
+
+    float tmax = -INFINITY;
+    if (limit >= BN - 1) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float x = __uint_as_float(v[c][i]) * scale_log2;
+                v[c][i] = __float_as_uint(x);
+                tmax = fmaxf(tmax, x);
+            }
+    } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                float x = __uint_as_float(v[c][i]) * scale_log2;
+                if (32 * c + i > limit) x = -INFINITY;
+                v[c][i] = __float_as_uint(x);
+                tmax = fmaxf(tmax, x);
+            }
+    }
+
+    const bool need = tmax > m_run + RESCALE_THRESHOLD;
+    const float m_new = need ? tmax : m_run;
+    const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;  // ex2(-inf) = 0
+    if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + 32 * c, o);
+        }
+    }
+    l_run *= alpha;
+    m_run = m_new;
+    const float m_sub = (m_run == -INFINITY) ? 0.0f : m_run;
+
+    float rs = 0.0f;
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int c = 2 * h2 + (i >> 4), e = (2 * i) & 31;
+            const float p0 = ex2_approx(__uint_as_float(v[c][e]) - m_sub);
+            const float p1 = ex2_approx(__uint_as_float(v[c][e + 1]) - m_sub);
+            rs += p0 + p1;
+            pk[i] = pack_half2(p0, p1);
+        }
+        tmem_st32(tS + 32 * h2, pk);
+    }
+    l_run += rs;
+    tmem_wait_st();
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_q1, const __grid_constant__ CUtensorMap tm_q2,
+                   const __grid_constant__ CUtensorMap tm_k1, const __grid_constant__ CUtensorMap tm_k2,
+                   const __grid_constant__ CUtensorMap tm_v, const PrefillParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    const uint32_t sbase = smem_addr(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const Work w = work_of(blockIdx.x, p);
+    const int nh = w.h / (p.H / p.H_N), vh = w.h / (p.H / p.H_V);
+    const int q0 = w.qt * BM;
+    const int nkv = p.causal ? w.qt + 1 : (p.N + BN - 1) / BN;
+
+    const uint32_t bar_q = sbase + OFF_BARS;
+    auto bar_full = [&](int s) { return sbase + OFF_BARS + 8 * (1 + s); };
+    auto bar_empty = [&](int s) { return sbase + OFF_BARS + 8 * (1 + STAGES + s); };
+    const uint32_t bar_s1 = sbase + OFF_BARS + 8 * (1 + 2 * STAGES);
+    const uint32_t bar_s2 = bar_s1 + 8, bar_p1 = bar_s1 + 16, bar_p2 = bar_s1 + 24;
+    const uint32_t bar_o = bar_s1 + 32;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_ABORT);
+    uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + OFF_TMEM_PTR);
+    float *sL2 = reinterpret_cast<float *>(smem + OFF_L2);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(bar_full(s), 1);
+            mbar_init(bar_empty(s), 1);
+        }
+        mbar_init(bar_s1, 1);
+        mbar_init(bar_s2, 1);
+        mbar_init(bar_p1, 128);
+        mbar_init(bar_p2, 128);
+        mbar_init(bar_o, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(sbase + OFF_TMEM_PTR, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_ptr;
+    const uint64_t lim = p.timeout_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tensormap(&tm_q1);
+            prefetch_tensormap(&tm_q2);
+            prefetch_tensormap(&tm_k1);
+            prefetch_tensormap(&tm_k2);
+            prefetch_tensormap(&tm_v);
+            const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
+            mbar_arrive_expect_tx(bar_q, 2 * Q_BYTES);
+            tma_load_4d(sbase + OFF_Q1, &tm_q1, bar_q, 0, q0, w.h, w.b, stream);
+            tma_load_4d(sbase + OFF_Q2, &tm_q2, bar_q, 0, q0, nh, w.b, stream);
+            int issued = 0;
+            for (int j = 0; j < nkv; ++j) {
+                const int s = j % STAGES;
+                if (j >= STAGES && !mbar_wait(bar_empty(s), ((j / STAGES) - 1) & 1, abort_flag, lim))
+                    break;
+                const uint32_t st = sbase + OFF_STAGE0 + s * STAGE_BYTES;
+                const int k0 = j * BN;
+                mbar_arrive_expect_tx(bar_full(s), STAGE_BYTES);
+                tma_load_4d(st, &tm_k1, bar_full(s), 0, k0, w.h, w.b, keep);
+                tma_load_4d(st + K_BYTES, &tm_k2, bar_full(s), 0, k0, nh, w.b, keep);
+                tma_load_4d(st + 2 * K_BYTES, &tm_v, bar_full(s), 0, k0, vh, w.b, keep);
+                tma_load_4d(st + 2 * K_BYTES + VHALF_BYTES, &tm_v, bar_full(s), 64, k0, vh, w.b, keep);
+                issued = j + 1;
+            }
+            // No load of ours may land after the CTA has gone: wait for all of them.
+            bool drained = mbar_wait_drain(bar_q, 0, lim);
+            for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+                drained &= mbar_wait_drain(bar_full(j % STAGES), (j / STAGES) & 1, lim);
+            if (!drained) *abort_flag = 1;
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t ID_S = idesc_f16(1, 1, 0, BM, BN);    // bf16 x bf16, both K-major
+            constexpr uint32_t ID_PV = idesc_f16(0, 0, 1, BM, HDV);  // f16 x f16, B (V) MN-major
+            auto issue_s = [&](int t, int s) {
+                const uint32_t qa = sbase + (t ? OFF_Q2 : OFF_Q1);
+                const uint32_t ka = sbase + OFF_STAGE0 + s * STAGE_BYTES + (t ? K_BYTES : 0);
+                const uint32_t d = tbase + (t ? TM_S2 : TM_S1);
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; ++kk)
+                    mma_ss(d, smem_desc_sw128(qa + 32 * kk, 16, 1024),
+                           smem_desc_sw128(ka + 32 * kk, 16, 1024), ID_S, kk > 0);
+            };
+            auto issue_pv = [&](int t, int s, bool acc) {
+                const uint32_t va = sbase + OFF_STAGE0 + s * STAGE_BYTES + 2 * K_BYTES;
+                const uint32_t d = tbase + (t ? TM_O2 : TM_O1);
+                const uint32_t a = tbase + (t ? TM_S2 : TM_S1);
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    mma_ts(d, a + 8 * kk, smem_desc_sw128(va + 2048 * kk, VHALF_BYTES, 1024), ID_PV,
+                           (acc || kk > 0) ? 1u : 0u);
+            };
+            bool ok = mbar_wait(bar_q, 0, abort_flag, lim);
+            tc_fence_after();
+            if (ok) ok = mbar_wait(bar_full(0), 0, abort_flag, lim);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                mma_commit(bar_s1);
+                issue_s(1, 0);
+                mma_commit(bar_s2);
+            }
+            for (int j = 0; ok && j < nkv; ++j) {
+                const int s = j % STAGES;
+                if (!(ok = mbar_wait(bar_p1, j & 1, abort_flag, lim))) break;
+                tc_fence_after();
+                issue_pv(0, s, j > 0);
+                const bool more = j + 1 < nkv;
+                const int s1 = (j + 1) % STAGES;
+                if (more) {
+                    if (!(ok = mbar_wait(bar_full(s1), ((j + 1) / STAGES) & 1, abort_flag, lim))) break;
+                    tc_fence_after();
+                    issue_s(0, s1);
+                    mma_commit(bar_s1);
+                }
+                if (!(ok = mbar_wait(bar_p2, j & 1, abort_flag, lim))) break;
+                tc_fence_after();
+                issue_pv(1, s, j > 0);
+                mma_commit(bar_empty(s));
+                if (more) {
+                    issue_s(1, s1);
+                    mma_commit(bar_s2);
+                }
+            }
+            mma_commit(bar_o);
+            // Nothing of ours may still run on the tensor cores at teardown.
+            if (!mbar_wait_drain(bar_o, 0, lim)) *abort_flag = 1;
+        }
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ softmax
+        const int t = (warp >= 8) ? 1 : 0;
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+        const uint32_t tS = tbase + lane_off + (t ? TM_S2 : TM_S1);
+        const uint32_t tO = tbase + lane_off + (t ? TM_O2 : TM_O1);
+        const uint32_t bar_s = t ? bar_s2 : bar_s1, bar_p = t ? bar_p2 : bar_p1;
+        const int qrow = q0 + r;
+        float m_run = -INFINITY, l_run = 0.0f;
+        for (int j = 0; j < nkv; ++j) {
+            if (!mbar_wait(bar_s, j & 1, abort_flag, lim)) break;
+            tc_fence_after();
+            const int k0 = j * BN;
+            const int limit = p.causal ? qrow - k0 : p.N - 1 - k0;
+            softmax_tile(tS, tO, j, limit, p.scale_log2, m_run, l_run);
+            tc_fence_before();
+            mbar_arrive(bar_p);
+        }
+        if (t == 1) {
+            sL2[r] = l_run;
+            named_barrier_sync(1, 256);
+        } else {
+            named_barrier_sync(1, 256);
+            const float l2 = sL2[r];
+            const bool ok = mbar_wait(bar_o, 0, abort_flag, lim);
+            tc_fence_after();
+            if (ok && !*abort_flag) {
+                // ---------------------------------------------------- epilogue
+                const float lam = p.lambda[w.h];
+                const float inv1 = 1.0f / l_run, c2 = lam / l2;
+                const uint32_t tO1 = tbase + lane_off + TM_O1, tO2 = tbase + lane_off + TM_O2;
+                float rn = 1.0f;
+                if (p.apply_norm) {
+                    float ss = 0.0f;
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t a[32], bb[32];
+                        tmem_ld32(tO1 + 32 * c, a);
+                        tmem_ld32(tO2 + 32 * c, bb);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float dd = __uint_as_float(a[i]) * inv1 - __uint_as_float(bb[i]) * c2;
+                            ss += dd * dd;
+                        }
+                    }
+                    rn = rsqrtf(ss * (1.0f / HDV) + p.eps);
+                }
+                const float *gain = p.gain ? p.gain + (size_t)w.h * HDV : nullptr;
+                uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) +
+                                2 * ((int64_t)w.b * p.out_sb + (int64_t)qrow * p.out_sn +
+                                     (int64_t)w.h * p.out_sh);
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t a[32], bb[32];
+                    tmem_ld32(tO1 + 32 * c, a);
+                    tmem_ld32(tO2 + 32 * c, bb);
+                    tmem_wait_ld();
+                    uint32_t y[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float y0 = (__uint_as_float(a[2 * i]) * inv1 - __uint_as_float(bb[2 * i]) * c2) * rn;
+                        float y1 = (__uint_as_float(a[2 * i + 1]) * inv1 - __uint_as_float(bb[2 * i + 1]) * c2) * rn;
+                        if (gain) {
+                            y0 *= __ldg(gain + 32 * c + 2 * i);
+                            y1 *= __ldg(gain + 32 * c + 2 * i + 1);
+                        }
+                        y[i] = pack_bf162(y0, y1);
+                    }
+                    if (qrow < p.N) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + 64 * c);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_flag) report_error(p.dev_status, DIFFATTN_ERR_TIMEOUT);
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tbase, TMEM_COLS);
+    }
+}
+
+__global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb, int64_t sn,
+                                int64_t sh, __half *__restrict__ dst, int B, int N, int H_V,
+                                int32_t *dev_status)
+{
+    // One thread per 8 consecutive V elements (16 bytes in, 16 bytes out).
+    const int64_t total = (int64_t)B * N * H_V * (HDV / 8);
+    bool overflow = false;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int c8 = int(i % (HDV / 8));
+        const int64_t row = i / (HDV / 8);
+        const int hv = int(row % H_V);
+        const int64_t bn = row / H_V;
+        const int n = int(bn % N), b = int(bn / N);
+        const uint4 src = __ldg(reinterpret_cast<const uint4 *>(v + b * sb + n * sn + hv * sh + 8 * c8));
+        const uint32_t in[4] = {src.x, src.y, src.z, src.w};
+        uint32_t out[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&in[k]);
+            const float2 f = __bfloat1622float2(x);
+            overflow |= fabsf(f.x) > 65504.0f || fabsf(f.y) > 65504.0f;
+            out[k] = pack_half2(f.x, f.y);
+        }
+        reinterpret_cast<uint4 *>(dst)[i] = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+    if (overflow) report_error(dev_status, DIFFATTN_ERR_UNSUPPORTED);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const CUtensorMap &k1,
+                           const CUtensorMap &k2, const CUtensorMap &v16, const PrefillParams &p,
+                           cudaStream_t stream, int *launches, const ProfileEvents &ev)
+{
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int grid = p.B * p.H * p.num_qt;
+    if (grid == 0) return cudaSuccess;
+    if (ev.start) cudaEventRecord(ev.start, stream);
+    prefill_kernel<<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, p);
+    ++*launches;
+    if (ev.stop) cudaEventRecord(ev.stop, stream);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, void *dst, int B,
+                            int N, int H_V, int32_t *dev_status, cudaStream_t stream, int *launches)
+{
+    const int64_t total = (int64_t)B * N * H_V * (HDV / 8);
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    int blocks = (int)((total + threads - 1) / threads);
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    v_to_f16_kernel<<<blocks, threads, 0, stream>>>(static_cast<const __nv_bfloat16 *>(v), sb, sn,
+                                                    sh, static_cast<__half *>(dst), B, N, H_V,
+                                                    dev_status);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+}  // namespace da

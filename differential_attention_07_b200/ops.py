@@ -1,0 +1,299 @@
+"""Python binding of libdiffattn (ctypes).  Argument marshalling only.
+
+Every step of the computation runs in the CUDA kernels behind the C ABI
+declared in include/diffattn.h; this module checks tensor properties, fills
+the argument structs with raw device pointers, strides and the current CUDA
+stream, and allocates the caller-owned workspace with torch.  There is no CPU
+fallback: without the built library or a CUDA device every call raises.
+
+Functions (same names as the C entry points):
+    diffattn_fwd(q1, q2, k1, k2, v, lam, gain=None, ...)          -> out
+    diffattn_grouped_fwd(q1, q2, k1, k2, v, lam, gain=None, ...)  -> out
+    diffattn_decode(q1, q2, k1, k2, v, lam, gain=None, ...)       -> out
+"""
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+LIB_PATH = _build.LIB
+
+DIFFATTN_FLAG_CAUSAL = 1
+DIFFATTN_FLAG_APPLY_NORM = 2
+
+STATUS = {
+    0: "DIFFATTN_OK",
+    1: "DIFFATTN_ERR_INVALID_ARG",
+    2: "DIFFATTN_ERR_UNSUPPORTED",
+    3: "DIFFATTN_ERR_ALIGNMENT",
+    4: "DIFFATTN_ERR_WORKSPACE",
+    5: "DIFFATTN_ERR_CUDA",
+    6: "DIFFATTN_ERR_TIMEOUT",
+}
+
+EXPORTED = [
+    "diffattn_fwd", "diffattn_grouped_fwd", "diffattn_fwd_workspace_size", "diffattn_fwd_validate",
+    "diffattn_decode", "diffattn_decode_workspace_size", "diffattn_decode_num_splits",
+    "diffattn_decode_validate", "diffattn_status_str", "diffattn_last_launch_count",
+    "diffattn_set_profile_events",
+]
+
+_i64 = ctypes.c_int64
+_p = ctypes.c_void_p
+_S3 = _i64 * 3
+_S2 = _i64 * 2
+
+
+class FwdArgs(ctypes.Structure):
+    """Mirror of struct diffattn_fwd_args."""
+    _fields_ = [
+        ("B", _i64), ("N", _i64), ("H", _i64), ("H_N", _i64), ("H_V", _i64),
+        ("d", _i64), ("dv", _i64),
+        ("scale", ctypes.c_float), ("eps", ctypes.c_float),
+        ("flags", ctypes.c_uint32), ("timeout_ms", ctypes.c_uint32),
+        ("q1", _p), ("q1_stride", _S3),
+        ("q2", _p), ("q2_stride", _S3),
+        ("k1", _p), ("k1_stride", _S3),
+        ("k2", _p), ("k2_stride", _S3),
+        ("v", _p), ("v_stride", _S3),
+        ("out", _p), ("out_stride", _S3),
+        ("lambda_", _p), ("gain", _p), ("dev_status", _p),
+    ]
+
+
+class DecodeArgs(ctypes.Structure):
+    """Mirror of struct diffattn_decode_args."""
+    _fields_ = [
+        ("B", _i64), ("H", _i64), ("L", _i64),
+        ("d", _i64), ("dv", _i64),
+        ("scale", ctypes.c_float), ("eps", ctypes.c_float),
+        ("flags", ctypes.c_uint32), ("num_splits", ctypes.c_int32),
+        ("q1", _p), ("q1_stride", _S2),
+        ("q2", _p), ("q2_stride", _S2),
+        ("k1", _p), ("k1_stride", _S3),
+        ("k2", _p), ("k2_stride", _S3),
+        ("v", _p), ("v_stride", _S3),
+        ("out", _p), ("out_stride", _S2),
+        ("kv_len", _p), ("lambda_", _p), ("gain", _p), ("dev_status", _p),
+    ]
+
+
+class DiffAttnError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+_LIB = None
+
+
+def lib():
+    """The loaded libdiffattn (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libdiffattn is not built ({LIB_PATH} missing); run "
+                               "`python -m differential_attention_07_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        fa, da = ctypes.POINTER(FwdArgs), ctypes.POINTER(DecodeArgs)
+        for name in ("diffattn_fwd", "diffattn_grouped_fwd"):
+            f = getattr(L, name)
+            f.argtypes = [fa, _p, ctypes.c_size_t, _p]
+            f.restype = ctypes.c_int
+        L.diffattn_fwd_workspace_size.argtypes = [fa]
+        L.diffattn_fwd_workspace_size.restype = ctypes.c_size_t
+        L.diffattn_fwd_validate.argtypes = [fa, ctypes.c_int]
+        L.diffattn_fwd_validate.restype = ctypes.c_int
+        L.diffattn_decode.argtypes = [da, _p, ctypes.c_size_t, _p]
+        L.diffattn_decode.restype = ctypes.c_int
+        L.diffattn_decode_workspace_size.argtypes = [_i64, _i64, _i64, ctypes.c_int32]
+        L.diffattn_decode_workspace_size.restype = ctypes.c_size_t
+        L.diffattn_decode_num_splits.argtypes = [_i64, _i64, _i64, ctypes.c_int32]
+        L.diffattn_decode_num_splits.restype = ctypes.c_int32
+        L.diffattn_decode_validate.argtypes = [da]
+        L.diffattn_decode_validate.restype = ctypes.c_int
+        L.diffattn_status_str.argtypes = [ctypes.c_int]
+        L.diffattn_status_str.restype = ctypes.c_char_p
+        L.diffattn_last_launch_count.argtypes = []
+        L.diffattn_last_launch_count.restype = ctypes.c_int32
+        L.diffattn_set_profile_events.argtypes = [_p, _p]
+        L.diffattn_set_profile_events.restype = None
+        _LIB = L
+    return _LIB
+
+
+def last_launch_count() -> int:
+    """Kernels launched by the last successful call on this thread."""
+    return int(lib().diffattn_last_launch_count())
+
+
+def set_profile_events(start=None, stop=None):
+    """Record torch.cuda.Event `start` / `stop` around the main kernel of every
+    later call on this thread (None, None switches it off)."""
+    lib().diffattn_set_profile_events(
+        ctypes.c_void_p(start.cuda_event) if start is not None else None,
+        ctypes.c_void_p(stop.cuda_event) if stop is not None else None)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check_bf16(name, t, ndim):
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if t.stride(-1) != 1:
+        raise ValueError(f"{name}: last dimension must be contiguous")
+
+
+def _stream_ptr(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _fwd_args(q1, q2, k1, k2, v, lam, gain, out, *, scale, eps, causal, apply_norm,
+              timeout_ms, dev_status):
+    for n, t in (("q1", q1), ("q2", q2), ("k1", k1), ("k2", k2), ("v", v), ("out", out)):
+        _check_bf16(n, t, 4)
+    B, N, H, d = q1.shape
+    a = FwdArgs()
+    a.B, a.N, a.H, a.H_N, a.H_V = B, N, H, q2.shape[2], v.shape[2]
+    a.d, a.dv = d, v.shape[3]
+    a.scale, a.eps = float(scale), float(eps)
+    a.flags = (DIFFATTN_FLAG_CAUSAL if causal else 0) | (DIFFATTN_FLAG_APPLY_NORM if apply_norm else 0)
+    a.timeout_ms = int(timeout_ms)
+    for n, t in (("q1", q1), ("q2", q2), ("k1", k1), ("k2", k2), ("v", v), ("out", out)):
+        setattr(a, n, t.data_ptr())
+        setattr(a, n + "_stride", _S3(*t.stride()[:3]))
+    if lam.dtype != torch.float32 or lam.shape != (H,):
+        raise ValueError("lam must be float32 [H]")
+    a.lambda_ = lam.data_ptr()
+    if gain is not None:
+        if gain.dtype != torch.float32 or tuple(gain.shape) != (H, a.dv) or not gain.is_contiguous():
+            raise ValueError("gain must be contiguous float32 [H, dv]")
+        a.gain = gain.data_ptr()
+    a.dev_status = dev_status.data_ptr() if dev_status is not None else None
+    return a
+
+
+def _check_shapes_fwd(q1, q2, k1, k2, v):
+    B, N, H, d = q1.shape
+    if k1.shape != q1.shape:
+        raise ValueError("k1 must have q1's shape")
+    if q2.shape != k2.shape or q2.shape[:2] != (B, N) or q2.shape[3] != d:
+        raise ValueError("q2/k2 must be [B, N, H_N, d]")
+    if v.shape[:2] != (B, N):
+        raise ValueError("v must be [B, N, H_V, dv]")
+
+
+def _run_fwd(entry, q1, q2, k1, k2, v, lam, gain, *, scale, eps, causal, apply_norm, out,
+             workspace, stream, timeout_ms, dev_status):
+    _check_shapes_fwd(q1, q2, k1, k2, v)
+    B, N, H, _ = q1.shape
+    if out is None:
+        out = torch.empty(B, N, H, v.shape[3], dtype=torch.bfloat16, device=q1.device)
+    a = _fwd_args(q1, q2, k1, k2, v, lam, gain, out, scale=scale, eps=eps, causal=causal,
+                  apply_norm=apply_norm, timeout_ms=timeout_ms, dev_status=dev_status)
+    L = lib()
+    need = L.diffattn_fwd_workspace_size(ctypes.byref(a))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q1.device)
+    st = getattr(L, entry)(ctypes.byref(a), _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    if st != 0:
+        raise DiffAttnError(st, entry)
+    return out
+
+
+def diffattn_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,
+                 apply_norm=True, out=None, workspace=None, stream=None, timeout_ms=0,
+                 dev_status=None):
+    """Differential-attention prefill.  q1,q2,k1,k2 [B,N,H,64], v [B,N,H,128]
+    bf16 CUDA tensors (token-major, last dim contiguous); lam [H] fp32; gain
+    [H,128] fp32 or None.  Returns out [B,N,H,128] bf16."""
+    return _run_fwd("diffattn_fwd", q1, q2, k1, k2, v, lam, gain, scale=scale, eps=eps,
+                    causal=causal, apply_norm=apply_norm, out=out, workspace=workspace,
+                    stream=stream, timeout_ms=timeout_ms, dev_status=dev_status)
+
+
+def diffattn_grouped_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,
+                         apply_norm=True, out=None, workspace=None, stream=None, timeout_ms=0,
+                         dev_status=None):
+    """Grouped prefill: q1,k1 [B,N,H,64]; q2,k2 [B,N,H_N,64]; v [B,N,H_V,128];
+    signal head h uses noise head h // (H // H_N) and V head h // (H // H_V)."""
+    return _run_fwd("diffattn_grouped_fwd", q1, q2, k1, k2, v, lam, gain, scale=scale, eps=eps,
+                    causal=causal, apply_norm=apply_norm, out=out, workspace=workspace,
+                    stream=stream, timeout_ms=timeout_ms, dev_status=dev_status)
+
+
+def fwd_workspace_size(B, N, H, H_V=None):
+    a = FwdArgs()
+    a.B, a.N, a.H, a.H_V, a.d, a.dv = B, N, H, H_V or H, 64, 128
+    return int(lib().diffattn_fwd_workspace_size(ctypes.byref(a)))
+
+
+def decode_workspace_size(B, H, L, num_splits=0):
+    return int(lib().diffattn_decode_workspace_size(B, H, L, num_splits))
+
+
+def decode_num_splits(B, H, L, num_splits=0):
+    return int(lib().diffattn_decode_num_splits(B, H, L, num_splits))
+
+
+def _decode_args(q1, q2, k1, k2, v, lam, gain, out, *, kv_len, num_splits, scale, eps,
+                 apply_norm, dev_status):
+    for n, t, nd in (("q1", q1, 3), ("q2", q2, 3), ("k1", k1, 4), ("k2", k2, 4), ("v", v, 4),
+                     ("out", out, 3)):
+        _check_bf16(n, t, nd)
+    B, H, L, d = k1.shape
+    if q1.shape != (B, H, d) or q2.shape != (B, H, d) or k2.shape != k1.shape:
+        raise ValueError("decode: q [B,H,d], k [B,H,L,d] expected")
+    if v.shape[:3] != (B, H, L):
+        raise ValueError("decode: v [B,H,L,dv] expected")
+    a = DecodeArgs()
+    a.B, a.H, a.L, a.d, a.dv = B, H, L, d, v.shape[3]
+    a.scale, a.eps = float(scale), float(eps)
+    a.flags = DIFFATTN_FLAG_APPLY_NORM if apply_norm else 0
+    a.num_splits = int(num_splits)
+    for n, t in (("q1", q1), ("q2", q2), ("out", out)):
+        setattr(a, n, t.data_ptr())
+        setattr(a, n + "_stride", _S2(*t.stride()[:2]))
+    for n, t in (("k1", k1), ("k2", k2), ("v", v)):
+        setattr(a, n, t.data_ptr())
+        setattr(a, n + "_stride", _S3(*t.stride()[:3]))
+    if kv_len is not None:
+        if kv_len.dtype != torch.int32 or kv_len.shape != (B,):
+            raise ValueError("kv_len must be int32 [B]")
+        a.kv_len = kv_len.data_ptr()
+    if lam.dtype != torch.float32 or lam.shape != (H,):
+        raise ValueError("lam must be float32 [H]")
+    a.lambda_ = lam.data_ptr()
+    if gain is not None:
+        if gain.dtype != torch.float32 or tuple(gain.shape) != (H, a.dv) or not gain.is_contiguous():
+            raise ValueError("gain must be contiguous float32 [H, dv]")
+        a.gain = gain.data_ptr()
+    a.dev_status = dev_status.data_ptr() if dev_status is not None else None
+    return a
+
+
+def diffattn_decode(q1, q2, k1, k2, v, lam, gain=None, *, kv_len=None, num_splits=0, scale=0.125,
+                    eps=1e-5, apply_norm=True, out=None, workspace=None, stream=None,
+                    dev_status=None):
+    """Single-query decode.  q1,q2 [B,H,64]; k1,k2 [B,H,L,64]; v [B,H,L,128]
+    bf16 CUDA tensors; kv_len int32 [B] or None.  Returns out [B,H,128] bf16."""
+    B, H, L, _ = k1.shape
+    if out is None:
+        out = torch.empty(B, H, v.shape[3], dtype=torch.bfloat16, device=q1.device)
+    a = _decode_args(q1, q2, k1, k2, v, lam, gain, out, kv_len=kv_len, num_splits=num_splits,
+                     scale=scale, eps=eps, apply_norm=apply_norm, dev_status=dev_status)
+    Lb = lib()
+    need = Lb.diffattn_decode_workspace_size(B, H, L, int(num_splits))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q1.device)
+    st = Lb.diffattn_decode(ctypes.byref(a), _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    if st != 0:
+        raise DiffAttnError(st, "diffattn_decode")
+    return out

@@ -1,0 +1,164 @@
+/*
+ * diffattn.h -- C ABI of libdiffattn, the B200 (sm_100a) differential-attention
+ * forward pass.
+ *
+ * The operation (Motif 2.6B explainer, section "Differential attention" and
+ * figure 1): per batch b, signal head h and query row i,
+ *
+ *   A_t = softmax(scale * Q_t[i] K_t^T) V          for the two maps t = 1, 2
+ *   D   = A_1 - lambda[h] * A_2                      (the subtraction)
+ *   Y   = D / sqrt(mean_c D[c]^2 + eps) * gain[h]    (the norm after it)
+ *
+ * with causal masking (key j is visible to query i when j <= i).  The pages
+ * call the norm "GroupNorm"; this library reads it as an RMS norm over each
+ * head's dv channels of each token, with a learned per-channel gain.
+ * The grouped variant (Motif 3 summary, section 2.2, eq. "grouped differential
+ * output" D_t = H_S,t - lambda_t (.) Repeat_g(H_N,t)) takes map 2 of signal
+ * head h from noise head h / (H / H_N) and V from V head h / (H / H_V).
+ *
+ * Conventions for every entry point:
+ *  - Element type of Q/K/V/out is bf16.  Only d = 64 (Q/K head dim) and
+ *    dv = 128 (V head dim) are built; anything else is DIFFATTN_ERR_UNSUPPORTED.
+ *  - Tensor pointers are DEVICE pointers owned by the caller.  Every base
+ *    pointer must be 16-byte aligned and every stride a multiple of 8 elements
+ *    (16 bytes); the last dimension is contiguous.  Strides are in elements.
+ *  - The library allocates no device memory.  Scratch is the caller's
+ *    `workspace` (device memory, 256-byte aligned) of at least the size the
+ *    matching *_workspace_size function returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *    is the legacy default stream).  Nothing is synchronised.
+ *  - Argument errors are reported by the return value before anything is
+ *    launched.  Errors that only the device can see (a bounded wait that ran
+ *    out, a V value outside the fp16 range, a kv_len out of range) are written
+ *    to `dev_status` (device int32, nullable): the first error code wins, 0
+ *    means none.  The caller reads it after synchronising.  A kernel that sees
+ *    such an error finishes without writing the rows it could not compute.
+ *  - Every device-side wait is bounded by `timeout_ms` (0 selects 2000 ms).
+ */
+#ifndef DIFFATTN_H
+#define DIFFATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum diffattn_status {
+    DIFFATTN_OK = 0,
+    DIFFATTN_ERR_INVALID_ARG = 1,  /* null pointer, bad size, inconsistent heads */
+    DIFFATTN_ERR_UNSUPPORTED = 2,  /* head dims other than 64 / 128, V beyond fp16 range */
+    DIFFATTN_ERR_ALIGNMENT = 3,    /* pointer not 16-byte aligned or stride not 8-element */
+    DIFFATTN_ERR_WORKSPACE = 4,    /* workspace missing or too small */
+    DIFFATTN_ERR_CUDA = 5,         /* a CUDA runtime / driver call failed */
+    DIFFATTN_ERR_TIMEOUT = 6       /* (device) a bounded wait ran out */
+} diffattn_status;
+
+#define DIFFATTN_FLAG_CAUSAL 1u      /* key j visible to query i iff j <= i */
+#define DIFFATTN_FLAG_APPLY_NORM 2u  /* apply the RMS norm + gain; else write D */
+
+/* Prefill arguments.  Layout of each tensor: element (b, n, head, c) sits at
+ * ptr + b*stride[0] + n*stride[1] + head*stride[2] + c.
+ *   q1, k1: [B, N, H,   64]     q2, k2: [B, N, H_N, 64]
+ *   v:      [B, N, H_V, 128]    out:    [B, N, H,   128]
+ *   lambda: [H] fp32 device     gain:   [H, 128] fp32 device, or NULL for 1. */
+typedef struct diffattn_fwd_args {
+    int64_t B, N, H, H_N, H_V;
+    int64_t d, dv;
+    float scale, eps;
+    uint32_t flags;
+    uint32_t timeout_ms;
+    const void *q1; int64_t q1_stride[3];
+    const void *q2; int64_t q2_stride[3];
+    const void *k1; int64_t k1_stride[3];
+    const void *k2; int64_t k2_stride[3];
+    const void *v;  int64_t v_stride[3];
+    void *out;      int64_t out_stride[3];
+    const float *lambda;
+    const float *gain;
+    int32_t *dev_status;
+} diffattn_fwd_args;
+
+/* Causal (or full) prefill, one noise map per signal head: H_N and H_V must be
+ * 0 or equal to H.  N_q == N_k == N.  Differential attention as defined in the
+ * Motif 2.6B explainer, section "Differential attention".                    */
+diffattn_status diffattn_fwd(const diffattn_fwd_args *args, void *workspace, size_t ws_bytes,
+                             void *stream);
+
+/* Grouped prefill: H % H_N == 0 and H % H_V == 0; signal head h uses Q2/K2 of
+ * noise head h / (H / H_N) and V head h / (H / H_V) (Motif 3 summary,
+ * section 2.2).  With H_N == H_V == H it is diffattn_fwd.                    */
+diffattn_status diffattn_grouped_fwd(const diffattn_fwd_args *args, void *workspace,
+                                     size_t ws_bytes, void *stream);
+
+/* Bytes of workspace diffattn_fwd / diffattn_grouped_fwd need for `args`
+ * (an fp16 copy of V for the tensor-core P.V product).                       */
+size_t diffattn_fwd_workspace_size(const diffattn_fwd_args *args);
+
+/* Host-only argument check of a prefill call: the status diffattn_fwd (or,
+ * with grouped != 0, diffattn_grouped_fwd) would return before launching,
+ * with the workspace check skipped.  Touches no device.                      */
+diffattn_status diffattn_fwd_validate(const diffattn_fwd_args *args, int grouped);
+
+/* Single-query decode arguments.  The query of sequence b sits at position
+ * kv_len[b]-1 and attends to cached keys 0..kv_len[b]-1 (no mask needed).
+ *   q1, q2: [B, H, 64]            element (b, h, c) at ptr + b*s[0] + h*s[1] + c
+ *   k1, k2: [B, H, L, 64]         element (b, h, j, c) at ptr + b*s[0] + h*s[1] + j*s[2] + c
+ *   v:      [B, H, L, 128]
+ *   out:    [B, H, 128]
+ *   kv_len: [B] int32 device, 1 <= kv_len[b] <= L, or NULL for L.
+ *   num_splits: KV splits per (b, h); 0 picks one. */
+typedef struct diffattn_decode_args {
+    int64_t B, H, L;
+    int64_t d, dv;
+    float scale, eps;
+    uint32_t flags;         /* DIFFATTN_FLAG_APPLY_NORM; CAUSAL is ignored */
+    int32_t num_splits;
+    const void *q1; int64_t q1_stride[2];
+    const void *q2; int64_t q2_stride[2];
+    const void *k1; int64_t k1_stride[3];
+    const void *k2; int64_t k2_stride[3];
+    const void *v;  int64_t v_stride[3];
+    void *out;      int64_t out_stride[2];
+    const int32_t *kv_len;
+    const float *lambda;
+    const float *gain;
+    int32_t *dev_status;
+} diffattn_decode_args;
+
+/* Split-KV decode: a split kernel writes per-split partial softmax states
+ * (running max, sum and unnormalised V sum for both maps) into the workspace;
+ * a combine kernel merges them and applies the subtraction and the norm.    */
+diffattn_status diffattn_decode(const diffattn_decode_args *args, void *workspace,
+                                size_t ws_bytes, void *stream);
+
+/* Workspace bytes diffattn_decode needs for these sizes (num_splits 0 = the
+ * count diffattn_decode picks).                                              */
+size_t diffattn_decode_workspace_size(int64_t B, int64_t H, int64_t L, int32_t num_splits);
+
+/* The split count diffattn_decode uses for these sizes.                     */
+int32_t diffattn_decode_num_splits(int64_t B, int64_t H, int64_t L, int32_t num_splits);
+
+/* Host-only argument check of a decode call (workspace check skipped).      */
+diffattn_status diffattn_decode_validate(const diffattn_decode_args *args);
+
+/* Static, human-readable name of a status code.                              */
+const char *diffattn_status_str(diffattn_status status);
+
+/* Number of kernels the last successful call on this thread launched (for
+ * launch accounting in benchmarks).                                          */
+int32_t diffattn_last_launch_count(void);
+
+/* Timing hook for benchmarks: while set (non-NULL), every later call on this
+ * thread records `start` (a cudaEvent_t passed as void*) on its stream just
+ * before its main kernel (the prefill kernel, or the decode split kernel) and
+ * `stop` just after it, so the caller can time that kernel alone.  Pass NULL,
+ * NULL to switch it off.  The events are the caller's.                       */
+void diffattn_set_profile_events(void *start, void *stop);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIFFATTN_H */

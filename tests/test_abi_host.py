@@ -1,0 +1,171 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library must load on a machine without a GPU, export every function that
+include/*.h declares, and reject bad arguments before launching anything.
+"""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+import torch
+
+from differential_attention_07_b200 import build, ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"\b(diffattn_[a-z0-9_]+)\s*\(", src):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return ops.lib()
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = _declared_functions()
+    assert "diffattn_fwd" in names and "diffattn_decode" in names
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+    assert set(ops.EXPORTED) <= set(names)
+
+
+def test_library_is_sm100a_build():
+    src = open(os.path.join(ROOT, "differential_attention_07_b200", "build.py")).read()
+    assert "arch=compute_100a,code=sm_100a" in src
+
+
+def test_status_strings(L):
+    for code in range(7):
+        assert L.diffattn_status_str(code)
+    assert L.diffattn_status_str(6) == b"device wait timed out"
+
+
+def _fake_fwd_args(B=2, N=300, H=4, H_N=None, H_V=None, d=64, dv=128, base=1 << 20):
+    """Argument struct with plausible, 16-byte-aligned fake device addresses.
+    Only host validation ever looks at it."""
+    H_N = H_N or H
+    H_V = H_V or H
+    a = ops.FwdArgs()
+    a.B, a.N, a.H, a.H_N, a.H_V, a.d, a.dv = B, N, H, H_N, H_V, d, dv
+    a.scale, a.eps = 0.125, 1e-5
+    a.flags = ops.DIFFATTN_FLAG_CAUSAL | ops.DIFFATTN_FLAG_APPLY_NORM
+    for i, (n, h, w) in enumerate((("q1", H, d), ("q2", H_N, d), ("k1", H, d), ("k2", H_N, d),
+                                   ("v", H_V, dv), ("out", H, dv))):
+        setattr(a, n, base * (i + 1))
+        setattr(a, n + "_stride", ops._S3(N * h * w, h * w, w))
+    a.lambda_ = base * 16
+    return a
+
+
+def _v(L, a, grouped=0):
+    return L.diffattn_fwd_validate(ctypes.byref(a), grouped)
+
+
+def test_fwd_validation(L):
+    assert _v(L, _fake_fwd_args()) == 0
+    a = _fake_fwd_args(d=32)
+    assert _v(L, a) == 2                          # unsupported head dim
+    a = _fake_fwd_args(dv=64)
+    assert _v(L, a) == 2
+    a = _fake_fwd_args()
+    a.q1 = 0
+    assert _v(L, a) == 1                          # null pointer
+    a = _fake_fwd_args()
+    a.k2 = a.k2 + 8
+    assert _v(L, a) == 3                          # misaligned
+    a = _fake_fwd_args()
+    a.v_stride[1] = 130
+    assert _v(L, a) == 3                          # stride not a multiple of 8
+    a = _fake_fwd_args()
+    a.lambda_ = 0
+    assert _v(L, a) == 1
+    a = _fake_fwd_args()
+    a.scale = 0.0
+    assert _v(L, a) == 1
+    a = _fake_fwd_args()
+    a.flags = 8
+    assert _v(L, a) == 1
+    a = _fake_fwd_args(B=0)
+    a.q1 = 0
+    assert _v(L, a) == 0                          # empty batch: nothing to check
+
+
+def test_grouped_validation(L):
+    a = _fake_fwd_args(H=24, H_N=8, H_V=8)
+    assert _v(L, a, 1) == 0
+    assert _v(L, a, 0) == 1                       # ungrouped entry needs H_N == H_V == H
+    assert _v(L, _fake_fwd_args(H=24, H_N=7, H_V=8), 1) == 1
+    assert _v(L, _fake_fwd_args(H=24, H_N=8, H_V=5), 1) == 1
+
+
+def test_fwd_rejects_before_launch(L):
+    """diffattn_fwd with a bad argument or no workspace returns the error
+    without any CUDA call (this machine may have no GPU)."""
+    a = _fake_fwd_args(d=32)
+    assert L.diffattn_fwd(ctypes.byref(a), None, 0, None) == 2
+    a = _fake_fwd_args()
+    assert L.diffattn_fwd(ctypes.byref(a), None, 0, None) == 4          # workspace missing
+    need = L.diffattn_fwd_workspace_size(ctypes.byref(a))
+    assert need == 2 * 300 * 4 * 128 * 2
+    assert L.diffattn_fwd(ctypes.byref(a), ctypes.c_void_p(1 << 30), need - 1, None) == 4
+    assert L.diffattn_fwd(ctypes.byref(a), ctypes.c_void_p((1 << 30) + 16), need, None) == 3
+    assert L.diffattn_grouped_fwd(ctypes.byref(_fake_fwd_args(H=6, H_N=4)), None, 0, None) == 1
+
+
+def _fake_decode_args(B=3, H=2, L=1000, base=1 << 20):
+    a = ops.DecodeArgs()
+    a.B, a.H, a.L, a.d, a.dv = B, H, L, 64, 128
+    a.scale, a.eps, a.flags = 0.125, 1e-5, ops.DIFFATTN_FLAG_APPLY_NORM
+    a.q1, a.q1_stride = base, ops._S2(H * 64, 64)
+    a.q2, a.q2_stride = 2 * base, ops._S2(H * 64, 64)
+    a.k1, a.k1_stride = 3 * base, ops._S3(H * L * 64, L * 64, 64)
+    a.k2, a.k2_stride = 4 * base, ops._S3(H * L * 64, L * 64, 64)
+    a.v, a.v_stride = 5 * base, ops._S3(H * L * 128, L * 128, 128)
+    a.out, a.out_stride = 6 * base, ops._S2(H * 128, 128)
+    a.lambda_ = 7 * base
+    return a
+
+
+def test_decode_validation_and_workspace(L):
+    assert L.diffattn_decode_validate(ctypes.byref(_fake_decode_args())) == 0
+    a = _fake_decode_args()
+    a.k1 = a.k1 + 2
+    assert L.diffattn_decode_validate(ctypes.byref(a)) == 3
+    a = _fake_decode_args()
+    a.num_splits = -1
+    assert L.diffattn_decode_validate(ctypes.byref(a)) == 1
+    a = _fake_decode_args()
+    assert L.diffattn_decode(ctypes.byref(a), None, 0, None) == 4
+    # splits: chunks of at most 2048 keys, a multiple of 64, none empty
+    for (B, H, Lk, req) in [(64, 16, 8192, 0), (1, 16, 8192, 0), (3, 2, 1000, 0), (1, 1, 1, 0),
+                            (2, 2, 5000, 7), (1, 1, 100000, 0), (4, 4, 130, 3)]:
+        s = L.diffattn_decode_num_splits(B, H, Lk, req)
+        chunk = ((Lk + s - 1) // s + 63) // 64 * 64
+        assert s >= 1 and chunk <= max(2048, 64) and (s - 1) * chunk < Lk <= s * chunk
+        ws = L.diffattn_decode_workspace_size(B, H, Lk, req)
+        assert ws >= B * H * s * 260 * 4 and ws % 256 == 0
+    assert L.diffattn_decode_num_splits(64, 16, 8192, 0) == 4
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(ops, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(ops, "_LIB", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        ops.lib()
+
+
+def test_binding_rejects_cpu_tensor_types():
+    x = torch.zeros(1, 4, 1, 64, dtype=torch.float32)
+    with pytest.raises(TypeError):
+        ops._check_bf16("q1", x, 4)
