@@ -46,9 +46,16 @@ def causal_pairs(N):
 
 
 def prefill_flops(w):
-    """Algorithmic FLOP of one prefill call (causal pairs only)."""
+    """Algorithmic FLOP of one prefill call (causal pairs only).
+
+    Per pair: 2*64 for each score map, 2*128 for each P.V product.  In the
+    grouped form a noise map is computed once per noise head; its P.V product
+    is shared by the group when the group shares one V head (H_V == H_N),
+    otherwise each signal head multiplies it by its own V."""
     pairs = causal_pairs(w.N) if w.causal else w.N * w.N
-    return FLOP_PER_PAIR * pairs * w.B * w.H
+    qk_maps = w.H + w.H_N
+    pv_maps = w.H + (w.H_N if w.H_V == w.H_N else w.H)
+    return (qk_maps * 2 * 64 + pv_maps * 2 * 128) * pairs * w.B
 
 
 def decode_bytes(w):

@@ -267,7 +267,8 @@ __global__ void __launch_bounds__(DHDV) decode_combine_kernel(const DecodeParams
         A2 = fmaf(ps[4 + DHDV + c], e2, A2);
     }
     float d = 0.0f;
-    if (L1 > 0.0f && L2 > 0.0f) d = A1 / L1 - p.lambda[h] * (A2 / L2);
+    // D = (A1 - r A2) / L1 with r = lambda L1 / L2 (one rounding in the difference).
+    if (L1 > 0.0f && L2 > 0.0f) d = fmaf(-(p.lambda[h] * L1 / L2), A2, A1) / L1;
     float y = d;
     if (p.apply_norm) {
         const float ss = warp_sum(d * d);

@@ -349,7 +349,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (ok && !*abort_flag) {
                 // ---------------------------------------------------- epilogue
                 const float lam = p.lambda[w.h];
-                const float inv1 = 1.0f / l_run, c2 = lam / l2;
+                // D = (O1 - r O2) / l1 with r = lambda l1 / l2: one fused multiply-add
+                // per element, and identical maps with lambda = 1 cancel exactly.
+                const float inv1 = 1.0f / l_run, r2 = lam * l_run / l2;
                 const uint32_t tO1 = tbase + lane_off + TM_O1, tO2 = tbase + lane_off + TM_O2;
                 float rn = 1.0f;
                 if (p.apply_norm) {
@@ -362,7 +364,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
-                            const float dd = __uint_as_float(a[i]) * inv1 - __uint_as_float(bb[i]) * c2;
+                            const float dd = fmaf(-r2, __uint_as_float(bb[i]), __uint_as_float(a[i])) * inv1;
                             ss += dd * dd;
                         }
                     }
@@ -381,8 +383,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     uint32_t y[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        float y0 = (__uint_as_float(a[2 * i]) * inv1 - __uint_as_float(bb[2 * i]) * c2) * rn;
-                        float y1 = (__uint_as_float(a[2 * i + 1]) * inv1 - __uint_as_float(bb[2 * i + 1]) * c2) * rn;
+                        float y0 = fmaf(-r2, __uint_as_float(bb[2 * i]), __uint_as_float(a[2 * i])) * (inv1 * rn);
+                        float y1 = fmaf(-r2, __uint_as_float(bb[2 * i + 1]), __uint_as_float(a[2 * i + 1])) * (inv1 * rn);
                         if (gain) {
                             y0 *= __ldg(gain + 32 * c + 2 * i);
                             y1 *= __ldg(gain + 32 * c + 2 * i + 1);
