@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -15,6 +16,17 @@
 namespace {
 
 thread_local int32_t g_last_launches = 0;
+thread_local char g_last_error[256] = "";
+
+// Map a CUDA error to the ABI status, keeping its text for diffattn_last_error.
+diffattn_status cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess) return DIFFATTN_OK;
+    if (g_last_error[0] == 0)
+        std::snprintf(g_last_error, sizeof g_last_error, "%s: %s", cudaGetErrorName(e),
+                      cudaGetErrorString(e));
+    return DIFFATTN_ERR_CUDA;
+}
 thread_local da::ProfileEvents g_events;
 
 constexpr uint32_t kDefaultTimeoutMs = 2000;
@@ -150,6 +162,7 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
                         int grouped)
 {
     g_last_launches = 0;
+    g_last_error[0] = 0;
     diffattn_status st = validate_fwd(a, grouped);
     if (st != DIFFATTN_OK) return st;
     if (a->B == 0 || a->N == 0) return DIFFATTN_OK;
@@ -171,12 +184,15 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
                  a->k2_stride[0], a->k2_stride[1], a->k2_stride[2]) &&
         make_map(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws, 128, a->N, HV, a->B, a->N * HV * 128,
                  HV * 128, 128);
-    if (!ok) return DIFFATTN_ERR_CUDA;
+    if (!ok) {
+        da::set_internal_error("cuTensorMapEncodeTiled failed");
+        return DIFFATTN_ERR_CUDA;
+    }
 
     int launches = 0;
     cudaError_t e = da::launch_v_to_f16(a->v, a->v_stride[0], a->v_stride[1], a->v_stride[2], ws,
                                         (int)a->B, (int)a->N, (int)HV, a->dev_status, s, &launches);
-    if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_status(e);
 
     da::PrefillParams p{};
     p.B = (int)a->B;
@@ -202,12 +218,17 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     p.dev_status = a->dev_status;
     p.timeout_ns = (uint64_t)(a->timeout_ms ? a->timeout_ms : kDefaultTimeoutMs) * 1000000ull;
     e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, p, s, &launches, g_events);
-    if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_status(e);
     g_last_launches = launches;
     return DIFFATTN_OK;
 }
 
 }  // namespace
+
+void da::set_internal_error(const char *text)
+{
+    std::snprintf(g_last_error, sizeof g_last_error, "%s", text);
+}
 
 extern "C" {
 
@@ -257,6 +278,7 @@ diffattn_status diffattn_decode(const diffattn_decode_args *a, void *workspace, 
                                 void *stream)
 {
     g_last_launches = 0;
+    g_last_error[0] = 0;
     diffattn_status st = validate_decode(a);
     if (st != DIFFATTN_OK) return st;
     if (a->B == 0) return DIFFATTN_OK;
@@ -300,7 +322,7 @@ diffattn_status diffattn_decode(const diffattn_decode_args *a, void *workspace, 
     p.dev_status = a->dev_status;
     int launches = 0;
     cudaError_t e = da::launch_decode(p, static_cast<cudaStream_t>(stream), &launches, g_events);
-    if (e != cudaSuccess) return DIFFATTN_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_status(e);
     g_last_launches = launches;
     return DIFFATTN_OK;
 }
@@ -320,6 +342,8 @@ const char *diffattn_status_str(diffattn_status s)
 }
 
 int32_t diffattn_last_launch_count(void) { return g_last_launches; }
+
+const char *diffattn_last_error(void) { return g_last_error; }
 
 void diffattn_set_profile_events(void *start, void *stop)
 {

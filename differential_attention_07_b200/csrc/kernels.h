@@ -8,6 +8,9 @@
 
 namespace da {
 
+// Record a library-side failure text for diffattn_last_error() (thread-local).
+void set_internal_error(const char *text);
+
 // Events to record around the main kernel of a call (benchmark timing hook);
 // both null when unused.
 struct ProfileEvents {

@@ -7,7 +7,7 @@
 // after it (same page, figure 1: GroupNorm after the subtraction, read as a
 // per-head RMS norm with gain).
 //
-// One CTA per (b, h, query tile), 384 threads, one CTA per SM:
+// One CTA per (b, h, query tile), 384 threads (three warpgroups), one CTA per SM:
 //   warp 0        TMA producer: Q1/Q2 once, then K1/K2/V per 128-key tile
 //                 into a 3-stage ring (64 KB per stage).
 //   warp 1        MMA issuer (one thread): S1 = Q1 K1^T and S2 = Q2 K2^T
@@ -16,7 +16,9 @@
 //                 shared-memory tile for both maps.
 //   warps 4-7     softmax of map 1 (one thread per query row) and the
 //                 epilogue: D = O1/l1 - lambda O2/l2, RMS norm, gain, bf16.
-//   warps 8-11    softmax of map 2.
+//   warps 8-11    softmax of map 2.  A warp reaches TMEM lanes 32 (warp % 4)
+//                 onwards, so each warpgroup covers all 128 rows.  Registers
+//                 are split 56 / 224 / 224 between the warpgroups (setmaxnreg).
 // TMEM (512 columns): O1 [0,128) O2 [128,256) S1/P1 [256,384) S2/P2 [384,512).
 // P (fp16, two per column) overwrites the first 64 columns of its S.
 //
@@ -67,6 +69,15 @@ constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignm
 constexpr uint32_t TM_O1 = 0, TM_O2 = 128, TM_S1 = 256, TM_S2 = 384;
 constexpr uint32_t TMEM_COLS = 512;
 
+// Registers per thread: at launch (the most __launch_bounds__(384, 1) allows:
+// three warps per SM sub-partition share its 16K registers), and after the
+// split between the producer/MMA warpgroup and the two softmax warpgroups.
+constexpr int REGS_LAUNCH = 168;
+constexpr int REGS_IO = 56;
+constexpr int REGS_SOFTMAX = 224;
+static_assert(REGS_IO + 2 * REGS_SOFTMAX == 3 * REGS_LAUNCH, "register split must use the pool exactly");
+static_assert(NTHREADS == 384, "three warpgroups");
+
 // P.V MMAs read a stale-max P of at most 2^RESCALE_THRESHOLD.
 constexpr float RESCALE_THRESHOLD = 8.0f;
 
@@ -103,6 +114,39 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// Software 2^x for two values at once on the FMA and integer pipes, to take
+// part of the exponentials off MUFU.  Cody-Waite style range reduction:
+// x = n + f with n = rint(x) from the 1.5 * 2^23 magic-number add (the
+// integer lands in the low mantissa bits of j), f = x - n in [-1/2, 1/2];
+// 2^f is a degree-3 polynomial whose coefficients minimise the relative error
+// on [-1/2, 1/2] (Remez exchange, fit_exp2_poly.py; max relative error
+// 7.5e-5 in float32, below the fp16 rounding of P); 2^n is added into the
+// exponent field as (bits(j) << 23).  Inputs are clamped to >= -125 so the
+// exponent never wraps; 2^-125 is zero once P is rounded to fp16.
+constexpr float EXP2_C0 = 0x1.fff692p-1f;
+constexpr float EXP2_C1 = 0x1.62f31ap-1f;
+constexpr float EXP2_C2 = 0x1.f0de1ap-3f;
+constexpr float EXP2_C3 = 0x1.c3f76p-5f;
+constexpr float EXP2_ROUND = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ float2 exp2_soft2(float2 x)
+{
+    x.x = fmaxf(x.x, -125.0f);
+    x.y = fmaxf(x.y, -125.0f);
+    const float2 j = fadd2(x, make_float2(EXP2_ROUND, EXP2_ROUND));
+    const float2 n = fadd2(j, make_float2(-EXP2_ROUND, -EXP2_ROUND));
+    const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);
+    float2 p = ffma2(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
+    p = ffma2(p, f, make_float2(EXP2_C1, EXP2_C1));
+    p = ffma2(p, f, make_float2(EXP2_C0, EXP2_C0));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(j.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(j.y) << 23)));
+}
+
+// Of every SOFT_EXP_PERIOD pairs of scores, the last goes through
+// exp2_soft2 and the others through MUFU ex2.
+constexpr int SOFT_EXP_PERIOD = 4;
+
 __device__ __forceinline__ uint32_t pack_bf162(float lo, float hi)
 {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -120,27 +164,26 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, int j, in
     for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, v[c]);
     tmem_wait_ld();
 
-    float tmax = -INFINITY;
-    if (limit >= BN - 1) {
+    if (limit < BN - 1) {  // diagonal (or ragged) tile: hide keys past the limit
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float x = __uint_as_float(v[c][i]) * scale_log2;
-                v[c][i] = __float_as_uint(x);
-                tmax = fmaxf(tmax, x);
-            }
-    } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                float x = __uint_as_float(v[c][i]) * scale_log2;
-                if (32 * c + i > limit) x = -INFINITY;
-                v[c][i] = __float_as_uint(x);
-                tmax = fmaxf(tmax, x);
-            }
+            for (int i = 0; i < 32; ++i)
+                if (32 * c + i > limit) v[c][i] = __float_as_uint(-INFINITY);
     }
+    // Row max of the raw scores (scale > 0 commutes with max): four
+    // independent chains of three-input maxima instead of one serial chain.
+    float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+            mx[(i >> 3) & 3] = fmax3(mx[(i >> 3) & 3], __uint_as_float(v[c][i]), __uint_as_float(v[c][i + 1]));
+            mx[(i >> 3) & 3] = fmax3(mx[(i >> 3) & 3], __uint_as_float(v[c][i + 2]), __uint_as_float(v[c][i + 3]));
+            mx[(i >> 3) & 3] = fmax3(mx[(i >> 3) & 3], __uint_as_float(v[c][i + 4]), __uint_as_float(v[c][i + 5]));
+            mx[(i >> 3) & 3] = fmax3(mx[(i >> 3) & 3], __uint_as_float(v[c][i + 6]), __uint_as_float(v[c][i + 7]));
+        }
+    const float tmax = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]) * scale_log2;
 
     const bool need = tmax > m_run + RESCALE_THRESHOLD;
     const float m_new = need ? tmax : m_run;
@@ -160,21 +203,28 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, int j, in
     m_run = m_new;
     const float m_sub = (m_run == -INFINITY) ? 0.0f : m_run;
 
-    float rs = 0.0f;
+    // p = 2^(s * scale_log2 - m): one packed FMA per two scores, then MUFU
+    // ex2; row sum in four packed accumulators (short dependency chains).
+    const float2 sc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_sub, -m_sub);
+    float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const int c = 2 * h2 + (i >> 4), e = (2 * i) & 31;
-            const float p0 = ex2_approx(__uint_as_float(v[c][e]) - m_sub);
-            const float p1 = ex2_approx(__uint_as_float(v[c][e + 1]) - m_sub);
-            rs += p0 + p1;
-            pk[i] = pack_half2(p0, p1);
+            const float2 x = ffma2(make_float2(__uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1])), sc, nm);
+            const float2 pp = (i % SOFT_EXP_PERIOD == SOFT_EXP_PERIOD - 1)
+                                  ? exp2_soft2(x)
+                                  : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            acc[i & 3] = fadd2(acc[i & 3], pp);
+            pk[i] = pack_half2(pp.x, pp.y);
         }
         tmem_st32(tS + 32 * h2, pk);
     }
-    l_run += rs;
+    const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+    const float2 a = fadd2(a01, a23);
+    l_run += a.x + a.y;
     tmem_wait_st();
 }
 
@@ -228,7 +278,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tbase = *tmem_ptr;
     const uint64_t lim = p.timeout_ns;
 
-    if (warp == 0) {
+    // Register split: 128 x REGS_LAUNCH = 128 x REGS_IO + 256 x REGS_SOFTMAX
+    // (the host launches only when the kernel was built with REGS_LAUNCH).
+    // Each budget change opens its role's branch so that the compiler
+    // allocates each branch within its own budget.
+    if (warp < 4) {
+      regs_decrease<REGS_IO>();
+      if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tensormap(&tm_q1);
@@ -260,7 +316,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 drained &= mbar_wait_drain(bar_full(j % STAGES), (j / STAGES) & 1, lim);
             if (!drained) *abort_flag = 1;
         }
-    } else if (warp == 1) {
+      } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t ID_S = idesc_f16(1, 1, 0, BM, BN);    // bf16 x bf16, both K-major
@@ -319,7 +375,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // Nothing of ours may still run on the tensor cores at teardown.
             if (!mbar_wait_drain(bar_o, 0, lim)) *abort_flag = 1;
         }
-    } else if (warp >= 4) {
+      }
+    } else {
+        regs_increase<REGS_SOFTMAX>();
         // ------------------------------------------------------------ softmax
         const int t = (warp >= 8) ? 1 : 0;
         const int r = (warp & 3) * 32 + lane;
@@ -448,8 +506,19 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
 {
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)SMEM_BYTES);
+        // The register split inside the kernel is only valid for a build that
+        // launches with exactly REGS_LAUNCH registers per thread: with fewer,
+        // the softmax warpgroups' increase could never be granted.  Refuse to
+        // launch such a build.
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != REGS_LAUNCH || fa.maxThreadsPerBlock < NTHREADS) {
+            set_internal_error("prefill_kernel built with an unexpected register count");
+            return cudaErrorInvalidConfiguration;
+        }
+        e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }

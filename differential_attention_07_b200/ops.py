@@ -37,7 +37,7 @@ EXPORTED = [
     "diffattn_fwd", "diffattn_grouped_fwd", "diffattn_fwd_workspace_size", "diffattn_fwd_validate",
     "diffattn_decode", "diffattn_decode_workspace_size", "diffattn_decode_num_splits",
     "diffattn_decode_validate", "diffattn_status_str", "diffattn_last_launch_count",
-    "diffattn_set_profile_events",
+    "diffattn_set_profile_events", "diffattn_last_error",
 ]
 
 _i64 = ctypes.c_int64
@@ -83,7 +83,12 @@ class DecodeArgs(ctypes.Structure):
 class DiffAttnError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
-        super().__init__(f"{where}: {STATUS.get(status, status)}")
+        msg = f"{where}: {STATUS.get(status, status)}"
+        if status == 5 and _LIB is not None:
+            detail = _LIB.diffattn_last_error()
+            if detail:
+                msg += f" ({detail.decode(errors='replace')})"
+        super().__init__(msg)
 
 
 _LIB = None
@@ -118,6 +123,8 @@ def lib():
         L.diffattn_status_str.restype = ctypes.c_char_p
         L.diffattn_last_launch_count.argtypes = []
         L.diffattn_last_launch_count.restype = ctypes.c_int32
+        L.diffattn_last_error.argtypes = []
+        L.diffattn_last_error.restype = ctypes.c_char_p
         L.diffattn_set_profile_events.argtypes = [_p, _p]
         L.diffattn_set_profile_events.restype = None
         _LIB = L

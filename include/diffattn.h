@@ -150,6 +150,11 @@ const char *diffattn_status_str(diffattn_status status);
  * launch accounting in benchmarks).                                          */
 int32_t diffattn_last_launch_count(void);
 
+/* Text of the CUDA error (or internal check) behind the last
+ * DIFFATTN_ERR_CUDA returned on this thread; "" when there was none.  The
+ * string is owned by the library and valid until the next call.             */
+const char *diffattn_last_error(void);
+
 /* Timing hook for benchmarks: while set (non-NULL), every later call on this
  * thread records `start` (a cudaEvent_t passed as void*) on its stream just
  * before its main kernel (the prefill kernel, or the decode split kernel) and
