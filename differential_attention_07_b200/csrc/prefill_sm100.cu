@@ -286,95 +286,110 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       regs_decrease<REGS_IO>();
       if (warp == 0) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
+        // The whole warp runs the loop; an elected lane issues the copies.
+        const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
+        if (elect_one()) {
             prefetch_tensormap(&tm_q1);
             prefetch_tensormap(&tm_q2);
             prefetch_tensormap(&tm_k1);
             prefetch_tensormap(&tm_k2);
             prefetch_tensormap(&tm_v);
-            const uint64_t keep = policy_evict_last(), stream = policy_evict_first();
             mbar_arrive_expect_tx(bar_q, 2 * Q_BYTES);
             tma_load_4d(sbase + OFF_Q1, &tm_q1, bar_q, 0, q0, w.h, w.b, stream);
             tma_load_4d(sbase + OFF_Q2, &tm_q2, bar_q, 0, q0, nh, w.b, stream);
-            int issued = 0;
-            for (int j = 0; j < nkv; ++j) {
-                const int s = j % STAGES;
-                if (j >= STAGES && !mbar_wait(bar_empty(s), ((j / STAGES) - 1) & 1, abort_flag, lim))
-                    break;
-                const uint32_t st = sbase + OFF_STAGE0 + s * STAGE_BYTES;
-                const int k0 = j * BN;
+        }
+        __syncwarp();
+        int issued = 0;
+        for (int j = 0; j < nkv; ++j) {
+            const int s = j % STAGES;
+            if (j >= STAGES && !mbar_wait_warp(bar_empty(s), ((j / STAGES) - 1) & 1, abort_flag, lim))
+                break;
+            const uint32_t st = sbase + OFF_STAGE0 + s * STAGE_BYTES;
+            const int k0 = j * BN;
+            if (elect_one()) {
                 mbar_arrive_expect_tx(bar_full(s), STAGE_BYTES);
                 tma_load_4d(st, &tm_k1, bar_full(s), 0, k0, w.h, w.b, keep);
                 tma_load_4d(st + K_BYTES, &tm_k2, bar_full(s), 0, k0, nh, w.b, keep);
                 tma_load_4d(st + 2 * K_BYTES, &tm_v, bar_full(s), 0, k0, vh, w.b, keep);
                 tma_load_4d(st + 2 * K_BYTES + VHALF_BYTES, &tm_v, bar_full(s), 64, k0, vh, w.b, keep);
-                issued = j + 1;
             }
-            // No load of ours may land after the CTA has gone: wait for all of them.
-            bool drained = mbar_wait_drain(bar_q, 0, lim);
-            for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
-                drained &= mbar_wait_drain(bar_full(j % STAGES), (j / STAGES) & 1, lim);
-            if (!drained) *abort_flag = 1;
+            __syncwarp();
+            issued = j + 1;
         }
+        // No load of ours may land after the CTA has gone: wait for all of them.
+        bool drained = mbar_wait_drain(bar_q, 0, lim);
+        for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
+            drained &= mbar_wait_drain(bar_full(j % STAGES), (j / STAGES) & 1, lim);
+        if (!__all_sync(0xffffffffu, drained) && lane == 0) *abort_flag = 1;
       } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t ID_S = idesc_f16(1, 1, 0, BM, BN);    // bf16 x bf16, both K-major
-            constexpr uint32_t ID_PV = idesc_f16(0, 0, 1, BM, HDV);  // f16 x f16, B (V) MN-major
-            auto issue_s = [&](int t, int s) {
-                const uint32_t qa = sbase + (t ? OFF_Q2 : OFF_Q1);
-                const uint32_t ka = sbase + OFF_STAGE0 + s * STAGE_BYTES + (t ? K_BYTES : 0);
-                const uint32_t d = tbase + (t ? TM_S2 : TM_S1);
+        // The whole warp runs the loop (descriptors stay warp-uniform); an
+        // elected lane issues each tcgen05 instruction.
+        constexpr uint32_t ID_S = idesc_f16(1, 1, 0, BM, BN);    // bf16 x bf16, both K-major
+        constexpr uint32_t ID_PV = idesc_f16(0, 0, 1, BM, HDV);  // f16 x f16, B (V) MN-major
+        auto issue_s = [&](int t, int s) {
+            const uint32_t qa = sbase + (t ? OFF_Q2 : OFF_Q1);
+            const uint32_t ka = sbase + OFF_STAGE0 + s * STAGE_BYTES + (t ? K_BYTES : 0);
+            const uint32_t d = tbase + (t ? TM_S2 : TM_S1);
 #pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
+            for (int kk = 0; kk < HD / 16; ++kk) {
+                if (elect_one())
                     mma_ss(d, smem_desc_sw128(qa + 32 * kk, 16, 1024),
                            smem_desc_sw128(ka + 32 * kk, 16, 1024), ID_S, kk > 0);
-            };
-            auto issue_pv = [&](int t, int s, bool acc) {
-                const uint32_t va = sbase + OFF_STAGE0 + s * STAGE_BYTES + 2 * K_BYTES;
-                const uint32_t d = tbase + (t ? TM_O2 : TM_O1);
-                const uint32_t a = tbase + (t ? TM_S2 : TM_S1);
+                __syncwarp();
+            }
+        };
+        auto issue_pv = [&](int t, int s, bool acc) {
+            const uint32_t va = sbase + OFF_STAGE0 + s * STAGE_BYTES + 2 * K_BYTES;
+            const uint32_t d = tbase + (t ? TM_O2 : TM_O1);
+            const uint32_t a = tbase + (t ? TM_S2 : TM_S1);
 #pragma unroll
-                for (int kk = 0; kk < BN / 16; ++kk)
+            for (int kk = 0; kk < BN / 16; ++kk) {
+                if (elect_one())
                     mma_ts(d, a + 8 * kk, smem_desc_sw128(va + 2048 * kk, VHALF_BYTES, 1024), ID_PV,
                            (acc || kk > 0) ? 1u : 0u);
-            };
-            bool ok = mbar_wait(bar_q, 0, abort_flag, lim);
-            tc_fence_after();
-            if (ok) ok = mbar_wait(bar_full(0), 0, abort_flag, lim);
-            if (ok) {
-                tc_fence_after();
-                issue_s(0, 0);
-                mma_commit(bar_s1);
-                issue_s(1, 0);
-                mma_commit(bar_s2);
+                __syncwarp();
             }
-            for (int j = 0; ok && j < nkv; ++j) {
-                const int s = j % STAGES;
-                if (!(ok = mbar_wait(bar_p1, j & 1, abort_flag, lim))) break;
-                tc_fence_after();
-                issue_pv(0, s, j > 0);
-                const bool more = j + 1 < nkv;
-                const int s1 = (j + 1) % STAGES;
-                if (more) {
-                    if (!(ok = mbar_wait(bar_full(s1), ((j + 1) / STAGES) & 1, abort_flag, lim))) break;
-                    tc_fence_after();
-                    issue_s(0, s1);
-                    mma_commit(bar_s1);
-                }
-                if (!(ok = mbar_wait(bar_p2, j & 1, abort_flag, lim))) break;
-                tc_fence_after();
-                issue_pv(1, s, j > 0);
-                mma_commit(bar_empty(s));
-                if (more) {
-                    issue_s(1, s1);
-                    mma_commit(bar_s2);
-                }
-            }
-            mma_commit(bar_o);
-            // Nothing of ours may still run on the tensor cores at teardown.
-            if (!mbar_wait_drain(bar_o, 0, lim)) *abort_flag = 1;
+        };
+        auto commit = [&](uint32_t bar) {
+            if (elect_one()) mma_commit(bar);
+            __syncwarp();
+        };
+        bool ok = mbar_wait_warp(bar_q, 0, abort_flag, lim);
+        if (ok) ok = mbar_wait_warp(bar_full(0), 0, abort_flag, lim);
+        tc_fence_after();
+        if (ok) {
+            issue_s(0, 0);
+            commit(bar_s1);
+            issue_s(1, 0);
+            commit(bar_s2);
         }
+        for (int j = 0; ok && j < nkv; ++j) {
+            const int s = j % STAGES;
+            if (!(ok = mbar_wait_warp(bar_p1, j & 1, abort_flag, lim))) break;
+            tc_fence_after();
+            issue_pv(0, s, j > 0);
+            const bool more = j + 1 < nkv;
+            const int s1 = (j + 1) % STAGES;
+            if (more) {
+                if (!(ok = mbar_wait_warp(bar_full(s1), ((j + 1) / STAGES) & 1, abort_flag, lim))) break;
+                tc_fence_after();
+                issue_s(0, s1);
+                commit(bar_s1);
+            }
+            if (!(ok = mbar_wait_warp(bar_p2, j & 1, abort_flag, lim))) break;
+            tc_fence_after();
+            issue_pv(1, s, j > 0);
+            commit(bar_empty(s));
+            if (more) {
+                issue_s(1, s1);
+                commit(bar_s2);
+            }
+        }
+        commit(bar_o);
+        // Nothing of ours may still run on the tensor cores at teardown.
+        const bool drained = mbar_wait_drain(bar_o, 0, lim);
+        if (!__all_sync(0xffffffffu, drained) && lane == 0) *abort_flag = 1;
       }
     } else {
         regs_increase<REGS_SOFTMAX>();

@@ -102,6 +102,29 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, u
     }
 }
 
+// True on exactly one lane of the (fully active) warp.  Issuing tcgen05 /
+// TMA instructions from an elected lane of a warp that runs the loop
+// together keeps descriptors and addresses warp-uniform; a loop run by one
+// lane alone issues tcgen05.mma at about half the tensor-core rate.
+__device__ __forceinline__ bool elect_one()
+{
+    uint32_t p;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(p));
+    return p != 0;
+}
+
+// Warp-wide bounded wait: every lane waits, and the warp agrees on success.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
+                                               volatile int *abort_flag, uint64_t limit_ns)
+{
+    const bool ok = mbar_wait(bar, parity, abort_flag, limit_ns);
+    return __all_sync(0xffffffffu, ok);
+}
+
 // ---------------------------------------------------------------- TMA
 // 4-D tiled bulk tensor load global -> shared, completion counted in bytes
 // on `bar`.  c0 is the innermost (contiguous) coordinate.
