@@ -52,9 +52,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 }
 
 // 4-D map over a [B, N, heads, inner] tensor (element strides sb, sn, sh;
-// inner contiguous), box {64, 128, 1, 1}, 128-byte swizzle, zero fill.
+// inner contiguous), box {64, rows, 1, 1}, 128-byte swizzle, zero fill.
 bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int64_t inner,
-              int64_t N, int64_t heads, int64_t B, int64_t sb, int64_t sn, int64_t sh)
+              int64_t N, int64_t heads, int64_t B, int64_t sb, int64_t sn, int64_t sh,
+              uint32_t rows)
 {
     auto fn = encode_fn();
     if (!fn) return false;
@@ -62,7 +63,7 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int64_t 
                                 (cuuint64_t)B};
     const cuuint64_t strides[3] = {(cuuint64_t)(sn * 2), (cuuint64_t)(sh * 2),
                                    (cuuint64_t)(sb * 2)};
-    const cuuint32_t box[4] = {64, 128, 1, 1};
+    const cuuint32_t box[4] = {64, rows, 1, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(m, dt, 4, const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -175,15 +176,15 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     CUtensorMap mq1, mq2, mk1, mk2, mv;
     const bool ok =
         make_map(&mq1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->q1, 64, a->N, a->H, a->B,
-                 a->q1_stride[0], a->q1_stride[1], a->q1_stride[2]) &&
+                 a->q1_stride[0], a->q1_stride[1], a->q1_stride[2], da::kPrefillQRows) &&
         make_map(&mq2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->q2, 64, a->N, HN, a->B,
-                 a->q2_stride[0], a->q2_stride[1], a->q2_stride[2]) &&
+                 a->q2_stride[0], a->q2_stride[1], a->q2_stride[2], da::kPrefillQRows) &&
         make_map(&mk1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->k1, 64, a->N, a->H, a->B,
-                 a->k1_stride[0], a->k1_stride[1], a->k1_stride[2]) &&
+                 a->k1_stride[0], a->k1_stride[1], a->k1_stride[2], da::kPrefillKeyRows) &&
         make_map(&mk2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->k2, 64, a->N, HN, a->B,
-                 a->k2_stride[0], a->k2_stride[1], a->k2_stride[2]) &&
+                 a->k2_stride[0], a->k2_stride[1], a->k2_stride[2], da::kPrefillKeyRows) &&
         make_map(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws, 128, a->N, HV, a->B, a->N * HV * 128,
-                 HV * 128, 128);
+                 HV * 128, 128, da::kPrefillKeyRows);
     if (!ok) {
         da::set_internal_error("cuTensorMapEncodeTiled failed");
         return DIFFATTN_ERR_CUDA;

@@ -8,26 +8,31 @@
 // per-head RMS norm with gain).
 //
 // One CTA per (b, h, query tile), 384 threads (three warpgroups), one CTA per SM:
-//   warp 0        TMA producer: Q1/Q2 once, then K1/K2/V per 128-key tile
-//                 into a 3-stage ring (64 KB per stage).
-//   warp 1        MMA issuer (one thread): S1 = Q1 K1^T and S2 = Q2 K2^T
-//                 (bf16, fp32 accumulate in TMEM), then O1 += P1 V and
-//                 O2 += P2 V with P read from TMEM and V (fp16) from the same
-//                 shared-memory tile for both maps.
+//   warp 0        TMA producer: Q1/Q2 once, then K1/K2/V per 64-key step
+//                 into a 6-stage ring (32 KB per stage).
+//   warps 1, 2    MMA issuers, one per map: S_t = Q_t K_t^T (bf16, fp32
+//                 accumulate in TMEM), then O_t += P_t V with P read from TMEM
+//                 and V (fp16) from the shared-memory tile both maps use.
 //   warps 4-7     softmax of map 1 (one thread per query row) and the
-//                 epilogue: D = O1/l1 - lambda O2/l2, RMS norm, gain, bf16.
+//                 epilogue: D = (O1 - r O2)/l1 with r = lambda l1/l2, RMS
+//                 norm, gain, bf16.
 //   warps 8-11    softmax of map 2.  A warp reaches TMEM lanes 32 (warp % 4)
 //                 onwards, so each warpgroup covers all 128 rows.  Registers
 //                 are split 56 / 224 / 224 between the warpgroups (setmaxnreg).
-// TMEM (512 columns): O1 [0,128) O2 [128,256) S1/P1 [256,384) S2/P2 [384,512).
-// P (fp16, two per column) overwrites the first 64 columns of its S.
+// TMEM (512 columns): O1 [0,128) O2 [128,256), and two 64-column S buffers
+// per map: S1 [256,320) [320,384), S2 [384,448) [448,512).  P (fp16, two per
+// column) overwrites the first 32 columns of its S buffer.
 //
-// The MMA issue order S1_0 S2_0 | PV1_0 S1_1 PV2_0 S2_1 | PV1_1 S1_2 ... makes
-// every "S_t ready" commit also certify that the previous P_t.V product has
-// finished, so the softmax thread may rescale O_t and overwrite P_t as soon as
-// it sees S_t.  The softmax keeps a stale row maximum until the new one
-// exceeds it by more than 2^8 (P stays <= 256, exact enough in fp16), so O is
-// rescaled only when the maximum really moves.
+// Pipeline.  Key steps alternate between the two S buffers of a map, and the
+// MMA warp computes S for step j+2 as soon as P.V of step j has been issued,
+// so the softmax of step j+1 need not wait for the tensor cores: the score
+// MMAs of the next step run while the current step's softmax runs.  Per map t
+// and step j the map's MMA warp does:
+//   wait P_t,j; O_t += P_t,j V_j; release stage j; S_t,j+2 -> buffer j%2.
+// MMAs from one thread execute in issue order, so S_{j+2} overwrites P_j only
+// after P_j.V has read it.  The softmax keeps a stale row maximum until a new
+// one exceeds it by more than 2^8 (P stays <= 256, exact enough in fp16); only
+// then does it rescale its O row, after waiting for the previous P.V product.
 //
 // Every wait is bounded (PrefillParams::timeout_ns); on expiry the CTA raises
 // an abort flag, reports DIFFATTN_ERR_TIMEOUT, drains its own TMA loads and
@@ -42,27 +47,32 @@ namespace da {
 namespace {
 
 constexpr int BM = 128;   // query rows per tile (MMA M)
-constexpr int BN = 128;   // keys per KV tile (MMA N of S, K of P.V)
+constexpr int BN = 64;    // keys per step (MMA N of S, K of P.V)
 constexpr int HD = 64;    // Q/K head dim
 constexpr int HDV = 128;  // V head dim (MMA N of P.V)
-constexpr int STAGES = 3;
+constexpr int STAGES = 6;
 constexpr int NTHREADS = 384;
 
 constexpr uint32_t Q_BYTES = BM * HD * 2;           // 16 KB
-constexpr uint32_t K_BYTES = BN * HD * 2;           // 16 KB
-constexpr uint32_t VHALF_BYTES = BN * 64 * 2;       // 16 KB: 64 of the 128 V columns
-constexpr uint32_t V_BYTES = 2 * VHALF_BYTES;       // 32 KB
+constexpr uint32_t K_BYTES = BN * HD * 2;           // 8 KB
+constexpr uint32_t VHALF_BYTES = BN * 64 * 2;       // 8 KB: 64 of the 128 V columns
+constexpr uint32_t V_BYTES = 2 * VHALF_BYTES;       // 16 KB
 constexpr uint32_t STAGE_BYTES = 2 * K_BYTES + V_BYTES;
 
 constexpr uint32_t OFF_Q1 = 0;
 constexpr uint32_t OFF_Q2 = Q_BYTES;
 constexpr uint32_t OFF_STAGE0 = 2 * Q_BYTES;
 constexpr uint32_t OFF_BARS = OFF_STAGE0 + STAGES * STAGE_BYTES;
-// barriers: q, full[S], empty[S], s1, s2, p1, p2, o
-constexpr int NBARS = 1 + 2 * STAGES + 5;
+// barriers: q, full[S], empty[S], s1[2], s2[2], p1[2], p2[2], pv1, pv2, o.
+// S and P barriers come one per S buffer: a softmax may run two steps ahead
+// of the MMA warp's wait, and with one P barrier per map the second arrival
+// would complete a phase the MMA warp had not yet waited for.  Per buffer,
+// the next use needs the MMA warp's action in between, so no barrier is ever
+// more than one phase ahead of its waiter.
+constexpr int NBARS = 1 + 2 * STAGES + 4 + 4 + 3;
 constexpr uint32_t OFF_TMEM_PTR = OFF_BARS + NBARS * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
-constexpr uint32_t OFF_L2 = OFF_ABORT + 12;  // 16-byte aligned
+constexpr uint32_t OFF_L2 = (OFF_ABORT + 4 + 15) & ~15u;
 constexpr uint32_t SMEM_USED = OFF_L2 + BM * 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
 
@@ -82,7 +92,9 @@ static_assert(NTHREADS == 384, "three warpgroups");
 constexpr float RESCALE_THRESHOLD = 8.0f;
 
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(OFF_STAGE0 % 1024 == 0 && STAGE_BYTES % 1024 == 0, "SW128 atoms need 1 KB alignment");
+static_assert(kPrefillQRows == BM && kPrefillKeyRows == BN, "TMA boxes match the tiles");
+static_assert(OFF_STAGE0 % 1024 == 0 && STAGE_BYTES % 1024 == 0 && K_BYTES % 1024 == 0,
+              "SW128 atoms need 1 KB alignment");
 
 struct Work {
     int b, h, qt;
@@ -111,6 +123,12 @@ __device__ __forceinline__ Work work_of(int idx, const PrefillParams &p)
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
 {
     __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ uint32_t pack_bf162(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
@@ -143,45 +161,45 @@ __device__ __forceinline__ float2 exp2_soft2(float2 x)
                        __int_as_float(__float_as_int(p.y) + (__float_as_int(j.y) << 23)));
 }
 
-// Of every SOFT_EXP_PERIOD pairs of scores, the last goes through
-// exp2_soft2 and the others through MUFU ex2.
-constexpr int SOFT_EXP_PERIOD = 4;
+// Which pairs of scores (index mod 8) take the software exp2; the rest use
+// MUFU ex2.  3 of 8 balances MUFU time against issue slots for two softmax
+// warps per SM sub-partition.
+constexpr uint32_t SOFT_EXP_MASK = 0xA4u;  // pairs 2, 5, 7 of every 8
 
-__device__ __forceinline__ uint32_t pack_bf162(float lo, float hi)
-{
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-
-// Softmax of one map for one KV tile, for the query row this thread owns.
+// Softmax of one map for one 64-key step, for the query row this thread owns.
 // Reads S (fp32) from TMEM, updates the running max / sum, rescales the O row
-// when the max moved, writes P (fp16) over the first 64 S columns.
-__device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, int j, int limit,
-                                             float scale_log2, float &m_run, float &l_run)
+// when the max moved (after the previous P.V product into it has finished),
+// and writes P (fp16) over the first 32 columns of the S buffer.  Returns
+// false if a bounded wait gave up.
+__device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, int j, int limit,
+                                             float scale_log2, float &m_run, float &l_run,
+                                             uint32_t bar_pv, volatile int *abort_flag,
+                                             uint64_t lim)
 {
-    uint32_t v[4][32];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, v[c]);
+    uint32_t v[2][32];
+    tmem_ld32(tS, v[0]);
+    tmem_ld32(tS + 32, v[1]);
     tmem_wait_ld();
 
-    if (limit < BN - 1) {  // diagonal (or ragged) tile: hide keys past the limit
+    if (limit < BN - 1) {  // diagonal (or ragged) step: hide keys past the limit
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
             for (int i = 0; i < 32; ++i)
                 if (32 * c + i > limit) v[c][i] = __float_as_uint(-INFINITY);
     }
     // Row max of the raw scores (scale > 0 commutes with max): four
-    // independent chains of three-input maxima instead of one serial chain.
+    // independent chains of three-input maxima.
     float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
+    for (int c = 0; c < 2; ++c)
 #pragma unroll
         for (int i = 0; i < 32; i += 8) {
-            mx[(i >> 3) & 3] = fmax3(mx[(i >> 3) & 3], __uint_as_float(v[c][i]), __uint_as_float(v[c][i + 1]));
-            mx[(i >> 3) & 3] = fmax3(mx[(i >> 3) & 3], __uint_as_float(v[c][i + 2]), __uint_as_float(v[c][i + 3]));
-            mx[(i >> 3) & 3] = fmax3(mx[(i >> 3) & 3], __uint_as_float(v[c][i + 4]), __uint_as_float(v[c][i + 5]));
-            mx[(i >> 3) & 3] = fmax3(mx[(i >> 3) & 3], __uint_as_float(v[c][i + 6]), __uint_as_float(v[c][i + 7]));
+            float &m = mx[(2 * c + (i >> 4)) & 3];
+            m = fmax3(m, __uint_as_float(v[c][i]), __uint_as_float(v[c][i + 1]));
+            m = fmax3(m, __uint_as_float(v[c][i + 2]), __uint_as_float(v[c][i + 3]));
+            m = fmax3(m, __uint_as_float(v[c][i + 4]), __uint_as_float(v[c][i + 5]));
+            m = fmax3(m, __uint_as_float(v[c][i + 6]), __uint_as_float(v[c][i + 7]));
         }
     const float tmax = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]) * scale_log2;
 
@@ -189,6 +207,9 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, int j, in
     const float m_new = need ? tmax : m_run;
     const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;  // ex2(-inf) = 0
     if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // O holds P.V products up to step j-1; the last one must be finished.
+        if (!mbar_wait_warp(bar_pv, (j - 1) & 1, abort_flag, lim)) return false;
+        tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
             uint32_t o[32];
@@ -203,29 +224,26 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, int j, in
     m_run = m_new;
     const float m_sub = (m_run == -INFINITY) ? 0.0f : m_run;
 
-    // p = 2^(s * scale_log2 - m): one packed FMA per two scores, then MUFU
-    // ex2; row sum in four packed accumulators (short dependency chains).
+    // p = 2^(s * scale_log2 - m): one packed FMA per two scores, then MUFU or
+    // software exp2; row sum in four packed accumulators.
     const float2 sc = make_float2(scale_log2, scale_log2), nm = make_float2(-m_sub, -m_sub);
     float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+    uint32_t pk[32];
 #pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int c = 2 * h2 + (i >> 4), e = (2 * i) & 31;
-            const float2 x = ffma2(make_float2(__uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1])), sc, nm);
-            const float2 pp = (i % SOFT_EXP_PERIOD == SOFT_EXP_PERIOD - 1)
-                                  ? exp2_soft2(x)
-                                  : make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            acc[i & 3] = fadd2(acc[i & 3], pp);
-            pk[i] = pack_half2(pp.x, pp.y);
-        }
-        tmem_st32(tS + 32 * h2, pk);
+    for (int i = 0; i < 32; ++i) {
+        const int c = i >> 4, e = (2 * i) & 31;
+        const float2 x = ffma2(make_float2(__uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1])), sc, nm);
+        const float2 pp = ((SOFT_EXP_MASK >> (i & 7)) & 1u)
+                              ? exp2_soft2(x)
+                              : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+        acc[i & 3] = fadd2(acc[i & 3], pp);
+        pk[i] = pack_half2(pp.x, pp.y);
     }
-    const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
-    const float2 a = fadd2(a01, a23);
+    tmem_st32(tS, pk);
+    const float2 a = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
     l_run += a.x + a.y;
     tmem_wait_st();
+    return true;
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -242,14 +260,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const Work w = work_of(blockIdx.x, p);
     const int nh = w.h / (p.H / p.H_N), vh = w.h / (p.H / p.H_V);
     const int q0 = w.qt * BM;
-    const int nkv = p.causal ? w.qt + 1 : (p.N + BN - 1) / BN;
+    const int n_steps_all = (p.N + BN - 1) / BN;
+    const int nkv = p.causal ? min(n_steps_all, (q0 + BM) / BN) : n_steps_all;
 
     const uint32_t bar_q = sbase + OFF_BARS;
     auto bar_full = [&](int s) { return sbase + OFF_BARS + 8 * (1 + s); };
     auto bar_empty = [&](int s) { return sbase + OFF_BARS + 8 * (1 + STAGES + s); };
-    const uint32_t bar_s1 = sbase + OFF_BARS + 8 * (1 + 2 * STAGES);
-    const uint32_t bar_s2 = bar_s1 + 8, bar_p1 = bar_s1 + 16, bar_p2 = bar_s1 + 24;
-    const uint32_t bar_o = bar_s1 + 32;
+    const uint32_t bar_s1_0 = sbase + OFF_BARS + 8 * (1 + 2 * STAGES);  // s1[2], then s2[2]
+    auto bar_s = [&](int t, int b) { return bar_s1_0 + 8 * (2 * t + b); };
+    auto bar_p = [&](int t, int b) { return bar_s1_0 + 32 + 8 * (2 * t + b); };
+    const uint32_t bar_pv1 = bar_s1_0 + 64, bar_pv2 = bar_s1_0 + 72;
+    const uint32_t bar_o = bar_s1_0 + 80;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_ABORT);
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + OFF_TMEM_PTR);
     float *sL2 = reinterpret_cast<float *>(smem + OFF_L2);
@@ -258,13 +279,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_init(bar_q, 1);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar_full(s), 1);
-            mbar_init(bar_empty(s), 1);
+            mbar_init(bar_empty(s), 2);  // one commit from each map's MMA warp
         }
-        mbar_init(bar_s1, 1);
-        mbar_init(bar_s2, 1);
-        mbar_init(bar_p1, 128);
-        mbar_init(bar_p2, 128);
-        mbar_init(bar_o, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(bar_s1_0 + 8 * i, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(bar_s1_0 + 32 + 8 * i, 128);
+        mbar_init(bar_pv1, 1);
+        mbar_init(bar_pv2, 1);
+        mbar_init(bar_o, 2);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -321,33 +342,35 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
             drained &= mbar_wait_drain(bar_full(j % STAGES), (j / STAGES) & 1, lim);
         if (!__all_sync(0xffffffffu, drained) && lane == 0) *abort_flag = 1;
-      } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        // The whole warp runs the loop (descriptors stay warp-uniform); an
-        // elected lane issues each tcgen05 instruction.
+      } else if (warp == 1 || warp == 2) {
+        // ------------------------------------------------------------ MMA issuers
+        // Warp 1 issues map 1's MMAs, warp 2 map 2's.  The maps use disjoint
+        // TMEM, so each warp only needs its own MMAs in order, and neither map
+        // waits for the other's softmax.  The whole warp runs the loop
+        // (descriptors stay warp-uniform); an elected lane issues.
+        const int t = warp - 1;
         constexpr uint32_t ID_S = idesc_f16(1, 1, 0, BM, BN);    // bf16 x bf16, both K-major
         constexpr uint32_t ID_PV = idesc_f16(0, 0, 1, BM, HDV);  // f16 x f16, B (V) MN-major
-        auto issue_s = [&](int t, int s) {
-            const uint32_t qa = sbase + (t ? OFF_Q2 : OFF_Q1);
+        const uint32_t qa = sbase + (t ? OFF_Q2 : OFF_Q1);
+        const uint32_t tS = tbase + (t ? TM_S2 : TM_S1), tO = tbase + (t ? TM_O2 : TM_O1);
+        const uint32_t bar_pv = t ? bar_pv2 : bar_pv1;
+        auto issue_s = [&](int s, int buf) {
             const uint32_t ka = sbase + OFF_STAGE0 + s * STAGE_BYTES + (t ? K_BYTES : 0);
-            const uint32_t d = tbase + (t ? TM_S2 : TM_S1);
 #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk) {
                 if (elect_one())
-                    mma_ss(d, smem_desc_sw128(qa + 32 * kk, 16, 1024),
+                    mma_ss(tS + BN * buf, smem_desc_sw128(qa + 32 * kk, 16, 1024),
                            smem_desc_sw128(ka + 32 * kk, 16, 1024), ID_S, kk > 0);
                 __syncwarp();
             }
         };
-        auto issue_pv = [&](int t, int s, bool acc) {
+        auto issue_pv = [&](int s, int buf, bool acc) {
             const uint32_t va = sbase + OFF_STAGE0 + s * STAGE_BYTES + 2 * K_BYTES;
-            const uint32_t d = tbase + (t ? TM_O2 : TM_O1);
-            const uint32_t a = tbase + (t ? TM_S2 : TM_S1);
 #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk) {
                 if (elect_one())
-                    mma_ts(d, a + 8 * kk, smem_desc_sw128(va + 2048 * kk, VHALF_BYTES, 1024), ID_PV,
-                           (acc || kk > 0) ? 1u : 0u);
+                    mma_ts(tO, tS + BN * buf + 8 * kk, smem_desc_sw128(va + 2048 * kk, VHALF_BYTES, 1024),
+                           ID_PV, (acc || kk > 0) ? 1u : 0u);
                 __syncwarp();
             }
         };
@@ -356,37 +379,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             __syncwarp();
         };
         bool ok = mbar_wait_warp(bar_q, 0, abort_flag, lim);
-        if (ok) ok = mbar_wait_warp(bar_full(0), 0, abort_flag, lim);
-        tc_fence_after();
-        if (ok) {
-            issue_s(0, 0);
-            commit(bar_s1);
-            issue_s(1, 0);
-            commit(bar_s2);
+        for (int jj = 0; ok && jj < 2 && jj < nkv; ++jj) {
+            if (!(ok = mbar_wait_warp(bar_full(jj), 0, abort_flag, lim))) break;
+            tc_fence_after();
+            issue_s(jj, jj);
+            commit(bar_s(t, jj));
         }
         for (int j = 0; ok && j < nkv; ++j) {
-            const int s = j % STAGES;
-            if (!(ok = mbar_wait_warp(bar_p1, j & 1, abort_flag, lim))) break;
+            const int s = j % STAGES, buf = j & 1;
+            if (!(ok = mbar_wait_warp(bar_p(t, buf), (j >> 1) & 1, abort_flag, lim))) break;
             tc_fence_after();
-            issue_pv(0, s, j > 0);
-            const bool more = j + 1 < nkv;
-            const int s1 = (j + 1) % STAGES;
-            if (more) {
-                if (!(ok = mbar_wait_warp(bar_full(s1), ((j + 1) / STAGES) & 1, abort_flag, lim))) break;
+            issue_pv(s, buf, j > 0);
+            commit(bar_pv);
+            commit(bar_empty(s));  // the stage is free once both maps' P.V have read it
+            if (j + 2 < nkv) {
+                const int s2 = (j + 2) % STAGES;
+                if (!(ok = mbar_wait_warp(bar_full(s2), ((j + 2) / STAGES) & 1, abort_flag, lim))) break;
                 tc_fence_after();
-                issue_s(0, s1);
-                commit(bar_s1);
-            }
-            if (!(ok = mbar_wait_warp(bar_p2, j & 1, abort_flag, lim))) break;
-            tc_fence_after();
-            issue_pv(1, s, j > 0);
-            commit(bar_empty(s));
-            if (more) {
-                issue_s(1, s1);
-                commit(bar_s2);
+                issue_s(s2, buf);
+                commit(bar_s(t, buf));
             }
         }
-        commit(bar_o);
+        commit(bar_o);  // bar_o completes when both maps' MMAs are done
         // Nothing of ours may still run on the tensor cores at teardown.
         const bool drained = mbar_wait_drain(bar_o, 0, lim);
         if (!__all_sync(0xffffffffu, drained) && lane == 0) *abort_flag = 1;
@@ -397,19 +411,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int t = (warp >= 8) ? 1 : 0;
         const int r = (warp & 3) * 32 + lane;
         const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
-        const uint32_t tS = tbase + lane_off + (t ? TM_S2 : TM_S1);
+        const uint32_t tS0 = tbase + lane_off + (t ? TM_S2 : TM_S1);
         const uint32_t tO = tbase + lane_off + (t ? TM_O2 : TM_O1);
-        const uint32_t bar_s = t ? bar_s2 : bar_s1, bar_p = t ? bar_p2 : bar_p1;
+        const uint32_t bar_pv = t ? bar_pv2 : bar_pv1;
         const int qrow = q0 + r;
         float m_run = -INFINITY, l_run = 0.0f;
         for (int j = 0; j < nkv; ++j) {
-            if (!mbar_wait(bar_s, j & 1, abort_flag, lim)) break;
+            const int buf = j & 1;
+            if (!mbar_wait_warp(bar_s(t, buf), (j >> 1) & 1, abort_flag, lim)) break;
             tc_fence_after();
             const int k0 = j * BN;
             const int limit = p.causal ? qrow - k0 : p.N - 1 - k0;
-            softmax_tile(tS, tO, j, limit, p.scale_log2, m_run, l_run);
+            if (!softmax_step(tS0 + BN * buf, tO, j, limit, p.scale_log2, m_run, l_run, bar_pv,
+                              abort_flag, lim))
+                break;
             tc_fence_before();
-            mbar_arrive(bar_p);
+            mbar_arrive(bar_p(t, buf));
         }
         if (t == 1) {
             sL2[r] = l_run;
@@ -417,7 +434,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         } else {
             named_barrier_sync(1, 256);
             const float l2 = sL2[r];
-            const bool ok = mbar_wait(bar_o, 0, abort_flag, lim);
+            const bool ok = mbar_wait_warp(bar_o, 0, abort_flag, lim);
             tc_fence_after();
             if (ok && !*abort_flag) {
                 // ---------------------------------------------------- epilogue
