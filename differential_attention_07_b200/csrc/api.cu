@@ -73,6 +73,13 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int64_t 
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Bytes of the fp16 V copy at the start of the prefill workspace.
+size_t v16_bytes(const diffattn_fwd_args *a)
+{
+    const int64_t HV = a->H_V ? a->H_V : a->H;
+    return align256((size_t)a->B * a->N * HV * 128 * 2);
+}
+
 diffattn_status validate_fwd(const diffattn_fwd_args *a, int grouped)
 {
     if (!a) return DIFFATTN_ERR_INVALID_ARG;
@@ -95,6 +102,7 @@ diffattn_status validate_fwd(const diffattn_fwd_args *a, int grouped)
     if (!a->lambda) return DIFFATTN_ERR_INVALID_ARG;
     for (const void *p : ptrs)
         if (!aligned16(p)) return DIFFATTN_ERR_ALIGNMENT;
+    if (a->gain && !aligned16(a->gain)) return DIFFATTN_ERR_ALIGNMENT;
     const int64_t *strides[6] = {a->q1_stride, a->q2_stride, a->k1_stride, a->k2_stride,
                                  a->v_stride, a->out_stride};
     for (const int64_t *s : strides)
@@ -191,8 +199,10 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     }
 
     int launches = 0;
+    int *tile_counter = reinterpret_cast<int *>(static_cast<char *>(ws) + v16_bytes(a));
     cudaError_t e = da::launch_v_to_f16(a->v, a->v_stride[0], a->v_stride[1], a->v_stride[2], ws,
-                                        (int)a->B, (int)a->N, (int)HV, a->dev_status, s, &launches);
+                                        (int)a->B, (int)a->N, (int)HV, a->dev_status,
+                                        tile_counter, s, &launches);
     if (e != cudaSuccess) return cuda_status(e);
 
     da::PrefillParams p{};
@@ -218,6 +228,7 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     p.out_sh = a->out_stride[2];
     p.dev_status = a->dev_status;
     p.timeout_ns = (uint64_t)(a->timeout_ms ? a->timeout_ms : kDefaultTimeoutMs) * 1000000ull;
+    p.tile_counter = tile_counter;
     e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, p, s, &launches, g_events);
     if (e != cudaSuccess) return cuda_status(e);
     g_last_launches = launches;
@@ -241,8 +252,7 @@ diffattn_status diffattn_fwd_validate(const diffattn_fwd_args *args, int grouped
 size_t diffattn_fwd_workspace_size(const diffattn_fwd_args *a)
 {
     if (!a || a->B <= 0 || a->N <= 0) return 0;
-    const int64_t HV = a->H_V ? a->H_V : a->H;
-    return align256((size_t)a->B * a->N * HV * 128 * 2);
+    return v16_bytes(a) + 256;  // fp16 V copy, then the work-item counter
 }
 
 diffattn_status diffattn_fwd(const diffattn_fwd_args *args, void *workspace, size_t ws_bytes,

@@ -31,6 +31,7 @@ struct PrefillParams {
     int64_t out_sb, out_sn, out_sh;
     int32_t *dev_status;
     uint64_t timeout_ns;
+    int *tile_counter;    // work-item counter in the workspace (zeroed by the V staging kernel)
 };
 
 // Rows per TMA box: a query tile, and a key step of the prefill kernel.
@@ -44,10 +45,11 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
                            const CUtensorMap &k2, const CUtensorMap &v16, const PrefillParams &p,
                            cudaStream_t stream, int *launches, const ProfileEvents &ev);
 
-// bf16 V [B, N, H_V, 128] (strided) -> contiguous fp16 copy in `dst`.
+// bf16 V [B, N, H_V, 128] (strided) -> contiguous fp16 copy in `dst`; also
+// zeroes the prefill kernel's work-item counter.
 cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, void *dst, int B,
-                            int N, int H_V, int32_t *dev_status, cudaStream_t stream,
-                            int *launches);
+                            int N, int H_V, int32_t *dev_status, int *tile_counter,
+                            cudaStream_t stream, int *launches);
 
 struct DecodeParams {
     int B, H, L;

@@ -63,18 +63,38 @@ constexpr uint32_t OFF_Q1 = 0;
 constexpr uint32_t OFF_Q2 = Q_BYTES;
 constexpr uint32_t OFF_STAGE0 = 2 * Q_BYTES;
 constexpr uint32_t OFF_BARS = OFF_STAGE0 + STAGES * STAGE_BYTES;
-// barriers: q, full[S], empty[S], s1[2], s2[2], p1[2], p2[2], pv1, pv2, o.
+// mbarriers, in this order:
+enum : int {
+    B_QFULL = 0,                 // Q1/Q2 of the current tile landed (TMA bytes)
+    B_QFREE = 1,                 // both maps' last score MMA of the tile done (2 commits)
+    B_FULL = 2,                  // [STAGES] K1/K2/V of a step landed (TMA bytes)
+    B_EMPTY = B_FULL + STAGES,   // [STAGES] both maps' P.V of the step done (2 commits)
+    B_S = B_EMPTY + STAGES,      // [2 maps][2 buffers] S ready (commit)
+    B_P = B_S + 4,               // [2 maps][2 buffers] P written (128 arrivals)
+    B_PV = B_P + 4,              // [2 maps] latest P.V into O done (commit)
+    B_O = B_PV + 2,              // all MMAs of the tile done (2 commits)
+    B_OFREE = B_O + 1,           // epilogue finished reading O (256 arrivals)
+    B_LX = B_OFREE + 1,          // row sums exchanged (256 arrivals)
+    B_SSX = B_LX + 1,            // partial sums of squares exchanged (256 arrivals)
+    B_ITEM = B_SSX + 1,          // [ITEM_SLOTS] work item published (1 arrival)
+    B_ITEMFREE = B_ITEM + 4,     // [ITEM_SLOTS] work item read by all 10 reader warps
+    NBARS = B_ITEMFREE + 4
+};
 // S and P barriers come one per S buffer: a softmax may run two steps ahead
-// of the MMA warp's wait, and with one P barrier per map the second arrival
+// of its MMA warp's wait, and with one P barrier per map the second arrival
 // would complete a phase the MMA warp had not yet waited for.  Per buffer,
 // the next use needs the MMA warp's action in between, so no barrier is ever
-// more than one phase ahead of its waiter.
-constexpr int NBARS = 1 + 2 * STAGES + 4 + 4 + 3;
+// more than one phase ahead of its waiter; the same holds for the per-tile
+// barriers because each tile's use of one depends on the previous tile's use
+// of another.
 constexpr uint32_t OFF_TMEM_PTR = OFF_BARS + NBARS * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
-constexpr uint32_t OFF_L2 = (OFF_ABORT + 4 + 15) & ~15u;
-constexpr uint32_t SMEM_USED = OFF_L2 + BM * 4;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for 1024-byte alignment
+constexpr int ITEM_SLOTS = 4;
+constexpr int ITEM_READERS = 10;                         // 2 MMA warps + 8 softmax warps
+constexpr uint32_t OFF_ITEM = OFF_ABORT + 4;             // int [ITEM_SLOTS] work-item ring
+constexpr uint32_t OFF_L = (OFF_ITEM + 4 * ITEM_SLOTS + 15) & ~15u;  // float [2][128] row sums
+constexpr uint32_t OFF_SS = OFF_L + 2 * BM * 4;          // float [2][128] partial sums of squares
+constexpr uint32_t SMEM_BYTES = OFF_SS + 2 * BM * 4;     // dynamic smem is 1024-byte aligned
 
 constexpr uint32_t TM_O1 = 0, TM_O2 = 128, TM_S1 = 256, TM_S2 = 384;
 constexpr uint32_t TMEM_COLS = 512;
@@ -88,10 +108,14 @@ constexpr int REGS_SOFTMAX = 224;
 static_assert(REGS_IO + 2 * REGS_SOFTMAX == 3 * REGS_LAUNCH, "register split must use the pool exactly");
 static_assert(NTHREADS == 384, "three warpgroups");
 
+// The producer warms L2 with the K/V of the step this many steps ahead.
+constexpr int L2_PREFETCH_STEPS = 8;
+
 // P.V MMAs read a stale-max P of at most 2^RESCALE_THRESHOLD.
 constexpr float RESCALE_THRESHOLD = 8.0f;
 
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(OFF_BARS % 8 == 0, "mbarriers are 8-byte aligned");
 static_assert(kPrefillQRows == BM && kPrefillKeyRows == BN, "TMA boxes match the tiles");
 static_assert(OFF_STAGE0 % 1024 == 0 && STAGE_BYTES % 1024 == 0 && K_BYTES % 1024 == 0,
               "SW128 atoms need 1 KB alignment");
@@ -171,10 +195,10 @@ constexpr uint32_t SOFT_EXP_MASK = 0xA4u;  // pairs 2, 5, 7 of every 8
 // when the max moved (after the previous P.V product into it has finished),
 // and writes P (fp16) over the first 32 columns of the S buffer.  Returns
 // false if a bounded wait gave up.
-__device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, int j, int limit,
+__device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, bool first, int limit,
                                              float scale_log2, float &m_run, float &l_run,
-                                             uint32_t bar_pv, volatile int *abort_flag,
-                                             uint64_t lim)
+                                             uint32_t bar_pv, uint32_t pv_parity,
+                                             volatile int *abort_flag, uint64_t lim)
 {
     uint32_t v[2][32];
     tmem_ld32(tS, v[0]);
@@ -206,9 +230,10 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, int j, in
     const bool need = tmax > m_run + RESCALE_THRESHOLD;
     const float m_new = need ? tmax : m_run;
     const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;  // ex2(-inf) = 0
-    if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // O holds P.V products up to step j-1; the last one must be finished.
-        if (!mbar_wait_warp(bar_pv, (j - 1) & 1, abort_flag, lim)) return false;
+    if (!first && __any_sync(0xffffffffu, need)) {
+        // O holds P.V products up to the previous step; the last one must be
+        // finished before the row is rescaled.
+        if (!mbar_wait_warp(bar_pv, pv_parity, abort_flag, lim)) return false;
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -251,41 +276,52 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                    const __grid_constant__ CUtensorMap tm_k1, const __grid_constant__ CUtensorMap tm_k2,
                    const __grid_constant__ CUtensorMap tm_v, const PrefillParams p)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_addr(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    const Work w = work_of(blockIdx.x, p);
-    const int nh = w.h / (p.H / p.H_N), vh = w.h / (p.H / p.H_V);
-    const int q0 = w.qt * BM;
+    if (sbase & 1023u) {  // the 128-byte-swizzled tiles need 1 KB alignment
+        if (threadIdx.x == 0) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
+        return;
+    }
+    const int total = p.B * p.H * p.num_qt;
+    int *sItem = reinterpret_cast<int *>(smem + OFF_ITEM);
     const int n_steps_all = (p.N + BN - 1) / BN;
-    const int nkv = p.causal ? min(n_steps_all, (q0 + BM) / BN) : n_steps_all;
+    auto steps_of = [&](const Work &w) {
+        const int q0 = w.qt * BM;
+        return p.causal ? min(n_steps_all, (q0 + BM) / BN) : n_steps_all;
+    };
 
-    const uint32_t bar_q = sbase + OFF_BARS;
-    auto bar_full = [&](int s) { return sbase + OFF_BARS + 8 * (1 + s); };
-    auto bar_empty = [&](int s) { return sbase + OFF_BARS + 8 * (1 + STAGES + s); };
-    const uint32_t bar_s1_0 = sbase + OFF_BARS + 8 * (1 + 2 * STAGES);  // s1[2], then s2[2]
-    auto bar_s = [&](int t, int b) { return bar_s1_0 + 8 * (2 * t + b); };
-    auto bar_p = [&](int t, int b) { return bar_s1_0 + 32 + 8 * (2 * t + b); };
-    const uint32_t bar_pv1 = bar_s1_0 + 64, bar_pv2 = bar_s1_0 + 72;
-    const uint32_t bar_o = bar_s1_0 + 80;
+    auto bar = [&](int i) { return sbase + OFF_BARS + 8 * i; };
+    auto bar_full = [&](int s) { return bar(B_FULL + s); };
+    auto bar_empty = [&](int s) { return bar(B_EMPTY + s); };
+    auto bar_s = [&](int t, int b) { return bar(B_S + 2 * t + b); };
+    auto bar_p = [&](int t, int b) { return bar(B_P + 2 * t + b); };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_ABORT);
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + OFF_TMEM_PTR);
-    float *sL2 = reinterpret_cast<float *>(smem + OFF_L2);
+    float *sL = reinterpret_cast<float *>(smem + OFF_L);
+    float *sSS = reinterpret_cast<float *>(smem + OFF_SS);
 
     if (threadIdx.x == 0) {
-        mbar_init(bar_q, 1);
+        mbar_init(bar(B_QFULL), 1);
+        mbar_init(bar(B_QFREE), 2);
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar_full(s), 1);
-            mbar_init(bar_empty(s), 2);  // one commit from each map's MMA warp
+            mbar_init(bar_empty(s), 2);
         }
-        for (int i = 0; i < 4; ++i) mbar_init(bar_s1_0 + 8 * i, 1);
-        for (int i = 0; i < 4; ++i) mbar_init(bar_s1_0 + 32 + 8 * i, 128);
-        mbar_init(bar_pv1, 1);
-        mbar_init(bar_pv2, 1);
-        mbar_init(bar_o, 2);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(bar(B_S + i), 1);
+            mbar_init(bar(B_P + i), 128);
+        }
+        mbar_init(bar(B_PV), 1);
+        mbar_init(bar(B_PV + 1), 1);
+        mbar_init(bar(B_O), 2);
+        mbar_init(bar(B_OFREE), 256);
+        mbar_init(bar(B_LX), 256);
+        mbar_init(bar(B_SSX), 256);
+        for (int i = 0; i < ITEM_SLOTS; ++i) {
+            mbar_init(bar(B_ITEM + i), 1);
+            mbar_init(bar(B_ITEMFREE + i), ITEM_READERS);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -298,6 +334,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_after();
     const uint32_t tbase = *tmem_ptr;
     const uint64_t lim = p.timeout_ns;
+
+    // Work items are handed out dynamically (an atomic counter in global
+    // memory, zeroed by the V staging kernel that runs first): the producer
+    // takes the next one and publishes it in a ring of ITEM_SLOTS; the other
+    // roles read item k from slot k % ITEM_SLOTS and release the slot.  The
+    // producer reuses a slot only after all ten reader warps released it (with
+    // short tiles it can run several tiles ahead).  A negative item ends the
+    // loop.
+    auto next_item = [&](int k) -> int {
+        const int slot = k % ITEM_SLOTS;
+        if (!mbar_wait_warp(bar(B_ITEM + slot), (k / ITEM_SLOTS) & 1, abort_flag, p.timeout_ns))
+            return -1;
+        const int item = *reinterpret_cast<volatile int *>(&sItem[slot]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_ITEMFREE + slot));
+        return item;
+    };
 
     // Register split: 128 x REGS_LAUNCH = 128 x REGS_IO + 256 x REGS_SOFTMAX
     // (the host launches only when the kernel was built with REGS_LAUNCH).
@@ -315,32 +368,70 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             prefetch_tensormap(&tm_k1);
             prefetch_tensormap(&tm_k2);
             prefetch_tensormap(&tm_v);
-            mbar_arrive_expect_tx(bar_q, 2 * Q_BYTES);
-            tma_load_4d(sbase + OFF_Q1, &tm_q1, bar_q, 0, q0, w.h, w.b, stream);
-            tma_load_4d(sbase + OFF_Q2, &tm_q2, bar_q, 0, q0, nh, w.b, stream);
         }
         __syncwarp();
-        int issued = 0;
-        for (int j = 0; j < nkv; ++j) {
-            const int s = j % STAGES;
-            if (j >= STAGES && !mbar_wait_warp(bar_empty(s), ((j / STAGES) - 1) & 1, abort_flag, lim))
+        int g = 0, tiles = 0;
+        bool ok = true;
+        for (;; ++tiles) {
+            const int slot = tiles % ITEM_SLOTS;
+            if (tiles >= ITEM_SLOTS &&
+                !(ok = mbar_wait_warp(bar(B_ITEMFREE + slot), ((tiles / ITEM_SLOTS) - 1) & 1, abort_flag, lim)))
                 break;
-            const uint32_t st = sbase + OFF_STAGE0 + s * STAGE_BYTES;
-            const int k0 = j * BN;
+            int item = -1;
+            if (lane == 0) {
+                item = *abort_flag ? total : atomicAdd(p.tile_counter, 1);
+                sItem[slot] = item < total ? item : -1;
+                mbar_arrive(bar(B_ITEM + slot));
+            }
+            item = __shfl_sync(0xffffffffu, item, 0);
+            if (item >= total) break;
+            const Work w = work_of(item, p);
+            const int nh = w.h / (p.H / p.H_N), vh = w.h / (p.H / p.H_V);
+            const int nkv = steps_of(w);
+            // The previous tile's score MMAs must be done with Q.
+            if (tiles > 0 && !(ok = mbar_wait_warp(bar(B_QFREE), (tiles - 1) & 1, abort_flag, lim)))
+                break;
             if (elect_one()) {
-                mbar_arrive_expect_tx(bar_full(s), STAGE_BYTES);
-                tma_load_4d(st, &tm_k1, bar_full(s), 0, k0, w.h, w.b, keep);
-                tma_load_4d(st + K_BYTES, &tm_k2, bar_full(s), 0, k0, nh, w.b, keep);
-                tma_load_4d(st + 2 * K_BYTES, &tm_v, bar_full(s), 0, k0, vh, w.b, keep);
-                tma_load_4d(st + 2 * K_BYTES + VHALF_BYTES, &tm_v, bar_full(s), 64, k0, vh, w.b, keep);
+                mbar_arrive_expect_tx(bar(B_QFULL), 2 * Q_BYTES);
+                tma_load_4d(sbase + OFF_Q1, &tm_q1, bar(B_QFULL), 0, w.qt * BM, w.h, w.b, stream);
+                tma_load_4d(sbase + OFF_Q2, &tm_q2, bar(B_QFULL), 0, w.qt * BM, nh, w.b, stream);
             }
             __syncwarp();
-            issued = j + 1;
+            for (int j = 0; j < nkv; ++j, ++g) {
+                const int s = g % STAGES;
+                if (g >= STAGES &&
+                    !(ok = mbar_wait_warp(bar_empty(s), ((g / STAGES) - 1) & 1, abort_flag, lim)))
+                    break;
+                const uint32_t st = sbase + OFF_STAGE0 + s * STAGE_BYTES;
+                const int k0 = j * BN;
+                if (elect_one()) {
+                    // Warm L2 with the K/V tiles of a later step of this tile
+                    // (the stage ring alone cannot hide an HBM miss).
+                    if (j + L2_PREFETCH_STEPS < nkv) {
+                        const int kp = k0 + L2_PREFETCH_STEPS * BN;
+                        tma_prefetch_l2_4d(&tm_k1, 0, kp, w.h, w.b);
+                        tma_prefetch_l2_4d(&tm_k2, 0, kp, nh, w.b);
+                        tma_prefetch_l2_4d(&tm_v, 0, kp, vh, w.b);
+                        tma_prefetch_l2_4d(&tm_v, 64, kp, vh, w.b);
+                    }
+                    mbar_arrive_expect_tx(bar_full(s), STAGE_BYTES);
+                    tma_load_4d(st, &tm_k1, bar_full(s), 0, k0, w.h, w.b, keep);
+                    tma_load_4d(st + K_BYTES, &tm_k2, bar_full(s), 0, k0, nh, w.b, keep);
+                    tma_load_4d(st + 2 * K_BYTES, &tm_v, bar_full(s), 0, k0, vh, w.b, keep);
+                    tma_load_4d(st + 2 * K_BYTES + VHALF_BYTES, &tm_v, bar_full(s), 64, k0, vh, w.b, keep);
+                }
+                __syncwarp();
+            }
+            if (!ok) {
+                ++tiles;
+                break;
+            }
         }
         // No load of ours may land after the CTA has gone: wait for all of them.
-        bool drained = mbar_wait_drain(bar_q, 0, lim);
-        for (int j = (issued > STAGES ? issued - STAGES : 0); j < issued; ++j)
-            drained &= mbar_wait_drain(bar_full(j % STAGES), (j / STAGES) & 1, lim);
+        bool drained = true;
+        if (tiles > 0) drained = mbar_wait_drain(bar(B_QFULL), (tiles - 1) & 1, lim);
+        for (int k = (g > STAGES ? g - STAGES : 0); k < g; ++k)
+            drained &= mbar_wait_drain(bar_full(k % STAGES), (k / STAGES) & 1, lim);
         if (!__all_sync(0xffffffffu, drained) && lane == 0) *abort_flag = 1;
       } else if (warp == 1 || warp == 2) {
         // ------------------------------------------------------------ MMA issuers
@@ -353,7 +444,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         constexpr uint32_t ID_PV = idesc_f16(0, 0, 1, BM, HDV);  // f16 x f16, B (V) MN-major
         const uint32_t qa = sbase + (t ? OFF_Q2 : OFF_Q1);
         const uint32_t tS = tbase + (t ? TM_S2 : TM_S1), tO = tbase + (t ? TM_O2 : TM_O1);
-        const uint32_t bar_pv = t ? bar_pv2 : bar_pv1;
+        const uint32_t bar_pv = bar(B_PV + t);
         auto issue_s = [&](int s, int buf) {
             const uint32_t ka = sbase + OFF_STAGE0 + s * STAGE_BYTES + (t ? K_BYTES : 0);
 #pragma unroll
@@ -374,119 +465,160 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 __syncwarp();
             }
         };
-        auto commit = [&](uint32_t bar) {
-            if (elect_one()) mma_commit(bar);
+        auto commit = [&](uint32_t b) {
+            if (elect_one()) mma_commit(b);
             __syncwarp();
         };
-        bool ok = mbar_wait_warp(bar_q, 0, abort_flag, lim);
-        for (int jj = 0; ok && jj < 2 && jj < nkv; ++jj) {
-            if (!(ok = mbar_wait_warp(bar_full(jj), 0, abort_flag, lim))) break;
-            tc_fence_after();
-            issue_s(jj, jj);
-            commit(bar_s(t, jj));
-        }
-        for (int j = 0; ok && j < nkv; ++j) {
-            const int s = j % STAGES, buf = j & 1;
-            if (!(ok = mbar_wait_warp(bar_p(t, buf), (j >> 1) & 1, abort_flag, lim))) break;
-            tc_fence_after();
-            issue_pv(s, buf, j > 0);
-            commit(bar_pv);
-            commit(bar_empty(s));  // the stage is free once both maps' P.V have read it
-            if (j + 2 < nkv) {
-                const int s2 = (j + 2) % STAGES;
-                if (!(ok = mbar_wait_warp(bar_full(s2), ((j + 2) / STAGES) & 1, abort_flag, lim))) break;
+        int g = 0;
+        bool ok = true;
+        for (int tiles = 0;; ++tiles) {
+            const int item = next_item(tiles);
+            if (item < 0) break;
+            const Work w = work_of(item, p);
+            const int nkv = steps_of(w);
+            if (!(ok = mbar_wait_warp(bar(B_QFULL), tiles & 1, abort_flag, lim))) break;
+            for (int jj = 0; jj < 2 && jj < nkv; ++jj) {
+                const int gg = g + jj;
+                if (!(ok = mbar_wait_warp(bar_full(gg % STAGES), (gg / STAGES) & 1, abort_flag, lim))) break;
                 tc_fence_after();
-                issue_s(s2, buf);
-                commit(bar_s(t, buf));
+                issue_s(gg % STAGES, gg & 1);
+                commit(bar_s(t, gg & 1));
+                if (jj == nkv - 1) commit(bar(B_QFREE));
             }
+            for (int j = 0; ok && j < nkv; ++j) {
+                const int gg = g + j, s = gg % STAGES, buf = gg & 1;
+                if (!(ok = mbar_wait_warp(bar_p(t, buf), (gg >> 1) & 1, abort_flag, lim))) break;
+                // The first P.V of a tile overwrites O: the previous tile's
+                // epilogue must have read it.
+                if (j == 0 && tiles > 0 &&
+                    !(ok = mbar_wait_warp(bar(B_OFREE), (tiles - 1) & 1, abort_flag, lim)))
+                    break;
+                tc_fence_after();
+                issue_pv(s, buf, j > 0);
+                commit(bar_pv);
+                commit(bar_empty(s));  // the stage is free once both maps' P.V have read it
+                if (j + 2 < nkv) {
+                    const int g2 = gg + 2;
+                    if (!(ok = mbar_wait_warp(bar_full(g2 % STAGES), (g2 / STAGES) & 1, abort_flag, lim)))
+                        break;
+                    tc_fence_after();
+                    issue_s(g2 % STAGES, buf);
+                    commit(bar_s(t, buf));
+                    if (j + 2 == nkv - 1) commit(bar(B_QFREE));
+                }
+            }
+            if (!ok) break;
+            commit(bar(B_O));  // completes once both maps' MMAs of the tile are done
+            g += nkv;
         }
-        commit(bar_o);  // bar_o completes when both maps' MMAs are done
         // Nothing of ours may still run on the tensor cores at teardown.
-        const bool drained = mbar_wait_drain(bar_o, 0, lim);
+        commit(bar(B_PV + t));
+        const bool drained = mbar_wait_drain(bar(B_PV + t), g & 1, lim);
         if (!__all_sync(0xffffffffu, drained) && lane == 0) *abort_flag = 1;
       }
     } else {
         regs_increase<REGS_SOFTMAX>();
-        // ------------------------------------------------------------ softmax
+        // ------------------------------------------------------------ softmax + epilogue
         const int t = (warp >= 8) ? 1 : 0;
         const int r = (warp & 3) * 32 + lane;
         const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
         const uint32_t tS0 = tbase + lane_off + (t ? TM_S2 : TM_S1);
         const uint32_t tO = tbase + lane_off + (t ? TM_O2 : TM_O1);
-        const uint32_t bar_pv = t ? bar_pv2 : bar_pv1;
-        const int qrow = q0 + r;
-        float m_run = -INFINITY, l_run = 0.0f;
-        for (int j = 0; j < nkv; ++j) {
-            const int buf = j & 1;
-            if (!mbar_wait_warp(bar_s(t, buf), (j >> 1) & 1, abort_flag, lim)) break;
+        const uint32_t tO1 = tbase + lane_off + TM_O1, tO2 = tbase + lane_off + TM_O2;
+        const uint32_t bar_pv = bar(B_PV + t);
+        int g = 0;
+        bool ok = true;
+        for (int tiles = 0;; ++tiles) {
+            const int item = next_item(tiles);
+            if (item < 0) break;
+            const Work w = work_of(item, p);
+            const int nkv = steps_of(w);
+            const int qrow = w.qt * BM + r;
+            // The epilogue's lambda and gain: load / prefetch them now so the
+            // global-memory latency hides behind the softmax loop.
+            const float lam = ld_early_f32(p.lambda + w.h);
+            const float *gain = p.gain ? p.gain + (size_t)w.h * HDV + 64 * t : nullptr;
+            if (gain && lane < 2) prefetch_l1(gain + 32 * lane);
+            float m_run = -INFINITY, l_run = 0.0f;
+            for (int j = 0; j < nkv; ++j) {
+                const int gg = g + j, buf = gg & 1;
+                if (!(ok = mbar_wait_warp(bar_s(t, buf), (gg >> 1) & 1, abort_flag, lim))) break;
+                tc_fence_after();
+                const int k0 = j * BN;
+                const int limit = p.causal ? qrow - k0 : p.N - 1 - k0;
+                if (!(ok = softmax_step(tS0 + BN * buf, tO, j == 0, limit, p.scale_log2, m_run, l_run,
+                                        bar_pv, (gg - 1) & 1, abort_flag, lim)))
+                    break;
+                tc_fence_before();
+                mbar_arrive(bar_p(t, buf));
+            }
+            if (!ok) break;
+            g += nkv;
+            // ---------------------------------------------------- epilogue
+            // Both warpgroups finish the tile: warpgroup t writes the output
+            // columns [64 t, 64 t + 64) of every row.  D = (O1 - r O2) / l1
+            // with r = lambda l1 / l2 (one fused multiply-add per element;
+            // identical maps with lambda = 1 cancel exactly), then the RMS
+            // norm over all 128 columns, whose sum of squares is exchanged.
+            sL[t * BM + r] = l_run;
+            mbar_arrive(bar(B_LX));
+            if (!(ok = mbar_wait_warp(bar(B_LX), tiles & 1, abort_flag, lim))) break;
+            if (!(ok = mbar_wait_warp(bar(B_O), tiles & 1, abort_flag, lim))) break;
             tc_fence_after();
-            const int k0 = j * BN;
-            const int limit = p.causal ? qrow - k0 : p.N - 1 - k0;
-            if (!softmax_step(tS0 + BN * buf, tO, j, limit, p.scale_log2, m_run, l_run, bar_pv,
-                              abort_flag, lim))
-                break;
+            const float l1 = sL[r], l2 = sL[BM + r];
+            const float inv1 = 1.0f / l1, r2 = lam * l1 / l2;
+            const uint32_t c0 = 64 * t;
+            // One read of this half of O1 and O2; D stays in registers, and O
+            // is released to the MMA warps (the next tile's first P.V
+            // overwrites it) as soon as the read has completed.
+            uint32_t oa[2][32], ob[2][32];
+            tmem_ld32(tO1 + c0, oa[0]);
+            tmem_ld32(tO1 + c0 + 32, oa[1]);
+            tmem_ld32(tO2 + c0, ob[0]);
+            tmem_ld32(tO2 + c0 + 32, ob[1]);
+            tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(bar_p(t, buf));
-        }
-        if (t == 1) {
-            sL2[r] = l_run;
-            named_barrier_sync(1, 256);
-        } else {
-            named_barrier_sync(1, 256);
-            const float l2 = sL2[r];
-            const bool ok = mbar_wait_warp(bar_o, 0, abort_flag, lim);
-            tc_fence_after();
-            if (ok && !*abort_flag) {
-                // ---------------------------------------------------- epilogue
-                const float lam = p.lambda[w.h];
-                // D = (O1 - r O2) / l1 with r = lambda l1 / l2: one fused multiply-add
-                // per element, and identical maps with lambda = 1 cancel exactly.
-                const float inv1 = 1.0f / l_run, r2 = lam * l_run / l2;
-                const uint32_t tO1 = tbase + lane_off + TM_O1, tO2 = tbase + lane_off + TM_O2;
-                float rn = 1.0f;
-                if (p.apply_norm) {
-                    float ss = 0.0f;
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t a[32], bb[32];
-                        tmem_ld32(tO1 + 32 * c, a);
-                        tmem_ld32(tO2 + 32 * c, bb);
-                        tmem_wait_ld();
+            mbar_arrive(bar(B_OFREE));
+            float d[64];
+            float ss = 0.0f;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const float dd = fmaf(-r2, __uint_as_float(bb[i]), __uint_as_float(a[i])) * inv1;
-                            ss += dd * dd;
-                        }
-                    }
-                    rn = rsqrtf(ss * (1.0f / HDV) + p.eps);
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    d[32 * c + i] = fmaf(-r2, __uint_as_float(ob[c][i]), __uint_as_float(oa[c][i])) * inv1;
+                    ss = fmaf(d[32 * c + i], d[32 * c + i], ss);
                 }
-                const float *gain = p.gain ? p.gain + (size_t)w.h * HDV : nullptr;
-                uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) +
-                                2 * ((int64_t)w.b * p.out_sb + (int64_t)qrow * p.out_sn +
-                                     (int64_t)w.h * p.out_sh);
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t a[32], bb[32];
-                    tmem_ld32(tO1 + 32 * c, a);
-                    tmem_ld32(tO2 + 32 * c, bb);
-                    tmem_wait_ld();
-                    uint32_t y[16];
+            sSS[t * BM + r] = ss;
+            mbar_arrive(bar(B_SSX));
+            float gv[64];  // this half's gain, loaded while the sums are exchanged
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        float y0 = fmaf(-r2, __uint_as_float(bb[2 * i]), __uint_as_float(a[2 * i])) * (inv1 * rn);
-                        float y1 = fmaf(-r2, __uint_as_float(bb[2 * i + 1]), __uint_as_float(a[2 * i + 1])) * (inv1 * rn);
-                        if (gain) {
-                            y0 *= __ldg(gain + 32 * c + 2 * i);
-                            y1 *= __ldg(gain + 32 * c + 2 * i + 1);
-                        }
-                        y[i] = pack_bf162(y0, y1);
-                    }
-                    if (qrow < p.N) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + 64 * c);
+            for (int i = 0; i < 16; ++i) {
+                const float4 g4 = gain ? __ldg(reinterpret_cast<const float4 *>(gain) + i)
+                                       : make_float4(1.f, 1.f, 1.f, 1.f);
+                gv[4 * i] = g4.x;
+                gv[4 * i + 1] = g4.y;
+                gv[4 * i + 2] = g4.z;
+                gv[4 * i + 3] = g4.w;
+            }
+            if (!(ok = mbar_wait_warp(bar(B_SSX), tiles & 1, abort_flag, lim))) break;
+            const float rn =
+                p.apply_norm ? rsqrtf((sSS[r] + sSS[BM + r]) * (1.0f / HDV) + p.eps) : 1.0f;
+            uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) +
+                            2 * ((int64_t)w.b * p.out_sb + (int64_t)qrow * p.out_sn +
+                                 (int64_t)w.h * p.out_sh + c0);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
-                    }
+            for (int c = 0; c < 2; ++c) {
+                uint32_t y[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    y[i] = pack_bf162(d[32 * c + 2 * i] * rn * gv[32 * c + 2 * i],
+                                      d[32 * c + 2 * i + 1] * rn * gv[32 * c + 2 * i + 1]);
+                }
+                if (qrow < p.N) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 64 * c);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
                 }
             }
         }
@@ -503,8 +635,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb, int64_t sn,
                                 int64_t sh, __half *__restrict__ dst, int B, int N, int H_V,
-                                int32_t *dev_status)
+                                int32_t *dev_status, int *tile_counter)
 {
+    // The prefill kernel that follows on the stream hands out its work items
+    // from this counter.
+    if (blockIdx.x == 0 && threadIdx.x == 0) *tile_counter = 0;
     // One thread per 8 consecutive V elements (16 bytes in, 16 bytes out).
     const int64_t total = (int64_t)B * N * H_V * (HDV / 8);
     bool overflow = false;
@@ -554,8 +689,16 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    const int grid = p.B * p.H * p.num_qt;
-    if (grid == 0) return cudaSuccess;
+    static int num_sms = 0;
+    if (num_sms == 0) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+    }
+    const int total = p.B * p.H * p.num_qt;
+    if (total == 0) return cudaSuccess;
+    const int grid = total < num_sms ? total : num_sms;  // persistent: one CTA per SM
     if (ev.start) cudaEventRecord(ev.start, stream);
     prefill_kernel<<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, p);
     ++*launches;
@@ -564,16 +707,17 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
 }
 
 cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, void *dst, int B,
-                            int N, int H_V, int32_t *dev_status, cudaStream_t stream, int *launches)
+                            int N, int H_V, int32_t *dev_status, int *tile_counter,
+                            cudaStream_t stream, int *launches)
 {
     const int64_t total = (int64_t)B * N * H_V * (HDV / 8);
-    if (total == 0) return cudaSuccess;
+    if (total == 0) return cudaSuccess;  // nothing to stage; the prefill is skipped too
     const int threads = 256;
     int blocks = (int)((total + threads - 1) / threads);
     if (blocks > 148 * 16) blocks = 148 * 16;
     v_to_f16_kernel<<<blocks, threads, 0, stream>>>(static_cast<const __nv_bfloat16 *>(v), sb, sn,
                                                     sh, static_cast<__half *>(dst), B, N, H_V,
-                                                    dev_status);
+                                                    dev_status, tile_counter);
     ++*launches;
     return cudaGetLastError();
 }

@@ -62,7 +62,8 @@ typedef enum diffattn_status {
  * ptr + b*stride[0] + n*stride[1] + head*stride[2] + c.
  *   q1, k1: [B, N, H,   64]     q2, k2: [B, N, H_N, 64]
  *   v:      [B, N, H_V, 128]    out:    [B, N, H,   128]
- *   lambda: [H] fp32 device     gain:   [H, 128] fp32 device, or NULL for 1. */
+ *   lambda: [H] fp32 device     gain:   [H, 128] fp32 device (16-byte aligned,
+ *                                       contiguous), or NULL for 1. */
 typedef struct diffattn_fwd_args {
     int64_t B, N, H, H_N, H_V;
     int64_t d, dv;
@@ -93,7 +94,7 @@ diffattn_status diffattn_grouped_fwd(const diffattn_fwd_args *args, void *worksp
                                      size_t ws_bytes, void *stream);
 
 /* Bytes of workspace diffattn_fwd / diffattn_grouped_fwd need for `args`
- * (an fp16 copy of V for the tensor-core P.V product).                       */
+ * (an fp16 copy of V for the tensor-core P.V product, and a work counter).  */
 size_t diffattn_fwd_workspace_size(const diffattn_fwd_args *args);
 
 /* Host-only argument check of a prefill call: the status diffattn_fwd (or,

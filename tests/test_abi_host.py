@@ -96,6 +96,9 @@ def test_fwd_validation(L):
     a = _fake_fwd_args()
     a.flags = 8
     assert _v(L, a) == 1
+    a = _fake_fwd_args()
+    a.gain = (1 << 22) + 4
+    assert _v(L, a) == 3                          # gain must be 16-byte aligned
     a = _fake_fwd_args(B=0)
     a.q1 = 0
     assert _v(L, a) == 0                          # empty batch: nothing to check
@@ -117,7 +120,7 @@ def test_fwd_rejects_before_launch(L):
     a = _fake_fwd_args()
     assert L.diffattn_fwd(ctypes.byref(a), None, 0, None) == 4          # workspace missing
     need = L.diffattn_fwd_workspace_size(ctypes.byref(a))
-    assert need == 2 * 300 * 4 * 128 * 2
+    assert need == 2 * 300 * 4 * 128 * 2 + 256
     assert L.diffattn_fwd(ctypes.byref(a), ctypes.c_void_p(1 << 30), need - 1, None) == 4
     assert L.diffattn_fwd(ctypes.byref(a), ctypes.c_void_p((1 << 30) + 16), need, None) == 3
     assert L.diffattn_grouped_fwd(ctypes.byref(_fake_fwd_args(H=6, H_N=4)), None, 0, None) == 1

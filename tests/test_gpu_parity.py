@@ -73,6 +73,18 @@ def test_prefill_multi_tile_many_heads(cuda_ok):
     _assert_parity(y, _oracle_prefill(x))
 
 
+@pytest.mark.parametrize("B,N,H", [(40, 100, 8), (64, 64, 6), (8, 700, 8)])
+def test_prefill_many_tiles_per_cta(cuda_ok, B, N, H):
+    """More query tiles than SMs, many of them one or two key steps long, so
+    each persistent CTA runs several tiles back to back and the work-item
+    ring wraps around."""
+    x = inputs.prefill_inputs(B, N, H, seed=B + N + H, lam=(0.0, 0.9), gain_std=0.1)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = _run_prefill(x, status=st)
+    assert st.item() == 0
+    _assert_parity(y, _oracle_prefill(x))
+
+
 @pytest.mark.parametrize("N", [100, 384, 450])
 def test_prefill_non_causal(cuda_ok, N):
     x = inputs.prefill_inputs(2, N, 2, seed=5 + N, lam=(0.2, 0.8), gain_std=0.1)
