@@ -73,6 +73,21 @@ def test_prefill_multi_tile_many_heads(cuda_ok):
     _assert_parity(y, _oracle_prefill(x))
 
 
+@pytest.mark.parametrize("N", [200, 640])
+def test_prefill_growing_scores_force_rescales(cuda_ok, N):
+    """Key magnitudes that grow along the sequence (and a late spike) make the
+    running maximum jump by more than 2^8 repeatedly, so the kernel's stale
+    maximum must be corrected (O rescaled, the step's exponentials redone)."""
+    x = inputs.prefill_inputs(2, N, 3, seed=N + 1, lam=(0.2, 0.8), gain_std=0.1)
+    grow = (1.0 + 5.0 * torch.arange(N, dtype=torch.float32) / N)[None, :, None, None]
+    x["k1"] = (x["k1"].float() * grow).to(torch.bfloat16)
+    x["k2"] = (x["k2"].float() * grow.flip(1)).to(torch.bfloat16)
+    spike = N - N // 5
+    x["k1"][:, spike] = (x["q1"][:, -1].float() * 4.0).to(torch.bfloat16)
+    y = _run_prefill(x)
+    _assert_parity(y, _oracle_prefill(x))
+
+
 @pytest.mark.parametrize("B,N,H", [(40, 100, 8), (64, 64, 6), (8, 700, 8)])
 def test_prefill_many_tiles_per_cta(cuda_ok, B, N, H):
     """More query tiles than SMs, many of them one or two key steps long, so
