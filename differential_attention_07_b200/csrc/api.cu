@@ -235,6 +235,52 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     return DIFFATTN_OK;
 }
 
+// Fill the decode parameters and launch (arguments already validated; the
+// partials buffer holds at least diffattn_decode_workspace_size bytes).
+diffattn_status run_decode(const diffattn_decode_args *a, float *partials, void *stream)
+{
+    da::DecodeParams p{};
+    p.B = (int)a->B;
+    p.H = (int)a->H;
+    p.L = (int)a->L;
+    p.splits = decode_splits(a->B, a->H, a->L, a->num_splits);
+    p.chunk = decode_chunk(a->L, p.splits);
+    p.scale_log2 = a->scale * 1.4426950408889634f;
+    p.eps = a->eps;
+    p.apply_norm = (a->flags & DIFFATTN_FLAG_APPLY_NORM) ? 1 : 0;
+    p.q1 = a->q1;
+    p.q2 = a->q2;
+    p.k1 = a->k1;
+    p.k2 = a->k2;
+    p.v = a->v;
+    p.q1_sb = a->q1_stride[0];
+    p.q1_sh = a->q1_stride[1];
+    p.q2_sb = a->q2_stride[0];
+    p.q2_sh = a->q2_stride[1];
+    p.k1_sb = a->k1_stride[0];
+    p.k1_sh = a->k1_stride[1];
+    p.k1_sl = a->k1_stride[2];
+    p.k2_sb = a->k2_stride[0];
+    p.k2_sh = a->k2_stride[1];
+    p.k2_sl = a->k2_stride[2];
+    p.v_sb = a->v_stride[0];
+    p.v_sh = a->v_stride[1];
+    p.v_sl = a->v_stride[2];
+    p.out = a->out;
+    p.out_sb = a->out_stride[0];
+    p.out_sh = a->out_stride[1];
+    p.kv_len = a->kv_len;
+    p.lambda = a->lambda;
+    p.gain = a->gain;
+    p.partials = partials;
+    p.dev_status = a->dev_status;
+    int launches = 0;
+    cudaError_t e = da::launch_decode(p, static_cast<cudaStream_t>(stream), &launches, g_events);
+    if (e != cudaSuccess) return cuda_status(e);
+    g_last_launches = launches;
+    return DIFFATTN_OK;
+}
+
 }  // namespace
 
 void da::set_internal_error(const char *text)
@@ -296,46 +342,27 @@ diffattn_status diffattn_decode(const diffattn_decode_args *a, void *workspace, 
     const size_t need = diffattn_decode_workspace_size(a->B, a->H, a->L, a->num_splits);
     if (!workspace || ws_bytes < need) return DIFFATTN_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return DIFFATTN_ERR_ALIGNMENT;
-    da::DecodeParams p{};
-    p.B = (int)a->B;
-    p.H = (int)a->H;
-    p.L = (int)a->L;
-    p.splits = decode_splits(a->B, a->H, a->L, a->num_splits);
-    p.chunk = decode_chunk(a->L, p.splits);
-    p.scale_log2 = a->scale * 1.4426950408889634f;
-    p.eps = a->eps;
-    p.apply_norm = (a->flags & DIFFATTN_FLAG_APPLY_NORM) ? 1 : 0;
-    p.q1 = a->q1;
-    p.q2 = a->q2;
-    p.k1 = a->k1;
-    p.k2 = a->k2;
-    p.v = a->v;
-    p.q1_sb = a->q1_stride[0];
-    p.q1_sh = a->q1_stride[1];
-    p.q2_sb = a->q2_stride[0];
-    p.q2_sh = a->q2_stride[1];
-    p.k1_sb = a->k1_stride[0];
-    p.k1_sh = a->k1_stride[1];
-    p.k1_sl = a->k1_stride[2];
-    p.k2_sb = a->k2_stride[0];
-    p.k2_sh = a->k2_stride[1];
-    p.k2_sl = a->k2_stride[2];
-    p.v_sb = a->v_stride[0];
-    p.v_sh = a->v_stride[1];
-    p.v_sl = a->v_stride[2];
-    p.out = a->out;
-    p.out_sb = a->out_stride[0];
-    p.out_sh = a->out_stride[1];
-    p.kv_len = a->kv_len;
-    p.lambda = a->lambda;
-    p.gain = a->gain;
-    p.partials = static_cast<float *>(workspace);
-    p.dev_status = a->dev_status;
-    int launches = 0;
-    cudaError_t e = da::launch_decode(p, static_cast<cudaStream_t>(stream), &launches, g_events);
+    return run_decode(a, static_cast<float *>(workspace), stream);
+}
+
+diffattn_status diffattn_decode_noalloc(const diffattn_decode_args *a, void *stream)
+{
+    g_last_launches = 0;
+    g_last_error[0] = 0;
+    diffattn_status st = validate_decode(a);
+    if (st != DIFFATTN_OK) return st;
+    if (a->B == 0) return DIFFATTN_OK;
+    const size_t need = diffattn_decode_workspace_size(a->B, a->H, a->L, a->num_splits);
+    if (need > da::kNoAllocScratchBytes) {
+        std::snprintf(g_last_error, sizeof g_last_error,
+                      "decode partials need %zu bytes; the no-allocation scratch holds %zu",
+                      need, da::kNoAllocScratchBytes);
+        return DIFFATTN_ERR_WORKSPACE;
+    }
+    float *scratch = nullptr;
+    const cudaError_t e = da::decode_noalloc_scratch(&scratch);
     if (e != cudaSuccess) return cuda_status(e);
-    g_last_launches = launches;
-    return DIFFATTN_OK;
+    return run_decode(a, scratch, stream);
 }
 
 const char *diffattn_status_str(diffattn_status s)

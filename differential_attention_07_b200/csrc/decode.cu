@@ -21,10 +21,19 @@
 //                then D = acc1/l1 - lambda acc2/l2, RMS norm, gain, bf16.
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
 namespace da {
+
+// Partial-state storage for diffattn_decode_noalloc, for callers that cannot
+// hand the library a workspace.  It lives in the module's static device
+// memory, so every GPU that loads this library holds it until the process
+// exits, and every no-allocation call on a device shares it.
+static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchBytes / sizeof(float)];
+
 namespace {
 
 constexpr int DHDV = 128;
@@ -283,6 +292,28 @@ __global__ void __launch_bounds__(DHDV) decode_combine_kernel(const DecodeParams
 }
 
 }  // namespace
+
+cudaError_t decode_noalloc_scratch(float **ptr)
+{
+    // Host code cannot use g_decode_scratch's name as a device address; ask
+    // the runtime for the address on the current device, once per device.
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static float *addr[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_decode_scratch);
+        if (e != cudaSuccess) return e;
+        addr[dev] = static_cast<float *>(p);
+    }
+    *ptr = addr[dev];
+    return cudaSuccess;
+}
 
 cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream, int *launches,
                           const ProfileEvents &ev)

@@ -6,6 +6,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "diffattn.h"
+
 namespace da {
 
 // Record a library-side failure text for diffattn_last_error() (thread-local).
@@ -73,5 +75,12 @@ constexpr int kDecodeMaxChunk = 2048;
 
 cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream, int *launches,
                           const ProfileEvents &ev);
+
+// Size of the static device array behind diffattn_decode_noalloc.
+constexpr size_t kNoAllocScratchBytes = DIFFATTN_DECODE_NOALLOC_SCRATCH_BYTES;
+
+// Device address of that array on the current device (looked up with
+// cudaGetSymbolAddress on the first call per device, then cached).
+cudaError_t decode_noalloc_scratch(float **ptr);
 
 }  // namespace da

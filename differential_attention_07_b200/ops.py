@@ -37,7 +37,7 @@ EXPORTED = [
     "diffattn_fwd", "diffattn_grouped_fwd", "diffattn_fwd_workspace_size", "diffattn_fwd_validate",
     "diffattn_decode", "diffattn_decode_workspace_size", "diffattn_decode_num_splits",
     "diffattn_decode_validate", "diffattn_status_str", "diffattn_last_launch_count",
-    "diffattn_set_profile_events", "diffattn_last_error",
+    "diffattn_set_profile_events", "diffattn_last_error", "diffattn_decode_noalloc",
 ]
 
 _i64 = ctypes.c_int64
@@ -84,7 +84,7 @@ class DiffAttnError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
         msg = f"{where}: {STATUS.get(status, status)}"
-        if status == 5 and _LIB is not None:
+        if status in (4, 5) and _LIB is not None:
             detail = _LIB.diffattn_last_error()
             if detail:
                 msg += f" ({detail.decode(errors='replace')})"
@@ -113,6 +113,8 @@ def lib():
         L.diffattn_fwd_validate.restype = ctypes.c_int
         L.diffattn_decode.argtypes = [da, _p, ctypes.c_size_t, _p]
         L.diffattn_decode.restype = ctypes.c_int
+        L.diffattn_decode_noalloc.argtypes = [da, _p]
+        L.diffattn_decode_noalloc.restype = ctypes.c_int
         L.diffattn_decode_workspace_size.argtypes = [_i64, _i64, _i64, ctypes.c_int32]
         L.diffattn_decode_workspace_size.restype = ctypes.c_size_t
         L.diffattn_decode_num_splits.argtypes = [_i64, _i64, _i64, ctypes.c_int32]
@@ -303,4 +305,18 @@ def diffattn_decode(q1, q2, k1, k2, v, lam, gain=None, *, kv_len=None, num_split
     st = Lb.diffattn_decode(ctypes.byref(a), _ptr(workspace), workspace.numel(), _stream_ptr(stream))
     if st != 0:
         raise DiffAttnError(st, "diffattn_decode")
+    return out
+
+
+def diffattn_decode_noalloc(q1, q2, k1, k2, v, lam, gain=None, *, out, kv_len=None, num_splits=0,
+                            scale=0.125, eps=1e-5, apply_norm=True, stream=None, dev_status=None):
+    """Single-query decode that allocates nothing: the caller passes the
+    output buffer, and the per-split partial states use the library's fixed
+    static scratch (see diffattn_decode_noalloc in include/diffattn.h).  For
+    callers that cannot allocate device memory or hand over a workspace."""
+    a = _decode_args(q1, q2, k1, k2, v, lam, gain, out, kv_len=kv_len, num_splits=num_splits,
+                     scale=scale, eps=eps, apply_norm=apply_norm, dev_status=dev_status)
+    st = lib().diffattn_decode_noalloc(ctypes.byref(a), _stream_ptr(stream))
+    if st != 0:
+        raise DiffAttnError(st, "diffattn_decode_noalloc")
     return out

@@ -134,6 +134,27 @@ typedef struct diffattn_decode_args {
 diffattn_status diffattn_decode(const diffattn_decode_args *args, void *workspace,
                                 size_t ws_bytes, void *stream);
 
+/* Decode without a workspace.  The pages have no counterpart to this entry
+ * point: it exists for callers that cannot allocate device memory or pass
+ * a workspace -- for instance code inside a serving engine whose allocator
+ * already owns all of the GPU's memory (a KV-cache pool), code on a
+ * latency-critical path that must not call cudaMalloc (which can
+ * synchronise the device), or a plugin that has no allocator handle to take
+ * a workspace from.  It computes exactly what diffattn_decode computes, with
+ * the per-split partial states kept in a fixed static device array of
+ * DIFFATTN_DECODE_NOALLOC_SCRATCH_BYTES that the library carries (every GPU
+ * that loads the library holds it until the process exits).
+ *  - Sizes whose partials (diffattn_decode_workspace_size) exceed that array
+ *    return DIFFATTN_ERR_WORKSPACE; diffattn_last_error() says by how much.
+ *  - The first call on a device looks up the array's device address; make
+ *    that first call before any stream capture.
+ *  - Every call on a device shares the one array and leaves its partials
+ *    there; nothing in it has to start at zero.  Calls that overlap on the
+ *    GPU (other streams, other host threads) race on it: serialise them.
+ *  - Nothing is allocated or freed, by the library or on its behalf.        */
+#define DIFFATTN_DECODE_NOALLOC_SCRATCH_BYTES (8u << 20)
+diffattn_status diffattn_decode_noalloc(const diffattn_decode_args *args, void *stream);
+
 /* Workspace bytes diffattn_decode needs for these sizes (num_splits 0 = the
  * count diffattn_decode picks).                                              */
 size_t diffattn_decode_workspace_size(int64_t B, int64_t H, int64_t L, int32_t num_splits);
