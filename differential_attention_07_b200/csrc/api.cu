@@ -89,7 +89,8 @@ diffattn_status validate_fwd(const diffattn_fwd_args *a, int grouped)
     if (!grouped && (HN != a->H || HV != a->H)) return DIFFATTN_ERR_INVALID_ARG;
     if (a->H % HN != 0 || a->H % HV != 0) return DIFFATTN_ERR_INVALID_ARG;
     if (a->d != 64 || a->dv != 128) return DIFFATTN_ERR_UNSUPPORTED;
-    if (a->flags & ~(DIFFATTN_FLAG_CAUSAL | DIFFATTN_FLAG_APPLY_NORM)) return DIFFATTN_ERR_INVALID_ARG;
+    if (a->flags & ~(DIFFATTN_FLAG_CAUSAL | DIFFATTN_FLAG_APPLY_NORM | DIFFATTN_FLAG_TEST_WITHHOLD_LOAD))
+        return DIFFATTN_ERR_INVALID_ARG;
     if (!(a->scale > 0.0f) || !std::isfinite(a->scale)) return DIFFATTN_ERR_INVALID_ARG;
     if (!(a->eps >= 0.0f) || !std::isfinite(a->eps)) return DIFFATTN_ERR_INVALID_ARG;
     // Index arithmetic inside the kernels is 32-bit for counts.
@@ -220,6 +221,7 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     p.eps = a->eps;
     p.causal = (a->flags & DIFFATTN_FLAG_CAUSAL) ? 1 : 0;
     p.apply_norm = (a->flags & DIFFATTN_FLAG_APPLY_NORM) ? 1 : 0;
+    p.withhold_load = (a->flags & DIFFATTN_FLAG_TEST_WITHHOLD_LOAD) ? 1 : 0;
     p.lambda = a->lambda;
     p.gain = a->gain;
     p.out = a->out;

@@ -27,6 +27,7 @@ struct PrefillParams {
     float scale_log2;     // softmax scale * log2(e)
     float eps;
     int causal, apply_norm;
+    int withhold_load;    // test hook: skip the first K/V load of the CTA's first tile
     const float *lambda;
     const float *gain;    // [H, 128] or nullptr
     void *out;            // bf16

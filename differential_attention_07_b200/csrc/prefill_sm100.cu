@@ -404,6 +404,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     break;
                 const uint32_t st = sbase + OFF_STAGE0 + s * STAGE_BYTES;
                 const int k0 = j * BN;
+                if (p.withhold_load && g == 0) continue;  // test hook: this stage never fills
                 if (elect_one()) {
                     // Warm L2 with the K/V tiles of a later step of this tile
                     // (the stage ring alone cannot hide an HBM miss).
@@ -431,7 +432,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         bool drained = true;
         if (tiles > 0) drained = mbar_wait_drain(bar(B_QFULL), (tiles - 1) & 1, lim);
         for (int k = (g > STAGES ? g - STAGES : 0); k < g; ++k)
-            drained &= mbar_wait_drain(bar_full(k % STAGES), (k / STAGES) & 1, lim);
+            if (!(p.withhold_load && k == 0))  // the withheld load was never issued
+                drained &= mbar_wait_drain(bar_full(k % STAGES), (k / STAGES) & 1, lim);
         if (!__all_sync(0xffffffffu, drained) && lane == 0) *abort_flag = 1;
       } else if (warp == 1 || warp == 2) {
         // ------------------------------------------------------------ MMA issuers

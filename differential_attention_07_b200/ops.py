@@ -22,6 +22,7 @@ LIB_PATH = _build.LIB
 
 DIFFATTN_FLAG_CAUSAL = 1
 DIFFATTN_FLAG_APPLY_NORM = 2
+DIFFATTN_FLAG_TEST_WITHHOLD_LOAD = 0x80000000
 
 STATUS = {
     0: "DIFFATTN_OK",
@@ -165,7 +166,7 @@ def _stream_ptr(stream):
 
 
 def _fwd_args(q1, q2, k1, k2, v, lam, gain, out, *, scale, eps, causal, apply_norm,
-              timeout_ms, dev_status):
+              timeout_ms, dev_status, test_withhold_load=False):
     for n, t in (("q1", q1), ("q2", q2), ("k1", k1), ("k2", k2), ("v", v), ("out", out)):
         _check_bf16(n, t, 4)
     B, N, H, d = q1.shape
@@ -174,6 +175,8 @@ def _fwd_args(q1, q2, k1, k2, v, lam, gain, out, *, scale, eps, causal, apply_no
     a.d, a.dv = d, v.shape[3]
     a.scale, a.eps = float(scale), float(eps)
     a.flags = (DIFFATTN_FLAG_CAUSAL if causal else 0) | (DIFFATTN_FLAG_APPLY_NORM if apply_norm else 0)
+    if test_withhold_load:
+        a.flags |= DIFFATTN_FLAG_TEST_WITHHOLD_LOAD
     a.timeout_ms = int(timeout_ms)
     for n, t in (("q1", q1), ("q2", q2), ("k1", k1), ("k2", k2), ("v", v), ("out", out)):
         setattr(a, n, t.data_ptr())
@@ -200,13 +203,14 @@ def _check_shapes_fwd(q1, q2, k1, k2, v):
 
 
 def _run_fwd(entry, q1, q2, k1, k2, v, lam, gain, *, scale, eps, causal, apply_norm, out,
-             workspace, stream, timeout_ms, dev_status):
+             workspace, stream, timeout_ms, dev_status, test_withhold_load=False):
     _check_shapes_fwd(q1, q2, k1, k2, v)
     B, N, H, _ = q1.shape
     if out is None:
         out = torch.empty(B, N, H, v.shape[3], dtype=torch.bfloat16, device=q1.device)
     a = _fwd_args(q1, q2, k1, k2, v, lam, gain, out, scale=scale, eps=eps, causal=causal,
-                  apply_norm=apply_norm, timeout_ms=timeout_ms, dev_status=dev_status)
+                  apply_norm=apply_norm, timeout_ms=timeout_ms, dev_status=dev_status,
+                  test_withhold_load=test_withhold_load)
     L = lib()
     need = L.diffattn_fwd_workspace_size(ctypes.byref(a))
     if workspace is None:
@@ -219,13 +223,16 @@ def _run_fwd(entry, q1, q2, k1, k2, v, lam, gain, *, scale, eps, causal, apply_n
 
 def diffattn_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,
                  apply_norm=True, out=None, workspace=None, stream=None, timeout_ms=0,
-                 dev_status=None):
+                 dev_status=None, test_withhold_load=False):
     """Differential-attention prefill.  q1,q2,k1,k2 [B,N,H,64], v [B,N,H,128]
     bf16 CUDA tensors (token-major, last dim contiguous); lam [H] fp32; gain
-    [H,128] fp32 or None.  Returns out [B,N,H,128] bf16."""
+    [H,128] fp32 or None.  Returns out [B,N,H,128] bf16.  test_withhold_load
+    sets the library's failure-path test hook (the call then reports a
+    timeout in dev_status)."""
     return _run_fwd("diffattn_fwd", q1, q2, k1, k2, v, lam, gain, scale=scale, eps=eps,
                     causal=causal, apply_norm=apply_norm, out=out, workspace=workspace,
-                    stream=stream, timeout_ms=timeout_ms, dev_status=dev_status)
+                    stream=stream, timeout_ms=timeout_ms, dev_status=dev_status,
+                    test_withhold_load=test_withhold_load)
 
 
 def diffattn_grouped_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,

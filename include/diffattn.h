@@ -57,6 +57,12 @@ typedef enum diffattn_status {
 
 #define DIFFATTN_FLAG_CAUSAL 1u      /* key j visible to query i iff j <= i */
 #define DIFFATTN_FLAG_APPLY_NORM 2u  /* apply the RMS norm + gain; else write D */
+/* Test hook for the failure path: the prefill kernel withholds the K/V load
+ * of the first key step of the first tile each CTA takes, so its bounded
+ * waits run out (after timeout_ms) and the call reports
+ * DIFFATTN_ERR_TIMEOUT in dev_status without writing the output.  Nothing
+ * faults or hangs; the device stays usable.  Not for production use.       */
+#define DIFFATTN_FLAG_TEST_WITHHOLD_LOAD 0x80000000u
 
 /* Prefill arguments.  Layout of each tensor: element (b, n, head, c) sits at
  * ptr + b*stride[0] + n*stride[1] + head*stride[2] + c.
