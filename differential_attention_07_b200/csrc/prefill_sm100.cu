@@ -186,9 +186,11 @@ __device__ __forceinline__ float2 exp2_soft2(float2 x)
 }
 
 // Which pairs of scores (index mod 8) take the software exp2; the rest use
-// MUFU ex2.  3 of 8 balances MUFU time against issue slots for two softmax
-// warps per SM sub-partition.
-constexpr uint32_t SOFT_EXP_MASK = 0xA4u;  // pairs 2, 5, 7 of every 8
+// MUFU ex2.  Measured on B200 (motif-4K / 16K prefill, TFLOP/s): 4 of 8
+// 790 / 931, 3 of 8 810 / 893, 2 of 8 860 / 909, 1 of 8 861 / 959, none
+// 843 / 996: with the pipeline overlapped, issue slots matter more than
+// MUFU time, so only one pair in eight goes to the FMA pipe.
+constexpr uint32_t SOFT_EXP_MASK = 0x20u;  // pair 5 of every 8
 
 // Softmax of one map for one 64-key step, for the query row this thread owns.
 // Reads S (fp32) from TMEM, updates the running max / sum, rescales the O row
