@@ -116,63 +116,88 @@ def aggregate_throughput(units_per_rank, elapsed_s_local, device, world):
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons sampled (NVML, every ~2 ms, from a
+    background thread) while the timed region runs."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
+    def __init__(self, device):
+        self.device = device
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
+        self._thread = None
+        self._handle = None
+
+    def _open(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            pr = torch.cuda.get_device_properties(self.device)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            self._handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            self._handle = pynvml.nvmlDeviceGetHandleByIndex(self.device.index or 0)
+        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM)
+        return pynvml
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            nv = self._open()
+        except Exception:
+            return self
+        self._stop = threading.Event()
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(self._handle, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._handle)
+                    self.samples.append((mhz, rs))
+                except Exception:
+                    pass
+                self._stop.wait(0.002)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
         return self
 
     def __exit__(self, *a):
-        self.out = ""
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                self.out, _ = self.proc.communicate()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
 
     def summary(self):
-        rows = [r.split(",") for r in (getattr(self, "out", "") or "").strip().splitlines()]
-        rows = [[c.strip() for c in r] for r in rows if len(r) >= 9]
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = sorted(float(r[1]) for r in rows if r[1].replace(".", "").isdigit())
-        mx = max((float(r[2]) for r in rows if r[2].replace(".", "").isdigit()), default=None)
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
-        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx,
-                "reasons": reasons, "samples": len(rows)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        mhz = sorted(m for m, _ in self.samples)
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        reasons = sorted(n for b, n in self.REASONS.items() if bits & b)
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
 
 
 # ------------------------------------------------------------------ timing helpers
-def time_loop(fn, steps, warmup, device, stream=None):
+def time_loop(fn, steps, warmup, device, stream=None, clocks=None):
     """Device time (s) of `steps` calls of fn after `warmup` calls; barrier and
-    synchronize on both sides; events on the launching stream."""
+    synchronize on both sides; events on the launching stream.  `clocks` (a
+    ClockSampler) samples the SM clock during the timed region only."""
+    import contextlib
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize(device)
     barrier(device)
     s = stream or torch.cuda.current_stream(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s)
-    for _ in range(steps):
-        fn()
-    e1.record(s)
-    torch.cuda.synchronize(device)
+    with (clocks if clocks is not None else contextlib.nullcontext()):
+        e0.record(s)
+        for _ in range(steps):
+            fn()
+        e1.record(s)
+        torch.cuda.synchronize(device)
     barrier(device)
     return e0.elapsed_time(e1) / 1e3
 
@@ -234,13 +259,13 @@ def to_dev(x, device):
     return {k: v.to(device, non_blocking=True) for k, v in x.items()}
 
 
-def run_prefill_workload(w, steps, warmup, device, ops, rank=0):
+def run_prefill_workload(w, steps, warmup, device, ops, rank=0, clocks=None):
     x = inputs.workload_inputs(inputs.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}))
     d = to_dev(x, device)
     grouped = w.kind == "grouped"
     f = ops.diffattn_grouped_fwd if grouped else ops.diffattn_fwd
     out = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=device)
-    ws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H, w.H_V), dtype=torch.uint8, device=device)
+    ws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H, w.H_V, w.H_N), dtype=torch.uint8, device=device)
     status = torch.zeros(1, dtype=torch.int32, device=device)
 
     def call():
@@ -249,7 +274,7 @@ def run_prefill_workload(w, steps, warmup, device, ops, rank=0):
 
     call()
     launches = ops.last_launch_count()
-    t = time_loop(call, steps, warmup, device)
+    t = time_loop(call, steps, warmup, device, clocks=clocks)
     tk = kernel_time(call, max(3, min(steps, 20)), ops)
     torch.cuda.synchronize(device)
     if status.item() != 0:
@@ -282,7 +307,7 @@ def e2e_prefill(w, steps, warmup, device, ops, x):
     dev = {k: torch.empty_like(v, device=device) for k, v in x.items()}
     out = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=device)
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    ws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H, w.H_V), dtype=torch.uint8, device=device)
+    ws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H, w.H_V, w.H_N), dtype=torch.uint8, device=device)
     f = ops.diffattn_grouped_fwd if w.kind == "grouped" else ops.diffattn_fwd
 
     def step():
@@ -311,8 +336,8 @@ def gpu_arm(args):
     w = inputs.WORKLOADS[args.workload]
     units = prefill_flops(w)
 
-    with ClockSampler(local) as clk:
-        r = run_prefill_workload(w, args.steps, args.warmup, device, ops, rank)
+    clk = ClockSampler(device)
+    r = run_prefill_workload(w, args.steps, args.warmup, device, ops, rank, clocks=clk)
     value, t_max = aggregate_throughput(units * args.steps, r["step_s"] * args.steps, device, world)
     value /= 1e12
     e2e_s, h2d, d2h = e2e_prefill(w, max(3, args.steps // 4), 2, device, ops, r["x"])

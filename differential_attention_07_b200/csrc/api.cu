@@ -73,6 +73,16 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int64_t 
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Grouped heads that run as (signal, noise) and (signal, signal) pairs: each
+// group of g = H / H_N signal heads shares one V head, with g odd and >= 3.
+bool grouped_pairs(const diffattn_fwd_args *a)
+{
+    const int64_t HN = a->H_N ? a->H_N : a->H, HV = a->H_V ? a->H_V : a->H;
+    if (HN <= 0 || a->H % HN != 0 || HV != HN) return false;
+    const int64_t g = a->H / HN;
+    return g >= 3 && g % 2 == 1;
+}
+
 // Bytes of the fp16 V copy at the start of the prefill workspace.
 size_t v16_bytes(const diffattn_fwd_args *a)
 {
@@ -213,10 +223,6 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     p.H_N = (int)HN;
     p.H_V = (int)HV;
     p.num_qt = (int)((a->N + 127) / 128);
-    int G = (2 * 148) / p.num_qt;
-    if (G < 1) G = 1;
-    if (G > p.B * p.H) G = p.B * p.H;
-    p.heads_per_group = G;
     p.scale_log2 = a->scale * 1.4426950408889634f;
     p.eps = a->eps;
     p.causal = (a->flags & DIFFATTN_FLAG_CAUSAL) ? 1 : 0;
@@ -230,8 +236,39 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     p.out_sh = a->out_stride[2];
     p.dev_status = a->dev_status;
     p.timeout_ns = (uint64_t)(a->timeout_ms ? a->timeout_ms : kDefaultTimeoutMs) * 1000000ull;
-    p.tile_counter = tile_counter;
-    e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, p, s, &launches, g_events);
+    // Grouped heads whose group shares one V head and holds an odd number g
+    // >= 3 of signal heads run as two launches that compute each map once:
+    // (last signal head, noise head) pairs that export the normalised noise
+    // output, then pairs of the remaining signal heads that import it.  Any
+    // other layout runs one launch, one signal head (and its noise map) per
+    // work unit.
+    const int64_t g = a->H / HN;
+    auto set_units = [&](int units) {
+        p.units = units;
+        int G = (2 * 148) / p.num_qt;  // (b, unit) pairs sharing K/V in L2 at a time
+        if (G < 1) G = 1;
+        if (G > p.B * units) G = p.B * units;
+        p.heads_per_group = G;
+    };
+    if (g_events.start) cudaEventRecord(g_events.start, s);
+    if (grouped_pairs(a)) {
+        p.noise_out = reinterpret_cast<float *>(static_cast<char *>(ws) + v16_bytes(a) + 256);
+        p.mode = 1;
+        set_units((int)HN);
+        p.tile_counter = tile_counter;
+        e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, p, s, &launches);
+        if (e != cudaSuccess) return cuda_status(e);
+        p.mode = 2;
+        set_units((int)(HN * ((g - 1) / 2)));
+        p.tile_counter = tile_counter + 1;
+        e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, p, s, &launches);
+    } else {
+        p.mode = 0;
+        set_units((int)a->H);
+        p.tile_counter = tile_counter;
+        e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, p, s, &launches);
+    }
+    if (g_events.stop) cudaEventRecord(g_events.stop, s);
     if (e != cudaSuccess) return cuda_status(e);
     g_last_launches = launches;
     return DIFFATTN_OK;
@@ -299,8 +336,15 @@ diffattn_status diffattn_fwd_validate(const diffattn_fwd_args *args, int grouped
 
 size_t diffattn_fwd_workspace_size(const diffattn_fwd_args *a)
 {
-    if (!a || a->B <= 0 || a->N <= 0) return 0;
-    return v16_bytes(a) + 256;  // fp16 V copy, then the work-item counter
+    if (!a || a->B <= 0 || a->N <= 0 || a->H <= 0) return 0;
+    // fp16 V copy, the work-item counters, and for paired grouped heads the
+    // normalised noise outputs [B, N, H_N, 128] fp32
+    size_t n = v16_bytes(a) + 256;
+    if (grouped_pairs(a)) {
+        const int64_t HN = a->H_N ? a->H_N : a->H;
+        n += align256((size_t)a->B * a->N * HN * 128 * sizeof(float));
+    }
+    return n;
 }
 
 diffattn_status diffattn_fwd(const diffattn_fwd_args *args, void *workspace, size_t ws_bytes,

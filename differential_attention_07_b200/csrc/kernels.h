@@ -28,6 +28,9 @@ struct PrefillParams {
     float eps;
     int causal, apply_norm;
     int withhold_load;    // test hook: skip the first K/V load of the CTA's first tile
+    int mode;             // 0: one signal head per unit; 1, 2: grouped pairs (see prefill_sm100.cu)
+    int units;            // work units per batch entry for this launch
+    float *noise_out;     // modes 1, 2: normalised noise outputs [B, N, H_N, 128] fp32
     const float *lambda;
     const float *gain;    // [H, 128] or nullptr
     void *out;            // bf16
@@ -46,10 +49,10 @@ constexpr unsigned kPrefillKeyRows = 64;
 // {64, rows, 1, 1} boxes (kPrefillQRows for Q, kPrefillKeyRows for K and V).
 cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const CUtensorMap &k1,
                            const CUtensorMap &k2, const CUtensorMap &v16, const PrefillParams &p,
-                           cudaStream_t stream, int *launches, const ProfileEvents &ev);
+                           cudaStream_t stream, int *launches);
 
 // bf16 V [B, N, H_V, 128] (strided) -> contiguous fp16 copy in `dst`; also
-// zeroes the prefill kernel's work-item counter.
+// zeroes the two work-item counters of the prefill launches that follow.
 cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, void *dst, int B,
                             int N, int H_V, int32_t *dev_status, int *tile_counter,
                             cudaStream_t stream, int *launches);

@@ -121,15 +121,42 @@ static_assert(OFF_STAGE0 % 1024 == 0 && STAGE_BYTES % 1024 == 0 && K_BYTES % 102
               "SW128 atoms need 1 KB alignment");
 
 struct Work {
-    int b, h, qt;
+    int b, u, qt;  // batch, unit (see heads_of), query tile
 };
+
+// The heads one work item computes.  Map 1 is always signal head a (Q1/K1);
+// map 2 is noise head b (Q2/K2) or, for a pair of signal heads, signal head
+// b (Q1/K1).  Modes (PrefillParams::mode):
+//   0  unit = signal head: map 2 is its noise head h / (H / H_N), V head
+//      h / (H / H_V); the tile's output is head a.
+//   1  unit = noise head n of a group whose g = H / H_N signal heads share
+//      V head n: map 1 is the group's last signal head; the output is that
+//      head, and the normalised noise output is exported for mode 2.
+//   2  unit = (noise head n, pair p): maps 1 and 2 are signal heads
+//      n g + 2p and n g + 2p + 1; each finishes against the exported noise
+//      output of its group.
+struct Heads {
+    int a, b, vh, n;
+    bool b_noise;
+};
+__device__ __forceinline__ Heads heads_of(int u, const PrefillParams &p)
+{
+    if (p.mode == 0) {
+        const int n = u / (p.H / p.H_N);
+        return Heads{u, n, u / (p.H / p.H_V), n, true};
+    }
+    const int g = p.H / p.H_N;
+    if (p.mode == 1) return Heads{u * g + g - 1, u, u, u, true};
+    const int pairs = (g - 1) / 2, n = u / pairs, pp = u % pairs;
+    return Heads{n * g + 2 * pp, n * g + 2 * pp + 1, n, n, false};
+}
 
 // Map the linear CTA index to (b, h, query tile).  (b, h) pairs are taken in
 // groups of heads_per_group so that the CTAs running at the same time share
 // K/V tiles in L2; inside a group the longest (latest) query tiles go first.
 __device__ __forceinline__ Work work_of(int idx, const PrefillParams &p)
 {
-    const int BH = p.B * p.H, G = p.heads_per_group, nq = p.num_qt;
+    const int BH = p.B * p.units, G = p.heads_per_group, nq = p.num_qt;
     const int full = BH / G, per_group = G * nq;
     int bh, qt;
     if (idx < full * per_group) {
@@ -141,7 +168,7 @@ __device__ __forceinline__ Work work_of(int idx, const PrefillParams &p)
         qt = nq - 1 - r / tail;
         bh = full * G + r % tail;
     }
-    return Work{bh / p.H, bh % p.H, qt};
+    return Work{bh / p.units, bh % p.units, qt};
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
@@ -285,7 +312,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (threadIdx.x == 0) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
         return;
     }
-    const int total = p.B * p.H * p.num_qt;
+    const int total = p.B * p.units * p.num_qt;
     int *sItem = reinterpret_cast<int *>(smem + OFF_ITEM);
     const int n_steps_all = (p.N + BN - 1) / BN;
     auto steps_of = [&](const Work &w) {
@@ -388,15 +415,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             item = __shfl_sync(0xffffffffu, item, 0);
             if (item >= total) break;
             const Work w = work_of(item, p);
-            const int nh = w.h / (p.H / p.H_N), vh = w.h / (p.H / p.H_V);
+            const Heads hd = heads_of(w.u, p);
+            const CUtensorMap *mq2 = hd.b_noise ? &tm_q2 : &tm_q1;
+            const CUtensorMap *mk2 = hd.b_noise ? &tm_k2 : &tm_k1;
             const int nkv = steps_of(w);
             // The previous tile's score MMAs must be done with Q.
             if (tiles > 0 && !(ok = mbar_wait_warp(bar(B_QFREE), (tiles - 1) & 1, abort_flag, lim)))
                 break;
             if (elect_one()) {
                 mbar_arrive_expect_tx(bar(B_QFULL), 2 * Q_BYTES);
-                tma_load_4d(sbase + OFF_Q1, &tm_q1, bar(B_QFULL), 0, w.qt * BM, w.h, w.b, stream);
-                tma_load_4d(sbase + OFF_Q2, &tm_q2, bar(B_QFULL), 0, w.qt * BM, nh, w.b, stream);
+                tma_load_4d(sbase + OFF_Q1, &tm_q1, bar(B_QFULL), 0, w.qt * BM, hd.a, w.b, stream);
+                tma_load_4d(sbase + OFF_Q2, mq2, bar(B_QFULL), 0, w.qt * BM, hd.b, w.b, stream);
             }
             __syncwarp();
             for (int j = 0; j < nkv; ++j, ++g) {
@@ -412,16 +441,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     // (the stage ring alone cannot hide an HBM miss).
                     if (j + L2_PREFETCH_STEPS < nkv) {
                         const int kp = k0 + L2_PREFETCH_STEPS * BN;
-                        tma_prefetch_l2_4d(&tm_k1, 0, kp, w.h, w.b);
-                        tma_prefetch_l2_4d(&tm_k2, 0, kp, nh, w.b);
-                        tma_prefetch_l2_4d(&tm_v, 0, kp, vh, w.b);
-                        tma_prefetch_l2_4d(&tm_v, 64, kp, vh, w.b);
+                        tma_prefetch_l2_4d(&tm_k1, 0, kp, hd.a, w.b);
+                        tma_prefetch_l2_4d(mk2, 0, kp, hd.b, w.b);
+                        tma_prefetch_l2_4d(&tm_v, 0, kp, hd.vh, w.b);
+                        tma_prefetch_l2_4d(&tm_v, 64, kp, hd.vh, w.b);
                     }
                     mbar_arrive_expect_tx(bar_full(s), STAGE_BYTES);
-                    tma_load_4d(st, &tm_k1, bar_full(s), 0, k0, w.h, w.b, keep);
-                    tma_load_4d(st + K_BYTES, &tm_k2, bar_full(s), 0, k0, nh, w.b, keep);
-                    tma_load_4d(st + 2 * K_BYTES, &tm_v, bar_full(s), 0, k0, vh, w.b, keep);
-                    tma_load_4d(st + 2 * K_BYTES + VHALF_BYTES, &tm_v, bar_full(s), 64, k0, vh, w.b, keep);
+                    tma_load_4d(st, &tm_k1, bar_full(s), 0, k0, hd.a, w.b, keep);
+                    tma_load_4d(st + K_BYTES, mk2, bar_full(s), 0, k0, hd.b, w.b, keep);
+                    tma_load_4d(st + 2 * K_BYTES, &tm_v, bar_full(s), 0, k0, hd.vh, w.b, keep);
+                    tma_load_4d(st + 2 * K_BYTES + VHALF_BYTES, &tm_v, bar_full(s), 64, k0, hd.vh, w.b, keep);
                 }
                 __syncwarp();
             }
@@ -538,11 +567,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const Work w = work_of(item, p);
             const int nkv = steps_of(w);
             const int qrow = w.qt * BM + r;
-            // The epilogue's lambda and gain: load / prefetch them now so the
-            // global-memory latency hides behind the softmax loop.
-            const float lam = ld_early_f32(p.lambda + w.h);
-            const float *gain = p.gain ? p.gain + (size_t)w.h * HDV + 64 * t : nullptr;
-            if (gain && lane < 2) prefetch_l1(gain + 32 * lane);
+            const Heads hd = heads_of(w.u, p);
+            // Output head of this warpgroup: both finish head a together in
+            // modes 0 and 1 (64 columns each); in mode 2 each finishes its own.
+            const bool own = p.mode == 2;
+            const int head = (own && t) ? hd.b : hd.a;
+            // The epilogue's lambda, gain (and in mode 2 the group's noise
+            // output row): load / prefetch them now so the global-memory
+            // latency hides behind the softmax loop.
+            const float lam = ld_early_f32(p.lambda + head);
+            const float *gain = p.gain ? p.gain + (size_t)head * HDV + (own ? 0 : 64 * t) : nullptr;
+            if (gain && lane < (own ? 4 : 2)) prefetch_l1(gain + 32 * lane);
+            const float *an_row =
+                own ? p.noise_out + (((size_t)w.b * p.N + min(qrow, p.N - 1)) * p.H_N + hd.n) * HDV
+                    : nullptr;
+            if (own) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) prefetch_l1(an_row + 32 * i);
+            }
             float m_run = -INFINITY, l_run = 0.0f;
             for (int j = 0; j < nkv; ++j) {
                 const int gg = g + j, buf = gg & 1;
@@ -558,6 +600,72 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (!ok) break;
             g += nkv;
+            if (own) {
+                // ------------------------------------------------ epilogue, mode 2
+                // This warpgroup's head alone: D = O / l - lambda A_N with A_N
+                // the group's normalised noise output (written by mode 1),
+                // then the RMS norm over the 128 columns of the row.
+                if (!(ok = mbar_wait_warp(bar(B_O), tiles & 1, abort_flag, lim))) break;
+                tc_fence_after();
+                const float inv = 1.0f / l_run;
+                // Pass 1: sum of squares of D over the row, 64 columns at a time.
+                float ss = 0.0f;
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t o[2][32];
+                    tmem_ld32(tO + 64 * hh, o[0]);
+                    tmem_ld32(tO + 64 * hh + 32, o[1]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i4 = 0; i4 < 16; ++i4) {
+                        const float4 a4 = __ldg(reinterpret_cast<const float4 *>(an_row) + 16 * hh + i4);
+                        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float dd = fmaf(-lam, av[e], __uint_as_float(o[i4 >> 3][4 * (i4 & 7) + e]) * inv);
+                            ss = fmaf(dd, dd, ss);
+                        }
+                    }
+                }
+                const float rn = p.apply_norm ? rsqrtf(ss * (1.0f / HDV) + p.eps) : 1.0f;
+                uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) +
+                                2 * ((int64_t)w.b * p.out_sb + (int64_t)qrow * p.out_sn +
+                                     (int64_t)head * p.out_sh);
+                // Pass 2: D again, normalised, gain, bf16, stored; O is released
+                // after its last read.
+#pragma unroll 1
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t o[2][32];
+                    tmem_ld32(tO + 64 * hh, o[0]);
+                    tmem_ld32(tO + 64 * hh + 32, o[1]);
+                    tmem_wait_ld();
+                    if (hh == 1) {
+                        tc_fence_before();
+                        mbar_arrive(bar(B_OFREE));
+                    }
+                    uint32_t y[32];
+#pragma unroll
+                    for (int i4 = 0; i4 < 16; ++i4) {
+                        const float4 a4 = __ldg(reinterpret_cast<const float4 *>(an_row) + 16 * hh + i4);
+                        const float4 g4 = gain ? __ldg(reinterpret_cast<const float4 *>(gain) + 16 * hh + i4)
+                                               : make_float4(1.f, 1.f, 1.f, 1.f);
+                        const uint32_t *oc = &o[i4 >> 3][4 * (i4 & 7)];
+                        const float d0 = fmaf(-lam, a4.x, __uint_as_float(oc[0]) * inv);
+                        const float d1 = fmaf(-lam, a4.y, __uint_as_float(oc[1]) * inv);
+                        const float d2 = fmaf(-lam, a4.z, __uint_as_float(oc[2]) * inv);
+                        const float d3 = fmaf(-lam, a4.w, __uint_as_float(oc[3]) * inv);
+                        y[2 * i4] = pack_bf162(d0 * rn * g4.x, d1 * rn * g4.y);
+                        y[2 * i4 + 1] = pack_bf162(d2 * rn * g4.z, d3 * rn * g4.w);
+                    }
+                    if (qrow < p.N) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + 128 * hh);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            dst[i] = make_uint4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+                    }
+                }
+                continue;
+            }
             // ---------------------------------------------------- epilogue
             // Both warpgroups finish the tile: warpgroup t writes the output
             // columns [64 t, 64 t + 64) of every row.  D = (O1 - r O2) / l1
@@ -583,6 +691,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar(B_OFREE));
+            if (p.mode == 1 && qrow < p.N) {
+                // Export this half of the normalised noise output O2 / l2 for
+                // the group's other signal heads (mode 2).
+                float4 *an = reinterpret_cast<float4 *>(
+                    p.noise_out + (((size_t)w.b * p.N + qrow) * p.H_N + hd.n) * HDV + c0);
+                const float inv2 = 1.0f / l2;
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4)
+                        an[8 * c + i4] = make_float4(__uint_as_float(ob[c][4 * i4]) * inv2,
+                                                     __uint_as_float(ob[c][4 * i4 + 1]) * inv2,
+                                                     __uint_as_float(ob[c][4 * i4 + 2]) * inv2,
+                                                     __uint_as_float(ob[c][4 * i4 + 3]) * inv2);
+            }
             float d[64];
             float ss = 0.0f;
 #pragma unroll
@@ -609,7 +732,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 p.apply_norm ? rsqrtf((sSS[r] + sSS[BM + r]) * (1.0f / HDV) + p.eps) : 1.0f;
             uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) +
                             2 * ((int64_t)w.b * p.out_sb + (int64_t)qrow * p.out_sn +
-                                 (int64_t)w.h * p.out_sh + c0);
+                                 (int64_t)hd.a * p.out_sh + c0);
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t y[16];
@@ -641,9 +764,9 @@ __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb,
                                 int64_t sh, __half *__restrict__ dst, int B, int N, int H_V,
                                 int32_t *dev_status, int *tile_counter)
 {
-    // The prefill kernel that follows on the stream hands out its work items
-    // from this counter.
-    if (blockIdx.x == 0 && threadIdx.x == 0) *tile_counter = 0;
+    // The prefill launches that follow on the stream hand out their work
+    // items from these two counters (one per launch).
+    if (blockIdx.x == 0 && threadIdx.x < 2) tile_counter[threadIdx.x] = 0;
     // One thread per 8 consecutive V elements (16 bytes in, 16 bytes out).
     const int64_t total = (int64_t)B * N * H_V * (HDV / 8);
     bool overflow = false;
@@ -673,7 +796,7 @@ __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb,
 
 cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const CUtensorMap &k1,
                            const CUtensorMap &k2, const CUtensorMap &v16, const PrefillParams &p,
-                           cudaStream_t stream, int *launches, const ProfileEvents &ev)
+                           cudaStream_t stream, int *launches)
 {
     static bool attr_set = false;
     if (!attr_set) {
@@ -700,13 +823,11 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
         if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
     }
-    const int total = p.B * p.H * p.num_qt;
+    const int total = p.B * p.units * p.num_qt;
     if (total == 0) return cudaSuccess;
     const int grid = total < num_sms ? total : num_sms;  // persistent: one CTA per SM
-    if (ev.start) cudaEventRecord(ev.start, stream);
     prefill_kernel<<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, p);
     ++*launches;
-    if (ev.stop) cudaEventRecord(ev.stop, stream);
     return cudaGetLastError();
 }
 

@@ -245,9 +245,10 @@ def diffattn_grouped_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=
                     stream=stream, timeout_ms=timeout_ms, dev_status=dev_status)
 
 
-def fwd_workspace_size(B, N, H, H_V=None):
+def fwd_workspace_size(B, N, H, H_V=None, H_N=None):
+    """Workspace bytes of a prefill call with these sizes."""
     a = FwdArgs()
-    a.B, a.N, a.H, a.H_V, a.d, a.dv = B, N, H, H_V or H, 64, 128
+    a.B, a.N, a.H, a.H_N, a.H_V, a.d, a.dv = B, N, H, H_N or H, H_V or H, 64, 128
     return int(lib().diffattn_fwd_workspace_size(ctypes.byref(a)))
 
 

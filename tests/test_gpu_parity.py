@@ -171,10 +171,17 @@ def test_row0_closed_form_on_gpu(cuda_ok):
     assert np.abs(y - ref).max() <= MAX_ABS
 
 
-@pytest.mark.parametrize("H,H_N,H_V", [(6, 2, 2), (6, 2, 6), (4, 1, 2), (3, 3, 1)])
-def test_grouped_small(cuda_ok, H, H_N, H_V):
-    x = inputs.prefill_inputs(2, 333, H, H_N, H_V, seed=47 + H_N + H_V, gain_std=0.1)
-    y = _run_prefill(x, grouped=True)
+@pytest.mark.parametrize("H,H_N,H_V,N", [(6, 2, 2, 333), (6, 2, 6, 333), (4, 1, 2, 333),
+                                         (3, 3, 1, 333), (10, 2, 2, 333), (15, 5, 5, 200),
+                                         (9, 3, 3, 700), (12, 2, 2, 260)])
+def test_grouped_small(cuda_ok, H, H_N, H_V, N):
+    """Groups of g = 3 or 5 signal heads sharing one V head run as (signal,
+    noise) and (signal, signal) pairs over two launches; other layouts (V per
+    signal head, even g, g = 1) one signal head per work unit."""
+    x = inputs.prefill_inputs(2, N, H, H_N, H_V, seed=47 + H + H_N + H_V, gain_std=0.1)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    y = _run_prefill(x, grouped=True, status=st)
+    assert st.item() == 0
     _assert_parity(y, _oracle_prefill(x))
 
 
