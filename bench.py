@@ -63,6 +63,24 @@ def decode_bytes(w):
     return w.B * w.H * w.N * (64 + 64 + 128) * 2
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one
+# prefill_kernel launch on the 4 x 4096 x 16-head workload, from one ncu
+# capture, keyed by a hash of the kernel sources it was taken on.  A kernel
+# whose sources no longer hash to this value reports null traffic.
+PREFILL_TRAFFIC = {"source_sha256_16": "926545ca555da600", "bytes": 203_687_936 + 45_298_944}
+
+
+def prefill_traffic():
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("prefill_sm100.cu", "sm100_ptx.cuh"):
+        with open(os.path.join(ROOT, "differential_attention_07_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != PREFILL_TRAFFIC["source_sha256_16"]:
+        return None
+    return PREFILL_TRAFFIC["bytes"]
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -367,7 +385,8 @@ def gpu_arm(args):
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(achieved / peaks["bf16_tflops"], 4),
                      "peak_source": peaks["source"] + " bf16 burst (MEASURED_PEAKS.json)",
-                     "kernel": "prefill_kernel", "traffic": None},
+                     "kernel": "prefill_kernel", "traffic": prefill_traffic(),
+                     "traffic_unit": "bytes per launch (ncu)"},
         "gpu_launches": r["launches"] * args.steps,
         "clocks": clk.summary(),
     }

@@ -78,3 +78,10 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     monkeypatch.setenv("WORLD_SIZE", "2")
     bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"])
     assert capsys.readouterr().out == ""
+
+
+def test_traffic_figure_is_dropped_when_the_kernel_source_changes(monkeypatch):
+    t = bench.prefill_traffic()
+    assert t is None or t > 0
+    monkeypatch.setitem(bench.PREFILL_TRAFFIC, "source_sha256_16", "0" * 16)
+    assert bench.prefill_traffic() is None
