@@ -321,12 +321,20 @@ cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream, int *launc
     const int BH = p.B * p.H;
     if (BH == 0) return cudaSuccess;
     const size_t smem = (size_t)(2 * p.chunk + 16 * 2 * DHDV) * sizeof(float);
-    static size_t smem_set = 0;
-    if (smem > 48 * 1024 && smem > smem_set) {
-        cudaError_t e = cudaFuncSetAttribute(decode_split_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024) {
+        // The opt-in shared-memory size is a per-device attribute of the
+        // kernel: remember the largest size set on each device.
+        constexpr int kMaxDevices = 64;
+        static size_t smem_set[kMaxDevices] = {};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return e;
-        smem_set = smem;
+        if (dev < 0 || dev >= kMaxDevices || smem > smem_set[dev]) {
+            e = cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem);
+            if (e != cudaSuccess) return e;
+            if (dev >= 0 && dev < kMaxDevices) smem_set[dev] = smem;
+        }
     }
     if (ev.start) cudaEventRecord(ev.start, stream);
     decode_split_kernel<<<BH * p.splits, SPLIT_THREADS, smem, stream>>>(p);

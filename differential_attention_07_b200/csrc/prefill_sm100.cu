@@ -7,18 +7,23 @@
 // after it (same page, figure 1: GroupNorm after the subtraction, read as a
 // per-head RMS norm with gain).
 //
-// One CTA per (b, h, query tile), 384 threads (three warpgroups), one CTA per SM:
-//   warp 0        TMA producer: Q1/Q2 once, then K1/K2/V per 64-key step
-//                 into a 6-stage ring (32 KB per stage).
+// A persistent kernel: one CTA per SM (384 threads, three warpgroups) takes
+// work items -- (b, unit, 128-row query tile) -- from a global counter until
+// none are left.
+//   warp 0        TMA producer: takes the next item, publishes it to the
+//                 other roles, loads Q1/Q2 once per item, then K1/K2/V per
+//                 64-key step into a 6-stage ring (32 KB per stage).
 //   warps 1, 2    MMA issuers, one per map: S_t = Q_t K_t^T (bf16, fp32
 //                 accumulate in TMEM), then O_t += P_t V with P read from TMEM
 //                 and V (fp16) from the shared-memory tile both maps use.
-//   warps 4-7     softmax of map 1 (one thread per query row) and the
-//                 epilogue: D = (O1 - r O2)/l1 with r = lambda l1/l2, RMS
-//                 norm, gain, bf16.
+//   warps 4-7     softmax of map 1 (one thread per query row).
 //   warps 8-11    softmax of map 2.  A warp reaches TMEM lanes 32 (warp % 4)
-//                 onwards, so each warpgroup covers all 128 rows.  Registers
-//                 are split 56 / 224 / 224 between the warpgroups (setmaxnreg).
+//                 onwards, so each warpgroup covers all 128 rows.  Both
+//                 softmax warpgroups then run the epilogue, 64 output columns
+//                 each: D = (O1 - r O2)/l1 with r = lambda l1/l2, RMS norm
+//                 (sum of squares exchanged through shared memory), gain, bf16.
+//                 Registers are split 56 / 224 / 224 between the warpgroups
+//                 (setmaxnreg).
 // TMEM (512 columns): O1 [0,128) O2 [128,256), and two 64-column S buffers
 // per map: S1 [256,320) [320,384), S2 [384,448) [448,512).  P (fp16, two per
 // column) overwrites the first 32 columns of its S buffer.
@@ -798,14 +803,24 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
                            const CUtensorMap &k2, const CUtensorMap &v16, const PrefillParams &p,
                            cudaStream_t stream, int *launches)
 {
-    static bool attr_set = false;
-    if (!attr_set) {
+    // Per device: the kernel attribute and the SM count.
+    constexpr int kMaxDevices = 64;
+    static bool attr_set[kMaxDevices] = {};
+    static int num_sms[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) {
+        set_internal_error("device ordinal beyond the library's table");
+        return cudaErrorInvalidDevice;
+    }
+    if (!attr_set[dev]) {
         // The register split inside the kernel is only valid for a build that
         // launches with exactly REGS_LAUNCH registers per thread: with fewer,
         // the softmax warpgroups' increase could never be granted.  Refuse to
         // launch such a build.
         cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel);
+        e = cudaFuncGetAttributes(&fa, prefill_kernel);
         if (e != cudaSuccess) return e;
         if (fa.numRegs != REGS_LAUNCH || fa.maxThreadsPerBlock < NTHREADS) {
             set_internal_error("prefill_kernel built with an unexpected register count");
@@ -814,18 +829,13 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
         e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
-    static int num_sms = 0;
-    if (num_sms == 0) {
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+        e = cudaDeviceGetAttribute(&num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
+        attr_set[dev] = true;
     }
     const int total = p.B * p.units * p.num_qt;
     if (total == 0) return cudaSuccess;
-    const int grid = total < num_sms ? total : num_sms;  // persistent: one CTA per SM
+    const int grid = total < num_sms[dev] ? total : num_sms[dev];  // persistent: one CTA per SM
     prefill_kernel<<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, p);
     ++*launches;
     return cudaGetLastError();
