@@ -11,6 +11,10 @@ Recipe (the same for every workload):
   ``[B, heads, N, dim]`` order, each rounded to bf16 (round to nearest even);
   then lambda (float32 uniform per signal head); then the RMS gain
   (float32 ``1 + 0.1 * randn`` of shape ``[H, dv]``, or ones).
+* Gated workloads (Motif 3's token-dependent lambda and output gate) draw,
+  from a second generator seeded with seed + 1000, lambda logits (float32
+  ``1.5 * randn``, [B, N, H]) and gate logits (``2 * randn`` rounded to
+  bf16, [B, N, H, 128]); see ``gate_inputs``.
 * The tensors handed out are permuted to the token-major layout
   ``[B, N, heads, dim]`` (``.contiguous()``), which is what the prefill entry
   points read.  Decode tensors stay head-major: q ``[B, H, d]``, K/V
@@ -45,6 +49,8 @@ class Workload:
     gain_std: float = 0.0                    # 0 => gain of ones
     seed: int = 0
     causal: bool = True
+    gated: bool = False            # token-dependent lambda logits and output-gate logits
+    apply_norm: bool = True
 
 
 WORKLOADS = {
@@ -58,6 +64,10 @@ WORKLOADS = {
                         gain_std=0.0, seed=3),
     "decode": Workload("decode", "decode", B=64, N=8192, H=16, H_N=16, H_V=16, lam=(0.2, 0.8),
                        gain_std=0.1, seed=4),
+    # Motif-3-style attention output (Motif 3 summary, section 2.2): grouped
+    # heads, token-dependent lambda, output gate, no norm.
+    "gated": Workload("gated", "grouped", B=2, N=4096, H=24, H_N=8, H_V=8, lam=(0.2, 0.8),
+                      gain_std=0.0, seed=5, gated=True, apply_norm=False),
 }
 
 
@@ -106,13 +116,34 @@ def decode_inputs(B, L, H, d=64, dv=128, *, seed=0, lam=(0.2, 0.8), lam_head0=No
     return dict(q1=q1, q2=q2, k1=k1, k2=k2, v=v, lam=lamv, gain=gain)
 
 
+def gate_inputs(B, N, H, dv=128, *, seed=0, lam_logit_std=1.5, gate_std=2.0):
+    """Token-dependent lambda logits and output-gate logits (random draws).
+
+    A generator seeded with ``seed + 1000``: lambda logits float32 ``randn *
+    lam_logit_std`` of shape [B, N, H] (prefill) or [B, H] (N = None,
+    decode), then gate logits ``randn * gate_std`` rounded to bf16, [B, N, H,
+    dv] or [B, H, dv].  These stand for the outputs of the projections
+    x_t W^lambda and c_t^Q W^G."""
+    g = torch.Generator().manual_seed(seed + 1000)
+    lead = (B, H) if N is None else (B, N, H)
+    lam_logits = lam_logit_std * torch.randn(*lead, generator=g, dtype=torch.float32)
+    gate = (gate_std * torch.randn(*lead, dv, generator=g, dtype=torch.float32)).to(torch.bfloat16)
+    return dict(lam_logits=lam_logits, gate=gate)
+
+
 def workload_inputs(w: Workload):
     """Inputs of a named workload (CPU tensors)."""
     if w.kind == "decode":
-        return decode_inputs(w.B, w.N, w.H, w.d, w.dv, seed=w.seed, lam=w.lam,
-                             lam_head0=w.lam_head0, gain_std=w.gain_std)
-    return prefill_inputs(w.B, w.N, w.H, w.H_N, w.H_V, w.d, w.dv, seed=w.seed, lam=w.lam,
+        x = decode_inputs(w.B, w.N, w.H, w.d, w.dv, seed=w.seed, lam=w.lam,
                           lam_head0=w.lam_head0, gain_std=w.gain_std)
+        if w.gated:
+            x.update(gate_inputs(w.B, None, w.H, w.dv, seed=w.seed))
+        return x
+    x = prefill_inputs(w.B, w.N, w.H, w.H_N, w.H_V, w.d, w.dv, seed=w.seed, lam=w.lam,
+                       lam_head0=w.lam_head0, gain_std=w.gain_std)
+    if w.gated:
+        x.update(gate_inputs(w.B, w.N, w.H, w.dv, seed=w.seed))
+    return x
 
 
 def sample_rows(B, N, H, count, seed=0, tile=128):

@@ -15,12 +15,19 @@ the noise map of signal head h taken from noise head h // g, and Norm the
 per-head RMS normalisation with gain (Motif 2.6B explainer, section
 "Differential attention" and figure 1; Motif 3 summary, section 2.2).
 
+With token-dependent lambda logits and output-gate logits (Motif 3 summary,
+section 2.2) lambda becomes sigma(logit) per (b, i, h), and the output is
+multiplied element-wise by sigma(G) after the norm.
+
 Pins (tests/test_oracle_pins.py): lambda = 0 against torch's scaled-dot-product
 attention plus torch's rms_norm; map 2 against the same library routine; the
 Q2=Q1, K2=K1 reduction; softmax rows summing to one; causal independence;
 SciPy-softmax brute force for N <= 8; the row-0 closed form; exact scale
 invariance; the grouped head map against repeat_interleave; decode against the
-last prefill row; a hand-derived golden example.  Parity unpinned: the choice of
+last prefill row; a hand-derived golden example; for the token-dependent
+lambda and the gate: saturated logits reducing to SDPA, sigma(0) = 1/2,
+the lambda logits' indexing against SDPA, the gate as the element-wise last
+step, decode against the last gated prefill row.  Parity unpinned: the choice of
 RMS normalisation for the pages' "GroupNorm" and the grouped V layout are
 readings of the pages, not facts the pages fix.
 """
@@ -40,12 +47,12 @@ def load(path):
     ip = ctypes.POINTER(ctypes.c_int64)
     i64 = ctypes.c_int64
     lib.diffattn_oracle_prefill.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, i64,
-                                            i64, i64, dp, dp, ctypes.c_double,
+                                            i64, i64, dp, dp, dp, dp, ctypes.c_double,
                                             ctypes.c_double, ctypes.c_int, ctypes.c_int,
                                             ip, i64, dp]
     lib.diffattn_oracle_prefill.restype = ctypes.c_int
     lib.diffattn_oracle_decode.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, i64,
-                                           ip, dp, dp, ctypes.c_double, ctypes.c_double,
+                                           ip, dp, dp, dp, dp, ctypes.c_double, ctypes.c_double,
                                            ctypes.c_int, dp]
     lib.diffattn_oracle_decode.restype = ctypes.c_int
     lib.diffattn_oracle_softmax_row.argtypes = [dp, dp, i64, i64, ctypes.c_double, dp]
@@ -92,27 +99,34 @@ def softmax_row(q, k, scale):
 
 
 def prefill(q1, q2, k1, k2, v, lam, gain=None, *, scale, eps, causal=True, apply_norm=True,
-            rows=None):
+            rows=None, lam_logits=None, gate=None):
     """Prefill oracle.
 
     q1, k1: [B, N, H, d]; q2, k2: [B, N, H_N, d]; v: [B, N, H_V, dv];
-    lam: [H]; gain: [H, dv] or None.  Returns float64 [B, N, H, dv].
-    rows: None (all rows) or an int array [R, 3] of (b, i, h); then only those
-    rows are computed and the rest of the result is NaN.
+    lam: [H] (ignored, may be None, when lam_logits is given); gain: [H, dv]
+    or None; lam_logits: token-dependent lambda logits [B, N, H] or None;
+    gate: output-gate logits [B, N, H, dv] or None.  Returns float64
+    [B, N, H, dv].  rows: None (all rows) or an int array [R, 3] of
+    (b, i, h); then only those rows are computed and the rest is NaN.
     """
     q1, q2, k1, k2, v = map(_f64, (q1, q2, k1, k2, v))
-    lam, gain = _f64(lam), _f64(gain)
+    lam, gain, lam_logits, gate = map(_f64, (lam, gain, lam_logits, gate))
     B, N, H, d = q1.shape
     H_N, H_V, dv = q2.shape[2], v.shape[2], v.shape[3]
     assert k1.shape == q1.shape and k2.shape == q2.shape and v.shape[:2] == (B, N)
-    assert lam.shape == (H,) and (gain is None or gain.shape == (H, dv))
+    assert (gain is None or gain.shape == (H, dv))
+    assert lam_logits is None or lam_logits.shape == (B, N, H)
+    assert gate is None or gate.shape == (B, N, H, dv)
+    if lam_logits is None:
+        assert lam is not None and lam.shape == (H,)
     out = np.full((B, N, H, dv), np.nan, dtype=np.float64)
     rp, nrows = None, 0
     if rows is not None:
         rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1, 3))
         rp, nrows = rows.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), rows.shape[0]
     rc = _lib().diffattn_oracle_prefill(_dp(q1), _dp(q2), _dp(k1), _dp(k2), _dp(v), B, N, H,
-                                        H_N, H_V, d, dv, _dp(lam), _dp(gain), float(scale),
+                                        H_N, H_V, d, dv, _dp(lam), _dp(gain), _dp(lam_logits),
+                                        _dp(gate), float(scale),
                                         float(eps), int(bool(causal)), int(bool(apply_norm)),
                                         rp, nrows, _dp(out))
     if rc != 0:
@@ -120,16 +134,23 @@ def prefill(q1, q2, k1, k2, v, lam, gain=None, *, scale, eps, causal=True, apply
     return out
 
 
-def decode(q1, q2, k1, k2, v, lam, gain=None, *, kv_len=None, scale, eps, apply_norm=True):
+def decode(q1, q2, k1, k2, v, lam, gain=None, *, kv_len=None, scale, eps, apply_norm=True,
+           lam_logits=None, gate=None):
     """Single-query decode oracle.
 
     q1, q2: [B, H, d]; k1, k2: [B, H, L, d]; v: [B, H, L, dv]; kv_len: [B] or
-    None; lam [H]; gain [H, dv] or None.  Returns float64 [B, H, dv].
+    None; lam [H] (or None with lam_logits); gain [H, dv] or None;
+    lam_logits: [B, H] or None; gate: [B, H, dv] or None.  Returns float64
+    [B, H, dv].
     """
     q1, q2, k1, k2, v = map(_f64, (q1, q2, k1, k2, v))
-    lam, gain = _f64(lam), _f64(gain)
+    lam, gain, lam_logits, gate = map(_f64, (lam, gain, lam_logits, gate))
     B, H, L, d = k1.shape
     dv = v.shape[3]
+    assert lam_logits is None or lam_logits.shape == (B, H)
+    assert gate is None or gate.shape == (B, H, dv)
+    if lam_logits is None:
+        assert lam is not None and lam.shape == (H,)
     kl = None
     if kv_len is not None:
         if hasattr(kv_len, "detach"):
@@ -140,7 +161,8 @@ def decode(q1, q2, k1, k2, v, lam, gain=None, *, kv_len=None, scale, eps, apply_
     rc = _lib().diffattn_oracle_decode(
         _dp(q1), _dp(q2), _dp(k1), _dp(k2), _dp(v), B, H, L, d, dv,
         kl.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)) if kl is not None else None,
-        _dp(lam), _dp(gain), float(scale), float(eps), int(bool(apply_norm)), _dp(out))
+        _dp(lam), _dp(gain), _dp(lam_logits), _dp(gate), float(scale), float(eps),
+        int(bool(apply_norm)), _dp(out))
     if rc != 0:
         raise ValueError("oracle decode: invalid arguments")
     return out

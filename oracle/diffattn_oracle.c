@@ -32,6 +32,15 @@
  *      read as one RMS group per head and token over its dv channels:
  *      Y[c] = D[c] / sqrt(mean_c D[c]^2 + eps) * gain[h][c].
  *      With apply_norm == 0 the pre-norm D is returned.
+ *   5. Token-dependent lambda and output gate (Motif 3 summary, section 2.2):
+ *      lambda_t = sigma(x_t W^lambda) per signal head and token, and
+ *      GDLA(x_t) = vec(sigma(G_t) (.) D_t) W^O.  The projections are outside
+ *      this path, so their outputs -- the logits x_t W^lambda [B][N][H] and
+ *      G_t [B][N][H][dv] -- are the inputs; sigma is the logistic function.
+ *      With lambda logits given they replace lambda[h] in step 3.  With gate
+ *      logits given, step 4's result (normalised or not) is multiplied
+ *      element-wise by sigma(G_t), i.e. the gate is the last operation before
+ *      W^O.
  *
  * Every input is float64 (the exact bf16 / fp32 values widened by the caller)
  * and every intermediate is float64.  Built with -ffp-contract=off so that the
@@ -39,9 +48,11 @@
  *
  * Layouts (all contiguous, row-major, element counts not bytes):
  *   prefill: q1,k1 [B][N][H][d]; q2,k2 [B][N][H_N][d]; v [B][N][H_V][dv];
- *            out [B][N][H][dv]; lambda [H]; gain [H][dv] or NULL (= 1).
+ *            out [B][N][H][dv]; lambda [H]; gain [H][dv] or NULL (= 1);
+ *            lambda_logit [B][N][H] or NULL; gate_logit [B][N][H][dv] or NULL.
  *   decode:  q1,q2 [B][H][d]; k1,k2 [B][H][L][d]; v [B][H][L][dv];
- *            kv_len [B] or NULL (= L); out [B][H][dv].
+ *            kv_len [B] or NULL (= L); out [B][H][dv];
+ *            lambda_logit [B][H] or NULL; gate_logit [B][H][dv] or NULL.
  */
 #include <math.h>
 #include <stdint.h>
@@ -72,13 +83,20 @@ static double softmax_weights(const double *q, const double *k, int64_t k_row_st
     return l;
 }
 
-/* One output row: steps 2-4 above.  a1, a2 are scratch of length dv; w1, w2 of
+/* The logistic function sigma(x) = 1 / (1 + e^-x) of step 5.                 */
+static double logistic(double x)
+{
+    return 1.0 / (1.0 + exp(-x));
+}
+
+/* One output row: steps 2-5 above.  a1, a2 are scratch of length dv; w1, w2 of
  * length nkeys.                                                               */
 static void diff_row(const double *q1, const double *k1, int64_t k1_rs,
                      const double *q2, const double *k2, int64_t k2_rs,
                      const double *v, int64_t v_rs,
                      int64_t nkeys, int64_t d, int64_t dv, double scale,
                      double lambda, const double *gain, double eps, int apply_norm,
+                     const double *gate_logit,
                      double *w1, double *w2, double *a1, double *a2, double *out)
 {
     double l1 = softmax_weights(q1, k1, k1_rs, nkeys, d, scale, w1);
@@ -92,11 +110,14 @@ static void diff_row(const double *q1, const double *k1, int64_t k1_rs,
         }
     }
     for (int64_t c = 0; c < dv; ++c) out[c] = a1[c] / l1 - lambda * (a2[c] / l2);
-    if (!apply_norm) return;
-    double ss = 0.0;
-    for (int64_t c = 0; c < dv; ++c) ss += out[c] * out[c];
-    double r = 1.0 / sqrt(ss / (double)dv + eps);
-    for (int64_t c = 0; c < dv; ++c) out[c] = out[c] * r * (gain ? gain[c] : 1.0);
+    if (apply_norm) {
+        double ss = 0.0;
+        for (int64_t c = 0; c < dv; ++c) ss += out[c] * out[c];
+        double r = 1.0 / sqrt(ss / (double)dv + eps);
+        for (int64_t c = 0; c < dv; ++c) out[c] = out[c] * r * (gain ? gain[c] : 1.0);
+    }
+    if (gate_logit)
+        for (int64_t c = 0; c < dv; ++c) out[c] = logistic(gate_logit[c]) * out[c];
 }
 
 /* Number of OpenMP threads the oracle will use (reported beside its timings). */
@@ -126,6 +147,7 @@ int diffattn_oracle_prefill(const double *q1, const double *q2, const double *k1
                             int64_t B, int64_t N, int64_t H, int64_t H_N, int64_t H_V,
                             int64_t d, int64_t dv,
                             const double *lambda, const double *gain,
+                            const double *lambda_logit, const double *gate_logit,
                             double scale, double eps, int causal, int apply_norm,
                             const int64_t *rows, int64_t nrows, double *out)
 {
@@ -154,9 +176,12 @@ int diffattn_oracle_prefill(const double *q1, const double *q2, const double *k1
             const double *k1b = k1 + ((b * N) * H + h) * d;
             const double *k2b = k2 + ((b * N) * H_N + n) * d;
             const double *vb = v + ((b * N) * H_V + hv) * dv;
+            const int64_t row = (b * N + i) * H + h;   /* index of (b, i, h) */
+            const double lam = lambda_logit ? logistic(lambda_logit[row]) : lambda[h];
+            const double *gate = gate_logit ? gate_logit + row * dv : NULL;
             diff_row(q1r, k1b, H * d, q2r, k2b, H_N * d, vb, H_V * dv, nkeys, d, dv, scale,
-                     lambda[h], gain ? gain + h * dv : NULL, eps, apply_norm, w1, w2, a1, a2,
-                     out + ((b * N + i) * H + h) * dv);
+                     lam, gain ? gain + h * dv : NULL, eps, apply_norm, gate, w1, w2, a1, a2,
+                     out + row * dv);
         }
         free(w1); free(w2); free(a1); free(a2);
     }
@@ -169,6 +194,7 @@ int diffattn_oracle_decode(const double *q1, const double *q2, const double *k1,
                            const double *k2, const double *v,
                            int64_t B, int64_t H, int64_t L, int64_t d, int64_t dv,
                            const int64_t *kv_len, const double *lambda, const double *gain,
+                           const double *lambda_logit, const double *gate_logit,
                            double scale, double eps, int apply_norm, double *out)
 {
     if (B < 0 || H <= 0 || L <= 0 || d <= 0 || dv <= 0) return -1;
@@ -184,9 +210,11 @@ int diffattn_oracle_decode(const double *q1, const double *q2, const double *k1,
         for (int64_t r = 0; r < B * H; ++r) {
             const int64_t b = r / H, h = r % H;
             const int64_t nkeys = kv_len ? kv_len[b] : L;
+            const double lam = lambda_logit ? logistic(lambda_logit[r]) : lambda[h];
             diff_row(q1 + r * d, k1 + r * L * d, d, q2 + r * d, k2 + r * L * d, d,
-                     v + r * L * dv, dv, nkeys, d, dv, scale, lambda[h],
-                     gain ? gain + h * dv : NULL, eps, apply_norm, w1, w2, a1, a2, out + r * dv);
+                     v + r * L * dv, dv, nkeys, d, dv, scale, lam,
+                     gain ? gain + h * dv : NULL, eps, apply_norm,
+                     gate_logit ? gate_logit + r * dv : NULL, w1, w2, a1, a2, out + r * dv);
         }
         free(w1); free(w2); free(a1); free(a2);
     }

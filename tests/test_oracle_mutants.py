@@ -30,13 +30,24 @@ MUTANTS = {
                       "const int64_t n = h / g, hv = h % H_V;"),
     "map2_uses_map1_weights": ("a2[c] += w2[j] * vj[c];", "a2[c] += w1[j] * vj[c];"),
     "mean_over_dv_minus_1": ("ss / (double)dv", "ss / (double)(dv - 1)"),
-    "gain_of_head0": ("gain ? gain + h * dv : NULL, eps, apply_norm, w1, w2, a1, a2,\n"
-                      "                     out",
-                      "gain ? gain : NULL, eps, apply_norm, w1, w2, a1, a2,\n"
-                      "                     out"),
+    "gain_of_head0": ("lam, gain ? gain + h * dv : NULL, eps, apply_norm, gate,",
+                      "lam, gain ? gain : NULL, eps, apply_norm, gate,"),
     "decode_drops_last_key": ("const int64_t nkeys = kv_len ? kv_len[b] : L;",
                               "const int64_t nkeys = kv_len ? kv_len[b] - (kv_len[b] > 1) : L;"),
     "map2_divided_by_l1": ("lambda * (a2[c] / l2)", "lambda * (a2[c] / l1)"),
+    "logistic_sign_flipped": ("return 1.0 / (1.0 + exp(-x));", "return 1.0 / (1.0 + exp(x));"),
+    "token_lambda_transposed": ("logistic(lambda_logit[row])",
+                                "logistic(lambda_logit[(b * H + h) * N + i])"),
+    "token_lambda_of_head0": ("logistic(lambda_logit[row])",
+                              "logistic(lambda_logit[row - h])"),
+    "gate_column_zero": ("logistic(gate_logit[c]) * out[c]", "logistic(gate_logit[0]) * out[c]"),
+    "gate_also_before_norm": (
+        "    for (int64_t c = 0; c < dv; ++c) out[c] = a1[c] / l1 - lambda * (a2[c] / l2);\n",
+        "    for (int64_t c = 0; c < dv; ++c) out[c] = a1[c] / l1 - lambda * (a2[c] / l2);\n"
+        "    if (gate_logit) for (int64_t c = 0; c < dv; ++c) out[c] *= logistic(gate_logit[c]);\n"),
+    "decode_gate_row_of_batch": ("gate_logit ? gate_logit + r * dv : NULL",
+                                 "gate_logit ? gate_logit + b * dv : NULL"),
+    "decode_token_lambda_of_head": ("logistic(lambda_logit[r])", "logistic(lambda_logit[h])"),
 }
 
 PIN_TESTS = [f for name, f in sorted(vars(pins).items())

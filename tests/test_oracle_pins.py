@@ -272,3 +272,85 @@ def test_oracle_rejects_bad_arguments():
         hm = lambda t: t.permute(0, 2, 1, 3).contiguous()
         oracle.decode(x["q1"][:, 0], x["q2"][:, 0], hm(x["k1"]), hm(x["k2"]), hm(x["v"]),
                       x["lam"], kv_len=[0], scale=1, eps=0)
+
+
+# ---------------------------------------------------------------------------
+# token-dependent lambda and output gate (Motif 3 summary, section 2.2:
+# lambda_t = sigma(x_t W^lambda); GDLA(x_t) = vec(sigma(G_t) (.) D_t) W^O)
+# ---------------------------------------------------------------------------
+def _gated_small(B=2, N=37, H=4, H_N=2, H_V=2, seed=91):
+    x = _small(B=B, N=N, H=H, H_N=H_N, H_V=H_V, seed=seed)
+    x.update({k: _f64(v) for k, v in inputs.gate_inputs(B, N, H, seed=seed).items()})
+    return x
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_saturated_logits_give_ordinary_attention(causal):
+    """lambda logits -40 (sigma = 4e-18) and gate logits +40 (sigma = 1 - 4e-18):
+    ordinary attention (torch SDPA) followed by the RMS norm with gain."""
+    x = _gated_small()
+    B, N, H = x["lam_logits"].shape
+    y = oracle.prefill(x["q1"], x["q2"], x["k1"], x["k2"], x["v"], None, x["gain"],
+                       scale=0.125, eps=1e-5, causal=causal,
+                       lam_logits=torch.full((B, N, H), -40.0, dtype=torch.float64),
+                       gate=torch.full((B, N, H, 128), 40.0, dtype=torch.float64))
+    a = _sdpa(x["q1"], x["k1"], x["v"].repeat_interleave(2, dim=2), 0.125, causal)
+    ref = torch.stack([F.rms_norm(a[:, :, h], (128,), weight=x["gain"][h], eps=1e-5)
+                       for h in range(H)], dim=2)
+    np.testing.assert_allclose(y, ref.numpy(), atol=1e-12, rtol=0)
+
+
+def test_zero_logits_are_one_half():
+    """sigma(0) = 1/2: zero lambda logits equal a per-head lambda of 1/2, and
+    zero gate logits halve every output element."""
+    x = _gated_small(seed=92)
+    B, N, H = x["lam_logits"].shape
+    a = (x["q1"], x["q2"], x["k1"], x["k2"], x["v"])
+    half = oracle.prefill(*a, torch.full((H,), 0.5, dtype=torch.float64), x["gain"],
+                          scale=0.125, eps=1e-5)
+    y = oracle.prefill(*a, None, x["gain"], scale=0.125, eps=1e-5,
+                       lam_logits=torch.zeros(B, N, H, dtype=torch.float64),
+                       gate=torch.zeros(B, N, H, 128, dtype=torch.float64))
+    np.testing.assert_allclose(y, 0.5 * half, atol=1e-15, rtol=0)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_token_lambda_against_sdpa(causal):
+    """Before the norm, D[b, i, h] = A1 - sigma(z[b, i, h]) A2 with A1, A2 from
+    torch SDPA (grouped: map 2 and V from head h // 2) and sigma = 1/(1+e^-z)
+    from torch.sigmoid: pins the [B, N, H] indexing of the logits."""
+    x = _gated_small(seed=93)
+    H = x["lam_logits"].shape[2]
+    y = oracle.prefill(x["q1"], x["q2"], x["k1"], x["k2"], x["v"], None, scale=0.125,
+                       eps=1e-5, causal=causal, apply_norm=False, lam_logits=x["lam_logits"])
+    rep = lambda t: t.repeat_interleave(H // t.shape[2], dim=2)
+    a1 = _sdpa(x["q1"], x["k1"], rep(x["v"]), 0.125, causal)
+    a2 = _sdpa(rep(x["q2"]), rep(x["k2"]), rep(x["v"]), 0.125, causal)
+    ref = a1 - torch.sigmoid(x["lam_logits"])[..., None] * a2
+    np.testing.assert_allclose(y, ref.numpy(), atol=1e-12, rtol=0)
+
+
+def test_gate_is_elementwise_after_the_norm():
+    """With the norm on, gated / ungated = sigma(G) element by element: the gate
+    is the last step before W^O (a gate before the norm would be partly
+    normalised away) and is indexed [b, i, h, c]."""
+    x = _gated_small(seed=94)
+    a = (x["q1"], x["q2"], x["k1"], x["k2"], x["v"], x["lam"], x["gain"])
+    y0 = oracle.prefill(*a, scale=0.125, eps=1e-5)
+    y = oracle.prefill(*a, scale=0.125, eps=1e-5, gate=x["gate"])
+    np.testing.assert_allclose(y, torch.sigmoid(x["gate"]).numpy() * y0, atol=1e-13, rtol=0)
+
+
+def test_decode_gated_equals_last_prefill_row():
+    """Decode with lambda logits [B, H] and gate logits [B, H, dv] equals the
+    last prefill row with the same logits at that row."""
+    B, L, H = 2, 41, 3
+    x = _small(B=B, N=L, H=H, seed=95)
+    gl = {k: _f64(v) for k, v in inputs.gate_inputs(B, L, H, seed=95).items()}
+    y = oracle.prefill(x["q1"], x["q2"], x["k1"], x["k2"], x["v"], None, x["gain"],
+                       scale=0.125, eps=1e-5, lam_logits=gl["lam_logits"], gate=gl["gate"])
+    hm = lambda t: t.permute(0, 2, 1, 3).contiguous()
+    yd = oracle.decode(x["q1"][:, L - 1], x["q2"][:, L - 1], hm(x["k1"]), hm(x["k2"]),
+                       hm(x["v"]), None, x["gain"], scale=0.125, eps=1e-5,
+                       lam_logits=gl["lam_logits"][:, L - 1], gate=gl["gate"][:, L - 1])
+    np.testing.assert_allclose(yd, y[:, L - 1], atol=1e-13, rtol=0)
