@@ -16,7 +16,9 @@ kernel.  Rank 0 prints one JSON line:
 * cpu_baseline the float64 oracle on a bounded sample of the same workload
                (rank 0, one GPU only);
 * extra        the other workloads at one pass each: long context (1 x 16384),
-               grouped (24 signal / 8 noise heads), decode (batch 64, 8192
+               grouped (24 signal / 8 noise heads), gated (the grouped shape
+               with token-dependent lambda and output gate, no norm: Motif 3
+               summary, section 2.2), decode (batch 64, 8192
                cached keys; GB/s against the measured HBM copy bandwidth).
 
 With more than one GPU (torchrun) every rank runs its own batch of the same
@@ -288,7 +290,8 @@ def run_prefill_workload(w, steps, warmup, device, ops, rank=0, clocks=None):
 
     def call():
         f(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"], scale=w.scale, eps=w.eps,
-          causal=w.causal, out=out, workspace=ws, dev_status=status)
+          causal=w.causal, apply_norm=w.apply_norm, out=out, workspace=ws, dev_status=status,
+          lam_logits=d.get("lam_logits"), gate=d.get("gate"))
 
     call()
     launches = ops.last_launch_count()
@@ -392,7 +395,7 @@ def gpu_arm(args):
     }
     if world == 1 and not args.no_extra:
         extra = {}
-        for name in ("lc16k", "grouped"):
+        for name in ("lc16k", "grouped", "gated"):
             wx = inputs.WORKLOADS[name]
             rx = run_prefill_workload(wx, max(3, args.steps // 5), 2, device, ops)
             fx = prefill_flops(wx)

@@ -110,16 +110,22 @@ diffattn_status validate_fwd(const diffattn_fwd_args *a, int grouped)
     const void *ptrs[6] = {a->q1, a->q2, a->k1, a->k2, a->v, a->out};
     for (const void *p : ptrs)
         if (!p) return DIFFATTN_ERR_INVALID_ARG;
-    if (!a->lambda) return DIFFATTN_ERR_INVALID_ARG;
+    if (!a->lambda && !a->lambda_logits) return DIFFATTN_ERR_INVALID_ARG;
     for (const void *p : ptrs)
         if (!aligned16(p)) return DIFFATTN_ERR_ALIGNMENT;
     if (a->gain && !aligned16(a->gain)) return DIFFATTN_ERR_ALIGNMENT;
-    const int64_t *strides[6] = {a->q1_stride, a->q2_stride, a->k1_stride, a->k2_stride,
-                                 a->v_stride, a->out_stride};
-    for (const int64_t *s : strides)
+    if (a->lambda_logits) {
+        if (reinterpret_cast<uintptr_t>(a->lambda_logits) % 4) return DIFFATTN_ERR_ALIGNMENT;
+        for (int i = 0; i < 3; ++i)
+            if (a->lambda_logits_stride[i] < 0) return DIFFATTN_ERR_INVALID_ARG;
+    }
+    if (a->gate && !aligned16(a->gate)) return DIFFATTN_ERR_ALIGNMENT;
+    const int64_t *strides[7] = {a->q1_stride, a->q2_stride, a->k1_stride, a->k2_stride,
+                                 a->v_stride, a->out_stride, a->gate_stride};
+    for (int t = 0; t < (a->gate ? 7 : 6); ++t)
         for (int i = 0; i < 3; ++i) {
-            if (s[i] < 0) return DIFFATTN_ERR_INVALID_ARG;
-            if (!stride8(s[i])) return DIFFATTN_ERR_ALIGNMENT;
+            if (strides[t][i] < 0) return DIFFATTN_ERR_INVALID_ARG;
+            if (!stride8(strides[t][i])) return DIFFATTN_ERR_ALIGNMENT;
         }
     return DIFFATTN_OK;
 }
@@ -138,9 +144,18 @@ diffattn_status validate_decode(const diffattn_decode_args *a)
     const void *ptrs[6] = {a->q1, a->q2, a->k1, a->k2, a->v, a->out};
     for (const void *p : ptrs)
         if (!p) return DIFFATTN_ERR_INVALID_ARG;
-    if (!a->lambda) return DIFFATTN_ERR_INVALID_ARG;
+    if (!a->lambda && !a->lambda_logits) return DIFFATTN_ERR_INVALID_ARG;
     for (const void *p : ptrs)
         if (!aligned16(p)) return DIFFATTN_ERR_ALIGNMENT;
+    if (a->lambda_logits) {
+        if (reinterpret_cast<uintptr_t>(a->lambda_logits) % 4) return DIFFATTN_ERR_ALIGNMENT;
+        if (a->lambda_logits_stride[0] < 0 || a->lambda_logits_stride[1] < 0)
+            return DIFFATTN_ERR_INVALID_ARG;
+    }
+    if (a->gate) {
+        if (a->gate_stride[0] < 0 || a->gate_stride[1] < 0) return DIFFATTN_ERR_INVALID_ARG;
+        if (!aligned16(a->gate)) return DIFFATTN_ERR_ALIGNMENT;
+    }
     const int64_t s2[4] = {a->q1_stride[0], a->q1_stride[1], a->q2_stride[0], a->q2_stride[1]};
     for (int64_t s : s2) {
         if (s < 0) return DIFFATTN_ERR_INVALID_ARG;
@@ -229,7 +244,15 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     p.apply_norm = (a->flags & DIFFATTN_FLAG_APPLY_NORM) ? 1 : 0;
     p.withhold_load = (a->flags & DIFFATTN_FLAG_TEST_WITHHOLD_LOAD) ? 1 : 0;
     p.lambda = a->lambda;
-    p.gain = a->gain;
+    p.gain = p.apply_norm ? a->gain : nullptr;  // the gain belongs to the norm
+    p.lam_logits = a->lambda_logits;
+    p.ll_sb = a->lambda_logits_stride[0];
+    p.ll_sn = a->lambda_logits_stride[1];
+    p.ll_sh = a->lambda_logits_stride[2];
+    p.gate = a->gate;
+    p.gate_sb = a->gate_stride[0];
+    p.gate_sn = a->gate_stride[1];
+    p.gate_sh = a->gate_stride[2];
     p.out = a->out;
     p.out_sb = a->out_stride[0];
     p.out_sn = a->out_stride[1];
@@ -311,6 +334,12 @@ diffattn_status run_decode(const diffattn_decode_args *a, float *partials, void 
     p.kv_len = a->kv_len;
     p.lambda = a->lambda;
     p.gain = a->gain;
+    p.lam_logits = a->lambda_logits;
+    p.ll_sb = a->lambda_logits_stride[0];
+    p.ll_sh = a->lambda_logits_stride[1];
+    p.gate = a->gate;
+    p.gate_sb = a->gate_stride[0];
+    p.gate_sh = a->gate_stride[1];
     p.partials = partials;
     p.dev_status = a->dev_status;
     int launches = 0;

@@ -18,7 +18,9 @@
 //                the chunk.  Logits are kept in the log2 domain.
 // combine kernel grid = B*H, 128 threads (one per V column): merges the
 //                chunks (m = max m_s, l = sum l_s 2^(m_s - m), same for acc),
-//                then D = acc1/l1 - lambda acc2/l2, RMS norm, gain, bf16.
+//                then D = acc1/l1 - lambda acc2/l2, RMS norm, gain, the optional
+//                output gate sigma(G) (lambda optionally sigma of a per-token
+//                logit; Motif 3 summary, section 2.2), bf16.
 #include <cuda_bf16.h>
 
 #include <mutex>
@@ -276,8 +278,11 @@ __global__ void __launch_bounds__(DHDV) decode_combine_kernel(const DecodeParams
         A2 = fmaf(ps[4 + DHDV + c], e2, A2);
     }
     float d = 0.0f;
+    // lambda of this (b, h): per head, or sigma of its token-dependent logit
+    // (Motif 3 summary, section 2.2).
+    const float lam = p.lam_logits ? logistic_fast(p.lam_logits[b * p.ll_sb + h * p.ll_sh]) : p.lambda[h];
     // D = (A1 - r A2) / L1 with r = lambda L1 / L2 (one rounding in the difference).
-    if (L1 > 0.0f && L2 > 0.0f) d = fmaf(-(p.lambda[h] * L1 / L2), A2, A1) / L1;
+    if (L1 > 0.0f && L2 > 0.0f) d = fmaf(-(lam * L1 / L2), A2, A1) / L1;
     float y = d;
     if (p.apply_norm) {
         const float ss = warp_sum(d * d);
@@ -286,6 +291,10 @@ __global__ void __launch_bounds__(DHDV) decode_combine_kernel(const DecodeParams
         const float tot = scratch[0] + scratch[1] + scratch[2] + scratch[3];
         y = d * rsqrtf(tot * (1.0f / DHDV) + p.eps);
         if (p.gain) y *= p.gain[h * DHDV + c];
+    }
+    if (p.gate) {  // output gate sigma(G) (same section, "Output Gating"), the last step
+        const __nv_bfloat16 *g = static_cast<const __nv_bfloat16 *>(p.gate) + b * p.gate_sb + h * p.gate_sh;
+        y *= logistic_tanh(__bfloat162float(g[c]));
     }
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.out) + b * p.out_sb + h * p.out_sh;
     o[c] = __float2bfloat16_rn(y);

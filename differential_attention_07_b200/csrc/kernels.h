@@ -31,8 +31,12 @@ struct PrefillParams {
     int mode;             // 0: one signal head per unit; 1, 2: grouped pairs (see prefill_sm100.cu)
     int units;            // work units per batch entry for this launch
     float *noise_out;     // modes 1, 2: normalised noise outputs [B, N, H_N, 128] fp32
-    const float *lambda;
+    const float *lambda;  // [H], unused when lam_logits is set
     const float *gain;    // [H, 128] or nullptr
+    const float *lam_logits;  // token-dependent lambda logits [B, N, H] or nullptr
+    int64_t ll_sb, ll_sn, ll_sh;
+    const void *gate;     // bf16 output-gate logits [B, N, H, 128] or nullptr
+    int64_t gate_sb, gate_sn, gate_sh;
     void *out;            // bf16
     int64_t out_sb, out_sn, out_sh;
     int32_t *dev_status;
@@ -69,6 +73,10 @@ struct DecodeParams {
     int64_t out_sb, out_sh;
     const int32_t *kv_len;
     const float *lambda, *gain;
+    const float *lam_logits;  // [B, H] or nullptr
+    int64_t ll_sb, ll_sh;
+    const void *gate;         // bf16 [B, H, 128] or nullptr
+    int64_t gate_sb, gate_sh;
     float *partials;      // [B*H][splits][4 + 2*128] fp32
     int32_t *dev_status;
 };

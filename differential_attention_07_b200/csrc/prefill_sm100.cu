@@ -21,7 +21,9 @@
 //                 onwards, so each warpgroup covers all 128 rows.  Both
 //                 softmax warpgroups then run the epilogue, 64 output columns
 //                 each: D = (O1 - r O2)/l1 with r = lambda l1/l2, RMS norm
-//                 (sum of squares exchanged through shared memory), gain, bf16.
+//                 (sum of squares exchanged through shared memory), gain,
+//                 optional output gate sigma(G) (lambda optionally sigma of a
+//                 per-token logit: Motif 3 summary, section 2.2), bf16.
 //                 Registers are split 56 / 224 / 224 between the warpgroups
 //                 (setmaxnreg).
 // TMEM (512 columns): O1 [0,128) O2 [128,256), and two 64-column S buffers
@@ -577,10 +579,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // modes 0 and 1 (64 columns each); in mode 2 each finishes its own.
             const bool own = p.mode == 2;
             const int head = (own && t) ? hd.b : hd.a;
-            // The epilogue's lambda, gain (and in mode 2 the group's noise
+            // The epilogue's lambda (per head, or the token-dependent logit of
+            // this row), gain, gate logits (and in mode 2 the group's noise
             // output row): load / prefetch them now so the global-memory
             // latency hides behind the softmax loop.
-            const float lam = ld_early_f32(p.lambda + head);
+            const int64_t qrow_c = min(qrow, p.N - 1);
+            const float lam_in = ld_early_f32(
+                p.lam_logits ? p.lam_logits + w.b * p.ll_sb + qrow_c * p.ll_sn + head * p.ll_sh
+                             : p.lambda + head);
+            const __nv_bfloat16 *grow =
+                p.gate ? static_cast<const __nv_bfloat16 *>(p.gate) + w.b * p.gate_sb +
+                             qrow_c * p.gate_sn + (int64_t)head * p.gate_sh + (own ? 0 : 64 * t)
+                       : nullptr;
+            if (grow) {
+                prefetch_l2(grow);
+                prefetch_l2(grow + 63);
+                if (own) {
+                    prefetch_l2(grow + 64);
+                    prefetch_l2(grow + 127);
+                }
+            }
             const float *gain = p.gain ? p.gain + (size_t)head * HDV + (own ? 0 : 64 * t) : nullptr;
             if (gain && lane < (own ? 4 : 2)) prefetch_l1(gain + 32 * lane);
             const float *an_row =
@@ -610,9 +628,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // This warpgroup's head alone: D = O / l - lambda A_N with A_N
                 // the group's normalised noise output (written by mode 1),
                 // then the RMS norm over the 128 columns of the row.
+                if (grow) {  // the row's gate logits (256 B) to L1 while the last P.V runs
+                    prefetch_l1(grow);
+                    prefetch_l1(grow + 64);
+                    prefetch_l1(grow + 127);
+                }
                 if (!(ok = mbar_wait_warp(bar(B_O), tiles & 1, abort_flag, lim))) break;
                 tc_fence_after();
                 const float inv = 1.0f / l_run;
+                const float lam = p.lam_logits ? logistic_fast(lam_in) : lam_in;
                 // Pass 1: sum of squares of D over the row, 64 columns at a time.
                 float ss = 0.0f;
 #pragma unroll 1
@@ -654,13 +678,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         const float4 a4 = __ldg(reinterpret_cast<const float4 *>(an_row) + 16 * hh + i4);
                         const float4 g4 = gain ? __ldg(reinterpret_cast<const float4 *>(gain) + 16 * hh + i4)
                                                : make_float4(1.f, 1.f, 1.f, 1.f);
+                        float4 s4 = make_float4(rn, rn, rn, rn);  // norm x output gate
+                        if (grow) {
+                            const uint2 gq = __ldg(reinterpret_cast<const uint2 *>(grow + 64 * hh) + i4);
+                            s4.x *= logistic_tanh(__uint_as_float(gq.x << 16));
+                            s4.y *= logistic_tanh(__uint_as_float(gq.x & 0xffff0000u));
+                            s4.z *= logistic_tanh(__uint_as_float(gq.y << 16));
+                            s4.w *= logistic_tanh(__uint_as_float(gq.y & 0xffff0000u));
+                        }
                         const uint32_t *oc = &o[i4 >> 3][4 * (i4 & 7)];
                         const float d0 = fmaf(-lam, a4.x, __uint_as_float(oc[0]) * inv);
                         const float d1 = fmaf(-lam, a4.y, __uint_as_float(oc[1]) * inv);
                         const float d2 = fmaf(-lam, a4.z, __uint_as_float(oc[2]) * inv);
                         const float d3 = fmaf(-lam, a4.w, __uint_as_float(oc[3]) * inv);
-                        y[2 * i4] = pack_bf162(d0 * rn * g4.x, d1 * rn * g4.y);
-                        y[2 * i4 + 1] = pack_bf162(d2 * rn * g4.z, d3 * rn * g4.w);
+                        y[2 * i4] = pack_bf162(d0 * s4.x * g4.x, d1 * s4.y * g4.y);
+                        y[2 * i4 + 1] = pack_bf162(d2 * s4.z * g4.z, d3 * s4.w * g4.w);
                     }
                     if (qrow < p.N) {
                         uint4 *dst = reinterpret_cast<uint4 *>(orow + 128 * hh);
@@ -677,12 +709,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // with r = lambda l1 / l2 (one fused multiply-add per element;
             // identical maps with lambda = 1 cancel exactly), then the RMS
             // norm over all 128 columns, whose sum of squares is exchanged.
+            if (grow) {  // bring this half's gate logits (128 B) to L1 while the last P.V runs
+                prefetch_l1(grow);
+                prefetch_l1(grow + 63);
+            }
             sL[t * BM + r] = l_run;
             mbar_arrive(bar(B_LX));
             if (!(ok = mbar_wait_warp(bar(B_LX), tiles & 1, abort_flag, lim))) break;
             if (!(ok = mbar_wait_warp(bar(B_O), tiles & 1, abort_flag, lim))) break;
             tc_fence_after();
             const float l1 = sL[r], l2 = sL[BM + r];
+            const float lam = p.lam_logits ? logistic_fast(lam_in) : lam_in;
             const float inv1 = 1.0f / l1, r2 = lam * l1 / l2;
             const uint32_t c0 = 64 * t;
             // One read of this half of O1 and O2; D stays in registers, and O
@@ -731,6 +768,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 gv[4 * i + 1] = g4.y;
                 gv[4 * i + 2] = g4.z;
                 gv[4 * i + 3] = g4.w;
+            }
+            if (grow) {  // the output gate sigma(G) folds into the gain
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint4 gq = __ldg(reinterpret_cast<const uint4 *>(grow) + i);
+                    const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        gv[8 * i + 2 * k] *= logistic_tanh(__uint_as_float(gw[k] << 16));
+                        gv[8 * i + 2 * k + 1] *= logistic_tanh(__uint_as_float(gw[k] & 0xffff0000u));
+                    }
+                }
             }
             if (!(ok = mbar_wait_warp(bar(B_SSX), tiles & 1, abort_flag, lim))) break;
             const float rn =

@@ -389,6 +389,32 @@ __device__ __forceinline__ void prefetch_l1(const void *p)
     asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
 
+__device__ __forceinline__ void prefetch_l2(const void *p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// The logistic function sigma(z) = 1 / (1 + e^-z) of Motif 3's token-dependent
+// lambda and output gate, as 1 / (1 + 2^(-z log2 e)) with MUFU ex2 and a fast
+// divide.  z is clamped to [-80, 80], where sigma is 0 or 1 to fp32 precision,
+// so the divide never sees an infinite or huge denominator.
+__device__ __forceinline__ float logistic_fast(float z)
+{
+    z = fminf(fmaxf(z, -80.0f), 80.0f);
+    return __fdividef(1.0f, 1.0f + ex2_approx(-1.4426950408889634f * z));
+}
+
+// sigma(z) = (1 + tanh(z / 2)) / 2 with one MUFU tanh.approx (absolute error
+// below 2.5e-4, under the bf16 rounding of an output it scales).  For the
+// output gate, which multiplies the result directly; lambda, whose error the
+// subtraction can amplify, uses logistic_fast.
+__device__ __forceinline__ float logistic_tanh(float z)
+{
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * z));
+    return fmaf(0.5f, t, 0.5f);
+}
+
 // Global fp32 load issued at this point of the program (the value is only
 // consumed much later, so its latency hides behind the work in between).
 __device__ __forceinline__ float ld_early_f32(const float *p)

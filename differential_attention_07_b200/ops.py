@@ -61,6 +61,8 @@ class FwdArgs(ctypes.Structure):
         ("v", _p), ("v_stride", _S3),
         ("out", _p), ("out_stride", _S3),
         ("lambda_", _p), ("gain", _p), ("dev_status", _p),
+        ("lambda_logits", _p), ("lambda_logits_stride", _S3),
+        ("gate", _p), ("gate_stride", _S3),
     ]
 
 
@@ -78,6 +80,8 @@ class DecodeArgs(ctypes.Structure):
         ("v", _p), ("v_stride", _S3),
         ("out", _p), ("out_stride", _S2),
         ("kv_len", _p), ("lambda_", _p), ("gain", _p), ("dev_status", _p),
+        ("lambda_logits", _p), ("lambda_logits_stride", _S2),
+        ("gate", _p), ("gate_stride", _S2),
     ]
 
 
@@ -165,8 +169,31 @@ def _stream_ptr(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _set_lambda_gate(a, lam, lam_logits, gate, lead, dv, S):
+    """Fill lambda (per head), the token-dependent lambda logits and the gate
+    logits.  lead: the leading dims (B, N, H) or (B, H); S: the stride type."""
+    H = lead[-1]
+    if lam_logits is not None:
+        if lam_logits.dtype != torch.float32 or tuple(lam_logits.shape) != tuple(lead):
+            raise ValueError(f"lam_logits must be float32 {list(lead)}")
+        a.lambda_logits = lam_logits.data_ptr()
+        a.lambda_logits_stride = S(*lam_logits.stride())
+    elif lam is None:
+        raise ValueError("lam (per head) or lam_logits (per token) is required")
+    if lam is not None:
+        if lam.dtype != torch.float32 or lam.shape != (H,):
+            raise ValueError("lam must be float32 [H]")
+        a.lambda_ = lam.data_ptr()
+    if gate is not None:
+        _check_bf16("gate", gate, len(lead) + 1)
+        if tuple(gate.shape) != tuple(lead) + (dv,):
+            raise ValueError(f"gate must be bf16 {list(lead) + [dv]}")
+        a.gate = gate.data_ptr()
+        a.gate_stride = S(*gate.stride()[:len(lead)])
+
+
 def _fwd_args(q1, q2, k1, k2, v, lam, gain, out, *, scale, eps, causal, apply_norm,
-              timeout_ms, dev_status, test_withhold_load=False):
+              timeout_ms, dev_status, test_withhold_load=False, lam_logits=None, gate=None):
     for n, t in (("q1", q1), ("q2", q2), ("k1", k1), ("k2", k2), ("v", v), ("out", out)):
         _check_bf16(n, t, 4)
     B, N, H, d = q1.shape
@@ -181,9 +208,7 @@ def _fwd_args(q1, q2, k1, k2, v, lam, gain, out, *, scale, eps, causal, apply_no
     for n, t in (("q1", q1), ("q2", q2), ("k1", k1), ("k2", k2), ("v", v), ("out", out)):
         setattr(a, n, t.data_ptr())
         setattr(a, n + "_stride", _S3(*t.stride()[:3]))
-    if lam.dtype != torch.float32 or lam.shape != (H,):
-        raise ValueError("lam must be float32 [H]")
-    a.lambda_ = lam.data_ptr()
+    _set_lambda_gate(a, lam, lam_logits, gate, (B, N, H), a.dv, _S3)
     if gain is not None:
         if gain.dtype != torch.float32 or tuple(gain.shape) != (H, a.dv) or not gain.is_contiguous():
             raise ValueError("gain must be contiguous float32 [H, dv]")
@@ -203,14 +228,15 @@ def _check_shapes_fwd(q1, q2, k1, k2, v):
 
 
 def _run_fwd(entry, q1, q2, k1, k2, v, lam, gain, *, scale, eps, causal, apply_norm, out,
-             workspace, stream, timeout_ms, dev_status, test_withhold_load=False):
+             workspace, stream, timeout_ms, dev_status, test_withhold_load=False,
+             lam_logits=None, gate=None):
     _check_shapes_fwd(q1, q2, k1, k2, v)
     B, N, H, _ = q1.shape
     if out is None:
         out = torch.empty(B, N, H, v.shape[3], dtype=torch.bfloat16, device=q1.device)
     a = _fwd_args(q1, q2, k1, k2, v, lam, gain, out, scale=scale, eps=eps, causal=causal,
                   apply_norm=apply_norm, timeout_ms=timeout_ms, dev_status=dev_status,
-                  test_withhold_load=test_withhold_load)
+                  test_withhold_load=test_withhold_load, lam_logits=lam_logits, gate=gate)
     L = lib()
     need = L.diffattn_fwd_workspace_size(ctypes.byref(a))
     if workspace is None:
@@ -223,26 +249,30 @@ def _run_fwd(entry, q1, q2, k1, k2, v, lam, gain, *, scale, eps, causal, apply_n
 
 def diffattn_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,
                  apply_norm=True, out=None, workspace=None, stream=None, timeout_ms=0,
-                 dev_status=None, test_withhold_load=False):
+                 dev_status=None, test_withhold_load=False, lam_logits=None, gate=None):
     """Differential-attention prefill.  q1,q2,k1,k2 [B,N,H,64], v [B,N,H,128]
-    bf16 CUDA tensors (token-major, last dim contiguous); lam [H] fp32; gain
-    [H,128] fp32 or None.  Returns out [B,N,H,128] bf16.  test_withhold_load
-    sets the library's failure-path test hook (the call then reports a
-    timeout in dev_status)."""
+    bf16 CUDA tensors (token-major, last dim contiguous); lam [H] fp32 (or
+    None with lam_logits); gain [H,128] fp32 or None; lam_logits: fp32
+    [B,N,H] token-dependent lambda logits or None; gate: bf16 [B,N,H,128]
+    output-gate logits or None.  Returns out [B,N,H,128] bf16.
+    test_withhold_load sets the library's failure-path test hook (the call
+    then reports a timeout in dev_status)."""
     return _run_fwd("diffattn_fwd", q1, q2, k1, k2, v, lam, gain, scale=scale, eps=eps,
                     causal=causal, apply_norm=apply_norm, out=out, workspace=workspace,
                     stream=stream, timeout_ms=timeout_ms, dev_status=dev_status,
-                    test_withhold_load=test_withhold_load)
+                    test_withhold_load=test_withhold_load, lam_logits=lam_logits, gate=gate)
 
 
 def diffattn_grouped_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,
                          apply_norm=True, out=None, workspace=None, stream=None, timeout_ms=0,
-                         dev_status=None):
+                         dev_status=None, lam_logits=None, gate=None):
     """Grouped prefill: q1,k1 [B,N,H,64]; q2,k2 [B,N,H_N,64]; v [B,N,H_V,128];
-    signal head h uses noise head h // (H // H_N) and V head h // (H // H_V)."""
+    signal head h uses noise head h // (H // H_N) and V head h // (H // H_V).
+    lam_logits [B,N,H] and gate [B,N,H,128] as in diffattn_fwd."""
     return _run_fwd("diffattn_grouped_fwd", q1, q2, k1, k2, v, lam, gain, scale=scale, eps=eps,
                     causal=causal, apply_norm=apply_norm, out=out, workspace=workspace,
-                    stream=stream, timeout_ms=timeout_ms, dev_status=dev_status)
+                    stream=stream, timeout_ms=timeout_ms, dev_status=dev_status,
+                    lam_logits=lam_logits, gate=gate)
 
 
 def fwd_workspace_size(B, N, H, H_V=None, H_N=None):
@@ -261,7 +291,7 @@ def decode_num_splits(B, H, L, num_splits=0):
 
 
 def _decode_args(q1, q2, k1, k2, v, lam, gain, out, *, kv_len, num_splits, scale, eps,
-                 apply_norm, dev_status):
+                 apply_norm, dev_status, lam_logits=None, gate=None):
     for n, t, nd in (("q1", q1, 3), ("q2", q2, 3), ("k1", k1, 4), ("k2", k2, 4), ("v", v, 4),
                      ("out", out, 3)):
         _check_bf16(n, t, nd)
@@ -285,9 +315,7 @@ def _decode_args(q1, q2, k1, k2, v, lam, gain, out, *, kv_len, num_splits, scale
         if kv_len.dtype != torch.int32 or kv_len.shape != (B,):
             raise ValueError("kv_len must be int32 [B]")
         a.kv_len = kv_len.data_ptr()
-    if lam.dtype != torch.float32 or lam.shape != (H,):
-        raise ValueError("lam must be float32 [H]")
-    a.lambda_ = lam.data_ptr()
+    _set_lambda_gate(a, lam, lam_logits, gate, (B, H), a.dv, _S2)
     if gain is not None:
         if gain.dtype != torch.float32 or tuple(gain.shape) != (H, a.dv) or not gain.is_contiguous():
             raise ValueError("gain must be contiguous float32 [H, dv]")
@@ -298,14 +326,16 @@ def _decode_args(q1, q2, k1, k2, v, lam, gain, out, *, kv_len, num_splits, scale
 
 def diffattn_decode(q1, q2, k1, k2, v, lam, gain=None, *, kv_len=None, num_splits=0, scale=0.125,
                     eps=1e-5, apply_norm=True, out=None, workspace=None, stream=None,
-                    dev_status=None):
+                    dev_status=None, lam_logits=None, gate=None):
     """Single-query decode.  q1,q2 [B,H,64]; k1,k2 [B,H,L,64]; v [B,H,L,128]
-    bf16 CUDA tensors; kv_len int32 [B] or None.  Returns out [B,H,128] bf16."""
+    bf16 CUDA tensors; kv_len int32 [B] or None; lam_logits fp32 [B,H] and
+    gate bf16 [B,H,128] optional.  Returns out [B,H,128] bf16."""
     B, H, L, _ = k1.shape
     if out is None:
         out = torch.empty(B, H, v.shape[3], dtype=torch.bfloat16, device=q1.device)
     a = _decode_args(q1, q2, k1, k2, v, lam, gain, out, kv_len=kv_len, num_splits=num_splits,
-                     scale=scale, eps=eps, apply_norm=apply_norm, dev_status=dev_status)
+                     scale=scale, eps=eps, apply_norm=apply_norm, dev_status=dev_status,
+                     lam_logits=lam_logits, gate=gate)
     Lb = lib()
     need = Lb.diffattn_decode_workspace_size(B, H, L, int(num_splits))
     if workspace is None:
@@ -317,13 +347,15 @@ def diffattn_decode(q1, q2, k1, k2, v, lam, gain=None, *, kv_len=None, num_split
 
 
 def diffattn_decode_noalloc(q1, q2, k1, k2, v, lam, gain=None, *, out, kv_len=None, num_splits=0,
-                            scale=0.125, eps=1e-5, apply_norm=True, stream=None, dev_status=None):
+                            scale=0.125, eps=1e-5, apply_norm=True, stream=None, dev_status=None,
+                            lam_logits=None, gate=None):
     """Single-query decode that allocates nothing: the caller passes the
     output buffer, and the per-split partial states use the library's fixed
     static scratch (see diffattn_decode_noalloc in include/diffattn.h).  For
     callers that cannot allocate device memory or hand over a workspace."""
     a = _decode_args(q1, q2, k1, k2, v, lam, gain, out, kv_len=kv_len, num_splits=num_splits,
-                     scale=scale, eps=eps, apply_norm=apply_norm, dev_status=dev_status)
+                     scale=scale, eps=eps, apply_norm=apply_norm, dev_status=dev_status,
+                     lam_logits=lam_logits, gate=gate)
     st = lib().diffattn_decode_noalloc(ctypes.byref(a), _stream_ptr(stream))
     if st != 0:
         raise DiffAttnError(st, "diffattn_decode_noalloc")

@@ -15,6 +15,12 @@
  * The grouped variant (Motif 3 summary, section 2.2, eq. "grouped differential
  * output" D_t = H_S,t - lambda_t (.) Repeat_g(H_N,t)) takes map 2 of signal
  * head h from noise head h / (H / H_N) and V from V head h / (H / H_V).
+ * The same section makes lambda token-dependent, lambda_t = sigma(x_t W^lambda),
+ * and gates the output, vec(sigma(G_t) (.) D_t) W^O ("Output Gating"): both
+ * are optional inputs of every entry point (the logits x_t W^lambda and G_t,
+ * produced by projections outside this library; sigma(z) = 1 / (1 + e^-z)).
+ * The gate multiplies the result element-wise as the last step: Y above when
+ * the norm is applied, D when it is not.
  *
  * Conventions for every entry point:
  *  - Element type of Q/K/V/out is bf16.  Only d = 64 (Q/K head dim) and
@@ -69,7 +75,13 @@ typedef enum diffattn_status {
  *   q1, k1: [B, N, H,   64]     q2, k2: [B, N, H_N, 64]
  *   v:      [B, N, H_V, 128]    out:    [B, N, H,   128]
  *   lambda: [H] fp32 device     gain:   [H, 128] fp32 device (16-byte aligned,
- *                                       contiguous), or NULL for 1. */
+ *                                       contiguous), or NULL for 1.
+ *   lambda_logits: [B, N, H] fp32 device, element (b, n, h) at
+ *       ptr + b*s[0] + n*s[1] + h*s[2] (4-byte aligned, any strides), or NULL.
+ *       When set, signal head h of token n uses lambda = sigma(logit) and
+ *       `lambda` may be NULL.
+ *   gate: [B, N, H, 128] bf16 device gate logits, laid out like `out` (16-byte
+ *       aligned base, strides multiples of 8 elements), or NULL for no gate. */
 typedef struct diffattn_fwd_args {
     int64_t B, N, H, H_N, H_V;
     int64_t d, dv;
@@ -85,6 +97,8 @@ typedef struct diffattn_fwd_args {
     const float *lambda;
     const float *gain;
     int32_t *dev_status;
+    const float *lambda_logits; int64_t lambda_logits_stride[3];
+    const void *gate;           int64_t gate_stride[3];
 } diffattn_fwd_args;
 
 /* Causal (or full) prefill, one noise map per signal head: H_N and H_V must be
@@ -115,7 +129,10 @@ diffattn_status diffattn_fwd_validate(const diffattn_fwd_args *args, int grouped
  *   v:      [B, H, L, 128]
  *   out:    [B, H, 128]
  *   kv_len: [B] int32 device, 1 <= kv_len[b] <= L, or NULL for L.
- *   num_splits: KV splits per (b, h); 0 picks one. */
+ *   num_splits: KV splits per (b, h); 0 picks one.
+ *   lambda_logits: [B, H] fp32 device (element (b, h) at ptr + b*s[0] + h*s[1])
+ *       or NULL; when set, lambda = sigma(logit) and `lambda` may be NULL.
+ *   gate: [B, H, 128] bf16 device gate logits laid out like `out`, or NULL. */
 typedef struct diffattn_decode_args {
     int64_t B, H, L;
     int64_t d, dv;
@@ -132,6 +149,8 @@ typedef struct diffattn_decode_args {
     const float *lambda;
     const float *gain;
     int32_t *dev_status;
+    const float *lambda_logits; int64_t lambda_logits_stride[2];
+    const void *gate;           int64_t gate_stride[2];
 } diffattn_decode_args;
 
 /* Split-KV decode: a split kernel writes per-split partial softmax states

@@ -168,6 +168,43 @@ def test_decode_validation_and_workspace(L):
     assert L.diffattn_decode_num_splits(64, 16, 8192, 0) == 4
 
 
+def test_token_lambda_and_gate_validation(L):
+    """Motif 3's token-dependent lambda logits and output gate: the per-head
+    lambda may be NULL only when logits are given; the gate follows the
+    output's alignment rules; the logits need 4-byte alignment."""
+    base = 1 << 20
+    a = _fake_fwd_args()
+    a.lambda_ = None
+    assert _v(L, a) == 1                              # no lambda at all
+    a.lambda_logits = 20 * base
+    a.lambda_logits_stride = ops._S3(300 * 4, 4, 1)
+    assert _v(L, a) == 0                              # logits alone are enough
+    a.lambda_logits = 20 * base + 2
+    assert _v(L, a) == 3                              # not 4-byte aligned
+    a.lambda_logits = 20 * base
+    a.lambda_logits_stride = ops._S3(300 * 4, -4, 1)
+    assert _v(L, a) == 1
+    a = _fake_fwd_args()
+    a.gate, a.gate_stride = 21 * base, ops._S3(300 * 4 * 128, 4 * 128, 128)
+    assert _v(L, a) == 0
+    a.gate = 21 * base + 8
+    assert _v(L, a) == 3                              # base not 16-byte aligned
+    a.gate = 21 * base
+    a.gate_stride = ops._S3(300 * 4 * 128, 4 * 128 + 4, 128)
+    assert _v(L, a) == 3                              # stride not a multiple of 8
+    a.gate_stride = ops._S3(300 * 4 * 128, -512, 128)
+    assert _v(L, a) == 1
+    d = _fake_decode_args()
+    d.lambda_ = None
+    assert L.diffattn_decode_validate(ctypes.byref(d)) == 1
+    d.lambda_logits, d.lambda_logits_stride = 8 * base, ops._S2(2, 1)
+    assert L.diffattn_decode_validate(ctypes.byref(d)) == 0
+    d.gate, d.gate_stride = 9 * base + 2, ops._S2(2 * 128, 128)
+    assert L.diffattn_decode_validate(ctypes.byref(d)) == 3
+    d.gate = 9 * base
+    assert L.diffattn_decode_validate(ctypes.byref(d)) == 0
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(ops, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(ops, "_LIB", None)
