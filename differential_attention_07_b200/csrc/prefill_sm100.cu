@@ -12,7 +12,7 @@
 // none are left.
 //   warp 0        TMA producer: takes the next item, publishes it to the
 //                 other roles, loads Q1/Q2 once per item, then K1/K2/V per
-//                 64-key step into a 6-stage ring (32 KB per stage).
+//                 64-key step into a 4-stage ring (32 KB per stage).
 //   warps 1, 2    MMA issuers, one per map: S_t = Q_t K_t^T (bf16, fp32
 //                 accumulate in TMEM), then O_t += P_t V with P read from TMEM
 //                 and V (fp16) from the shared-memory tile both maps use.
@@ -57,7 +57,7 @@ constexpr int BM = 128;   // query rows per tile (MMA M)
 constexpr int BN = 64;    // keys per step (MMA N of S, K of P.V)
 constexpr int HD = 64;    // Q/K head dim
 constexpr int HDV = 128;  // V head dim (MMA N of P.V)
-constexpr int STAGES = 6;
+constexpr int STAGES = 4;
 constexpr int NTHREADS = 384;
 
 constexpr uint32_t Q_BYTES = BM * HD * 2;           // 16 KB
@@ -77,10 +77,10 @@ enum : int {
     B_FULL = 2,                  // [STAGES] K1/K2/V of a step landed (TMA bytes)
     B_EMPTY = B_FULL + STAGES,   // [STAGES] both maps' P.V of the step done (2 commits)
     B_S = B_EMPTY + STAGES,      // [2 maps][2 buffers] S ready (commit)
-    B_P = B_S + 4,               // [2 maps][2 buffers] P written (128 arrivals)
+    B_P = B_S + 4,               // [2 maps][2 buffers] P written (4 softmax warps)
     B_PV = B_P + 4,              // [2 maps] latest P.V into O done (commit)
     B_O = B_PV + 2,              // all MMAs of the tile done (2 commits)
-    B_OFREE = B_O + 1,           // epilogue finished reading O (256 arrivals)
+    B_OFREE = B_O + 1,           // epilogue finished reading O (8 softmax warps)
     B_LX = B_OFREE + 1,          // row sums exchanged (256 arrivals)
     B_SSX = B_LX + 1,            // partial sums of squares exchanged (256 arrivals)
     B_ITEM = B_SSX + 1,          // [ITEM_SLOTS] work item published (1 arrival)
@@ -265,8 +265,10 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, bool firs
 
     const bool need = tmax > m_run + RESCALE_THRESHOLD;
     const float m_new = need ? tmax : m_run;
-    const float alpha = need ? ex2_approx(m_run - m_new) : 1.0f;  // ex2(-inf) = 0
-    if (!first && __any_sync(0xffffffffu, need)) {
+    float alpha = 1.0f;
+    if (__any_sync(0xffffffffu, need)) {  // rare after a row's first step
+      alpha = need ? ex2_approx(m_run - m_new) : 1.0f;  // ex2(-inf) = 0
+      if (!first) {
         // O holds P.V products up to the previous step; the last one must be
         // finished before the row is rescaled.
         if (!mbar_wait_warp(bar_pv, pv_parity, abort_flag, lim)) return false;
@@ -280,6 +282,7 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, bool firs
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
             tmem_st32(tO + 32 * c, o);
         }
+      }
     }
     l_run *= alpha;
     m_run = m_new;
@@ -346,12 +349,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         for (int i = 0; i < 4; ++i) {
             mbar_init(bar(B_S + i), 1);
-            mbar_init(bar(B_P + i), 128);
+            mbar_init(bar(B_P + i), 4);   // one arrival per softmax warp
         }
         mbar_init(bar(B_PV), 1);
         mbar_init(bar(B_PV + 1), 1);
         mbar_init(bar(B_O), 2);
-        mbar_init(bar(B_OFREE), 256);
+        mbar_init(bar(B_OFREE), 8);   // one arrival per softmax warp
         mbar_init(bar(B_LX), 256);
         mbar_init(bar(B_SSX), 256);
         for (int i = 0; i < ITEM_SLOTS; ++i) {
@@ -618,8 +621,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (!(ok = softmax_step(tS0 + BN * buf, tO, j == 0, limit, p.scale_log2, m_run, l_run,
                                         bar_pv, (gg - 1) & 1, abort_flag, lim)))
                     break;
+                // Every lane's P store has completed (tcgen05.wait::st in the
+                // step); after the warp sync one arrival stands for the warp.
                 tc_fence_before();
-                mbar_arrive(bar_p(t, buf));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_p(t, buf));
             }
             if (!ok) break;
             g += nkv;
@@ -668,9 +674,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tmem_ld32(tO + 64 * hh, o[0]);
                     tmem_ld32(tO + 64 * hh + 32, o[1]);
                     tmem_wait_ld();
-                    if (hh == 1) {
+                    if (hh == 1) {  // O read to registers by every lane: release it, once per warp
                         tc_fence_before();
-                        mbar_arrive(bar(B_OFREE));
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(B_OFREE));
                     }
                     uint32_t y[32];
 #pragma unroll
@@ -732,7 +739,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tmem_ld32(tO2 + c0 + 32, ob[1]);
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(bar(B_OFREE));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_OFREE));  // once per warp, after every lane's read
             if (p.mode == 1 && qrow < p.N) {
                 // Export this half of the normalised noise output O2 / l2 for
                 // the group's other signal heads (mode 2).
