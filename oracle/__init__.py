@@ -48,12 +48,12 @@ def load(path):
     i64 = ctypes.c_int64
     lib.diffattn_oracle_prefill.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, i64,
                                             i64, i64, dp, dp, dp, dp, ctypes.c_double,
-                                            ctypes.c_double, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_double, ctypes.c_int, ctypes.c_int, i64,
                                             ip, i64, dp]
     lib.diffattn_oracle_prefill.restype = ctypes.c_int
     lib.diffattn_oracle_decode.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, i64,
                                            ip, dp, dp, dp, dp, ctypes.c_double, ctypes.c_double,
-                                           ctypes.c_int, dp]
+                                           ctypes.c_int, i64, dp]
     lib.diffattn_oracle_decode.restype = ctypes.c_int
     lib.diffattn_oracle_softmax_row.argtypes = [dp, dp, i64, i64, ctypes.c_double, dp]
     lib.diffattn_oracle_softmax_row.restype = None
@@ -99,13 +99,15 @@ def softmax_row(q, k, scale):
 
 
 def prefill(q1, q2, k1, k2, v, lam, gain=None, *, scale, eps, causal=True, apply_norm=True,
-            rows=None, lam_logits=None, gate=None):
+            rows=None, lam_logits=None, gate=None, window=0):
     """Prefill oracle.
 
     q1, k1: [B, N, H, d]; q2, k2: [B, N, H_N, d]; v: [B, N, H_V, dv];
     lam: [H] (ignored, may be None, when lam_logits is given); gain: [H, dv]
     or None; lam_logits: token-dependent lambda logits [B, N, H] or None;
-    gate: output-gate logits [B, N, H, dv] or None.  Returns float64
+    gate: output-gate logits [B, N, H, dv] or None; window: 0, or a causal
+    sliding window of that many keys (query i sees keys i-W < j <= i).
+    Returns float64
     [B, N, H, dv].  rows: None (all rows) or an int array [R, 3] of
     (b, i, h); then only those rows are computed and the rest is NaN.
     """
@@ -128,19 +130,20 @@ def prefill(q1, q2, k1, k2, v, lam, gain=None, *, scale, eps, causal=True, apply
                                         H_N, H_V, d, dv, _dp(lam), _dp(gain), _dp(lam_logits),
                                         _dp(gate), float(scale),
                                         float(eps), int(bool(causal)), int(bool(apply_norm)),
-                                        rp, nrows, _dp(out))
+                                        int(window), rp, nrows, _dp(out))
     if rc != 0:
         raise ValueError("oracle prefill: invalid arguments")
     return out
 
 
 def decode(q1, q2, k1, k2, v, lam, gain=None, *, kv_len=None, scale, eps, apply_norm=True,
-           lam_logits=None, gate=None):
+           lam_logits=None, gate=None, window=0):
     """Single-query decode oracle.
 
     q1, q2: [B, H, d]; k1, k2: [B, H, L, d]; v: [B, H, L, dv]; kv_len: [B] or
     None; lam [H] (or None with lam_logits); gain [H, dv] or None;
-    lam_logits: [B, H] or None; gate: [B, H, dv] or None.  Returns float64
+    lam_logits: [B, H] or None; gate: [B, H, dv] or None; window: 0 or the
+    number of most recent cached keys the query sees.  Returns float64
     [B, H, dv].
     """
     q1, q2, k1, k2, v = map(_f64, (q1, q2, k1, k2, v))
@@ -162,7 +165,7 @@ def decode(q1, q2, k1, k2, v, lam, gain=None, *, kv_len=None, scale, eps, apply_
         _dp(q1), _dp(q2), _dp(k1), _dp(k2), _dp(v), B, H, L, d, dv,
         kl.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)) if kl is not None else None,
         _dp(lam), _dp(gain), _dp(lam_logits), _dp(gate), float(scale), float(eps),
-        int(bool(apply_norm)), _dp(out))
+        int(bool(apply_norm)), int(window), _dp(out))
     if rc != 0:
         raise ValueError("oracle decode: invalid arguments")
     return out

@@ -12,7 +12,10 @@
  *
  *   1. Key range J.  Causal prefill: keys 0..i (the diagonal is included, so
  *      no row is empty).  Non-causal prefill: keys 0..N-1.  Decode: the query
- *      sits at position kv_len-1 and sees keys 0..kv_len-1.
+ *      sits at position kv_len-1 and sees keys 0..kv_len-1.  A sliding window
+ *      of W > 0 keys (causal only; Motif 3 summary, sections 2.1 and
+ *      "Practical Implications": sliding-window layers with 128-token
+ *      windows) keeps the W most recent of those keys: i-W < j <= i.
  *      (Motif 2.6B is a decoder-only Transformer: edgentiq Motif-2.6B blog;
  *      Motif 3 summary, section 2.1 "full causal-attention layer".)
  *   2. For each map t in {1,2}: z_j = s * <q_t, k_t[j]>, m = max_j z_j,
@@ -148,10 +151,11 @@ int diffattn_oracle_prefill(const double *q1, const double *q2, const double *k1
                             int64_t d, int64_t dv,
                             const double *lambda, const double *gain,
                             const double *lambda_logit, const double *gate_logit,
-                            double scale, double eps, int causal, int apply_norm,
+                            double scale, double eps, int causal, int apply_norm, int64_t window,
                             const int64_t *rows, int64_t nrows, double *out)
 {
     if (B < 0 || N < 0 || H <= 0 || H_N <= 0 || H_V <= 0 || d <= 0 || dv <= 0) return -1;
+    if (window < 0 || (window > 0 && !causal)) return -1;
     if (H % H_N != 0 || H % H_V != 0) return -1;
     const int64_t g = H / H_N;       /* signal heads per noise head */
     const int64_t gv = H / H_V;      /* signal heads per V head */
@@ -171,15 +175,17 @@ int diffattn_oracle_prefill(const double *q1, const double *q2, const double *k1
             if (b < 0 || b >= B || i < 0 || i >= N || h < 0 || h >= H) { bad = 1; continue; }
             const int64_t n = h / g, hv = h / gv;
             const int64_t nkeys = causal ? i + 1 : N;
+            /* first visible key: i - W + 1 under a window of W keys */
+            const int64_t j0 = (window > 0 && i + 1 > window) ? i + 1 - window : 0;
             const double *q1r = q1 + ((b * N + i) * H + h) * d;
             const double *q2r = q2 + ((b * N + i) * H_N + n) * d;
-            const double *k1b = k1 + ((b * N) * H + h) * d;
-            const double *k2b = k2 + ((b * N) * H_N + n) * d;
-            const double *vb = v + ((b * N) * H_V + hv) * dv;
+            const double *k1b = k1 + ((b * N + j0) * H + h) * d;
+            const double *k2b = k2 + ((b * N + j0) * H_N + n) * d;
+            const double *vb = v + ((b * N + j0) * H_V + hv) * dv;
             const int64_t row = (b * N + i) * H + h;   /* index of (b, i, h) */
             const double lam = lambda_logit ? logistic(lambda_logit[row]) : lambda[h];
             const double *gate = gate_logit ? gate_logit + row * dv : NULL;
-            diff_row(q1r, k1b, H * d, q2r, k2b, H_N * d, vb, H_V * dv, nkeys, d, dv, scale,
+            diff_row(q1r, k1b, H * d, q2r, k2b, H_N * d, vb, H_V * dv, nkeys - j0, d, dv, scale,
                      lam, gain ? gain + h * dv : NULL, eps, apply_norm, gate, w1, w2, a1, a2,
                      out + row * dv);
         }
@@ -195,9 +201,9 @@ int diffattn_oracle_decode(const double *q1, const double *q2, const double *k1,
                            int64_t B, int64_t H, int64_t L, int64_t d, int64_t dv,
                            const int64_t *kv_len, const double *lambda, const double *gain,
                            const double *lambda_logit, const double *gate_logit,
-                           double scale, double eps, int apply_norm, double *out)
+                           double scale, double eps, int apply_norm, int64_t window, double *out)
 {
-    if (B < 0 || H <= 0 || L <= 0 || d <= 0 || dv <= 0) return -1;
+    if (B < 0 || H <= 0 || L <= 0 || d <= 0 || dv <= 0 || window < 0) return -1;
     for (int64_t b = 0; b < B; ++b)
         if (kv_len && (kv_len[b] < 1 || kv_len[b] > L)) return -1;
 #pragma omp parallel
@@ -210,9 +216,11 @@ int diffattn_oracle_decode(const double *q1, const double *q2, const double *k1,
         for (int64_t r = 0; r < B * H; ++r) {
             const int64_t b = r / H, h = r % H;
             const int64_t nkeys = kv_len ? kv_len[b] : L;
+            /* under a window of W keys: the W most recent cached keys */
+            const int64_t j0 = (window > 0 && nkeys > window) ? nkeys - window : 0;
             const double lam = lambda_logit ? logistic(lambda_logit[r]) : lambda[h];
-            diff_row(q1 + r * d, k1 + r * L * d, d, q2 + r * d, k2 + r * L * d, d,
-                     v + r * L * dv, dv, nkeys, d, dv, scale, lam,
+            diff_row(q1 + r * d, k1 + (r * L + j0) * d, d, q2 + r * d, k2 + (r * L + j0) * d, d,
+                     v + (r * L + j0) * dv, dv, nkeys - j0, d, dv, scale, lam,
                      gain ? gain + h * dv : NULL, eps, apply_norm,
                      gate_logit ? gate_logit + r * dv : NULL, w1, w2, a1, a2, out + r * dv);
         }

@@ -48,6 +48,8 @@ MUTANTS = {
     "decode_gate_row_of_batch": ("gate_logit ? gate_logit + r * dv : NULL",
                                  "gate_logit ? gate_logit + b * dv : NULL"),
     "decode_token_lambda_of_head": ("logistic(lambda_logit[r])", "logistic(lambda_logit[h])"),
+    "window_one_key_too_many": ("? i + 1 - window : 0;", "? i - window : 0;"),
+    "decode_window_one_key_too_few": ("? nkeys - window : 0;", "? nkeys - window + 1 : 0;"),
 }
 
 PIN_TESTS = [f for name, f in sorted(vars(pins).items())
@@ -55,12 +57,19 @@ PIN_TESTS = [f for name, f in sorted(vars(pins).items())
 
 
 def _run_pin(f):
-    sig = inspect.signature(f)
-    if "causal" in sig.parameters:
-        for c in (True, False):
-            f(causal=c)
-    else:
-        f()
+    """Run a pin over every combination of its pytest parametrize values."""
+    import itertools
+    grids = []
+    for mark in getattr(f, "pytestmark", []):
+        if mark.name == "parametrize":
+            names, values = mark.args[0], mark.args[1]
+            names = [n.strip() for n in names.split(",")] if isinstance(names, str) else list(names)
+            grids.append([dict(zip(names, v if len(names) > 1 else (v,))) for v in values])
+    for combo in itertools.product(*grids) if grids else [()]:
+        kw = {}
+        for part in combo:
+            kw.update(part)
+        f(**kw)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))

@@ -354,3 +354,88 @@ def test_decode_gated_equals_last_prefill_row():
                        hm(x["v"]), None, x["gain"], scale=0.125, eps=1e-5,
                        lam_logits=gl["lam_logits"][:, L - 1], gate=gl["gate"][:, L - 1])
     np.testing.assert_allclose(yd, y[:, L - 1], atol=1e-13, rtol=0)
+
+
+# ---------------------------------------------------------------------------
+# sliding window (Motif 3 summary: sliding-window layers, 128-token windows);
+# read as: query i sees the W most recent keys, i - W < j <= i
+# ---------------------------------------------------------------------------
+def _window_mask(N, W):
+    i = torch.arange(N)[:, None]
+    j = torch.arange(N)[None, :]
+    return (j <= i) & (j > i - W)
+
+
+def test_window_covering_everything_is_plain_causal():
+    x = _small(B=2, N=30, H=2, seed=101)
+    a = (x["q1"], x["q2"], x["k1"], x["k2"], x["v"], x["lam"], x["gain"])
+    ref = oracle.prefill(*a, scale=0.125, eps=1e-5)
+    for W in (30, 31, 1000):
+        np.testing.assert_array_equal(oracle.prefill(*a, scale=0.125, eps=1e-5, window=W), ref)
+
+
+def test_window_of_one_is_the_row_itself():
+    """W = 1: every map attends to its own key only, D = (1 - lambda) V[i] and
+    Y = V[i] / rms(V[i]) * gain (eps = 0)."""
+    x = _small(B=2, N=9, H=3, seed=102)
+    y = oracle.prefill(x["q1"], x["q2"], x["k1"], x["k2"], x["v"], x["lam"], x["gain"],
+                       scale=0.125, eps=0.0, window=1)
+    v = x["v"].numpy()
+    ref = v / np.sqrt((v ** 2).mean(-1, keepdims=True)) * x["gain"].numpy()[None, None]
+    np.testing.assert_allclose(y, ref, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("W", [2, 5, 17])
+def test_window_against_masked_sdpa(W):
+    """lambda = 0 against torch SDPA with the explicit window mask, then the
+    norm; map 2 through D(0) - D(1) against the same masked SDPA."""
+    B, N, H = 2, 40, 2
+    x = _small(B=B, N=N, H=H, seed=103 + W)
+    mask = _window_mask(N, W)
+    sdpa = lambda q, k: F.scaled_dot_product_attention(
+        q.permute(0, 2, 1, 3), k.permute(0, 2, 1, 3), x["v"].permute(0, 2, 1, 3), attn_mask=mask,
+        scale=0.125).permute(0, 2, 1, 3)
+    a = (x["q1"], x["q2"], x["k1"], x["k2"], x["v"])
+    y = oracle.prefill(*a, torch.zeros(H, dtype=torch.float64), x["gain"], scale=0.125, eps=1e-5,
+                       window=W)
+    a1 = sdpa(x["q1"], x["k1"])
+    ref = torch.stack([F.rms_norm(a1[:, :, h], (128,), weight=x["gain"][h], eps=1e-5)
+                       for h in range(H)], dim=2)
+    np.testing.assert_allclose(y, ref.numpy(), atol=1e-12, rtol=0)
+    d0 = oracle.prefill(*a, torch.zeros(H, dtype=torch.float64), scale=0.125, eps=1e-5,
+                        apply_norm=False, window=W)
+    d1 = oracle.prefill(*a, torch.ones(H, dtype=torch.float64), scale=0.125, eps=1e-5,
+                        apply_norm=False, window=W)
+    np.testing.assert_allclose(d0 - d1, sdpa(x["q2"], x["k2"]).numpy(), atol=1e-12, rtol=0)
+
+
+def test_window_edges():
+    """Row i under window W ignores keys up to i - W and depends on key i - W + 1."""
+    N, W, i = 40, 7, 25
+    x = _small(B=1, N=N, H=1, seed=107)
+    a = lambda k1, v: (x["q1"], x["q2"], k1, x["k2"], v, x["lam"], x["gain"])
+    y = oracle.prefill(*a(x["k1"], x["v"]), scale=0.125, eps=1e-5, window=W)
+    k1, v = x["k1"].clone(), x["v"].clone()
+    k1[:, : i - W + 1] += 4.0
+    v[:, : i - W + 1] *= -3.0
+    y2 = oracle.prefill(*a(k1, v), scale=0.125, eps=1e-5, window=W)
+    np.testing.assert_array_equal(y[0, i], y2[0, i])
+    v3 = x["v"].clone()
+    v3[:, i - W + 1] *= -3.0
+    y3 = oracle.prefill(*a(x["k1"], v3), scale=0.125, eps=1e-5, window=W)
+    assert np.abs(y[0, i] - y3[0, i]).max() > 1e-3
+
+
+def test_decode_window_equals_last_prefill_row():
+    B, L, H, W = 3, 50, 2, 11
+    x = _small(B=B, N=L, H=H, seed=109)
+    y = oracle.prefill(x["q1"], x["q2"], x["k1"], x["k2"], x["v"], x["lam"], x["gain"],
+                       scale=0.125, eps=1e-5, window=W)
+    hm = lambda t: t.permute(0, 2, 1, 3).contiguous()
+    kv_len = np.array([L, 5, 23])
+    q1 = torch.stack([x["q1"][b, kv_len[b] - 1] for b in range(B)])
+    q2 = torch.stack([x["q2"][b, kv_len[b] - 1] for b in range(B)])
+    yd = oracle.decode(q1, q2, hm(x["k1"]), hm(x["k2"]), hm(x["v"]), x["lam"], x["gain"],
+                       kv_len=kv_len, scale=0.125, eps=1e-5, window=W)
+    for b in range(B):
+        np.testing.assert_allclose(yd[b], y[b, kv_len[b] - 1], atol=1e-13, rtol=0)
