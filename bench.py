@@ -43,8 +43,19 @@ from differential_attention_07_b200 import inputs  # noqa: E402
 FLOP_PER_PAIR = 768  # 2*64 + 2*64 (two QK^T) + 2*128 + 2*128 (two P.V)
 
 
-def causal_pairs(N):
-    return N * (N + 1) // 2
+def causal_pairs(N, window=0):
+    """Visible (query, key) pairs of one head: key j <= query i, and under a
+    sliding window of W keys also j > i - W."""
+    if window <= 0 or window >= N:
+        return N * (N + 1) // 2
+    return window * (window + 1) // 2 + (N - window) * window
+
+
+def prefill_bytes(w):
+    """Algorithmic HBM bytes of one prefill call: Q1, Q2, K1, K2, V read once
+    and the output written once (bf16)."""
+    per_token = (w.H + w.H_N) * w.d * 2 * 2 + w.H_V * w.dv * 2 + w.H * w.dv * 2
+    return w.B * w.N * per_token
 
 
 def prefill_flops(w):
@@ -54,7 +65,7 @@ def prefill_flops(w):
     grouped form a noise map is computed once per noise head; its P.V product
     is shared by the group when the group shares one V head (H_V == H_N),
     otherwise each signal head multiplies it by its own V."""
-    pairs = causal_pairs(w.N) if w.causal else w.N * w.N
+    pairs = causal_pairs(w.N, w.window) if w.causal else w.N * w.N
     qk_maps = w.H + w.H_N
     pv_maps = w.H + (w.H_N if w.H_V == w.H_N else w.H)
     return (qk_maps * 2 * 64 + pv_maps * 2 * 128) * pairs * w.B
@@ -291,6 +302,7 @@ def run_prefill_workload(w, steps, warmup, device, ops, rank=0, clocks=None):
     def call():
         f(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"], scale=w.scale, eps=w.eps,
           causal=w.causal, apply_norm=w.apply_norm, out=out, workspace=ws, dev_status=status,
+          window=w.window,
           lam_logits=d.get("lam_logits"), gate=d.get("gate"))
 
     call()
@@ -395,7 +407,7 @@ def gpu_arm(args):
     }
     if world == 1 and not args.no_extra:
         extra = {}
-        for name in ("lc16k", "grouped", "gated"):
+        for name in ("lc16k", "grouped", "gated", "swa16k"):
             wx = inputs.WORKLOADS[name]
             rx = run_prefill_workload(wx, max(3, args.steps // 5), 2, device, ops)
             fx = prefill_flops(wx)
@@ -403,6 +415,10 @@ def gpu_arm(args):
                            "kernel_tflops": round(fx / rx["kernel_s"] / 1e12, 2),
                            "frac_of_peak": round(fx / rx["kernel_s"] / 1e12 / peaks["bf16_tflops"], 4),
                            "ms": round(rx["step_s"] * 1e3, 4)}
+            if wx.window:  # few keys per query: the HBM bytes bound it, not the tensor cores
+                gb = prefill_bytes(wx) / rx["step_s"] / 1e9
+                extra[name]["gbs"] = round(gb, 1)
+                extra[name]["hbm_frac"] = round(gb / peaks["hbm_gbs"], 4)
             del rx
         wd = inputs.WORKLOADS["decode"]
         rd = run_decode_workload(wd, max(5, args.steps), 3, device, ops)

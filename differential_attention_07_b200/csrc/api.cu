@@ -103,6 +103,8 @@ diffattn_status validate_fwd(const diffattn_fwd_args *a, int grouped)
         return DIFFATTN_ERR_INVALID_ARG;
     if (!(a->scale > 0.0f) || !std::isfinite(a->scale)) return DIFFATTN_ERR_INVALID_ARG;
     if (!(a->eps >= 0.0f) || !std::isfinite(a->eps)) return DIFFATTN_ERR_INVALID_ARG;
+    if (a->window < 0 || (a->window > 0 && !(a->flags & DIFFATTN_FLAG_CAUSAL)))
+        return DIFFATTN_ERR_INVALID_ARG;
     // Index arithmetic inside the kernels is 32-bit for counts.
     if (a->N > (1 << 24) || a->B > (1 << 16) || a->H > 4096) return DIFFATTN_ERR_UNSUPPORTED;
     if ((a->B * a->H * ((a->N + 127) / 128)) > INT32_MAX) return DIFFATTN_ERR_UNSUPPORTED;
@@ -136,7 +138,7 @@ diffattn_status validate_decode(const diffattn_decode_args *a)
     if (a->B < 0 || a->H <= 0 || a->L <= 0) return DIFFATTN_ERR_INVALID_ARG;
     if (a->d != 64 || a->dv != 128) return DIFFATTN_ERR_UNSUPPORTED;
     if (a->flags & ~(DIFFATTN_FLAG_CAUSAL | DIFFATTN_FLAG_APPLY_NORM)) return DIFFATTN_ERR_INVALID_ARG;
-    if (a->num_splits < 0) return DIFFATTN_ERR_INVALID_ARG;
+    if (a->num_splits < 0 || a->window < 0) return DIFFATTN_ERR_INVALID_ARG;
     if (!(a->scale > 0.0f) || !std::isfinite(a->scale)) return DIFFATTN_ERR_INVALID_ARG;
     if (!(a->eps >= 0.0f) || !std::isfinite(a->eps)) return DIFFATTN_ERR_INVALID_ARG;
     if (a->L > (1 << 26) || a->B > (1 << 16) || a->H > 4096) return DIFFATTN_ERR_UNSUPPORTED;
@@ -242,6 +244,7 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     p.eps = a->eps;
     p.causal = (a->flags & DIFFATTN_FLAG_CAUSAL) ? 1 : 0;
     p.apply_norm = (a->flags & DIFFATTN_FLAG_APPLY_NORM) ? 1 : 0;
+    p.window = a->window;
     p.withhold_load = (a->flags & DIFFATTN_FLAG_TEST_WITHHOLD_LOAD) ? 1 : 0;
     p.lambda = a->lambda;
     p.gain = p.apply_norm ? a->gain : nullptr;  // the gain belongs to the norm
@@ -307,6 +310,16 @@ diffattn_status run_decode(const diffattn_decode_args *a, float *partials, void 
     p.L = (int)a->L;
     p.splits = decode_splits(a->B, a->H, a->L, a->num_splits);
     p.chunk = decode_chunk(a->L, p.splits);
+    p.window = a->window;
+    if (a->window > 0 && a->window < a->L) {
+        // Only the window's keys are split.  The workspace holds the split
+        // count for L, so use no more splits than that.
+        const int64_t Lw = a->window;
+        int s = decode_splits(a->B, a->H, Lw, a->num_splits);
+        if (s > p.splits) s = p.splits;
+        p.chunk = decode_chunk(Lw, s);
+        p.splits = (int)((Lw + p.chunk - 1) / p.chunk);
+    }
     p.scale_log2 = a->scale * 1.4426950408889634f;
     p.eps = a->eps;
     p.apply_norm = (a->flags & DIFFATTN_FLAG_APPLY_NORM) ? 1 : 0;

@@ -27,6 +27,7 @@ struct PrefillParams {
     float scale_log2;     // softmax scale * log2(e)
     float eps;
     int causal, apply_norm;
+    int window;           // sliding window in keys (query i sees i-window < j <= i), 0 = none
     int withhold_load;    // test hook: skip the first K/V load of the CTA's first tile
     int mode;             // 0: one signal head per unit; 1, 2: grouped pairs (see prefill_sm100.cu)
     int units;            // work units per batch entry for this launch
@@ -64,6 +65,7 @@ cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, v
 struct DecodeParams {
     int B, H, L;
     int splits, chunk;    // keys per split (multiple of 64)
+    int window;           // the query sees the `window` most recent keys, 0 = all
     float scale_log2, eps;
     int apply_norm;
     const void *q1, *q2, *k1, *k2, *v;

@@ -47,6 +47,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <climits>
+
 #include "kernels.h"
 #include "sm100_ptx.cuh"
 
@@ -226,12 +228,15 @@ __device__ __forceinline__ float2 exp2_soft2(float2 x)
 // MUFU time, so only one pair in eight goes to the FMA pipe.
 constexpr uint32_t SOFT_EXP_MASK = 0x20u;  // pair 5 of every 8
 
-// Softmax of one map for one 64-key step, for the query row this thread owns.
+// Softmax of one map for one 64-key step, for the query row this thread owns;
+// keys lo..hi of the step are visible to it (a row may see none of a step's
+// keys under a sliding window: its max stays -inf and its P row is 0).
 // Reads S (fp32) from TMEM, updates the running max / sum, rescales the O row
 // when the max moved (after the previous P.V product into it has finished),
 // and writes P (fp16) over the first 32 columns of the S buffer.  Returns
 // false if a bounded wait gave up.
-__device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, bool first, int limit,
+template <bool WINDOW>
+__device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, bool first, int lo, int hi,
                                              float scale_log2, float &m_run, float &l_run,
                                              uint32_t bar_pv, uint32_t pv_parity,
                                              volatile int *abort_flag, uint64_t lim)
@@ -241,12 +246,19 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, bool firs
     tmem_ld32(tS + 32, v[1]);
     tmem_wait_ld();
 
-    if (limit < BN - 1) {  // diagonal (or ragged) step: hide keys past the limit
+    if (hi < BN - 1) {  // diagonal (or ragged) step: hide keys past hi
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-                if (32 * c + i > limit) v[c][i] = __float_as_uint(-INFINITY);
+                if (32 * c + i > hi) v[c][i] = __float_as_uint(-INFINITY);
+    }
+    if (WINDOW && lo > 0) {  // sliding-window edge: hide keys before lo
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (32 * c + i < lo) v[c][i] = __float_as_uint(-INFINITY);
     }
     // Row max of the raw scores (scale > 0 commutes with max): four
     // independent chains of three-input maxima.
@@ -310,6 +322,10 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, bool firs
     return true;
 }
 
+// WINDOW: the kernel of sliding-window calls (p.window > 0).  Without a
+// window the lower-edge mask code is left out altogether: even untaken, it
+// cost the unwindowed kernel 2-5 % (measured).
+template <bool WINDOW>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q1, const __grid_constant__ CUtensorMap tm_q2,
                    const __grid_constant__ CUtensorMap tm_k1, const __grid_constant__ CUtensorMap tm_k2,
@@ -325,9 +341,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int total = p.B * p.units * p.num_qt;
     int *sItem = reinterpret_cast<int *>(smem + OFF_ITEM);
     const int n_steps_all = (p.N + BN - 1) / BN;
+    // Key steps of a work item: [kv_first, kv_first + steps_of).  Causal tiles
+    // stop at the diagonal; under a sliding window of W keys they start at
+    // the step holding key q0 - W + 1, the first one row q0 sees.
+    auto kv_first = [&](const Work &w) {
+        return WINDOW ? max(0, w.qt * BM - p.window + 1) / BN : 0;
+    };
     auto steps_of = [&](const Work &w) {
         const int q0 = w.qt * BM;
-        return p.causal ? min(n_steps_all, (q0 + BM) / BN) : n_steps_all;
+        return (p.causal ? min(n_steps_all, (q0 + BM) / BN) : n_steps_all) - kv_first(w);
     };
 
     auto bar = [&](int i) { return sbase + OFF_BARS + 8 * i; };
@@ -428,7 +450,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const Heads hd = heads_of(w.u, p);
             const CUtensorMap *mq2 = hd.b_noise ? &tm_q2 : &tm_q1;
             const CUtensorMap *mk2 = hd.b_noise ? &tm_k2 : &tm_k1;
-            const int nkv = steps_of(w);
+            const int nkv = steps_of(w), kv0 = kv_first(w);
             // The previous tile's score MMAs must be done with Q.
             if (tiles > 0 && !(ok = mbar_wait_warp(bar(B_QFREE), (tiles - 1) & 1, abort_flag, lim)))
                 break;
@@ -444,7 +466,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     !(ok = mbar_wait_warp(bar_empty(s), ((g / STAGES) - 1) & 1, abort_flag, lim)))
                     break;
                 const uint32_t st = sbase + OFF_STAGE0 + s * STAGE_BYTES;
-                const int k0 = j * BN;
+                const int k0 = (kv0 + j) * BN;
                 if (p.withhold_load && g == 0) continue;  // test hook: this stage never fills
                 if (elect_one()) {
                     // Warm L2 with the K/V tiles of a later step of this tile
@@ -575,7 +597,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int item = next_item(tiles);
             if (item < 0) break;
             const Work w = work_of(item, p);
-            const int nkv = steps_of(w);
+            const int nkv = steps_of(w), kv0 = kv_first(w);
             const int qrow = w.qt * BM + r;
             const Heads hd = heads_of(w.u, p);
             // Output head of this warpgroup: both finish head a together in
@@ -616,9 +638,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 const int gg = g + j, buf = gg & 1;
                 if (!(ok = mbar_wait_warp(bar_s(t, buf), (gg >> 1) & 1, abort_flag, lim))) break;
                 tc_fence_after();
-                const int k0 = j * BN;
-                const int limit = p.causal ? qrow - k0 : p.N - 1 - k0;
-                if (!(ok = softmax_step(tS0 + BN * buf, tO, j == 0, limit, p.scale_log2, m_run, l_run,
+                const int k0 = (kv0 + j) * BN;
+                const int hi = p.causal ? qrow - k0 : p.N - 1 - k0;
+                const int lo = WINDOW ? qrow - p.window + 1 - k0 : INT_MIN;
+                if (!(ok = softmax_step<WINDOW>(tS0 + BN * buf, tO, j == 0, lo, hi, p.scale_log2, m_run, l_run,
                                         bar_pv, (gg - 1) & 1, abort_flag, lim)))
                     break;
                 // Every lane's P store has completed (tcgen05.wait::st in the
@@ -876,16 +899,17 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
         // launches with exactly REGS_LAUNCH registers per thread: with fewer,
         // the softmax warpgroups' increase could never be granted.  Refuse to
         // launch such a build.
-        cudaFuncAttributes fa;
-        e = cudaFuncGetAttributes(&fa, prefill_kernel);
-        if (e != cudaSuccess) return e;
-        if (fa.numRegs != REGS_LAUNCH || fa.maxThreadsPerBlock < NTHREADS) {
-            set_internal_error("prefill_kernel built with an unexpected register count");
-            return cudaErrorInvalidConfiguration;
+        for (const void *k : {(const void *)prefill_kernel<false>, (const void *)prefill_kernel<true>}) {
+            cudaFuncAttributes fa;
+            e = cudaFuncGetAttributes(&fa, k);
+            if (e != cudaSuccess) return e;
+            if (fa.numRegs != REGS_LAUNCH || fa.maxThreadsPerBlock < NTHREADS) {
+                set_internal_error("prefill_kernel built with an unexpected register count");
+                return cudaErrorInvalidConfiguration;
+            }
+            e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+            if (e != cudaSuccess) return e;
         }
-        e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)SMEM_BYTES);
-        if (e != cudaSuccess) return e;
         e = cudaDeviceGetAttribute(&num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
@@ -893,7 +917,10 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
     const int total = p.B * p.units * p.num_qt;
     if (total == 0) return cudaSuccess;
     const int grid = total < num_sms[dev] ? total : num_sms[dev];  // persistent: one CTA per SM
-    prefill_kernel<<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, p);
+    if (p.window > 0)
+        prefill_kernel<true><<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, p);
+    else
+        prefill_kernel<false><<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, p);
     ++*launches;
     return cudaGetLastError();
 }

@@ -51,6 +51,7 @@ class Workload:
     causal: bool = True
     gated: bool = False            # token-dependent lambda logits and output-gate logits
     apply_norm: bool = True
+    window: int = 0                # causal sliding window in keys (0 = none)
 
 
 WORKLOADS = {
@@ -68,6 +69,10 @@ WORKLOADS = {
     # heads, token-dependent lambda, output gate, no norm.
     "gated": Workload("gated", "grouped", B=2, N=4096, H=24, H_N=8, H_V=8, lam=(0.2, 0.8),
                       gain_std=0.0, seed=5, gated=True, apply_norm=False),
+    # A sliding-window layer (Motif 3 summary: 128-token windows) over the
+    # long-context shape.
+    "swa16k": Workload("swa16k", "prefill", B=1, N=16384, H=16, H_N=16, H_V=16, lam=(0.2, 0.8),
+                       gain_std=0.1, seed=6, window=128),
 }
 
 

@@ -63,6 +63,7 @@ class FwdArgs(ctypes.Structure):
         ("lambda_", _p), ("gain", _p), ("dev_status", _p),
         ("lambda_logits", _p), ("lambda_logits_stride", _S3),
         ("gate", _p), ("gate_stride", _S3),
+        ("window", ctypes.c_int32),
     ]
 
 
@@ -82,6 +83,7 @@ class DecodeArgs(ctypes.Structure):
         ("kv_len", _p), ("lambda_", _p), ("gain", _p), ("dev_status", _p),
         ("lambda_logits", _p), ("lambda_logits_stride", _S2),
         ("gate", _p), ("gate_stride", _S2),
+        ("window", ctypes.c_int32),
     ]
 
 
@@ -193,7 +195,8 @@ def _set_lambda_gate(a, lam, lam_logits, gate, lead, dv, S):
 
 
 def _fwd_args(q1, q2, k1, k2, v, lam, gain, out, *, scale, eps, causal, apply_norm,
-              timeout_ms, dev_status, test_withhold_load=False, lam_logits=None, gate=None):
+              timeout_ms, dev_status, test_withhold_load=False, lam_logits=None, gate=None,
+              window=0):
     for n, t in (("q1", q1), ("q2", q2), ("k1", k1), ("k2", k2), ("v", v), ("out", out)):
         _check_bf16(n, t, 4)
     B, N, H, d = q1.shape
@@ -205,6 +208,7 @@ def _fwd_args(q1, q2, k1, k2, v, lam, gain, out, *, scale, eps, causal, apply_no
     if test_withhold_load:
         a.flags |= DIFFATTN_FLAG_TEST_WITHHOLD_LOAD
     a.timeout_ms = int(timeout_ms)
+    a.window = int(window)
     for n, t in (("q1", q1), ("q2", q2), ("k1", k1), ("k2", k2), ("v", v), ("out", out)):
         setattr(a, n, t.data_ptr())
         setattr(a, n + "_stride", _S3(*t.stride()[:3]))
@@ -229,14 +233,15 @@ def _check_shapes_fwd(q1, q2, k1, k2, v):
 
 def _run_fwd(entry, q1, q2, k1, k2, v, lam, gain, *, scale, eps, causal, apply_norm, out,
              workspace, stream, timeout_ms, dev_status, test_withhold_load=False,
-             lam_logits=None, gate=None):
+             lam_logits=None, gate=None, window=0):
     _check_shapes_fwd(q1, q2, k1, k2, v)
     B, N, H, _ = q1.shape
     if out is None:
         out = torch.empty(B, N, H, v.shape[3], dtype=torch.bfloat16, device=q1.device)
     a = _fwd_args(q1, q2, k1, k2, v, lam, gain, out, scale=scale, eps=eps, causal=causal,
                   apply_norm=apply_norm, timeout_ms=timeout_ms, dev_status=dev_status,
-                  test_withhold_load=test_withhold_load, lam_logits=lam_logits, gate=gate)
+                  test_withhold_load=test_withhold_load, lam_logits=lam_logits, gate=gate,
+                  window=window)
     L = lib()
     need = L.diffattn_fwd_workspace_size(ctypes.byref(a))
     if workspace is None:
@@ -249,30 +254,33 @@ def _run_fwd(entry, q1, q2, k1, k2, v, lam, gain, *, scale, eps, causal, apply_n
 
 def diffattn_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,
                  apply_norm=True, out=None, workspace=None, stream=None, timeout_ms=0,
-                 dev_status=None, test_withhold_load=False, lam_logits=None, gate=None):
+                 dev_status=None, test_withhold_load=False, lam_logits=None, gate=None,
+                 window=0):
     """Differential-attention prefill.  q1,q2,k1,k2 [B,N,H,64], v [B,N,H,128]
     bf16 CUDA tensors (token-major, last dim contiguous); lam [H] fp32 (or
     None with lam_logits); gain [H,128] fp32 or None; lam_logits: fp32
     [B,N,H] token-dependent lambda logits or None; gate: bf16 [B,N,H,128]
-    output-gate logits or None.  Returns out [B,N,H,128] bf16.
+    output-gate logits or None; window: 0, or a causal sliding window of that
+    many keys.  Returns out [B,N,H,128] bf16.
     test_withhold_load sets the library's failure-path test hook (the call
     then reports a timeout in dev_status)."""
     return _run_fwd("diffattn_fwd", q1, q2, k1, k2, v, lam, gain, scale=scale, eps=eps,
                     causal=causal, apply_norm=apply_norm, out=out, workspace=workspace,
                     stream=stream, timeout_ms=timeout_ms, dev_status=dev_status,
-                    test_withhold_load=test_withhold_load, lam_logits=lam_logits, gate=gate)
+                    test_withhold_load=test_withhold_load, lam_logits=lam_logits, gate=gate,
+                    window=window)
 
 
 def diffattn_grouped_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,
                          apply_norm=True, out=None, workspace=None, stream=None, timeout_ms=0,
-                         dev_status=None, lam_logits=None, gate=None):
+                         dev_status=None, lam_logits=None, gate=None, window=0):
     """Grouped prefill: q1,k1 [B,N,H,64]; q2,k2 [B,N,H_N,64]; v [B,N,H_V,128];
     signal head h uses noise head h // (H // H_N) and V head h // (H // H_V).
     lam_logits [B,N,H] and gate [B,N,H,128] as in diffattn_fwd."""
     return _run_fwd("diffattn_grouped_fwd", q1, q2, k1, k2, v, lam, gain, scale=scale, eps=eps,
                     causal=causal, apply_norm=apply_norm, out=out, workspace=workspace,
                     stream=stream, timeout_ms=timeout_ms, dev_status=dev_status,
-                    lam_logits=lam_logits, gate=gate)
+                    lam_logits=lam_logits, gate=gate, window=window)
 
 
 def fwd_workspace_size(B, N, H, H_V=None, H_N=None):
@@ -291,7 +299,7 @@ def decode_num_splits(B, H, L, num_splits=0):
 
 
 def _decode_args(q1, q2, k1, k2, v, lam, gain, out, *, kv_len, num_splits, scale, eps,
-                 apply_norm, dev_status, lam_logits=None, gate=None):
+                 apply_norm, dev_status, lam_logits=None, gate=None, window=0):
     for n, t, nd in (("q1", q1, 3), ("q2", q2, 3), ("k1", k1, 4), ("k2", k2, 4), ("v", v, 4),
                      ("out", out, 3)):
         _check_bf16(n, t, nd)
@@ -305,6 +313,7 @@ def _decode_args(q1, q2, k1, k2, v, lam, gain, out, *, kv_len, num_splits, scale
     a.scale, a.eps = float(scale), float(eps)
     a.flags = DIFFATTN_FLAG_APPLY_NORM if apply_norm else 0
     a.num_splits = int(num_splits)
+    a.window = int(window)
     for n, t in (("q1", q1), ("q2", q2), ("out", out)):
         setattr(a, n, t.data_ptr())
         setattr(a, n + "_stride", _S2(*t.stride()[:2]))
@@ -326,7 +335,7 @@ def _decode_args(q1, q2, k1, k2, v, lam, gain, out, *, kv_len, num_splits, scale
 
 def diffattn_decode(q1, q2, k1, k2, v, lam, gain=None, *, kv_len=None, num_splits=0, scale=0.125,
                     eps=1e-5, apply_norm=True, out=None, workspace=None, stream=None,
-                    dev_status=None, lam_logits=None, gate=None):
+                    dev_status=None, lam_logits=None, gate=None, window=0):
     """Single-query decode.  q1,q2 [B,H,64]; k1,k2 [B,H,L,64]; v [B,H,L,128]
     bf16 CUDA tensors; kv_len int32 [B] or None; lam_logits fp32 [B,H] and
     gate bf16 [B,H,128] optional.  Returns out [B,H,128] bf16."""
@@ -335,7 +344,7 @@ def diffattn_decode(q1, q2, k1, k2, v, lam, gain=None, *, kv_len=None, num_split
         out = torch.empty(B, H, v.shape[3], dtype=torch.bfloat16, device=q1.device)
     a = _decode_args(q1, q2, k1, k2, v, lam, gain, out, kv_len=kv_len, num_splits=num_splits,
                      scale=scale, eps=eps, apply_norm=apply_norm, dev_status=dev_status,
-                     lam_logits=lam_logits, gate=gate)
+                     lam_logits=lam_logits, gate=gate, window=window)
     Lb = lib()
     need = Lb.diffattn_decode_workspace_size(B, H, L, int(num_splits))
     if workspace is None:
@@ -348,14 +357,14 @@ def diffattn_decode(q1, q2, k1, k2, v, lam, gain=None, *, kv_len=None, num_split
 
 def diffattn_decode_noalloc(q1, q2, k1, k2, v, lam, gain=None, *, out, kv_len=None, num_splits=0,
                             scale=0.125, eps=1e-5, apply_norm=True, stream=None, dev_status=None,
-                            lam_logits=None, gate=None):
+                            lam_logits=None, gate=None, window=0):
     """Single-query decode that allocates nothing: the caller passes the
     output buffer, and the per-split partial states use the library's fixed
     static scratch (see diffattn_decode_noalloc in include/diffattn.h).  For
     callers that cannot allocate device memory or hand over a workspace."""
     a = _decode_args(q1, q2, k1, k2, v, lam, gain, out, kv_len=kv_len, num_splits=num_splits,
                      scale=scale, eps=eps, apply_norm=apply_norm, dev_status=dev_status,
-                     lam_logits=lam_logits, gate=gate)
+                     lam_logits=lam_logits, gate=gate, window=window)
     st = lib().diffattn_decode_noalloc(ctypes.byref(a), _stream_ptr(stream))
     if st != 0:
         raise DiffAttnError(st, "diffattn_decode_noalloc")

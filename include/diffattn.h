@@ -63,6 +63,11 @@ typedef enum diffattn_status {
 
 #define DIFFATTN_FLAG_CAUSAL 1u      /* key j visible to query i iff j <= i */
 #define DIFFATTN_FLAG_APPLY_NORM 2u  /* apply the RMS norm + gain; else write D */
+/* Sliding window (Motif 3 summary, section 2.1: sliding-window attention
+ * layers; "Practical Implications": 128-token windows): with `window` = W > 0
+ * the query at position i sees only keys i-W < j <= i, the W most recent
+ * including itself (prefill: needs DIFFATTN_FLAG_CAUSAL; decode: the W most
+ * recent cached keys).  0 means no window.                                   */
 /* Test hook for the failure path: the prefill kernel withholds the K/V load
  * of the first key step of the first tile each CTA takes, so its bounded
  * waits run out (after timeout_ms) and the call reports
@@ -99,6 +104,7 @@ typedef struct diffattn_fwd_args {
     int32_t *dev_status;
     const float *lambda_logits; int64_t lambda_logits_stride[3];
     const void *gate;           int64_t gate_stride[3];
+    int32_t window;             /* sliding window in keys, 0 = none (causal only) */
 } diffattn_fwd_args;
 
 /* Causal (or full) prefill, one noise map per signal head: H_N and H_V must be
@@ -151,6 +157,7 @@ typedef struct diffattn_decode_args {
     int32_t *dev_status;
     const float *lambda_logits; int64_t lambda_logits_stride[2];
     const void *gate;           int64_t gate_stride[2];
+    int32_t window;             /* the query sees the `window` most recent keys; 0 = all */
 } diffattn_decode_args;
 
 /* Split-KV decode: a split kernel writes per-split partial softmax states

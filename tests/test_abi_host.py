@@ -205,6 +205,23 @@ def test_token_lambda_and_gate_validation(L):
     assert L.diffattn_decode_validate(ctypes.byref(d)) == 0
 
 
+def test_window_validation(L):
+    a = _fake_fwd_args()
+    a.window = 128
+    assert _v(L, a) == 0
+    a.window = -1
+    assert _v(L, a) == 1
+    a = _fake_fwd_args()
+    a.window = 16
+    a.flags = ops.DIFFATTN_FLAG_APPLY_NORM          # a window needs the causal mask
+    assert _v(L, a) == 1
+    d = _fake_decode_args()
+    d.window = 100
+    assert L.diffattn_decode_validate(ctypes.byref(d)) == 0
+    d.window = -5
+    assert L.diffattn_decode_validate(ctypes.byref(d)) == 1
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(ops, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(ops, "_LIB", None)

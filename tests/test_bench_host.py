@@ -85,3 +85,12 @@ def test_traffic_figure_is_dropped_when_the_kernel_source_changes(monkeypatch):
     assert t is None or t > 0
     monkeypatch.setitem(bench.PREFILL_TRAFFIC, "source_sha256_16", "0" * 16)
     assert bench.prefill_traffic() is None
+
+
+def test_window_pair_count():
+    # W(W+1)/2 pairs for the first W queries, then W per query
+    assert bench.causal_pairs(16384, 128) == 128 * 129 // 2 + (16384 - 128) * 128
+    assert bench.causal_pairs(100, 0) == bench.causal_pairs(100, 100) == 5050
+    w = inputs.WORKLOADS["swa16k"]
+    assert bench.prefill_flops(w) == 768 * 16 * bench.causal_pairs(16384, 128)
+    assert bench.prefill_bytes(w) == 16384 * 16 * 1024
