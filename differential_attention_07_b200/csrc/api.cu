@@ -209,7 +209,7 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     const int64_t HN = a->H_N ? a->H_N : a->H, HV = a->H_V ? a->H_V : a->H;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-    CUtensorMap mq1, mq2, mk1, mk2, mv;
+    CUtensorMap mq1, mq2, mk1, mk2, mv, mo;
     const bool ok =
         make_map(&mq1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->q1, 64, a->N, a->H, a->B,
                  a->q1_stride[0], a->q1_stride[1], a->q1_stride[2], da::kPrefillQRows) &&
@@ -220,7 +220,9 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
         make_map(&mk2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->k2, 64, a->N, HN, a->B,
                  a->k2_stride[0], a->k2_stride[1], a->k2_stride[2], da::kPrefillKeyRows) &&
         make_map(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws, 128, a->N, HV, a->B, a->N * HV * 128,
-                 HV * 128, 128, da::kPrefillKeyRows);
+                 HV * 128, 128, da::kPrefillKeyRows) &&
+        make_map(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->out, 128, a->N, a->H, a->B,
+                 a->out_stride[0], a->out_stride[1], a->out_stride[2], da::kPrefillOutRows);
     if (!ok) {
         da::set_internal_error("cuTensorMapEncodeTiled failed");
         return DIFFATTN_ERR_CUDA;
@@ -282,17 +284,17 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
         p.mode = 1;
         set_units((int)HN);
         p.tile_counter = tile_counter;
-        e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, p, s, &launches);
+        e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, mo, p, s, &launches);
         if (e != cudaSuccess) return cuda_status(e);
         p.mode = 2;
         set_units((int)(HN * ((g - 1) / 2)));
         p.tile_counter = tile_counter + 1;
-        e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, p, s, &launches);
+        e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, mo, p, s, &launches);
     } else {
         p.mode = 0;
         set_units((int)a->H);
         p.tile_counter = tile_counter;
-        e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, p, s, &launches);
+        e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, mo, p, s, &launches);
     }
     if (g_events.stop) cudaEventRecord(g_events.stop, s);
     if (e != cudaSuccess) return cuda_status(e);

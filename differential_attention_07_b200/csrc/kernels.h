@@ -48,12 +48,14 @@ struct PrefillParams {
 // Rows per TMA box: a query tile, and a key step of the prefill kernel.
 constexpr unsigned kPrefillQRows = 128;
 constexpr unsigned kPrefillKeyRows = 64;
+constexpr unsigned kPrefillOutRows = 32;  // rows of an output store box (one warp's rows)
 
 // Tensor maps: Q1/K1 over [B, N, H, 64] bf16, Q2/K2 over [B, N, H_N, 64]
 // bf16, V over the fp16 copy [B, N, H_V, 128]; all with 128-byte swizzle and
 // {64, rows, 1, 1} boxes (kPrefillQRows for Q, kPrefillKeyRows for K and V).
 cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const CUtensorMap &k1,
-                           const CUtensorMap &k2, const CUtensorMap &v16, const PrefillParams &p,
+                           const CUtensorMap &k2, const CUtensorMap &v16, const CUtensorMap &out,
+                           const PrefillParams &p,
                            cudaStream_t stream, int *launches);
 
 // bf16 V [B, N, H_V, 128] (strided) -> contiguous fp16 copy in `dst`; also

@@ -83,8 +83,8 @@ enum : int {
     B_PV = B_P + 4,              // [2 maps] latest P.V into O done (commit)
     B_O = B_PV + 2,              // all MMAs of the tile done (2 commits)
     B_OFREE = B_O + 1,           // epilogue finished reading O (8 softmax warps)
-    B_LX = B_OFREE + 1,          // row sums exchanged (256 arrivals)
-    B_SSX = B_LX + 1,            // partial sums of squares exchanged (256 arrivals)
+    B_LX = B_OFREE + 1,          // row sums exchanged (8 softmax warps)
+    B_SSX = B_LX + 1,            // partial sums of squares exchanged (8 softmax warps)
     B_ITEM = B_SSX + 1,          // [ITEM_SLOTS] work item published (1 arrival)
     B_ITEMFREE = B_ITEM + 4,     // [ITEM_SLOTS] work item read by all 10 reader warps
     NBARS = B_ITEMFREE + 4
@@ -103,7 +103,12 @@ constexpr int ITEM_READERS = 10;                         // 2 MMA warps + 8 soft
 constexpr uint32_t OFF_ITEM = OFF_ABORT + 4;             // int [ITEM_SLOTS] work-item ring
 constexpr uint32_t OFF_L = (OFF_ITEM + 4 * ITEM_SLOTS + 15) & ~15u;  // float [2][128] row sums
 constexpr uint32_t OFF_SS = OFF_L + 2 * BM * 4;          // float [2][128] partial sums of squares
-constexpr uint32_t SMEM_BYTES = OFF_SS + 2 * BM * 4;     // dynamic smem is 1024-byte aligned
+// Output staging: per softmax warp 32 rows x 128 columns bf16 (two 4 KB
+// halves, each one 128-byte-swizzled TMA store box of 32 rows x 64 columns).
+constexpr uint32_t OUT_HALF_BYTES = 32 * 64 * 2;
+constexpr uint32_t OUT_WARP_BYTES = 2 * OUT_HALF_BYTES;
+constexpr uint32_t OFF_OUT = (OFF_SS + 2 * BM * 4 + 1023) & ~1023u;
+constexpr uint32_t SMEM_BYTES = OFF_OUT + 8 * OUT_WARP_BYTES;  // dynamic smem is 1024-byte aligned
 
 constexpr uint32_t TM_O1 = 0, TM_O2 = 128, TM_S1 = 256, TM_S2 = 384;
 constexpr uint32_t TMEM_COLS = 512;
@@ -125,7 +130,8 @@ constexpr float RESCALE_THRESHOLD = 8.0f;
 
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(OFF_BARS % 8 == 0, "mbarriers are 8-byte aligned");
-static_assert(kPrefillQRows == BM && kPrefillKeyRows == BN, "TMA boxes match the tiles");
+static_assert(kPrefillQRows == BM && kPrefillKeyRows == BN && kPrefillOutRows == 32,
+              "TMA boxes match the tiles");
 static_assert(OFF_STAGE0 % 1024 == 0 && STAGE_BYTES % 1024 == 0 && K_BYTES % 1024 == 0,
               "SW128 atoms need 1 KB alignment");
 
@@ -329,7 +335,8 @@ template <bool WINDOW>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q1, const __grid_constant__ CUtensorMap tm_q2,
                    const __grid_constant__ CUtensorMap tm_k1, const __grid_constant__ CUtensorMap tm_k2,
-                   const __grid_constant__ CUtensorMap tm_v, const PrefillParams p)
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
+                   const PrefillParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_addr(smem);
@@ -377,8 +384,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_init(bar(B_PV + 1), 1);
         mbar_init(bar(B_O), 2);
         mbar_init(bar(B_OFREE), 8);   // one arrival per softmax warp
-        mbar_init(bar(B_LX), 256);
-        mbar_init(bar(B_SSX), 256);
+        mbar_init(bar(B_LX), 8);    // one arrival per softmax warp
+        mbar_init(bar(B_SSX), 8);
         for (int i = 0; i < ITEM_SLOTS; ++i) {
             mbar_init(bar(B_ITEM + i), 1);
             mbar_init(bar(B_ITEMFREE + i), ITEM_READERS);
@@ -686,9 +693,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                 }
                 const float rn = p.apply_norm ? rsqrtf(ss * (1.0f / HDV) + p.eps) : 1.0f;
-                uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) +
-                                2 * ((int64_t)w.b * p.out_sb + (int64_t)qrow * p.out_sn +
-                                     (int64_t)head * p.out_sh);
+                // This warp's staging buffer: the previous tile's store must
+                // have read it.
+                const uint32_t obuf = sbase + OFF_OUT + (warp - 4) * OUT_WARP_BYTES;
+                if (lane == 0) bulk_wait_read_all();
+                __syncwarp();
                 // Pass 2: D again, normalised, gain, bf16, stored; O is released
                 // after its last read.
 #pragma unroll 1
@@ -724,12 +733,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         y[2 * i4] = pack_bf162(d0 * s4.x * g4.x, d1 * s4.y * g4.y);
                         y[2 * i4 + 1] = pack_bf162(d2 * s4.z * g4.z, d3 * s4.w * g4.w);
                     }
-                    if (qrow < p.N) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + 128 * hh);
+                    // 16-byte chunk i of this row goes to chunk i ^ (row % 8)
+                    // of its 128-byte line (the TMA 128-byte swizzle).
+                    const uint32_t rowb = obuf + OUT_HALF_BYTES * hh + 128 * lane;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            dst[i] = make_uint4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
-                    }
+                    for (int i = 0; i < 8; ++i)
+                        st_shared_v4(rowb + ((i ^ (lane & 7)) << 4), y[4 * i], y[4 * i + 1], y[4 * i + 2],
+                                     y[4 * i + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                const int r0 = w.qt * BM + 32 * (warp & 3);
+                if (lane == 0 && r0 < p.N) {  // a box wholly past N is not issued
+                    tma_store_4d(&tm_out, obuf, 0, r0, head, w.b);
+                    tma_store_4d(&tm_out, obuf + OUT_HALF_BYTES, 64, r0, head, w.b);
+                    bulk_commit_group();
                 }
                 continue;
             }
@@ -744,7 +762,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 prefetch_l1(grow + 63);
             }
             sL[t * BM + r] = l_run;
-            mbar_arrive(bar(B_LX));
+            __syncwarp();  // every lane's row sum is written: one arrival for the warp
+            if (lane == 0) mbar_arrive(bar(B_LX));
             if (!(ok = mbar_wait_warp(bar(B_LX), tiles & 1, abort_flag, lim))) break;
             if (!(ok = mbar_wait_warp(bar(B_O), tiles & 1, abort_flag, lim))) break;
             tc_fence_after();
@@ -789,7 +808,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     ss = fmaf(d[32 * c + i], d[32 * c + i], ss);
                 }
             sSS[t * BM + r] = ss;
-            mbar_arrive(bar(B_SSX));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_SSX));
             float gv[64];  // this half's gain, loaded while the sums are exchanged
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -815,9 +835,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!(ok = mbar_wait_warp(bar(B_SSX), tiles & 1, abort_flag, lim))) break;
             const float rn =
                 p.apply_norm ? rsqrtf((sSS[r] + sSS[BM + r]) * (1.0f / HDV) + p.eps) : 1.0f;
-            uint8_t *orow = reinterpret_cast<uint8_t *>(p.out) +
-                            2 * ((int64_t)w.b * p.out_sb + (int64_t)qrow * p.out_sn +
-                                 (int64_t)hd.a * p.out_sh + c0);
+            // Stage this warp's 32 rows x 64 columns in shared memory (the
+            // 128-byte swizzle: 16-byte chunk i of a row at i ^ (row % 8)),
+            // then one TMA store; rows past N are clipped by the store.
+            const uint32_t obuf = sbase + OFF_OUT + (warp - 4) * OUT_WARP_BYTES;
+            if (lane == 0) bulk_wait_read_all();  // the previous tile's store has read the buffer
+            __syncwarp();
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t y[16];
@@ -826,16 +849,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     y[i] = pack_bf162(d[32 * c + 2 * i] * rn * gv[32 * c + 2 * i],
                                       d[32 * c + 2 * i + 1] * rn * gv[32 * c + 2 * i + 1]);
                 }
-                if (qrow < p.N) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + 64 * c);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+                for (int i = 0; i < 4; ++i) {
+                    const int ch = 4 * c + i;
+                    st_shared_v4(obuf + 128 * lane + ((ch ^ (lane & 7)) << 4), y[4 * i], y[4 * i + 1],
+                                 y[4 * i + 2], y[4 * i + 3]);
                 }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && w.qt * BM + 32 * (warp & 3) < p.N) {  // a box wholly past N is not issued
+                tma_store_4d(&tm_out, obuf, c0, w.qt * BM + 32 * (warp & 3), hd.a, w.b);
+                bulk_commit_group();
             }
         }
     }
 
+    if (warp >= 4 && lane == 0) bulk_wait_all();  // output stores done before the CTA exits
     tc_fence_before();
     __syncthreads();
     if (threadIdx.x == 0 && *abort_flag) report_error(p.dev_status, DIFFATTN_ERR_TIMEOUT);
@@ -880,7 +910,8 @@ __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb,
 }  // namespace
 
 cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const CUtensorMap &k1,
-                           const CUtensorMap &k2, const CUtensorMap &v16, const PrefillParams &p,
+                           const CUtensorMap &k2, const CUtensorMap &v16, const CUtensorMap &out,
+                           const PrefillParams &p,
                            cudaStream_t stream, int *launches)
 {
     // Per device: the kernel attribute and the SM count.
@@ -918,9 +949,9 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
     if (total == 0) return cudaSuccess;
     const int grid = total < num_sms[dev] ? total : num_sms[dev];  // persistent: one CTA per SM
     if (p.window > 0)
-        prefill_kernel<true><<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, p);
+        prefill_kernel<true><<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, out, p);
     else
-        prefill_kernel<false><<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, p);
+        prefill_kernel<false><<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, out, p);
     ++*launches;
     return cudaGetLastError();
 }
