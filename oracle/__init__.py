@@ -49,7 +49,7 @@ def load(path):
     lib.diffattn_oracle_prefill.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, i64,
                                             i64, i64, dp, dp, dp, dp, ctypes.c_double,
                                             ctypes.c_double, ctypes.c_int, ctypes.c_int, i64,
-                                            ip, i64, dp]
+                                            ctypes.c_double, ip, i64, dp]
     lib.diffattn_oracle_prefill.restype = ctypes.c_int
     lib.diffattn_oracle_decode.argtypes = [dp, dp, dp, dp, dp, i64, i64, i64, i64, i64,
                                            ip, dp, dp, dp, dp, ctypes.c_double, ctypes.c_double,
@@ -99,15 +99,16 @@ def softmax_row(q, k, scale):
 
 
 def prefill(q1, q2, k1, k2, v, lam, gain=None, *, scale, eps, causal=True, apply_norm=True,
-            rows=None, lam_logits=None, gate=None, window=0):
+            rows=None, lam_logits=None, gate=None, window=0, rope_theta=0.0):
     """Prefill oracle.
 
     q1, k1: [B, N, H, d]; q2, k2: [B, N, H_N, d]; v: [B, N, H_V, dv];
     lam: [H] (ignored, may be None, when lam_logits is given); gain: [H, dv]
     or None; lam_logits: token-dependent lambda logits [B, N, H] or None;
     gate: output-gate logits [B, N, H, dv] or None; window: 0, or a causal
-    sliding window of that many keys (query i sees keys i-W < j <= i).
-    Returns float64
+    sliding window of that many keys (query i sees keys i-W < j <= i);
+    rope_theta: 0, or the base of the rotary embedding applied to Q1, K1,
+    Q2, K2 by token position (interleaved pairs).  Returns float64
     [B, N, H, dv].  rows: None (all rows) or an int array [R, 3] of
     (b, i, h); then only those rows are computed and the rest is NaN.
     """
@@ -130,7 +131,7 @@ def prefill(q1, q2, k1, k2, v, lam, gain=None, *, scale, eps, causal=True, apply
                                         H_N, H_V, d, dv, _dp(lam), _dp(gain), _dp(lam_logits),
                                         _dp(gate), float(scale),
                                         float(eps), int(bool(causal)), int(bool(apply_norm)),
-                                        int(window), rp, nrows, _dp(out))
+                                        int(window), float(rope_theta), rp, nrows, _dp(out))
     if rc != 0:
         raise ValueError("oracle prefill: invalid arguments")
     return out

@@ -35,6 +35,14 @@
  *      read as one RMS group per head and token over its dv channels:
  *      Y[c] = D[c] / sqrt(mean_c D[c]^2 + eps) * gain[h][c].
  *      With apply_norm == 0 the pre-norm D is returned.
+ *   0. Rotary position embedding (optional; Motif 2.6B explainer, "The
+ *      block": RoPE with theta = 500,000).  With rope_theta > 0 every 64-wide
+ *      row of Q1, K1, Q2, K2 at token position n is rotated before step 2,
+ *      pair by pair: for c < d/2, with angle a = n * theta^(-2c/d),
+ *        x'[2c]   = x[2c] cos a - x[2c+1] sin a
+ *        x'[2c+1] = x[2c] sin a + x[2c+1] cos a.
+ *      (The pages give the base only; interleaved pairs within each map's
+ *      own 64 dimensions are this oracle's reading.)
  *   5. Token-dependent lambda and output gate (Motif 3 summary, section 2.2):
  *      lambda_t = sigma(x_t W^lambda) per signal head and token, and
  *      GDLA(x_t) = vec(sigma(G_t) (.) D_t) W^O.  The projections are outside
@@ -84,6 +92,28 @@ static double softmax_weights(const double *q, const double *k, int64_t k_row_st
         l += w[j];
     }
     return l;
+}
+
+/* Step 0: rotate every d-wide row of x [B][N][heads][d] by its token
+ * position; returns a new array (caller frees) or NULL on allocation failure. */
+static double *rope_copy(const double *x, int64_t B, int64_t N, int64_t heads, int64_t d,
+                         double theta)
+{
+    double *y = (double *)malloc(sizeof(double) * (size_t)(B * N * heads * d > 0 ? B * N * heads * d : 1));
+    if (!y) return NULL;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t h = 0; h < heads; ++h) {
+                const double *xr = x + ((b * N + n) * heads + h) * d;
+                double *yr = y + ((b * N + n) * heads + h) * d;
+                for (int64_t c = 0; c < d / 2; ++c) {
+                    const double a = (double)n * pow(theta, -2.0 * (double)c / (double)d);
+                    const double cs = cos(a), sn = sin(a);
+                    yr[2 * c] = xr[2 * c] * cs - xr[2 * c + 1] * sn;
+                    yr[2 * c + 1] = xr[2 * c] * sn + xr[2 * c + 1] * cs;
+                }
+            }
+    return y;
 }
 
 /* The logistic function sigma(x) = 1 / (1 + e^-x) of step 5.                 */
@@ -152,10 +182,22 @@ int diffattn_oracle_prefill(const double *q1, const double *q2, const double *k1
                             const double *lambda, const double *gain,
                             const double *lambda_logit, const double *gate_logit,
                             double scale, double eps, int causal, int apply_norm, int64_t window,
-                            const int64_t *rows, int64_t nrows, double *out)
+                            double rope_theta, const int64_t *rows, int64_t nrows, double *out)
 {
     if (B < 0 || N < 0 || H <= 0 || H_N <= 0 || H_V <= 0 || d <= 0 || dv <= 0) return -1;
-    if (window < 0 || (window > 0 && !causal)) return -1;
+    if (window < 0 || (window > 0 && !causal) || rope_theta < 0 || (rope_theta > 0 && d % 2)) return -1;
+    double *rq1 = NULL, *rq2 = NULL, *rk1 = NULL, *rk2 = NULL;
+    if (rope_theta > 0) {  /* step 0 */
+        rq1 = rope_copy(q1, B, N, H, d, rope_theta);
+        rk1 = rope_copy(k1, B, N, H, d, rope_theta);
+        rq2 = rope_copy(q2, B, N, H_N, d, rope_theta);
+        rk2 = rope_copy(k2, B, N, H_N, d, rope_theta);
+        if (!rq1 || !rk1 || !rq2 || !rk2) {
+            free(rq1); free(rk1); free(rq2); free(rk2);
+            return -1;
+        }
+        q1 = rq1; k1 = rk1; q2 = rq2; k2 = rk2;
+    }
     if (H % H_N != 0 || H % H_V != 0) return -1;
     const int64_t g = H / H_N;       /* signal heads per noise head */
     const int64_t gv = H / H_V;      /* signal heads per V head */
@@ -191,6 +233,7 @@ int diffattn_oracle_prefill(const double *q1, const double *q2, const double *k1
         }
         free(w1); free(w2); free(a1); free(a2);
     }
+    free(rq1); free(rk1); free(rq2); free(rk2);
     return bad ? -1 : 0;
 }
 

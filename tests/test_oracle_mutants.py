@@ -50,6 +50,13 @@ MUTANTS = {
     "decode_token_lambda_of_head": ("logistic(lambda_logit[r])", "logistic(lambda_logit[h])"),
     "window_one_key_too_many": ("? i + 1 - window : 0;", "? i - window : 0;"),
     "decode_window_one_key_too_few": ("? nkeys - window : 0;", "? nkeys - window + 1 : 0;"),
+    "rope_sin_sign": ("yr[2 * c] = xr[2 * c] * cs - xr[2 * c + 1] * sn;",
+                      "yr[2 * c] = xr[2 * c] * cs + xr[2 * c + 1] * sn;"),
+    "rope_frequency_exponent": ("pow(theta, -2.0 * (double)c / (double)d)",
+                                "pow(theta, -1.0 * (double)c / (double)d)"),
+    # (A uniform shift of every position is not a mistake: attention with
+    # rotary embeddings depends on relative positions only.)
+    "rope_keys_not_rotated": ("q1 = rq1; k1 = rk1; q2 = rq2; k2 = rk2;", "q1 = rq1; q2 = rq2;"),
 }
 
 PIN_TESTS = [f for name, f in sorted(vars(pins).items())

@@ -439,3 +439,62 @@ def test_decode_window_equals_last_prefill_row():
                        kv_len=kv_len, scale=0.125, eps=1e-5, window=W)
     for b in range(B):
         np.testing.assert_allclose(yd[b], y[b, kv_len[b] - 1], atol=1e-13, rtol=0)
+
+
+# ---------------------------------------------------------------------------
+# rotary position embedding (Motif 2.6B explainer, "The block": RoPE with
+# theta = 500,000); read as interleaved pairs within each 64-wide map vector
+# ---------------------------------------------------------------------------
+def _rope_complex(x, theta):
+    """Rotation written as complex multiplication: pair (x[2c], x[2c+1]) is the
+    number x[2c] + i x[2c+1], times exp(i n theta^(-2c/d)) at token n.
+    x: [B, N, heads, d] float64."""
+    B, N, Hh, d = x.shape
+    z = torch.view_as_complex(x.reshape(B, N, Hh, d // 2, 2).contiguous())
+    n = torch.arange(N, dtype=torch.float64)[:, None]
+    freq = theta ** (-2.0 * torch.arange(d // 2, dtype=torch.float64) / d)
+    rot = torch.polar(torch.ones(N, d // 2, dtype=torch.float64), n * freq)
+    return torch.view_as_real(z * rot[None, :, None, :]).reshape(B, N, Hh, d)
+
+
+@pytest.mark.parametrize("theta", [500000.0, 10000.0])
+def test_rope_equals_complex_rotation_then_plain(theta):
+    """The oracle with RoPE equals the plain oracle on Q/K rotated by the
+    complex-number form (grouped shape, so both maps and heads are covered)."""
+    x = _small(B=2, N=45, H=4, H_N=2, H_V=2, seed=111)
+    y = oracle.prefill(x["q1"], x["q2"], x["k1"], x["k2"], x["v"], x["lam"], x["gain"],
+                       scale=0.125, eps=1e-5, rope_theta=theta)
+    r = lambda t: _rope_complex(t, theta)
+    ref = oracle.prefill(r(x["q1"]), r(x["q2"]), r(x["k1"]), r(x["k2"]), x["v"], x["lam"],
+                         x["gain"], scale=0.125, eps=1e-5)
+    np.testing.assert_allclose(y, ref, atol=1e-12, rtol=0)
+
+
+def test_rope_leaves_row_zero_and_depends_on_relative_position():
+    """Token 0 is not rotated, so row 0 is unchanged.  And with the same q at
+    every position and the same k at every position, the score of (i, j)
+    depends only on i - j: with V one-hot over the keys the output row is the
+    weight vector, whose log-weights by distance differ between rows only by
+    a constant (the row's normaliser)."""
+    x = _small(B=1, N=12, H=1, seed=112)
+    a = (x["q1"], x["q2"], x["k1"], x["k2"], x["v"], x["lam"], x["gain"])
+    y0 = oracle.prefill(*a, scale=0.125, eps=1e-5)
+    yr = oracle.prefill(*a, scale=0.125, eps=1e-5, rope_theta=500000.0)
+    np.testing.assert_allclose(yr[:, 0], y0[:, 0], atol=1e-14, rtol=0)
+    assert np.abs(yr[:, 5:] - y0[:, 5:]).max() > 1e-4
+    # relative position: constant q and k, V = one-hot of the key index, no
+    # norm, lambda = 0: the output of row i is the weight vector over keys,
+    # and weight(i, j) depends only on i - j
+    N = 12
+    q = x["q1"][:, :1].repeat(1, N, 1, 1)
+    k = x["k1"][:, :1].repeat(1, N, 1, 1)
+    v = torch.zeros(1, N, 1, 128, dtype=torch.float64)
+    v[0, torch.arange(N), 0, torch.arange(N)] = 1.0
+    w = oracle.prefill(q, q, k, k, v, torch.zeros(1, dtype=torch.float64), scale=0.125, eps=1e-5,
+                       apply_norm=False, rope_theta=500000.0)[0, :, 0, :N]
+    s = np.log(w + 1e-300)   # log-weights: s(i, j) - logsumexp_i
+    for i in range(2, N):
+        d = s[i, :i + 1][::-1]          # by distance i - j = 0, 1, ...
+        d_prev = s[i - 1, :i][::-1]
+        # differences between distances are the same in both rows
+        np.testing.assert_allclose(d[1:i] - d[0], d_prev[1:i] - d_prev[0], atol=1e-9, rtol=0)
