@@ -296,13 +296,13 @@ def run_prefill_workload(w, steps, warmup, device, ops, rank=0, clocks=None):
     grouped = w.kind == "grouped"
     f = ops.diffattn_grouped_fwd if grouped else ops.diffattn_fwd
     out = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=device)
-    ws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H, w.H_V, w.H_N), dtype=torch.uint8, device=device)
+    ws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H, w.H_V, w.H_N, w.rope_theta), dtype=torch.uint8, device=device)
     status = torch.zeros(1, dtype=torch.int32, device=device)
 
     def call():
         f(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"], scale=w.scale, eps=w.eps,
           causal=w.causal, apply_norm=w.apply_norm, out=out, workspace=ws, dev_status=status,
-          window=w.window,
+          window=w.window, rope_theta=w.rope_theta,
           lam_logits=d.get("lam_logits"), gate=d.get("gate"))
 
     call()
@@ -340,7 +340,7 @@ def e2e_prefill(w, steps, warmup, device, ops, x):
     dev = {k: torch.empty_like(v, device=device) for k, v in x.items()}
     out = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=device)
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    ws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H, w.H_V, w.H_N), dtype=torch.uint8, device=device)
+    ws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H, w.H_V, w.H_N, w.rope_theta), dtype=torch.uint8, device=device)
     f = ops.diffattn_grouped_fwd if w.kind == "grouped" else ops.diffattn_fwd
 
     def step():
@@ -407,7 +407,7 @@ def gpu_arm(args):
     }
     if world == 1 and not args.no_extra:
         extra = {}
-        for name in ("lc16k", "grouped", "gated", "swa16k"):
+        for name in ("lc16k", "grouped", "gated", "swa16k", "rope4k"):
             wx = inputs.WORKLOADS[name]
             rx = run_prefill_workload(wx, max(3, args.steps // 5), 2, device, ops)
             fx = prefill_flops(wx)

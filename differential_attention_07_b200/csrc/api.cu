@@ -72,6 +72,14 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int64_t 
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+bool grouped_pairs(const diffattn_fwd_args *a);
+// Normalised noise outputs of paired grouped heads, fp32 [B, N, H_N, 128].
+size_t noise_bytes(const diffattn_fwd_args *a)
+{
+    if (!grouped_pairs(a)) return 0;
+    const int64_t HN = a->H_N ? a->H_N : a->H;
+    return align256((size_t)a->B * a->N * HN * 128 * sizeof(float));
+}
 
 // Grouped heads that run as (signal, noise) and (signal, signal) pairs: each
 // group of g = H / H_N signal heads shares one V head, with g odd and >= 3.
@@ -81,6 +89,25 @@ bool grouped_pairs(const diffattn_fwd_args *a)
     if (HN <= 0 || a->H % HN != 0 || HV != HN) return false;
     const int64_t g = a->H / HN;
     return g >= 3 && g % 2 == 1;
+}
+
+// Prefill workspace: [fp16 V][256 B work counters][noise outputs, paired
+// grouped heads only: [B, N, H_N, 128] fp32][rotated Q1, K1, Q2, K2 when
+// rope_theta > 0: contiguous [B, N, heads, 64] bf16 each].
+size_t v16_bytes(const diffattn_fwd_args *a);
+size_t noise_bytes(const diffattn_fwd_args *a);
+size_t rope_copy_bytes(const diffattn_fwd_args *a, int t)
+{
+    const int64_t HN = a->H_N ? a->H_N : a->H;
+    return align256((size_t)a->B * a->N * (t < 2 ? a->H : HN) * 64 * 2);
+}
+size_t rope_offset(const diffattn_fwd_args *a) { return v16_bytes(a) + 256 + noise_bytes(a); }
+size_t rope_bytes(const diffattn_fwd_args *a)
+{
+    if (!(a->rope_theta > 0.0f)) return 0;
+    size_t n = 0;
+    for (int t = 0; t < 4; ++t) n += rope_copy_bytes(a, t);
+    return n;
 }
 
 // Bytes of the fp16 V copy at the start of the prefill workspace.
@@ -105,6 +132,7 @@ diffattn_status validate_fwd(const diffattn_fwd_args *a, int grouped)
     if (!(a->eps >= 0.0f) || !std::isfinite(a->eps)) return DIFFATTN_ERR_INVALID_ARG;
     if (a->window < 0 || (a->window > 0 && !(a->flags & DIFFATTN_FLAG_CAUSAL)))
         return DIFFATTN_ERR_INVALID_ARG;
+    if (!(a->rope_theta >= 0.0f) || !std::isfinite(a->rope_theta)) return DIFFATTN_ERR_INVALID_ARG;
     // Index arithmetic inside the kernels is 32-bit for counts.
     if (a->N > (1 << 24) || a->B > (1 << 16) || a->H > 4096) return DIFFATTN_ERR_UNSUPPORTED;
     if ((a->B * a->H * ((a->N + 127) / 128)) > INT32_MAX) return DIFFATTN_ERR_UNSUPPORTED;
@@ -209,16 +237,48 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     const int64_t HN = a->H_N ? a->H_N : a->H, HV = a->H_V ? a->H_V : a->H;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
 
+    // Q/K sources of the tensor maps: the caller's tensors, or with a rotary
+    // embedding their rotated copies in the workspace (written by the
+    // staging kernel that runs first on the stream).
+    const void *qk[4] = {a->q1, a->k1, a->q2, a->k2};
+    const int64_t *qks[4] = {a->q1_stride, a->k1_stride, a->q2_stride, a->k2_stride};
+    int64_t qk_stride[4][3];
+    da::RopeStage rope{};
+    for (int t = 0; t < 4; ++t) {
+        const int64_t heads = t < 2 ? a->H : HN;
+        for (int i = 0; i < 3; ++i) qk_stride[t][i] = qks[t][i];
+        if (!(a->rope_theta > 0.0f)) continue;
+        char *dst = static_cast<char *>(ws) + rope_offset(a);
+        for (int u = 0; u < t; ++u) dst += rope_copy_bytes(a, u);
+        rope.src[t] = qk[t];
+        rope.sb[t] = qks[t][0];
+        rope.sn[t] = qks[t][1];
+        rope.sh[t] = qks[t][2];
+        rope.dst[t] = dst;
+        rope.heads[t] = (int)heads;
+        qk[t] = dst;
+        qk_stride[t][0] = a->N * heads * 64;
+        qk_stride[t][1] = heads * 64;
+        qk_stride[t][2] = 64;
+    }
+    if (a->rope_theta > 0.0f) {
+        rope.enabled = 1;
+        for (int c = 0; c < 32; ++c)  // turns per token of pair c: theta^(-2c/64) / (2 pi)
+            rope.g[c] = std::pow((double)a->rope_theta, -2.0 * c / 64.0) / 6.283185307179586;
+    }
+
+    const CUtensorMapDataType qkt =
+        a->rope_theta > 0.0f ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     CUtensorMap mq1, mq2, mk1, mk2, mv, mo;
     const bool ok =
-        make_map(&mq1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->q1, 64, a->N, a->H, a->B,
-                 a->q1_stride[0], a->q1_stride[1], a->q1_stride[2], da::kPrefillQRows) &&
-        make_map(&mq2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->q2, 64, a->N, HN, a->B,
-                 a->q2_stride[0], a->q2_stride[1], a->q2_stride[2], da::kPrefillQRows) &&
-        make_map(&mk1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->k1, 64, a->N, a->H, a->B,
-                 a->k1_stride[0], a->k1_stride[1], a->k1_stride[2], da::kPrefillKeyRows) &&
-        make_map(&mk2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->k2, 64, a->N, HN, a->B,
-                 a->k2_stride[0], a->k2_stride[1], a->k2_stride[2], da::kPrefillKeyRows) &&
+        make_map(&mq1, qkt, qk[0], 64, a->N, a->H, a->B,
+                 qk_stride[0][0], qk_stride[0][1], qk_stride[0][2], da::kPrefillQRows) &&
+        make_map(&mq2, qkt, qk[2], 64, a->N, HN, a->B,
+                 qk_stride[2][0], qk_stride[2][1], qk_stride[2][2], da::kPrefillQRows) &&
+        make_map(&mk1, qkt, qk[1], 64, a->N, a->H, a->B,
+                 qk_stride[1][0], qk_stride[1][1], qk_stride[1][2], da::kPrefillKeyRows) &&
+        make_map(&mk2, qkt, qk[3], 64, a->N, HN, a->B,
+                 qk_stride[3][0], qk_stride[3][1], qk_stride[3][2], da::kPrefillKeyRows) &&
         make_map(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws, 128, a->N, HV, a->B, a->N * HV * 128,
                  HV * 128, 128, da::kPrefillKeyRows) &&
         make_map(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->out, 128, a->N, a->H, a->B,
@@ -232,7 +292,7 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     int *tile_counter = reinterpret_cast<int *>(static_cast<char *>(ws) + v16_bytes(a));
     cudaError_t e = da::launch_v_to_f16(a->v, a->v_stride[0], a->v_stride[1], a->v_stride[2], ws,
                                         (int)a->B, (int)a->N, (int)HV, a->dev_status,
-                                        tile_counter, s, &launches);
+                                        tile_counter, rope, s, &launches);
     if (e != cudaSuccess) return cuda_status(e);
 
     da::PrefillParams p{};
@@ -247,6 +307,7 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     p.causal = (a->flags & DIFFATTN_FLAG_CAUSAL) ? 1 : 0;
     p.apply_norm = (a->flags & DIFFATTN_FLAG_APPLY_NORM) ? 1 : 0;
     p.window = a->window;
+    p.qk_f16 = a->rope_theta > 0.0f ? 1 : 0;
     p.withhold_load = (a->flags & DIFFATTN_FLAG_TEST_WITHHOLD_LOAD) ? 1 : 0;
     p.lambda = a->lambda;
     p.gain = p.apply_norm ? a->gain : nullptr;  // the gain belongs to the norm
@@ -280,7 +341,7 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     };
     if (g_events.start) cudaEventRecord(g_events.start, s);
     if (grouped_pairs(a)) {
-        p.noise_out = reinterpret_cast<float *>(static_cast<char *>(ws) + v16_bytes(a) + 256);
+        p.noise_out = reinterpret_cast<float *>(static_cast<char *>(ws) + v16_bytes(a) + 256);  // noise_bytes(a)
         p.mode = 1;
         set_units((int)HN);
         p.tile_counter = tile_counter;
@@ -381,14 +442,7 @@ diffattn_status diffattn_fwd_validate(const diffattn_fwd_args *args, int grouped
 size_t diffattn_fwd_workspace_size(const diffattn_fwd_args *a)
 {
     if (!a || a->B <= 0 || a->N <= 0 || a->H <= 0) return 0;
-    // fp16 V copy, the work-item counters, and for paired grouped heads the
-    // normalised noise outputs [B, N, H_N, 128] fp32
-    size_t n = v16_bytes(a) + 256;
-    if (grouped_pairs(a)) {
-        const int64_t HN = a->H_N ? a->H_N : a->H;
-        n += align256((size_t)a->B * a->N * HN * 128 * sizeof(float));
-    }
-    return n;
+    return rope_offset(a) + rope_bytes(a);
 }
 
 diffattn_status diffattn_fwd(const diffattn_fwd_args *args, void *workspace, size_t ws_bytes,

@@ -28,6 +28,7 @@ struct PrefillParams {
     float eps;
     int causal, apply_norm;
     int window;           // sliding window in keys (query i sees i-window < j <= i), 0 = none
+    int qk_f16;           // Q/K are fp16 (the rotated copies) rather than bf16
     int withhold_load;    // test hook: skip the first K/V load of the CTA's first tile
     int mode;             // 0: one signal head per unit; 1, 2: grouped pairs (see prefill_sm100.cu)
     int units;            // work units per batch entry for this launch
@@ -60,8 +61,21 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
 
 // bf16 V [B, N, H_V, 128] (strided) -> contiguous fp16 copy in `dst`; also
 // zeroes the two work-item counters of the prefill launches that follow.
+// Rotary-embedding part of the staging kernel: tensors 0..3 are Q1, K1, Q2,
+// K2 (heads H, H, H_N, H_N); each 64-wide row at token n is rotated into a
+// contiguous [B, N, heads, 64] fp16 copy.  g[c] = theta^(-2c/64) / (2 pi).
+struct RopeStage {
+    const void *src[4];
+    int64_t sb[4], sn[4], sh[4];
+    void *dst[4];
+    int heads[4];
+    double g[32];
+    int enabled;
+};
+
 cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, void *dst, int B,
                             int N, int H_V, int32_t *dev_status, int *tile_counter,
+                            const RopeStage &rope,
                             cudaStream_t stream, int *launches);
 
 struct DecodeParams {

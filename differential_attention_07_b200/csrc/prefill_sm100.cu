@@ -512,7 +512,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // waits for the other's softmax.  The whole warp runs the loop
         // (descriptors stay warp-uniform); an elected lane issues.
         const int t = warp - 1;
-        constexpr uint32_t ID_S = idesc_f16(1, 1, 0, BM, BN);    // bf16 x bf16, both K-major
+        // Scores: bf16 x bf16, or f16 x f16 on rotated fp16 copies; both K-major.
+        const uint32_t ID_S = p.qk_f16 ? idesc_f16(0, 0, 0, BM, BN) : idesc_f16(1, 1, 0, BM, BN);
         constexpr uint32_t ID_PV = idesc_f16(0, 0, 1, BM, HDV);  // f16 x f16, B (V) MN-major
         const uint32_t qa = sbase + (t ? OFF_Q2 : OFF_Q1);
         const uint32_t tS = tbase + (t ? TM_S2 : TM_S1), tO = tbase + (t ? TM_O2 : TM_O1);
@@ -877,7 +878,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb, int64_t sn,
                                 int64_t sh, __half *__restrict__ dst, int B, int N, int H_V,
-                                int32_t *dev_status, int *tile_counter)
+                                int32_t *dev_status, int *tile_counter, const RopeStage rope)
 {
     // The prefill launches that follow on the stream hand out their work
     // items from these two counters (one per launch).
@@ -903,6 +904,43 @@ __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb,
             out[k] = pack_half2(f.x, f.y);
         }
         reinterpret_cast<uint4 *>(dst)[i] = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+    if (overflow) report_error(dev_status, DIFFATTN_ERR_UNSUPPORTED);
+    if (!rope.enabled) return;
+    // Rotary embedding of Q1, K1, Q2, K2 (Motif 2.6B explainer, "The block"):
+    // one thread per 8 consecutive elements = 4 interleaved pairs of a 64-wide
+    // row, written as fp16 (2^-11 rounding: bf16 copies added enough logit
+    // error to break the mean tolerance).  The angle n g[c] 2 pi is reduced to a fraction of a turn in double
+    // precision (n up to 2^24), so the float sincos sees an angle in [-pi, pi).
+    for (int t = 0; t < 4; ++t) {
+        const int heads = rope.heads[t];
+        const int64_t tot = (int64_t)B * N * heads * 8;
+        const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(rope.src[t]);
+        uint4 *out = static_cast<uint4 *>(rope.dst[t]);
+        for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < tot;
+             i += (int64_t)gridDim.x * blockDim.x) {
+            const int c8 = int(i % 8);
+            const int64_t row = i / 8;
+            const int h = int(row % heads);
+            const int64_t bn = row / heads;
+            const int n = int(bn % N), b = int(bn / N);
+            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(src + b * rope.sb[t] + n * rope.sn[t] +
+                                                                  h * rope.sh[t] + 8 * c8));
+            const uint32_t in[4] = {x.x, x.y, x.z, x.w};
+            uint32_t o[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const double turns = (double)n * rope.g[4 * c8 + k];
+                const float frac = (float)(turns - rint(turns));  // in [-1/2, 1/2]
+                float sn_, cs;  // |angle| <= pi: the fast intrinsic errs by ~2^-21, below fp16 rounding
+                __sincosf(6.283185307179586f * frac, &sn_, &cs);
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&in[k]));
+                const float r0 = f.x * cs - f.y * sn_, r1 = f.x * sn_ + f.y * cs;
+                overflow |= fabsf(r0) > 65504.0f || fabsf(r1) > 65504.0f;
+                o[k] = pack_half2(r0, r1);
+            }
+            out[i] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
     }
     if (overflow) report_error(dev_status, DIFFATTN_ERR_UNSUPPORTED);
 }
@@ -958,7 +996,7 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
 
 cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, void *dst, int B,
                             int N, int H_V, int32_t *dev_status, int *tile_counter,
-                            cudaStream_t stream, int *launches)
+                            const RopeStage &rope, cudaStream_t stream, int *launches)
 {
     const int64_t total = (int64_t)B * N * H_V * (HDV / 8);
     if (total == 0) return cudaSuccess;  // nothing to stage; the prefill is skipped too
@@ -967,7 +1005,7 @@ cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, v
     if (blocks > 148 * 16) blocks = 148 * 16;
     v_to_f16_kernel<<<blocks, threads, 0, stream>>>(static_cast<const __nv_bfloat16 *>(v), sb, sn,
                                                     sh, static_cast<__half *>(dst), B, N, H_V,
-                                                    dev_status, tile_counter);
+                                                    dev_status, tile_counter, rope);
     ++*launches;
     return cudaGetLastError();
 }

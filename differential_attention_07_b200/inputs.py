@@ -52,6 +52,7 @@ class Workload:
     gated: bool = False            # token-dependent lambda logits and output-gate logits
     apply_norm: bool = True
     window: int = 0                # causal sliding window in keys (0 = none)
+    rope_theta: float = 0.0        # rotary embedding base (0 = none)
 
 
 WORKLOADS = {
@@ -73,6 +74,10 @@ WORKLOADS = {
     # long-context shape.
     "swa16k": Workload("swa16k", "prefill", B=1, N=16384, H=16, H_N=16, H_V=16, lam=(0.2, 0.8),
                        gain_std=0.1, seed=6, window=128),
+    # The 4K shape with Motif 2.6B's rotary embedding (theta = 500,000)
+    # applied by the library.
+    "rope4k": Workload("rope4k", "prefill", B=4, N=4096, H=16, H_N=16, H_V=16, lam=(0.2, 0.8),
+                       gain_std=0.1, seed=7, rope_theta=500000.0),
 }
 
 

@@ -64,6 +64,7 @@ class FwdArgs(ctypes.Structure):
         ("lambda_logits", _p), ("lambda_logits_stride", _S3),
         ("gate", _p), ("gate_stride", _S3),
         ("window", ctypes.c_int32),
+        ("rope_theta", ctypes.c_float),
     ]
 
 
@@ -196,7 +197,7 @@ def _set_lambda_gate(a, lam, lam_logits, gate, lead, dv, S):
 
 def _fwd_args(q1, q2, k1, k2, v, lam, gain, out, *, scale, eps, causal, apply_norm,
               timeout_ms, dev_status, test_withhold_load=False, lam_logits=None, gate=None,
-              window=0):
+              window=0, rope_theta=0.0):
     for n, t in (("q1", q1), ("q2", q2), ("k1", k1), ("k2", k2), ("v", v), ("out", out)):
         _check_bf16(n, t, 4)
     B, N, H, d = q1.shape
@@ -209,6 +210,7 @@ def _fwd_args(q1, q2, k1, k2, v, lam, gain, out, *, scale, eps, causal, apply_no
         a.flags |= DIFFATTN_FLAG_TEST_WITHHOLD_LOAD
     a.timeout_ms = int(timeout_ms)
     a.window = int(window)
+    a.rope_theta = float(rope_theta)
     for n, t in (("q1", q1), ("q2", q2), ("k1", k1), ("k2", k2), ("v", v), ("out", out)):
         setattr(a, n, t.data_ptr())
         setattr(a, n + "_stride", _S3(*t.stride()[:3]))
@@ -233,7 +235,7 @@ def _check_shapes_fwd(q1, q2, k1, k2, v):
 
 def _run_fwd(entry, q1, q2, k1, k2, v, lam, gain, *, scale, eps, causal, apply_norm, out,
              workspace, stream, timeout_ms, dev_status, test_withhold_load=False,
-             lam_logits=None, gate=None, window=0):
+             lam_logits=None, gate=None, window=0, rope_theta=0.0):
     _check_shapes_fwd(q1, q2, k1, k2, v)
     B, N, H, _ = q1.shape
     if out is None:
@@ -241,7 +243,7 @@ def _run_fwd(entry, q1, q2, k1, k2, v, lam, gain, *, scale, eps, causal, apply_n
     a = _fwd_args(q1, q2, k1, k2, v, lam, gain, out, scale=scale, eps=eps, causal=causal,
                   apply_norm=apply_norm, timeout_ms=timeout_ms, dev_status=dev_status,
                   test_withhold_load=test_withhold_load, lam_logits=lam_logits, gate=gate,
-                  window=window)
+                  window=window, rope_theta=rope_theta)
     L = lib()
     need = L.diffattn_fwd_workspace_size(ctypes.byref(a))
     if workspace is None:
@@ -255,38 +257,40 @@ def _run_fwd(entry, q1, q2, k1, k2, v, lam, gain, *, scale, eps, causal, apply_n
 def diffattn_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,
                  apply_norm=True, out=None, workspace=None, stream=None, timeout_ms=0,
                  dev_status=None, test_withhold_load=False, lam_logits=None, gate=None,
-                 window=0):
+                 window=0, rope_theta=0.0):
     """Differential-attention prefill.  q1,q2,k1,k2 [B,N,H,64], v [B,N,H,128]
     bf16 CUDA tensors (token-major, last dim contiguous); lam [H] fp32 (or
     None with lam_logits); gain [H,128] fp32 or None; lam_logits: fp32
     [B,N,H] token-dependent lambda logits or None; gate: bf16 [B,N,H,128]
     output-gate logits or None; window: 0, or a causal sliding window of that
-    many keys.  Returns out [B,N,H,128] bf16.
+    many keys; rope_theta: 0, or the base of the rotary embedding applied to
+    Q1, K1, Q2, K2 by token position.  Returns out [B,N,H,128] bf16.
     test_withhold_load sets the library's failure-path test hook (the call
     then reports a timeout in dev_status)."""
     return _run_fwd("diffattn_fwd", q1, q2, k1, k2, v, lam, gain, scale=scale, eps=eps,
                     causal=causal, apply_norm=apply_norm, out=out, workspace=workspace,
                     stream=stream, timeout_ms=timeout_ms, dev_status=dev_status,
                     test_withhold_load=test_withhold_load, lam_logits=lam_logits, gate=gate,
-                    window=window)
+                    window=window, rope_theta=rope_theta)
 
 
 def diffattn_grouped_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,
                          apply_norm=True, out=None, workspace=None, stream=None, timeout_ms=0,
-                         dev_status=None, lam_logits=None, gate=None, window=0):
+                         dev_status=None, lam_logits=None, gate=None, window=0, rope_theta=0.0):
     """Grouped prefill: q1,k1 [B,N,H,64]; q2,k2 [B,N,H_N,64]; v [B,N,H_V,128];
     signal head h uses noise head h // (H // H_N) and V head h // (H // H_V).
     lam_logits [B,N,H] and gate [B,N,H,128] as in diffattn_fwd."""
     return _run_fwd("diffattn_grouped_fwd", q1, q2, k1, k2, v, lam, gain, scale=scale, eps=eps,
                     causal=causal, apply_norm=apply_norm, out=out, workspace=workspace,
                     stream=stream, timeout_ms=timeout_ms, dev_status=dev_status,
-                    lam_logits=lam_logits, gate=gate, window=window)
+                    lam_logits=lam_logits, gate=gate, window=window, rope_theta=rope_theta)
 
 
-def fwd_workspace_size(B, N, H, H_V=None, H_N=None):
+def fwd_workspace_size(B, N, H, H_V=None, H_N=None, rope_theta=0.0):
     """Workspace bytes of a prefill call with these sizes."""
     a = FwdArgs()
     a.B, a.N, a.H, a.H_N, a.H_V, a.d, a.dv = B, N, H, H_N or H, H_V or H, 64, 128
+    a.rope_theta = float(rope_theta)
     return int(lib().diffattn_fwd_workspace_size(ctypes.byref(a)))
 
 

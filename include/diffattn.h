@@ -105,6 +105,17 @@ typedef struct diffattn_fwd_args {
     const float *lambda_logits; int64_t lambda_logits_stride[3];
     const void *gate;           int64_t gate_stride[3];
     int32_t window;             /* sliding window in keys, 0 = none (causal only) */
+    /* Rotary position embedding (Motif 2.6B explainer, "The block": RoPE with
+     * theta = 500,000): with rope_theta > 0 every 64-wide row of Q1, K1, Q2
+     * and K2 at token position n is rotated before the scores, in interleaved
+     * pairs: (x[2c], x[2c+1]) turned by the angle n * rope_theta^(-2c/64).
+     * The rotated copies live in the workspace as fp16 (see
+     * diffattn_fwd_workspace_size); the caller's tensors are not modified.
+     * Rotated values beyond the fp16 range report DIFFATTN_ERR_UNSUPPORTED
+     * in dev_status.
+     * 0 = no rotation.  Decode has no rotation: it reads its cache as
+     * stored.                                                               */
+    float rope_theta;
 } diffattn_fwd_args;
 
 /* Causal (or full) prefill, one noise map per signal head: H_N and H_V must be
@@ -120,7 +131,9 @@ diffattn_status diffattn_grouped_fwd(const diffattn_fwd_args *args, void *worksp
                                      size_t ws_bytes, void *stream);
 
 /* Bytes of workspace diffattn_fwd / diffattn_grouped_fwd need for `args`
- * (an fp16 copy of V for the tensor-core P.V product, and a work counter).  */
+ * (an fp16 copy of V for the tensor-core P.V product, the work counters, and
+ * depending on the arguments the grouped heads' noise outputs and the
+ * rotated copies of Q1, K1, Q2, K2).                                        */
 size_t diffattn_fwd_workspace_size(const diffattn_fwd_args *args);
 
 /* Host-only argument check of a prefill call: the status diffattn_fwd (or,

@@ -222,6 +222,19 @@ def test_window_validation(L):
     assert L.diffattn_decode_validate(ctypes.byref(d)) == 1
 
 
+def test_rope_validation_and_workspace(L):
+    a = _fake_fwd_args(B=2, N=300, H=4)
+    base = L.diffattn_fwd_workspace_size(ctypes.byref(a))
+    a.rope_theta = 500000.0
+    assert _v(L, a) == 0
+    # rotated copies of Q1, K1, Q2, K2: 4 x [B, N, H, 64] bf16
+    assert L.diffattn_fwd_workspace_size(ctypes.byref(a)) == base + 4 * 2 * 300 * 4 * 64 * 2
+    a.rope_theta = -1.0
+    assert _v(L, a) == 1
+    a.rope_theta = float("inf")
+    assert _v(L, a) == 1
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(ops, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(ops, "_LIB", None)
