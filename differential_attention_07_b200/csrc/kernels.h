@@ -56,7 +56,7 @@ constexpr unsigned kPrefillOutRows = 32;  // rows of an output store box (one wa
 // {64, rows, 1, 1} boxes (kPrefillQRows for Q, kPrefillKeyRows for K and V).
 cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const CUtensorMap &k1,
                            const CUtensorMap &k2, const CUtensorMap &v16, const CUtensorMap &out,
-                           const PrefillParams &p,
+                           const CUtensorMap &gate, const PrefillParams &p,
                            cudaStream_t stream, int *launches);
 
 // bf16 V [B, N, H_V, 128] (strided) -> contiguous fp16 copy in `dst`; also

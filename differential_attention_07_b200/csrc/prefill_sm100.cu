@@ -87,7 +87,8 @@ enum : int {
     B_SSX = B_LX + 1,            // partial sums of squares exchanged (8 softmax warps)
     B_ITEM = B_SSX + 1,          // [ITEM_SLOTS] work item published (1 arrival)
     B_ITEMFREE = B_ITEM + 4,     // [ITEM_SLOTS] work item read by all 10 reader warps
-    NBARS = B_ITEMFREE + 4
+    B_GATE = B_ITEMFREE + 4,     // [8 softmax warps] the warp's gate-logit box landed (TMA bytes)
+    NBARS = B_GATE + 8
 };
 // S and P barriers come one per S buffer: a softmax may run two steps ahead
 // of its MMA warp's wait, and with one P barrier per map the second arrival
@@ -328,15 +329,16 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, bool firs
     return true;
 }
 
-// WINDOW: the kernel of sliding-window calls (p.window > 0).  Without a
-// window the lower-edge mask code is left out altogether: even untaken, it
-// cost the unwindowed kernel 2-5 % (measured).
-template <bool WINDOW>
+// WINDOW: the kernel of sliding-window calls (p.window > 0); GATED: of calls
+// with an output gate (p.gate).  Without them their code is left out
+// altogether: even untaken, the window's lower-edge mask cost the plain
+// kernel 2-5 % and the gate's loads 2-5 % (measured).
+template <bool WINDOW, bool GATED>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q1, const __grid_constant__ CUtensorMap tm_q2,
                    const __grid_constant__ CUtensorMap tm_k1, const __grid_constant__ CUtensorMap tm_k2,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
-                   const PrefillParams p)
+                   const __grid_constant__ CUtensorMap tm_gate, const PrefillParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_addr(smem);
@@ -390,6 +392,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(bar(B_ITEM + i), 1);
             mbar_init(bar(B_ITEMFREE + i), ITEM_READERS);
         }
+        for (int i = 0; i < 8; ++i) mbar_init(bar(B_GATE + i), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -620,18 +623,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const float lam_in = ld_early_f32(
                 p.lam_logits ? p.lam_logits + w.b * p.ll_sb + qrow_c * p.ll_sn + head * p.ll_sh
                              : p.lambda + head);
-            const __nv_bfloat16 *grow =
-                p.gate ? static_cast<const __nv_bfloat16 *>(p.gate) + w.b * p.gate_sb +
-                             qrow_c * p.gate_sn + (int64_t)head * p.gate_sh + (own ? 0 : 64 * t)
-                       : nullptr;
-            if (grow) {
-                prefetch_l2(grow);
-                prefetch_l2(grow + 63);
-                if (own) {
-                    prefetch_l2(grow + 64);
-                    prefetch_l2(grow + 127);
-                }
-            }
+            // (Gate logits arrive by TMA into this warp's output staging
+            // buffer, one 32-row box per 64 columns, when the epilogue starts.)
             const float *gain = p.gain ? p.gain + (size_t)head * HDV + (own ? 0 : 64 * t) : nullptr;
             if (gain && lane < (own ? 4 : 2)) prefetch_l1(gain + 32 * lane);
             const float *an_row =
@@ -665,12 +658,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // This warpgroup's head alone: D = O / l - lambda A_N with A_N
                 // the group's normalised noise output (written by mode 1),
                 // then the RMS norm over the 128 columns of the row.
-                if (grow) {  // the row's gate logits (256 B) to L1 while the last P.V runs
-                    prefetch_l1(grow);
-                    prefetch_l1(grow + 64);
-                    prefetch_l1(grow + 127);
+                if constexpr (GATED) {  // once the previous store has read this warp's buffer
+                    if (elect_one()) {
+                        const uint32_t gbuf = sbase + OFF_OUT + (warp - 4) * OUT_WARP_BYTES;
+                        const uint32_t gbar = bar(B_GATE + (warp - 4));
+                        bulk_wait_read_all();
+                        mbar_arrive_expect_tx(gbar, OUT_WARP_BYTES);
+                        tma_load_4d_nohint(gbuf, &tm_gate, gbar, 0, w.qt * BM + 32 * (warp & 3), head, w.b);
+                        tma_load_4d_nohint(gbuf + OUT_HALF_BYTES, &tm_gate, gbar, 64, w.qt * BM + 32 * (warp & 3),
+                                           head, w.b);
+                    }
+                    __syncwarp();
                 }
                 if (!(ok = mbar_wait_warp(bar(B_O), tiles & 1, abort_flag, lim))) break;
+                // The gate box (issued above) has had the last P.V's time to land.
+                if (GATED && !(ok = mbar_wait_warp(bar(B_GATE + (warp - 4)), tiles & 1, abort_flag, lim)))
+                    break;
                 tc_fence_after();
                 const float inv = 1.0f / l_run;
                 const float lam = p.lam_logits ? logistic_fast(lam_in) : lam_in;
@@ -695,7 +698,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 const float rn = p.apply_norm ? rsqrtf(ss * (1.0f / HDV) + p.eps) : 1.0f;
                 // This warp's staging buffer: the previous tile's store must
-                // have read it.
+                // have read it (and the gate box must have landed in it).
                 const uint32_t obuf = sbase + OFF_OUT + (warp - 4) * OUT_WARP_BYTES;
                 if (lane == 0) bulk_wait_read_all();
                 __syncwarp();
@@ -719,8 +722,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         const float4 g4 = gain ? __ldg(reinterpret_cast<const float4 *>(gain) + 16 * hh + i4)
                                                : make_float4(1.f, 1.f, 1.f, 1.f);
                         float4 s4 = make_float4(rn, rn, rn, rn);  // norm x output gate
-                        if (grow) {
-                            const uint2 gq = __ldg(reinterpret_cast<const uint2 *>(grow + 64 * hh) + i4);
+                        if constexpr (GATED) {  // gate columns 4 i4 .. 4 i4 + 3 of this half, from the box
+                            const uint2 gq = ld_shared_v2(obuf + OUT_HALF_BYTES * hh + 128 * lane +
+                                                          ((((i4 >> 1) ^ (lane & 7)) << 4) | (8 * (i4 & 1))));
                             s4.x *= logistic_tanh(__uint_as_float(gq.x << 16));
                             s4.y *= logistic_tanh(__uint_as_float(gq.x & 0xffff0000u));
                             s4.z *= logistic_tanh(__uint_as_float(gq.y << 16));
@@ -758,9 +762,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // with r = lambda l1 / l2 (one fused multiply-add per element;
             // identical maps with lambda = 1 cancel exactly), then the RMS
             // norm over all 128 columns, whose sum of squares is exchanged.
-            if (grow) {  // bring this half's gate logits (128 B) to L1 while the last P.V runs
-                prefetch_l1(grow);
-                prefetch_l1(grow + 63);
+            if constexpr (GATED) {  // once the previous store has read this warp's buffer
+                if (elect_one()) {
+                    const uint32_t gbuf = sbase + OFF_OUT + (warp - 4) * OUT_WARP_BYTES;
+                    const uint32_t gbar = bar(B_GATE + (warp - 4));
+                    bulk_wait_read_all();
+                    mbar_arrive_expect_tx(gbar, OUT_HALF_BYTES);
+                    tma_load_4d_nohint(gbuf, &tm_gate, gbar, 64 * t, w.qt * BM + 32 * (warp & 3), hd.a, w.b);
+                }
+                __syncwarp();
             }
             sL[t * BM + r] = l_run;
             __syncwarp();  // every lane's row sum is written: one arrival for the warp
@@ -821,10 +831,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 gv[4 * i + 2] = g4.z;
                 gv[4 * i + 3] = g4.w;
             }
-            if (grow) {  // the output gate sigma(G) folds into the gain
+            if constexpr (GATED) {  // the output gate sigma(G), from the landed box, folds into the gain
+                if (!(ok = mbar_wait_warp(bar(B_GATE + (warp - 4)), tiles & 1, abort_flag, lim))) break;
+                const uint32_t gbuf = sbase + OFF_OUT + (warp - 4) * OUT_WARP_BYTES;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const uint4 gq = __ldg(reinterpret_cast<const uint4 *>(grow) + i);
+                    const uint4 gq = ld_shared_v4(gbuf + 128 * lane + ((i ^ (lane & 7)) << 4));
                     const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
@@ -949,7 +961,7 @@ __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb,
 
 cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const CUtensorMap &k1,
                            const CUtensorMap &k2, const CUtensorMap &v16, const CUtensorMap &out,
-                           const PrefillParams &p,
+                           const CUtensorMap &gate, const PrefillParams &p,
                            cudaStream_t stream, int *launches)
 {
     // Per device: the kernel attribute and the SM count.
@@ -968,7 +980,8 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
         // launches with exactly REGS_LAUNCH registers per thread: with fewer,
         // the softmax warpgroups' increase could never be granted.  Refuse to
         // launch such a build.
-        for (const void *k : {(const void *)prefill_kernel<false>, (const void *)prefill_kernel<true>}) {
+        for (const void *k : {(const void *)prefill_kernel<false, false>, (const void *)prefill_kernel<true, false>,
+                              (const void *)prefill_kernel<false, true>, (const void *)prefill_kernel<true, true>}) {
             cudaFuncAttributes fa;
             e = cudaFuncGetAttributes(&fa, k);
             if (e != cudaSuccess) return e;
@@ -986,10 +999,9 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
     const int total = p.B * p.units * p.num_qt;
     if (total == 0) return cudaSuccess;
     const int grid = total < num_sms[dev] ? total : num_sms[dev];  // persistent: one CTA per SM
-    if (p.window > 0)
-        prefill_kernel<true><<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, out, p);
-    else
-        prefill_kernel<false><<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, out, p);
+    auto kernel = p.gate ? (p.window > 0 ? prefill_kernel<true, true> : prefill_kernel<false, true>)
+                         : (p.window > 0 ? prefill_kernel<true, false> : prefill_kernel<false, false>);
+    kernel<<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, out, gate, p);
     ++*launches;
     return cudaGetLastError();
 }
