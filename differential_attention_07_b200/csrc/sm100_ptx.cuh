@@ -181,12 +181,7 @@ __device__ __forceinline__ uint64_t policy_evict_first()
 }
 
 // ---------------------------------------------------------------- tcgen05
-// TMEM address: bits [31:16] lane, [15:0] column.
-__device__ __forceinline__ uint32_t tmem_addr(uint32_t base, uint32_t lane, uint32_t col)
-{
-    return base + (lane << 16) + col;
-}
-
+// TMEM addresses: bits [31:16] lane, [15:0] column.
 // Warp-wide: allocate `ncols` TMEM columns, address written to smem `dst`.
 __device__ __forceinline__ void tmem_alloc(uint32_t dst, uint32_t ncols)
 {
@@ -370,19 +365,6 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
 }
-__device__ __forceinline__ float2 fmul2(float2 a, float2 b)
-{
-    float2 d;
-    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-        "mov.b64 ra, {%2, %3};\n\t"
-        "mov.b64 rb, {%4, %5};\n\t"
-        "mul.rn.f32x2 rd, ra, rb;\n\t"
-        "mov.b64 {%0, %1}, rd;\n\t}"
-        : "=f"(d.x), "=f"(d.y)
-        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-
 // Bring a global line into L1 ahead of use.
 __device__ __forceinline__ void prefetch_l1(const void *p)
 {
@@ -428,11 +410,6 @@ __device__ __forceinline__ uint2 ld_shared_v2(uint32_t addr)
 // async-proxy (TMA) reads of them.
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
-__device__ __forceinline__ void prefetch_l2(const void *p)
-{
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
 // The logistic function sigma(z) = 1 / (1 + e^-z) of Motif 3's token-dependent
 // lambda and output gate, as 1 / (1 + 2^(-z log2 e)) with MUFU ex2 and a fast
 // divide.  z is clamped to [-80, 80], where sigma is 0 or 1 to fp32 precision,
@@ -461,11 +438,6 @@ __device__ __forceinline__ float ld_early_f32(const float *p)
     float v;
     asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
     return v;
-}
-
-__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 }  // namespace da
