@@ -341,7 +341,10 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     const int64_t g = a->H / HN;
     auto set_units = [&](int units) {
         p.units = units;
-        int G = (2 * 148) / p.num_qt;  // (b, unit) pairs sharing K/V in L2 at a time
+        // (b, unit) pairs whose tiles run together, sharing their K/V in L2:
+        // about four query tiles per SM in flight (measured best at the 4K and
+        // 16K shapes: 18 and 4 heads, 36 and 32 MB of K/V)
+        int G = (4 * 148) / p.num_qt;
         if (G < 1) G = 1;
         if (G > p.B * units) G = p.B * units;
         p.heads_per_group = G;
