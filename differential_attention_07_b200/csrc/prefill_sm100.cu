@@ -23,7 +23,9 @@
 //                 each: D = (O1 - r O2)/l1 with r = lambda l1/l2, RMS norm
 //                 (sum of squares exchanged through shared memory), gain,
 //                 optional output gate sigma(G) (lambda optionally sigma of a
-//                 per-token logit: Motif 3 summary, section 2.2), bf16.
+//                 per-token logit: Motif 3 summary, section 2.2), bf16, staged
+//                 in each warp's shared-memory buffer and written by TMA
+//                 stores.
 //                 Registers are split 56 / 224 / 224 between the warpgroups
 //                 (setmaxnreg).
 // TMEM (512 columns): O1 [0,128) O2 [128,256), and two 64-column S buffers
