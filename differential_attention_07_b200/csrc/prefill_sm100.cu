@@ -918,16 +918,25 @@ __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb,
     // items from these two counters (one per launch).
     if (blockIdx.x == 0 && threadIdx.x < 2) tile_counter[threadIdx.x] = 0;
     // One thread per 8 consecutive V elements (16 bytes in, 16 bytes out).
+    // A dense V ([B, N, H_V, 128] with no gaps, the common case) is one flat
+    // array, so its chunk i needs no index arithmetic; otherwise chunk i is
+    // decomposed into (b, n, head, column) -- 64-bit divisions that made the
+    // pass compute-bound.
     const int64_t total = (int64_t)B * N * H_V * (HDV / 8);
+    const bool dense = sh == HDV && sn == (int64_t)H_V * HDV && sb == (int64_t)N * H_V * HDV;
     bool overflow = false;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
          i += (int64_t)gridDim.x * blockDim.x) {
-        const int c8 = int(i % (HDV / 8));
-        const int64_t row = i / (HDV / 8);
-        const int hv = int(row % H_V);
-        const int64_t bn = row / H_V;
-        const int n = int(bn % N), b = int(bn / N);
-        const uint4 src = __ldg(reinterpret_cast<const uint4 *>(v + b * sb + n * sn + hv * sh + 8 * c8));
+        int64_t off = 8 * i;
+        if (!dense) {
+            const int c8 = int(i % (HDV / 8));
+            const int64_t row = i / (HDV / 8);
+            const int hv = int(row % H_V);
+            const int64_t bn = row / H_V;
+            const int n = int(bn % N), b = int(bn / N);
+            off = b * sb + n * sn + hv * sh + 8 * c8;
+        }
+        const uint4 src = __ldg(reinterpret_cast<const uint4 *>(v + off));
         const uint32_t in[4] = {src.x, src.y, src.z, src.w};
         uint32_t out[4];
 #pragma unroll
@@ -951,15 +960,22 @@ __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb,
         const int64_t tot = (int64_t)B * N * heads * 8;
         const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(rope.src[t]);
         uint4 *out = static_cast<uint4 *>(rope.dst[t]);
+        const bool qk_dense = rope.sh[t] == 64 && rope.sn[t] == (int64_t)heads * 64 &&
+                              rope.sb[t] == (int64_t)N * heads * 64;
         for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < tot;
              i += (int64_t)gridDim.x * blockDim.x) {
-            const int c8 = int(i % 8);
-            const int64_t row = i / 8;
-            const int h = int(row % heads);
+            const int c8 = int(i & 7);
+            const int64_t row = i >> 3;
+            // the token position n is needed for the angle in any case; the
+            // source offset needs the full decomposition only when not dense
             const int64_t bn = row / heads;
-            const int n = int(bn % N), b = int(bn / N);
-            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(src + b * rope.sb[t] + n * rope.sn[t] +
-                                                                  h * rope.sh[t] + 8 * c8));
+            const int n = int(bn % N);
+            int64_t off = 8 * i;
+            if (!qk_dense) {
+                const int h = int(row - bn * heads), b = int(bn / N);
+                off = b * rope.sb[t] + n * rope.sn[t] + h * rope.sh[t] + 8 * c8;
+            }
+            const uint4 x = __ldg(reinterpret_cast<const uint4 *>(src + off));
             const uint32_t in[4] = {x.x, x.y, x.z, x.w};
             uint32_t o[4];
 #pragma unroll
