@@ -426,6 +426,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_ptr;
+    // The prologue above overlaps the end of the staging kernel (or, for the
+    // second grouped launch, of the first): everything below reads what they
+    // wrote -- the fp16 V and rotated Q/K copies, the work counters, the
+    // exported noise outputs.
+    grid_dependency_wait();
     const uint64_t lim = p.timeout_ns;
 
     // Work items are handed out dynamically (an atomic counter in global
@@ -914,6 +919,9 @@ __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb,
                                 int64_t sh, __half *__restrict__ dst, int B, int N, int H_V,
                                 int32_t *dev_status, int *tile_counter, const RopeStage rope)
 {
+    // The prefill launch that follows may become resident and run its
+    // prologue now; it waits for this kernel to finish before reading.
+    grid_launch_dependents();
     // The prefill launches that follow on the stream hand out their work
     // items from these two counters (one per launch).
     if (blockIdx.x == 0 && threadIdx.x < 2) tile_counter[threadIdx.x] = 0;
@@ -1039,7 +1047,21 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
     const int grid = total < num_sms[dev] ? total : num_sms[dev];  // persistent: one CTA per SM
     auto kernel = p.gate ? (p.window > 0 ? prefill_kernel<true, true> : prefill_kernel<false, true>)
                          : (p.window > 0 ? prefill_kernel<true, false> : prefill_kernel<false, false>);
-    kernel<<<grid, NTHREADS, SMEM_BYTES, stream>>>(q1, q2, k1, k2, v16, out, gate, p);
+    // Programmatic dependent launch: the prologue (barriers, TMEM) overlaps
+    // the tail of the kernel before it; the kernel waits (griddepcontrol)
+    // before touching that kernel's results.
+    cudaLaunchAttribute attr{};
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NTHREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = stream;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    cudaError_t le = cudaLaunchKernelEx(&cfg, kernel, q1, q2, k1, k2, v16, out, gate, p);
+    if (le != cudaSuccess) return le;
     ++*launches;
     return cudaGetLastError();
 }

@@ -406,6 +406,14 @@ __device__ __forceinline__ uint2 ld_shared_v2(uint32_t addr)
     asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
     return v;
 }
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while the kernel before it on the stream is still
+// running; it waits here until that kernel has completed and its memory
+// operations are visible.  The earlier kernel lets its dependents start
+// early by signalling launch_dependents.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Order this thread's generic-proxy shared-memory writes before later
 // async-proxy (TMA) reads of them.
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
