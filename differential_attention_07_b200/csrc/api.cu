@@ -75,12 +75,14 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int64_t 
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 bool grouped_pairs(const diffattn_fwd_args *a);
-// Normalised noise outputs of paired grouped heads, fp32 [B, N, H_N, 128].
+// Normalised noise outputs of paired grouped heads, fp32, per (b, noise
+// head, 128-row query tile) a tile-transposed 128 x 128 block.
 size_t noise_bytes(const diffattn_fwd_args *a)
 {
     if (!grouped_pairs(a)) return 0;
     const int64_t HN = a->H_N ? a->H_N : a->H;
-    return align256((size_t)a->B * a->N * HN * 128 * sizeof(float));
+    const int64_t tiles = (a->N + 127) / 128;
+    return align256((size_t)a->B * HN * tiles * 128 * 128 * sizeof(float));
 }
 
 // Grouped heads that run as (signal, noise) and (signal, signal) pairs: each

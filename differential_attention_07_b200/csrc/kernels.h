@@ -32,7 +32,8 @@ struct PrefillParams {
     int withhold_load;    // test hook: skip the first K/V load of the CTA's first tile
     int mode;             // 0: one signal head per unit; 1, 2: grouped pairs (see prefill_sm100.cu)
     int units;            // work units per batch entry for this launch
-    float *noise_out;     // modes 1, 2: normalised noise outputs [B, N, H_N, 128] fp32
+    float *noise_out;     // modes 1, 2: normalised noise outputs, fp32, per (b, noise head,
+                          // query tile) 32 float4 chunks x 128 rows (chunk-major)
     const float *lambda;  // [H], unused when lam_logits is set
     const float *gain;    // [H, 128] or nullptr
     const float *lam_logits;  // token-dependent lambda logits [B, N, H] or nullptr

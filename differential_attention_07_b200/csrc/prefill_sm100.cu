@@ -654,13 +654,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // buffer, one 32-row box per 64 columns, when the epilogue starts.)
             const float *gain = p.gain ? p.gain + (size_t)head * HDV + (own ? 0 : 64 * t) : nullptr;
             if (gain && lane < (own ? 4 : 2)) prefetch_l1(gain + 32 * lane);
-            const float *an_row =
-                own ? p.noise_out + (((size_t)w.b * p.N + min(qrow, p.N - 1)) * p.H_N + hd.n) * HDV
+            // The group's noise outputs of this tile, stored tile-transposed:
+            // float4 chunk c (columns 4c .. 4c + 3) of tile row r at c * 128 + r,
+            // so a warp reading chunk c of its 32 rows reads 512 contiguous bytes.
+            const float4 *an_tile =
+                own ? reinterpret_cast<const float4 *>(p.noise_out) +
+                          (((size_t)w.b * p.H_N + hd.n) * p.num_qt + w.qt) * (HDV / 4) * BM
                     : nullptr;
-            if (own) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) prefetch_l1(an_row + 32 * i);
-            }
             float m_run = -INFINITY, l_run = 0.0f;
             for (int j = 0; j < nkv; ++j) {
                 const int gg = g + j, buf = gg & 1;
@@ -714,7 +714,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tmem_wait_ld();
 #pragma unroll
                     for (int i4 = 0; i4 < 16; ++i4) {
-                        const float4 a4 = __ldg(reinterpret_cast<const float4 *>(an_row) + 16 * hh + i4);
+                        const float4 a4 = __ldg(an_tile + (16 * hh + i4) * BM + r);
                         const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -745,7 +745,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     uint32_t y[32];
 #pragma unroll
                     for (int i4 = 0; i4 < 16; ++i4) {
-                        const float4 a4 = __ldg(reinterpret_cast<const float4 *>(an_row) + 16 * hh + i4);
+                        const float4 a4 = __ldg(an_tile + (16 * hh + i4) * BM + r);
                         const float4 g4 = gain ? __ldg(reinterpret_cast<const float4 *>(gain) + 16 * hh + i4)
                                                : make_float4(1.f, 1.f, 1.f, 1.f);
                         float4 s4 = make_float4(rn, rn, rn, rn);  // norm x output gate
@@ -821,17 +821,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_OFREE));  // once per warp, after every lane's read
-            if (p.mode == 1 && qrow < p.N) {
+            if (p.mode == 1) {
                 // Export this half of the normalised noise output O2 / l2 for
-                // the group's other signal heads (mode 2).
-                float4 *an = reinterpret_cast<float4 *>(
-                    p.noise_out + (((size_t)w.b * p.N + qrow) * p.H_N + hd.n) * HDV + c0);
+                // the group's other signal heads (mode 2), tile-transposed
+                // (chunk c of row r at c * 128 + r: the warp's stores of one
+                // chunk are 512 contiguous bytes).  Rows past N go to the
+                // tile's padding.
+                float4 *an = reinterpret_cast<float4 *>(p.noise_out) +
+                             (((size_t)w.b * p.H_N + hd.n) * p.num_qt + w.qt) * (HDV / 4) * BM +
+                             (c0 / 4) * BM + r;
                 const float inv2 = 1.0f / l2;
 #pragma unroll
                 for (int c = 0; c < 2; ++c)
 #pragma unroll
                     for (int i4 = 0; i4 < 8; ++i4)
-                        an[8 * c + i4] = make_float4(__uint_as_float(ob[c][4 * i4]) * inv2,
+                        an[(8 * c + i4) * BM] = make_float4(__uint_as_float(ob[c][4 * i4]) * inv2,
                                                      __uint_as_float(ob[c][4 * i4 + 1]) * inv2,
                                                      __uint_as_float(ob[c][4 * i4 + 2]) * inv2,
                                                      __uint_as_float(ob[c][4 * i4 + 3]) * inv2);

@@ -125,10 +125,11 @@ def test_fwd_rejects_before_launch(L):
     assert L.diffattn_fwd(ctypes.byref(a), ctypes.c_void_p((1 << 30) + 16), need, None) == 3
     assert L.diffattn_grouped_fwd(ctypes.byref(_fake_fwd_args(H=6, H_N=4)), None, 0, None) == 1
     # groups of 3 signal heads sharing one V head also hold the exported
-    # noise outputs (fp32) in the workspace
+    # noise outputs (fp32, whole 128-row query tiles: 300 rows take 3) in the
+    # workspace
     g = _fake_fwd_args(H=24, H_N=8, H_V=8)
     assert L.diffattn_fwd_workspace_size(ctypes.byref(g)) == (2 * 300 * 8 * 128 * 2 + 256
-                                                             + 2 * 300 * 8 * 128 * 4)
+                                                             + 2 * 8 * 3 * 128 * 128 * 4)
     g = _fake_fwd_args(H=24, H_N=8, H_V=24)
     assert L.diffattn_fwd_workspace_size(ctypes.byref(g)) == 2 * 300 * 24 * 128 * 2 + 256
 
