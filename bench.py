@@ -80,7 +80,7 @@ def decode_bytes(w):
 # prefill_kernel launch on the 4 x 4096 x 16-head workload, from one ncu
 # capture, keyed by a hash of the kernel sources it was taken on.  A kernel
 # whose sources no longer hash to this value reports null traffic.
-PREFILL_TRAFFIC = {"source_sha256_16": "c84f8fbfd5103d8f", "bytes": 268_455_424 + 47_300_096}
+PREFILL_TRAFFIC = {"source_sha256_16": "45f80504a5d26214", "bytes": 268_578_048 + 46_927_872}
 
 
 def prefill_traffic():
