@@ -27,7 +27,9 @@ invariance; the grouped head map against repeat_interleave; decode against the
 last prefill row; a hand-derived golden example; for the token-dependent
 lambda and the gate: saturated logits reducing to SDPA, sigma(0) = 1/2,
 the lambda logits' indexing against SDPA, the gate as the element-wise last
-step, decode against the last gated prefill row.  Parity unpinned: the choice of
+step, decode against the last gated prefill row.  The backward pass
+(``oracle/backward.py``) has pins of its own (tests/test_oracle_bwd_pins.py).
+Parity unpinned: the choice of
 RMS normalisation for the pages' "GroupNorm" and the grouped V layout are
 readings of the pages, not facts the pages fix.
 """
@@ -36,6 +38,7 @@ import ctypes
 import numpy as np
 
 from . import build as _build
+from .backward import prefill_backward  # noqa: F401  (gradient of prefill, float64 NumPy)
 
 _LIB = None
 
