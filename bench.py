@@ -41,6 +41,11 @@ if ROOT not in sys.path:
 from differential_attention_07_b200 import inputs  # noqa: E402
 
 FLOP_PER_PAIR = 768  # 2*64 + 2*64 (two QK^T) + 2*128 + 2*128 (two P.V)
+# Backward, the products it cannot do without: the two score maps again
+# (2*64 each), dP = dD V^T (2*128, shared by both maps), dV = (P_1 - lambda
+# P_2)^T dD (2*128, shared), dK_1, dK_2, dQ_1, dQ_2 (2*64 each).  The kernels
+# execute 1792: the query-tile kernel recomputes both score maps and dP.
+BWD_FLOP_PER_PAIR = 1280
 
 
 def causal_pairs(N, window=0):
@@ -384,6 +389,42 @@ def e2e_prefill(w, steps, warmup, device, ops, x):
     return t / steps, h2d, d2h
 
 
+def run_backward_workload(w, steps, warmup, device, ops):
+    """Time diffattn_bwd (and the forward that saves its state) on workload w."""
+    x = inputs.workload_inputs(w)
+    d = to_dev(x, device)
+    dy = inputs.grad_output(w.B, w.N, w.H, w.dv, seed=w.seed).to(device)
+    save = torch.empty(ops.fwd_save_size(w.B, w.N, w.H), dtype=torch.uint8, device=device)
+    out = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=device)
+    fws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H), dtype=torch.uint8, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def fwd():
+        ops.diffattn_fwd(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"],
+                         scale=w.scale, eps=w.eps, causal=w.causal, out=out, workspace=fws,
+                         save=save, dev_status=status)
+
+    fwd()
+    grads = ops.diffattn_bwd(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"], dy,
+                             save, scale=w.scale, eps=w.eps, causal=w.causal, dev_status=status)
+    bws = torch.empty(ops.bwd_workspace_size(w.B, w.N, w.H), dtype=torch.uint8, device=device)
+
+    def bwd():
+        ops.diffattn_bwd(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"], dy, save,
+                         scale=w.scale, eps=w.eps, causal=w.causal, grads=grads, workspace=bws,
+                         dev_status=status)
+
+    bwd()
+    launches = ops.last_launch_count()
+    tb = time_loop(bwd, steps, warmup, device) / steps
+    tk = kernel_time(bwd, max(3, min(steps, 20)), ops)
+    tf = time_loop(fwd, steps, warmup, device) / steps
+    torch.cuda.synchronize(device)
+    if status.item() != 0:
+        raise RuntimeError(f"device status {status.item()} in the backward of {w.name}")
+    return dict(bwd_s=tb, kernel_s=tk, fwd_save_s=tf, launches=launches)
+
+
 def gpu_arm(args):
     world, rank, local = dist_env()
     device = torch.device("cuda", local)
@@ -448,6 +489,18 @@ def gpu_arm(args):
                 extra[name]["gbs"] = round(gb, 1)
                 extra[name]["hbm_frac"] = round(gb / peaks["hbm_gbs"], 4)
             del rx
+        wb = inputs.WORKLOADS["motif4k"]
+        rb = run_backward_workload(wb, max(3, args.steps // 5), 2, device, ops)
+        pb = causal_pairs(wb.N) * wb.B * wb.H
+        extra["bwd4k"] = {"tflops": round(pb * BWD_FLOP_PER_PAIR / rb["bwd_s"] / 1e12, 2),
+                          "kernel_tflops": round(pb * BWD_FLOP_PER_PAIR / rb["kernel_s"] / 1e12, 2),
+                          "frac_of_peak": round(pb * BWD_FLOP_PER_PAIR / rb["kernel_s"] / 1e12
+                                                / peaks["bf16_tflops"], 4),
+                          "ms": round(rb["bwd_s"] * 1e3, 4),
+                          "fwd_save_ms": round(rb["fwd_save_s"] * 1e3, 4),
+                          "train_step_tflops": round(pb * (FLOP_PER_PAIR + BWD_FLOP_PER_PAIR)
+                                                     / (rb["bwd_s"] + rb["fwd_save_s"]) / 1e12, 2),
+                          "flop_per_pair": BWD_FLOP_PER_PAIR, "launches": rb["launches"]}
         wd = inputs.WORKLOADS["decode"]
         rd = run_decode_workload(wd, max(5, args.steps), 3, device, ops)
         bd = decode_bytes(wd)

@@ -73,6 +73,23 @@ bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int64_t 
     return r == CUDA_SUCCESS;
 }
 
+// 4-D map over the backward pass's row statistics, fp32 [B, H, 4, n_pad]:
+// box {64 rows, 4 arrays}, no swizzle.
+bool make_stats_map(CUtensorMap *m, const float *base, int64_t n_pad, int64_t H, int64_t B)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)n_pad, 4, (cuuint64_t)H, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)(n_pad * 4), (cuuint64_t)(4 * n_pad * 4),
+                                   (cuuint64_t)(H * 4 * n_pad * 4)};
+    const cuuint32_t box[4] = {64, 4, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float *>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 bool grouped_pairs(const diffattn_fwd_args *a);
 // Normalised noise outputs of paired grouped heads, fp32, per (b, noise
@@ -160,6 +177,60 @@ diffattn_status validate_fwd(const diffattn_fwd_args *a, int grouped)
         for (int i = 0; i < 3; ++i) {
             if (strides[t][i] < 0) return DIFFATTN_ERR_INVALID_ARG;
             if (!stride8(strides[t][i])) return DIFFATTN_ERR_ALIGNMENT;
+        }
+    if (a->save) {
+        // The saved state serves the one-noise-map-per-head forward with a
+        // per-head lambda.
+        if (!aligned16(a->save)) return DIFFATTN_ERR_ALIGNMENT;
+        if (HN != a->H || HV != a->H || a->lambda_logits || a->gate || a->window > 0 ||
+            a->rope_theta > 0.0f || !a->lambda)
+            return DIFFATTN_ERR_UNSUPPORTED;
+    }
+    return DIFFATTN_OK;
+}
+
+// ---------------------------------------------------------------- backward
+// Workspace of the backward pass: [fp16 V copy][fp16 dD][row statistics
+// fp32 [B, H, 4, n_pad]][256 B: the staging kernel's counters].
+size_t bwd_half_bytes(const diffattn_bwd_args *a)
+{
+    return align256((size_t)a->B * a->N * a->H * 128 * 2);
+}
+size_t bwd_stats_bytes(const diffattn_bwd_args *a)
+{
+    return align256((size_t)a->B * a->H * 4 * ((a->N + 127) / 128) * 128 * sizeof(float));
+}
+
+diffattn_status validate_bwd(const diffattn_bwd_args *a)
+{
+    if (!a) return DIFFATTN_ERR_INVALID_ARG;
+    if (a->B < 0 || a->N < 0 || a->H <= 0) return DIFFATTN_ERR_INVALID_ARG;
+    if (a->d != 64 || a->dv != 128) return DIFFATTN_ERR_UNSUPPORTED;
+    if (a->flags & ~(DIFFATTN_FLAG_CAUSAL | DIFFATTN_FLAG_APPLY_NORM)) return DIFFATTN_ERR_INVALID_ARG;
+    if (!(a->scale > 0.0f) || !std::isfinite(a->scale)) return DIFFATTN_ERR_INVALID_ARG;
+    if (!(a->eps >= 0.0f) || !std::isfinite(a->eps)) return DIFFATTN_ERR_INVALID_ARG;
+    if (a->N > (1 << 24) || a->B > (1 << 16) || a->H > 4096) return DIFFATTN_ERR_UNSUPPORTED;
+    if ((a->B * a->H * ((a->N + 127) / 128)) > INT32_MAX) return DIFFATTN_ERR_UNSUPPORTED;
+    if (a->B == 0 || a->N == 0) return DIFFATTN_OK;
+    const void *ptrs[12] = {a->q1, a->q2, a->k1, a->k2, a->v, a->dout,
+                            a->grad_q1, a->grad_q2, a->grad_k1, a->grad_k2, a->grad_v, a->save};
+    for (const void *p : ptrs)
+        if (!p) return DIFFATTN_ERR_INVALID_ARG;
+    if (!a->lambda) return DIFFATTN_ERR_INVALID_ARG;
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return DIFFATTN_ERR_ALIGNMENT;
+    if (a->gain && !aligned16(a->gain)) return DIFFATTN_ERR_ALIGNMENT;
+    if ((a->grad_lambda && reinterpret_cast<uintptr_t>(a->grad_lambda) % 4) ||
+        (a->grad_gain && reinterpret_cast<uintptr_t>(a->grad_gain) % 4))
+        return DIFFATTN_ERR_ALIGNMENT;
+    const int64_t *strides[11] = {a->q1_stride, a->q2_stride, a->k1_stride, a->k2_stride,
+                                  a->v_stride, a->dout_stride, a->grad_q1_stride,
+                                  a->grad_q2_stride, a->grad_k1_stride, a->grad_k2_stride,
+                                  a->grad_v_stride};
+    for (const int64_t *s : strides)
+        for (int i = 0; i < 3; ++i) {
+            if (s[i] < 0) return DIFFATTN_ERR_INVALID_ARG;
+            if (!stride8(s[i])) return DIFFATTN_ERR_ALIGNMENT;
         }
     return DIFFATTN_OK;
 }
@@ -369,8 +440,112 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
         p.mode = 0;
         set_units((int)a->H);
         p.tile_counter = tile_counter;
+        p.save = static_cast<float *>(a->save);
         e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, mo, mg, p, s, &launches);
     }
+    if (g_events.stop) cudaEventRecord(g_events.stop, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    g_last_launches = launches;
+    return DIFFATTN_OK;
+}
+
+diffattn_status run_bwd(const diffattn_bwd_args *a, void *ws, size_t ws_bytes, void *stream)
+{
+    g_last_launches = 0;
+    g_last_error[0] = 0;
+    diffattn_status st = validate_bwd(a);
+    if (st != DIFFATTN_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // dlambda and dgain are sums over rows: start them at zero (and leave
+    // them there for an empty problem).
+    if (a->grad_lambda) {
+        cudaError_t e = cudaMemsetAsync(a->grad_lambda, 0, (size_t)a->H * sizeof(float), s);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    if (a->grad_gain) {
+        cudaError_t e = cudaMemsetAsync(a->grad_gain, 0, (size_t)a->H * 128 * sizeof(float), s);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    if (a->B == 0 || a->N == 0) return DIFFATTN_OK;
+    const size_t need = diffattn_bwd_workspace_size(a);
+    if (!ws || ws_bytes < need) return DIFFATTN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return DIFFATTN_ERR_ALIGNMENT;
+
+    char *w = static_cast<char *>(ws);
+    void *v16 = w;
+    void *dd = w + bwd_half_bytes(a);
+    float *stats = reinterpret_cast<float *>(w + 2 * bwd_half_bytes(a));
+    int *counters = reinterpret_cast<int *>(w + 2 * bwd_half_bytes(a) + bwd_stats_bytes(a));
+    const int64_t num_qt = (a->N + 127) / 128, n_pad = num_qt * 128;
+    const int64_t hs = a->N * a->H * 128;  // batch stride of the contiguous fp16 copies
+
+    da::BwdKeyMaps km;
+    da::BwdQueryMaps qm;
+    const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    const bool ok =
+        make_map(&km.k1, bf, a->k1, 64, a->N, a->H, a->B, a->k1_stride[0], a->k1_stride[1], a->k1_stride[2], 128) &&
+        make_map(&km.k2, bf, a->k2, 64, a->N, a->H, a->B, a->k2_stride[0], a->k2_stride[1], a->k2_stride[2], 128) &&
+        make_map(&km.v, f16, v16, 128, a->N, a->H, a->B, hs, a->H * 128, 128, 128) &&
+        make_map(&km.q1, bf, a->q1, 64, a->N, a->H, a->B, a->q1_stride[0], a->q1_stride[1], a->q1_stride[2], 64) &&
+        make_map(&km.q2, bf, a->q2, 64, a->N, a->H, a->B, a->q2_stride[0], a->q2_stride[1], a->q2_stride[2], 64) &&
+        make_map(&km.dd, f16, dd, 128, a->N, a->H, a->B, hs, a->H * 128, 128, 64) &&
+        make_stats_map(&km.stats, stats, n_pad, a->H, a->B) &&
+        make_map(&qm.q1, bf, a->q1, 64, a->N, a->H, a->B, a->q1_stride[0], a->q1_stride[1], a->q1_stride[2], 128) &&
+        make_map(&qm.q2, bf, a->q2, 64, a->N, a->H, a->B, a->q2_stride[0], a->q2_stride[1], a->q2_stride[2], 128) &&
+        make_map(&qm.dd, f16, dd, 128, a->N, a->H, a->B, hs, a->H * 128, 128, 128) &&
+        make_map(&qm.k1, bf, a->k1, 64, a->N, a->H, a->B, a->k1_stride[0], a->k1_stride[1], a->k1_stride[2], 64) &&
+        make_map(&qm.k2, bf, a->k2, 64, a->N, a->H, a->B, a->k2_stride[0], a->k2_stride[1], a->k2_stride[2], 64) &&
+        make_map(&qm.v, f16, v16, 128, a->N, a->H, a->B, hs, a->H * 128, 128, 64);
+    if (!ok) {
+        da::set_internal_error("cuTensorMapEncodeTiled failed");
+        return DIFFATTN_ERR_CUDA;
+    }
+
+    int launches = 0;
+    const da::RopeStage no_rope{};
+    cudaError_t e = da::launch_v_to_f16(a->v, a->v_stride[0], a->v_stride[1], a->v_stride[2], v16,
+                                        (int)a->B, (int)a->N, (int)a->H, a->dev_status, counters,
+                                        no_rope, s, &launches);
+    if (e != cudaSuccess) return cuda_status(e);
+
+    da::BwdParams p{};
+    p.B = (int)a->B;
+    p.N = (int)a->N;
+    p.H = (int)a->H;
+    p.num_qt = (int)num_qt;
+    p.n_pad = (int)n_pad;
+    p.scale = a->scale;
+    p.scale_log2 = a->scale * 1.4426950408889634f;
+    p.eps = a->eps;
+    p.causal = (a->flags & DIFFATTN_FLAG_CAUSAL) ? 1 : 0;
+    p.apply_norm = (a->flags & DIFFATTN_FLAG_APPLY_NORM) ? 1 : 0;
+    p.save = static_cast<const float *>(a->save);
+    p.dout = a->dout;
+    p.do_sb = a->dout_stride[0];
+    p.do_sn = a->dout_stride[1];
+    p.do_sh = a->dout_stride[2];
+    p.lambda = a->lambda;
+    p.gain = a->gain;
+    p.dd = dd;
+    p.stats = stats;
+    p.dq1 = a->grad_q1;
+    p.dq2 = a->grad_q2;
+    p.dk1 = a->grad_k1;
+    p.dk2 = a->grad_k2;
+    p.dv = a->grad_v;
+    for (int i = 0; i < 3; ++i) {
+        p.dq1_s[i] = a->grad_q1_stride[i];
+        p.dq2_s[i] = a->grad_q2_stride[i];
+        p.dk1_s[i] = a->grad_k1_stride[i];
+        p.dk2_s[i] = a->grad_k2_stride[i];
+        p.dv_s[i] = a->grad_v_stride[i];
+    }
+    p.dlambda = a->grad_lambda;
+    p.dgain = a->grad_gain;
+    p.dev_status = a->dev_status;
+    p.timeout_ns = (uint64_t)(a->timeout_ms ? a->timeout_ms : kDefaultTimeoutMs) * 1000000ull;
+    if (g_events.start) cudaEventRecord(g_events.start, s);
+    e = da::launch_bwd(km, qm, p, s, &launches);
     if (g_events.stop) cudaEventRecord(g_events.stop, s);
     if (e != cudaSuccess) return cuda_status(e);
     g_last_launches = launches;
@@ -459,6 +634,18 @@ size_t diffattn_fwd_workspace_size(const diffattn_fwd_args *a)
     return rope_offset(a) + rope_bytes(a);
 }
 
+size_t diffattn_fwd_save_size(const diffattn_fwd_args *a)
+{
+    if (!a || a->B <= 0 || a->N <= 0 || a->H <= 0) return 0;
+    return (size_t)a->B * a->H * ((a->N + 127) / 128) * da::kSaveTileFloats * sizeof(float);
+}
+
+size_t diffattn_bwd_workspace_size(const diffattn_bwd_args *a)
+{
+    if (!a || a->B <= 0 || a->N <= 0 || a->H <= 0) return 0;
+    return 2 * bwd_half_bytes(a) + bwd_stats_bytes(a) + 256;
+}
+
 // A named NVTX range around each entry point, for timeline profilers (a
 // no-op unless one is attached).
 struct NvtxRange {
@@ -478,6 +665,13 @@ diffattn_status diffattn_grouped_fwd(const diffattn_fwd_args *args, void *worksp
 {
     NvtxRange range("diffattn_grouped_fwd");
     return run_fwd(args, workspace, ws_bytes, stream, 1);
+}
+
+diffattn_status diffattn_bwd(const diffattn_bwd_args *args, void *workspace, size_t ws_bytes,
+                             void *stream)
+{
+    NvtxRange range("diffattn_bwd");
+    return run_bwd(args, workspace, ws_bytes, stream);
 }
 
 diffattn_status diffattn_decode_validate(const diffattn_decode_args *args)

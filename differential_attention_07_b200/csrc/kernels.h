@@ -45,7 +45,14 @@ struct PrefillParams {
     int32_t *dev_status;
     uint64_t timeout_ns;
     int *tile_counter;    // work-item counter in the workspace (zeroed by the V staging kernel)
+    float *save;          // mode 0: state saved for the backward pass, or nullptr
 };
+
+// The forward's saved state, per (b, h, 128-row query tile): A_1 and A_2 as
+// fp32 float4 chunks, chunk c of map t and tile row r at float4 index
+// (32 t + c) * 128 + r, then lse_t (log2 of the softmax denominator, in the
+// units of scale * log2(e) * score) at float index 2 * 128 * 128 + 128 t + r.
+constexpr int kSaveTileFloats = 2 * 128 * 128 + 2 * 128;
 
 // Rows per TMA box: a query tile, and a key step of the prefill kernel.
 constexpr unsigned kPrefillQRows = 128;
@@ -78,6 +85,45 @@ cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, v
                             int N, int H_V, int32_t *dev_status, int *tile_counter,
                             const RopeStage &rope,
                             cudaStream_t stream, int *launches);
+
+// Backward pass (backward_sm100.cu).  H_N == H_V == H.
+struct BwdParams {
+    int B, N, H;
+    int num_qt, n_pad;    // 128-row tiles per (b, h) and n_pad = 128 num_qt
+    float scale, scale_log2, eps;
+    int causal, apply_norm;
+    const float *save;    // the forward's saved state (kSaveTileFloats per tile)
+    const void *dout;     // bf16 [B, N, H, 128]
+    int64_t do_sb, do_sn, do_sh;
+    const float *lambda;  // [H]
+    const float *gain;    // [H, 128] or nullptr (1)
+    void *dd;             // workspace: dD as fp16, contiguous [B, N, H, 128]
+    float *stats;         // workspace: [B, H, 4, n_pad] fp32 (lse_1, lse_2, Delta_1, Delta_2)
+    void *dq1, *dq2, *dk1, *dk2, *dv;  // bf16 outputs
+    int64_t dq1_s[3], dq2_s[3], dk1_s[3], dk2_s[3], dv_s[3];
+    float *dlambda;       // [H] (zeroed before the call) or nullptr
+    float *dgain;         // [H, 128] (zeroed before the call) or nullptr
+    int32_t *dev_status;
+    uint64_t timeout_ns;
+};
+
+// Tensor maps of the key-tile kernel (dK_1, dK_2, dV): K_1, K_2 and the fp16
+// V copy in 128-row boxes; Q_1, Q_2 and dD in 64-row boxes; the statistics
+// (fp32, no swizzle) in {64, 4} boxes.  All 128-byte swizzled, {64, rows}.
+struct BwdKeyMaps {
+    CUtensorMap k1, k2, v, q1, q2, dd, stats;
+};
+// Tensor maps of the query-tile kernel (dQ_1, dQ_2): Q_1, Q_2, dD in 128-row
+// boxes; K_1, K_2 and the fp16 V copy in 64-row boxes.
+struct BwdQueryMaps {
+    CUtensorMap q1, q2, dd, k1, k2, v;
+};
+
+// Launch the backward kernels after the V staging: the row preparation
+// (dD, statistics, dlambda, dgain), the key-tile kernel and the query-tile
+// kernel.
+cudaError_t launch_bwd(const BwdKeyMaps &km, const BwdQueryMaps &qm, const BwdParams &p,
+                       cudaStream_t stream, int *launches);
 
 struct DecodeParams {
     int B, H, L;

@@ -209,18 +209,6 @@ __device__ __forceinline__ Work work_of(int idx, const PrefillParams &p)
     return Work{bh / p.units, bh % p.units, qt};
 }
 
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
-{
-    __half2 h = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-
-__device__ __forceinline__ uint32_t pack_bf162(float lo, float hi)
-{
-    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-
 // Software 2^x for two values at once on the FMA and integer pipes, to take
 // part of the exponentials off MUFU.  Cody-Waite style range reduction:
 // x = n + f with n = rint(x) from the 1.5 * 2^23 magic-number add (the
@@ -352,10 +340,11 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, bool firs
 }
 
 // WINDOW: the kernel of sliding-window calls (p.window > 0); GATED: of calls
-// with an output gate (p.gate).  Without them their code is left out
+// with an output gate (p.gate); SAVE: of calls that also save the state of
+// the backward pass (p.save).  Without them their code is left out
 // altogether: even untaken, the window's lower-edge mask cost the plain
 // kernel 2-5 % and the gate's loads 2-5 % (measured).
-template <bool WINDOW, bool GATED>
+template <bool WINDOW, bool GATED, bool SAVE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q1, const __grid_constant__ CUtensorMap tm_q2,
                    const __grid_constant__ CUtensorMap tm_k1, const __grid_constant__ CUtensorMap tm_k2,
@@ -821,6 +810,27 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_OFREE));  // once per warp, after every lane's read
+            if constexpr (SAVE) {
+                // Saved for the backward pass (mode 0): this half's columns of
+                // A_1 = O1 / l1 and A_2 = O2 / l2, chunk-major like the noise
+                // outputs, and this warpgroup's map's lse = m + log2(l) (the
+                // running max and sum are in units of scale * log2(e) * score).
+                float *tile = p.save + ((size_t)(w.b * p.H + hd.a) * p.num_qt + w.qt) * kSaveTileFloats;
+                float4 *sa = reinterpret_cast<float4 *>(tile) + (c0 / 4) * BM + r;
+                const float inv2 = 1.0f / l2;
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                        sa[(8 * c + i4) * BM] = make_float4(
+                            __uint_as_float(oa[c][4 * i4]) * inv1, __uint_as_float(oa[c][4 * i4 + 1]) * inv1,
+                            __uint_as_float(oa[c][4 * i4 + 2]) * inv1, __uint_as_float(oa[c][4 * i4 + 3]) * inv1);
+                        sa[(32 + 8 * c + i4) * BM] = make_float4(
+                            __uint_as_float(ob[c][4 * i4]) * inv2, __uint_as_float(ob[c][4 * i4 + 1]) * inv2,
+                            __uint_as_float(ob[c][4 * i4 + 2]) * inv2, __uint_as_float(ob[c][4 * i4 + 3]) * inv2);
+                    }
+                tile[2 * BM * HDV + t * BM + r] = m_run + log2f(l_run);
+            }
             if (p.mode == 1) {
                 // Export this half of the normalised noise output O2 / l2 for
                 // the group's other signal heads (mode 2), tile-transposed
@@ -1030,8 +1040,11 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
         // launches with exactly REGS_LAUNCH registers per thread: with fewer,
         // the softmax warpgroups' increase could never be granted.  Refuse to
         // launch such a build.
-        for (const void *k : {(const void *)prefill_kernel<false, false>, (const void *)prefill_kernel<true, false>,
-                              (const void *)prefill_kernel<false, true>, (const void *)prefill_kernel<true, true>}) {
+        for (const void *k : {(const void *)prefill_kernel<false, false, false>,
+                              (const void *)prefill_kernel<true, false, false>,
+                              (const void *)prefill_kernel<false, true, false>,
+                              (const void *)prefill_kernel<true, true, false>,
+                              (const void *)prefill_kernel<false, false, true>}) {
             cudaFuncAttributes fa;
             e = cudaFuncGetAttributes(&fa, k);
             if (e != cudaSuccess) return e;
@@ -1049,8 +1062,9 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
     const int total = p.B * p.units * p.num_qt;
     if (total == 0) return cudaSuccess;
     const int grid = total < num_sms[dev] ? total : num_sms[dev];  // persistent: one CTA per SM
-    auto kernel = p.gate ? (p.window > 0 ? prefill_kernel<true, true> : prefill_kernel<false, true>)
-                         : (p.window > 0 ? prefill_kernel<true, false> : prefill_kernel<false, false>);
+    auto kernel = p.save ? prefill_kernel<false, false, true>
+                  : p.gate ? (p.window > 0 ? prefill_kernel<true, true, false> : prefill_kernel<false, true, false>)
+                           : (p.window > 0 ? prefill_kernel<true, false, false> : prefill_kernel<false, false, false>);
     // Programmatic dependent launch: the prologue (barriers, TMEM) overlaps
     // the tail of the kernel before it; the kernel waits (griddepcontrol)
     // before touching that kernel's results.

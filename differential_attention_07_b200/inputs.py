@@ -141,6 +141,14 @@ def gate_inputs(B, N, H, dv=128, *, seed=0, lam_logit_std=1.5, gate_std=2.0):
     return dict(lam_logits=lam_logits, gate=gate)
 
 
+def grad_output(B, N, H, dv=128, *, seed=0, std=1.0):
+    """Gradient of a loss with respect to the prefill output, dY [B, N, H, dv]
+    bf16: a generator seeded with ``seed + 2000``, ``randn * std`` rounded to
+    bf16 (the upstream gradient a training step hands the backward pass)."""
+    g = torch.Generator().manual_seed(seed + 2000)
+    return (std * torch.randn(B, N, H, dv, generator=g, dtype=torch.float32)).to(torch.bfloat16)
+
+
 def workload_inputs(w: Workload):
     """Inputs of a named workload (CPU tensors)."""
     if w.kind == "decode":

@@ -10,6 +10,9 @@ Functions (same names as the C entry points):
     diffattn_fwd(q1, q2, k1, k2, v, lam, gain=None, ...)          -> out
     diffattn_grouped_fwd(q1, q2, k1, k2, v, lam, gain=None, ...)  -> out
     diffattn_decode(q1, q2, k1, k2, v, lam, gain=None, ...)       -> out
+    diffattn_bwd(q1, q2, k1, k2, v, lam, gain, dout, save, ...)   -> gradients
+and DiffAttention / diff_attention, a torch.autograd.Function over
+diffattn_fwd (with the saved state) and diffattn_bwd, for training.
 """
 import ctypes
 import os
@@ -39,6 +42,7 @@ EXPORTED = [
     "diffattn_decode", "diffattn_decode_workspace_size", "diffattn_decode_num_splits",
     "diffattn_decode_validate", "diffattn_status_str", "diffattn_last_launch_count",
     "diffattn_set_profile_events", "diffattn_last_error", "diffattn_decode_noalloc",
+    "diffattn_bwd", "diffattn_bwd_workspace_size", "diffattn_fwd_save_size",
 ]
 
 _i64 = ctypes.c_int64
@@ -65,6 +69,30 @@ class FwdArgs(ctypes.Structure):
         ("gate", _p), ("gate_stride", _S3),
         ("window", ctypes.c_int32),
         ("rope_theta", ctypes.c_float),
+        ("save", _p),
+    ]
+
+
+class BwdArgs(ctypes.Structure):
+    """Mirror of struct diffattn_bwd_args."""
+    _fields_ = [
+        ("B", _i64), ("N", _i64), ("H", _i64),
+        ("d", _i64), ("dv", _i64),
+        ("scale", ctypes.c_float), ("eps", ctypes.c_float),
+        ("flags", ctypes.c_uint32), ("timeout_ms", ctypes.c_uint32),
+        ("q1", _p), ("q1_stride", _S3),
+        ("q2", _p), ("q2_stride", _S3),
+        ("k1", _p), ("k1_stride", _S3),
+        ("k2", _p), ("k2_stride", _S3),
+        ("v", _p), ("v_stride", _S3),
+        ("dout", _p), ("dout_stride", _S3),
+        ("save", _p), ("lambda_", _p), ("gain", _p),
+        ("grad_q1", _p), ("grad_q1_stride", _S3),
+        ("grad_q2", _p), ("grad_q2_stride", _S3),
+        ("grad_k1", _p), ("grad_k1_stride", _S3),
+        ("grad_k2", _p), ("grad_k2_stride", _S3),
+        ("grad_v", _p), ("grad_v_stride", _S3),
+        ("grad_lambda", _p), ("grad_gain", _p), ("dev_status", _p),
     ]
 
 
@@ -110,13 +138,19 @@ def lib():
             raise RuntimeError(f"libdiffattn is not built ({LIB_PATH} missing); run "
                                "`python -m differential_attention_07_b200.build`")
         L = ctypes.CDLL(LIB_PATH)
-        fa, da = ctypes.POINTER(FwdArgs), ctypes.POINTER(DecodeArgs)
+        fa, da, ba = ctypes.POINTER(FwdArgs), ctypes.POINTER(DecodeArgs), ctypes.POINTER(BwdArgs)
         for name in ("diffattn_fwd", "diffattn_grouped_fwd"):
             f = getattr(L, name)
             f.argtypes = [fa, _p, ctypes.c_size_t, _p]
             f.restype = ctypes.c_int
         L.diffattn_fwd_workspace_size.argtypes = [fa]
         L.diffattn_fwd_workspace_size.restype = ctypes.c_size_t
+        L.diffattn_fwd_save_size.argtypes = [fa]
+        L.diffattn_fwd_save_size.restype = ctypes.c_size_t
+        L.diffattn_bwd.argtypes = [ba, _p, ctypes.c_size_t, _p]
+        L.diffattn_bwd.restype = ctypes.c_int
+        L.diffattn_bwd_workspace_size.argtypes = [ba]
+        L.diffattn_bwd_workspace_size.restype = ctypes.c_size_t
         L.diffattn_fwd_validate.argtypes = [fa, ctypes.c_int]
         L.diffattn_fwd_validate.restype = ctypes.c_int
         L.diffattn_decode.argtypes = [da, _p, ctypes.c_size_t, _p]
@@ -197,7 +231,7 @@ def _set_lambda_gate(a, lam, lam_logits, gate, lead, dv, S):
 
 def _fwd_args(q1, q2, k1, k2, v, lam, gain, out, *, scale, eps, causal, apply_norm,
               timeout_ms, dev_status, test_withhold_load=False, lam_logits=None, gate=None,
-              window=0, rope_theta=0.0):
+              window=0, rope_theta=0.0, save=None):
     for n, t in (("q1", q1), ("q2", q2), ("k1", k1), ("k2", k2), ("v", v), ("out", out)):
         _check_bf16(n, t, 4)
     B, N, H, d = q1.shape
@@ -220,6 +254,11 @@ def _fwd_args(q1, q2, k1, k2, v, lam, gain, out, *, scale, eps, causal, apply_no
             raise ValueError("gain must be contiguous float32 [H, dv]")
         a.gain = gain.data_ptr()
     a.dev_status = dev_status.data_ptr() if dev_status is not None else None
+    if save is not None:
+        need = int(lib().diffattn_fwd_save_size(ctypes.byref(a)))
+        if not save.is_cuda or save.numel() * save.element_size() < need or not save.is_contiguous():
+            raise ValueError(f"save must be a contiguous CUDA buffer of at least {need} bytes")
+        a.save = save.data_ptr()
     return a
 
 
@@ -235,7 +274,7 @@ def _check_shapes_fwd(q1, q2, k1, k2, v):
 
 def _run_fwd(entry, q1, q2, k1, k2, v, lam, gain, *, scale, eps, causal, apply_norm, out,
              workspace, stream, timeout_ms, dev_status, test_withhold_load=False,
-             lam_logits=None, gate=None, window=0, rope_theta=0.0):
+             lam_logits=None, gate=None, window=0, rope_theta=0.0, save=None):
     _check_shapes_fwd(q1, q2, k1, k2, v)
     B, N, H, _ = q1.shape
     if out is None:
@@ -243,7 +282,7 @@ def _run_fwd(entry, q1, q2, k1, k2, v, lam, gain, *, scale, eps, causal, apply_n
     a = _fwd_args(q1, q2, k1, k2, v, lam, gain, out, scale=scale, eps=eps, causal=causal,
                   apply_norm=apply_norm, timeout_ms=timeout_ms, dev_status=dev_status,
                   test_withhold_load=test_withhold_load, lam_logits=lam_logits, gate=gate,
-                  window=window, rope_theta=rope_theta)
+                  window=window, rope_theta=rope_theta, save=save)
     L = lib()
     need = L.diffattn_fwd_workspace_size(ctypes.byref(a))
     if workspace is None:
@@ -257,7 +296,7 @@ def _run_fwd(entry, q1, q2, k1, k2, v, lam, gain, *, scale, eps, causal, apply_n
 def diffattn_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,
                  apply_norm=True, out=None, workspace=None, stream=None, timeout_ms=0,
                  dev_status=None, test_withhold_load=False, lam_logits=None, gate=None,
-                 window=0, rope_theta=0.0):
+                 window=0, rope_theta=0.0, save=None):
     """Differential-attention prefill.  q1,q2,k1,k2 [B,N,H,64], v [B,N,H,128]
     bf16 CUDA tensors (token-major, last dim contiguous); lam [H] fp32 (or
     None with lam_logits); gain [H,128] fp32 or None; lam_logits: fp32
@@ -265,13 +304,15 @@ def diffattn_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, ca
     output-gate logits or None; window: 0, or a causal sliding window of that
     many keys; rope_theta: 0, or the base of the rotary embedding applied to
     Q1, K1, Q2, K2 by token position.  Returns out [B,N,H,128] bf16.
+    save: None, or a CUDA buffer of fwd_save_size(B, N, H) bytes that the
+    call also fills with the state diffattn_bwd needs.
     test_withhold_load sets the library's failure-path test hook (the call
     then reports a timeout in dev_status)."""
     return _run_fwd("diffattn_fwd", q1, q2, k1, k2, v, lam, gain, scale=scale, eps=eps,
                     causal=causal, apply_norm=apply_norm, out=out, workspace=workspace,
                     stream=stream, timeout_ms=timeout_ms, dev_status=dev_status,
                     test_withhold_load=test_withhold_load, lam_logits=lam_logits, gate=gate,
-                    window=window, rope_theta=rope_theta)
+                    window=window, rope_theta=rope_theta, save=save)
 
 
 def diffattn_grouped_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,
@@ -373,3 +414,116 @@ def diffattn_decode_noalloc(q1, q2, k1, k2, v, lam, gain=None, *, out, kv_len=No
     if st != 0:
         raise DiffAttnError(st, "diffattn_decode_noalloc")
     return out
+
+
+def fwd_save_size(B, N, H):
+    """Bytes of the state a prefill call with these sizes saves for diffattn_bwd."""
+    a = FwdArgs()
+    a.B, a.N, a.H, a.H_N, a.H_V, a.d, a.dv = B, N, H, H, H, 64, 128
+    return int(lib().diffattn_fwd_save_size(ctypes.byref(a)))
+
+
+def bwd_workspace_size(B, N, H):
+    """Workspace bytes of a diffattn_bwd call with these sizes."""
+    a = BwdArgs()
+    a.B, a.N, a.H, a.d, a.dv = B, N, H, 64, 128
+    return int(lib().diffattn_bwd_workspace_size(ctypes.byref(a)))
+
+
+def _bwd_args(q1, q2, k1, k2, v, lam, gain, dout, save, grads, *, scale, eps, causal, apply_norm,
+              timeout_ms, dev_status):
+    named = (("q1", q1), ("q2", q2), ("k1", k1), ("k2", k2), ("v", v), ("dout", dout),
+             ("grad_q1", grads["dq1"]), ("grad_q2", grads["dq2"]), ("grad_k1", grads["dk1"]),
+             ("grad_k2", grads["dk2"]), ("grad_v", grads["dv"]))
+    for n, t in named:
+        _check_bf16(n, t, 4)
+    B, N, H, d = q1.shape
+    for n, t in named:
+        if tuple(t.shape[:3]) != (B, N, H):
+            raise ValueError(f"{n} must be [B, N, H, *] with q1's B, N, H")
+    a = BwdArgs()
+    a.B, a.N, a.H, a.d, a.dv = B, N, H, d, v.shape[3]
+    a.scale, a.eps = float(scale), float(eps)
+    a.flags = (DIFFATTN_FLAG_CAUSAL if causal else 0) | (DIFFATTN_FLAG_APPLY_NORM if apply_norm else 0)
+    a.timeout_ms = int(timeout_ms)
+    for n, t in named:
+        setattr(a, n, t.data_ptr())
+        setattr(a, n + "_stride", _S3(*t.stride()[:3]))
+    if lam is None or lam.dtype != torch.float32 or lam.shape != (H,):
+        raise ValueError("lam must be float32 [H]")
+    a.lambda_ = lam.data_ptr()
+    if gain is not None:
+        if gain.dtype != torch.float32 or tuple(gain.shape) != (H, a.dv) or not gain.is_contiguous():
+            raise ValueError("gain must be contiguous float32 [H, dv]")
+        a.gain = gain.data_ptr()
+    if not save.is_cuda or not save.is_contiguous() or save.numel() * save.element_size() < fwd_save_size(B, N, H):
+        raise ValueError("save must be the buffer a diffattn_fwd call with these sizes filled")
+    a.save = save.data_ptr()
+    a.grad_lambda = grads["dlam"].data_ptr() if grads.get("dlam") is not None else None
+    a.grad_gain = grads["dgain"].data_ptr() if grads.get("dgain") is not None else None
+    a.dev_status = dev_status.data_ptr() if dev_status is not None else None
+    return a
+
+
+def diffattn_bwd(q1, q2, k1, k2, v, lam, gain, dout, save, *, scale=0.125, eps=1e-5, causal=True,
+                 apply_norm=True, grads=None, workspace=None, stream=None, timeout_ms=0,
+                 dev_status=None):
+    """Backward pass of diffattn_fwd: gradients of sum(dout * out).
+
+    Inputs as in the forward call that filled `save` (same scale, eps,
+    causal, apply_norm); dout [B,N,H,128] bf16.  Returns a dict: dq1, dq2,
+    dk1, dk2 [B,N,H,64] and dv [B,N,H,128] bf16; dlam [H] and dgain [H,128]
+    fp32.  grads: optional dict of preallocated outputs with those keys."""
+    B, N, H, d = q1.shape
+    dev = q1.device
+    if grads is None:
+        grads = {k: torch.empty(B, N, H, d, dtype=torch.bfloat16, device=dev)
+                 for k in ("dq1", "dq2", "dk1", "dk2")}
+        grads["dv"] = torch.empty(B, N, H, v.shape[3], dtype=torch.bfloat16, device=dev)
+        grads["dlam"] = torch.empty(H, dtype=torch.float32, device=dev)
+        grads["dgain"] = torch.empty(H, v.shape[3], dtype=torch.float32, device=dev)
+    a = _bwd_args(q1, q2, k1, k2, v, lam, gain, dout, save, grads, scale=scale, eps=eps,
+                  causal=causal, apply_norm=apply_norm, timeout_ms=timeout_ms,
+                  dev_status=dev_status)
+    L = lib()
+    need = L.diffattn_bwd_workspace_size(ctypes.byref(a))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    st = L.diffattn_bwd(ctypes.byref(a), _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    if st != 0:
+        raise DiffAttnError(st, "diffattn_bwd")
+    return grads
+
+
+class DiffAttention(torch.autograd.Function):
+    """Differential attention as an autograd function: the forward runs
+    diffattn_fwd with the saved state, the backward runs diffattn_bwd."""
+
+    @staticmethod
+    def forward(ctx, q1, q2, k1, k2, v, lam, gain, scale, eps, causal, apply_norm):
+        B, N, H, _ = q1.shape
+        save = torch.empty(max(fwd_save_size(B, N, H), 16), dtype=torch.uint8, device=q1.device)
+        out = diffattn_fwd(q1, q2, k1, k2, v, lam, gain, scale=scale, eps=eps, causal=causal,
+                           apply_norm=apply_norm, save=save)
+        ctx.save_for_backward(q1, q2, k1, k2, v, lam, gain, save)
+        ctx.cfg = (scale, eps, causal, apply_norm)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q1, q2, k1, k2, v, lam, gain, save = ctx.saved_tensors
+        scale, eps, causal, apply_norm = ctx.cfg
+        dout = dout.to(torch.bfloat16)
+        if dout.stride(-1) != 1:
+            dout = dout.contiguous()
+        g = diffattn_bwd(q1, q2, k1, k2, v, lam, gain, dout, save, scale=scale, eps=eps,
+                         causal=causal, apply_norm=apply_norm)
+        dgain = g["dgain"] if gain is not None else None
+        return g["dq1"], g["dq2"], g["dk1"], g["dk2"], g["dv"], g["dlam"], dgain, None, None, None, None
+
+
+def diff_attention(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,
+                   apply_norm=True):
+    """Differentiable differential attention (bf16 q/k/v [B,N,H,64|128], fp32
+    lam [H] and gain [H,128]); gradients flow to every tensor input."""
+    return DiffAttention.apply(q1, q2, k1, k2, v, lam, gain, scale, eps, causal, apply_norm)

@@ -116,6 +116,16 @@ typedef struct diffattn_fwd_args {
      * 0 = no rotation.  Decode has no rotation: it reads its cache as
      * stored.                                                               */
     float rope_theta;
+    /* State saved for diffattn_bwd: NULL, or device memory (16-byte aligned)
+     * of diffattn_fwd_save_size(args) bytes that the forward fills, besides
+     * `out`, with what the backward pass needs: per row and map the
+     * normalised map output A_t = softmax(scale Q_t K_t^T) V (fp32) and the
+     * base-2 log of the row's softmax denominator.  Its layout is private to
+     * the library; it stays valid until the caller reuses the memory.
+     * Supported for diffattn_fwd (H_N == H_V == H) with per-head lambda and
+     * no lambda_logits, gate, window or rope_theta; other combinations
+     * return DIFFATTN_ERR_UNSUPPORTED.                                       */
+    void *save;
 } diffattn_fwd_args;
 
 /* Causal (or full) prefill, one noise map per signal head: H_N and H_V must be
@@ -135,6 +145,64 @@ diffattn_status diffattn_grouped_fwd(const diffattn_fwd_args *args, void *worksp
  * depending on the arguments the grouped heads' noise outputs and the
  * rotated copies of Q1, K1, Q2, K2).                                        */
 size_t diffattn_fwd_workspace_size(const diffattn_fwd_args *args);
+
+/* Bytes of the `save` buffer a diffattn_fwd call with `args` fills (0 for
+ * an empty problem).                                                        */
+size_t diffattn_fwd_save_size(const diffattn_fwd_args *args);
+
+/* Backward pass of diffattn_fwd: the gradients of sum(dout * out) with
+ * respect to q1, q2, k1, k2, v, lambda and gain.  The pages define the
+ * forward pass only (Motif 2.6B explainer, section "Differential attention";
+ * the model is trained with it), so this is its exact gradient:
+ *
+ *   dgain = sum_i dY D r,  dD = r (dY gain) - (r^3 / dv) D sum_c(dY gain D)
+ *   dA_1 = dD, dA_2 = -lambda dD, dlambda = -sum dD A_2
+ *   per map: dP = dA_t V^T, dS = P (dP - rowsum(dA_t A_t)),
+ *            dQ_t = scale dS K_t, dK_t = scale dS^T Q_t, dV += P^T dA_t
+ *
+ * (r = (mean_c D^2 + eps)^-1/2; without DIFFATTN_FLAG_APPLY_NORM, dD = dY and
+ * dgain = 0).  Inputs are those of the forward call that filled `save`, with
+ * the same B, N, H, scale, eps and flags.  Layouts as in the forward:
+ *   q1, q2, k1, k2, grad_q1, grad_q2, grad_k1, grad_k2: [B, N, H, 64] bf16
+ *   v, dout, grad_v: [B, N, H, 128] bf16
+ *   lambda: [H] fp32 device; gain: [H, 128] fp32 device or NULL for 1.
+ *   grad_lambda: [H] fp32 device or NULL; grad_gain: [H, 128] fp32 device,
+ *   contiguous, or NULL.
+ * Every gradient is overwritten, not accumulated into.  Intermediate
+ * quantities beyond the fp16 range (the normalised-output gradient dD is
+ * staged in fp16 for the tensor cores) report DIFFATTN_ERR_UNSUPPORTED in
+ * dev_status.                                                               */
+typedef struct diffattn_bwd_args {
+    int64_t B, N, H;
+    int64_t d, dv;
+    float scale, eps;
+    uint32_t flags;         /* CAUSAL, APPLY_NORM: as in the forward call */
+    uint32_t timeout_ms;
+    const void *q1; int64_t q1_stride[3];
+    const void *q2; int64_t q2_stride[3];
+    const void *k1; int64_t k1_stride[3];
+    const void *k2; int64_t k2_stride[3];
+    const void *v;  int64_t v_stride[3];
+    const void *dout; int64_t dout_stride[3];
+    const void *save;       /* filled by the forward call */
+    const float *lambda;
+    const float *gain;
+    void *grad_q1; int64_t grad_q1_stride[3];
+    void *grad_q2; int64_t grad_q2_stride[3];
+    void *grad_k1; int64_t grad_k1_stride[3];
+    void *grad_k2; int64_t grad_k2_stride[3];
+    void *grad_v;  int64_t grad_v_stride[3];
+    float *grad_lambda;
+    float *grad_gain;
+    int32_t *dev_status;
+} diffattn_bwd_args;
+
+diffattn_status diffattn_bwd(const diffattn_bwd_args *args, void *workspace, size_t ws_bytes,
+                             void *stream);
+
+/* Workspace bytes of diffattn_bwd (fp16 copies of V and of dD, and per-row
+ * statistics).                                                              */
+size_t diffattn_bwd_workspace_size(const diffattn_bwd_args *args);
 
 /* Host-only argument check of a prefill call: the status diffattn_fwd (or,
  * with grouped != 0, diffattn_grouped_fwd) would return before launching,

@@ -247,3 +247,62 @@ def test_binding_rejects_cpu_tensor_types():
     x = torch.zeros(1, 4, 1, 64, dtype=torch.float32)
     with pytest.raises(TypeError):
         ops._check_bf16("q1", x, 4)
+
+
+def _fake_bwd_args(B=2, N=300, H=4, base=1 << 20):
+    a = ops.BwdArgs()
+    a.B, a.N, a.H, a.d, a.dv = B, N, H, 64, 128
+    a.scale, a.eps = 0.125, 1e-5
+    a.flags = ops.DIFFATTN_FLAG_CAUSAL | ops.DIFFATTN_FLAG_APPLY_NORM
+    for i, (n, w) in enumerate((("q1", 64), ("q2", 64), ("k1", 64), ("k2", 64), ("v", 128),
+                                ("dout", 128), ("grad_q1", 64), ("grad_q2", 64), ("grad_k1", 64),
+                                ("grad_k2", 64), ("grad_v", 128))):
+        setattr(a, n, base * (i + 1))
+        setattr(a, n + "_stride", ops._S3(N * H * w, H * w, w))
+    a.save, a.lambda_ = base * 20, base * 21
+    return a
+
+
+def test_bwd_rejects_before_launch(L):
+    """diffattn_bwd checks its arguments and workspace before any CUDA call.
+    (The empty-problem case zeroes dlambda / dgain on the device, so it is
+    left to the GPU tests.)"""
+    b = lambda a, ws=None, n=0: L.diffattn_bwd(ctypes.byref(a), ws, n, None)
+    a = _fake_bwd_args()
+    need = L.diffattn_bwd_workspace_size(ctypes.byref(a))
+    # fp16 copies of V and dD, then [B, H, 4, 3 tiles * 128] fp32 statistics, then 256 B
+    assert need == 2 * (2 * 300 * 4 * 128 * 2) + 2 * 4 * 4 * 384 * 4 + 256
+    assert b(a) == 4                                               # workspace missing
+    assert b(a, ctypes.c_void_p(1 << 30), need - 1) == 4
+    assert b(a, ctypes.c_void_p((1 << 30) + 16), need) == 3         # workspace not 256-aligned
+    for field, value, code in (("d", 32, 2), ("dv", 64, 2), ("save", 0, 1), ("dout", 0, 1),
+                               ("grad_v", 0, 1), ("lambda_", 0, 1), ("grad_k2", (1 << 20) + 8, 3),
+                               ("save", (1 << 20) + 4, 3), ("grad_gain", (1 << 20) + 2, 3),
+                               ("flags", 8, 1), ("scale", 0.0, 1)):
+        a = _fake_bwd_args()
+        setattr(a, field, value)
+        assert b(a, ctypes.c_void_p(1 << 30), need) == code, field
+    a = _fake_bwd_args()
+    a.dout_stride[1] = 130
+    assert b(a, ctypes.c_void_p(1 << 30), need) == 3                # stride not a multiple of 8
+
+
+def test_fwd_save_size_and_support(L):
+    a = _fake_fwd_args()
+    # per (b, h, 128-row tile): A_1, A_2 (2 x 128 x 128 fp32) and lse_1, lse_2 (2 x 128 fp32)
+    assert L.diffattn_fwd_save_size(ctypes.byref(a)) == 2 * 4 * 3 * (2 * 128 * 128 + 2 * 128) * 4
+    a.save = 1 << 28
+    assert _v(L, a) == 0
+    a.save = (1 << 28) + 8
+    assert _v(L, a) == 3                                           # 16-byte alignment
+    for field, value in (("window", 64), ("rope_theta", 1e4), ("gate", 1 << 27),
+                         ("lambda_logits", 1 << 27)):
+        a = _fake_fwd_args()
+        a.save = 1 << 28
+        setattr(a, field, value)
+        if field == "gate":
+            a.gate_stride = ops._S3(300 * 4 * 128, 4 * 128, 128)
+        assert _v(L, a) == 2, field                                # no saved state for these
+    g = _fake_fwd_args(H=24, H_N=8, H_V=8)
+    g.save = 1 << 28
+    assert _v(L, g, 1) == 2                                        # nor for grouped heads
