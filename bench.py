@@ -1,4 +1,4 @@
-"""Benchmark of the differential-attention forward pass on B200.
+"""Benchmark of differential attention on B200 (headline: the forward pass).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -18,8 +18,11 @@ kernel.  Rank 0 prints one JSON line:
 * extra        the other workloads at one pass each: long context (1 x 16384),
                grouped (24 signal / 8 noise heads), gated (the grouped shape
                with token-dependent lambda and output gate, no norm: Motif 3
-               summary, section 2.2), decode (batch 64, 8192
-               cached keys; GB/s against the measured HBM copy bandwidth).
+               summary, section 2.2), sliding window (1 x 16384, W = 128),
+               RoPE (the 4K shape, theta = 500,000), the backward pass of the
+               4K shape (1280 FLOP per pair; also the saving forward and a
+               training step of both), decode (batch 64, 8192 cached keys;
+               GB/s against the measured HBM copy bandwidth).
 
 With more than one GPU (torchrun) every rank runs its own batch of the same
 shape (weak scaling; the path has no exchange step) and the time is the max
@@ -85,7 +88,7 @@ def decode_bytes(w):
 # prefill_kernel launch on the 4 x 4096 x 16-head workload, from one ncu
 # capture, keyed by a hash of the kernel sources it was taken on.  A kernel
 # whose sources no longer hash to this value reports null traffic.
-PREFILL_TRAFFIC = {"source_sha256_16": "45f80504a5d26214", "bytes": 268_578_048 + 46_927_872}
+PREFILL_TRAFFIC = {"source_sha256_16": "3a8691558a24655b", "bytes": 268_728_320 + 45_776_128}
 
 
 def prefill_traffic():

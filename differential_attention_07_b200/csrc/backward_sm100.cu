@@ -2,8 +2,9 @@
 // prefill on B200 (sm_100a).
 //
 // The pages define the forward pass (Motif 2.6B explainer, section
-// "Differential attention", figure 1) and train the model with it; the
-// backward pass here is its exact gradient.  With A_t = P_t V the two map
+// "Differential attention", figure 1) and train the model with it (same
+// page, "A schedule for the data"); the backward pass here is its exact
+// gradient.  With A_t = P_t V the two map
 // outputs, D = A_1 - lambda A_2, r = (mean_c D^2 + eps)^-1/2, Y = D r gain:
 //
 //   dgain = sum_i dY D r                 dD = r (dY gain) - (r^3/128) D sum_c(dY gain D)

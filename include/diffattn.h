@@ -153,7 +153,8 @@ size_t diffattn_fwd_save_size(const diffattn_fwd_args *args);
 /* Backward pass of diffattn_fwd: the gradients of sum(dout * out) with
  * respect to q1, q2, k1, k2, v, lambda and gain.  The pages define the
  * forward pass only (Motif 2.6B explainer, section "Differential attention";
- * the model is trained with it), so this is its exact gradient:
+ * the model is trained with it, same page, "A schedule for the data"), so
+ * this is its exact gradient:
  *
  *   dgain = sum_i dY D r,  dD = r (dY gain) - (r^3 / dv) D sum_c(dY gain D)
  *   dA_1 = dD, dA_2 = -lambda dD, dlambda = -sum dD A_2

@@ -6,8 +6,9 @@ shares no code with the CUDA path.
 
 The pages give the forward pass only (Motif 2.6B explainer, section
 "Differential attention" and figure 1; Motif 3 summary, section 2.2, for the
-grouped head map); they use it for training, so the backward pass is the
-gradient of that forward pass, nothing more.  This module writes the chain
+grouped head map); the model is trained with it (Motif 2.6B explainer,
+section "A schedule for the data"), so the backward pass is the gradient of
+that forward pass, nothing more.  This module writes the chain
 rule out step by step, per batch entry and signal head, on whole N x N
 matrices (NumPy matmuls are the only library steps):
 
