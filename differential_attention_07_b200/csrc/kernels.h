@@ -108,8 +108,9 @@ struct BwdParams {
 };
 
 // Tensor maps of the key-tile kernel (dK_1, dK_2, dV): K_1, K_2 and the fp16
-// V copy in 128-row boxes; Q_1, Q_2 and dD in 64-row boxes; the statistics
-// (fp32, no swizzle) in {64, 4} boxes.  All 128-byte swizzled, {64, rows}.
+// V copy in 128-row boxes; Q_1, Q_2 and dD in 64-row boxes (all 128-byte
+// swizzled, {64 columns, rows} boxes); the statistics in {64 rows, 4 arrays}
+// boxes of fp32, not swizzled.
 struct BwdKeyMaps {
     CUtensorMap k1, k2, v, q1, q2, dd, stats;
 };
