@@ -186,6 +186,7 @@ int diffattn_oracle_prefill(const double *q1, const double *q2, const double *k1
 {
     if (B < 0 || N < 0 || H <= 0 || H_N <= 0 || H_V <= 0 || d <= 0 || dv <= 0) return -1;
     if (window < 0 || (window > 0 && !causal) || rope_theta < 0 || (rope_theta > 0 && d % 2)) return -1;
+    if (H % H_N != 0 || H % H_V != 0) return -1;  /* before anything is allocated */
     double *rq1 = NULL, *rq2 = NULL, *rk1 = NULL, *rk2 = NULL;
     if (rope_theta > 0) {  /* step 0 */
         rq1 = rope_copy(q1, B, N, H, d, rope_theta);
@@ -198,7 +199,6 @@ int diffattn_oracle_prefill(const double *q1, const double *q2, const double *k1
         }
         q1 = rq1; k1 = rk1; q2 = rq2; k2 = rk2;
     }
-    if (H % H_N != 0 || H % H_V != 0) return -1;
     const int64_t g = H / H_N;       /* signal heads per noise head */
     const int64_t gv = H / H_V;      /* signal heads per V head */
     const int64_t total = rows ? nrows : B * N * H;
