@@ -2,38 +2,52 @@
 // prefill on B200 (sm_100a).
 //
 // The pages define the forward pass (Motif 2.6B explainer, section
-// "Differential attention", figure 1) and train the model with it (same
-// page, "A schedule for the data"); the backward pass here is its exact
-// gradient.  With A_t = P_t V the two map
-// outputs, D = A_1 - lambda A_2, r = (mean_c D^2 + eps)^-1/2, Y = D r gain:
+// "Differential attention", figure 1; Motif 3 summary, section 2.2, for the
+// grouped heads, the token-dependent lambda and the output gate, section 2.1
+// for sliding-window layers; Motif 2.6B explainer, "The block", for the
+// rotary embedding) and train the model with it (Motif 2.6B explainer, "A
+// schedule for the data"); the backward pass here is its exact gradient.
+// With A_t = P_t V the two map outputs, lambda_i the row's lambda (per head,
+// or sigma of the token's logit), D = A_1 - lambda_i A_2,
+// r = (mean_c D^2 + eps)^-1/2, Yn = D r gain, Y = sigma(G) Yn:
 //
-//   dgain = sum_i dY D r                 dD = r (dY gain) - (r^3/128) D sum_c(dY gain D)
-//   dA_1 = dD, dA_2 = -lambda dD         dlambda = -sum dD A_2
-//   per map t: dP_t = dA_t V^T = (1, -lambda) x dP with dP = dD V^T (one product)
+//   dYn = dY sigma(G),  dG = dY Yn sigma'(G)           (gate; else dYn = dY)
+//   dgain = sum_i dYn D r,  dD = r (dYn gain) - (r^3/128) D sum_c(dYn gain D)
+//   dA_1 = dD, dA_2 = -lambda_i dD,  dlambda_i = -sum_c dD A_2
+//   per map t: dP_t = dA_t V^T = (1, -lambda_i) x dP with dP = dD V^T (one product)
 //              Delta_t = rowsum(dA_t A_t), dS_t = P_t (dP_t - Delta_t)
 //              dQ_t = scale dS_t K_t, dK_t = scale dS_t^T Q_t
 //   dV = P_1^T dA_1 + P_2^T dA_2 = (P_1 - lambda P_2)^T dD (one product)
 //
-// Three kernels after the fp16 staging of V (the forward's staging kernel):
+// (with the rotary embedding the products run on the rotated Q/K, and dQ,
+// dK are rotated back).  After the staging pass (fp16 V, rotated Q/K),
+// three or four kernels:
 //  1. bwd_prep_kernel, one thread per row: reads the forward's saved A_1, A_2
-//     and lse, and dY; writes dD (fp16, the tensor-core operand), the row
-//     statistics (lse_1, lse_2, Delta_1, Delta_2), and adds into dlambda and
+//     and lse, dY and the gate logits; writes dD (fp16, the tensor-core
+//     operand), the row statistics (lse_1, lse_2, Delta_1, Delta_2, lambda),
+//     the gate's and the lambda logits' gradients, and adds into dlambda and
 //     dgain.
 //  2. bwd_key_kernel, one CTA per (b, h, 128-key tile), keys on the 128 TMEM
-//     lanes: loops over 64-query blocks; per block three tcgen05 products
-//     into TMEM (S_1^T = K_1 Q_1^T, S_2^T = K_2 Q_2^T, dP^T = V dD^T), the
-//     element-wise step in registers (P_t from the saved lse, the dV operand
-//     P_1 - lambda P_2 in fp16, dS_1, dS_2 in bf16, written back to TMEM),
-//     then three accumulating products with A from TMEM (dV += (P_1 -
-//     lambda P_2)^T dD, dK_t += dS_t^T Q_t).
-//  3. bwd_query_kernel, one CTA per (b, h, 128-query tile), queries on the
-//     lanes: loops over 64-key blocks; S_1, S_2, dP = dD V^T, the element-wise
-//     step, dQ_t += dS_t K_t.
-// Both loops double-buffer their block loads (TMA) against the element-wise
-// step; the tensor core and the CUDA cores take turns within a CTA (no warp
-// specialisation), so the speed comes from one CTA per SM over many CTAs.
+//     lanes, over the 64-query blocks that see them.  Warp-specialised:
+//     warp 0 loads (TMA), warp 1 issues the tcgen05 products, warps 2-9
+//     (two warpgroups, 32 queries of each block apiece) run the element-wise
+//     step.  Per block: S_1^T = K_1 Q_1^T, S_2^T = K_2 Q_2^T, dP^T = V dD^T
+//     into TMEM; the element-wise warps load them to registers and release
+//     the TMEM at once, so the next block's products run during this
+//     block's element-wise step; they write P_1 - lambda P_2 (fp16) and
+//     dS_1, dS_2 to shared memory as the A operands of dV += (P_1 - lambda
+//     P_2)^T dD and dK_t += dS_t^T Q_t.
+//  3. bwd_query_kernel, the same shape per (b, h, 128-query tile) over
+//     64-key blocks: S_1, S_2, dP = dD V^T, the element-wise step, dQ_t +=
+//     dS_t K_t.
+//  4. bwd_convert_kernel, only when noise or V heads are shared by several
+//     signal heads: their gradients are summed in fp32 (vector atomics from
+//     the tile kernels) and converted to bf16 here.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+
+#include <atomic>
+#include <mutex>
 
 #include "kernels.h"
 #include "sm100_ptx.cuh"
@@ -41,48 +55,68 @@
 namespace da {
 namespace {
 
-constexpr int BT = 128;   // rows of a tile: MMA M, one per TMEM lane / thread
+constexpr int BT = 128;   // rows of a tile: MMA M, one per TMEM lane
 constexpr int BB = 64;    // rows of a block: MMA N of the score products
 constexpr int HD = 64;    // Q/K head dim
 constexpr int HDV = 128;  // V head dim
-constexpr int NT = 128;   // threads per CTA of the tile kernels
-constexpr int NBARS = 5;  // tile, full[2], S, M
+constexpr int NT = 320;   // 10 warps: producer, MMA issuer, two element-wise warpgroups
+constexpr int NEW = 8;    // element-wise warps
+
+// mbarriers of both tile kernels.
+enum : int {
+    B_TILE = 0,   // the tile's operands landed (TMA bytes)
+    B_FULL = 1,   // [2] a block's operands landed (TMA bytes)
+    B_EMPTY = 3,  // [2] the block's last products have read its stage (commit)
+    B_SFULL = 5,  // the block's score and dP products are in TMEM (commit)
+    B_SFREE = 6,  // the element-wise warps loaded them (8 arrivals)
+    B_AFULL = 7,  // the element-wise warps wrote the A operands (8 arrivals)
+    B_AFREE = 8,  // the accumulating products have read the A operands (commit)
+    B_DONE = 9,   // every product of the CTA has completed (commit)
+    NBARS = 10
+};
 
 // ---------------------------------------------------------------- key-tile kernel
-// Shared memory: the tile's K_1, K_2 (bf16 [128][64]) and V (fp16 [128][128]
-// as two [128][64] column halves), then two block buffers of Q_1, Q_2 (bf16
-// [64][64]), dD (fp16 [64][128] as two halves) and the statistics [4][64].
-constexpr uint32_t KT_K1 = 0, KT_K2 = 16384, KT_V = 32768, KT_BUF = 65536;
-constexpr uint32_t KB_Q1 = 0, KB_Q2 = 8192, KB_DD = 16384, KB_ST = 32768, KB_BYTES = 33792;
-constexpr uint32_t KT_BARS = KT_BUF + 2 * KB_BYTES;
-constexpr uint32_t KT_SMEM = KT_BARS + 8 * NBARS + 8;
-// TMEM columns: dV accumulator, dK_1, dK_2, then S_1^T, S_2^T, dP^T.  The
-// element-wise step writes the dV operand over the first half of S_1^T, dS_1
-// over the first half of S_2^T and dS_2 over the first half of dP^T.
+// Shared memory: the tile's K_1, K_2 ([128][64]) and fp16 V ([128][128] as
+// two [128][64] column halves); two block stages of Q_1, Q_2 ([64][64]), dD
+// (fp16 [64][128] as two halves) and the statistics [kBwdStats][64] fp32;
+// the A operands P_1 - lambda P_2, dS_1, dS_2 ([128 keys][64 queries]).
+constexpr uint32_t KT_K1 = 0, KT_K2 = 16384, KT_V = 32768, KT_STAGE0 = 65536;
+constexpr uint32_t KB_Q1 = 0, KB_Q2 = 8192, KB_DD = 16384, KB_ST = 32768;
+constexpr uint32_t KB_LOAD = KB_ST + kBwdStats * BB * 4;  // bytes a stage receives
+constexpr uint32_t KB_BYTES = (KB_LOAD + 1023) & ~1023u;   // stages stay 1 KB aligned
+constexpr uint32_t KT_A = KT_STAGE0 + 2 * KB_BYTES;
+constexpr uint32_t KA_PV = 0, KA_DS1 = 16384, KA_DS2 = 32768;
+constexpr uint32_t KT_BARS = KT_A + 3 * 16384;
+constexpr uint32_t KT_SMEM = KT_BARS + 8 * NBARS + 16;
+// TMEM columns: dV, dK_1, dK_2 accumulators, then S_1^T, S_2^T, dP^T.
 constexpr uint32_t KM_DV = 0, KM_DK1 = 128, KM_DK2 = 192, KM_S1 = 256, KM_S2 = 320, KM_DP = 384;
 
 // ---------------------------------------------------------------- query-tile kernel
-// Shared memory: the tile's Q_1, Q_2 (bf16 [128][64]) and dD (fp16 [128][128]
-// as two halves), then two block buffers of K_1, K_2 (bf16 [64][64]) and V
-// (fp16 [64][128] as two halves).
-constexpr uint32_t QT_Q1 = 0, QT_Q2 = 16384, QT_DD = 32768, QT_BUF = 65536;
+// Shared memory: the tile's Q_1, Q_2 ([128][64]) and dD (fp16 [128][128] as
+// two halves); two block stages of K_1, K_2 ([64][64]) and fp16 V ([64][128]
+// as two halves); the A operands dS_1, dS_2 ([128 queries][64 keys]).
+constexpr uint32_t QT_Q1 = 0, QT_Q2 = 16384, QT_DD = 32768, QT_STAGE0 = 65536;
 constexpr uint32_t QB_K1 = 0, QB_K2 = 8192, QB_V = 16384, QB_BYTES = 32768;
-constexpr uint32_t QT_BARS = QT_BUF + 2 * QB_BYTES;
-constexpr uint32_t QT_SMEM = QT_BARS + 8 * NBARS + 8;
-// TMEM columns: dQ_1, dQ_2, then S_1, S_2, dP; dS_1 goes over the first half
-// of S_1 and dS_2 over the first half of S_2.
+constexpr uint32_t QT_A = QT_STAGE0 + 2 * QB_BYTES;
+constexpr uint32_t QA_DS1 = 0, QA_DS2 = 16384;
+constexpr uint32_t QT_BARS = QT_A + 2 * 16384;
+constexpr uint32_t QT_SMEM = QT_BARS + 8 * NBARS + 16;
+// TMEM columns: dQ_1, dQ_2 accumulators, then S_1, S_2, dP.
 constexpr uint32_t QM_DQ1 = 0, QM_DQ2 = 64, QM_S1 = 128, QM_S2 = 192, QM_DP = 256;
 
-// Both tile kernels use more than half an SM's shared memory, so one CTA per
-// SM holds the 512 TMEM columns it allocates.
-static_assert(KT_SMEM > 116 * 1024 && KT_SMEM <= 227 * 1024, "key-tile kernel: one CTA per SM");
-static_assert(QT_SMEM > 116 * 1024 && QT_SMEM <= 227 * 1024, "query-tile kernel: one CTA per SM");
+static_assert(KT_SMEM <= 232448 && QT_SMEM <= 232448, "shared memory budget");
+static_assert(KT_A % 1024 == 0 && QT_A % 1024 == 0 && KB_BYTES % 1024 == 0, "SW128 tiles are 1 KB aligned");
+static_assert(KT_SMEM > 116 * 1024 && QT_SMEM > 116 * 1024, "one CTA per SM owns the 512 TMEM columns");
 
-// Instruction descriptors (fp32 accumulate).
-constexpr uint32_t ID_S = idesc_f16(1, 1, 0, BT, BB);     // bf16 x bf16, both K-major
-constexpr uint32_t ID_DP = idesc_f16(0, 0, 0, BT, BB);    // fp16 x fp16, both K-major
-constexpr uint32_t ID_DV = idesc_f16(0, 0, 1, BT, HDV);   // fp16 (TMEM) x fp16, B MN-major
-constexpr uint32_t ID_ACC64 = idesc_f16(1, 1, 1, BT, HD); // bf16 (TMEM) x bf16, B MN-major
+// Instruction descriptors (fp32 accumulate).  F16QK: Q/K are the rotated
+// fp16 copies (and dS is fp16 to match them in the dQ / dK products).
+template <bool F16QK>
+struct Ids {
+    static constexpr uint32_t S = F16QK ? idesc_f16(0, 0, 0, BT, BB) : idesc_f16(1, 1, 0, BT, BB);
+    static constexpr uint32_t DS = F16QK ? idesc_f16(0, 0, 1, BT, HD) : idesc_f16(1, 1, 1, BT, HD);
+};
+constexpr uint32_t ID_DP = idesc_f16(0, 0, 0, BT, BB);   // fp16 x fp16, both K-major
+constexpr uint32_t ID_DV = idesc_f16(0, 0, 1, BT, HDV);  // fp16 A (K-major) x fp16 B (MN-major)
 
 // Descriptor of a 128-byte-swizzled operand tile (rows of 128 bytes, 8-row
 // atoms of 1 KB); `lbo` is the byte distance between 64-element column
@@ -93,34 +127,82 @@ __device__ __forceinline__ uint64_t sw128(uint32_t addr, uint32_t lbo = 16)
 }
 
 // One elected lane of a fully active warp issues; the warp stays converged.
-struct Issuer {
-    __device__ __forceinline__ void ss(uint32_t d, uint64_t a, uint64_t b, uint32_t id, bool acc) const
-    {
-        if (elect_one()) mma_ss(d, a, b, id, acc ? 1u : 0u);
-        __syncwarp();
-    }
-    __device__ __forceinline__ void ts(uint32_t d, uint32_t a, uint64_t b, uint32_t id, bool acc) const
-    {
-        if (elect_one()) mma_ts(d, a, b, id, acc ? 1u : 0u);
-        __syncwarp();
-    }
-    __device__ __forceinline__ void commit(uint32_t bar) const
-    {
-        if (elect_one()) mma_commit(bar);
-        __syncwarp();
-    }
-};
-
-// Store 2 x 32 fp32 values (scaled) of one row as bf16 to `dst` (16-byte aligned).
-__device__ __forceinline__ void store_row_bf16(__nv_bfloat16 *dst, const uint32_t (&v)[32], float s)
+__device__ __forceinline__ void mma_issue(uint32_t d, uint64_t a, uint64_t b, uint32_t id, bool acc)
 {
+    if (elect_one()) mma_ss(d, a, b, id, acc ? 1u : 0u);
+    __syncwarp();
+}
+__device__ __forceinline__ void commit_to(uint32_t bar)
+{
+    if (elect_one()) mma_commit(bar);
+    __syncwarp();
+}
+
+__device__ __forceinline__ uint32_t pack_ds(float lo, float hi, bool f16)
+{
+    return f16 ? pack_half2(lo, hi) : pack_bf162(lo, hi);
+}
+
+// Row r's 32-column half `half` of a [128 rows][64 columns] 16-bit operand
+// tile in the 128-byte swizzle (16-byte chunk c of row r at c ^ (r % 8)).
+__device__ __forceinline__ void st_operand_half(uint32_t tile, int r, int half, const uint32_t (&w)[16])
+{
+    const uint32_t row = tile + 128u * r;
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        st_shared_v4(row + ((((4 * half + c) ^ (r & 7)) & 7) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2],
+                     w[4 * c + 3]);
+}
+
+// The inverse rotary rotation of one 64-wide row at token position `pos`:
+// the pair (x[2c], x[2c+1]) turned back by pos * theta^(-2c/64).  The angle
+// is reduced to a fraction of a turn in double precision (pos up to 2^24).
+__device__ __forceinline__ void unrotate64(float (&x)[64], int pos, const double *g)
+{
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        const double turns = (double)pos * g[c];
+        const float frac = (float)(turns - rint(turns));
+        float sn, cs;
+        __sincosf(6.283185307179586f * frac, &sn, &cs);
+        const float a = x[2 * c], b = x[2 * c + 1];
+        x[2 * c] = a * cs + b * sn;
+        x[2 * c + 1] = b * cs - a * sn;
+    }
+}
+
+// Write one row of `cols` values (scaled by s) to a bf16 row (16-byte
+// aligned), or add it to an fp32 row of sums with vector atomics.
+template <int COLS>
+__device__ __forceinline__ void put_row(const float *x, float s, __nv_bfloat16 *dst, float *acc)
+{
+    if (acc) {
+#pragma unroll
+        for (int i = 0; i < COLS; i += 4)
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(acc + i), "f"(x[i] * s),
+                         "f"(x[i + 1] * s), "f"(x[i + 2] * s), "f"(x[i + 3] * s)
+                         : "memory");
+        return;
+    }
     uint4 *d4 = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-        d4[i] = make_uint4(pack_bf162(__uint_as_float(v[8 * i]) * s, __uint_as_float(v[8 * i + 1]) * s),
-                           pack_bf162(__uint_as_float(v[8 * i + 2]) * s, __uint_as_float(v[8 * i + 3]) * s),
-                           pack_bf162(__uint_as_float(v[8 * i + 4]) * s, __uint_as_float(v[8 * i + 5]) * s),
-                           pack_bf162(__uint_as_float(v[8 * i + 6]) * s, __uint_as_float(v[8 * i + 7]) * s));
+    for (int i = 0; i < COLS / 8; ++i)
+        d4[i] = make_uint4(pack_bf162(x[8 * i] * s, x[8 * i + 1] * s), pack_bf162(x[8 * i + 2] * s, x[8 * i + 3] * s),
+                           pack_bf162(x[8 * i + 4] * s, x[8 * i + 5] * s), pack_bf162(x[8 * i + 6] * s, x[8 * i + 7] * s));
+}
+
+// Load 64 fp32 TMEM columns of this warp's lanes into x.
+__device__ __forceinline__ void tmem_row64(uint32_t taddr, float (&x)[64])
+{
+    uint32_t v[2][32];
+    tmem_ld32(taddr, v[0]);
+    tmem_ld32(taddr + 32, v[1]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        x[i] = __uint_as_float(v[0][i]);
+        x[32 + i] = __uint_as_float(v[1][i]);
+    }
 }
 
 // ---------------------------------------------------------------- 1. row preparation
@@ -136,32 +218,53 @@ __global__ void __launch_bounds__(128)
     const int qt = blockIdx.x % p.num_qt, h = (blockIdx.x / p.num_qt) % p.H, b = blockIdx.x / (p.num_qt * p.H);
     const int r = threadIdx.x, row = qt * BT + r;
     const bool valid = row < p.N;
+    const int rowc = valid ? row : 0;
     const float *tile = p.save + ((size_t)(b * p.H + h) * p.num_qt + qt) * kSaveTileFloats;
     const float4 *a1p = reinterpret_cast<const float4 *>(tile) + r;   // chunk c at c * 128
     const float4 *a2p = a1p + 32 * BT;
-    const float lam = p.lambda[h];
+    const float ll = p.lam_logits ? p.lam_logits[b * p.ll_sb + (int64_t)rowc * p.ll_sn + h * p.ll_sh] : 0.0f;
+    const float lam = p.lam_logits ? logistic_fast(ll) : p.lambda[h];
     const float4 *g4p = p.gain ? reinterpret_cast<const float4 *>(p.gain + (size_t)h * HDV) : nullptr;
     const __nv_bfloat16 *dy = static_cast<const __nv_bfloat16 *>(p.dout) + (size_t)b * p.do_sb +
-                              (size_t)(valid ? row : 0) * p.do_sn + (size_t)h * p.do_sh;
+                              (size_t)rowc * p.do_sn + (size_t)h * p.do_sh;
+    const __nv_bfloat16 *gl = p.gate ? static_cast<const __nv_bfloat16 *>(p.gate) + (size_t)b * p.gate_sb +
+                                           (size_t)rowc * p.gate_sn + (size_t)h * p.gate_sh
+                                     : nullptr;
     const bool want_dgain = p.apply_norm && p.dgain;
 
-    auto load_dy4 = [&](int c, float (&y)[4]) {
-        const uint2 u = *reinterpret_cast<const uint2 *>(dy + 4 * c);
+    auto load4 = [](const __nv_bfloat16 *src, int c, float (&y)[4]) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(src + 4 * c);
         y[0] = __uint_as_float(u.x << 16);
         y[1] = __uint_as_float(u.x & 0xffff0000u);
         y[2] = __uint_as_float(u.y << 16);
         y[3] = __uint_as_float(u.y & 0xffff0000u);
     };
     auto gain4 = [&](int c) { return g4p ? __ldg(g4p + c) : make_float4(1.f, 1.f, 1.f, 1.f); };
+    // dYn = dY sigma(G) (the gate is the forward's last step), and sigma(G)
+    auto dyn4 = [&](int c, float (&y)[4], float (&sg)[4]) {
+        load4(dy, c, y);
+        if (gl) {
+            float g[4];
+            load4(gl, c, g);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                sg[e] = logistic_fast(g[e]);
+                y[e] *= sg[e];
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sg[e] = 1.0f;
+        }
+    };
 
-    // Pass 1: sum of squares of D and sum_c dY gain D.
+    // Pass 1: sum of squares of D and sum_c dYn gain D.
     float ss = 0.f, tg = 0.f;
     if (valid && p.apply_norm) {
 #pragma unroll 4
         for (int c = 0; c < 32; ++c) {
             const float4 a1 = a1p[c * BT], a2 = a2p[c * BT], g = gain4(c);
-            float y[4];
-            load_dy4(c, y);
+            float y[4], sg[4];
+            dyn4(c, y, sg);
             const float d[4] = {fmaf(-lam, a2.x, a1.x), fmaf(-lam, a2.y, a1.y), fmaf(-lam, a2.z, a1.z),
                                 fmaf(-lam, a2.w, a1.w)};
             const float gg[4] = {g.x, g.y, g.z, g.w};
@@ -175,29 +278,46 @@ __global__ void __launch_bounds__(128)
     const float rn = p.apply_norm ? 1.0f / sqrtf(ss * (1.0f / HDV) + p.eps) : 1.0f;
     const float coef = rn * rn * rn * (1.0f / HDV) * tg;
 
-    // Pass 2: dD, Delta_1 = dD . A_1, dD . A_2, the dgain terms.
-    float delta1 = 0.f, dot2 = 0.f;
+    // Pass 2: dD, Delta_1 = dD . A_1, Delta_2 = -lambda dD . A_2, dlambda =
+    // -dD . A_2, the dgain terms, dG.  The Deltas take dD as rounded to
+    // fp16, the operand the tile kernels' dP = dD V^T products see: then
+    // dS = P (dP - Delta) sums to zero over a row to fp32 rounding, and a
+    // row whose softmax is constant (one visible key) gets dS = 0 (exact
+    // in the gradient).  dlambda takes dD itself.
+    float delta1 = 0.f, dot2 = 0.f, dot2h = 0.f;
     bool bad = false;
-    __half *ddrow = static_cast<__half *>(p.dd) + (((size_t)b * p.N + (valid ? row : 0)) * p.H + h) * HDV;
-#pragma unroll 4
+    __half *ddrow = static_cast<__half *>(p.dd) + (((size_t)b * p.N + rowc) * p.H + h) * HDV;
+    __nv_bfloat16 *dgrow = p.dgate ? static_cast<__nv_bfloat16 *>(p.dgate) + (size_t)b * p.dg_sb +
+                                         (size_t)rowc * p.dg_sn + (size_t)h * p.dg_sh
+                                   : nullptr;
+#pragma unroll 2
     for (int c = 0; c < 32; ++c) {
         float dd[4] = {0.f, 0.f, 0.f, 0.f}, gt[4] = {0.f, 0.f, 0.f, 0.f};
         if (valid) {
             const float4 a1 = a1p[c * BT], a2 = a2p[c * BT], g = gain4(c);
-            float y[4];
-            load_dy4(c, y);
+            float y[4], sg[4];
+            dyn4(c, y, sg);
             const float av1[4] = {a1.x, a1.y, a1.z, a1.w}, av2[4] = {a2.x, a2.y, a2.z, a2.w};
             const float gg[4] = {g.x, g.y, g.z, g.w};
+            float dgv[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float d = fmaf(-lam, av2[e], av1[e]);
                 dd[e] = p.apply_norm ? fmaf(rn * gg[e], y[e], -coef * d) : y[e];
-                delta1 = fmaf(dd[e], av1[e], delta1);
+                const float ddh = __half2float(__float2half_rn(dd[e]));
+                delta1 = fmaf(ddh, av1[e], delta1);
+                dot2h = fmaf(ddh, av2[e], dot2h);
                 dot2 = fmaf(dd[e], av2[e], dot2);
                 gt[e] = y[e] * d * rn;
                 bad |= !(fabsf(dd[e]) <= 65504.0f);
+                // dG = dY Yn sigma'(G) = dYn Yn (1 - sigma(G)), Yn = D r gain (or D)
+                const float yn = p.apply_norm ? d * rn * gg[e] : d;
+                dgv[e] = y[e] * yn * (1.0f - sg[e]);
             }
             *reinterpret_cast<uint2 *>(ddrow + 4 * c) = make_uint2(pack_half2(dd[0], dd[1]), pack_half2(dd[2], dd[3]));
+            if (dgrow)
+                *reinterpret_cast<uint2 *>(dgrow + 4 * c) =
+                    make_uint2(pack_bf162(dgv[0], dgv[1]), pack_bf162(dgv[2], dgv[3]));
         }
         if (want_dgain) {
 #pragma unroll
@@ -206,23 +326,30 @@ __global__ void __launch_bounds__(128)
     }
     if (bad) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
 
-    // Row statistics; rows past N get zeros (the tile kernels mask them).
-    float *st = p.stats + (size_t)(b * p.H + h) * 4 * p.n_pad + row;
+    // Row statistics; rows past N get zeros (the tile kernels' products see
+    // zero operands there).
+    float *st = p.stats + (size_t)(b * p.H + h) * kBwdStats * p.n_pad + row;
     const float *lse = tile + 2 * BT * HDV;
     st[0] = valid ? lse[r] : 0.f;
     st[p.n_pad] = valid ? lse[BT + r] : 0.f;
     st[2 * p.n_pad] = delta1;
-    st[3 * p.n_pad] = -lam * dot2;
+    st[3 * p.n_pad] = -lam * dot2h;
+    st[4 * p.n_pad] = valid ? lam : 0.f;
 
-    // dlambda += -sum dD . A_2 over the tile's rows.
-    if (p.dlambda) {
+    // dlambda_i = -dD . A_2: per token through sigma' with lambda logits,
+    // else summed over the tile's rows into the head's dlambda.
+    if (p.lam_logits) {
+        if (p.dlam_logits && valid)
+            p.dlam_logits[b * p.dll_sb + (int64_t)row * p.dll_sn + h * p.dll_sh] = -dot2 * lam * (1.0f - lam);
+    } else if (p.dlambda) {
         float v = -dot2;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         if ((r & 31) == 0) warp_sum[r >> 5] = v;
     }
     __syncthreads();
-    if (p.dlambda && r == 0) atomicAdd(p.dlambda + h, warp_sum[0] + warp_sum[1] + warp_sum[2] + warp_sum[3]);
+    if (!p.lam_logits && p.dlambda && r == 0)
+        atomicAdd(p.dlambda + h, warp_sum[0] + warp_sum[1] + warp_sum[2] + warp_sum[3]);
     // dgain[h][c] += sum over the tile's rows (thread r sums column r).
     if (want_dgain) {
         float v = 0.f;
@@ -232,13 +359,25 @@ __global__ void __launch_bounds__(128)
     }
 }
 
+// Roles shared by both tile kernels.
+struct Roles {
+    int warp, lane;
+    __device__ __forceinline__ bool producer() const { return warp == 0; }
+    __device__ __forceinline__ bool issuer() const { return warp == 1; }
+    // element-wise warpgroup (0 or 1) and the TMEM lane / tile row of this thread
+    __device__ __forceinline__ int wg() const { return (warp - 2) >> 2; }
+    __device__ __forceinline__ int row() const { return (warp & 3) * 32 + lane; }
+    __device__ __forceinline__ uint32_t lane_off() const { return uint32_t((warp & 3) * 32) << 16; }
+};
+
 // ---------------------------------------------------------------- 2. key tiles
+template <bool F16QK>
 __global__ void __launch_bounds__(NT, 1)
     bwd_key_kernel(const __grid_constant__ BwdKeyMaps m, const BwdParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_addr(smem);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Roles R{(int)(threadIdx.x >> 5), (int)(threadIdx.x & 31)};
     if (sbase & 1023u) {  // the 128-byte-swizzled tiles need 1 KB alignment
         if (threadIdx.x == 0) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
         return;
@@ -246,22 +385,34 @@ __global__ void __launch_bounds__(NT, 1)
     // Heavy tiles first: under the causal mask key tile 0 meets every query.
     const int BH = p.B * p.H;
     const int kt = blockIdx.x / BH, bh = blockIdx.x % BH, b = bh / p.H, h = bh % p.H;
+    const int hn = h / (p.H / p.H_N), hv = h / (p.H / p.H_V);
     const int k0 = kt * BT;
-    const int nqb = (p.N + BB - 1) / BB;
+    // Query blocks that see a key of the tile: causal from the block holding
+    // k0; under a window of W keys up to the one holding k0 + 127 + W - 1.
+    const int nqb_all = (p.N + BB - 1) / BB;
     const int qb0 = p.causal ? k0 / BB : 0;
-    const int nit = nqb - qb0;  // >= 1: k0 < N
+    const int qb1 = p.window > 0 ? min(nqb_all, (k0 + BT - 1 + p.window - 1) / BB + 1) : nqb_all;
+    const int nit = qb1 - qb0;  // >= 1: k0 < N
     auto bar = [&](int i) { return sbase + KT_BARS + 8 * i; };
-    enum { B_TILE = 0, B_FULL = 1, B_S = 3, B_M = 4 };
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + KT_BARS + 8 * NBARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + KT_BARS + 8 * NBARS + 4);
     const uint64_t lim = p.timeout_ns;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), 1);
+        mbar_init(bar(B_TILE), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(B_FULL + s), 1);
+            mbar_init(bar(B_EMPTY + s), 1);
+        }
+        mbar_init(bar(B_SFULL), 1);
+        mbar_init(bar(B_SFREE), NEW);
+        mbar_init(bar(B_AFULL), NEW);
+        mbar_init(bar(B_AFREE), 1);
+        mbar_init(bar(B_DONE), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0) {
+    if (R.warp == 0) {
         tmem_alloc(smem_addr(tmem_ptr), 512);
         tmem_relinquish();
     }
@@ -269,191 +420,216 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_ptr;
-    const Issuer is;
 
-    auto load_block = [&](int j) {  // query block qb0 + j into buffer j & 1 (elected lane)
-        const uint32_t buf = sbase + KT_BUF + (j & 1) * KB_BYTES, fb = bar(B_FULL + (j & 1));
-        const int q0 = (qb0 + j) * BB;
-        mbar_arrive_expect_tx(fb, KB_BYTES);
-        tma_load_4d_nohint(buf + KB_Q1, &m.q1, fb, 0, q0, h, b);
-        tma_load_4d_nohint(buf + KB_Q2, &m.q2, fb, 0, q0, h, b);
-        tma_load_4d_nohint(buf + KB_DD, &m.dd, fb, 0, q0, h, b);
-        tma_load_4d_nohint(buf + KB_DD + 8192, &m.dd, fb, 64, q0, h, b);
-        tma_load_4d_nohint(buf + KB_ST, &m.stats, fb, q0, 0, h, b);
-    };
-    int loads = 0;  // blocks whose loads were issued
-    if (warp == 0) {
+    if (R.producer()) {
+        // ------------------------------------------------------------ TMA producer
         if (elect_one()) {
-            mbar_arrive_expect_tx(bar(B_TILE), KT_BUF);
+            mbar_arrive_expect_tx(bar(B_TILE), KT_STAGE0);
             tma_load_4d_nohint(sbase + KT_K1, &m.k1, bar(B_TILE), 0, k0, h, b);
-            tma_load_4d_nohint(sbase + KT_K2, &m.k2, bar(B_TILE), 0, k0, h, b);
-            tma_load_4d_nohint(sbase + KT_V, &m.v, bar(B_TILE), 0, k0, h, b);
-            tma_load_4d_nohint(sbase + KT_V + 16384, &m.v, bar(B_TILE), 64, k0, h, b);
-            load_block(0);
+            tma_load_4d_nohint(sbase + KT_K2, &m.k2, bar(B_TILE), 0, k0, hn, b);
+            tma_load_4d_nohint(sbase + KT_V, &m.v, bar(B_TILE), 0, k0, hv, b);
+            tma_load_4d_nohint(sbase + KT_V + 16384, &m.v, bar(B_TILE), 64, k0, hv, b);
         }
         __syncwarp();
-    }
-    loads = 1;
-
-    const int kj = k0 + warp * 32 + lane;  // this thread's key
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
-    const float lam = p.lambda[h];
-    int consumed = 0, commits_s = 0, commits_m = 0;
-    bool tile_waited = false, ok = true;
-    for (int j = 0; j < nit; ++j) {
-        const uint32_t buf = sbase + KT_BUF + (j & 1) * KB_BYTES;
-        bool ok_w = true;
-        if (warp == 0) {
-            if (!tile_waited) ok_w = tile_waited = mbar_wait_warp(bar(B_TILE), 0, abort_flag, lim);
-            ok_w = ok_w && mbar_wait_warp(bar(B_FULL + (j & 1)), (j >> 1) & 1, abort_flag, lim);
-            if (ok_w) {
-                consumed = j + 1;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                    is.ss(tbase + KM_S1, sw128(sbase + KT_K1 + 32 * kk), sw128(buf + KB_Q1 + 32 * kk), ID_S, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                    is.ss(tbase + KM_S2, sw128(sbase + KT_K2 + 32 * kk), sw128(buf + KB_Q2 + 32 * kk), ID_S, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < HDV / 16; ++kk) {
-                    const uint32_t o = 32 * (kk & 3);
-                    is.ss(tbase + KM_DP, sw128(sbase + KT_V + (kk >> 2) * 16384 + o),
-                          sw128(buf + KB_DD + (kk >> 2) * 8192 + o), ID_DP, kk > 0);
-                }
-                is.commit(bar(B_S));
-                ++commits_s;
+        int loads = 0;
+        for (int j = 0; j < nit; ++j) {
+            const int s = j & 1;
+            if (j >= 2 && !mbar_wait_warp(bar(B_EMPTY + s), ((j >> 1) - 1) & 1, abort_flag, lim)) break;
+            if (elect_one()) {
+                const uint32_t st = sbase + KT_STAGE0 + s * KB_BYTES, fb = bar(B_FULL + s);
+                const int q0 = (qb0 + j) * BB;
+                mbar_arrive_expect_tx(fb, KB_LOAD);
+                tma_load_4d_nohint(st + KB_Q1, &m.q1, fb, 0, q0, h, b);
+                tma_load_4d_nohint(st + KB_Q2, &m.q2, fb, 0, q0, hn, b);
+                tma_load_4d_nohint(st + KB_DD, &m.dd, fb, 0, q0, h, b);
+                tma_load_4d_nohint(st + KB_DD + 8192, &m.dd, fb, 64, q0, h, b);
+                tma_load_4d_nohint(st + KB_ST, &m.stats, fb, q0, 0, h, b);
             }
-        }
-        // Everyone: the three products of this block are in TMEM (and, as
-        // the commit covers all earlier MMAs, the previous block's
-        // accumulations have read their operands).
-        bool ok_s = ok_w && mbar_wait_warp(bar(B_S), j & 1, abort_flag, lim);
-        if (!__syncthreads_and(ok_s)) {
-            ok = false;
-            break;
-        }
-        tc_fence_after();
-        if (warp == 0 && j + 1 < nit) {
-            if (elect_one()) load_block(j + 1);
             __syncwarp();
-            loads = j + 2;
+            loads = j + 1;
         }
-
-        // Element-wise step for this thread's key against the block's 64
-        // queries, 32 at a time.
-        const float *st = reinterpret_cast<const float *>(smem + KT_BUF + (j & 1) * KB_BYTES + KB_ST);
-        const int q0 = (qb0 + j) * BB;
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {
-            uint32_t s1[32], s2[32], dp[32];
-            tmem_ld32(tbase + lane_off + KM_S1 + 32 * ch, s1);
-            tmem_ld32(tbase + lane_off + KM_S2 + 32 * ch, s2);
-            tmem_ld32(tbase + lane_off + KM_DP + 32 * ch, dp);
-            tmem_wait_ld();
-            uint32_t pc[16], ds1[16], ds2[16];
+        // No load of ours may land after the CTA has gone.
+        bool drained = mbar_wait_drain(bar(B_TILE), 0, lim);
+        for (int k = (loads > 2 ? loads - 2 : 0); k < loads; ++k)
+            drained &= mbar_wait_drain(bar(B_FULL + (k & 1)), (k >> 1) & 1, lim);
+        if (!__all_sync(0xffffffffu, drained) && R.lane == 0) *abort_flag = 1;
+    } else if (R.issuer()) {
+        // ------------------------------------------------------------ MMA issuer
+        // Per block j: the score and dP products of block j (once the
+        // element-wise warps have taken block j-1's out of TMEM), then the
+        // accumulating products of block j-1 (once its A operands are
+        // written).  The tensor pipe runs them in that order.
+        auto issue_s = [&](int j) {
+            const uint32_t st = sbase + KT_STAGE0 + (j & 1) * KB_BYTES;
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-                float pv[2], d1[2], d2[2];
+            for (int kk = 0; kk < HD / 16; ++kk)
+                mma_issue(tbase + KM_S1, sw128(sbase + KT_K1 + 32 * kk), sw128(st + KB_Q1 + 32 * kk), Ids<F16QK>::S,
+                          kk > 0);
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int qi = 32 * ch + i + e, q = q0 + qi;
-                    const bool vis = q < p.N && kj < p.N && (!p.causal || q >= kj);
-                    const float p1 = vis ? ex2_approx(fmaf(__uint_as_float(s1[i + e]), p.scale_log2, -st[qi])) : 0.f;
-                    const float p2 = vis ? ex2_approx(fmaf(__uint_as_float(s2[i + e]), p.scale_log2, -st[BB + qi])) : 0.f;
-                    const float g = __uint_as_float(dp[i + e]);
-                    pv[e] = fmaf(-lam, p2, p1);
-                    d1[e] = p1 * (g - st[2 * BB + qi]);
-                    d2[e] = p2 * fmaf(-lam, g, -st[3 * BB + qi]);
-                }
-                pc[i >> 1] = pack_half2(pv[0], pv[1]);
-                ds1[i >> 1] = pack_bf162(d1[0], d1[1]);
-                ds2[i >> 1] = pack_bf162(d2[0], d2[1]);
+            for (int kk = 0; kk < HD / 16; ++kk)
+                mma_issue(tbase + KM_S2, sw128(sbase + KT_K2 + 32 * kk), sw128(st + KB_Q2 + 32 * kk), Ids<F16QK>::S,
+                          kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < HDV / 16; ++kk) {
+                const uint32_t o = 32 * (kk & 3);
+                mma_issue(tbase + KM_DP, sw128(sbase + KT_V + (kk >> 2) * 16384 + o),
+                          sw128(st + KB_DD + (kk >> 2) * 8192 + o), ID_DP, kk > 0);
             }
-            tmem_st16(tbase + lane_off + KM_S1 + 16 * ch, pc);
-            tmem_st16(tbase + lane_off + KM_S2 + 16 * ch, ds1);
-            tmem_st16(tbase + lane_off + KM_DP + 16 * ch, ds2);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncthreads();
-        if (warp == 0) {
+            commit_to(bar(B_SFULL));
+        };
+        auto issue_acc = [&](int j) {
+            const uint32_t st = sbase + KT_STAGE0 + (j & 1) * KB_BYTES;
+            // dV += (P_1 - lambda P_2)^T dD; dK_t += dS_t^T Q_t (B MN-major).
+#pragma unroll
+            for (int kk = 0; kk < BB / 16; ++kk)
+                mma_issue(tbase + KM_DV, sw128(sbase + KT_A + KA_PV + 32 * kk), sw128(st + KB_DD + 2048 * kk, 8192),
+                          ID_DV, j > 0 || kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < BB / 16; ++kk)
+                mma_issue(tbase + KM_DK1, sw128(sbase + KT_A + KA_DS1 + 32 * kk), sw128(st + KB_Q1 + 2048 * kk, 8192),
+                          Ids<F16QK>::DS, j > 0 || kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < BB / 16; ++kk)
+                mma_issue(tbase + KM_DK2, sw128(sbase + KT_A + KA_DS2 + 32 * kk), sw128(st + KB_Q2 + 2048 * kk, 8192),
+                          Ids<F16QK>::DS, j > 0 || kk > 0);
+            commit_to(bar(B_AFREE));
+            commit_to(bar(B_EMPTY + (j & 1)));
+        };
+        bool ok = mbar_wait_warp(bar(B_TILE), 0, abort_flag, lim);
+        for (int j = 0; ok && j < nit; ++j) {
+            if (!(ok = mbar_wait_warp(bar(B_FULL + (j & 1)), (j >> 1) & 1, abort_flag, lim))) break;
+            if (j > 0 && !(ok = mbar_wait_warp(bar(B_SFREE), (j - 1) & 1, abort_flag, lim))) break;
             tc_fence_after();
-            // dV += (P_1 - lambda P_2)^T dD; dK_t += dS_t^T Q_t (A from TMEM).
-#pragma unroll
-            for (int kk = 0; kk < BB / 16; ++kk)
-                is.ts(tbase + KM_DV, tbase + KM_S1 + 8 * kk, sw128(buf + KB_DD + 2048 * kk, 8192), ID_DV,
-                      j > 0 || kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < BB / 16; ++kk)
-                is.ts(tbase + KM_DK1, tbase + KM_S2 + 8 * kk, sw128(buf + KB_Q1 + 2048 * kk, 8192), ID_ACC64,
-                      j > 0 || kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < BB / 16; ++kk)
-                is.ts(tbase + KM_DK2, tbase + KM_DP + 8 * kk, sw128(buf + KB_Q2 + 2048 * kk, 8192), ID_ACC64,
-                      j > 0 || kk > 0);
-            is.commit(bar(B_M));
-            ++commits_m;
+            issue_s(j);
+            if (j > 0) {
+                if (!(ok = mbar_wait_warp(bar(B_AFULL), (j - 1) & 1, abort_flag, lim))) break;
+                tc_fence_after();
+                issue_acc(j - 1);
+            }
         }
-    }
-    // The last accumulations, then the tile's rows of dV, dK_1, dK_2.
-    if (ok) ok = __syncthreads_and(mbar_wait_warp(bar(B_M), (nit - 1) & 1, abort_flag, lim));
-    if (ok) {
-        // Every lane takes part in the TMEM loads (warp-collective); only
-        // rows of keys below N are stored.
-        tc_fence_after();
-        const bool own = kj < p.N;
-        const int krow = own ? kj : 0;
-        uint32_t v[32];
-        __nv_bfloat16 *dvr = static_cast<__nv_bfloat16 *>(p.dv) + (size_t)b * p.dv_s[0] +
-                             (size_t)krow * p.dv_s[1] + (size_t)h * p.dv_s[2];
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-            tmem_ld32(tbase + lane_off + KM_DV + 32 * c, v);
-            tmem_wait_ld();
-            if (own) store_row_bf16(dvr + 32 * c, v, 1.0f);
+        if (ok && mbar_wait_warp(bar(B_AFULL), (nit - 1) & 1, abort_flag, lim)) {
+            tc_fence_after();
+            issue_acc(nit - 1);
         }
-        __nv_bfloat16 *dk1 = static_cast<__nv_bfloat16 *>(p.dk1) + (size_t)b * p.dk1_s[0] +
-                             (size_t)krow * p.dk1_s[1] + (size_t)h * p.dk1_s[2];
-        __nv_bfloat16 *dk2 = static_cast<__nv_bfloat16 *>(p.dk2) + (size_t)b * p.dk2_s[0] +
-                             (size_t)krow * p.dk2_s[1] + (size_t)h * p.dk2_s[2];
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-            tmem_ld32(tbase + lane_off + KM_DK1 + 32 * c, v);
+        // DONE completes once everything issued has: the epilogue's signal,
+        // and the teardown's guarantee that no product still runs.
+        commit_to(bar(B_DONE));
+        if (!__all_sync(0xffffffffu, mbar_wait_drain(bar(B_DONE), 0, lim)) && R.lane == 0) *abort_flag = 1;
+    } else {
+        // ------------------------------------------------------------ element-wise + epilogue
+        const int wg = R.wg(), r = R.row();
+        const uint32_t lo = R.lane_off();
+        const int kj = k0 + r;  // this thread's key
+        const float c = p.scale_log2;
+        bool ok = true, big = false;
+        for (int j = 0; j < nit; ++j) {
+            if (!(ok = mbar_wait_warp(bar(B_SFULL), j & 1, abort_flag, lim))) break;
+            tc_fence_after();
+            uint32_t s1[32], s2[32], dp[32];
+            tmem_ld32(tbase + lo + KM_S1 + 32 * wg, s1);
+            tmem_ld32(tbase + lo + KM_S2 + 32 * wg, s2);
+            tmem_ld32(tbase + lo + KM_DP + 32 * wg, dp);
             tmem_wait_ld();
-            if (own) store_row_bf16(dk1 + 32 * c, v, p.scale);
-            tmem_ld32(tbase + lane_off + KM_DK2 + 32 * c, v);
-            tmem_wait_ld();
-            if (own) store_row_bf16(dk2 + 32 * c, v, p.scale);
+            tc_fence_before();
+            __syncwarp();
+            if (R.lane == 0) mbar_arrive(bar(B_SFREE));
+            // This warpgroup's 32 queries of the block, and their statistics.
+            const int qb = (qb0 + j) * BB + 32 * wg;
+            const uint32_t st = sbase + KT_STAGE0 + (j & 1) * KB_BYTES + KB_ST + 4 * 32 * wg;
+            const bool mask = (p.causal && qb < k0 + BT - 1) || (p.window > 0 && qb + 31 - k0 >= p.window);
+            uint32_t pv[16], d1p[16], d2p[16];
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+                const uint4 ul1 = ld_shared_v4(st + 4 * i), ul2 = ld_shared_v4(st + 256 + 4 * i);
+                const uint4 ud1 = ld_shared_v4(st + 512 + 4 * i), ud2 = ld_shared_v4(st + 768 + 4 * i);
+                const uint4 ulm = ld_shared_v4(st + 1024 + 4 * i);
+                const uint32_t l1[4] = {ul1.x, ul1.y, ul1.z, ul1.w}, l2[4] = {ul2.x, ul2.y, ul2.z, ul2.w};
+                const uint32_t D1[4] = {ud1.x, ud1.y, ud1.z, ud1.w}, D2[4] = {ud2.x, ud2.y, ud2.z, ud2.w};
+                const uint32_t LM[4] = {ulm.x, ulm.y, ulm.z, ulm.w};
+                float vp[4], v1[4], v2[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float p1 = ex2_approx(fmaf(__uint_as_float(s1[i + e]), c, -__uint_as_float(l1[e])));
+                    float p2 = ex2_approx(fmaf(__uint_as_float(s2[i + e]), c, -__uint_as_float(l2[e])));
+                    if (mask) {
+                        const int q = qb + i + e;
+                        const bool vis = (!p.causal || q >= kj) && (p.window <= 0 || q - kj < p.window);
+                        p1 = vis ? p1 : 0.f;
+                        p2 = vis ? p2 : 0.f;
+                    }
+                    const float g = __uint_as_float(dp[i + e]), lam = __uint_as_float(LM[e]);
+                    vp[e] = fmaf(-lam, p2, p1);
+                    v1[e] = p1 * (g - __uint_as_float(D1[e]));
+                    v2[e] = p2 * fmaf(-lam, g, -__uint_as_float(D2[e]));
+                    if (F16QK) big |= !(fabsf(v1[e]) <= 65504.0f && fabsf(v2[e]) <= 65504.0f);
+                }
+                pv[i / 2] = pack_half2(vp[0], vp[1]);
+                pv[i / 2 + 1] = pack_half2(vp[2], vp[3]);
+                d1p[i / 2] = pack_ds(v1[0], v1[1], F16QK);
+                d1p[i / 2 + 1] = pack_ds(v1[2], v1[3], F16QK);
+                d2p[i / 2] = pack_ds(v2[0], v2[1], F16QK);
+                d2p[i / 2 + 1] = pack_ds(v2[2], v2[3], F16QK);
+            }
+            // The previous block's accumulating products must have read the
+            // A operands before they are overwritten.
+            if (j > 0 && !(ok = mbar_wait_warp(bar(B_AFREE), (j - 1) & 1, abort_flag, lim))) break;
+            st_operand_half(sbase + KT_A + KA_PV, r, wg, pv);
+            st_operand_half(sbase + KT_A + KA_DS1, r, wg, d1p);
+            st_operand_half(sbase + KT_A + KA_DS2, r, wg, d2p);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (R.lane == 0) mbar_arrive(bar(B_AFULL));
         }
-    } else if (threadIdx.x == 0) {
-        report_error(p.dev_status, DIFFATTN_ERR_TIMEOUT);
-    }
-    // Nothing of ours may be in flight when the CTA frees TMEM and exits.
-    if (warp == 0) {
-        bool drained = true;
-        if (!tile_waited) drained &= mbar_wait_drain(bar(B_TILE), 0, lim);
-        for (int jj = consumed; jj < loads; ++jj)
-            drained &= mbar_wait_drain(bar(B_FULL + (jj & 1)), (jj >> 1) & 1, lim);
-        if (commits_s > 0) drained &= mbar_wait_drain(bar(B_S), (commits_s - 1) & 1, lim);
-        if (commits_m > 0) drained &= mbar_wait_drain(bar(B_M), (commits_m - 1) & 1, lim);
-        if (!__all_sync(0xffffffffu, drained) && lane == 0) report_error(p.dev_status, DIFFATTN_ERR_TIMEOUT);
+        if (big) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
+        if (ok) ok = mbar_wait_warp(bar(B_DONE), 0, abort_flag, lim);
+        if (ok) {
+            // Warpgroup 0 writes dV columns [0, 64) and dK_1; warpgroup 1 dV
+            // columns [64, 128) and dK_2.  Every lane takes part in the TMEM
+            // loads (warp-collective); only rows of keys below N are stored.
+            tc_fence_after();
+            const bool own = kj < p.N;
+            const int krow = own ? kj : 0;
+            float x[64];
+            tmem_row64(tbase + lo + KM_DV + 64 * wg, x);
+            if (own) {
+                __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dv) + (size_t)b * p.dv_s[0] +
+                                     (size_t)krow * p.dv_s[1] + (size_t)hv * p.dv_s[2] + 64 * wg;
+                float *acc = p.acc_dv ? p.acc_dv + (((size_t)b * p.N + krow) * p.H_V + hv) * HDV + 64 * wg : nullptr;
+                put_row<64>(x, 1.0f, dst, acc);
+            }
+            tmem_row64(tbase + lo + (wg ? KM_DK2 : KM_DK1), x);
+            if (own) {
+                if (F16QK) unrotate64(x, krow, p.rope_g);
+                if (wg == 0) {
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dk1) + (size_t)b * p.dk1_s[0] +
+                                         (size_t)krow * p.dk1_s[1] + (size_t)h * p.dk1_s[2];
+                    put_row<64>(x, p.scale, dst, nullptr);
+                } else {
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dk2) + (size_t)b * p.dk2_s[0] +
+                                         (size_t)krow * p.dk2_s[1] + (size_t)hn * p.dk2_s[2];
+                    float *acc = p.acc_dk2 ? p.acc_dk2 + (((size_t)b * p.N + krow) * p.H_N + hn) * HD : nullptr;
+                    put_row<64>(x, p.scale, dst, acc);
+                }
+            }
+        }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (threadIdx.x == 0 && *abort_flag) report_error(p.dev_status, DIFFATTN_ERR_TIMEOUT);
+    if (R.warp == 0) {
         tc_fence_after();
         tmem_dealloc(tbase, 512);
     }
 }
 
 // ---------------------------------------------------------------- 3. query tiles
+template <bool F16QK>
 __global__ void __launch_bounds__(NT, 1)
     bwd_query_kernel(const __grid_constant__ BwdQueryMaps m, const BwdParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_addr(smem);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Roles R{(int)(threadIdx.x >> 5), (int)(threadIdx.x & 31)};
     if (sbase & 1023u) {
         if (threadIdx.x == 0) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
         return;
@@ -461,21 +637,34 @@ __global__ void __launch_bounds__(NT, 1)
     // Heavy tiles first: under the causal mask the last query tile meets every key.
     const int BH = p.B * p.H;
     const int qt = p.num_qt - 1 - (int)(blockIdx.x / BH), bh = blockIdx.x % BH, b = bh / p.H, h = bh % p.H;
+    const int hn = h / (p.H / p.H_N), hv = h / (p.H / p.H_V);
     const int q0 = qt * BT;
+    // Key blocks the tile's queries see: up to the diagonal when causal;
+    // under a window of W keys from the block holding key q0 - W + 1.
     const int nkb_all = (p.N + BB - 1) / BB;
-    const int nit = p.causal ? min(nkb_all, (q0 + BT) / BB) : nkb_all;
+    const int kb0 = p.window > 0 ? max(0, q0 - p.window + 1) / BB : 0;
+    const int kb1 = p.causal ? min(nkb_all, (q0 + BT - 1) / BB + 1) : nkb_all;
+    const int nit = kb1 - kb0;  // >= 1
     auto bar = [&](int i) { return sbase + QT_BARS + 8 * i; };
-    enum { B_TILE = 0, B_FULL = 1, B_S = 3, B_M = 4 };
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + QT_BARS + 8 * NBARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + QT_BARS + 8 * NBARS + 4);
     const uint64_t lim = p.timeout_ns;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NBARS; ++i) mbar_init(bar(i), 1);
+        mbar_init(bar(B_TILE), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(B_FULL + s), 1);
+            mbar_init(bar(B_EMPTY + s), 1);
+        }
+        mbar_init(bar(B_SFULL), 1);
+        mbar_init(bar(B_SFREE), NEW);
+        mbar_init(bar(B_AFULL), NEW);
+        mbar_init(bar(B_AFREE), 1);
+        mbar_init(bar(B_DONE), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 0) {
+    if (R.warp == 0) {
         tmem_alloc(smem_addr(tmem_ptr), 512);
         tmem_relinquish();
     }
@@ -483,168 +672,218 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_ptr;
-    const Issuer is;
 
-    auto load_block = [&](int j) {  // key block j into buffer j & 1 (elected lane)
-        const uint32_t buf = sbase + QT_BUF + (j & 1) * QB_BYTES, fb = bar(B_FULL + (j & 1));
-        const int kb = j * BB;
-        mbar_arrive_expect_tx(fb, QB_BYTES);
-        tma_load_4d_nohint(buf + QB_K1, &m.k1, fb, 0, kb, h, b);
-        tma_load_4d_nohint(buf + QB_K2, &m.k2, fb, 0, kb, h, b);
-        tma_load_4d_nohint(buf + QB_V, &m.v, fb, 0, kb, h, b);
-        tma_load_4d_nohint(buf + QB_V + 8192, &m.v, fb, 64, kb, h, b);
-    };
-    int loads = 0;
-    if (warp == 0) {
+    if (R.producer()) {
         if (elect_one()) {
-            mbar_arrive_expect_tx(bar(B_TILE), QT_BUF);
+            mbar_arrive_expect_tx(bar(B_TILE), QT_STAGE0);
             tma_load_4d_nohint(sbase + QT_Q1, &m.q1, bar(B_TILE), 0, q0, h, b);
-            tma_load_4d_nohint(sbase + QT_Q2, &m.q2, bar(B_TILE), 0, q0, h, b);
+            tma_load_4d_nohint(sbase + QT_Q2, &m.q2, bar(B_TILE), 0, q0, hn, b);
             tma_load_4d_nohint(sbase + QT_DD, &m.dd, bar(B_TILE), 0, q0, h, b);
             tma_load_4d_nohint(sbase + QT_DD + 16384, &m.dd, bar(B_TILE), 64, q0, h, b);
-            load_block(0);
         }
         __syncwarp();
-    }
-    loads = 1;
-
-    const int qrow = q0 + warp * 32 + lane;  // this thread's query
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
-    const float lam = p.lambda[h];
-    const float *strow = p.stats + (size_t)(b * p.H + h) * 4 * p.n_pad + qrow;
-    const float lse1 = strow[0], lse2 = strow[p.n_pad], del1 = strow[2 * p.n_pad], del2 = strow[3 * p.n_pad];
-    int consumed = 0, commits_s = 0, commits_m = 0;
-    bool tile_waited = false, ok = true;
-    for (int j = 0; j < nit; ++j) {
-        const uint32_t buf = sbase + QT_BUF + (j & 1) * QB_BYTES;
-        bool ok_w = true;
-        if (warp == 0) {
-            if (!tile_waited) ok_w = tile_waited = mbar_wait_warp(bar(B_TILE), 0, abort_flag, lim);
-            ok_w = ok_w && mbar_wait_warp(bar(B_FULL + (j & 1)), (j >> 1) & 1, abort_flag, lim);
-            if (ok_w) {
-                consumed = j + 1;
+        int loads = 0;
+        for (int j = 0; j < nit; ++j) {
+            const int s = j & 1;
+            if (j >= 2 && !mbar_wait_warp(bar(B_EMPTY + s), ((j >> 1) - 1) & 1, abort_flag, lim)) break;
+            if (elect_one()) {
+                const uint32_t st = sbase + QT_STAGE0 + s * QB_BYTES, fb = bar(B_FULL + s);
+                const int k0 = (kb0 + j) * BB;
+                mbar_arrive_expect_tx(fb, QB_BYTES);
+                tma_load_4d_nohint(st + QB_K1, &m.k1, fb, 0, k0, h, b);
+                tma_load_4d_nohint(st + QB_K2, &m.k2, fb, 0, k0, hn, b);
+                tma_load_4d_nohint(st + QB_V, &m.v, fb, 0, k0, hv, b);
+                tma_load_4d_nohint(st + QB_V + 8192, &m.v, fb, 64, k0, hv, b);
+            }
+            __syncwarp();
+            loads = j + 1;
+        }
+        bool drained = mbar_wait_drain(bar(B_TILE), 0, lim);
+        for (int k = (loads > 2 ? loads - 2 : 0); k < loads; ++k)
+            drained &= mbar_wait_drain(bar(B_FULL + (k & 1)), (k >> 1) & 1, lim);
+        if (!__all_sync(0xffffffffu, drained) && R.lane == 0) *abort_flag = 1;
+    } else if (R.issuer()) {
+        auto issue_s = [&](int j) {
+            const uint32_t st = sbase + QT_STAGE0 + (j & 1) * QB_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < HD / 16; ++kk)
+                mma_issue(tbase + QM_S1, sw128(sbase + QT_Q1 + 32 * kk), sw128(st + QB_K1 + 32 * kk), Ids<F16QK>::S,
+                          kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < HD / 16; ++kk)
+                mma_issue(tbase + QM_S2, sw128(sbase + QT_Q2 + 32 * kk), sw128(st + QB_K2 + 32 * kk), Ids<F16QK>::S,
+                          kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < HDV / 16; ++kk) {
+                const uint32_t o = 32 * (kk & 3);
+                mma_issue(tbase + QM_DP, sw128(sbase + QT_DD + (kk >> 2) * 16384 + o),
+                          sw128(st + QB_V + (kk >> 2) * 8192 + o), ID_DP, kk > 0);
+            }
+            commit_to(bar(B_SFULL));
+        };
+        auto issue_acc = [&](int j) {
+            const uint32_t st = sbase + QT_STAGE0 + (j & 1) * QB_BYTES;
+            // dQ_t += dS_t K_t (B: the K block, MN-major).
+#pragma unroll
+            for (int kk = 0; kk < BB / 16; ++kk)
+                mma_issue(tbase + QM_DQ1, sw128(sbase + QT_A + QA_DS1 + 32 * kk), sw128(st + QB_K1 + 2048 * kk, 8192),
+                          Ids<F16QK>::DS, j > 0 || kk > 0);
+#pragma unroll
+            for (int kk = 0; kk < BB / 16; ++kk)
+                mma_issue(tbase + QM_DQ2, sw128(sbase + QT_A + QA_DS2 + 32 * kk), sw128(st + QB_K2 + 2048 * kk, 8192),
+                          Ids<F16QK>::DS, j > 0 || kk > 0);
+            commit_to(bar(B_AFREE));
+            commit_to(bar(B_EMPTY + (j & 1)));
+        };
+        bool ok = mbar_wait_warp(bar(B_TILE), 0, abort_flag, lim);
+        for (int j = 0; ok && j < nit; ++j) {
+            if (!(ok = mbar_wait_warp(bar(B_FULL + (j & 1)), (j >> 1) & 1, abort_flag, lim))) break;
+            if (j > 0 && !(ok = mbar_wait_warp(bar(B_SFREE), (j - 1) & 1, abort_flag, lim))) break;
+            tc_fence_after();
+            issue_s(j);
+            if (j > 0) {
+                if (!(ok = mbar_wait_warp(bar(B_AFULL), (j - 1) & 1, abort_flag, lim))) break;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                    is.ss(tbase + QM_S1, sw128(sbase + QT_Q1 + 32 * kk), sw128(buf + QB_K1 + 32 * kk), ID_S, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < HD / 16; ++kk)
-                    is.ss(tbase + QM_S2, sw128(sbase + QT_Q2 + 32 * kk), sw128(buf + QB_K2 + 32 * kk), ID_S, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < HDV / 16; ++kk) {
-                    const uint32_t o = 32 * (kk & 3);
-                    is.ss(tbase + QM_DP, sw128(sbase + QT_DD + (kk >> 2) * 16384 + o),
-                          sw128(buf + QB_V + (kk >> 2) * 8192 + o), ID_DP, kk > 0);
-                }
-                is.commit(bar(B_S));
-                ++commits_s;
+                issue_acc(j - 1);
             }
         }
-        bool ok_s = ok_w && mbar_wait_warp(bar(B_S), j & 1, abort_flag, lim);
-        if (!__syncthreads_and(ok_s)) {
-            ok = false;
-            break;
+        if (ok && mbar_wait_warp(bar(B_AFULL), (nit - 1) & 1, abort_flag, lim)) {
+            tc_fence_after();
+            issue_acc(nit - 1);
         }
-        tc_fence_after();
-        if (warp == 0 && j + 1 < nit) {
-            if (elect_one()) load_block(j + 1);
-            __syncwarp();
-            loads = j + 2;
-        }
-
-        const int kb = j * BB;
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {
+        commit_to(bar(B_DONE));
+        if (!__all_sync(0xffffffffu, mbar_wait_drain(bar(B_DONE), 0, lim)) && R.lane == 0) *abort_flag = 1;
+    } else {
+        const int wg = R.wg(), r = R.row();
+        const uint32_t lo = R.lane_off();
+        const int qrow = q0 + r;  // this thread's query
+        const float c = p.scale_log2;
+        const float *strow = p.stats + (size_t)(b * p.H + h) * kBwdStats * p.n_pad + qrow;
+        const float lse1 = strow[0], lse2 = strow[p.n_pad], del1 = strow[2 * p.n_pad], del2 = strow[3 * p.n_pad];
+        const float lam = strow[4 * p.n_pad];
+        bool ok = true, big = false;
+        for (int j = 0; j < nit; ++j) {
+            if (!(ok = mbar_wait_warp(bar(B_SFULL), j & 1, abort_flag, lim))) break;
+            tc_fence_after();
             uint32_t s1[32], s2[32], dp[32];
-            tmem_ld32(tbase + lane_off + QM_S1 + 32 * ch, s1);
-            tmem_ld32(tbase + lane_off + QM_S2 + 32 * ch, s2);
-            tmem_ld32(tbase + lane_off + QM_DP + 32 * ch, dp);
+            tmem_ld32(tbase + lo + QM_S1 + 32 * wg, s1);
+            tmem_ld32(tbase + lo + QM_S2 + 32 * wg, s2);
+            tmem_ld32(tbase + lo + QM_DP + 32 * wg, dp);
             tmem_wait_ld();
-            uint32_t ds1[16], ds2[16];
+            tc_fence_before();
+            __syncwarp();
+            if (R.lane == 0) mbar_arrive(bar(B_SFREE));
+            const int kb = (kb0 + j) * BB + 32 * wg;  // this warpgroup's 32 keys of the block
+            const bool mask = (p.causal && kb + 31 > q0) || (p.window > 0 && q0 + BT - 1 - kb >= p.window);
+            uint32_t d1p[16], d2p[16];
 #pragma unroll
             for (int i = 0; i < 32; i += 2) {
-                float d1[2], d2[2];
+                float v1[2], v2[2];
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    const int key = kb + 32 * ch + i + e;
-                    const bool vis = key < p.N && (!p.causal || key <= qrow);
-                    const float p1 = vis ? ex2_approx(fmaf(__uint_as_float(s1[i + e]), p.scale_log2, -lse1)) : 0.f;
-                    const float p2 = vis ? ex2_approx(fmaf(__uint_as_float(s2[i + e]), p.scale_log2, -lse2)) : 0.f;
+                    float p1 = ex2_approx(fmaf(__uint_as_float(s1[i + e]), c, -lse1));
+                    float p2 = ex2_approx(fmaf(__uint_as_float(s2[i + e]), c, -lse2));
+                    if (mask) {
+                        const int key = kb + i + e;
+                        const bool vis = (!p.causal || key <= qrow) && (p.window <= 0 || qrow - key < p.window);
+                        p1 = vis ? p1 : 0.f;
+                        p2 = vis ? p2 : 0.f;
+                    }
                     const float g = __uint_as_float(dp[i + e]);
-                    d1[e] = p1 * (g - del1);
-                    d2[e] = p2 * fmaf(-lam, g, -del2);
+                    v1[e] = p1 * (g - del1);
+                    v2[e] = p2 * fmaf(-lam, g, -del2);
+                    if (F16QK) big |= !(fabsf(v1[e]) <= 65504.0f && fabsf(v2[e]) <= 65504.0f);
                 }
-                ds1[i >> 1] = pack_bf162(d1[0], d1[1]);
-                ds2[i >> 1] = pack_bf162(d2[0], d2[1]);
+                d1p[i / 2] = pack_ds(v1[0], v1[1], F16QK);
+                d2p[i / 2] = pack_ds(v2[0], v2[1], F16QK);
             }
-            tmem_st16(tbase + lane_off + QM_S1 + 16 * ch, ds1);
-            tmem_st16(tbase + lane_off + QM_S2 + 16 * ch, ds2);
+            if (j > 0 && !(ok = mbar_wait_warp(bar(B_AFREE), (j - 1) & 1, abort_flag, lim))) break;
+            st_operand_half(sbase + QT_A + QA_DS1, r, wg, d1p);
+            st_operand_half(sbase + QT_A + QA_DS2, r, wg, d2p);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (R.lane == 0) mbar_arrive(bar(B_AFULL));
         }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncthreads();
-        if (warp == 0) {
+        if (big) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
+        if (ok) ok = mbar_wait_warp(bar(B_DONE), 0, abort_flag, lim);
+        if (ok) {
+            // Warpgroup 0 writes dQ_1, warpgroup 1 dQ_2; rows below N only.
             tc_fence_after();
-            // dQ_t += dS_t K_t (A from TMEM, K block as MN-major B).
-#pragma unroll
-            for (int kk = 0; kk < BB / 16; ++kk)
-                is.ts(tbase + QM_DQ1, tbase + QM_S1 + 8 * kk, sw128(buf + QB_K1 + 2048 * kk, 8192), ID_ACC64,
-                      j > 0 || kk > 0);
-#pragma unroll
-            for (int kk = 0; kk < BB / 16; ++kk)
-                is.ts(tbase + QM_DQ2, tbase + QM_S2 + 8 * kk, sw128(buf + QB_K2 + 2048 * kk, 8192), ID_ACC64,
-                      j > 0 || kk > 0);
-            is.commit(bar(B_M));
-            ++commits_m;
+            const bool own = qrow < p.N;
+            const int qr = own ? qrow : 0;
+            float x[64];
+            tmem_row64(tbase + lo + (wg ? QM_DQ2 : QM_DQ1), x);
+            if (own) {
+                if (F16QK) unrotate64(x, qr, p.rope_g);
+                if (wg == 0) {
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dq1) + (size_t)b * p.dq1_s[0] +
+                                         (size_t)qr * p.dq1_s[1] + (size_t)h * p.dq1_s[2];
+                    put_row<64>(x, p.scale, dst, nullptr);
+                } else {
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dq2) + (size_t)b * p.dq2_s[0] +
+                                         (size_t)qr * p.dq2_s[1] + (size_t)hn * p.dq2_s[2];
+                    float *acc = p.acc_dq2 ? p.acc_dq2 + (((size_t)b * p.N + qr) * p.H_N + hn) * HD : nullptr;
+                    put_row<64>(x, p.scale, dst, acc);
+                }
+            }
         }
-    }
-    if (ok) ok = __syncthreads_and(mbar_wait_warp(bar(B_M), (nit - 1) & 1, abort_flag, lim));
-    if (ok) {
-        // Every lane takes part in the TMEM loads; rows below N are stored.
-        tc_fence_after();
-        const bool own = qrow < p.N;
-        const int qr = own ? qrow : 0;
-        uint32_t v[32];
-        __nv_bfloat16 *dq1 = static_cast<__nv_bfloat16 *>(p.dq1) + (size_t)b * p.dq1_s[0] +
-                             (size_t)qr * p.dq1_s[1] + (size_t)h * p.dq1_s[2];
-        __nv_bfloat16 *dq2 = static_cast<__nv_bfloat16 *>(p.dq2) + (size_t)b * p.dq2_s[0] +
-                             (size_t)qr * p.dq2_s[1] + (size_t)h * p.dq2_s[2];
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-            tmem_ld32(tbase + lane_off + QM_DQ1 + 32 * c, v);
-            tmem_wait_ld();
-            if (own) store_row_bf16(dq1 + 32 * c, v, p.scale);
-            tmem_ld32(tbase + lane_off + QM_DQ2 + 32 * c, v);
-            tmem_wait_ld();
-            if (own) store_row_bf16(dq2 + 32 * c, v, p.scale);
-        }
-    } else if (threadIdx.x == 0) {
-        report_error(p.dev_status, DIFFATTN_ERR_TIMEOUT);
-    }
-    if (warp == 0) {
-        bool drained = true;
-        if (!tile_waited) drained &= mbar_wait_drain(bar(B_TILE), 0, lim);
-        for (int jj = consumed; jj < loads; ++jj)
-            drained &= mbar_wait_drain(bar(B_FULL + (jj & 1)), (jj >> 1) & 1, lim);
-        if (commits_s > 0) drained &= mbar_wait_drain(bar(B_S), (commits_s - 1) & 1, lim);
-        if (commits_m > 0) drained &= mbar_wait_drain(bar(B_M), (commits_m - 1) & 1, lim);
-        if (!__all_sync(0xffffffffu, drained) && lane == 0) report_error(p.dev_status, DIFFATTN_ERR_TIMEOUT);
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (threadIdx.x == 0 && *abort_flag) report_error(p.dev_status, DIFFATTN_ERR_TIMEOUT);
+    if (R.warp == 0) {
         tc_fence_after();
         tmem_dealloc(tbase, 512);
+    }
+}
+
+// ---------------------------------------------------------------- 4. conversion of shared-head sums
+// The fp32 sums of dK_2, dQ_2 (noise heads) and dV (V heads) that several
+// signal heads added into, written as bf16 rows (8 elements per thread).
+__global__ void bwd_convert_kernel(const BwdParams p)
+{
+    const int64_t n_qk = p.acc_dk2 ? (int64_t)p.B * p.N * p.H_N * (HD / 8) : 0;
+    const int64_t n_v = p.acc_dv ? (int64_t)p.B * p.N * p.H_V * (HDV / 8) : 0;
+    const int64_t total = 2 * n_qk + n_v;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const float *src;
+        __nv_bfloat16 *dst;
+        int64_t k = i;
+        if (k < 2 * n_qk) {
+            const bool q = k >= n_qk;
+            k -= q ? n_qk : 0;
+            const int c8 = int(k % (HD / 8));
+            const int64_t rowi = k / (HD / 8);
+            const int hn = int(rowi % p.H_N);
+            const int64_t bn = rowi / p.H_N;
+            const int n = int(bn % p.N), b = int(bn / p.N);
+            src = (q ? p.acc_dq2 : p.acc_dk2) + rowi * HD + 8 * c8;
+            const int64_t *s = q ? p.dq2_s : p.dk2_s;
+            dst = static_cast<__nv_bfloat16 *>(q ? p.dq2 : p.dk2) + b * s[0] + (int64_t)n * s[1] + hn * s[2] + 8 * c8;
+        } else {
+            k -= 2 * n_qk;
+            const int c8 = int(k % (HDV / 8));
+            const int64_t rowi = k / (HDV / 8);
+            const int hv = int(rowi % p.H_V);
+            const int64_t bn = rowi / p.H_V;
+            const int n = int(bn % p.N), b = int(bn / p.N);
+            src = p.acc_dv + rowi * HDV + 8 * c8;
+            dst = static_cast<__nv_bfloat16 *>(p.dv) + b * p.dv_s[0] + (int64_t)n * p.dv_s[1] + hv * p.dv_s[2] + 8 * c8;
+        }
+        const float4 a = *reinterpret_cast<const float4 *>(src), c = *reinterpret_cast<const float4 *>(src + 4);
+        *reinterpret_cast<uint4 *>(dst) =
+            make_uint4(pack_bf162(a.x, a.y), pack_bf162(a.z, a.w), pack_bf162(c.x, c.y), pack_bf162(c.z, c.w));
     }
 }
 
 }  // namespace
 
 cudaError_t launch_bwd(const BwdKeyMaps &km, const BwdQueryMaps &qm, const BwdParams &p,
-                       cudaStream_t stream, int *launches)
+                       cudaStream_t stream, int *launches, const ProfileEvents &ev)
 {
     constexpr int kMaxDevices = 64;
-    static bool attr_set[kMaxDevices] = {};
+    static std::atomic<bool> attr_set[kMaxDevices] = {};
+    static std::mutex attr_mutex;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -653,14 +892,21 @@ cudaError_t launch_bwd(const BwdKeyMaps &km, const BwdQueryMaps &qm, const BwdPa
         return cudaErrorInvalidDevice;
     }
     const int red_bytes = BT * (HDV + 1) * (int)sizeof(float);
-    if (!attr_set[dev]) {
-        e = cudaFuncSetAttribute(bwd_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, red_bytes);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(bwd_key_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KT_SMEM);
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(bwd_query_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QT_SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
+        std::lock_guard<std::mutex> lock(attr_mutex);  // first calls from several host threads
+        if (!attr_set[dev].load(std::memory_order_relaxed)) {
+            e = cudaFuncSetAttribute(bwd_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, red_bytes);
+            if (e != cudaSuccess) return e;
+            for (const void *k : {(const void *)bwd_key_kernel<false>, (const void *)bwd_key_kernel<true>}) {
+                e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KT_SMEM);
+                if (e != cudaSuccess) return e;
+            }
+            for (const void *k : {(const void *)bwd_query_kernel<false>, (const void *)bwd_query_kernel<true>}) {
+                e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QT_SMEM);
+                if (e != cudaSuccess) return e;
+            }
+            attr_set[dev].store(true, std::memory_order_release);
+        }
     }
     if ((int64_t)p.B * p.H * p.num_qt == 0) return cudaSuccess;
     const bool want_dgain = p.apply_norm && p.dgain;
@@ -669,13 +915,28 @@ cudaError_t launch_bwd(const BwdKeyMaps &km, const BwdQueryMaps &qm, const BwdPa
     ++*launches;
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bwd_key_kernel<<<tiles, NT, KT_SMEM, stream>>>(km, p);
+    if (ev.start) cudaEventRecord(ev.start, stream);
+    if (p.qk_f16)
+        bwd_key_kernel<true><<<tiles, NT, KT_SMEM, stream>>>(km, p);
+    else
+        bwd_key_kernel<false><<<tiles, NT, KT_SMEM, stream>>>(km, p);
     ++*launches;
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    bwd_query_kernel<<<tiles, NT, QT_SMEM, stream>>>(qm, p);
+    if (p.qk_f16)
+        bwd_query_kernel<true><<<tiles, NT, QT_SMEM, stream>>>(qm, p);
+    else
+        bwd_query_kernel<false><<<tiles, NT, QT_SMEM, stream>>>(qm, p);
     ++*launches;
-    return cudaGetLastError();
+    if (ev.stop) cudaEventRecord(ev.stop, stream);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (p.acc_dk2 || p.acc_dv) {
+        bwd_convert_kernel<<<device_sm_count() * 8, 256, 0, stream>>>(p);
+        ++*launches;
+        e = cudaGetLastError();
+    }
+    return e;
 }
 
 }  // namespace da

@@ -338,9 +338,12 @@ cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream, int *launc
     const size_t smem = (size_t)(2 * p.chunk + 16 * 2 * DHDV) * sizeof(float);
     if (smem > 48 * 1024) {
         // The opt-in shared-memory size is a per-device attribute of the
-        // kernel: remember the largest size set on each device.
+        // kernel: remember the largest size set on each device (under a
+        // mutex, for first calls from several host threads).
         constexpr int kMaxDevices = 64;
         static size_t smem_set[kMaxDevices] = {};
+        static std::mutex smem_mutex;
+        std::lock_guard<std::mutex> lock(smem_mutex);
         int dev = 0;
         cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return e;

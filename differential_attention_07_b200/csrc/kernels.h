@@ -30,10 +30,14 @@ struct PrefillParams {
     int window;           // sliding window in keys (query i sees i-window < j <= i), 0 = none
     int qk_f16;           // Q/K are fp16 (the rotated copies) rather than bf16
     int withhold_load;    // test hook: skip the first K/V load of the CTA's first tile
-    int mode;             // 0: one signal head per unit; 1, 2: grouped pairs (see prefill_sm100.cu)
-    int units;            // work units per batch entry for this launch
-    float *noise_out;     // modes 1, 2: normalised noise outputs, fp32, per (b, noise head,
+    int mode;             // 0: one signal head per item; 1: grouped pairs (see prefill_sm100.cu)
+    int units;            // tile units per batch entry: signal heads (mode 0), noise heads (mode 1)
+    int pairs;            // mode 1: (signal, signal) pairs per group, (H / H_N - 1) / 2
+    int lag;              // mode 1: tiles by which a group's pair items trail its export item
+    float *noise_out;     // mode 1: normalised noise outputs, fp32, per (b, noise head,
                           // query tile) 32 float4 chunks x 128 rows (chunk-major)
+    int *noise_ready;     // mode 1: per (b, noise head, query tile) count of the 8 epilogue
+                          // warps that have exported their part (zeroed by the staging kernel)
     const float *lambda;  // [H], unused when lam_logits is set
     const float *gain;    // [H, 128] or nullptr
     const float *lam_logits;  // token-dependent lambda logits [B, N, H] or nullptr
@@ -81,36 +85,58 @@ struct RopeStage {
     int enabled;
 };
 
+// `zero`/`n_zero`: ints the staging kernel also clears (the grouped pairs'
+// ready counts), or nullptr / 0.  `sm_count`: SMs of the device (grid size).
 cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, void *dst, int B,
                             int N, int H_V, int32_t *dev_status, int *tile_counter,
-                            const RopeStage &rope,
+                            int *zero, int64_t n_zero, const RopeStage &rope, int sm_count,
                             cudaStream_t stream, int *launches);
 
-// Backward pass (backward_sm100.cu).  H_N == H_V == H.
+// SM count of the current device, looked up once per device (thread-safe);
+// 148 (a B200) when no device is visible, for host-only size queries.
+int device_sm_count();
+
+// Backward pass (backward_sm100.cu).
 struct BwdParams {
-    int B, N, H;
+    int B, N, H, H_N, H_V;
     int num_qt, n_pad;    // 128-row tiles per (b, h) and n_pad = 128 num_qt
     float scale, scale_log2, eps;
     int causal, apply_norm;
+    int window;           // sliding window in keys, 0 = none
     const float *save;    // the forward's saved state (kSaveTileFloats per tile)
     const void *dout;     // bf16 [B, N, H, 128]
     int64_t do_sb, do_sn, do_sh;
-    const float *lambda;  // [H]
+    const float *lambda;  // [H], unused with lam_logits
+    const float *lam_logits;  // [B, N, H] or nullptr
+    int64_t ll_sb, ll_sn, ll_sh;
+    const void *gate;     // bf16 gate logits [B, N, H, 128] or nullptr
+    int64_t gate_sb, gate_sn, gate_sh;
     const float *gain;    // [H, 128] or nullptr (1)
     void *dd;             // workspace: dD as fp16, contiguous [B, N, H, 128]
-    float *stats;         // workspace: [B, H, 4, n_pad] fp32 (lse_1, lse_2, Delta_1, Delta_2)
+    float *stats;         // workspace: [B, H, kBwdStats, n_pad] fp32
     void *dq1, *dq2, *dk1, *dk2, *dv;  // bf16 outputs
     int64_t dq1_s[3], dq2_s[3], dk1_s[3], dk2_s[3], dv_s[3];
+    float *acc_dq2, *acc_dk2, *acc_dv;  // fp32 [B, N, heads, dim] sums when heads are shared, else nullptr
     float *dlambda;       // [H] (zeroed before the call) or nullptr
     float *dgain;         // [H, 128] (zeroed before the call) or nullptr
+    float *dlam_logits;   // [B, N, H] or nullptr
+    int64_t dll_sb, dll_sn, dll_sh;
+    void *dgate;          // bf16 [B, N, H, 128] or nullptr
+    int64_t dg_sb, dg_sn, dg_sh;
+    int qk_f16;           // Q/K operands are the rotated fp16 copies (rotary embedding)
+    double rope_g[32];    // turns per token of pair c: theta^(-2c/64) / (2 pi)
     int32_t *dev_status;
     uint64_t timeout_ns;
 };
 
+// Row statistics of the backward pass, per (b, h): lse_1, lse_2, Delta_1,
+// Delta_2 and the row's lambda, each n_pad floats.
+constexpr int kBwdStats = 5;
+
 // Tensor maps of the key-tile kernel (dK_1, dK_2, dV): K_1, K_2 and the fp16
 // V copy in 128-row boxes; Q_1, Q_2 and dD in 64-row boxes (all 128-byte
-// swizzled, {64 columns, rows} boxes); the statistics in {64 rows, 4 arrays}
-// boxes of fp32, not swizzled.
+// swizzled, {64 columns, rows} boxes); the statistics in {64 rows,
+// kBwdStats arrays} boxes of fp32, not swizzled.
 struct BwdKeyMaps {
     CUtensorMap k1, k2, v, q1, q2, dd, stats;
 };
@@ -120,11 +146,12 @@ struct BwdQueryMaps {
     CUtensorMap q1, q2, dd, k1, k2, v;
 };
 
-// Launch the backward kernels after the V staging: the row preparation
-// (dD, statistics, dlambda, dgain), the key-tile kernel and the query-tile
-// kernel.
+// Launch the backward kernels after the staging pass: the row preparation
+// (dD, statistics, dlambda or the lambda logits' gradient, dgain, the gate's
+// gradient), the key-tile kernel, the query-tile kernel and, when heads are
+// shared, the conversion of the fp32 sums.
 cudaError_t launch_bwd(const BwdKeyMaps &km, const BwdQueryMaps &qm, const BwdParams &p,
-                       cudaStream_t stream, int *launches);
+                       cudaStream_t stream, int *launches, const ProfileEvents &ev);
 
 struct DecodeParams {
     int B, H, L;

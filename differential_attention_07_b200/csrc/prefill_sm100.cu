@@ -49,7 +49,9 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <atomic>
 #include <climits>
+#include <mutex>
 
 #include "kernels.h"
 #include "sm100_ptx.cuh"
@@ -147,26 +149,28 @@ struct Work {
 // b (Q1/K1).  Modes (PrefillParams::mode):
 //   0  unit = signal head: map 2 is its noise head h / (H / H_N), V head
 //      h / (H / H_V); the tile's output is head a.
-//   1  unit = noise head n of a group whose g = H / H_N signal heads share
-//      V head n: map 1 is the group's last signal head; the output is that
-//      head, and the normalised noise output is exported for mode 2.
-//   2  unit = (noise head n, pair p): maps 1 and 2 are signal heads
-//      n g + 2p and n g + 2p + 1; each finishes against the exported noise
-//      output of its group.
+//   1  grouped pairs, for groups of g = H / H_N (odd, >= 3) signal heads
+//      that share V head n with their noise head n.  Two kinds of unit:
+//      u < H_N, the export unit of group u: map 1 is the group's last
+//      signal head, map 2 the noise head; the output is that signal head,
+//      and the normalised noise output A_N is exported for the group;
+//      u = H_N + n P + q (P = (g - 1) / 2 pairs per group), a pair unit:
+//      maps 1 and 2 are signal heads n g + 2q and n g + 2q + 1, and each
+//      finishes against the exported A_N of its group (own = true).
 struct Heads {
     int a, b, vh, n;
-    bool b_noise;
+    bool b_noise, own;
 };
 __device__ __forceinline__ Heads heads_of(int u, const PrefillParams &p)
 {
     if (p.mode == 0) {
         const int n = u / (p.H / p.H_N);
-        return Heads{u, n, u / (p.H / p.H_V), n, true};
+        return Heads{u, n, u / (p.H / p.H_V), n, true, false};
     }
     const int g = p.H / p.H_N;
-    if (p.mode == 1) return Heads{u * g + g - 1, u, u, u, true};
-    const int pairs = (g - 1) / 2, n = u / pairs, pp = u % pairs;
-    return Heads{n * g + 2 * pp, n * g + 2 * pp + 1, n, n, false};
+    if (u < p.H_N) return Heads{u * g + g - 1, u, u, u, true, false};
+    const int up = u - p.H_N, n = up / p.pairs, q = up - n * p.pairs;
+    return Heads{n * g + 2 * q, n * g + 2 * q + 1, n, n, false, true};
 }
 
 // Map the linear CTA index to (b, h, query tile).  (b, h) pairs are taken in
@@ -184,7 +188,7 @@ __device__ __forceinline__ Heads heads_of(int u, const PrefillParams &p)
 //    of the kernel idle, measured.)  The light half re-reads the first half
 //    of each head's K/V, which costs little against the kernel's 6 % DRAM
 //    use.
-__device__ __forceinline__ Work work_of(int idx, const PrefillParams &p)
+__device__ __forceinline__ Work tile_of(int idx, const PrefillParams &p)
 {
     const int BH = p.B * p.units, G = p.heads_per_group, nq = p.num_qt;
     const int n_light = p.causal ? nq / 2 : 0, n_heavy = nq - n_light;
@@ -207,6 +211,64 @@ __device__ __forceinline__ Work work_of(int idx, const PrefillParams &p)
         bh = full * G + r % tail;
     }
     return Work{bh / p.units, bh % p.units, qt};
+}
+
+// Work items of one launch.  Mode 0: the tiles above, one item each.  Mode
+// 1: the tiles are (b, noise head, query tile) triples T[0..NT); each has an
+// export item and P pair items, and a pair item's epilogue needs its tile's
+// export.  The export items run D = PrefillParams::lag tiles ahead of the
+// pair items of the same tile:
+//   T[0] .. T[D-1] export;  then per s in [D, NT): export of T[s], the P
+//   pair items of T[s - D];  then the pair items of T[NT-D] .. T[NT-1].
+// With D about the number of CTAs, an export item has finished long before
+// the pair items of its tile reach their epilogue.  Because every item comes
+// after the items it waits for, and each CTA takes its items in that order,
+// the earliest unfinished item can always proceed: the launch cannot
+// deadlock, whatever the number of resident CTAs.
+__device__ __forceinline__ Work work_of(int idx, const PrefillParams &p)
+{
+    if (p.mode == 0) return tile_of(idx, p);
+    const int NT = p.B * p.units * p.num_qt, P = p.pairs, S = P + 1, D = p.lag;
+    int s, k;
+    if (idx < D) {
+        s = idx;
+        k = 0;
+    } else if (idx < D + (NT - D) * S) {
+        const int r = idx - D;
+        s = D + r / S;
+        k = r - (r / S) * S;
+        if (k) s -= D;
+    } else {
+        const int r = idx - D - (NT - D) * S;
+        s = NT - D + r / P;
+        k = 1 + r % P;
+    }
+    Work w = tile_of(s, p);
+    if (k) w.u = p.units + w.u * P + (k - 1);
+    return w;
+}
+
+// Spin (bounded) until *flag >= target; the acquire load orders the caller's
+// later reads after the writes the flag's producers released.
+__device__ __forceinline__ bool wait_flag_geq(const int *flag, int target, volatile int *abort_flag,
+                                              uint64_t limit_ns)
+{
+    auto ld_acquire = [](const int *f) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+        return v;
+    };
+    if (ld_acquire(flag) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        __nanosleep(64);
+        if (ld_acquire(flag) >= target) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            *abort_flag = 1;
+            return false;
+        }
+    }
 }
 
 // Software 2^x for two values at once on the FMA and integer pipes, to take
@@ -358,7 +420,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (threadIdx.x == 0) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
         return;
     }
-    const int total = p.B * p.units * p.num_qt;
+    const int total = p.B * p.units * p.num_qt * (p.mode == 1 ? p.pairs + 1 : 1);
     int *sItem = reinterpret_cast<int *>(smem + OFF_ITEM);
     const int n_steps_all = (p.N + BN - 1) / BN;
     // Key steps of a work item: [kv_first, kv_first + steps_of).  Causal tiles
@@ -619,6 +681,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t tO1 = tbase + lane_off + TM_O1, tO2 = tbase + lane_off + TM_O2;
         const uint32_t bar_pv = bar(B_PV + t);
         int g = 0;
+        int shared_eps = 0;  // tiles finished by the shared epilogue (phases of B_LX, B_SSX)
         bool ok = true;
         for (int tiles = 0;; ++tiles) {
             const int item = next_item(tiles);
@@ -627,12 +690,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int nkv = steps_of(w), kv0 = kv_first(w);
             const int qrow = w.qt * BM + r;
             const Heads hd = heads_of(w.u, p);
-            // Output head of this warpgroup: both finish head a together in
-            // modes 0 and 1 (64 columns each); in mode 2 each finishes its own.
-            const bool own = p.mode == 2;
+            // Output head of this warpgroup: both finish head a together (64
+            // columns each), except in a pair item, where each finishes its own.
+            const bool own = hd.own;
             const int head = (own && t) ? hd.b : hd.a;
             // The epilogue's lambda (per head, or the token-dependent logit of
-            // this row), gain, gate logits (and in mode 2 the group's noise
+            // this row), gain, gate logits (and in a pair item the group's noise
             // output row): load / prefetch them now so the global-memory
             // latency hides behind the softmax loop.
             const int64_t qrow_c = min(qrow, p.N - 1);
@@ -646,10 +709,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // The group's noise outputs of this tile, stored tile-transposed:
             // float4 chunk c (columns 4c .. 4c + 3) of tile row r at c * 128 + r,
             // so a warp reading chunk c of its 32 rows reads 512 contiguous bytes.
+            const size_t noise_tile = ((size_t)w.b * p.H_N + hd.n) * p.num_qt + w.qt;
             const float4 *an_tile =
-                own ? reinterpret_cast<const float4 *>(p.noise_out) +
-                          (((size_t)w.b * p.H_N + hd.n) * p.num_qt + w.qt) * (HDV / 4) * BM
-                    : nullptr;
+                own ? reinterpret_cast<const float4 *>(p.noise_out) + noise_tile * (HDV / 4) * BM : nullptr;
             float m_run = -INFINITY, l_run = 0.0f;
             for (int j = 0; j < nkv; ++j) {
                 const int gg = g + j, buf = gg & 1;
@@ -670,10 +732,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!ok) break;
             g += nkv;
             if (own) {
-                // ------------------------------------------------ epilogue, mode 2
+                // ------------------------------------------------ epilogue, pair item
                 // This warpgroup's head alone: D = O / l - lambda A_N with A_N
-                // the group's normalised noise output (written by mode 1),
-                // then the RMS norm over the 128 columns of the row.
+                // the group's normalised noise output (written by the tile's
+                // export item), then the RMS norm over the 128 columns of the row.
                 if constexpr (GATED) {  // once the previous store has read this warp's buffer
                     if (elect_one()) {
                         const uint32_t gbuf = sbase + OFF_OUT + (warp - 4) * OUT_WARP_BYTES;
@@ -690,6 +752,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // The gate box (issued above) has had the last P.V's time to land.
                 if (GATED && !(ok = mbar_wait_warp(bar(B_GATE + (warp - 4)), tiles & 1, abort_flag, lim)))
                     break;
+                // The export item of this tile ran about one wave of items
+                // earlier; its eight epilogue warps have normally all
+                // published their half-rows by now.  (Plain L2 loads below: the
+                // data was written during this launch.)
+                bool ready = true;
+                if (lane == 0) ready = wait_flag_geq(p.noise_ready + noise_tile, 8, abort_flag, lim);
+                if (!(ok = __shfl_sync(0xffffffffu, ready, 0))) break;
                 tc_fence_after();
                 const float inv = 1.0f / l_run;
                 const float lam = p.lam_logits ? logistic_fast(lam_in) : lam_in;
@@ -703,7 +772,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tmem_wait_ld();
 #pragma unroll
                     for (int i4 = 0; i4 < 16; ++i4) {
-                        const float4 a4 = __ldg(an_tile + (16 * hh + i4) * BM + r);
+                        const float4 a4 = __ldcg(an_tile + (16 * hh + i4) * BM + r);
                         const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -734,7 +803,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     uint32_t y[32];
 #pragma unroll
                     for (int i4 = 0; i4 < 16; ++i4) {
-                        const float4 a4 = __ldg(an_tile + (16 * hh + i4) * BM + r);
+                        const float4 a4 = __ldcg(an_tile + (16 * hh + i4) * BM + r);
                         const float4 g4 = gain ? __ldg(reinterpret_cast<const float4 *>(gain) + 16 * hh + i4)
                                                : make_float4(1.f, 1.f, 1.f, 1.f);
                         float4 s4 = make_float4(rn, rn, rn, rn);  // norm x output gate
@@ -791,7 +860,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             sL[t * BM + r] = l_run;
             __syncwarp();  // every lane's row sum is written: one arrival for the warp
             if (lane == 0) mbar_arrive(bar(B_LX));
-            if (!(ok = mbar_wait_warp(bar(B_LX), tiles & 1, abort_flag, lim))) break;
+            if (!(ok = mbar_wait_warp(bar(B_LX), shared_eps & 1, abort_flag, lim))) break;
             if (!(ok = mbar_wait_warp(bar(B_O), tiles & 1, abort_flag, lim))) break;
             tc_fence_after();
             const float l1 = sL[r], l2 = sL[BM + r];
@@ -833,12 +902,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (p.mode == 1) {
                 // Export this half of the normalised noise output O2 / l2 for
-                // the group's other signal heads (mode 2), tile-transposed
-                // (chunk c of row r at c * 128 + r: the warp's stores of one
-                // chunk are 512 contiguous bytes).  Rows past N go to the
-                // tile's padding.
-                float4 *an = reinterpret_cast<float4 *>(p.noise_out) +
-                             (((size_t)w.b * p.H_N + hd.n) * p.num_qt + w.qt) * (HDV / 4) * BM +
+                // the group's pair items, tile-transposed (chunk c of row r at
+                // c * 128 + r: the warp's stores of one chunk are 512
+                // contiguous bytes).  Rows past N go to the tile's padding.
+                float4 *an = reinterpret_cast<float4 *>(p.noise_out) + noise_tile * (HDV / 4) * BM +
                              (c0 / 4) * BM + r;
                 const float inv2 = 1.0f / l2;
 #pragma unroll
@@ -849,6 +916,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                                      __uint_as_float(ob[c][4 * i4 + 1]) * inv2,
                                                      __uint_as_float(ob[c][4 * i4 + 2]) * inv2,
                                                      __uint_as_float(ob[c][4 * i4 + 3]) * inv2);
+                // Publish: every lane's stores, then one release per warp (the
+                // pair items wait for all eight warps of the tile).
+                __syncwarp();
+                if (lane == 0) {
+                    __threadfence();
+                    atomicAdd(p.noise_ready + noise_tile, 1);
+                }
             }
             float d[64];
             float ss = 0.0f;
@@ -886,7 +960,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                 }
             }
-            if (!(ok = mbar_wait_warp(bar(B_SSX), tiles & 1, abort_flag, lim))) break;
+            if (!(ok = mbar_wait_warp(bar(B_SSX), shared_eps & 1, abort_flag, lim))) break;
+            ++shared_eps;
             const float rn =
                 p.apply_norm ? rsqrtf((sSS[r] + sSS[BM + r]) * (1.0f / HDV) + p.eps) : 1.0f;
             // Stage this warp's 32 rows x 64 columns in shared memory (the
@@ -931,14 +1006,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
 __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb, int64_t sn,
                                 int64_t sh, __half *__restrict__ dst, int B, int N, int H_V,
-                                int32_t *dev_status, int *tile_counter, const RopeStage rope)
+                                int32_t *dev_status, int *tile_counter, int *zero, int64_t n_zero,
+                                const RopeStage rope)
 {
     // The prefill launch that follows may become resident and run its
     // prologue now; it waits for this kernel to finish before reading.
     grid_launch_dependents();
     // The prefill launches that follow on the stream hand out their work
-    // items from these two counters (one per launch).
+    // items from these two counters (one per launch), and the grouped pairs
+    // count their exports in `zero`.
     if (blockIdx.x == 0 && threadIdx.x < 2) tile_counter[threadIdx.x] = 0;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_zero;
+         i += (int64_t)gridDim.x * blockDim.x)
+        zero[i] = 0;
     // One thread per 8 consecutive V elements (16 bytes in, 16 bytes out).
     // A dense V ([B, N, H_V, 128] with no gaps, the common case) is one flat
     // array, so its chunk i needs no index arithmetic; otherwise chunk i is
@@ -1024,10 +1104,11 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
                            const CUtensorMap &gate, const PrefillParams &p,
                            cudaStream_t stream, int *launches)
 {
-    // Per device: the kernel attribute and the SM count.
+    // Per device, once (first calls from several host threads serialise on
+    // the mutex): the kernel attributes.
     constexpr int kMaxDevices = 64;
-    static bool attr_set[kMaxDevices] = {};
-    static int num_sms[kMaxDevices] = {};
+    static std::atomic<bool> attr_set[kMaxDevices] = {};
+    static std::mutex attr_mutex;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -1035,7 +1116,9 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
         set_internal_error("device ordinal beyond the library's table");
         return cudaErrorInvalidDevice;
     }
-    if (!attr_set[dev]) {
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
+      std::lock_guard<std::mutex> lock(attr_mutex);
+      if (!attr_set[dev].load(std::memory_order_relaxed)) {
         // The register split inside the kernel is only valid for a build that
         // launches with exactly REGS_LAUNCH registers per thread: with fewer,
         // the softmax warpgroups' increase could never be granted.  Refuse to
@@ -1044,7 +1127,10 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
                               (const void *)prefill_kernel<true, false, false>,
                               (const void *)prefill_kernel<false, true, false>,
                               (const void *)prefill_kernel<true, true, false>,
-                              (const void *)prefill_kernel<false, false, true>}) {
+                              (const void *)prefill_kernel<false, false, true>,
+                              (const void *)prefill_kernel<true, false, true>,
+                              (const void *)prefill_kernel<false, true, true>,
+                              (const void *)prefill_kernel<true, true, true>}) {
             cudaFuncAttributes fa;
             e = cudaFuncGetAttributes(&fa, k);
             if (e != cudaSuccess) return e;
@@ -1055,16 +1141,20 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
             e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
             if (e != cudaSuccess) return e;
         }
-        e = cudaDeviceGetAttribute(&num_sms[dev], cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_release);
+      }
     }
-    const int total = p.B * p.units * p.num_qt;
+    const int sms = device_sm_count();
+    const int total = p.B * p.units * p.num_qt * (p.mode == 1 ? p.pairs + 1 : 1);
     if (total == 0) return cudaSuccess;
-    const int grid = total < num_sms[dev] ? total : num_sms[dev];  // persistent: one CTA per SM
-    auto kernel = p.save ? prefill_kernel<false, false, true>
-                  : p.gate ? (p.window > 0 ? prefill_kernel<true, true, false> : prefill_kernel<false, true, false>)
-                           : (p.window > 0 ? prefill_kernel<true, false, false> : prefill_kernel<false, false, false>);
+    const int grid = total < sms ? total : sms;  // persistent: one CTA per SM
+    using Kernel = decltype(&prefill_kernel<false, false, false>);
+    static const Kernel kernels[2][2][2] = {  // [save][gate][window]
+        {{prefill_kernel<false, false, false>, prefill_kernel<true, false, false>},
+         {prefill_kernel<false, true, false>, prefill_kernel<true, true, false>}},
+        {{prefill_kernel<false, false, true>, prefill_kernel<true, false, true>},
+         {prefill_kernel<false, true, true>, prefill_kernel<true, true, true>}}};
+    const Kernel kernel = kernels[p.save != nullptr][p.gate != nullptr][p.window > 0];
     // Programmatic dependent launch: the prologue (barriers, TMEM) overlaps
     // the tail of the kernel before it; the kernel waits (griddepcontrol)
     // before touching that kernel's results.
@@ -1086,16 +1176,17 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
 
 cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, void *dst, int B,
                             int N, int H_V, int32_t *dev_status, int *tile_counter,
-                            const RopeStage &rope, cudaStream_t stream, int *launches)
+                            int *zero, int64_t n_zero, const RopeStage &rope, int sm_count,
+                            cudaStream_t stream, int *launches)
 {
     const int64_t total = (int64_t)B * N * H_V * (HDV / 8);
     if (total == 0) return cudaSuccess;  // nothing to stage; the prefill is skipped too
     const int threads = 256;
     int blocks = (int)((total + threads - 1) / threads);
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks > sm_count * 16) blocks = sm_count * 16;  // grid-stride beyond 16 blocks per SM
     v_to_f16_kernel<<<blocks, threads, 0, stream>>>(static_cast<const __nv_bfloat16 *>(v), sb, sn,
                                                     sh, static_cast<__half *>(dst), B, N, H_V,
-                                                    dev_status, tile_counter, rope);
+                                                    dev_status, tile_counter, zero, n_zero, rope);
     ++*launches;
     return cudaGetLastError();
 }

@@ -93,6 +93,12 @@ class BwdArgs(ctypes.Structure):
         ("grad_k2", _p), ("grad_k2_stride", _S3),
         ("grad_v", _p), ("grad_v_stride", _S3),
         ("grad_lambda", _p), ("grad_gain", _p), ("dev_status", _p),
+        ("H_N", _i64), ("H_V", _i64),
+        ("lambda_logits", _p), ("lambda_logits_stride", _S3),
+        ("gate", _p), ("gate_stride", _S3),
+        ("window", ctypes.c_int32), ("rope_theta", ctypes.c_float),
+        ("grad_lambda_logits", _p), ("grad_lambda_logits_stride", _S3),
+        ("grad_gate", _p), ("grad_gate_stride", _S3),
     ]
 
 
@@ -317,14 +323,16 @@ def diffattn_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, ca
 
 def diffattn_grouped_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,
                          apply_norm=True, out=None, workspace=None, stream=None, timeout_ms=0,
-                         dev_status=None, lam_logits=None, gate=None, window=0, rope_theta=0.0):
+                         dev_status=None, lam_logits=None, gate=None, window=0, rope_theta=0.0,
+                         save=None, test_withhold_load=False):
     """Grouped prefill: q1,k1 [B,N,H,64]; q2,k2 [B,N,H_N,64]; v [B,N,H_V,128];
     signal head h uses noise head h // (H // H_N) and V head h // (H // H_V).
-    lam_logits [B,N,H] and gate [B,N,H,128] as in diffattn_fwd."""
+    lam_logits [B,N,H], gate [B,N,H,128] and save as in diffattn_fwd."""
     return _run_fwd("diffattn_grouped_fwd", q1, q2, k1, k2, v, lam, gain, scale=scale, eps=eps,
                     causal=causal, apply_norm=apply_norm, out=out, workspace=workspace,
                     stream=stream, timeout_ms=timeout_ms, dev_status=dev_status,
-                    lam_logits=lam_logits, gate=gate, window=window, rope_theta=rope_theta)
+                    lam_logits=lam_logits, gate=gate, window=window, rope_theta=rope_theta,
+                    save=save, test_withhold_load=test_withhold_load)
 
 
 def fwd_workspace_size(B, N, H, H_V=None, H_N=None, rope_theta=0.0):
@@ -423,35 +431,41 @@ def fwd_save_size(B, N, H):
     return int(lib().diffattn_fwd_save_size(ctypes.byref(a)))
 
 
-def bwd_workspace_size(B, N, H):
+def bwd_workspace_size(B, N, H, H_N=None, H_V=None, rope_theta=0.0):
     """Workspace bytes of a diffattn_bwd call with these sizes."""
     a = BwdArgs()
     a.B, a.N, a.H, a.d, a.dv = B, N, H, 64, 128
+    a.H_N, a.H_V = H_N or H, H_V or H
+    a.rope_theta = float(rope_theta)
     return int(lib().diffattn_bwd_workspace_size(ctypes.byref(a)))
 
 
 def _bwd_args(q1, q2, k1, k2, v, lam, gain, dout, save, grads, *, scale, eps, causal, apply_norm,
-              timeout_ms, dev_status):
+              timeout_ms, dev_status, lam_logits=None, gate=None, window=0, rope_theta=0.0):
     named = (("q1", q1), ("q2", q2), ("k1", k1), ("k2", k2), ("v", v), ("dout", dout),
              ("grad_q1", grads["dq1"]), ("grad_q2", grads["dq2"]), ("grad_k1", grads["dk1"]),
              ("grad_k2", grads["dk2"]), ("grad_v", grads["dv"]))
     for n, t in named:
         _check_bf16(n, t, 4)
     B, N, H, d = q1.shape
+    H_N, H_V = q2.shape[2], v.shape[2]
+    heads = {"q1": H, "k1": H, "dout": H, "grad_q1": H, "grad_k1": H, "q2": H_N, "k2": H_N,
+             "grad_q2": H_N, "grad_k2": H_N, "v": H_V, "grad_v": H_V}
     for n, t in named:
-        if tuple(t.shape[:3]) != (B, N, H):
-            raise ValueError(f"{n} must be [B, N, H, *] with q1's B, N, H")
+        if tuple(t.shape[:3]) != (B, N, heads[n]):
+            raise ValueError(f"{n} must be [B, N, {heads[n]}, *] (as in the forward call)")
     a = BwdArgs()
     a.B, a.N, a.H, a.d, a.dv = B, N, H, d, v.shape[3]
+    a.H_N, a.H_V = H_N, H_V
     a.scale, a.eps = float(scale), float(eps)
     a.flags = (DIFFATTN_FLAG_CAUSAL if causal else 0) | (DIFFATTN_FLAG_APPLY_NORM if apply_norm else 0)
     a.timeout_ms = int(timeout_ms)
+    a.window = int(window)
+    a.rope_theta = float(rope_theta)
     for n, t in named:
         setattr(a, n, t.data_ptr())
         setattr(a, n + "_stride", _S3(*t.stride()[:3]))
-    if lam is None or lam.dtype != torch.float32 or lam.shape != (H,):
-        raise ValueError("lam must be float32 [H]")
-    a.lambda_ = lam.data_ptr()
+    _set_lambda_gate(a, lam, lam_logits, gate, (B, N, H), a.dv, _S3)
     if gain is not None:
         if gain.dtype != torch.float32 or tuple(gain.shape) != (H, a.dv) or not gain.is_contiguous():
             raise ValueError("gain must be contiguous float32 [H, dv]")
@@ -461,30 +475,54 @@ def _bwd_args(q1, q2, k1, k2, v, lam, gain, dout, save, grads, *, scale, eps, ca
     a.save = save.data_ptr()
     a.grad_lambda = grads["dlam"].data_ptr() if grads.get("dlam") is not None else None
     a.grad_gain = grads["dgain"].data_ptr() if grads.get("dgain") is not None else None
+    if lam_logits is not None and grads.get("dlam_logits") is not None:
+        t = grads["dlam_logits"]
+        if t.dtype != torch.float32 or tuple(t.shape) != (B, N, H):
+            raise ValueError("dlam_logits must be float32 [B, N, H]")
+        a.grad_lambda_logits = t.data_ptr()
+        a.grad_lambda_logits_stride = _S3(*t.stride())
+    if gate is not None and grads.get("dgate") is not None:
+        t = grads["dgate"]
+        _check_bf16("dgate", t, 4)
+        if tuple(t.shape) != (B, N, H, a.dv):
+            raise ValueError("dgate must be bf16 [B, N, H, dv]")
+        a.grad_gate = t.data_ptr()
+        a.grad_gate_stride = _S3(*t.stride()[:3])
     a.dev_status = dev_status.data_ptr() if dev_status is not None else None
     return a
 
 
 def diffattn_bwd(q1, q2, k1, k2, v, lam, gain, dout, save, *, scale=0.125, eps=1e-5, causal=True,
                  apply_norm=True, grads=None, workspace=None, stream=None, timeout_ms=0,
-                 dev_status=None):
-    """Backward pass of diffattn_fwd: gradients of sum(dout * out).
+                 dev_status=None, lam_logits=None, gate=None, window=0, rope_theta=0.0):
+    """Backward pass of diffattn_fwd / diffattn_grouped_fwd: gradients of
+    sum(dout * out).
 
     Inputs as in the forward call that filled `save` (same scale, eps,
-    causal, apply_norm); dout [B,N,H,128] bf16.  Returns a dict: dq1, dq2,
-    dk1, dk2 [B,N,H,64] and dv [B,N,H,128] bf16; dlam [H] and dgain [H,128]
-    fp32.  grads: optional dict of preallocated outputs with those keys."""
+    causal, apply_norm, lam / lam_logits, gate, window, rope_theta); dout
+    [B,N,H,128] bf16.  Returns a dict: dq1, dk1 [B,N,H,64], dq2, dk2
+    [B,N,H_N,64], dv [B,N,H_V,128] bf16; dlam [H] and dgain [H,128] fp32;
+    with lam_logits also dlam_logits [B,N,H] fp32, with a gate dgate
+    [B,N,H,128] bf16.  grads: optional dict of preallocated outputs."""
     B, N, H, d = q1.shape
+    H_N, H_V, dv = q2.shape[2], v.shape[2], v.shape[3]
     dev = q1.device
     if grads is None:
-        grads = {k: torch.empty(B, N, H, d, dtype=torch.bfloat16, device=dev)
-                 for k in ("dq1", "dq2", "dk1", "dk2")}
-        grads["dv"] = torch.empty(B, N, H, v.shape[3], dtype=torch.bfloat16, device=dev)
-        grads["dlam"] = torch.empty(H, dtype=torch.float32, device=dev)
-        grads["dgain"] = torch.empty(H, v.shape[3], dtype=torch.float32, device=dev)
+        grads = {"dq1": torch.empty(B, N, H, d, dtype=torch.bfloat16, device=dev),
+                 "dk1": torch.empty(B, N, H, d, dtype=torch.bfloat16, device=dev),
+                 "dq2": torch.empty(B, N, H_N, d, dtype=torch.bfloat16, device=dev),
+                 "dk2": torch.empty(B, N, H_N, d, dtype=torch.bfloat16, device=dev),
+                 "dv": torch.empty(B, N, H_V, dv, dtype=torch.bfloat16, device=dev),
+                 "dlam": torch.empty(H, dtype=torch.float32, device=dev),
+                 "dgain": torch.empty(H, dv, dtype=torch.float32, device=dev)}
+        if lam_logits is not None:
+            grads["dlam_logits"] = torch.empty(B, N, H, dtype=torch.float32, device=dev)
+        if gate is not None:
+            grads["dgate"] = torch.empty(B, N, H, dv, dtype=torch.bfloat16, device=dev)
     a = _bwd_args(q1, q2, k1, k2, v, lam, gain, dout, save, grads, scale=scale, eps=eps,
                   causal=causal, apply_norm=apply_norm, timeout_ms=timeout_ms,
-                  dev_status=dev_status)
+                  dev_status=dev_status, lam_logits=lam_logits, gate=gate, window=window,
+                  rope_theta=rope_theta)
     L = lib()
     need = L.diffattn_bwd_workspace_size(ctypes.byref(a))
     if workspace is None:
@@ -497,33 +535,44 @@ def diffattn_bwd(q1, q2, k1, k2, v, lam, gain, dout, save, *, scale=0.125, eps=1
 
 class DiffAttention(torch.autograd.Function):
     """Differential attention as an autograd function: the forward runs
-    diffattn_fwd with the saved state, the backward runs diffattn_bwd."""
+    diffattn_fwd (diffattn_grouped_fwd with shared noise or V heads) with the
+    saved state, the backward runs diffattn_bwd."""
 
     @staticmethod
-    def forward(ctx, q1, q2, k1, k2, v, lam, gain, scale, eps, causal, apply_norm):
+    def forward(ctx, q1, q2, k1, k2, v, lam, gain, lam_logits, gate, scale, eps, causal, apply_norm,
+                window, rope_theta):
         B, N, H, _ = q1.shape
         save = torch.empty(max(fwd_save_size(B, N, H), 16), dtype=torch.uint8, device=q1.device)
-        out = diffattn_fwd(q1, q2, k1, k2, v, lam, gain, scale=scale, eps=eps, causal=causal,
-                           apply_norm=apply_norm, save=save)
-        ctx.save_for_backward(q1, q2, k1, k2, v, lam, gain, save)
-        ctx.cfg = (scale, eps, causal, apply_norm)
+        grouped = q2.shape[2] != H or v.shape[2] != H
+        f = diffattn_grouped_fwd if grouped else diffattn_fwd
+        out = f(q1, q2, k1, k2, v, lam, gain, scale=scale, eps=eps, causal=causal,
+                apply_norm=apply_norm, save=save, lam_logits=lam_logits, gate=gate, window=window,
+                rope_theta=rope_theta)
+        ctx.save_for_backward(q1, q2, k1, k2, v, lam, gain, lam_logits, gate, save)
+        ctx.cfg = (scale, eps, causal, apply_norm, window, rope_theta)
         return out
 
     @staticmethod
     def backward(ctx, dout):
-        q1, q2, k1, k2, v, lam, gain, save = ctx.saved_tensors
-        scale, eps, causal, apply_norm = ctx.cfg
+        q1, q2, k1, k2, v, lam, gain, lam_logits, gate, save = ctx.saved_tensors
+        scale, eps, causal, apply_norm, window, rope_theta = ctx.cfg
         dout = dout.to(torch.bfloat16)
         if dout.stride(-1) != 1:
             dout = dout.contiguous()
         g = diffattn_bwd(q1, q2, k1, k2, v, lam, gain, dout, save, scale=scale, eps=eps,
-                         causal=causal, apply_norm=apply_norm)
+                         causal=causal, apply_norm=apply_norm, lam_logits=lam_logits, gate=gate,
+                         window=window, rope_theta=rope_theta)
+        dlam = g["dlam"] if lam is not None else None
         dgain = g["dgain"] if gain is not None else None
-        return g["dq1"], g["dq2"], g["dk1"], g["dk2"], g["dv"], g["dlam"], dgain, None, None, None, None
+        return (g["dq1"], g["dq2"], g["dk1"], g["dk2"], g["dv"], dlam, dgain, g.get("dlam_logits"),
+                g.get("dgate"), None, None, None, None, None, None)
 
 
 def diff_attention(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=1e-5, causal=True,
-                   apply_norm=True):
-    """Differentiable differential attention (bf16 q/k/v [B,N,H,64|128], fp32
-    lam [H] and gain [H,128]); gradients flow to every tensor input."""
-    return DiffAttention.apply(q1, q2, k1, k2, v, lam, gain, scale, eps, causal, apply_norm)
+                   apply_norm=True, lam_logits=None, gate=None, window=0, rope_theta=0.0):
+    """Differentiable differential attention (bf16 q1, k1 [B,N,H,64], q2, k2
+    [B,N,H_N,64], v [B,N,H_V,128]; fp32 lam [H] and gain [H,128]; optional
+    lambda logits fp32 [B,N,H], gate logits bf16 [B,N,H,128], a causal
+    window, a rotary base); gradients flow to every tensor input."""
+    return DiffAttention.apply(q1, q2, k1, k2, v, lam, gain, lam_logits, gate, scale, eps, causal,
+                               apply_norm, window, rope_theta)

@@ -122,9 +122,9 @@ typedef struct diffattn_fwd_args {
      * normalised map output A_t = softmax(scale Q_t K_t^T) V (fp32) and the
      * base-2 log of the row's softmax denominator.  Its layout is private to
      * the library; it stays valid until the caller reuses the memory.
-     * Supported for diffattn_fwd (H_N == H_V == H) with per-head lambda and
-     * no lambda_logits, gate, window or rope_theta; other combinations
-     * return DIFFATTN_ERR_UNSUPPORTED.                                       */
+     * Every option of the forward call can save.  A grouped call that saves
+     * computes each noise map once per signal head (the state is per signal
+     * head), not once per group.                                            */
     void *save;
 } diffattn_fwd_args;
 
@@ -150,29 +150,43 @@ size_t diffattn_fwd_workspace_size(const diffattn_fwd_args *args);
  * an empty problem).                                                        */
 size_t diffattn_fwd_save_size(const diffattn_fwd_args *args);
 
-/* Backward pass of diffattn_fwd: the gradients of sum(dout * out) with
- * respect to q1, q2, k1, k2, v, lambda and gain.  The pages define the
- * forward pass only (Motif 2.6B explainer, section "Differential attention";
- * the model is trained with it, same page, "A schedule for the data"), so
- * this is its exact gradient:
+/* Backward pass of diffattn_fwd / diffattn_grouped_fwd: the gradients of
+ * sum(dout * out) with respect to q1, q2, k1, k2, v, lambda (or the lambda
+ * logits), gain and the gate logits.  The pages define the forward pass only
+ * (Motif 2.6B explainer, section "Differential attention"; the model is
+ * trained with it, same page, "A schedule for the data"), so this is its
+ * exact gradient.  With lambda_i the row's lambda, Yn the output before the
+ * gate and r = (mean_c D^2 + eps)^-1/2:
  *
- *   dgain = sum_i dY D r,  dD = r (dY gain) - (r^3 / dv) D sum_c(dY gain D)
- *   dA_1 = dD, dA_2 = -lambda dD, dlambda = -sum dD A_2
+ *   dYn = dY sigma(G), dG = dY Yn sigma(G) (1 - sigma(G))   (no gate: dYn = dY)
+ *   dgain = sum_i dYn D r,  dD = r (dYn gain) - (r^3 / dv) D sum_c(dYn gain D)
+ *   dA_1 = dD, dA_2 = -lambda_i dD, dlambda_i = -sum_c dD A_2
  *   per map: dP = dA_t V^T, dS = P (dP - rowsum(dA_t A_t)),
  *            dQ_t = scale dS K_t, dK_t = scale dS^T Q_t, dV += P^T dA_t
  *
- * (r = (mean_c D^2 + eps)^-1/2; without DIFFATTN_FLAG_APPLY_NORM, dD = dY and
- * dgain = 0).  Inputs are those of the forward call that filled `save`, with
- * the same B, N, H, scale, eps and flags.  Layouts as in the forward:
- *   q1, q2, k1, k2, grad_q1, grad_q2, grad_k1, grad_k2: [B, N, H, 64] bf16
- *   v, dout, grad_v: [B, N, H, 128] bf16
- *   lambda: [H] fp32 device; gain: [H, 128] fp32 device or NULL for 1.
+ * (without DIFFATTN_FLAG_APPLY_NORM, dD = dYn and dgain = 0; with lambda
+ * logits, dlogit_i = dlambda_i sigma'(logit_i) and grad_lambda = 0; with a
+ * window, the masked pairs take no part; with rope_theta, the products use
+ * the rotated Q/K and dQ, dK are rotated back).  Grouped heads (H_N, H_V as
+ * in the forward) sum the gradients of a shared noise or V head over its
+ * signal heads.  Inputs are those of the forward call that filled `save`,
+ * with the same sizes, scale, eps, flags, lambda / logits, gate, window and
+ * rope_theta.  Layouts as in the forward:
+ *   q1, k1, grad_q1, grad_k1: [B, N, H, 64] bf16
+ *   q2, k2, grad_q2, grad_k2: [B, N, H_N, 64] bf16
+ *   v, grad_v: [B, N, H_V, 128] bf16;  dout: [B, N, H, 128] bf16
+ *   lambda: [H] fp32 device (or NULL with lambda_logits); gain: [H, 128]
+ *   fp32 device or NULL for 1.
  *   grad_lambda: [H] fp32 device or NULL; grad_gain: [H, 128] fp32 device,
  *   contiguous, or NULL.
+ *   lambda_logits / grad_lambda_logits: [B, N, H] fp32 (any strides), or
+ *   NULL; gate / grad_gate: [B, N, H, 128] bf16 laid out like dout, or NULL.
  * Every gradient is overwritten, not accumulated into.  Intermediate
  * quantities beyond the fp16 range (the normalised-output gradient dD is
- * staged in fp16 for the tensor cores) report DIFFATTN_ERR_UNSUPPORTED in
- * dev_status.                                                               */
+ * staged in fp16 for the tensor cores, and with rope_theta so are the score
+ * gradients) report DIFFATTN_ERR_UNSUPPORTED in dev_status; the kernels
+ * still run to the end, and every gradient of such a call is undefined (it
+ * may hold inf or NaN).  Check dev_status before using the gradients.       */
 typedef struct diffattn_bwd_args {
     int64_t B, N, H;
     int64_t d, dv;
@@ -196,13 +210,21 @@ typedef struct diffattn_bwd_args {
     float *grad_lambda;
     float *grad_gain;
     int32_t *dev_status;
+    int64_t H_N, H_V;       /* noise / V heads; 0 means H */
+    const float *lambda_logits; int64_t lambda_logits_stride[3];
+    const void *gate;           int64_t gate_stride[3];
+    int32_t window;             /* as in the forward call; 0 = none */
+    float rope_theta;           /* as in the forward call; 0 = none */
+    float *grad_lambda_logits;  int64_t grad_lambda_logits_stride[3];
+    void *grad_gate;            int64_t grad_gate_stride[3];
 } diffattn_bwd_args;
 
 diffattn_status diffattn_bwd(const diffattn_bwd_args *args, void *workspace, size_t ws_bytes,
                              void *stream);
 
-/* Workspace bytes of diffattn_bwd (fp16 copies of V and of dD, and per-row
- * statistics).                                                              */
+/* Workspace bytes of diffattn_bwd (fp16 copies of V and of dD, per-row
+ * statistics, and depending on the arguments the rotated copies of Q1, K1,
+ * Q2, K2 and fp32 sums of the gradients of shared noise and V heads).      */
 size_t diffattn_bwd_workspace_size(const diffattn_bwd_args *args);
 
 /* Host-only argument check of a prefill call: the status diffattn_fwd (or,
@@ -260,8 +282,11 @@ diffattn_status diffattn_decode(const diffattn_decode_args *args, void *workspac
  * that loads the library holds it until the process exits).
  *  - Sizes whose partials (diffattn_decode_workspace_size) exceed that array
  *    return DIFFATTN_ERR_WORKSPACE; diffattn_last_error() says by how much.
- *  - The first call on a device looks up the array's device address; make
- *    that first call before any stream capture.
+ *  - The first call on a device looks up the array's device address and
+ *    keeps it for the rest of the process; make that first call before any
+ *    stream capture.  The kept address dies with the device's context: after
+ *    cudaDeviceReset (or anything else that destroys and recreates the
+ *    primary context) do not call this entry point on that device again.
  *  - Every call on a device shares the one array and leaves its partials
  *    there; nothing in it has to start at zero.  Calls that overlap on the
  *    GPU (other streams, other host threads) race on it: serialise them.
@@ -273,7 +298,8 @@ diffattn_status diffattn_decode_noalloc(const diffattn_decode_args *args, void *
  * count diffattn_decode picks).                                              */
 size_t diffattn_decode_workspace_size(int64_t B, int64_t H, int64_t L, int32_t num_splits);
 
-/* The split count diffattn_decode uses for these sizes.                     */
+/* The split count diffattn_decode uses for these sizes (chosen for about
+ * four CTAs per SM of the current device).                                   */
 int32_t diffattn_decode_num_splits(int64_t B, int64_t H, int64_t L, int32_t num_splits);
 
 /* Host-only argument check of a decode call (workspace check skipped).      */

@@ -126,10 +126,10 @@ def test_fwd_rejects_before_launch(L):
     assert L.diffattn_grouped_fwd(ctypes.byref(_fake_fwd_args(H=6, H_N=4)), None, 0, None) == 1
     # groups of 3 signal heads sharing one V head also hold the exported
     # noise outputs (fp32, whole 128-row query tiles: 300 rows take 3) in the
-    # workspace
+    # workspace, then one ready count per (b, noise head, tile), 256-B aligned
     g = _fake_fwd_args(H=24, H_N=8, H_V=8)
     assert L.diffattn_fwd_workspace_size(ctypes.byref(g)) == (2 * 300 * 8 * 128 * 2 + 256
-                                                             + 2 * 8 * 3 * 128 * 128 * 4)
+                                                             + 2 * 8 * 3 * 128 * 128 * 4 + 256)
     g = _fake_fwd_args(H=24, H_N=8, H_V=24)
     assert L.diffattn_fwd_workspace_size(ctypes.byref(g)) == 2 * 300 * 24 * 128 * 2 + 256
 
@@ -270,15 +270,27 @@ def test_bwd_rejects_before_launch(L):
     b = lambda a, ws=None, n=0: L.diffattn_bwd(ctypes.byref(a), ws, n, None)
     a = _fake_bwd_args()
     need = L.diffattn_bwd_workspace_size(ctypes.byref(a))
-    # fp16 copies of V and dD, then [B, H, 4, 3 tiles * 128] fp32 statistics, then 256 B
-    assert need == 2 * (2 * 300 * 4 * 128 * 2) + 2 * 4 * 4 * 384 * 4 + 256
+    # fp16 copies of V and dD, then [B, H, 5, 3 tiles * 128] fp32 statistics, then 256 B
+    assert need == 2 * (2 * 300 * 4 * 128 * 2) + 2 * 4 * 5 * 384 * 4 + 256
+    # grouped heads add fp32 sums of the shared heads' gradients: dK2 and dQ2
+    # [B, N, H_N, 64], dV [B, N, H_V, 128]; rope_theta the rotated fp16 copies
+    g = _fake_bwd_args()
+    g.H_N, g.H_V = 2, 2
+    assert L.diffattn_bwd_workspace_size(ctypes.byref(g)) == (
+        300 * 2 * 2 * 128 * 2 + 2 * 300 * 4 * 128 * 2 + 2 * 4 * 5 * 384 * 4 + 256
+        + 2 * (2 * 300 * 2 * 64 * 4) + 2 * 300 * 2 * 128 * 4)
+    g = _fake_bwd_args()
+    g.rope_theta = 1e4
+    assert L.diffattn_bwd_workspace_size(ctypes.byref(g)) == need + 4 * (2 * 300 * 4 * 64 * 2)
     assert b(a) == 4                                               # workspace missing
     assert b(a, ctypes.c_void_p(1 << 30), need - 1) == 4
     assert b(a, ctypes.c_void_p((1 << 30) + 16), need) == 3         # workspace not 256-aligned
     for field, value, code in (("d", 32, 2), ("dv", 64, 2), ("save", 0, 1), ("dout", 0, 1),
                                ("grad_v", 0, 1), ("lambda_", 0, 1), ("grad_k2", (1 << 20) + 8, 3),
                                ("save", (1 << 20) + 4, 3), ("grad_gain", (1 << 20) + 2, 3),
-                               ("flags", 8, 1), ("scale", 0.0, 1)):
+                               ("flags", 8, 1), ("scale", 0.0, 1), ("H_N", 3, 1), ("H_V", -1, 1),
+                               ("window", -1, 1), ("grad_gate", 1 << 27, 1),
+                               ("lambda_logits", (1 << 20) + 2, 3)):
         a = _fake_bwd_args()
         setattr(a, field, value)
         assert b(a, ctypes.c_void_p(1 << 30), need) == code, field
@@ -302,7 +314,9 @@ def test_fwd_save_size_and_support(L):
         setattr(a, field, value)
         if field == "gate":
             a.gate_stride = ops._S3(300 * 4 * 128, 4 * 128, 128)
-        assert _v(L, a) == 2, field                                # no saved state for these
+        assert _v(L, a) == 0, field                                # every option saves
     g = _fake_fwd_args(H=24, H_N=8, H_V=8)
+    ws = L.diffattn_fwd_workspace_size(ctypes.byref(g))
     g.save = 1 << 28
-    assert _v(L, g, 1) == 2                                        # nor for grouped heads
+    assert _v(L, g, 1) == 0                                        # grouped heads too,
+    assert L.diffattn_fwd_workspace_size(ctypes.byref(g)) < ws     # one signal head per item

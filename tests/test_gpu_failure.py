@@ -37,3 +37,29 @@ def test_withheld_load_reports_timeout_and_device_stays_usable(cuda_ok):
                          scale=0.125, eps=1e-5)
     err = np.abs(y.float().cpu().double().numpy() - ref)
     assert err.max() <= 2e-2 and err.mean() <= 2e-3
+
+
+def test_grouped_pairs_time_out_together_and_device_stays_usable(cuda_ok):
+    """Grouped pairs in one launch: pair items wait (bounded) for their
+    tile's export item.  With every CTA's first load withheld, export items
+    never publish, so the pair items' waits run out too; the call reports
+    DIFFATTN_ERR_TIMEOUT, stores nothing, and the next call is correct."""
+    x = inputs.prefill_inputs(2, 300, 6, 2, 2, seed=12, gain_std=0.1)
+    d = {k: v.cuda() for k, v in x.items()}
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.zeros(2, 300, 6, 128, dtype=torch.bfloat16, device="cuda")
+    ops.diffattn_grouped_fwd(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"],
+                             out=out, dev_status=st, timeout_ms=50, test_withhold_load=True)
+    torch.cuda.synchronize()
+    assert st.item() == 6  # DIFFATTN_ERR_TIMEOUT
+    assert torch.count_nonzero(out).item() == 0
+
+    st.zero_()
+    y = ops.diffattn_grouped_fwd(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"],
+                                 dev_status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    ref = oracle.prefill(x["q1"], x["q2"], x["k1"], x["k2"], x["v"], x["lam"], x["gain"],
+                         scale=0.125, eps=1e-5)
+    err = np.abs(y.float().cpu().double().numpy() - ref)
+    assert err.max() <= 2e-2 and err.mean() <= 2e-3

@@ -70,17 +70,13 @@ def test_window_requires_causal(cuda_ok):
         _run(x, 16, causal=False)
 
 
-def test_window_full_size_sampled(cuda_ok):
+def test_window_workload_full(cuda_ok):
     """The sliding-window workload (1 x 16384, 16 heads, W = 128) in the
-    benchmark's launch configuration, checked on sampled rows."""
+    benchmark's launch configuration, every element against the oracle."""
     w = inputs.WORKLOADS["swa16k"]
     x = inputs.workload_inputs(w)
     y = _run(x, w.window)
-    rows = inputs.sample_rows(w.B, w.N, w.H, 150, seed=w.seed)
-    b, i, h = rows[:, 0], rows[:, 1], rows[:, 2]
-    ref = _oracle(x, w.window, rows=rows)[b.numpy(), i.numpy(), h.numpy()]
-    _check(y[b.cuda(), i.cuda(), h.cuda()], ref)
-    assert torch.isfinite(y.float()).all()
+    _check(y, _oracle(x, w.window))
 
 
 @pytest.mark.parametrize("W", [1, 100, 2048, 3000, 10000])

@@ -7,13 +7,16 @@ with no allocator handle to take a workspace from.  diffattn_decode_noalloc
 serves them by keeping the decode's per-split partial states in a fixed
 static device array inside the library.  This test calls it through the C ABI
 twice in a row, with different inputs and split counts, and checks each
-result against diffattn_decode (which uses a caller-owned workspace) within
-the parity tolerance of the other GPU tests.  It lives in its own file that
+result against diffattn_decode (which uses a caller-owned workspace) and
+against the float64 oracle, within the parity tolerance of the other GPU
+tests.  It lives in its own file that
 sorts last, so a run stopping at the first failure has run everything else.
 """
+import numpy as np
 import pytest
 import torch
 
+import oracle
 from differential_attention_07_b200 import inputs, ops
 
 pytestmark = pytest.mark.gpu
@@ -40,10 +43,17 @@ def test_noalloc_decode_matches_workspace_decode_twice(cuda_ok):
     got1, ref1 = _both(x1, 0)
     x2 = inputs.decode_inputs(3, 777, 2, seed=456, gain_std=0.1)
     got2, ref2 = _both(x2, 5, kv_len=torch.tensor([777, 1, 400], dtype=torch.int32))
-    for got, ref in ((got1, ref1), (got2, ref2)):
+    kv2 = torch.tensor([777, 1, 400], dtype=torch.int32)
+    exact1 = oracle.decode(x1["q1"], x1["q2"], x1["k1"], x1["k2"], x1["v"], x1["lam"], x1["gain"],
+                           scale=0.125, eps=1e-5)
+    exact2 = oracle.decode(x2["q1"], x2["q2"], x2["k1"], x2["k2"], x2["v"], x2["lam"], x2["gain"],
+                           kv_len=kv2, scale=0.125, eps=1e-5)
+    for got, ref, exact in ((got1, ref1, exact1), (got2, ref2, exact2)):
         assert torch.isfinite(got).all()
         err = (got - ref).abs()
         assert err.max().item() <= 2e-2 and err.mean().item() <= 2e-3
+        e64 = np.abs(got.cpu().double().numpy() - exact)
+        assert e64.max() <= 2e-2 and e64.mean() <= 2e-3, (e64.max(), e64.mean())
 
 
 def test_noalloc_decode_rejects_sizes_beyond_its_scratch(cuda_ok):
