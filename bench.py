@@ -20,13 +20,17 @@ kernel.  Rank 0 prints one JSON line:
                with token-dependent lambda and output gate, no norm: Motif 3
                summary, section 2.2), sliding window (1 x 16384, W = 128),
                RoPE (the 4K shape, theta = 500,000), the backward pass of the
-               4K shape (1280 FLOP per pair; also the saving forward and a
-               training step of both), decode (batch 64, 8192 cached keys;
-               GB/s against the measured HBM copy bandwidth).
+               4K shape and of the gated grouped shape (1280 FLOP per pair per
+               signal head; also the saving forward and a training step of
+               both), decode (batch 64, 8192 cached keys; GB/s against the
+               measured HBM copy bandwidth).
 
 With more than one GPU (torchrun) every rank runs its own batch of the same
-shape (weak scaling; the path has no exchange step) and the time is the max
-over ranks.  `--impl reference` times the oracle itself on the host cores.
+shape by default (weak scaling; the path has no exchange step); `--shard
+batch|heads` instead splits one global problem by batch entries or by
+(whole groups of) heads through strided views, and `--gather` assembles the
+output afterwards.  The time is the max over ranks.  `--impl reference`
+times the oracle itself on the host cores.
 """
 import argparse
 import json
@@ -49,6 +53,24 @@ FLOP_PER_PAIR = 768  # 2*64 + 2*64 (two QK^T) + 2*128 + 2*128 (two P.V)
 # P_2)^T dD (2*128, shared), dK_1, dK_2, dQ_1, dQ_2 (2*64 each).  The kernels
 # execute 1792: the query-tile kernel recomputes both score maps and dP.
 BWD_FLOP_PER_PAIR = 1280
+# Timed steps of each secondary workload: at least 20 steps and about 25 ms
+# of device time (the grouped prefill takes about 0.25 ms a step, the 16K
+# prefill 1.6 ms).
+EXTRA_STEPS = 20
+EXTRA_SECONDS = 0.025
+
+
+def extra_steps(call, device, minimum=EXTRA_STEPS):
+    """Steps for a secondary workload: one untimed call sizes the loop to
+    about EXTRA_SECONDS of device time, at least `minimum` steps."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    call()
+    e0.record()
+    call()
+    e1.record()
+    torch.cuda.synchronize(device)
+    t = max(e0.elapsed_time(e1) / 1e3, 1e-6)
+    return max(minimum, int(EXTRA_SECONDS / t + 0.999))
 
 
 def causal_pairs(N, window=0):
@@ -151,6 +173,88 @@ def aggregate_throughput(units_per_rank, elapsed_s_local, device, world):
     """Whole-job throughput: every rank's units over the slowest rank's time."""
     t = max_over_ranks(elapsed_s_local, device)
     return units_per_rank * world / t, t
+
+
+def sum_over_ranks(x, device):
+    """Sum of a float over ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ partition
+SHARD_MODES = ("replica", "batch", "heads")
+
+
+def shard_plan(w, world, rank, mode):
+    """The part of a workload that `rank` of `world` computes.
+
+    * replica: the whole workload, on inputs of the rank's own seed (every
+      rank one independent problem: weak scaling);
+    * batch: batch entries [b0, b1) of one global problem;
+    * heads: heads of one global problem, whole groups at a time: noise heads
+      [n0, n1), their signal heads [h0, h1) and V heads [v0, v1).  A group
+      is the least run of signal heads that owns whole noise and V heads
+      (lcm of H / H_N and H / H_V signal heads).
+
+    Every (b, signal head) of the global problem falls to exactly one rank
+    in the batch and heads modes; the work (b, h) units need no exchange.
+    Returns a dict of the index ranges (empty ranges when a rank gets no
+    work)."""
+    import math
+    g_n, g_v = w.H // w.H_N, w.H // w.H_V
+    full = dict(b0=0, b1=w.B, h0=0, h1=w.H, n0=0, n1=w.H_N, v0=0, v1=w.H_V)
+    if mode == "replica" or world == 1:
+        return full
+    if mode == "batch":
+        return {**full, "b0": rank * w.B // world, "b1": (rank + 1) * w.B // world}
+    if mode != "heads":
+        raise ValueError(mode)
+    unit = g_n * g_v // math.gcd(g_n, g_v)
+    units = w.H // unit
+    u0, u1 = rank * units // world, (rank + 1) * units // world
+    h0, h1 = u0 * unit, u1 * unit
+    return {**full, "h0": h0, "h1": h1, "n0": h0 // g_n, "n1": h1 // g_n,
+            "v0": h0 // g_v, "v1": h1 // g_v}
+
+
+def shard_inputs(x, plan):
+    """Views of a workload's [B, N, heads, dim] tensors (and the per-head
+    lambda / gain, per-token logits and gate) restricted to a shard plan.
+    The views keep the global tensors' strides."""
+    b = slice(plan["b0"], plan["b1"])
+    sig, noise, vh = (slice(plan["h0"], plan["h1"]), slice(plan["n0"], plan["n1"]),
+                      slice(plan["v0"], plan["v1"]))
+    heads = {"q1": sig, "k1": sig, "q2": noise, "k2": noise, "v": vh, "lam_logits": sig, "gate": sig}
+    out = {}
+    for k, t in x.items():
+        if t is None:
+            out[k] = None
+        elif k in ("lam", "gain"):
+            out[k] = t[sig]
+        else:
+            out[k] = t[b, :, heads[k]]
+    return out
+
+
+def shard_work(w, plan):
+    """The workload restricted to a shard (for its FLOP count)."""
+    import dataclasses
+    return dataclasses.replace(w, B=plan["b1"] - plan["b0"], H=plan["h1"] - plan["h0"],
+                               H_N=max(1, plan["n1"] - plan["n0"]), H_V=max(1, plan["v1"] - plan["v0"]))
+
+
+def gather_output(out_full, device):
+    """Assemble the ranks' output slices: each rank holds the global output
+    layout with only its own slice written and zeros elsewhere, so a sum over
+    ranks is the unsharded output exactly.  Runs outside the timed region."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.all_reduce(out_full, op=dist.ReduceOp.SUM)
+    return out_full
 
 
 # ------------------------------------------------------------------ clocks
@@ -298,33 +402,49 @@ def to_dev(x, device):
     return {k: v.to(device, non_blocking=True) for k, v in x.items()}
 
 
-def run_prefill_workload(w, steps, warmup, device, ops, rank=0, clocks=None):
-    x = inputs.workload_inputs(inputs.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}))
-    d = to_dev(x, device)
+def run_prefill_workload(w, steps, warmup, device, ops, rank=0, clocks=None, plan=None,
+                         shard="replica"):
+    """Time the prefill of workload w.  With a shard plan (batch or heads
+    mode) every rank draws the same global inputs and computes its slice of
+    them through strided views, writing its slice of a global output."""
+    seed = w.seed + 1000 * rank if shard == "replica" else w.seed
+    x = inputs.workload_inputs(inputs.Workload(**{**w.__dict__, "seed": seed}))
+    d_full = to_dev(x, device)
+    plan = plan or shard_plan(w, 1, 0, "replica")
+    d = shard_inputs(d_full, plan)
+    sw = shard_work(w, plan)
+    empty = plan["b1"] <= plan["b0"] or plan["h1"] <= plan["h0"]
     grouped = w.kind == "grouped"
     f = ops.diffattn_grouped_fwd if grouped else ops.diffattn_fwd
-    out = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=device)
-    ws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H, w.H_V, w.H_N, w.rope_theta), dtype=torch.uint8, device=device)
+    out_full = torch.zeros(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=device)
+    out = out_full[plan["b0"]:plan["b1"], :, plan["h0"]:plan["h1"]]
+    ws = torch.empty(max(1, ops.fwd_workspace_size(sw.B, sw.N, sw.H, sw.H_V, sw.H_N, sw.rope_theta)
+                         if not empty else 1), dtype=torch.uint8, device=device)
     status = torch.zeros(1, dtype=torch.int32, device=device)
 
     def call():
+        if empty:
+            return
         f(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"], scale=w.scale, eps=w.eps,
           causal=w.causal, apply_norm=w.apply_norm, out=out, workspace=ws, dev_status=status,
           window=w.window, rope_theta=w.rope_theta,
           lam_logits=d.get("lam_logits"), gate=d.get("gate"))
 
     call()
-    launches = ops.last_launch_count()
+    launches = ops.last_launch_count() if not empty else 0
+    if steps is None:
+        steps = extra_steps(call, device)
     t = time_loop(call, steps, warmup, device, clocks=clocks)
-    tk = kernel_time(call, max(3, min(steps, 20)), ops)
+    tk = kernel_time(call, max(3, steps), ops)
     torch.cuda.synchronize(device)
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()} in {w.name}")
-    return dict(step_s=t / steps, kernel_s=tk, launches=launches, x=x, d=d, call=call, out=out,
-                ws=ws, f=f)
+    return dict(step_s=t / steps, kernel_s=tk, launches=launches, steps=steps, x=shard_inputs(x, plan), d=d,
+                call=call, out=out, out_full=out_full, ws=ws, f=f, work=sw, empty=empty,
+                flops=0 if empty else prefill_flops(sw))
 
 
-def run_decode_workload(w, steps, warmup, device, ops):
+def run_decode_workload(w, steps, warmup, device, ops, clocks=None):
     x = inputs.workload_inputs(w)
     d = to_dev(x, device)
     out = torch.empty(w.B, w.H, w.dv, dtype=torch.bfloat16, device=device)
@@ -336,9 +456,11 @@ def run_decode_workload(w, steps, warmup, device, ops):
 
     call()
     launches = ops.last_launch_count()
-    t = time_loop(call, steps, warmup, device)
-    tk = kernel_time(call, max(3, min(steps, 20)), ops)
-    return dict(step_s=t / steps, kernel_s=tk, launches=launches)
+    if steps is None:
+        steps = extra_steps(call, device)
+    t = time_loop(call, steps, warmup, device, clocks=clocks)
+    tk = kernel_time(call, max(3, steps), ops)
+    return dict(step_s=t / steps, kernel_s=tk, launches=launches, steps=steps)
 
 
 def e2e_prefill(w, steps, warmup, device, ops, x):
@@ -349,8 +471,8 @@ def e2e_prefill(w, steps, warmup, device, ops, x):
     serving loop would use the call: entry b's inputs are copied in while
     entry b-1 is computed and entry b-2's output is copied out.  Copies and
     calls of one step never overlap the next step's."""
-    host = {k: v.pin_memory() for k, v in x.items()}
-    dev = {k: torch.empty_like(v, device=device) for k, v in x.items()}
+    host = {k: v.contiguous().pin_memory() for k, v in x.items() if v is not None}
+    dev = {k: torch.empty_like(v, device=device) for k, v in host.items()}
     out = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=device)
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     ws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H, w.H_V, w.H_N, w.rope_theta), dtype=torch.uint8, device=device)
@@ -392,40 +514,70 @@ def e2e_prefill(w, steps, warmup, device, ops, x):
     return t / steps, h2d, d2h
 
 
-def run_backward_workload(w, steps, warmup, device, ops):
-    """Time diffattn_bwd (and the forward that saves its state) on workload w."""
+def run_backward_workload(w, steps, warmup, device, ops, clocks=None):
+    """Time diffattn_bwd (and the forward that saves its state) on workload w
+    (any of its options: grouped heads, token lambda, gate, window, RoPE)."""
     x = inputs.workload_inputs(w)
     d = to_dev(x, device)
     dy = inputs.grad_output(w.B, w.N, w.H, w.dv, seed=w.seed).to(device)
     save = torch.empty(ops.fwd_save_size(w.B, w.N, w.H), dtype=torch.uint8, device=device)
     out = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=device)
-    fws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H), dtype=torch.uint8, device=device)
     status = torch.zeros(1, dtype=torch.int32, device=device)
+    f = ops.diffattn_grouped_fwd if w.kind == "grouped" else ops.diffattn_fwd
+    opts = dict(lam_logits=d.get("lam_logits"), gate=d.get("gate"), window=w.window,
+                rope_theta=w.rope_theta)
+    fws = torch.empty(1, dtype=torch.uint8, device=device)
 
     def fwd():
-        ops.diffattn_fwd(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"],
-                         scale=w.scale, eps=w.eps, causal=w.causal, out=out, workspace=fws,
-                         save=save, dev_status=status)
+        f(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"], scale=w.scale, eps=w.eps,
+          causal=w.causal, apply_norm=w.apply_norm, out=out, workspace=fws, save=save,
+          dev_status=status, **opts)
 
+    # the saving forward's workspace (a grouped call that saves needs no noise outputs)
+    a = ops._fwd_args(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"], out,
+                      scale=w.scale, eps=w.eps, causal=w.causal, apply_norm=w.apply_norm,
+                      timeout_ms=0, dev_status=None, save=save, **opts)
+    fws = torch.empty(max(1, ops.lib().diffattn_fwd_workspace_size(ops.ctypes.byref(a))),
+                      dtype=torch.uint8, device=device)
     fwd()
     grads = ops.diffattn_bwd(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"], dy,
-                             save, scale=w.scale, eps=w.eps, causal=w.causal, dev_status=status)
-    bws = torch.empty(ops.bwd_workspace_size(w.B, w.N, w.H), dtype=torch.uint8, device=device)
+                             save, scale=w.scale, eps=w.eps, causal=w.causal,
+                             apply_norm=w.apply_norm, dev_status=status, **opts)
+    bws = torch.empty(ops.bwd_workspace_size(w.B, w.N, w.H, w.H_N, w.H_V, w.rope_theta),
+                      dtype=torch.uint8, device=device)
 
     def bwd():
         ops.diffattn_bwd(d["q1"], d["q2"], d["k1"], d["k2"], d["v"], d["lam"], d["gain"], dy, save,
-                         scale=w.scale, eps=w.eps, causal=w.causal, grads=grads, workspace=bws,
-                         dev_status=status)
+                         scale=w.scale, eps=w.eps, causal=w.causal, apply_norm=w.apply_norm,
+                         grads=grads, workspace=bws, dev_status=status, **opts)
 
     bwd()
     launches = ops.last_launch_count()
-    tb = time_loop(bwd, steps, warmup, device) / steps
-    tk = kernel_time(bwd, max(3, min(steps, 20)), ops)
+    if steps is None:
+        steps = extra_steps(bwd, device)
+    tb = time_loop(bwd, steps, warmup, device, clocks=clocks) / steps
+    tk = kernel_time(bwd, max(3, steps), ops)
     tf = time_loop(fwd, steps, warmup, device) / steps
     torch.cuda.synchronize(device)
     if status.item() != 0:
         raise RuntimeError(f"device status {status.item()} in the backward of {w.name}")
-    return dict(bwd_s=tb, kernel_s=tk, fwd_save_s=tf, launches=launches)
+    return dict(bwd_s=tb, kernel_s=tk, fwd_save_s=tf, launches=launches, steps=steps)
+
+
+def backward_line(w, rb, peaks):
+    """The bench's record of one backward workload: 1280 FLOP per visible
+    (query, key) pair per signal head (every product the gradient needs:
+    both score maps again, dP, dV, dK_1, dK_2, dQ_1, dQ_2)."""
+    pairs = (causal_pairs(w.N, w.window) if w.causal else w.N * w.N) * w.B * w.H
+    fl = pairs * BWD_FLOP_PER_PAIR
+    return {"tflops": round(fl / rb["bwd_s"] / 1e12, 2),
+            "kernel_tflops": round(fl / rb["kernel_s"] / 1e12, 2),
+            "frac_of_peak": round(fl / rb["kernel_s"] / 1e12 / peaks["bf16_tflops"], 4),
+            "ms": round(rb["bwd_s"] * 1e3, 4), "fwd_save_ms": round(rb["fwd_save_s"] * 1e3, 4),
+            "train_step_tflops": round(pairs * (FLOP_PER_PAIR + BWD_FLOP_PER_PAIR)
+                                       / (rb["bwd_s"] + rb["fwd_save_s"]) / 1e12, 2),
+            "flop_per_pair": BWD_FLOP_PER_PAIR, "launches": rb["launches"], "steps": rb["steps"],
+            "kernels_timed": "bwd_key_kernel + bwd_query_kernel"}
 
 
 def gpu_arm(args):
@@ -439,16 +591,24 @@ def gpu_arm(args):
     barrier(device)
     peaks = measured_peaks()
     w = inputs.WORKLOADS[args.workload]
-    units = prefill_flops(w)
+    plan = shard_plan(w, world, rank, args.shard)
 
     clk = ClockSampler(device)
-    r = run_prefill_workload(w, args.steps, args.warmup, device, ops, rank, clocks=clk)
-    value, t_max = aggregate_throughput(units * args.steps, r["step_s"] * args.steps, device, world)
-    value /= 1e12
-    e2e_s, h2d, d2h = e2e_prefill(w, max(3, args.steps // 4), 2, device, ops, r["x"])
-    e2e_value, _ = aggregate_throughput(units, e2e_s, device, world)
+    r = run_prefill_workload(w, args.steps, args.warmup, device, ops, rank, clocks=clk, plan=plan,
+                             shard=args.shard)
+    units = r["flops"]                        # this rank's algorithmic FLOP per step
+    total_units = sum_over_ranks(units, device)
+    t_max = max_over_ranks(r["step_s"] * args.steps, device)
+    value = total_units * args.steps / t_max / 1e12
+    gathered = None
+    if args.gather and args.shard != "replica":  # outside the timed region
+        gather_output(r["out_full"], device)
+        gathered = bool(torch.isfinite(r["out_full"].float()).all().item())
+    e2e_s, h2d, d2h = (e2e_prefill(r["work"], max(3, args.steps // 4), 2, device, ops, r["x"])
+                       if not r["empty"] else (0.0, 0, 0))
+    e2e_value = total_units / max_over_ranks(e2e_s, device)
 
-    achieved = units / r["kernel_s"] / 1e12
+    achieved = units / r["kernel_s"] / 1e12 if not r["empty"] else 0.0
     result = {
         "metric": "diff-attn fwd TFLOP/s (bf16 causal)",
         "value": round(value, 2),
@@ -458,13 +618,16 @@ def gpu_arm(args):
         "warmup": args.warmup,
         "ms_per_step": round(t_max / args.steps * 1e3, 4),
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "weak" if args.shard == "replica" else "strong",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": f"{w.name}: B{w.B} N{w.N} H{w.H} d64 dv128 causal prefill",
-                   "global_batch": w.B * world, "seq_len": w.N, "heads": w.H,
-                   "parallelism": f"dp{world} (independent batches)",
+                   "global_batch": w.B * world if args.shard == "replica" else w.B,
+                   "seq_len": w.N, "heads": w.H,
+                   "parallelism": {"replica": f"dp{world} (independent batches)",
+                                   "batch": f"batch split over {world} ranks (one global problem)",
+                                   "heads": f"heads split over {world} ranks (one global problem)"}[args.shard],
                    "l2": "inputs 201 MB per rank, larger than the 126 MB L2; no flush"},
         "e2e": {"value": round(e2e_value / 1e12, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -477,42 +640,44 @@ def gpu_arm(args):
         "gpu_launches": r["launches"] * args.steps,
         "clocks": clk.summary(),
     }
+    if gathered is not None:
+        result["gathered"] = gathered
     if world == 1 and not args.no_extra:
         extra = {}
         for name in ("lc16k", "grouped", "gated", "swa16k", "rope4k"):
             wx = inputs.WORKLOADS[name]
-            rx = run_prefill_workload(wx, max(3, args.steps // 5), 2, device, ops)
+            cx = ClockSampler(device)
+            rx = run_prefill_workload(wx, None, 3, device, ops, clocks=cx)
             fx = prefill_flops(wx)
             extra[name] = {"tflops": round(fx / rx["step_s"] / 1e12, 2),
                            "kernel_tflops": round(fx / rx["kernel_s"] / 1e12, 2),
                            "frac_of_peak": round(fx / rx["kernel_s"] / 1e12 / peaks["bf16_tflops"], 4),
-                           "ms": round(rx["step_s"] * 1e3, 4)}
+                           "ms": round(rx["step_s"] * 1e3, 4), "steps": rx["steps"],
+                           "sm_mhz": cx.summary()["sm_mhz"]}
             if wx.window:  # few keys per query: the HBM bytes bound it, not the tensor cores
                 gb = prefill_bytes(wx) / rx["step_s"] / 1e9
                 extra[name]["gbs"] = round(gb, 1)
                 extra[name]["hbm_frac"] = round(gb / peaks["hbm_gbs"], 4)
             del rx
-        wb = inputs.WORKLOADS["motif4k"]
-        rb = run_backward_workload(wb, max(3, args.steps // 5), 2, device, ops)
-        pb = causal_pairs(wb.N) * wb.B * wb.H
-        extra["bwd4k"] = {"tflops": round(pb * BWD_FLOP_PER_PAIR / rb["bwd_s"] / 1e12, 2),
-                          "kernel_tflops": round(pb * BWD_FLOP_PER_PAIR / rb["kernel_s"] / 1e12, 2),
-                          "frac_of_peak": round(pb * BWD_FLOP_PER_PAIR / rb["kernel_s"] / 1e12
-                                                / peaks["bf16_tflops"], 4),
-                          "ms": round(rb["bwd_s"] * 1e3, 4),
-                          "fwd_save_ms": round(rb["fwd_save_s"] * 1e3, 4),
-                          "train_step_tflops": round(pb * (FLOP_PER_PAIR + BWD_FLOP_PER_PAIR)
-                                                     / (rb["bwd_s"] + rb["fwd_save_s"]) / 1e12, 2),
-                          "flop_per_pair": BWD_FLOP_PER_PAIR, "launches": rb["launches"]}
+        for key, name in (("bwd4k", "motif4k"), ("bwd_gated", "gated")):
+            # the gated workload is Motif 3's attention: grouped, token lambda, gate
+            wb = inputs.WORKLOADS[name]
+            cb = ClockSampler(device)
+            rb = run_backward_workload(wb, None, 3, device, ops, clocks=cb)
+            extra[key] = backward_line(wb, rb, peaks)
+            extra[key]["sm_mhz"] = cb.summary()["sm_mhz"]
+            del rb
         wd = inputs.WORKLOADS["decode"]
-        rd = run_decode_workload(wd, max(5, args.steps), 3, device, ops)
+        cd = ClockSampler(device)
+        rd = run_decode_workload(wd, None, 3, device, ops, clocks=cd)
         bd = decode_bytes(wd)
         extra["decode"] = {"gbs": round(bd / rd["step_s"] / 1e9, 1),
                            "split_kernel_gbs": round(bd / rd["kernel_s"] / 1e9, 1),
                            "roofline": {"bound": "hbm", "achieved": round(bd / rd["step_s"] / 1e9, 1),
                                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                         "frac": round(bd / rd["step_s"] / 1e9 / peaks["hbm_gbs"], 4)},
-                           "us": round(rd["step_s"] * 1e6, 2), "launches": rd["launches"]}
+                           "us": round(rd["step_s"] * 1e6, 2), "launches": rd["launches"],
+                           "steps": rd["steps"], "sm_mhz": cd.summary()["sm_mhz"]}
         result["extra"] = extra
     if world == 1 and rank == 0 and not args.no_cpu:
         v, sample, cores = cpu_baseline(w, budget_s=args.cpu_budget)
@@ -582,6 +747,11 @@ def main(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-baseline leg")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--shard", choices=SHARD_MODES, default="replica",
+                    help="multi-GPU split: independent problems per rank (replica), or one global "
+                         "problem split by batch entries or by heads")
+    ap.add_argument("--gather", action="store_true",
+                    help="with --shard batch|heads, assemble the output on every rank afterwards")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     if args.impl == "reference":
