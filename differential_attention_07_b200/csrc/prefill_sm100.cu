@@ -748,54 +748,62 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     }
                     __syncwarp();
                 }
+                // The export item of this tile ran about one wave of items
+                // earlier; its eight epilogue warps have normally all
+                // published their half-rows by now.  (Plain L2 loads below: the
+                // data was written during this launch.)  The first half of
+                // this row's A_N is loaded while the tile's last P.V runs.
+                bool ready = true;
+                if (lane == 0) ready = wait_flag_geq(p.noise_ready + noise_tile, 8, abort_flag, lim);
+                if (!(ok = __shfl_sync(0xffffffffu, ready, 0))) break;
+                float4 an[16];
+#pragma unroll
+                for (int i4 = 0; i4 < 16; ++i4) an[i4] = __ldcg(an_tile + i4 * BM + r);
                 if (!(ok = mbar_wait_warp(bar(B_O), tiles & 1, abort_flag, lim))) break;
                 // The gate box (issued above) has had the last P.V's time to land.
                 if (GATED && !(ok = mbar_wait_warp(bar(B_GATE + (warp - 4)), tiles & 1, abort_flag, lim)))
                     break;
-                // The export item of this tile ran about one wave of items
-                // earlier; its eight epilogue warps have normally all
-                // published their half-rows by now.  (Plain L2 loads below: the
-                // data was written during this launch.)
-                bool ready = true;
-                if (lane == 0) ready = wait_flag_geq(p.noise_ready + noise_tile, 8, abort_flag, lim);
-                if (!(ok = __shfl_sync(0xffffffffu, ready, 0))) break;
                 tc_fence_after();
                 const float inv = 1.0f / l_run;
                 const float lam = p.lam_logits ? logistic_fast(lam_in) : lam_in;
-                // Pass 1: sum of squares of D over the row, 64 columns at a time.
+                // Pass 1: sum of squares of D over the row, 64 columns at a
+                // time (the first half with the prefetched A_N, then the
+                // second half, whose A_N stays in registers for pass 2).
                 float ss = 0.0f;
-#pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
+                auto sum_sq = [&](int hh) {
                     uint32_t o[2][32];
                     tmem_ld32(tO + 64 * hh, o[0]);
                     tmem_ld32(tO + 64 * hh + 32, o[1]);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i4 = 0; i4 < 16; ++i4) {
-                        const float4 a4 = __ldcg(an_tile + (16 * hh + i4) * BM + r);
-                        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+                        const float av[4] = {an[i4].x, an[i4].y, an[i4].z, an[i4].w};
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float dd = fmaf(-lam, av[e], __uint_as_float(o[i4 >> 3][4 * (i4 & 7) + e]) * inv);
                             ss = fmaf(dd, dd, ss);
                         }
                     }
-                }
+                };
+                sum_sq(0);
+#pragma unroll
+                for (int i4 = 0; i4 < 16; ++i4) an[i4] = __ldcg(an_tile + (16 + i4) * BM + r);
+                sum_sq(1);
                 const float rn = p.apply_norm ? rsqrtf(ss * (1.0f / HDV) + p.eps) : 1.0f;
                 // This warp's staging buffer: the previous tile's store must
                 // have read it (and the gate box must have landed in it).
                 const uint32_t obuf = sbase + OFF_OUT + (warp - 4) * OUT_WARP_BYTES;
                 if (lane == 0) bulk_wait_read_all();
                 __syncwarp();
-                // Pass 2: D again, normalised, gain, bf16, stored; O is released
-                // after its last read.
-#pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
+                // Pass 2: D again, normalised, gain, bf16, stored; the second
+                // half first (its A_N is still in registers), and O is
+                // released after its last read.
+                auto write_half = [&](int hh) {
                     uint32_t o[2][32];
                     tmem_ld32(tO + 64 * hh, o[0]);
                     tmem_ld32(tO + 64 * hh + 32, o[1]);
                     tmem_wait_ld();
-                    if (hh == 1) {  // O read to registers by every lane: release it, once per warp
+                    if (hh == 0) {  // O read to registers by every lane: release it, once per warp
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar(B_OFREE));
@@ -803,7 +811,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     uint32_t y[32];
 #pragma unroll
                     for (int i4 = 0; i4 < 16; ++i4) {
-                        const float4 a4 = __ldcg(an_tile + (16 * hh + i4) * BM + r);
+                        const float4 a4 = an[i4];
                         const float4 g4 = gain ? __ldg(reinterpret_cast<const float4 *>(gain) + 16 * hh + i4)
                                                : make_float4(1.f, 1.f, 1.f, 1.f);
                         float4 s4 = make_float4(rn, rn, rn, rn);  // norm x output gate
@@ -830,7 +838,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     for (int i = 0; i < 8; ++i)
                         st_shared_v4(rowb + ((i ^ (lane & 7)) << 4), y[4 * i], y[4 * i + 1], y[4 * i + 2],
                                      y[4 * i + 3]);
-                }
+                };
+                write_half(1);
+#pragma unroll
+                for (int i4 = 0; i4 < 16; ++i4) an[i4] = __ldcg(an_tile + i4 * BM + r);
+                write_half(0);
                 fence_proxy_async_smem();
                 __syncwarp();
                 const int r0 = w.qt * BM + 32 * (warp & 3);
@@ -916,13 +928,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                                      __uint_as_float(ob[c][4 * i4 + 1]) * inv2,
                                                      __uint_as_float(ob[c][4 * i4 + 2]) * inv2,
                                                      __uint_as_float(ob[c][4 * i4 + 3]) * inv2);
-                // Publish: every lane's stores, then one release per warp (the
-                // pair items wait for all eight warps of the tile).
-                __syncwarp();
-                if (lane == 0) {
-                    __threadfence();
-                    atomicAdd(p.noise_ready + noise_tile, 1);
-                }
             }
             float d[64];
             float ss = 0.0f;
@@ -990,6 +995,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (lane == 0 && w.qt * BM + 32 * (warp & 3) < p.N) {  // a box wholly past N is not issued
                 tma_store_4d(&tm_out, obuf, c0, w.qt * BM + 32 * (warp & 3), hd.a, w.b);
                 bulk_commit_group();
+            }
+            if (p.mode == 1) {
+                // Publish this warp's part of the noise output (stored above,
+                // before the norm, so the stores have had the rest of the
+                // epilogue to drain): every lane's stores, then one release
+                // per warp; the pair items wait for all eight warps of the tile.
+                __syncwarp();
+                if (lane == 0) {
+                    __threadfence();
+                    atomicAdd(p.noise_ready + noise_tile, 1);
+                }
             }
         }
     }

@@ -248,7 +248,21 @@ def test_token_lambda_and_gate(cuda_ok, apply_norm):
 def test_window(cuda_ok, W):
     x, dy = _ext(2, 600, 2, 2, 2, seed=51 + W, window=W)
     _, g = _run(x, dy)
-    _check(g, _ref(x, dy))
+    ref = _ref(x, dy)
+    if W > 1:
+        _check(g, ref)
+        return
+    # W = 1: every query sees only itself, so each softmax is constant and
+    # dQ, dK are exactly zero; the GPU's are fp32 rounding residue of
+    # dP - Delta (both from the same fp16 dD), far below the scale of dV.
+    # And D = (1 - lambda) V_i, so the norm leaves only eps to depend on
+    # lambda: dlambda sums, over B N rows, near-cancellations of 128 fp32
+    # products of order one (about 1e-5 each), checked to 1e-4 sqrt(B N)
+    # absolute, as a random walk of those residues.
+    _check(g, ref, names=("dv",), sums=("dgain",))
+    assert np.abs(g["dlam"] - ref["dlam"]).max() <= 1e-4 * np.sqrt(2 * 600)
+    for n in ("dq1", "dq2", "dk1", "dk2"):
+        assert np.abs(g[n]).max() <= 1e-3 * np.abs(ref["dv"]).max(), n
 
 
 @pytest.mark.parametrize("N", [1, 77, 300])
