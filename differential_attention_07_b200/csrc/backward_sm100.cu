@@ -59,32 +59,37 @@ constexpr int BT = 128;   // rows of a tile: MMA M, one per TMEM lane
 constexpr int BB = 64;    // rows of a block: MMA N of the score products
 constexpr int HD = 64;    // Q/K head dim
 constexpr int HDV = 128;  // V head dim
-constexpr int NT = 320;   // 10 warps: producer, MMA issuer, two element-wise warpgroups
+constexpr int NT = 352;   // 11 warps: producer, two MMA issuers, two element-wise warpgroups
 constexpr int NEW = 8;    // element-wise warps
+
+// Block stages of the two tile kernels' load rings (as many as fit in
+// shared memory: a block's load is issued STAGES - 1 blocks ahead).
+constexpr int KSTAGES = 3, QSTAGES = 3, MAXSTAGES = 3;
 
 // mbarriers of both tile kernels.
 enum : int {
-    B_TILE = 0,   // the tile's operands landed (TMA bytes)
-    B_FULL = 1,   // [2] a block's operands landed (TMA bytes)
-    B_EMPTY = 3,  // [2] the block's last products have read its stage (commit)
-    B_SFULL = 5,  // the block's score and dP products are in TMEM (commit)
-    B_SFREE = 6,  // the element-wise warps loaded them (8 arrivals)
-    B_AFULL = 7,  // the element-wise warps wrote the A operands (8 arrivals)
-    B_AFREE = 8,  // the accumulating products have read the A operands (commit)
-    B_DONE = 9,   // every product of the CTA has completed (commit)
-    NBARS = 10
+    B_TILE = 0,                     // the tile's operands landed (TMA bytes)
+    B_FULL = 1,                     // [stages] a block's operands landed (TMA bytes)
+    B_EMPTY = B_FULL + MAXSTAGES,   // [stages] the block's last products have read its stage (commit)
+    B_SFULL = B_EMPTY + MAXSTAGES,  // the block's score and dP products are in TMEM (commit)
+    B_SFREE,                        // the element-wise warps loaded them (8 arrivals)
+    B_AFULL,                        // the element-wise warps wrote the A operands (8 arrivals)
+    B_AFREE,                        // the accumulating products have read the A operands (commit)
+    B_DONE,                         // every product of the CTA has completed (commit)
+    B_SDRAIN,                       // the score issuer's products have completed (commit)
+    NBARS
 };
 
 // ---------------------------------------------------------------- key-tile kernel
 // Shared memory: the tile's K_1, K_2 ([128][64]) and fp16 V ([128][128] as
-// two [128][64] column halves); two block stages of Q_1, Q_2 ([64][64]), dD
-// (fp16 [64][128] as two halves) and the statistics [kBwdStats][64] fp32;
-// the A operands P_1 - lambda P_2, dS_1, dS_2 ([128 keys][64 queries]).
+// two [128][64] column halves); KSTAGES block stages of Q_1, Q_2 ([64][64]),
+// dD (fp16 [64][128] as two halves) and the statistics [kBwdStats][64]
+// fp32; the A operands P_1 - lambda P_2, dS_1, dS_2 ([128 keys][64 queries]).
 constexpr uint32_t KT_K1 = 0, KT_K2 = 16384, KT_V = 32768, KT_STAGE0 = 65536;
 constexpr uint32_t KB_Q1 = 0, KB_Q2 = 8192, KB_DD = 16384, KB_ST = 32768;
 constexpr uint32_t KB_LOAD = KB_ST + kBwdStats * BB * 4;  // bytes a stage receives
 constexpr uint32_t KB_BYTES = (KB_LOAD + 1023) & ~1023u;   // stages stay 1 KB aligned
-constexpr uint32_t KT_A = KT_STAGE0 + 2 * KB_BYTES;
+constexpr uint32_t KT_A = KT_STAGE0 + KSTAGES * KB_BYTES;
 constexpr uint32_t KA_PV = 0, KA_DS1 = 16384, KA_DS2 = 32768;
 constexpr uint32_t KT_BARS = KT_A + 3 * 16384;
 constexpr uint32_t KT_SMEM = KT_BARS + 8 * NBARS + 16;
@@ -93,11 +98,12 @@ constexpr uint32_t KM_DV = 0, KM_DK1 = 128, KM_DK2 = 192, KM_S1 = 256, KM_S2 = 3
 
 // ---------------------------------------------------------------- query-tile kernel
 // Shared memory: the tile's Q_1, Q_2 ([128][64]) and dD (fp16 [128][128] as
-// two halves); two block stages of K_1, K_2 ([64][64]) and fp16 V ([64][128]
-// as two halves); the A operands dS_1, dS_2 ([128 queries][64 keys]).
+// two halves); QSTAGES block stages of K_1, K_2 ([64][64]) and fp16 V
+// ([64][128] as two halves); the A operands dS_1, dS_2 ([128 queries][64
+// keys]).
 constexpr uint32_t QT_Q1 = 0, QT_Q2 = 16384, QT_DD = 32768, QT_STAGE0 = 65536;
 constexpr uint32_t QB_K1 = 0, QB_K2 = 8192, QB_V = 16384, QB_BYTES = 32768;
-constexpr uint32_t QT_A = QT_STAGE0 + 2 * QB_BYTES;
+constexpr uint32_t QT_A = QT_STAGE0 + QSTAGES * QB_BYTES;
 constexpr uint32_t QA_DS1 = 0, QA_DS2 = 16384;
 constexpr uint32_t QT_BARS = QT_A + 2 * 16384;
 constexpr uint32_t QT_SMEM = QT_BARS + 8 * NBARS + 16;
@@ -363,12 +369,56 @@ __global__ void __launch_bounds__(128)
 struct Roles {
     int warp, lane;
     __device__ __forceinline__ bool producer() const { return warp == 0; }
-    __device__ __forceinline__ bool issuer() const { return warp == 1; }
-    // element-wise warpgroup (0 or 1) and the TMEM lane / tile row of this thread
-    __device__ __forceinline__ int wg() const { return (warp - 2) >> 2; }
+    __device__ __forceinline__ bool score_issuer() const { return warp == 1; }
+    __device__ __forceinline__ bool acc_issuer() const { return warp == 2; }
+    // element-wise warpgroup (0 or 1) and the TMEM lane / tile row of this
+    // thread (warps 3-6 and 7-10: each group covers the four lane quarters)
+    __device__ __forceinline__ int wg() const { return (warp - 3) >> 2; }
     __device__ __forceinline__ int row() const { return (warp & 3) * 32 + lane; }
     __device__ __forceinline__ uint32_t lane_off() const { return uint32_t((warp & 3) * 32) << 16; }
 };
+
+// The two MMA issuers of a tile kernel, one warp each, so that neither
+// kind of product waits behind the other in one warp's program order:
+//  * the score issuer: block j's score and dP products, once its stage has
+//    landed and the element-wise warps have taken block j-1's products out
+//    of TMEM (early in their step);
+//  * the accumulating issuer: block j's accumulating products, once the
+//    element-wise warps have written their A operands (at the end of their
+//    step).
+// Block j's score products are complete before its accumulating products
+// are issued (the element-wise warps waited for them), so the accumulating
+// issuer's last commit covers every product of the tile.  Every wait is
+// bounded; each issuer drains what it issued before the CTA tears down.
+template <int ST, class IssueS>
+__device__ __forceinline__ void score_issuer(int nit, uint32_t bar_tile, uint32_t bar_full, uint32_t bar_sfree,
+                                             uint32_t bar_drain, volatile int *abort_flag, uint64_t lim,
+                                             IssueS issue_s, int lane)
+{
+    bool ok = mbar_wait_warp(bar_tile, 0, abort_flag, lim);
+    for (int j = 0; ok && j < nit; ++j) {
+        if (!(ok = mbar_wait_warp(bar_full + 8 * (j % ST), (j / ST) & 1, abort_flag, lim))) break;
+        if (j > 0 && !(ok = mbar_wait_warp(bar_sfree, (j - 1) & 1, abort_flag, lim))) break;
+        tc_fence_after();
+        issue_s(j);
+    }
+    commit_to(bar_drain);
+    if (!__all_sync(0xffffffffu, mbar_wait_drain(bar_drain, 0, lim)) && lane == 0) *abort_flag = 1;
+}
+template <class IssueAcc>
+__device__ __forceinline__ void acc_issuer(int nit, uint32_t bar_afull, uint32_t bar_done, volatile int *abort_flag,
+                                           uint64_t lim, IssueAcc issue_acc, int lane)
+{
+    for (int j = 0; j < nit; ++j) {
+        if (!mbar_wait_warp(bar_afull, j & 1, abort_flag, lim)) break;
+        tc_fence_after();
+        issue_acc(j);
+    }
+    // DONE completes once everything issued has: the epilogue's signal,
+    // and the teardown's guarantee that no product still runs.
+    commit_to(bar_done);
+    if (!__all_sync(0xffffffffu, mbar_wait_drain(bar_done, 0, lim)) && lane == 0) *abort_flag = 1;
+}
 
 // ---------------------------------------------------------------- 2. key tiles
 template <bool F16QK>
@@ -400,7 +450,7 @@ __global__ void __launch_bounds__(NT, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_TILE), 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < MAXSTAGES; ++s) {
             mbar_init(bar(B_FULL + s), 1);
             mbar_init(bar(B_EMPTY + s), 1);
         }
@@ -409,6 +459,7 @@ __global__ void __launch_bounds__(NT, 1)
         mbar_init(bar(B_AFULL), NEW);
         mbar_init(bar(B_AFREE), 1);
         mbar_init(bar(B_DONE), 1);
+        mbar_init(bar(B_SDRAIN), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -433,8 +484,8 @@ __global__ void __launch_bounds__(NT, 1)
         __syncwarp();
         int loads = 0;
         for (int j = 0; j < nit; ++j) {
-            const int s = j & 1;
-            if (j >= 2 && !mbar_wait_warp(bar(B_EMPTY + s), ((j >> 1) - 1) & 1, abort_flag, lim)) break;
+            const int s = j % KSTAGES;
+            if (j >= KSTAGES && !mbar_wait_warp(bar(B_EMPTY + s), ((j / KSTAGES) - 1) & 1, abort_flag, lim)) break;
             if (elect_one()) {
                 const uint32_t st = sbase + KT_STAGE0 + s * KB_BYTES, fb = bar(B_FULL + s);
                 const int q0 = (qb0 + j) * BB;
@@ -450,17 +501,15 @@ __global__ void __launch_bounds__(NT, 1)
         }
         // No load of ours may land after the CTA has gone.
         bool drained = mbar_wait_drain(bar(B_TILE), 0, lim);
-        for (int k = (loads > 2 ? loads - 2 : 0); k < loads; ++k)
-            drained &= mbar_wait_drain(bar(B_FULL + (k & 1)), (k >> 1) & 1, lim);
+        for (int k = (loads > KSTAGES ? loads - KSTAGES : 0); k < loads; ++k)
+            drained &= mbar_wait_drain(bar(B_FULL + k % KSTAGES), (k / KSTAGES) & 1, lim);
         if (!__all_sync(0xffffffffu, drained) && R.lane == 0) *abort_flag = 1;
-    } else if (R.issuer()) {
-        // ------------------------------------------------------------ MMA issuer
-        // Per block j: the score and dP products of block j (once the
-        // element-wise warps have taken block j-1's out of TMEM), then the
-        // accumulating products of block j-1 (once its A operands are
-        // written).  The tensor pipe runs them in that order.
+    } else if (R.score_issuer() || R.acc_issuer()) {
+        // ------------------------------------------------------------ MMA issuers
+        // Warp 1 issues the score and dP products, warp 2 the accumulating
+        // products (see score_issuer / acc_issuer).
         auto issue_s = [&](int j) {
-            const uint32_t st = sbase + KT_STAGE0 + (j & 1) * KB_BYTES;
+            const uint32_t st = sbase + KT_STAGE0 + (j % KSTAGES) * KB_BYTES;
 #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk)
                 mma_issue(tbase + KM_S1, sw128(sbase + KT_K1 + 32 * kk), sw128(st + KB_Q1 + 32 * kk), Ids<F16QK>::S,
@@ -478,7 +527,7 @@ __global__ void __launch_bounds__(NT, 1)
             commit_to(bar(B_SFULL));
         };
         auto issue_acc = [&](int j) {
-            const uint32_t st = sbase + KT_STAGE0 + (j & 1) * KB_BYTES;
+            const uint32_t st = sbase + KT_STAGE0 + (j % KSTAGES) * KB_BYTES;
             // dV += (P_1 - lambda P_2)^T dD; dK_t += dS_t^T Q_t (B MN-major).
 #pragma unroll
             for (int kk = 0; kk < BB / 16; ++kk)
@@ -493,28 +542,13 @@ __global__ void __launch_bounds__(NT, 1)
                 mma_issue(tbase + KM_DK2, sw128(sbase + KT_A + KA_DS2 + 32 * kk), sw128(st + KB_Q2 + 2048 * kk, 8192),
                           Ids<F16QK>::DS, j > 0 || kk > 0);
             commit_to(bar(B_AFREE));
-            commit_to(bar(B_EMPTY + (j & 1)));
+            commit_to(bar(B_EMPTY + j % KSTAGES));
         };
-        bool ok = mbar_wait_warp(bar(B_TILE), 0, abort_flag, lim);
-        for (int j = 0; ok && j < nit; ++j) {
-            if (!(ok = mbar_wait_warp(bar(B_FULL + (j & 1)), (j >> 1) & 1, abort_flag, lim))) break;
-            if (j > 0 && !(ok = mbar_wait_warp(bar(B_SFREE), (j - 1) & 1, abort_flag, lim))) break;
-            tc_fence_after();
-            issue_s(j);
-            if (j > 0) {
-                if (!(ok = mbar_wait_warp(bar(B_AFULL), (j - 1) & 1, abort_flag, lim))) break;
-                tc_fence_after();
-                issue_acc(j - 1);
-            }
-        }
-        if (ok && mbar_wait_warp(bar(B_AFULL), (nit - 1) & 1, abort_flag, lim)) {
-            tc_fence_after();
-            issue_acc(nit - 1);
-        }
-        // DONE completes once everything issued has: the epilogue's signal,
-        // and the teardown's guarantee that no product still runs.
-        commit_to(bar(B_DONE));
-        if (!__all_sync(0xffffffffu, mbar_wait_drain(bar(B_DONE), 0, lim)) && R.lane == 0) *abort_flag = 1;
+        if (R.score_issuer())
+            score_issuer<KSTAGES>(nit, bar(B_TILE), bar(B_FULL), bar(B_SFREE), bar(B_SDRAIN), abort_flag, lim, issue_s,
+                               R.lane);
+        else
+            acc_issuer(nit, bar(B_AFULL), bar(B_DONE), abort_flag, lim, issue_acc, R.lane);
     } else {
         // ------------------------------------------------------------ element-wise + epilogue
         const int wg = R.wg(), r = R.row();
@@ -535,7 +569,7 @@ __global__ void __launch_bounds__(NT, 1)
             if (R.lane == 0) mbar_arrive(bar(B_SFREE));
             // This warpgroup's 32 queries of the block, and their statistics.
             const int qb = (qb0 + j) * BB + 32 * wg;
-            const uint32_t st = sbase + KT_STAGE0 + (j & 1) * KB_BYTES + KB_ST + 4 * 32 * wg;
+            const uint32_t st = sbase + KT_STAGE0 + (j % KSTAGES) * KB_BYTES + KB_ST + 4 * 32 * wg;
             const bool mask = (p.causal && qb < k0 + BT - 1) || (p.window > 0 && qb + 31 - k0 >= p.window);
             uint32_t pv[16], d1p[16], d2p[16];
 #pragma unroll
@@ -569,6 +603,9 @@ __global__ void __launch_bounds__(NT, 1)
                 d1p[i / 2 + 1] = pack_ds(v1[2], v1[3], F16QK);
                 d2p[i / 2] = pack_ds(v2[0], v2[1], F16QK);
                 d2p[i / 2 + 1] = pack_ds(v2[2], v2[3], F16QK);
+                // Keep the next four queries' statistics loads below this
+                // point: hoisted all at once they would need 160 registers.
+                asm volatile("" ::: "memory");
             }
             // The previous block's accumulating products must have read the
             // A operands before they are overwritten.
@@ -652,7 +689,7 @@ __global__ void __launch_bounds__(NT, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_TILE), 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < MAXSTAGES; ++s) {
             mbar_init(bar(B_FULL + s), 1);
             mbar_init(bar(B_EMPTY + s), 1);
         }
@@ -661,6 +698,7 @@ __global__ void __launch_bounds__(NT, 1)
         mbar_init(bar(B_AFULL), NEW);
         mbar_init(bar(B_AFREE), 1);
         mbar_init(bar(B_DONE), 1);
+        mbar_init(bar(B_SDRAIN), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -684,8 +722,8 @@ __global__ void __launch_bounds__(NT, 1)
         __syncwarp();
         int loads = 0;
         for (int j = 0; j < nit; ++j) {
-            const int s = j & 1;
-            if (j >= 2 && !mbar_wait_warp(bar(B_EMPTY + s), ((j >> 1) - 1) & 1, abort_flag, lim)) break;
+            const int s = j % QSTAGES;
+            if (j >= QSTAGES && !mbar_wait_warp(bar(B_EMPTY + s), ((j / QSTAGES) - 1) & 1, abort_flag, lim)) break;
             if (elect_one()) {
                 const uint32_t st = sbase + QT_STAGE0 + s * QB_BYTES, fb = bar(B_FULL + s);
                 const int k0 = (kb0 + j) * BB;
@@ -699,12 +737,12 @@ __global__ void __launch_bounds__(NT, 1)
             loads = j + 1;
         }
         bool drained = mbar_wait_drain(bar(B_TILE), 0, lim);
-        for (int k = (loads > 2 ? loads - 2 : 0); k < loads; ++k)
-            drained &= mbar_wait_drain(bar(B_FULL + (k & 1)), (k >> 1) & 1, lim);
+        for (int k = (loads > QSTAGES ? loads - QSTAGES : 0); k < loads; ++k)
+            drained &= mbar_wait_drain(bar(B_FULL + k % QSTAGES), (k / QSTAGES) & 1, lim);
         if (!__all_sync(0xffffffffu, drained) && R.lane == 0) *abort_flag = 1;
-    } else if (R.issuer()) {
+    } else if (R.score_issuer() || R.acc_issuer()) {
         auto issue_s = [&](int j) {
-            const uint32_t st = sbase + QT_STAGE0 + (j & 1) * QB_BYTES;
+            const uint32_t st = sbase + QT_STAGE0 + (j % QSTAGES) * QB_BYTES;
 #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk)
                 mma_issue(tbase + QM_S1, sw128(sbase + QT_Q1 + 32 * kk), sw128(st + QB_K1 + 32 * kk), Ids<F16QK>::S,
@@ -722,7 +760,7 @@ __global__ void __launch_bounds__(NT, 1)
             commit_to(bar(B_SFULL));
         };
         auto issue_acc = [&](int j) {
-            const uint32_t st = sbase + QT_STAGE0 + (j & 1) * QB_BYTES;
+            const uint32_t st = sbase + QT_STAGE0 + (j % QSTAGES) * QB_BYTES;
             // dQ_t += dS_t K_t (B: the K block, MN-major).
 #pragma unroll
             for (int kk = 0; kk < BB / 16; ++kk)
@@ -733,26 +771,13 @@ __global__ void __launch_bounds__(NT, 1)
                 mma_issue(tbase + QM_DQ2, sw128(sbase + QT_A + QA_DS2 + 32 * kk), sw128(st + QB_K2 + 2048 * kk, 8192),
                           Ids<F16QK>::DS, j > 0 || kk > 0);
             commit_to(bar(B_AFREE));
-            commit_to(bar(B_EMPTY + (j & 1)));
+            commit_to(bar(B_EMPTY + j % QSTAGES));
         };
-        bool ok = mbar_wait_warp(bar(B_TILE), 0, abort_flag, lim);
-        for (int j = 0; ok && j < nit; ++j) {
-            if (!(ok = mbar_wait_warp(bar(B_FULL + (j & 1)), (j >> 1) & 1, abort_flag, lim))) break;
-            if (j > 0 && !(ok = mbar_wait_warp(bar(B_SFREE), (j - 1) & 1, abort_flag, lim))) break;
-            tc_fence_after();
-            issue_s(j);
-            if (j > 0) {
-                if (!(ok = mbar_wait_warp(bar(B_AFULL), (j - 1) & 1, abort_flag, lim))) break;
-                tc_fence_after();
-                issue_acc(j - 1);
-            }
-        }
-        if (ok && mbar_wait_warp(bar(B_AFULL), (nit - 1) & 1, abort_flag, lim)) {
-            tc_fence_after();
-            issue_acc(nit - 1);
-        }
-        commit_to(bar(B_DONE));
-        if (!__all_sync(0xffffffffu, mbar_wait_drain(bar(B_DONE), 0, lim)) && R.lane == 0) *abort_flag = 1;
+        if (R.score_issuer())
+            score_issuer<QSTAGES>(nit, bar(B_TILE), bar(B_FULL), bar(B_SFREE), bar(B_SDRAIN), abort_flag, lim, issue_s,
+                               R.lane);
+        else
+            acc_issuer(nit, bar(B_AFULL), bar(B_DONE), abort_flag, lim, issue_acc, R.lane);
     } else {
         const int wg = R.wg(), r = R.row();
         const uint32_t lo = R.lane_off();
