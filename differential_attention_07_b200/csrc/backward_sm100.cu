@@ -77,6 +77,7 @@ enum : int {
     B_AFREE,                        // the accumulating products have read the A operands (commit)
     B_DONE,                         // every product of the CTA has completed (commit)
     B_SDRAIN,                       // the score issuer's products have completed (commit)
+    B_AOP,                          // the tile's A operands are in TMEM (8 arrivals)
     NBARS
 };
 
@@ -93,8 +94,12 @@ constexpr uint32_t KT_A = KT_STAGE0 + KSTAGES * KB_BYTES;
 constexpr uint32_t KA_PV = 0, KA_DS1 = 16384, KA_DS2 = 32768;
 constexpr uint32_t KT_BARS = KT_A + 3 * 16384;
 constexpr uint32_t KT_SMEM = KT_BARS + 8 * NBARS + 16;
-// TMEM columns: dV, dK_1, dK_2 accumulators, then S_1^T, S_2^T, dP^T.
-constexpr uint32_t KM_DV = 0, KM_DK1 = 128, KM_DK2 = 192, KM_S1 = 256, KM_S2 = 320, KM_DP = 384;
+// TMEM columns: dV, dK_1, dK_2 accumulators, then S_1^T, S_2^T, dP^T, then
+// the tile's K_1 and K_2 (bf16 / fp16 pairs) as the A operand of the score
+// products, so that every block's score products read only Q from shared
+// memory (the kernel is bound by shared-memory bandwidth).
+constexpr uint32_t KM_DV = 0, KM_DK1 = 128, KM_DK2 = 192, KM_S1 = 256, KM_S2 = 320, KM_DP = 384,
+                   KM_AK1 = 448, KM_AK2 = 480;
 
 // ---------------------------------------------------------------- query-tile kernel
 // Shared memory: the tile's Q_1, Q_2 ([128][64]) and dD (fp16 [128][128] as
@@ -107,8 +112,12 @@ constexpr uint32_t QT_A = QT_STAGE0 + QSTAGES * QB_BYTES;
 constexpr uint32_t QA_DS1 = 0, QA_DS2 = 16384;
 constexpr uint32_t QT_BARS = QT_A + 2 * 16384;
 constexpr uint32_t QT_SMEM = QT_BARS + 8 * NBARS + 16;
-// TMEM columns: dQ_1, dQ_2 accumulators, then S_1, S_2, dP.
-constexpr uint32_t QM_DQ1 = 0, QM_DQ2 = 64, QM_S1 = 128, QM_S2 = 192, QM_DP = 256;
+// TMEM columns: dQ_1, dQ_2 accumulators, then S_1, S_2, dP, then the tile's
+// Q_1, Q_2 and dD (16-bit pairs) as the A operands of the score and dP
+// products, so that every block's products read only K and V from shared
+// memory (the kernel is bound by shared-memory bandwidth).
+constexpr uint32_t QM_DQ1 = 0, QM_DQ2 = 64, QM_S1 = 128, QM_S2 = 192, QM_DP = 256, QM_AQ1 = 320,
+                   QM_AQ2 = 352, QM_ADD = 384;
 
 static_assert(KT_SMEM <= 232448 && QT_SMEM <= 232448, "shared memory budget");
 static_assert(KT_A % 1024 == 0 && QT_A % 1024 == 0 && KB_BYTES % 1024 == 0, "SW128 tiles are 1 KB aligned");
@@ -136,6 +145,11 @@ __device__ __forceinline__ uint64_t sw128(uint32_t addr, uint32_t lbo = 16)
 __device__ __forceinline__ void mma_issue(uint32_t d, uint64_t a, uint64_t b, uint32_t id, bool acc)
 {
     if (elect_one()) mma_ss(d, a, b, id, acc ? 1u : 0u);
+    __syncwarp();
+}
+__device__ __forceinline__ void mma_issue_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t id, bool acc)
+{
+    if (elect_one()) mma_ts(d, a_tmem, b, id, acc ? 1u : 0u);
     __syncwarp();
 }
 __device__ __forceinline__ void commit_to(uint32_t bar)
@@ -175,6 +189,25 @@ __device__ __forceinline__ void unrotate64(float (&x)[64], int pos, const double
         x[2 * c] = a * cs + b * sn;
         x[2 * c + 1] = b * cs - a * sn;
     }
+}
+
+// Copy this thread's row r of a [128 rows][64 columns] 16-bit tile in the
+// 128-byte swizzle (16-byte chunk c of row r at c ^ (r % 8)) to 32 TMEM
+// columns of its lane: column i holds elements 2i, 2i + 1, the layout of an
+// A operand read from TMEM.
+__device__ __forceinline__ void tile_row_to_tmem(uint32_t tile, int r, uint32_t taddr)
+{
+    uint32_t w[32];
+    const uint32_t row = tile + 128u * r;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint4 v = ld_shared_v4(row + (((c ^ (r & 7)) & 7) << 4));
+        w[4 * c] = v.x;
+        w[4 * c + 1] = v.y;
+        w[4 * c + 2] = v.z;
+        w[4 * c + 3] = v.w;
+    }
+    tmem_st32(taddr, w);
 }
 
 // Write one row of `cols` values (scaled by s) to a bf16 row (16-byte
@@ -391,11 +424,11 @@ struct Roles {
 // issuer's last commit covers every product of the tile.  Every wait is
 // bounded; each issuer drains what it issued before the CTA tears down.
 template <int ST, class IssueS>
-__device__ __forceinline__ void score_issuer(int nit, uint32_t bar_tile, uint32_t bar_full, uint32_t bar_sfree,
+__device__ __forceinline__ void score_issuer(int nit, uint32_t bar_aop, uint32_t bar_full, uint32_t bar_sfree,
                                              uint32_t bar_drain, volatile int *abort_flag, uint64_t lim,
                                              IssueS issue_s, int lane)
 {
-    bool ok = mbar_wait_warp(bar_tile, 0, abort_flag, lim);
+    bool ok = mbar_wait_warp(bar_aop, 0, abort_flag, lim);  // the tile's A operands are in TMEM
     for (int j = 0; ok && j < nit; ++j) {
         if (!(ok = mbar_wait_warp(bar_full + 8 * (j % ST), (j / ST) & 1, abort_flag, lim))) break;
         if (j > 0 && !(ok = mbar_wait_warp(bar_sfree, (j - 1) & 1, abort_flag, lim))) break;
@@ -460,6 +493,7 @@ __global__ void __launch_bounds__(NT, 1)
         mbar_init(bar(B_AFREE), 1);
         mbar_init(bar(B_DONE), 1);
         mbar_init(bar(B_SDRAIN), 1);
+        mbar_init(bar(B_AOP), NEW);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -512,12 +546,12 @@ __global__ void __launch_bounds__(NT, 1)
             const uint32_t st = sbase + KT_STAGE0 + (j % KSTAGES) * KB_BYTES;
 #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk)
-                mma_issue(tbase + KM_S1, sw128(sbase + KT_K1 + 32 * kk), sw128(st + KB_Q1 + 32 * kk), Ids<F16QK>::S,
-                          kk > 0);
+                mma_issue_ts(tbase + KM_S1, tbase + KM_AK1 + 8 * kk, sw128(st + KB_Q1 + 32 * kk), Ids<F16QK>::S,
+                             kk > 0);
 #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk)
-                mma_issue(tbase + KM_S2, sw128(sbase + KT_K2 + 32 * kk), sw128(st + KB_Q2 + 32 * kk), Ids<F16QK>::S,
-                          kk > 0);
+                mma_issue_ts(tbase + KM_S2, tbase + KM_AK2 + 8 * kk, sw128(st + KB_Q2 + 32 * kk), Ids<F16QK>::S,
+                             kk > 0);
 #pragma unroll
             for (int kk = 0; kk < HDV / 16; ++kk) {
                 const uint32_t o = 32 * (kk & 3);
@@ -545,8 +579,8 @@ __global__ void __launch_bounds__(NT, 1)
             commit_to(bar(B_EMPTY + j % KSTAGES));
         };
         if (R.score_issuer())
-            score_issuer<KSTAGES>(nit, bar(B_TILE), bar(B_FULL), bar(B_SFREE), bar(B_SDRAIN), abort_flag, lim, issue_s,
-                               R.lane);
+            score_issuer<KSTAGES>(nit, bar(B_AOP), bar(B_FULL), bar(B_SFREE), bar(B_SDRAIN), abort_flag, lim, issue_s,
+                                  R.lane);
         else
             acc_issuer(nit, bar(B_AFULL), bar(B_DONE), abort_flag, lim, issue_acc, R.lane);
     } else {
@@ -555,8 +589,17 @@ __global__ void __launch_bounds__(NT, 1)
         const uint32_t lo = R.lane_off();
         const int kj = k0 + r;  // this thread's key
         const float c = p.scale_log2;
-        bool ok = true, big = false;
-        for (int j = 0; j < nit; ++j) {
+        // The tile's K_1 (warpgroup 0) and K_2 (warpgroup 1) rows into TMEM,
+        // the A operand of every block's score products.
+        bool ok = mbar_wait_warp(bar(B_TILE), 0, abort_flag, lim), big = false;
+        if (ok) {
+            tile_row_to_tmem(sbase + (wg ? KT_K2 : KT_K1), r, tbase + lo + (wg ? KM_AK2 : KM_AK1));
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (R.lane == 0) mbar_arrive(bar(B_AOP));
+        }
+        for (int j = 0; ok && j < nit; ++j) {
             if (!(ok = mbar_wait_warp(bar(B_SFULL), j & 1, abort_flag, lim))) break;
             tc_fence_after();
             uint32_t s1[32], s2[32], dp[32];
@@ -699,6 +742,7 @@ __global__ void __launch_bounds__(NT, 1)
         mbar_init(bar(B_AFREE), 1);
         mbar_init(bar(B_DONE), 1);
         mbar_init(bar(B_SDRAIN), 1);
+        mbar_init(bar(B_AOP), NEW);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -745,17 +789,17 @@ __global__ void __launch_bounds__(NT, 1)
             const uint32_t st = sbase + QT_STAGE0 + (j % QSTAGES) * QB_BYTES;
 #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk)
-                mma_issue(tbase + QM_S1, sw128(sbase + QT_Q1 + 32 * kk), sw128(st + QB_K1 + 32 * kk), Ids<F16QK>::S,
-                          kk > 0);
+                mma_issue_ts(tbase + QM_S1, tbase + QM_AQ1 + 8 * kk, sw128(st + QB_K1 + 32 * kk), Ids<F16QK>::S,
+                             kk > 0);
 #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk)
-                mma_issue(tbase + QM_S2, sw128(sbase + QT_Q2 + 32 * kk), sw128(st + QB_K2 + 32 * kk), Ids<F16QK>::S,
-                          kk > 0);
+                mma_issue_ts(tbase + QM_S2, tbase + QM_AQ2 + 8 * kk, sw128(st + QB_K2 + 32 * kk), Ids<F16QK>::S,
+                             kk > 0);
 #pragma unroll
             for (int kk = 0; kk < HDV / 16; ++kk) {
                 const uint32_t o = 32 * (kk & 3);
-                mma_issue(tbase + QM_DP, sw128(sbase + QT_DD + (kk >> 2) * 16384 + o),
-                          sw128(st + QB_V + (kk >> 2) * 8192 + o), ID_DP, kk > 0);
+                mma_issue_ts(tbase + QM_DP, tbase + QM_ADD + 8 * kk, sw128(st + QB_V + (kk >> 2) * 8192 + o), ID_DP,
+                             kk > 0);
             }
             commit_to(bar(B_SFULL));
         };
@@ -774,8 +818,8 @@ __global__ void __launch_bounds__(NT, 1)
             commit_to(bar(B_EMPTY + j % QSTAGES));
         };
         if (R.score_issuer())
-            score_issuer<QSTAGES>(nit, bar(B_TILE), bar(B_FULL), bar(B_SFREE), bar(B_SDRAIN), abort_flag, lim, issue_s,
-                               R.lane);
+            score_issuer<QSTAGES>(nit, bar(B_AOP), bar(B_FULL), bar(B_SFREE), bar(B_SDRAIN), abort_flag, lim, issue_s,
+                                  R.lane);
         else
             acc_issuer(nit, bar(B_AFULL), bar(B_DONE), abort_flag, lim, issue_acc, R.lane);
     } else {
@@ -786,8 +830,23 @@ __global__ void __launch_bounds__(NT, 1)
         const float *strow = p.stats + (size_t)(b * p.H + h) * kBwdStats * p.n_pad + qrow;
         const float lse1 = strow[0], lse2 = strow[p.n_pad], del1 = strow[2 * p.n_pad], del2 = strow[3 * p.n_pad];
         const float lam = strow[4 * p.n_pad];
-        bool ok = true, big = false;
-        for (int j = 0; j < nit; ++j) {
+        // The tile's Q_1, Q_2 (warpgroup 0) and dD (warpgroup 1) rows into
+        // TMEM, the A operands of every block's score and dP products.
+        bool ok = mbar_wait_warp(bar(B_TILE), 0, abort_flag, lim), big = false;
+        if (ok) {
+            if (wg == 0) {
+                tile_row_to_tmem(sbase + QT_Q1, r, tbase + lo + QM_AQ1);
+                tile_row_to_tmem(sbase + QT_Q2, r, tbase + lo + QM_AQ2);
+            } else {
+                tile_row_to_tmem(sbase + QT_DD, r, tbase + lo + QM_ADD);
+                tile_row_to_tmem(sbase + QT_DD + 16384, r, tbase + lo + QM_ADD + 32);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (R.lane == 0) mbar_arrive(bar(B_AOP));
+        }
+        for (int j = 0; ok && j < nit; ++j) {
             if (!(ok = mbar_wait_warp(bar(B_SFULL), j & 1, abort_flag, lim))) break;
             tc_fence_after();
             uint32_t s1[32], s2[32], dp[32];
