@@ -129,9 +129,11 @@ def measured_peaks():
     if os.path.exists(p):
         j = json.load(open(p))
         return dict(hbm_gbs=j["hbm_gbs"], bf16_tflops=j["bf16_tflops"],
-                    bf16_tflops_sustained=j.get("bf16_tflops_sustained"), source="measured")
+                    bf16_tflops_sustained=j.get("bf16_tflops_sustained"),
+                    source="measured (MEASURED_PEAKS.json)")
+    # The pool's earlier measurement, used when the per-pod file is absent.
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
-                source="fallback")
+                source="fallback (MEASURED_PEAKS.json absent)")
 
 
 # ------------------------------------------------------------------ distributed
@@ -645,7 +647,7 @@ def gpu_arm(args):
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1),
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(achieved / peaks["bf16_tflops"], 4),
-                     "peak_source": peaks["source"] + " bf16 burst (MEASURED_PEAKS.json)",
+                     "peak_source": "bf16 burst, " + peaks["source"],
                      "kernel": "prefill_kernel", "traffic": prefill_traffic(),
                      "traffic_unit": "bytes per launch (ncu)"},
         "gpu_launches": r["launches"] * args.steps,
@@ -686,6 +688,7 @@ def gpu_arm(args):
                            "split_kernel_gbs": round(bd / rd["kernel_s"] / 1e9, 1),
                            "roofline": {"bound": "hbm", "achieved": round(bd / rd["step_s"] / 1e9, 1),
                                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                        "peak_source": "HBM copy, " + peaks["source"],
                                         "frac": round(bd / rd["step_s"] / 1e9 / peaks["hbm_gbs"], 4)},
                            "us": round(rd["step_s"] * 1e6, 2), "launches": rd["launches"],
                            "steps": rd["steps"], "sm_mhz": cd.summary()["sm_mhz"]}
