@@ -409,14 +409,7 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
                  HV * 128, 128, da::kPrefillKeyRows) &&
         make_map(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->out, 128, a->N, a->H, a->B,
                  a->out_stride[0], a->out_stride[1], a->out_stride[2], da::kPrefillOutRows);
-    // Gate logits, laid out like the output: read by TMA boxes of the same
-    // shape (the output's map stands in when there is no gate; unused then).
-    CUtensorMap mg = mo;
-    const bool ok_gate =
-        !a->gate || make_map(&mg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->gate, 128, a->N, a->H, a->B,
-                             a->gate_stride[0], a->gate_stride[1], a->gate_stride[2],
-                             da::kPrefillOutRows);
-    if (!ok || !ok_gate) {
+    if (!ok) {
         da::set_internal_error("cuTensorMapEncodeTiled failed");
         return DIFFATTN_ERR_CUDA;
     }
@@ -495,7 +488,7 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
         p.save = static_cast<float *>(a->save);
     }
     if (g_events.start) cudaEventRecord(g_events.start, s);
-    e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, mo, mg, p, s, &launches);
+    e = da::launch_prefill(mq1, mq2, mk1, mk2, mv, mo, p, s, &launches);
     if (g_events.stop) cudaEventRecord(g_events.stop, s);
     if (e != cudaSuccess) return cuda_status(e);
     g_last_launches = launches;

@@ -36,7 +36,7 @@ struct PrefillParams {
     int lag;              // mode 1: tiles by which a group's pair items trail its export item
     float *noise_out;     // mode 1: normalised noise outputs, fp32, per (b, noise head,
                           // query tile) 32 float4 chunks x 128 rows (chunk-major)
-    int *noise_ready;     // mode 1: per (b, noise head, query tile) count of the 8 epilogue
+    int *noise_ready;     // mode 1: per (b, noise head, query tile) count of the 4 epilogue
                           // warps that have exported their part (zeroed by the staging kernel)
     const float *lambda;  // [H], unused when lam_logits is set
     const float *gain;    // [H, 128] or nullptr
@@ -68,7 +68,7 @@ constexpr unsigned kPrefillOutRows = 32;  // rows of an output store box (one wa
 // {64, rows, 1, 1} boxes (kPrefillQRows for Q, kPrefillKeyRows for K and V).
 cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const CUtensorMap &k1,
                            const CUtensorMap &k2, const CUtensorMap &v16, const CUtensorMap &out,
-                           const CUtensorMap &gate, const PrefillParams &p,
+                           const PrefillParams &p,
                            cudaStream_t stream, int *launches);
 
 // bf16 V [B, N, H_V, 128] (strided) -> contiguous fp16 copy in `dst`; also

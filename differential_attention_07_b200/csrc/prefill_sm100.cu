@@ -7,7 +7,7 @@
 // after it (same page, figure 1: GroupNorm after the subtraction, read as a
 // per-head RMS norm with gain).
 //
-// A persistent kernel: one CTA per SM (384 threads, three warpgroups) takes
+// A persistent kernel: one CTA per SM (512 threads, four warpgroups) takes
 // work items -- (b, unit, 128-row query tile) -- from a global counter until
 // none are left.
 //   warp 0        TMA producer: takes the next item, publishes it to the
@@ -18,16 +18,18 @@
 //                 and V (fp16) from the shared-memory tile both maps use.
 //   warps 4-7     softmax of map 1 (one thread per query row).
 //   warps 8-11    softmax of map 2.  A warp reaches TMEM lanes 32 (warp % 4)
-//                 onwards, so each warpgroup covers all 128 rows.  Both
-//                 softmax warpgroups then run the epilogue, 64 output columns
-//                 each: D = (O1 - r O2)/l1 with r = lambda l1/l2, RMS norm
-//                 (sum of squares exchanged through shared memory), gain,
-//                 optional output gate sigma(G) (lambda optionally sigma of a
-//                 per-token logit: Motif 3 summary, section 2.2), bf16, staged
-//                 in each warp's shared-memory buffer and written by TMA
-//                 stores.
-//                 Registers are split 56 / 224 / 224 between the warpgroups
-//                 (setmaxnreg).
+//                 onwards, so each warpgroup covers all 128 rows.  At the end
+//                 of a tile the softmax warps hand their row sums to the
+//                 epilogue warps and go straight on to the next tile.
+//   warps 12-15   epilogue, 32 rows per warp, overlapping the next tile's
+//                 softmax: D = (O1 - r O2)/l1 with r = lambda l1/l2, RMS norm
+//                 over the row's 128 columns, gain, optional output gate
+//                 sigma(G) (lambda optionally sigma of a per-token logit:
+//                 Motif 3 summary, section 2.2), bf16, staged in each warp's
+//                 shared-memory buffer and written by TMA stores.  O goes
+//                 back to the MMA warps as soon as it has been read.
+//                 Registers are split 56 / 152 / 152 / 152 between the
+//                 warpgroups (setmaxnreg).
 // TMEM (512 columns): O1 [0,128) O2 [128,256), and two 64-column S buffers
 // per map: S1 [256,320) [320,384), S2 [384,448) [448,512).  P (fp16, two per
 // column) overwrites the first 32 columns of its S buffer.
@@ -64,7 +66,7 @@ constexpr int BN = 64;    // keys per step (MMA N of S, K of P.V)
 constexpr int HD = 64;    // Q/K head dim
 constexpr int HDV = 128;  // V head dim (MMA N of P.V)
 constexpr int STAGES = 4;
-constexpr int NTHREADS = 384;
+constexpr int NTHREADS = 512;
 
 constexpr uint32_t Q_BYTES = BM * HD * 2;           // 16 KB
 constexpr uint32_t K_BYTES = BN * HD * 2;           // 8 KB
@@ -86,13 +88,12 @@ enum : int {
     B_P = B_S + 4,               // [2 maps][2 buffers] P written (4 softmax warps)
     B_PV = B_P + 4,              // [2 maps] latest P.V into O done (commit)
     B_O = B_PV + 2,              // all MMAs of the tile done (2 commits)
-    B_OFREE = B_O + 1,           // epilogue finished reading O (8 softmax warps)
-    B_LX = B_OFREE + 1,          // row sums exchanged (8 softmax warps)
-    B_SSX = B_LX + 1,            // partial sums of squares exchanged (8 softmax warps)
-    B_ITEM = B_SSX + 1,          // [ITEM_SLOTS] work item published (1 arrival)
+    B_OFREE = B_O + 1,           // epilogue finished reading O (4 epilogue warps)
+    B_STAT = B_OFREE + 1,        // [2 tile parities] row sums written (8 softmax warps)
+    B_ITEM = B_STAT + 2,         // [ITEM_SLOTS] work item published (1 arrival)
     B_ITEMFREE = B_ITEM + 4,     // [ITEM_SLOTS] work item read by all 10 reader warps
-    B_GATE = B_ITEMFREE + 4,     // [8 softmax warps] the warp's gate-logit box landed (TMA bytes)
-    NBARS = B_GATE + 8
+    B_AN = B_ITEMFREE + 4,       // [4 epilogue warps] the warp's A_N rows landed (bulk-copy bytes)
+    NBARS = B_AN + 4
 };
 // S and P barriers come one per S buffer: a softmax may run two steps ahead
 // of its MMA warp's wait, and with one P barrier per map the second arrival
@@ -104,28 +105,32 @@ enum : int {
 constexpr uint32_t OFF_TMEM_PTR = OFF_BARS + NBARS * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
 constexpr int ITEM_SLOTS = 4;
-constexpr int ITEM_READERS = 10;                         // 2 MMA warps + 8 softmax warps
+constexpr int ITEM_READERS = 14;                         // 2 MMA, 8 softmax and 4 epilogue warps
 constexpr uint32_t OFF_ITEM = OFF_ABORT + 4;             // int [ITEM_SLOTS] work-item ring
-constexpr uint32_t OFF_L = (OFF_ITEM + 4 * ITEM_SLOTS + 15) & ~15u;  // float [2][128] row sums
-constexpr uint32_t OFF_SS = OFF_L + 2 * BM * 4;          // float [2][128] partial sums of squares
-// Output staging: per softmax warp 32 rows x 128 columns bf16 (two 4 KB
-// halves, each one 128-byte-swizzled TMA store box of 32 rows x 64 columns).
+// float [2 tile parities][l1, l2][128]: the softmax warps' row sums
+constexpr uint32_t OFF_STAT = (OFF_ITEM + 4 * ITEM_SLOTS + 15) & ~15u;
+// Epilogue buffers: per epilogue warp 16 KB.  A one-head item keeps its 32
+// rows of D there in fp32 and then the staged output, two 32 x 64 bf16 TMA
+// store boxes of 4 KB with the 128-byte swizzle; a pair item keeps its 32
+// rows of the group's noise output A_N (fp32) there.
 constexpr uint32_t OUT_HALF_BYTES = 32 * 64 * 2;
-constexpr uint32_t OUT_WARP_BYTES = 2 * OUT_HALF_BYTES;
-constexpr uint32_t OFF_OUT = (OFF_SS + 2 * BM * 4 + 1023) & ~1023u;
-constexpr uint32_t SMEM_BYTES = OFF_OUT + 8 * OUT_WARP_BYTES;  // dynamic smem is 1024-byte aligned
+constexpr uint32_t EPI_WARP_BYTES = 4 * OUT_HALF_BYTES;
+constexpr uint32_t OFF_OUT = (OFF_STAT + 2 * 2 * BM * 4 + 1023) & ~1023u;
+constexpr uint32_t SMEM_BYTES = OFF_OUT + 4 * EPI_WARP_BYTES;  // dynamic smem is 1024-byte aligned
 
 constexpr uint32_t TM_O1 = 0, TM_O2 = 128, TM_S1 = 256, TM_S2 = 384;
 constexpr uint32_t TMEM_COLS = 512;
 
-// Registers per thread: at launch (the most __launch_bounds__(384, 1) allows:
-// three warps per SM sub-partition share its 16K registers), and after the
-// split between the producer/MMA warpgroup and the two softmax warpgroups.
-constexpr int REGS_LAUNCH = 168;
+// Registers per thread: at launch (the most __launch_bounds__(512, 1) allows:
+// four warps per SM sub-partition share its 16K registers), and after the
+// split between the producer/MMA warpgroup, the two softmax warpgroups and
+// the epilogue warpgroup.  Each sub-partition holds one warp of each.
+constexpr int REGS_LAUNCH = 128;
 constexpr int REGS_IO = 56;
-constexpr int REGS_SOFTMAX = 224;
-static_assert(REGS_IO + 2 * REGS_SOFTMAX == 3 * REGS_LAUNCH, "register split must use the pool exactly");
-static_assert(NTHREADS == 384, "three warpgroups");
+constexpr int REGS_SOFTMAX = 152;
+constexpr int REGS_EPI = 152;
+static_assert(REGS_IO + 2 * REGS_SOFTMAX + REGS_EPI == 4 * REGS_LAUNCH, "register split must use the pool exactly");
+static_assert(NTHREADS == 512, "four warpgroups");
 
 // The producer warms L2 with the K/V of the step this many steps ahead.
 constexpr int L2_PREFETCH_STEPS = 8;
@@ -356,9 +361,13 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, bool firs
 
     const bool need = tmax > m_run + RESCALE_THRESHOLD;
     const float m_new = need ? tmax : m_run;
+    // A row that has seen no key yet (m_run = -inf: every P of it so far was
+    // 0, so its O row and l are 0) takes its first maximum without a rescale.
+    // Under a sliding window that is most rows of a tile's first steps.
+    const bool scale_o = need && m_run != -INFINITY;
     float alpha = 1.0f;
-    if (__any_sync(0xffffffffu, need)) {  // rare after a row's first step
-      alpha = need ? ex2_approx(m_run - m_new) : 1.0f;  // ex2(-inf) = 0
+    if (__any_sync(0xffffffffu, scale_o)) {  // rare after a row's first visible step
+      alpha = scale_o ? ex2_approx(m_run - m_new) : 1.0f;
       if (!first) {
         // O holds P.V products up to the previous step; the last one must be
         // finished before the row is rescaled.
@@ -411,7 +420,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q1, const __grid_constant__ CUtensorMap tm_q2,
                    const __grid_constant__ CUtensorMap tm_k1, const __grid_constant__ CUtensorMap tm_k2,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
-                   const __grid_constant__ CUtensorMap tm_gate, const PrefillParams p)
+                   const PrefillParams p)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_addr(smem);
@@ -441,8 +450,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     auto bar_p = [&](int t, int b) { return bar(B_P + 2 * t + b); };
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_ABORT);
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + OFF_TMEM_PTR);
-    float *sL = reinterpret_cast<float *>(smem + OFF_L);
-    float *sSS = reinterpret_cast<float *>(smem + OFF_SS);
+    float *sStat = reinterpret_cast<float *>(smem + OFF_STAT);
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_QFULL), 1);
@@ -458,14 +466,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_init(bar(B_PV), 1);
         mbar_init(bar(B_PV + 1), 1);
         mbar_init(bar(B_O), 2);
-        mbar_init(bar(B_OFREE), 8);   // one arrival per softmax warp
-        mbar_init(bar(B_LX), 8);    // one arrival per softmax warp
-        mbar_init(bar(B_SSX), 8);
+        mbar_init(bar(B_OFREE), 4);   // one arrival per epilogue warp
+        mbar_init(bar(B_STAT), 8);    // one arrival per softmax warp
+        mbar_init(bar(B_STAT + 1), 8);
+        for (int i = 0; i < 4; ++i) mbar_init(bar(B_AN + i), 1);
         for (int i = 0; i < ITEM_SLOTS; ++i) {
             mbar_init(bar(B_ITEM + i), 1);
             mbar_init(bar(B_ITEMFREE + i), ITEM_READERS);
         }
-        for (int i = 0; i < 8; ++i) mbar_init(bar(B_GATE + i), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -501,7 +509,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         return item;
     };
 
-    // Register split: 128 x REGS_LAUNCH = 128 x REGS_IO + 256 x REGS_SOFTMAX
+    // Register split: 4 x REGS_LAUNCH = REGS_IO + 2 x REGS_SOFTMAX + REGS_EPI per thread slot
     // (the host launches only when the kernel was built with REGS_LAUNCH).
     // Each budget change opens its role's branch so that the compiler
     // allocates each branch within its own budget.
@@ -670,18 +678,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const bool drained = mbar_wait_drain(bar(B_PV + t), g & 1, lim);
         if (!__all_sync(0xffffffffu, drained) && lane == 0) *abort_flag = 1;
       }
-    } else {
+    } else if (warp < 12) {
         regs_increase<REGS_SOFTMAX>();
-        // ------------------------------------------------------------ softmax + epilogue
+        // ------------------------------------------------------------ softmax
         const int t = (warp >= 8) ? 1 : 0;
         const int r = (warp & 3) * 32 + lane;
         const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
         const uint32_t tS0 = tbase + lane_off + (t ? TM_S2 : TM_S1);
         const uint32_t tO = tbase + lane_off + (t ? TM_O2 : TM_O1);
-        const uint32_t tO1 = tbase + lane_off + TM_O1, tO2 = tbase + lane_off + TM_O2;
         const uint32_t bar_pv = bar(B_PV + t);
         int g = 0;
-        int shared_eps = 0;  // tiles finished by the shared epilogue (phases of B_LX, B_SSX)
         bool ok = true;
         for (int tiles = 0;; ++tiles) {
             const int item = next_item(tiles);
@@ -689,29 +695,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const Work w = work_of(item, p);
             const int nkv = steps_of(w), kv0 = kv_first(w);
             const int qrow = w.qt * BM + r;
-            const Heads hd = heads_of(w.u, p);
-            // Output head of this warpgroup: both finish head a together (64
-            // columns each), except in a pair item, where each finishes its own.
-            const bool own = hd.own;
-            const int head = (own && t) ? hd.b : hd.a;
-            // The epilogue's lambda (per head, or the token-dependent logit of
-            // this row), gain, gate logits (and in a pair item the group's noise
-            // output row): load / prefetch them now so the global-memory
-            // latency hides behind the softmax loop.
-            const int64_t qrow_c = min(qrow, p.N - 1);
-            const float lam_in = ld_early_f32(
-                p.lam_logits ? p.lam_logits + w.b * p.ll_sb + qrow_c * p.ll_sn + head * p.ll_sh
-                             : p.lambda + head);
-            // (Gate logits arrive by TMA into this warp's output staging
-            // buffer, one 32-row box per 64 columns, when the epilogue starts.)
-            const float *gain = p.gain ? p.gain + (size_t)head * HDV + (own ? 0 : 64 * t) : nullptr;
-            if (gain && lane < (own ? 4 : 2)) prefetch_l1(gain + 32 * lane);
-            // The group's noise outputs of this tile, stored tile-transposed:
-            // float4 chunk c (columns 4c .. 4c + 3) of tile row r at c * 128 + r,
-            // so a warp reading chunk c of its 32 rows reads 512 contiguous bytes.
-            const size_t noise_tile = ((size_t)w.b * p.H_N + hd.n) * p.num_qt + w.qt;
-            const float4 *an_tile =
-                own ? reinterpret_cast<const float4 *>(p.noise_out) + noise_tile * (HDV / 4) * BM : nullptr;
             float m_run = -INFINITY, l_run = 0.0f;
             for (int j = 0; j < nkv; ++j) {
                 const int gg = g + j, buf = gg & 1;
@@ -731,276 +714,373 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (!ok) break;
             g += nkv;
-            if (own) {
-                // ------------------------------------------------ epilogue, pair item
-                // This warpgroup's head alone: D = O / l - lambda A_N with A_N
-                // the group's normalised noise output (written by the tile's
-                // export item), then the RMS norm over the 128 columns of the row.
-                if constexpr (GATED) {  // once the previous store has read this warp's buffer
-                    if (elect_one()) {
-                        const uint32_t gbuf = sbase + OFF_OUT + (warp - 4) * OUT_WARP_BYTES;
-                        const uint32_t gbar = bar(B_GATE + (warp - 4));
-                        bulk_wait_read_all();
-                        mbar_arrive_expect_tx(gbar, OUT_WARP_BYTES);
-                        tma_load_4d_nohint(gbuf, &tm_gate, gbar, 0, w.qt * BM + 32 * (warp & 3), head, w.b);
-                        tma_load_4d_nohint(gbuf + OUT_HALF_BYTES, &tm_gate, gbar, 64, w.qt * BM + 32 * (warp & 3),
-                                           head, w.b);
-                    }
-                    __syncwarp();
+            if constexpr (SAVE) {
+                // Saved for the backward pass: this map's lse = m + log2(l)
+                // (the running max and sum are in units of scale * log2(e) *
+                // score), at float 2 * 128 * 128 + 128 t + r of the tile's state.
+                const int head = heads_of(w.u, p).a;
+                p.save[((size_t)(w.b * p.H + head) * p.num_qt + w.qt) * kSaveTileFloats + 2 * BM * HDV + t * BM + r] =
+                    m_run + log2f(l_run);
+            }
+            // The row's running sum goes to the epilogue warps, in the slot of
+            // the tile's parity.  The epilogue reads the slot before it
+            // releases O; this warp writes the slot again two tiles later,
+            // after the MMA warps have waited for that release.
+            sStat[(tiles & 1) * (2 * BM) + t * BM + r] = l_run;
+            __syncwarp();  // every lane's sum is written: one arrival for the warp
+            if (lane == 0) mbar_arrive(bar(B_STAT + (tiles & 1)));
+        }
+    } else {
+        regs_increase<REGS_EPI>();
+        // ------------------------------------------------------------ epilogue
+        // Warp 12 + e finishes tile rows 32 e .. 32 e + 31 (its TMEM lanes)
+        // over all 128 output columns, while the softmax warps run the next
+        // tile.  Per item it waits for the softmax warps' row sums and for
+        // the tile's last P.V, reads O1 and O2, and writes the output rows.
+        const int ew = warp & 3;
+        const int r = 32 * ew + lane;
+        const uint32_t lane_off = uint32_t(32 * ew) << 16;
+        const uint32_t tO1 = tbase + lane_off + TM_O1, tO2 = tbase + lane_off + TM_O2;
+        // This warp's 16 KB of shared memory: the staged output boxes (two 32
+        // x 64 bf16 boxes per output head, 128-byte swizzle) and, in a
+        // one-head item, first D itself in fp32.
+        const uint32_t wbuf = sbase + OFF_OUT + ew * EPI_WARP_BYTES;
+        // 16-byte chunk ch of row `lane` of an output box (the TMA swizzle).
+        auto box_at = [&](uint32_t box, int ch) { return box + 128 * lane + ((ch ^ (lane & 7)) << 4); };
+        const uint32_t abar = bar(B_AN + ew);  // this warp's A_N copies landed
+        int an_loads = 0;
+        bool ok = true;
+        for (int tiles = 0;; ++tiles) {
+            const int item = next_item(tiles);
+            if (item < 0) break;
+            const Work w = work_of(item, p);
+            const Heads hd = heads_of(w.u, p);
+            const bool own = hd.own;
+            const int qrow = w.qt * BM + r;
+            const int64_t qrow_c = min(qrow, p.N - 1);
+            const int r0 = w.qt * BM + 32 * ew;  // first row of this warp's boxes
+            // The per-item inputs of the epilogue -- lambda (per head, or the
+            // token-dependent logit of this row), the gain rows, the gate
+            // logits' rows -- are loaded or prefetched now: the wait below
+            // hides their latency.
+            auto lam_load = [&](int head) {
+                return ld_early_f32(p.lam_logits ? p.lam_logits + w.b * p.ll_sb + qrow_c * p.ll_sn + head * p.ll_sh
+                                                 : p.lambda + head);
+            };
+            const float lam_a = lam_load(hd.a);
+            const float lam_b = own ? lam_load(hd.b) : 0.0f;
+            const float *gain_a = p.gain ? p.gain + (size_t)hd.a * HDV : nullptr;
+            const float *gain_b = p.gain ? p.gain + (size_t)hd.b * HDV : nullptr;
+            if (gain_a && lane < 4) prefetch_l1(gain_a + 32 * lane);
+            if (own && gain_b && lane < 4) prefetch_l1(gain_b + 32 * lane);
+            const uint4 *gate_a = nullptr, *gate_b = nullptr;  // this row's 128 logits: 16 chunks of 8
+            if constexpr (GATED) {
+                const __nv_bfloat16 *g0 =
+                    static_cast<const __nv_bfloat16 *>(p.gate) + w.b * p.gate_sb + qrow_c * p.gate_sn;
+                gate_a = reinterpret_cast<const uint4 *>(g0 + hd.a * p.gate_sh);
+                prefetch_l2(gate_a);
+                prefetch_l2(gate_a + 8);
+                if (own) {
+                    gate_b = reinterpret_cast<const uint4 *>(g0 + hd.b * p.gate_sh);
+                    prefetch_l2(gate_b);
+                    prefetch_l2(gate_b + 8);
                 }
-                // The export item of this tile ran about one wave of items
-                // earlier; its eight epilogue warps have normally all
-                // published their half-rows by now.  (Plain L2 loads below: the
-                // data was written during this launch.)  The first half of
-                // this row's A_N is loaded while the tile's last P.V runs.
-                bool ready = true;
-                if (lane == 0) ready = wait_flag_geq(p.noise_ready + noise_tile, 8, abort_flag, lim);
-                if (!(ok = __shfl_sync(0xffffffffu, ready, 0))) break;
-                float4 an[16];
+            }
+            const size_t noise_tile = ((size_t)w.b * p.H_N + hd.n) * p.num_qt + w.qt;
+            // Gain times output gate for 16 columns (16 c ..) of one head; gq:
+            // the gate logits of those columns, loaded one step ahead.
+            auto scale16 = [&](const float *gain, const uint4 (&gq)[2], int c, float (&gv)[16]) {
 #pragma unroll
-                for (int i4 = 0; i4 < 16; ++i4) an[i4] = __ldcg(an_tile + i4 * BM + r);
-                if (!(ok = mbar_wait_warp(bar(B_O), tiles & 1, abort_flag, lim))) break;
-                // The gate box (issued above) has had the last P.V's time to land.
-                if (GATED && !(ok = mbar_wait_warp(bar(B_GATE + (warp - 4)), tiles & 1, abort_flag, lim)))
-                    break;
-                tc_fence_after();
-                const float inv = 1.0f / l_run;
-                const float lam = p.lam_logits ? logistic_fast(lam_in) : lam_in;
-                // Pass 1: sum of squares of D over the row, 64 columns at a
-                // time (the first half with the prefetched A_N, then the
-                // second half, whose A_N stays in registers for pass 2).
-                float ss = 0.0f;
-                auto sum_sq = [&](int hh) {
-                    uint32_t o[2][32];
-                    tmem_ld32(tO + 64 * hh, o[0]);
-                    tmem_ld32(tO + 64 * hh + 32, o[1]);
-                    tmem_wait_ld();
+                for (int k = 0; k < 4; ++k) {
+                    const float4 g4 = gain ? __ldg(reinterpret_cast<const float4 *>(gain) + 4 * c + k)
+                                           : make_float4(1.f, 1.f, 1.f, 1.f);
+                    gv[4 * k] = g4.x;
+                    gv[4 * k + 1] = g4.y;
+                    gv[4 * k + 2] = g4.z;
+                    gv[4 * k + 3] = g4.w;
+                }
+                if constexpr (GATED) {
 #pragma unroll
-                    for (int i4 = 0; i4 < 16; ++i4) {
-                        const float av[4] = {an[i4].x, an[i4].y, an[i4].z, an[i4].w};
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t qw[4] = {gq[h].x, gq[h].y, gq[h].z, gq[h].w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float dd = fmaf(-lam, av[e], __uint_as_float(o[i4 >> 3][4 * (i4 & 7) + e]) * inv);
-                            ss = fmaf(dd, dd, ss);
+                        for (int k = 0; k < 4; ++k) {
+                            gv[8 * h + 2 * k] *= logistic_tanh(__uint_as_float(qw[k] << 16));
+                            gv[8 * h + 2 * k + 1] *= logistic_tanh(__uint_as_float(qw[k] & 0xffff0000u));
                         }
                     }
-                };
-                sum_sq(0);
-#pragma unroll
-                for (int i4 = 0; i4 < 16; ++i4) an[i4] = __ldcg(an_tile + (16 + i4) * BM + r);
-                sum_sq(1);
-                const float rn = p.apply_norm ? rsqrtf(ss * (1.0f / HDV) + p.eps) : 1.0f;
-                // This warp's staging buffer: the previous tile's store must
-                // have read it (and the gate box must have landed in it).
-                const uint32_t obuf = sbase + OFF_OUT + (warp - 4) * OUT_WARP_BYTES;
-                if (lane == 0) bulk_wait_read_all();
-                __syncwarp();
-                // Pass 2: D again, normalised, gain, bf16, stored; the second
-                // half first (its A_N is still in registers), and O is
-                // released after its last read.
-                auto write_half = [&](int hh) {
-                    uint32_t o[2][32];
-                    tmem_ld32(tO + 64 * hh, o[0]);
-                    tmem_ld32(tO + 64 * hh + 32, o[1]);
+                }
+            };
+            // Row sums of the tile, from the softmax warps.
+            if (!(ok = mbar_wait_warp(bar(B_STAT + (tiles & 1)), (tiles >> 1) & 1, abort_flag, lim))) break;
+            const float l1 = sStat[(tiles & 1) * (2 * BM) + r], l2 = sStat[(tiles & 1) * (2 * BM) + BM + r];
+            // The previous item's output stores must have read the buffer.
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+            if (!own) {
+                // -------------------------------------------- one output head
+                // D = (O1 - r2 O2) / l1 with r2 = lambda l1 / l2 (identical
+                // maps with lambda = 1 cancel exactly), then the RMS norm over
+                // the row's 128 columns, gain, gate, bf16.
+                if (!(ok = mbar_wait_warp(bar(B_O), tiles & 1, abort_flag, lim))) break;
+                tc_fence_after();
+                const float lam = p.lam_logits ? logistic_fast(lam_a) : lam_a;
+                const float inv1 = 1.0f / l1, inv2 = 1.0f / l2, r2 = lam * l1 / l2;
+                const uint32_t drow = wbuf + 64 * lane;
+                const int rot = (lane >> 1) & 3;
+                float4 *sa = SAVE ? reinterpret_cast<float4 *>(p.save + ((size_t)(w.b * p.H + hd.a) * p.num_qt + w.qt) *
+                                                                            kSaveTileFloats) + r
+                                  : nullptr;
+                float4 *an = p.mode == 1
+                                 ? reinterpret_cast<float4 *>(p.noise_out) + noise_tile * (HDV / 4) * BM + r
+                                 : nullptr;
+                float ss = 0.0f;
+#pragma unroll 2
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t oa[16], ob[16];
+                    tmem_ld16(tO1 + 16 * c, oa);
+                    tmem_ld16(tO2 + 16 * c, ob);
                     tmem_wait_ld();
-                    if (hh == 0) {  // O read to registers by every lane: release it, once per warp
+                    if (c == 7) {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(bar(B_OFREE));
                     }
-                    uint32_t y[32];
+                    float d[16];
 #pragma unroll
-                    for (int i4 = 0; i4 < 16; ++i4) {
-                        const float4 a4 = an[i4];
-                        const float4 g4 = gain ? __ldg(reinterpret_cast<const float4 *>(gain) + 16 * hh + i4)
-                                               : make_float4(1.f, 1.f, 1.f, 1.f);
-                        float4 s4 = make_float4(rn, rn, rn, rn);  // norm x output gate
-                        if constexpr (GATED) {  // gate columns 4 i4 .. 4 i4 + 3 of this half, from the box
-                            const uint2 gq = ld_shared_v2(obuf + OUT_HALF_BYTES * hh + 128 * lane +
-                                                          ((((i4 >> 1) ^ (lane & 7)) << 4) | (8 * (i4 & 1))));
-                            s4.x *= logistic_tanh(__uint_as_float(gq.x << 16));
-                            s4.y *= logistic_tanh(__uint_as_float(gq.x & 0xffff0000u));
-                            s4.z *= logistic_tanh(__uint_as_float(gq.y << 16));
-                            s4.w *= logistic_tanh(__uint_as_float(gq.y & 0xffff0000u));
-                        }
-                        const uint32_t *oc = &o[i4 >> 3][4 * (i4 & 7)];
-                        const float d0 = fmaf(-lam, a4.x, __uint_as_float(oc[0]) * inv);
-                        const float d1 = fmaf(-lam, a4.y, __uint_as_float(oc[1]) * inv);
-                        const float d2 = fmaf(-lam, a4.z, __uint_as_float(oc[2]) * inv);
-                        const float d3 = fmaf(-lam, a4.w, __uint_as_float(oc[3]) * inv);
-                        y[2 * i4] = pack_bf162(d0 * s4.x * g4.x, d1 * s4.y * g4.y);
-                        y[2 * i4 + 1] = pack_bf162(d2 * s4.z * g4.z, d3 * s4.w * g4.w);
+                    for (int i = 0; i < 16; ++i) {
+                        d[i] = fmaf(-r2, __uint_as_float(ob[i]), __uint_as_float(oa[i]));
+                        ss = fmaf(d[i], d[i], ss);
                     }
-                    // 16-byte chunk i of this row goes to chunk i ^ (row % 8)
-                    // of its 128-byte line (the TMA 128-byte swizzle).
-                    const uint32_t rowb = obuf + OUT_HALF_BYTES * hh + 128 * lane;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        st_shared_v4(rowb + ((i ^ (lane & 7)) << 4), y[4 * i], y[4 * i + 1], y[4 * i + 2],
-                                     y[4 * i + 3]);
-                };
-                write_half(1);
+                    for (int k = 0; k < 4; ++k)
+                        st_shared_v4(drow + 2048 * c + ((k ^ rot) << 4), __float_as_uint(d[4 * k]),
+                                     __float_as_uint(d[4 * k + 1]), __float_as_uint(d[4 * k + 2]),
+                                     __float_as_uint(d[4 * k + 3]));
+                    if constexpr (SAVE) {
 #pragma unroll
-                for (int i4 = 0; i4 < 16; ++i4) an[i4] = __ldcg(an_tile + i4 * BM + r);
-                write_half(0);
+                        for (int k = 0; k < 4; ++k) {
+                            sa[(4 * c + k) * BM] = make_float4(
+                                __uint_as_float(oa[4 * k]) * inv1, __uint_as_float(oa[4 * k + 1]) * inv1,
+                                __uint_as_float(oa[4 * k + 2]) * inv1, __uint_as_float(oa[4 * k + 3]) * inv1);
+                            sa[(32 + 4 * c + k) * BM] = make_float4(
+                                __uint_as_float(ob[4 * k]) * inv2, __uint_as_float(ob[4 * k + 1]) * inv2,
+                                __uint_as_float(ob[4 * k + 2]) * inv2, __uint_as_float(ob[4 * k + 3]) * inv2);
+                        }
+                    }
+                    if (an) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            an[(4 * c + k) * BM] = make_float4(
+                                __uint_as_float(ob[4 * k]) * inv2, __uint_as_float(ob[4 * k + 1]) * inv2,
+                                __uint_as_float(ob[4 * k + 2]) * inv2, __uint_as_float(ob[4 * k + 3]) * inv2);
+                    }
+                }
+                ss *= inv1 * inv1;
+                const float rn = (p.apply_norm ? rsqrtf(ss * (1.0f / HDV) + p.eps) : 1.0f) * inv1;
+                // Pass 2, 32 columns at a time: D' back from shared memory,
+                // normalised, scaled and rounded to bf16 into the output boxes,
+                // which overlay the first 8 KB of the buffer: box half h holds
+                // columns 64 h .. 64 h + 63 over D chunks 2 h and 2 h + 1.
+                // Columns 32 q .. 32 q + 31 go to box half q / 2, whose D chunks
+                // every lane has read by then (this pass or the one before),
+                // hence the warp sync between the reads and the writes.
+                uint4 gcur[2][2], gnext[2][2];  // gate logits of columns 32 q .. 32 q + 31, then of the next q
+                if constexpr (GATED) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        gcur[h][0] = __ldg(gate_a + 2 * h);
+                        gcur[h][1] = __ldg(gate_a + 2 * h + 1);
+                    }
+                }
+#pragma unroll 1
+                for (int q = 0; q < 4; ++q) {
+                    if (GATED && q < 3) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            gnext[h][0] = __ldg(gate_a + 4 * (q + 1) + 2 * h);
+                            gnext[h][1] = __ldg(gate_a + 4 * (q + 1) + 2 * h + 1);
+                        }
+                    }
+                    float d[2][16];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint4 v = ld_shared_v4(drow + 2048 * (2 * q + h) + ((k ^ rot) << 4));
+                            d[h][4 * k] = __uint_as_float(v.x);
+                            d[h][4 * k + 1] = __uint_as_float(v.y);
+                            d[h][4 * k + 2] = __uint_as_float(v.z);
+                            d[h][4 * k + 3] = __uint_as_float(v.w);
+                        }
+                    __syncwarp();
+                    const uint32_t box = wbuf + (q >> 1) * OUT_HALF_BYTES;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        float gv[16];
+                        scale16(gain_a, gcur[h], 2 * q + h, gv);
+                        uint32_t y[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            y[i] = pack_bf162(d[h][2 * i] * rn * gv[2 * i], d[h][2 * i + 1] * rn * gv[2 * i + 1]);
+                        const int ch = 4 * (q & 1) + 2 * h;  // 16-byte chunk of the box row
+                        st_shared_v4(box_at(box, ch), y[0], y[1], y[2], y[3]);
+                        st_shared_v4(box_at(box, ch + 1), y[4], y[5], y[6], y[7]);
+                    }
+                    if constexpr (GATED) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            gcur[h][0] = gnext[h][0];
+                            gcur[h][1] = gnext[h][1];
+                        }
+                    }
+                }
+            } else {
+                // -------------------------------------------- pair item
+                // Two output heads, one per map: D_h = O_h / l_h - lambda_h A_N
+                // with A_N the group's normalised noise output (written by the
+                // tile's export item), then each head's RMS norm.  This warp's
+                // 32 rows of A_N (16 KB) come into its buffer by bulk copies,
+                // 512 contiguous bytes per float4 chunk (chunk j of row `lane`
+                // at 512 j + 16 lane).  O is read twice (sums of squares, then
+                // the output) and released after the second read; the output
+                // rows go straight from registers to global memory.
+                bool ready = true;
+                if (lane == 0) ready = wait_flag_geq(p.noise_ready + noise_tile, 4, abort_flag, lim);
+                if (!(ok = __shfl_sync(0xffffffffu, ready, 0))) break;
+                // The buffer's last generic-proxy reads and writes (the previous
+                // item's) come before the copies into it; the acquired A_N
+                // comes before the copies' reads of it.
                 fence_proxy_async_smem();
                 __syncwarp();
-                const int r0 = w.qt * BM + 32 * (warp & 3);
-                if (lane == 0 && r0 < p.N) {  // a box wholly past N is not issued
-                    tma_store_4d(&tm_out, obuf, 0, r0, head, w.b);
-                    tma_store_4d(&tm_out, obuf + OUT_HALF_BYTES, 64, r0, head, w.b);
-                    bulk_commit_group();
-                }
-                continue;
-            }
-            // ---------------------------------------------------- epilogue
-            // Both warpgroups finish the tile: warpgroup t writes the output
-            // columns [64 t, 64 t + 64) of every row.  D = (O1 - r O2) / l1
-            // with r = lambda l1 / l2 (one fused multiply-add per element;
-            // identical maps with lambda = 1 cancel exactly), then the RMS
-            // norm over all 128 columns, whose sum of squares is exchanged.
-            if constexpr (GATED) {  // once the previous store has read this warp's buffer
                 if (elect_one()) {
-                    const uint32_t gbuf = sbase + OFF_OUT + (warp - 4) * OUT_WARP_BYTES;
-                    const uint32_t gbar = bar(B_GATE + (warp - 4));
-                    bulk_wait_read_all();
-                    mbar_arrive_expect_tx(gbar, OUT_HALF_BYTES);
-                    tma_load_4d_nohint(gbuf, &tm_gate, gbar, 64 * t, w.qt * BM + 32 * (warp & 3), hd.a, w.b);
+                    fence_proxy_async_global();
+                    const float4 *src = reinterpret_cast<const float4 *>(p.noise_out) + noise_tile * (HDV / 4) * BM +
+                                        32 * ew;
+                    mbar_arrive_expect_tx(abar, 32 * 512);
+                    for (int j = 0; j < 32; ++j) bulk_load_g2s(wbuf + 512 * j, src + j * BM, 512, abar);
                 }
                 __syncwarp();
-            }
-            sL[t * BM + r] = l_run;
-            __syncwarp();  // every lane's row sum is written: one arrival for the warp
-            if (lane == 0) mbar_arrive(bar(B_LX));
-            if (!(ok = mbar_wait_warp(bar(B_LX), shared_eps & 1, abort_flag, lim))) break;
-            if (!(ok = mbar_wait_warp(bar(B_O), tiles & 1, abort_flag, lim))) break;
-            tc_fence_after();
-            const float l1 = sL[r], l2 = sL[BM + r];
-            const float lam = p.lam_logits ? logistic_fast(lam_in) : lam_in;
-            const float inv1 = 1.0f / l1, r2 = lam * l1 / l2;
-            const uint32_t c0 = 64 * t;
-            // One read of this half of O1 and O2; D stays in registers, and O
-            // is released to the MMA warps (the next tile's first P.V
-            // overwrites it) as soon as the read has completed.
-            uint32_t oa[2][32], ob[2][32];
-            tmem_ld32(tO1 + c0, oa[0]);
-            tmem_ld32(tO1 + c0 + 32, oa[1]);
-            tmem_ld32(tO2 + c0, ob[0]);
-            tmem_ld32(tO2 + c0 + 32, ob[1]);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_OFREE));  // once per warp, after every lane's read
-            if constexpr (SAVE) {
-                // Saved for the backward pass (mode 0): this half's columns of
-                // A_1 = O1 / l1 and A_2 = O2 / l2, chunk-major like the noise
-                // outputs, and this warpgroup's map's lse = m + log2(l) (the
-                // running max and sum are in units of scale * log2(e) * score).
-                float *tile = p.save + ((size_t)(w.b * p.H + hd.a) * p.num_qt + w.qt) * kSaveTileFloats;
-                float4 *sa = reinterpret_cast<float4 *>(tile) + (c0 / 4) * BM + r;
-                const float inv2 = 1.0f / l2;
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-#pragma unroll
-                    for (int i4 = 0; i4 < 8; ++i4) {
-                        sa[(8 * c + i4) * BM] = make_float4(
-                            __uint_as_float(oa[c][4 * i4]) * inv1, __uint_as_float(oa[c][4 * i4 + 1]) * inv1,
-                            __uint_as_float(oa[c][4 * i4 + 2]) * inv1, __uint_as_float(oa[c][4 * i4 + 3]) * inv1);
-                        sa[(32 + 8 * c + i4) * BM] = make_float4(
-                            __uint_as_float(ob[c][4 * i4]) * inv2, __uint_as_float(ob[c][4 * i4 + 1]) * inv2,
-                            __uint_as_float(ob[c][4 * i4 + 2]) * inv2, __uint_as_float(ob[c][4 * i4 + 3]) * inv2);
-                    }
-                tile[2 * BM * HDV + t * BM + r] = m_run + log2f(l_run);
-            }
-            if (p.mode == 1) {
-                // Export this half of the normalised noise output O2 / l2 for
-                // the group's pair items, tile-transposed (chunk c of row r at
-                // c * 128 + r: the warp's stores of one chunk are 512
-                // contiguous bytes).  Rows past N go to the tile's padding.
-                float4 *an = reinterpret_cast<float4 *>(p.noise_out) + noise_tile * (HDV / 4) * BM +
-                             (c0 / 4) * BM + r;
-                const float inv2 = 1.0f / l2;
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-#pragma unroll
-                    for (int i4 = 0; i4 < 8; ++i4)
-                        an[(8 * c + i4) * BM] = make_float4(__uint_as_float(ob[c][4 * i4]) * inv2,
-                                                     __uint_as_float(ob[c][4 * i4 + 1]) * inv2,
-                                                     __uint_as_float(ob[c][4 * i4 + 2]) * inv2,
-                                                     __uint_as_float(ob[c][4 * i4 + 3]) * inv2);
-            }
-            float d[64];
-            float ss = 0.0f;
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    d[32 * c + i] = fmaf(-r2, __uint_as_float(ob[c][i]), __uint_as_float(oa[c][i])) * inv1;
-                    ss = fmaf(d[32 * c + i], d[32 * c + i], ss);
-                }
-            sSS[t * BM + r] = ss;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_SSX));
-            float gv[64];  // this half's gain, loaded while the sums are exchanged
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float4 g4 = gain ? __ldg(reinterpret_cast<const float4 *>(gain) + i)
-                                       : make_float4(1.f, 1.f, 1.f, 1.f);
-                gv[4 * i] = g4.x;
-                gv[4 * i + 1] = g4.y;
-                gv[4 * i + 2] = g4.z;
-                gv[4 * i + 3] = g4.w;
-            }
-            if constexpr (GATED) {  // the output gate sigma(G), from the landed box, folds into the gain
-                if (!(ok = mbar_wait_warp(bar(B_GATE + (warp - 4)), tiles & 1, abort_flag, lim))) break;
-                const uint32_t gbuf = sbase + OFF_OUT + (warp - 4) * OUT_WARP_BYTES;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint4 gq = ld_shared_v4(gbuf + 128 * lane + ((i ^ (lane & 7)) << 4));
-                    const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+                ++an_loads;
+                if (!(ok = mbar_wait_warp(bar(B_O), tiles & 1, abort_flag, lim))) break;
+                tc_fence_after();
+                if (!(ok = mbar_wait_warp(abar, (an_loads - 1) & 1, abort_flag, lim))) break;
+                const float la = p.lam_logits ? logistic_fast(lam_a) : lam_a;
+                const float lb = p.lam_logits ? logistic_fast(lam_b) : lam_b;
+                const float inv1 = 1.0f / l1, inv2 = 1.0f / l2;
+                // D_h' = O_h - (lambda_h l_h) A_N = l_h D_h: one fused
+                // multiply-add per element; 1 / l_h goes into the output scale.
+                const float2 ka = make_float2(-la * l1, -la * l1), kb = make_float2(-lb * l2, -lb * l2);
+                auto an16 = [&](int c, float (&av)[16]) {  // A_N of columns 16 c .. 16 c + 15
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        gv[8 * i + 2 * k] *= logistic_tanh(__uint_as_float(gw[k] << 16));
-                        gv[8 * i + 2 * k + 1] *= logistic_tanh(__uint_as_float(gw[k] & 0xffff0000u));
+                        const uint4 v = ld_shared_v4(wbuf + 512 * (4 * c + k) + 16 * lane);
+                        av[4 * k] = __uint_as_float(v.x);
+                        av[4 * k + 1] = __uint_as_float(v.y);
+                        av[4 * k + 2] = __uint_as_float(v.z);
+                        av[4 * k + 3] = __uint_as_float(v.w);
+                    }
+                };
+                float2 ssa2 = make_float2(0.0f, 0.0f), ssb2 = make_float2(0.0f, 0.0f);
+#pragma unroll 1
+                for (int c2 = 0; c2 < 4; ++c2) {  // pass 1, 32 columns at a time
+                    uint32_t oa[32], ob[32];
+                    tmem_ld32(tO1 + 32 * c2, oa);
+                    tmem_ld32(tO2 + 32 * c2, ob);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        float av[16];
+                        an16(2 * c2 + h, av);
+                        if (h == 0) tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float2 a2 = make_float2(av[2 * i], av[2 * i + 1]);
+                            const float2 da = ffma2(a2, ka, make_float2(__uint_as_float(oa[16 * h + 2 * i]),
+                                                                        __uint_as_float(oa[16 * h + 2 * i + 1])));
+                            const float2 db = ffma2(a2, kb, make_float2(__uint_as_float(ob[16 * h + 2 * i]),
+                                                                        __uint_as_float(ob[16 * h + 2 * i + 1])));
+                            ssa2 = ffma2(da, da, ssa2);
+                            ssb2 = ffma2(db, db, ssb2);
+                        }
+                    }
+                }
+                const float rna = (p.apply_norm ? rsqrtf((ssa2.x + ssa2.y) * inv1 * inv1 * (1.0f / HDV) + p.eps) : 1.0f) * inv1;
+                const float rnb = (p.apply_norm ? rsqrtf((ssb2.x + ssb2.y) * inv2 * inv2 * (1.0f / HDV) + p.eps) : 1.0f) * inv2;
+                const bool row_ok = qrow < p.N;
+                __nv_bfloat16 *out_row = static_cast<__nv_bfloat16 *>(p.out) + w.b * p.out_sb + qrow_c * p.out_sn;
+                uint4 gcur[2][2], gnext[2][2];  // [head][half]: gate logits of the current / next chunk
+                if constexpr (GATED) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        gcur[0][h] = __ldg(gate_a + h);
+                        gcur[1][h] = __ldg(gate_b + h);
+                    }
+                }
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t oa[16], ob[16];
+                    tmem_ld16(tO1 + 16 * c, oa);
+                    tmem_ld16(tO2 + 16 * c, ob);
+                    if (GATED && c < 7) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            gnext[0][h] = __ldg(gate_a + 2 * (c + 1) + h);
+                            gnext[1][h] = __ldg(gate_b + 2 * (c + 1) + h);
+                        }
+                    }
+                    float av[16];
+                    an16(c, av);
+                    tmem_wait_ld();
+                    if (c == 7) {  // every lane has read all of O: release it, once per warp
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(bar(B_OFREE));
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t *o = h ? ob : oa;
+                        const float2 kl = h ? kb : ka;
+                        const float rn = h ? rnb : rna;
+                        float gv[16];
+                        scale16(h ? gain_b : gain_a, gcur[h], c, gv);
+                        uint32_t y[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float2 dd = ffma2(make_float2(av[2 * i], av[2 * i + 1]), kl,
+                                                    make_float2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])));
+                            y[i] = pack_bf162(dd.x * rn * gv[2 * i], dd.y * rn * gv[2 * i + 1]);
+                        }
+                        if (row_ok) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(out_row + (h ? hd.b : hd.a) * p.out_sh + 16 * c);
+                            dst[0] = make_uint4(y[0], y[1], y[2], y[3]);
+                            dst[1] = make_uint4(y[4], y[5], y[6], y[7]);
+                        }
+                    }
+                    if constexpr (GATED) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            gcur[h][0] = gnext[h][0];
+                            gcur[h][1] = gnext[h][1];
+                        }
                     }
                 }
             }
-            if (!(ok = mbar_wait_warp(bar(B_SSX), shared_eps & 1, abort_flag, lim))) break;
-            ++shared_eps;
-            const float rn =
-                p.apply_norm ? rsqrtf((sSS[r] + sSS[BM + r]) * (1.0f / HDV) + p.eps) : 1.0f;
-            // Stage this warp's 32 rows x 64 columns in shared memory (the
-            // 128-byte swizzle: 16-byte chunk i of a row at i ^ (row % 8)),
-            // then one TMA store; rows past N are clipped by the store.
-            const uint32_t obuf = sbase + OFF_OUT + (warp - 4) * OUT_WARP_BYTES;
-            if (lane == 0) bulk_wait_read_all();  // the previous tile's store has read the buffer
-            __syncwarp();
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t y[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    y[i] = pack_bf162(d[32 * c + 2 * i] * rn * gv[32 * c + 2 * i],
-                                      d[32 * c + 2 * i + 1] * rn * gv[32 * c + 2 * i + 1]);
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int ch = 4 * c + i;
-                    st_shared_v4(obuf + 128 * lane + ((ch ^ (lane & 7)) << 4), y[4 * i], y[4 * i + 1],
-                                 y[4 * i + 2], y[4 * i + 3]);
+            if (!own) {
+                // The staged boxes go out by TMA (rows past N are clipped; a
+                // box wholly past N is not issued).
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && r0 < p.N) {
+                    tma_store_4d(&tm_out, wbuf, 0, r0, hd.a, w.b);
+                    tma_store_4d(&tm_out, wbuf + OUT_HALF_BYTES, 64, r0, hd.a, w.b);
+                    bulk_commit_group();
                 }
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0 && w.qt * BM + 32 * (warp & 3) < p.N) {  // a box wholly past N is not issued
-                tma_store_4d(&tm_out, obuf, c0, w.qt * BM + 32 * (warp & 3), hd.a, w.b);
-                bulk_commit_group();
-            }
-            if (p.mode == 1) {
-                // Publish this warp's part of the noise output (stored above,
-                // before the norm, so the stores have had the rest of the
-                // epilogue to drain): every lane's stores, then one release
-                // per warp; the pair items wait for all eight warps of the tile.
+            if (p.mode == 1 && !own) {
+                // Publish this warp's rows of the noise output (stored in pass
+                // 1, so the stores have had pass 2 to drain): every lane's
+                // stores, then one release per warp; the pair items wait for
+                // all four epilogue warps of the tile.
                 __syncwarp();
                 if (lane == 0) {
                     __threadfence();
@@ -1008,9 +1088,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
             }
         }
+        // No copy of ours may land after the CTA has gone.
+        if (an_loads > 0 && !__all_sync(0xffffffffu, mbar_wait_drain(abar, (an_loads - 1) & 1, lim)) && lane == 0)
+            *abort_flag = 1;
     }
 
-    if (warp >= 4 && lane == 0) bulk_wait_all();  // output stores done before the CTA exits
+    if (warp >= 12 && lane == 0) bulk_wait_all();  // output stores done before the CTA exits
     tc_fence_before();
     __syncthreads();
     if (threadIdx.x == 0 && *abort_flag) report_error(p.dev_status, DIFFATTN_ERR_TIMEOUT);
@@ -1117,7 +1200,7 @@ __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb,
 
 cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const CUtensorMap &k1,
                            const CUtensorMap &k2, const CUtensorMap &v16, const CUtensorMap &out,
-                           const CUtensorMap &gate, const PrefillParams &p,
+                           const PrefillParams &p,
                            cudaStream_t stream, int *launches)
 {
     // Per device, once (first calls from several host threads serialise on
@@ -1184,7 +1267,7 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
     cfg.stream = stream;
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
-    cudaError_t le = cudaLaunchKernelEx(&cfg, kernel, q1, q2, k1, k2, v16, out, gate, p);
+    cudaError_t le = cudaLaunchKernelEx(&cfg, kernel, q1, q2, k1, k2, v16, out, p);
     if (le != cudaSuccess) return le;
     ++*launches;
     return cudaGetLastError();
