@@ -106,9 +106,10 @@ constexpr uint32_t OFF_TMEM_PTR = OFF_BARS + NBARS * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
 constexpr int ITEM_SLOTS = 4;
 constexpr int ITEM_READERS = 14;                         // 2 MMA, 8 softmax and 4 epilogue warps
-constexpr uint32_t OFF_ITEM = OFF_ABORT + 4;             // int [ITEM_SLOTS] work-item ring
+constexpr uint32_t ITEM_BYTES = 48;                      // one published work item: three int4
+constexpr uint32_t OFF_ITEM = (OFF_ABORT + 4 + 15) & ~15u;  // [ITEM_SLOTS] work-item ring
 // float [2 tile parities][l1, l2][128]: the softmax warps' row sums
-constexpr uint32_t OFF_STAT = (OFF_ITEM + 4 * ITEM_SLOTS + 15) & ~15u;
+constexpr uint32_t OFF_STAT = (OFF_ITEM + ITEM_BYTES * ITEM_SLOTS + 15) & ~15u;
 // Epilogue buffers: per epilogue warp 16 KB.  A one-head item keeps its 32
 // rows of D there in fp32 and then the staged output, two 32 x 64 bf16 TMA
 // store boxes of 4 KB with the 128-byte swizzle; a pair item keeps its 32
@@ -430,7 +431,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         return;
     }
     const int total = p.B * p.units * p.num_qt * (p.mode == 1 ? p.pairs + 1 : 1);
-    int *sItem = reinterpret_cast<int *>(smem + OFF_ITEM);
     const int n_steps_all = (p.N + BN - 1) / BN;
     // Key steps of a work item: [kv_first, kv_first + steps_of).  Causal tiles
     // stop at the diagonal; under a sliding window of W keys they start at
@@ -494,19 +494,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
     // Work items are handed out dynamically (an atomic counter in global
     // memory, zeroed by the V staging kernel that runs first): the producer
-    // takes the next one and publishes it in a ring of ITEM_SLOTS; the other
-    // roles read item k from slot k % ITEM_SLOTS and release the slot.  The
-    // producer reuses a slot only after all ten reader warps released it (with
-    // short tiles it can run several tiles ahead).  A negative item ends the
-    // loop.
-    auto next_item = [&](int k) -> int {
+    // takes the next one, decodes it (tile, heads, key steps) and publishes
+    // it in a ring of ITEM_SLOTS; the other roles read item k from slot
+    // k % ITEM_SLOTS and release the slot.  The producer reuses a slot only
+    // after all fourteen reader warps released it (with short tiles it can
+    // run several tiles ahead).  b < 0 ends the loop.
+    struct Item {
+        Work w;
+        Heads hd;
+        int nkv, kv0;
+    };
+    auto read_item = [&](int k, Item &it) -> bool {
         const int slot = k % ITEM_SLOTS;
-        if (!mbar_wait_warp(bar(B_ITEM + slot), (k / ITEM_SLOTS) & 1, abort_flag, p.timeout_ns))
-            return -1;
-        const int item = *reinterpret_cast<volatile int *>(&sItem[slot]);
+        if (!mbar_wait_warp(bar(B_ITEM + slot), (k / ITEM_SLOTS) & 1, abort_flag, p.timeout_ns)) return false;
+        const uint32_t a = sbase + OFF_ITEM + ITEM_BYTES * slot;
+        const uint4 x = ld_shared_v4(a), y = ld_shared_v4(a + 16), z = ld_shared_v4(a + 32);
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(B_ITEMFREE + slot));
-        return item;
+        it.w = Work{int(x.x), int(x.y), int(x.z)};
+        it.nkv = int(x.w);
+        it.kv0 = int(y.x);
+        it.hd = Heads{int(y.y), int(y.z), int(y.w), int(z.x), (z.y & 1u) != 0, (z.y & 2u) != 0};
+        return it.w.b >= 0;
     };
 
     // Register split: 4 x REGS_LAUNCH = REGS_IO + 2 x REGS_SOFTMAX + REGS_EPI per thread slot
@@ -535,18 +544,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 !(ok = mbar_wait_warp(bar(B_ITEMFREE + slot), ((tiles / ITEM_SLOTS) - 1) & 1, abort_flag, lim)))
                 break;
             int item = -1;
-            if (lane == 0) {
-                item = *abort_flag ? total : atomicAdd(p.tile_counter, 1);
-                sItem[slot] = item < total ? item : -1;
+            if (lane == 0) item = *abort_flag ? total : atomicAdd(p.tile_counter, 1);
+            item = __shfl_sync(0xffffffffu, item, 0);
+            const Work w = item < total ? work_of(item, p) : Work{-1, 0, 0};
+            const Heads hd = heads_of(item < total ? w.u : 0, p);
+            const int nkv = item < total ? steps_of(w) : 0, kv0 = item < total ? kv_first(w) : 0;
+            if (lane == 0) {  // the decoded item, for the other roles
+                const uint32_t a = sbase + OFF_ITEM + ITEM_BYTES * slot;
+                st_shared_v4(a, uint32_t(w.b), uint32_t(w.u), uint32_t(w.qt), uint32_t(nkv));
+                st_shared_v4(a + 16, uint32_t(kv0), uint32_t(hd.a), uint32_t(hd.b), uint32_t(hd.vh));
+                st_shared_v4(a + 32, uint32_t(hd.n), (hd.b_noise ? 1u : 0u) | (hd.own ? 2u : 0u), 0u, 0u);
                 mbar_arrive(bar(B_ITEM + slot));
             }
-            item = __shfl_sync(0xffffffffu, item, 0);
             if (item >= total) break;
-            const Work w = work_of(item, p);
-            const Heads hd = heads_of(w.u, p);
             const CUtensorMap *mq2 = hd.b_noise ? &tm_q2 : &tm_q1;
             const CUtensorMap *mk2 = hd.b_noise ? &tm_k2 : &tm_k1;
-            const int nkv = steps_of(w), kv0 = kv_first(w);
             // The previous tile's score MMAs must be done with Q.
             if (tiles > 0 && !(ok = mbar_wait_warp(bar(B_QFREE), (tiles - 1) & 1, abort_flag, lim)))
                 break;
@@ -633,11 +645,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         };
         int g = 0;
         bool ok = true;
-        for (int tiles = 0;; ++tiles) {
-            const int item = next_item(tiles);
-            if (item < 0) break;
-            const Work w = work_of(item, p);
-            const int nkv = steps_of(w);
+        // The next item is read during the current tile's last step (while
+        // this warp waits for its P), so that the first score MMAs of the
+        // next tile follow the tile's last P.V at once.
+        Item nxt;
+        bool have = read_item(0, nxt);
+        for (int tiles = 0; have; ++tiles) {
+            const int nkv = nxt.nkv;
             if (!(ok = mbar_wait_warp(bar(B_QFULL), tiles & 1, abort_flag, lim))) break;
             for (int jj = 0; jj < 2 && jj < nkv; ++jj) {
                 const int gg = g + jj;
@@ -649,6 +663,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             for (int j = 0; ok && j < nkv; ++j) {
                 const int gg = g + j, s = gg % STAGES, buf = gg & 1;
+                if (j == nkv - 1) have = read_item(tiles + 1, nxt);
                 if (!(ok = mbar_wait_warp(bar_p(t, buf), (gg >> 1) & 1, abort_flag, lim))) break;
                 // The first P.V of a tile overwrites O: the previous tile's
                 // epilogue must have read it.
@@ -690,10 +705,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int g = 0;
         bool ok = true;
         for (int tiles = 0;; ++tiles) {
-            const int item = next_item(tiles);
-            if (item < 0) break;
-            const Work w = work_of(item, p);
-            const int nkv = steps_of(w), kv0 = kv_first(w);
+            Item it;
+            if (!read_item(tiles, it)) break;
+            const Work w = it.w;
+            const int nkv = it.nkv, kv0 = it.kv0;
             const int qrow = w.qt * BM + r;
             float m_run = -INFINITY, l_run = 0.0f;
             for (int j = 0; j < nkv; ++j) {
@@ -718,7 +733,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 // Saved for the backward pass: this map's lse = m + log2(l)
                 // (the running max and sum are in units of scale * log2(e) *
                 // score), at float 2 * 128 * 128 + 128 t + r of the tile's state.
-                const int head = heads_of(w.u, p).a;
+                const int head = it.hd.a;
                 p.save[((size_t)(w.b * p.H + head) * p.num_qt + w.qt) * kSaveTileFloats + 2 * BM * HDV + t * BM + r] =
                     m_run + log2f(l_run);
             }
@@ -751,10 +766,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         int an_loads = 0;
         bool ok = true;
         for (int tiles = 0;; ++tiles) {
-            const int item = next_item(tiles);
-            if (item < 0) break;
-            const Work w = work_of(item, p);
-            const Heads hd = heads_of(w.u, p);
+            Item it;
+            if (!read_item(tiles, it)) break;
+            const Work w = it.w;
+            const Heads hd = it.hd;
             const bool own = hd.own;
             const int qrow = w.qt * BM + r;
             const int64_t qrow_c = min(qrow, p.N - 1);
