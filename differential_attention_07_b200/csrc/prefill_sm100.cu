@@ -1135,24 +1135,13 @@ __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb,
         zero[i] = 0;
     // One thread per 8 consecutive V elements (16 bytes in, 16 bytes out).
     // A dense V ([B, N, H_V, 128] with no gaps, the common case) is one flat
-    // array, so its chunk i needs no index arithmetic; otherwise chunk i is
-    // decomposed into (b, n, head, column) -- 64-bit divisions that made the
-    // pass compute-bound.
+    // array, so its chunk i needs no index arithmetic, and each thread keeps
+    // four loads in flight; otherwise chunk i is decomposed into (b, n, head,
+    // column) -- 64-bit divisions that made the pass compute-bound.
     const int64_t total = (int64_t)B * N * H_V * (HDV / 8);
     const bool dense = sh == HDV && sn == (int64_t)H_V * HDV && sb == (int64_t)N * H_V * HDV;
     bool overflow = false;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        int64_t off = 8 * i;
-        if (!dense) {
-            const int c8 = int(i % (HDV / 8));
-            const int64_t row = i / (HDV / 8);
-            const int hv = int(row % H_V);
-            const int64_t bn = row / H_V;
-            const int n = int(bn % N), b = int(bn / N);
-            off = b * sb + n * sn + hv * sh + 8 * c8;
-        }
-        const uint4 src = __ldg(reinterpret_cast<const uint4 *>(v + off));
+    auto to_f16 = [&](const uint4 src) {
         const uint32_t in[4] = {src.x, src.y, src.z, src.w};
         uint32_t out[4];
 #pragma unroll
@@ -1162,7 +1151,31 @@ __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb,
             overflow |= fabsf(f.x) > 65504.0f || fabsf(f.y) > 65504.0f;
             out[k] = pack_half2(f.x, f.y);
         }
-        reinterpret_cast<uint4 *>(dst)[i] = make_uint4(out[0], out[1], out[2], out[3]);
+        return make_uint4(out[0], out[1], out[2], out[3]);
+    };
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (dense) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(v);
+        uint4 *out = reinterpret_cast<uint4 *>(dst);
+        for (; i + 3 * stride < total; i += 4 * stride) {
+            uint4 x[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) x[u] = __ldcs(src + i + u * stride);  // read once: streaming
+#pragma unroll
+            for (int u = 0; u < 4; ++u) out[i + u * stride] = to_f16(x[u]);
+        }
+        for (; i < total; i += stride) out[i] = to_f16(__ldcs(src + i));
+    } else {
+        for (; i < total; i += stride) {
+            const int c8 = int(i % (HDV / 8));
+            const int64_t row = i / (HDV / 8);
+            const int hv = int(row % H_V);
+            const int64_t bn = row / H_V;
+            const int n = int(bn % N), b = int(bn / N);
+            const int64_t off = b * sb + n * sn + hv * sh + 8 * c8;
+            reinterpret_cast<uint4 *>(dst)[i] = to_f16(__ldg(reinterpret_cast<const uint4 *>(v + off)));
+        }
     }
     if (overflow) report_error(dev_status, DIFFATTN_ERR_UNSUPPORTED);
     if (!rope.enabled) return;
@@ -1297,7 +1310,7 @@ cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, v
     if (total == 0) return cudaSuccess;  // nothing to stage; the prefill is skipped too
     const int threads = 256;
     int blocks = (int)((total + threads - 1) / threads);
-    if (blocks > sm_count * 16) blocks = sm_count * 16;  // grid-stride beyond 16 blocks per SM
+    if (blocks > sm_count * 8) blocks = sm_count * 8;  // resident at once (2048 threads per SM); grid-stride beyond
     v_to_f16_kernel<<<blocks, threads, 0, stream>>>(static_cast<const __nv_bfloat16 *>(v), sb, sn,
                                                     sh, static_cast<__half *>(dst), B, N, H_V,
                                                     dev_status, tile_counter, zero, n_zero, rope);
