@@ -536,7 +536,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             prefetch_tensormap(&tm_v);
         }
         __syncwarp();
-        int g = 0, tiles = 0;
+        int g = 0, tiles = 0, q_loads = 0;
         bool ok = true;
         for (;; ++tiles) {
             const int slot = tiles % ITEM_SLOTS;
@@ -559,16 +559,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (item >= total) break;
             const CUtensorMap *mq2 = hd.b_noise ? &tm_q2 : &tm_q1;
             const CUtensorMap *mk2 = hd.b_noise ? &tm_k2 : &tm_k1;
-            // The previous tile's score MMAs must be done with Q.
-            if (tiles > 0 && !(ok = mbar_wait_warp(bar(B_QFREE), (tiles - 1) & 1, abort_flag, lim)))
-                break;
-            if (elect_one()) {
-                mbar_arrive_expect_tx(bar(B_QFULL), 2 * Q_BYTES);
-                tma_load_4d(sbase + OFF_Q1, &tm_q1, bar(B_QFULL), 0, w.qt * BM, hd.a, w.b, stream);
-                tma_load_4d(sbase + OFF_Q2, mq2, bar(B_QFULL), 0, w.qt * BM, hd.b, w.b, stream);
-            }
-            __syncwarp();
+            // Q waits until the previous tile's last score MMAs are done with
+            // it.  The first two key steps' stages were last used by the
+            // previous tile, so their loads go out first (often while that
+            // tile still runs); a stage that this tile's own steps free is
+            // only waited for once Q is on its way.
+            auto load_q = [&]() -> bool {
+                if (tiles > 0 && !mbar_wait_warp(bar(B_QFREE), (tiles - 1) & 1, abort_flag, lim)) return false;
+                if (elect_one()) {
+                    mbar_arrive_expect_tx(bar(B_QFULL), 2 * Q_BYTES);
+                    tma_load_4d(sbase + OFF_Q1, &tm_q1, bar(B_QFULL), 0, w.qt * BM, hd.a, w.b, stream);
+                    tma_load_4d(sbase + OFF_Q2, mq2, bar(B_QFULL), 0, w.qt * BM, hd.b, w.b, stream);
+                }
+                __syncwarp();
+                ++q_loads;
+                return true;
+            };
+            const int q_at = nkv < 2 ? nkv : 2;
+            static_assert(STAGES > 2, "the steps loaded before Q must not depend on this tile");
             for (int j = 0; j < nkv; ++j, ++g) {
+                if (j == q_at && !(ok = load_q())) break;
                 const int s = g % STAGES;
                 if (g >= STAGES &&
                     !(ok = mbar_wait_warp(bar_empty(s), ((g / STAGES) - 1) & 1, abort_flag, lim)))
@@ -594,6 +604,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 __syncwarp();
             }
+            if (ok && q_at == nkv) ok = load_q();
             if (!ok) {
                 ++tiles;
                 break;
@@ -601,7 +612,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         // No load of ours may land after the CTA has gone: wait for all of them.
         bool drained = true;
-        if (tiles > 0) drained = mbar_wait_drain(bar(B_QFULL), (tiles - 1) & 1, lim);
+        if (q_loads > 0) drained = mbar_wait_drain(bar(B_QFULL), (q_loads - 1) & 1, lim);
         for (int k = (g > STAGES ? g - STAGES : 0); k < g; ++k)
             if (!(p.withhold_load && k == 0))  // the withheld load was never issued
                 drained &= mbar_wait_drain(bar_full(k % STAGES), (k / STAGES) & 1, lim);
