@@ -66,6 +66,11 @@ constexpr int NEW = 8;    // element-wise warps
 // shared memory: a block's load is issued STAGES - 1 blocks ahead).
 constexpr int KSTAGES = 3, QSTAGES = 3, MAXSTAGES = 3;
 
+// Which pairs of exponentials (pair index mod 8) the element-wise step
+// computes with the software exp2 (FMA pipe) rather than MUFU ex2: the step
+// needs two exponentials per (key, query) pair against 1280 MMA FLOP.
+constexpr uint32_t BWD_SOFT_EXP_MASK = 0x02u;  // one pair in eight (measured: none 457, 1/8 462, 2/8 456, 4/8 451 TFLOP/s)
+
 // mbarriers of both tile kernels.
 enum : int {
     B_TILE = 0,                     // the tile's operands landed (TMA bytes)
@@ -365,15 +370,16 @@ __global__ void __launch_bounds__(128)
     }
     if (bad) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
 
-    // Row statistics; rows past N get zeros (the tile kernels' products see
-    // zero operands there).
+    // Row statistics, negated (-lse_1, -lse_2, -Delta_1, -Delta_2, -lambda:
+    // the tile kernels add them in packed fused multiply-adds); rows past N
+    // get zeros (the tile kernels' products see zero operands there).
     float *st = p.stats + (size_t)(b * p.H + h) * kBwdStats * p.n_pad + row;
     const float *lse = tile + 2 * BT * HDV;
-    st[0] = valid ? lse[r] : 0.f;
-    st[p.n_pad] = valid ? lse[BT + r] : 0.f;
-    st[2 * p.n_pad] = delta1;
-    st[3 * p.n_pad] = -lam * dot2h;
-    st[4 * p.n_pad] = valid ? lam : 0.f;
+    st[0] = valid ? -lse[r] : 0.f;
+    st[p.n_pad] = valid ? -lse[BT + r] : 0.f;
+    st[2 * p.n_pad] = -delta1;
+    st[3 * p.n_pad] = lam * dot2h;
+    st[4 * p.n_pad] = valid ? -lam : 0.f;
 
     // dlambda_i = -dD . A_2: per token through sigma' with lambda logits,
     // else summed over the tile's rows into the head's dlambda.
@@ -615,37 +621,52 @@ __global__ void __launch_bounds__(NT, 1)
             const uint32_t st = sbase + KT_STAGE0 + (j % KSTAGES) * KB_BYTES + KB_ST + 4 * 32 * wg;
             const bool mask = (p.causal && qb < k0 + BT - 1) || (p.window > 0 && qb + 31 - k0 >= p.window);
             uint32_t pv[16], d1p[16], d2p[16];
+            const float2 c2 = make_float2(c, c);
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
+                // the four queries' statistics, negated: -lse_1, -lse_2,
+                // -Delta_1, -Delta_2, -lambda
                 const uint4 ul1 = ld_shared_v4(st + 4 * i), ul2 = ld_shared_v4(st + 256 + 4 * i);
                 const uint4 ud1 = ld_shared_v4(st + 512 + 4 * i), ud2 = ld_shared_v4(st + 768 + 4 * i);
                 const uint4 ulm = ld_shared_v4(st + 1024 + 4 * i);
                 const uint32_t l1[4] = {ul1.x, ul1.y, ul1.z, ul1.w}, l2[4] = {ul2.x, ul2.y, ul2.z, ul2.w};
                 const uint32_t D1[4] = {ud1.x, ud1.y, ud1.z, ud1.w}, D2[4] = {ud2.x, ud2.y, ud2.z, ud2.w};
                 const uint32_t LM[4] = {ulm.x, ulm.y, ulm.z, ulm.w};
-                float vp[4], v1[4], v2[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float p1 = ex2_approx(fmaf(__uint_as_float(s1[i + e]), c, -__uint_as_float(l1[e])));
-                    float p2 = ex2_approx(fmaf(__uint_as_float(s2[i + e]), c, -__uint_as_float(l2[e])));
-                    if (mask) {
-                        const int q = qb + i + e;
-                        const bool vis = (!p.causal || q >= kj) && (p.window <= 0 || q - kj < p.window);
-                        p1 = vis ? p1 : 0.f;
-                        p2 = vis ? p2 : 0.f;
+                for (int e = 0; e < 4; e += 2) {  // two queries at a time, in packed arithmetic
+                    auto f2 = [](const uint32_t *a, int k) { return make_float2(__uint_as_float(a[k]), __uint_as_float(a[k + 1])); };
+                    const float2 x1 = ffma2(f2(s1, i + e), c2, f2(l1, e));
+                    const float2 x2 = ffma2(f2(s2, i + e), c2, f2(l2, e));
+                    float2 p1, p2;
+                    if ((BWD_SOFT_EXP_MASK >> (((i + e) >> 1) & 7)) & 1u) {
+                        p1 = exp2_soft2(x1);
+                        p2 = exp2_soft2(x2);
+                    } else {
+                        p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+                        p2 = make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
                     }
-                    const float g = __uint_as_float(dp[i + e]), lam = __uint_as_float(LM[e]);
-                    vp[e] = fmaf(-lam, p2, p1);
-                    v1[e] = p1 * (g - __uint_as_float(D1[e]));
-                    v2[e] = p2 * fmaf(-lam, g, -__uint_as_float(D2[e]));
-                    if (F16QK) big |= !(fabsf(v1[e]) <= 65504.0f && fabsf(v2[e]) <= 65504.0f);
+                    if (mask) {
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int q = qb + i + e + u;
+                            const bool vis = (!p.causal || q >= kj) && (p.window <= 0 || q - kj < p.window);
+                            if (!vis) {
+                                if (u) p1.y = p2.y = 0.f;
+                                else p1.x = p2.x = 0.f;
+                            }
+                        }
+                    }
+                    const float2 g = f2(dp, i + e), nlam = f2(LM, e);
+                    const float2 vp = ffma2(nlam, p2, p1);                     // P_1 - lambda P_2
+                    const float2 v1 = fmul2(p1, fadd2(g, f2(D1, e)));          // P_1 (dP - Delta_1)
+                    const float2 v2 = fmul2(p2, ffma2(nlam, g, f2(D2, e)));    // P_2 (-lambda dP - Delta_2)
+                    if (F16QK)
+                        big |= !(fabsf(v1.x) <= 65504.0f && fabsf(v1.y) <= 65504.0f && fabsf(v2.x) <= 65504.0f &&
+                                 fabsf(v2.y) <= 65504.0f);
+                    pv[(i + e) / 2] = pack_half2(vp.x, vp.y);
+                    d1p[(i + e) / 2] = pack_ds(v1.x, v1.y, F16QK);
+                    d2p[(i + e) / 2] = pack_ds(v2.x, v2.y, F16QK);
                 }
-                pv[i / 2] = pack_half2(vp[0], vp[1]);
-                pv[i / 2 + 1] = pack_half2(vp[2], vp[3]);
-                d1p[i / 2] = pack_ds(v1[0], v1[1], F16QK);
-                d1p[i / 2 + 1] = pack_ds(v1[2], v1[3], F16QK);
-                d2p[i / 2] = pack_ds(v2[0], v2[1], F16QK);
-                d2p[i / 2 + 1] = pack_ds(v2[2], v2[3], F16QK);
                 // Keep the next four queries' statistics loads below this
                 // point: hoisted all at once they would need 160 registers.
                 asm volatile("" ::: "memory");
@@ -828,8 +849,9 @@ __global__ void __launch_bounds__(NT, 1)
         const int qrow = q0 + r;  // this thread's query
         const float c = p.scale_log2;
         const float *strow = p.stats + (size_t)(b * p.H + h) * kBwdStats * p.n_pad + qrow;
-        const float lse1 = strow[0], lse2 = strow[p.n_pad], del1 = strow[2 * p.n_pad], del2 = strow[3 * p.n_pad];
-        const float lam = strow[4 * p.n_pad];
+        // (stored negated: -lse_1, -lse_2, -Delta_1, -Delta_2, -lambda)
+        const float nlse1 = strow[0], nlse2 = strow[p.n_pad], ndel1 = strow[2 * p.n_pad], ndel2 = strow[3 * p.n_pad];
+        const float nlam = strow[4 * p.n_pad];
         // The tile's Q_1, Q_2 (warpgroup 0) and dD (warpgroup 1) rows into
         // TMEM, the A operands of every block's score and dP products.
         bool ok = mbar_wait_warp(bar(B_TILE), 0, abort_flag, lim), big = false;
@@ -860,26 +882,39 @@ __global__ void __launch_bounds__(NT, 1)
             const int kb = (kb0 + j) * BB + 32 * wg;  // this warpgroup's 32 keys of the block
             const bool mask = (p.causal && kb + 31 > q0) || (p.window > 0 && q0 + BT - 1 - kb >= p.window);
             uint32_t d1p[16], d2p[16];
+            const float2 c2 = make_float2(c, c), nl1 = make_float2(nlse1, nlse1), nl2 = make_float2(nlse2, nlse2);
+            const float2 nd1 = make_float2(ndel1, ndel1), nd2 = make_float2(ndel2, ndel2), nlm = make_float2(nlam, nlam);
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-                float v1[2], v2[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    float p1 = ex2_approx(fmaf(__uint_as_float(s1[i + e]), c, -lse1));
-                    float p2 = ex2_approx(fmaf(__uint_as_float(s2[i + e]), c, -lse2));
-                    if (mask) {
-                        const int key = kb + i + e;
-                        const bool vis = (!p.causal || key <= qrow) && (p.window <= 0 || qrow - key < p.window);
-                        p1 = vis ? p1 : 0.f;
-                        p2 = vis ? p2 : 0.f;
-                    }
-                    const float g = __uint_as_float(dp[i + e]);
-                    v1[e] = p1 * (g - del1);
-                    v2[e] = p2 * fmaf(-lam, g, -del2);
-                    if (F16QK) big |= !(fabsf(v1[e]) <= 65504.0f && fabsf(v2[e]) <= 65504.0f);
+            for (int i = 0; i < 32; i += 2) {  // two keys at a time, in packed arithmetic
+                const float2 x1 = ffma2(make_float2(__uint_as_float(s1[i]), __uint_as_float(s1[i + 1])), c2, nl1);
+                const float2 x2 = ffma2(make_float2(__uint_as_float(s2[i]), __uint_as_float(s2[i + 1])), c2, nl2);
+                float2 p1, p2;
+                if ((BWD_SOFT_EXP_MASK >> ((i >> 1) & 7)) & 1u) {
+                    p1 = exp2_soft2(x1);
+                    p2 = exp2_soft2(x2);
+                } else {
+                    p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+                    p2 = make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
                 }
-                d1p[i / 2] = pack_ds(v1[0], v1[1], F16QK);
-                d2p[i / 2] = pack_ds(v2[0], v2[1], F16QK);
+                if (mask) {
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int key = kb + i + u;
+                        const bool vis = (!p.causal || key <= qrow) && (p.window <= 0 || qrow - key < p.window);
+                        if (!vis) {
+                            if (u) p1.y = p2.y = 0.f;
+                            else p1.x = p2.x = 0.f;
+                        }
+                    }
+                }
+                const float2 g = make_float2(__uint_as_float(dp[i]), __uint_as_float(dp[i + 1]));
+                const float2 v1 = fmul2(p1, fadd2(g, nd1));        // P_1 (dP - Delta_1)
+                const float2 v2 = fmul2(p2, ffma2(nlm, g, nd2));   // P_2 (-lambda dP - Delta_2)
+                if (F16QK)
+                    big |= !(fabsf(v1.x) <= 65504.0f && fabsf(v1.y) <= 65504.0f && fabsf(v2.x) <= 65504.0f &&
+                             fabsf(v2.y) <= 65504.0f);
+                d1p[i / 2] = pack_ds(v1.x, v1.y, F16QK);
+                d2p[i / 2] = pack_ds(v2.x, v2.y, F16QK);
             }
             if (j > 0 && !(ok = mbar_wait_warp(bar(B_AFREE), (j - 1) & 1, abort_flag, lim))) break;
             st_operand_half(sbase + QT_A + QA_DS1, r, wg, d1p);

@@ -277,35 +277,6 @@ __device__ __forceinline__ bool wait_flag_geq(const int *flag, int target, volat
     }
 }
 
-// Software 2^x for two values at once on the FMA and integer pipes, to take
-// part of the exponentials off MUFU.  Cody-Waite style range reduction:
-// x = n + f with n = rint(x) from the 1.5 * 2^23 magic-number add (the
-// integer lands in the low mantissa bits of j), f = x - n in [-1/2, 1/2];
-// 2^f is a degree-3 polynomial whose coefficients minimise the relative error
-// on [-1/2, 1/2] (Remez exchange, fit_exp2_poly.py; max relative error
-// 7.5e-5 in float32, below the fp16 rounding of P); 2^n is added into the
-// exponent field as (bits(j) << 23).  Inputs are clamped to >= -125 so the
-// exponent never wraps; 2^-125 is zero once P is rounded to fp16.
-constexpr float EXP2_C0 = 0x1.fff692p-1f;
-constexpr float EXP2_C1 = 0x1.62f31ap-1f;
-constexpr float EXP2_C2 = 0x1.f0de1ap-3f;
-constexpr float EXP2_C3 = 0x1.c3f76p-5f;
-constexpr float EXP2_ROUND = 12582912.0f;  // 1.5 * 2^23
-
-__device__ __forceinline__ float2 exp2_soft2(float2 x)
-{
-    x.x = fmaxf(x.x, -125.0f);
-    x.y = fmaxf(x.y, -125.0f);
-    const float2 j = fadd2(x, make_float2(EXP2_ROUND, EXP2_ROUND));
-    const float2 n = fadd2(j, make_float2(-EXP2_ROUND, -EXP2_ROUND));
-    const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);
-    float2 p = ffma2(make_float2(EXP2_C3, EXP2_C3), f, make_float2(EXP2_C2, EXP2_C2));
-    p = ffma2(p, f, make_float2(EXP2_C1, EXP2_C1));
-    p = ffma2(p, f, make_float2(EXP2_C0, EXP2_C0));
-    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(j.x) << 23)),
-                       __int_as_float(__float_as_int(p.y) + (__float_as_int(j.y) << 23)));
-}
-
 // Which pairs of scores (index mod 8) take the software exp2; the rest use
 // MUFU ex2.  Measured on B200 (motif-4K / 16K prefill, TFLOP/s): 4 of 8
 // 790 / 931, 3 of 8 810 / 893, 2 of 8 860 / 909, 1 of 8 861 / 959, none

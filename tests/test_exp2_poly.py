@@ -1,6 +1,6 @@
-"""The prefill kernel's software exp2 (CPU emulation of its exact steps).
+"""The software exp2 of the prefill and backward kernels (CPU emulation of its exact steps).
 
-The kernel computes part of the softmax exponentials as 2^x = 2^n * p(f)
+The kernels compute part of the softmax exponentials as 2^x = 2^n * p(f)
 (range reduction x = n + f by the 1.5*2^23 magic-number add, a degree-3
 polynomial p fitted by Remez exchange, 2^n added into the exponent bits).
 These tests check that the constants in the CUDA source are the ones the
@@ -20,7 +20,7 @@ CSRC = os.path.join(ROOT, "differential_attention_07_b200", "csrc")
 
 
 def _kernel_constants():
-    src = open(os.path.join(CSRC, "prefill_sm100.cu")).read()
+    src = open(os.path.join(CSRC, "sm100_ptx.cuh")).read()
     c = {}
     for k in range(4):
         m = re.search(rf"constexpr float EXP2_C{k} = (0x[0-9a-fA-Fp.+-]+)f;", src)
