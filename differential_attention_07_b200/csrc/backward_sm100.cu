@@ -257,8 +257,11 @@ __device__ __forceinline__ void tmem_row64(uint32_t taddr, float (&x)[64])
 __global__ void __launch_bounds__(128)
     bwd_prep_kernel(const BwdParams p)
 {
+    // dgain reduction: a group of 32 columns of every row ([128][33] floats,
+    // padded against bank conflicts), then per-warp partial column sums.
     extern __shared__ float red[];
     __shared__ float warp_sum[4];
+    __shared__ float col_part[4][32];
     const int qt = blockIdx.x % p.num_qt, h = (blockIdx.x / p.num_qt) % p.H, b = blockIdx.x / (p.num_qt * p.H);
     const int r = threadIdx.x, row = qt * BT + r;
     const bool valid = row < p.N;
@@ -334,6 +337,7 @@ __global__ void __launch_bounds__(128)
     __nv_bfloat16 *dgrow = p.dgate ? static_cast<__nv_bfloat16 *>(p.dgate) + (size_t)b * p.dg_sb +
                                          (size_t)rowc * p.dg_sn + (size_t)h * p.dg_sh
                                    : nullptr;
+    float dgc0 = 0.f, dgc1 = 0.f, dgc2 = 0.f, dgc3 = 0.f;  // thread r < 32: columns r, 32 + r, 64 + r, 96 + r
 #pragma unroll 2
     for (int c = 0; c < 32; ++c) {
         float dd[4] = {0.f, 0.f, 0.f, 0.f}, gt[4] = {0.f, 0.f, 0.f, 0.f};
@@ -364,8 +368,28 @@ __global__ void __launch_bounds__(128)
                     make_uint2(pack_bf162(dgv[0], dgv[1]), pack_bf162(dgv[2], dgv[3]));
         }
         if (want_dgain) {
+            // This row's terms of columns 4c .. 4c + 3; after every eighth
+            // chunk the CTA sums the group's 32 columns over its 128 rows
+            // (a quarter of the rows per warp, then the four partials).
 #pragma unroll
-            for (int e = 0; e < 4; ++e) red[r * (HDV + 1) + 4 * c + e] = gt[e];
+            for (int e = 0; e < 4; ++e) red[r * 33 + 4 * (c & 7) + e] = gt[e];
+            if ((c & 7) == 7) {
+                __syncthreads();
+                const int col = r & 31, r0 = (r >> 5) * 32;
+                float v = 0.f;
+#pragma unroll 8
+                for (int i = 0; i < 32; ++i) v += red[(r0 + i) * 33 + col];
+                col_part[r >> 5][col] = v;
+                __syncthreads();
+                if (r < 32) {
+                    const float t = col_part[0][r] + col_part[1][r] + col_part[2][r] + col_part[3][r];
+                    const int grp = c >> 3;
+                    dgc0 = grp == 0 ? t : dgc0;
+                    dgc1 = grp == 1 ? t : dgc1;
+                    dgc2 = grp == 2 ? t : dgc2;
+                    dgc3 = grp == 3 ? t : dgc3;
+                }
+            }
         }
     }
     if (bad) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
@@ -395,12 +419,13 @@ __global__ void __launch_bounds__(128)
     __syncthreads();
     if (!p.lam_logits && p.dlambda && r == 0)
         atomicAdd(p.dlambda + h, warp_sum[0] + warp_sum[1] + warp_sum[2] + warp_sum[3]);
-    // dgain[h][c] += sum over the tile's rows (thread r sums column r).
-    if (want_dgain) {
-        float v = 0.f;
-#pragma unroll 8
-        for (int i = 0; i < BT; ++i) v += red[i * (HDV + 1) + r];
-        atomicAdd(p.dgain + (size_t)h * HDV + r, v);
+    // dgain[h][c] += the tile's column sums.
+    if (want_dgain && r < 32) {
+        float *dg = p.dgain + (size_t)h * HDV + r;
+        atomicAdd(dg, dgc0);
+        atomicAdd(dg + 32, dgc1);
+        atomicAdd(dg + 64, dgc2);
+        atomicAdd(dg + 96, dgc3);
     }
 }
 
@@ -1010,7 +1035,7 @@ cudaError_t launch_bwd(const BwdKeyMaps &km, const BwdQueryMaps &qm, const BwdPa
         set_internal_error("device ordinal beyond the library's table");
         return cudaErrorInvalidDevice;
     }
-    const int red_bytes = BT * (HDV + 1) * (int)sizeof(float);
+    const int red_bytes = BT * 33 * (int)sizeof(float);  // one group of 32 columns
     if (!attr_set[dev].load(std::memory_order_acquire)) {
         std::lock_guard<std::mutex> lock(attr_mutex);  // first calls from several host threads
         if (!attr_set[dev].load(std::memory_order_relaxed)) {
