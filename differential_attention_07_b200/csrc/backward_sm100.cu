@@ -279,46 +279,54 @@ __global__ void __launch_bounds__(128)
                                      : nullptr;
     const bool want_dgain = p.apply_norm && p.dgain;
 
-    auto load4 = [](const __nv_bfloat16 *src, int c, float (&y)[4]) {
-        const uint2 u = *reinterpret_cast<const uint2 *>(src + 4 * c);
-        y[0] = __uint_as_float(u.x << 16);
-        y[1] = __uint_as_float(u.x & 0xffff0000u);
-        y[2] = __uint_as_float(u.y << 16);
-        y[3] = __uint_as_float(u.y & 0xffff0000u);
+    // 8 columns (8 c8 .. 8 c8 + 7) of a bf16 row: one 16-byte load.
+    auto load8 = [](const __nv_bfloat16 *src, int c8, float (&y)[8]) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(src + 8 * c8);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            y[2 * k] = __uint_as_float(w[k] << 16);
+            y[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+        }
     };
     auto gain4 = [&](int c) { return g4p ? __ldg(g4p + c) : make_float4(1.f, 1.f, 1.f, 1.f); };
     // dYn = dY sigma(G) (the gate is the forward's last step), and sigma(G)
-    auto dyn4 = [&](int c, float (&y)[4], float (&sg)[4]) {
-        load4(dy, c, y);
+    auto dyn8 = [&](int c8, float (&y)[8], float (&sg)[8]) {
+        load8(dy, c8, y);
         if (gl) {
-            float g[4];
-            load4(gl, c, g);
+            float g[8];
+            load8(gl, c8, g);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
+            for (int e = 0; e < 8; ++e) {
                 sg[e] = logistic_fast(g[e]);
                 y[e] *= sg[e];
             }
         } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) sg[e] = 1.0f;
+            for (int e = 0; e < 8; ++e) sg[e] = 1.0f;
         }
     };
 
-    // Pass 1: sum of squares of D and sum_c dYn gain D.
+    // Pass 1: sum of squares of D and sum_c dYn gain D, 8 columns (two float4
+    // chunks of A_1, A_2) at a time.
     float ss = 0.f, tg = 0.f;
     if (valid && p.apply_norm) {
-#pragma unroll 4
-        for (int c = 0; c < 32; ++c) {
-            const float4 a1 = a1p[c * BT], a2 = a2p[c * BT], g = gain4(c);
-            float y[4], sg[4];
-            dyn4(c, y, sg);
-            const float d[4] = {fmaf(-lam, a2.x, a1.x), fmaf(-lam, a2.y, a1.y), fmaf(-lam, a2.z, a1.z),
-                                fmaf(-lam, a2.w, a1.w)};
-            const float gg[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll 2
+        for (int c8 = 0; c8 < 16; ++c8) {
+            float y[8], sg[8];
+            dyn8(c8, y, sg);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                ss = fmaf(d[e], d[e], ss);
-                tg = fmaf(gg[e] * y[e], d[e], tg);
+            for (int hh = 0; hh < 2; ++hh) {
+                const int c = 2 * c8 + hh;
+                const float4 a1 = a1p[c * BT], a2 = a2p[c * BT], g = gain4(c);
+                const float d[4] = {fmaf(-lam, a2.x, a1.x), fmaf(-lam, a2.y, a1.y), fmaf(-lam, a2.z, a1.z),
+                                    fmaf(-lam, a2.w, a1.w)};
+                const float gg[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    ss = fmaf(d[e], d[e], ss);
+                    tg = fmaf(gg[e] * y[4 * hh + e], d[e], tg);
+                }
             }
         }
     }
@@ -339,41 +347,50 @@ __global__ void __launch_bounds__(128)
                                    : nullptr;
     float dgc0 = 0.f, dgc1 = 0.f, dgc2 = 0.f, dgc3 = 0.f;  // thread r < 32: columns r, 32 + r, 64 + r, 96 + r
 #pragma unroll 2
-    for (int c = 0; c < 32; ++c) {
-        float dd[4] = {0.f, 0.f, 0.f, 0.f}, gt[4] = {0.f, 0.f, 0.f, 0.f};
-        if (valid) {
-            const float4 a1 = a1p[c * BT], a2 = a2p[c * BT], g = gain4(c);
-            float y[4], sg[4];
-            dyn4(c, y, sg);
-            const float av1[4] = {a1.x, a1.y, a1.z, a1.w}, av2[4] = {a2.x, a2.y, a2.z, a2.w};
-            const float gg[4] = {g.x, g.y, g.z, g.w};
-            float dgv[4];
+    for (int c8 = 0; c8 < 16; ++c8) {
+        float dd[8], gt[8], dgv[8];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float d = fmaf(-lam, av2[e], av1[e]);
-                dd[e] = p.apply_norm ? fmaf(rn * gg[e], y[e], -coef * d) : y[e];
-                const float ddh = __half2float(__float2half_rn(dd[e]));
-                delta1 = fmaf(ddh, av1[e], delta1);
-                dot2h = fmaf(ddh, av2[e], dot2h);
-                dot2 = fmaf(dd[e], av2[e], dot2);
-                gt[e] = y[e] * d * rn;
-                bad |= !(fabsf(dd[e]) <= 65504.0f);
-                // dG = dY Yn sigma'(G) = dYn Yn (1 - sigma(G)), Yn = D r gain (or D)
-                const float yn = p.apply_norm ? d * rn * gg[e] : d;
-                dgv[e] = y[e] * yn * (1.0f - sg[e]);
+        for (int e = 0; e < 8; ++e) dd[e] = gt[e] = dgv[e] = 0.f;
+        if (valid) {
+            float y[8], sg[8];
+            dyn8(c8, y, sg);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int c = 2 * c8 + hh;
+                const float4 a1 = a1p[c * BT], a2 = a2p[c * BT], g = gain4(c);
+                const float av1[4] = {a1.x, a1.y, a1.z, a1.w}, av2[4] = {a2.x, a2.y, a2.z, a2.w};
+                const float gg[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int k = 4 * hh + e;
+                    const float d = fmaf(-lam, av2[e], av1[e]);
+                    dd[k] = p.apply_norm ? fmaf(rn * gg[e], y[k], -coef * d) : y[k];
+                    const float ddh = __half2float(__float2half_rn(dd[k]));
+                    delta1 = fmaf(ddh, av1[e], delta1);
+                    dot2h = fmaf(ddh, av2[e], dot2h);
+                    dot2 = fmaf(dd[k], av2[e], dot2);
+                    gt[k] = y[k] * d * rn;
+                    bad |= !(fabsf(dd[k]) <= 65504.0f);
+                    // dG = dY Yn sigma'(G) = dYn Yn (1 - sigma(G)), Yn = D r gain (or D)
+                    const float yn = p.apply_norm ? d * rn * gg[e] : d;
+                    dgv[k] = y[k] * yn * (1.0f - sg[k]);
+                }
             }
-            *reinterpret_cast<uint2 *>(ddrow + 4 * c) = make_uint2(pack_half2(dd[0], dd[1]), pack_half2(dd[2], dd[3]));
+            *reinterpret_cast<uint4 *>(ddrow + 8 * c8) =
+                make_uint4(pack_half2(dd[0], dd[1]), pack_half2(dd[2], dd[3]), pack_half2(dd[4], dd[5]),
+                           pack_half2(dd[6], dd[7]));
             if (dgrow)
-                *reinterpret_cast<uint2 *>(dgrow + 4 * c) =
-                    make_uint2(pack_bf162(dgv[0], dgv[1]), pack_bf162(dgv[2], dgv[3]));
+                *reinterpret_cast<uint4 *>(dgrow + 8 * c8) =
+                    make_uint4(pack_bf162(dgv[0], dgv[1]), pack_bf162(dgv[2], dgv[3]), pack_bf162(dgv[4], dgv[5]),
+                               pack_bf162(dgv[6], dgv[7]));
         }
         if (want_dgain) {
-            // This row's terms of columns 4c .. 4c + 3; after every eighth
-            // chunk the CTA sums the group's 32 columns over its 128 rows
-            // (a quarter of the rows per warp, then the four partials).
+            // This row's terms of columns 8 c8 .. 8 c8 + 7; after every fourth
+            // step the CTA sums the group's 32 columns over its 128 rows (a
+            // quarter of the rows per warp, then the four partials).
 #pragma unroll
-            for (int e = 0; e < 4; ++e) red[r * 33 + 4 * (c & 7) + e] = gt[e];
-            if ((c & 7) == 7) {
+            for (int e = 0; e < 8; ++e) red[r * 33 + 8 * (c8 & 3) + e] = gt[e];
+            if ((c8 & 3) == 3) {
                 __syncthreads();
                 const int col = r & 31, r0 = (r >> 5) * 32;
                 float v = 0.f;
@@ -383,7 +400,7 @@ __global__ void __launch_bounds__(128)
                 __syncthreads();
                 if (r < 32) {
                     const float t = col_part[0][r] + col_part[1][r] + col_part[2][r] + col_part[3][r];
-                    const int grp = c >> 3;
+                    const int grp = c8 >> 2;
                     dgc0 = grp == 0 ? t : dgc0;
                     dgc1 = grp == 1 ? t : dgc1;
                     dgc2 = grp == 2 ? t : dgc2;
