@@ -575,6 +575,7 @@ diffattn_status run_bwd(const diffattn_bwd_args *a, void *ws, size_t ws_bytes, v
     if (e != cudaSuccess) return cuda_status(e);
 
     da::BwdParams p{};
+    p.tile_counter = counters;
     p.B = (int)a->B;
     p.N = (int)a->N;
     p.H = (int)a->H;

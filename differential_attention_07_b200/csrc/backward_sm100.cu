@@ -83,7 +83,12 @@ enum : int {
     B_DONE,                         // every product of the CTA has completed (commit)
     B_SDRAIN,                       // the score issuer's products have completed (commit)
     B_AOP,                          // the tile's A operands are in TMEM (8 arrivals)
-    NBARS
+    B_TILEFREE,                     // key tiles: the tile's score products are done with its K and V (commit)
+    B_ACCFREE,                      // key tiles: the epilogue has read the accumulators (8 arrivals)
+    B_ADRAIN,                       // key tiles: the accumulating issuer's products have completed (commit)
+    B_ITEM,                         // key tiles: [4] a tile index published (1 arrival)
+    B_ITEMFREE = B_ITEM + 4,        // key tiles: [4] the tile index read by all ten reader warps
+    NBARS = B_ITEMFREE + 4
 };
 
 // ---------------------------------------------------------------- key-tile kernel
@@ -98,7 +103,7 @@ constexpr uint32_t KB_BYTES = (KB_LOAD + 1023) & ~1023u;   // stages stay 1 KB a
 constexpr uint32_t KT_A = KT_STAGE0 + KSTAGES * KB_BYTES;
 constexpr uint32_t KA_PV = 0, KA_DS1 = 16384, KA_DS2 = 32768;
 constexpr uint32_t KT_BARS = KT_A + 3 * 16384;
-constexpr uint32_t KT_SMEM = KT_BARS + 8 * NBARS + 16;
+constexpr uint32_t KT_SMEM = KT_BARS + 8 * NBARS + 32;  // + TMEM address, abort flag, 4-slot tile ring
 // TMEM columns: dV, dK_1, dK_2 accumulators, then S_1^T, S_2^T, dP^T, then
 // the tile's K_1 and K_2 (bf16 / fp16 pairs) as the A operand of the score
 // products, so that every block's score products read only Q from shared
@@ -502,6 +507,19 @@ __device__ __forceinline__ void acc_issuer(int nit, uint32_t bar_afull, uint32_t
 }
 
 // ---------------------------------------------------------------- 2. key tiles
+// A persistent kernel: one CTA per SM takes key tiles, heaviest first (under
+// the causal mask key tile 0 meets every query), from a counter in the
+// workspace (zeroed by the staging kernel); the producer publishes each to
+// the other roles in a 4-slot ring.  The next tile's operands load, and its K rows go into TMEM,
+// while the element-wise warps write out the finished tile's dV and dK; its
+// first block's score products run during that epilogue.  Per tile:
+//   producer: TILEFREE (previous tile) -> the tile's K_1, K_2, V -> its blocks;
+//   score issuer: AOP (tile) -> the blocks' score and dP products -> TILEFREE;
+//   accumulating issuer: per block AFULL (block 0 also ACCFREE, previous
+//     tile) -> dV, dK_1, dK_2 products -> DONE (tile) after the last block;
+//   element-wise warps: TILE -> K rows into TMEM, AOP -> the previous tile's
+//     epilogue (DONE, TMEM reads, stores), ACCFREE -> the tile's blocks.
+// Block barriers count blocks over the CTA's whole sequence (G below).
 template <bool F16QK>
 __global__ void __launch_bounds__(NT, 1)
     bwd_key_kernel(const __grid_constant__ BwdKeyMaps m, const BwdParams p)
@@ -513,24 +531,49 @@ __global__ void __launch_bounds__(NT, 1)
         if (threadIdx.x == 0) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
         return;
     }
-    // Heavy tiles first: under the causal mask key tile 0 meets every query.
-    const int BH = p.B * p.H;
-    const int kt = blockIdx.x / BH, bh = blockIdx.x % BH, b = bh / p.H, h = bh % p.H;
-    const int hn = h / (p.H / p.H_N), hv = h / (p.H / p.H_V);
-    const int k0 = kt * BT;
-    // Query blocks that see a key of the tile: causal from the block holding
-    // k0; under a window of W keys up to the one holding k0 + 127 + W - 1.
+    const int BH = p.B * p.H, n_tiles = p.num_qt * BH;
     const int nqb_all = (p.N + BB - 1) / BB;
-    const int qb0 = p.causal ? k0 / BB : 0;
-    const int qb1 = p.window > 0 ? min(nqb_all, (k0 + BT - 1 + p.window - 1) / BB + 1) : nqb_all;
-    const int nit = qb1 - qb0;  // >= 1: k0 < N
+    struct Tile {
+        int b, h, hn, hv, k0, qb0, nit;
+    };
+    auto tile_of = [&](int t) {
+        Tile T;
+        const int kt = t / BH, bh = t % BH;
+        T.b = bh / p.H;
+        T.h = bh % p.H;
+        T.hn = T.h / (p.H / p.H_N);
+        T.hv = T.h / (p.H / p.H_V);
+        T.k0 = kt * BT;
+        // Query blocks that see a key of the tile: causal from the block
+        // holding k0; under a window of W keys up to the one holding
+        // k0 + 127 + W - 1.
+        T.qb0 = p.causal ? T.k0 / BB : 0;
+        const int qb1 = p.window > 0 ? min(nqb_all, (T.k0 + BT - 1 + p.window - 1) / BB + 1) : nqb_all;
+        T.nit = qb1 - T.qb0;  // >= 1: k0 < N
+        return T;
+    };
     auto bar = [&](int i) { return sbase + KT_BARS + 8 * i; };
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + KT_BARS + 8 * NBARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + KT_BARS + 8 * NBARS + 4);
+    int *sItem = reinterpret_cast<int *>(smem + KT_BARS + 8 * NBARS + 16);
     const uint64_t lim = p.timeout_ns;
+    // Tile k of this CTA from ring slot k % 4; -1 ends the loop (also when
+    // a bounded wait gives up).
+    auto read_tile = [&](int k) -> int {
+        const int slot = k & 3;
+        if (!mbar_wait_warp(bar(B_ITEM + slot), (k >> 2) & 1, abort_flag, lim)) return -1;
+        const int t = *reinterpret_cast<volatile int *>(&sItem[slot]);
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(bar(B_ITEMFREE + slot));
+        return t;
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_TILE), 1);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(bar(B_ITEM + i), 1);
+            mbar_init(bar(B_ITEMFREE + i), 2 + NEW);  // the two issuers and the element-wise warps
+        }
         for (int s = 0; s < MAXSTAGES; ++s) {
             mbar_init(bar(B_FULL + s), 1);
             mbar_init(bar(B_EMPTY + s), 1);
@@ -542,6 +585,9 @@ __global__ void __launch_bounds__(NT, 1)
         mbar_init(bar(B_DONE), 1);
         mbar_init(bar(B_SDRAIN), 1);
         mbar_init(bar(B_AOP), NEW);
+        mbar_init(bar(B_TILEFREE), 1);
+        mbar_init(bar(B_ACCFREE), NEW);
+        mbar_init(bar(B_ADRAIN), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -556,42 +602,64 @@ __global__ void __launch_bounds__(NT, 1)
 
     if (R.producer()) {
         // ------------------------------------------------------------ TMA producer
-        if (elect_one()) {
-            mbar_arrive_expect_tx(bar(B_TILE), KT_STAGE0);
-            tma_load_4d_nohint(sbase + KT_K1, &m.k1, bar(B_TILE), 0, k0, h, b);
-            tma_load_4d_nohint(sbase + KT_K2, &m.k2, bar(B_TILE), 0, k0, hn, b);
-            tma_load_4d_nohint(sbase + KT_V, &m.v, bar(B_TILE), 0, k0, hv, b);
-            tma_load_4d_nohint(sbase + KT_V + 16384, &m.v, bar(B_TILE), 64, k0, hv, b);
-        }
-        __syncwarp();
-        int loads = 0;
-        for (int j = 0; j < nit; ++j) {
-            const int s = j % KSTAGES;
-            if (j >= KSTAGES && !mbar_wait_warp(bar(B_EMPTY + s), ((j / KSTAGES) - 1) & 1, abort_flag, lim)) break;
+        int G = 0, ti = 0, tile_loads = 0;
+        bool ok = true;
+        for (;; ++ti) {
+            const int slot = ti & 3;
+            if (ti >= 4 && !(ok = mbar_wait_warp(bar(B_ITEMFREE + slot), ((ti >> 2) - 1) & 1, abort_flag, lim)))
+                break;
+            int t = 0;
+            if (R.lane == 0) {
+                t = *abort_flag ? n_tiles : atomicAdd(p.tile_counter, 1);
+                sItem[slot] = t < n_tiles ? t : -1;
+                mbar_arrive(bar(B_ITEM + slot));
+            }
+            t = __shfl_sync(0xffffffffu, t, 0);
+            if (t >= n_tiles) break;
+            const Tile T = tile_of(t);
+            // The previous tile's score products must be done with its K
+            // (in TMEM) and V.
+            if (ti > 0 && !(ok = mbar_wait_warp(bar(B_TILEFREE), (ti - 1) & 1, abort_flag, lim))) break;
             if (elect_one()) {
-                const uint32_t st = sbase + KT_STAGE0 + s * KB_BYTES, fb = bar(B_FULL + s);
-                const int q0 = (qb0 + j) * BB;
-                mbar_arrive_expect_tx(fb, KB_LOAD);
-                tma_load_4d_nohint(st + KB_Q1, &m.q1, fb, 0, q0, h, b);
-                tma_load_4d_nohint(st + KB_Q2, &m.q2, fb, 0, q0, hn, b);
-                tma_load_4d_nohint(st + KB_DD, &m.dd, fb, 0, q0, h, b);
-                tma_load_4d_nohint(st + KB_DD + 8192, &m.dd, fb, 64, q0, h, b);
-                tma_load_4d_nohint(st + KB_ST, &m.stats, fb, q0, 0, h, b);
+                mbar_arrive_expect_tx(bar(B_TILE), KT_STAGE0);
+                tma_load_4d_nohint(sbase + KT_K1, &m.k1, bar(B_TILE), 0, T.k0, T.h, T.b);
+                tma_load_4d_nohint(sbase + KT_K2, &m.k2, bar(B_TILE), 0, T.k0, T.hn, T.b);
+                tma_load_4d_nohint(sbase + KT_V, &m.v, bar(B_TILE), 0, T.k0, T.hv, T.b);
+                tma_load_4d_nohint(sbase + KT_V + 16384, &m.v, bar(B_TILE), 64, T.k0, T.hv, T.b);
             }
             __syncwarp();
-            loads = j + 1;
+            ++tile_loads;
+            for (int j = 0; j < T.nit; ++j) {
+                const int s = G % KSTAGES;
+                if (G >= KSTAGES &&
+                    !(ok = mbar_wait_warp(bar(B_EMPTY + s), ((G / KSTAGES) - 1) & 1, abort_flag, lim)))
+                    break;
+                if (elect_one()) {
+                    const uint32_t st = sbase + KT_STAGE0 + s * KB_BYTES, fb = bar(B_FULL + s);
+                    const int q0 = (T.qb0 + j) * BB;
+                    mbar_arrive_expect_tx(fb, KB_LOAD);
+                    tma_load_4d_nohint(st + KB_Q1, &m.q1, fb, 0, q0, T.h, T.b);
+                    tma_load_4d_nohint(st + KB_Q2, &m.q2, fb, 0, q0, T.hn, T.b);
+                    tma_load_4d_nohint(st + KB_DD, &m.dd, fb, 0, q0, T.h, T.b);
+                    tma_load_4d_nohint(st + KB_DD + 8192, &m.dd, fb, 64, q0, T.h, T.b);
+                    tma_load_4d_nohint(st + KB_ST, &m.stats, fb, q0, 0, T.h, T.b);
+                }
+                __syncwarp();
+                ++G;
+            }
         }
         // No load of ours may land after the CTA has gone.
-        bool drained = mbar_wait_drain(bar(B_TILE), 0, lim);
-        for (int k = (loads > KSTAGES ? loads - KSTAGES : 0); k < loads; ++k)
+        bool drained = true;
+        if (tile_loads > 0) drained = mbar_wait_drain(bar(B_TILE), (tile_loads - 1) & 1, lim);
+        for (int k = (G > KSTAGES ? G - KSTAGES : 0); k < G; ++k)
             drained &= mbar_wait_drain(bar(B_FULL + k % KSTAGES), (k / KSTAGES) & 1, lim);
         if (!__all_sync(0xffffffffu, drained) && R.lane == 0) *abort_flag = 1;
     } else if (R.score_issuer() || R.acc_issuer()) {
         // ------------------------------------------------------------ MMA issuers
         // Warp 1 issues the score and dP products, warp 2 the accumulating
-        // products (see score_issuer / acc_issuer).
-        auto issue_s = [&](int j) {
-            const uint32_t st = sbase + KT_STAGE0 + (j % KSTAGES) * KB_BYTES;
+        // products; neither waits behind the other in one program order.
+        auto issue_s = [&](int G) {
+            const uint32_t st = sbase + KT_STAGE0 + (G % KSTAGES) * KB_BYTES;
 #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk)
                 mma_issue_ts(tbase + KM_S1, tbase + KM_AK1 + 8 * kk, sw128(st + KB_Q1 + 32 * kk), Ids<F16QK>::S,
@@ -608,48 +676,136 @@ __global__ void __launch_bounds__(NT, 1)
             }
             commit_to(bar(B_SFULL));
         };
-        auto issue_acc = [&](int j) {
-            const uint32_t st = sbase + KT_STAGE0 + (j % KSTAGES) * KB_BYTES;
+        auto issue_acc = [&](int G, bool first) {
+            const uint32_t st = sbase + KT_STAGE0 + (G % KSTAGES) * KB_BYTES;
             // dV += (P_1 - lambda P_2)^T dD; dK_t += dS_t^T Q_t (B MN-major).
 #pragma unroll
             for (int kk = 0; kk < BB / 16; ++kk)
                 mma_issue(tbase + KM_DV, sw128(sbase + KT_A + KA_PV + 32 * kk), sw128(st + KB_DD + 2048 * kk, 8192),
-                          ID_DV, j > 0 || kk > 0);
+                          ID_DV, !first || kk > 0);
 #pragma unroll
             for (int kk = 0; kk < BB / 16; ++kk)
                 mma_issue(tbase + KM_DK1, sw128(sbase + KT_A + KA_DS1 + 32 * kk), sw128(st + KB_Q1 + 2048 * kk, 8192),
-                          Ids<F16QK>::DS, j > 0 || kk > 0);
+                          Ids<F16QK>::DS, !first || kk > 0);
 #pragma unroll
             for (int kk = 0; kk < BB / 16; ++kk)
                 mma_issue(tbase + KM_DK2, sw128(sbase + KT_A + KA_DS2 + 32 * kk), sw128(st + KB_Q2 + 2048 * kk, 8192),
-                          Ids<F16QK>::DS, j > 0 || kk > 0);
+                          Ids<F16QK>::DS, !first || kk > 0);
             commit_to(bar(B_AFREE));
-            commit_to(bar(B_EMPTY + j % KSTAGES));
+            commit_to(bar(B_EMPTY + G % KSTAGES));
         };
-        if (R.score_issuer())
-            score_issuer<KSTAGES>(nit, bar(B_AOP), bar(B_FULL), bar(B_SFREE), bar(B_SDRAIN), abort_flag, lim, issue_s,
-                                  R.lane);
-        else
-            acc_issuer(nit, bar(B_AFULL), bar(B_DONE), abort_flag, lim, issue_acc, R.lane);
+        int G = 0, ti = 0;
+        bool ok = true;
+        if (R.score_issuer()) {
+            for (;; ++ti) {
+                const int t = read_tile(ti);
+                if (t < 0) break;
+                const Tile T = tile_of(t);
+                // the tile's K rows are in TMEM (the A operand of its score products)
+                if (!(ok = mbar_wait_warp(bar(B_AOP), ti & 1, abort_flag, lim))) break;
+                for (int j = 0; ok && j < T.nit; ++j, ++G) {
+                    if (!(ok = mbar_wait_warp(bar(B_FULL + G % KSTAGES), (G / KSTAGES) & 1, abort_flag, lim))) break;
+                    if (G > 0 && !(ok = mbar_wait_warp(bar(B_SFREE), (G - 1) & 1, abort_flag, lim))) break;
+                    tc_fence_after();
+                    issue_s(G);
+                }
+                if (ok) commit_to(bar(B_TILEFREE));  // the tile's K (TMEM) and V may be replaced once these are done
+            }
+            // Nothing of ours may still run on the tensor cores at teardown.
+            commit_to(bar(B_SDRAIN));
+            if (!__all_sync(0xffffffffu, mbar_wait_drain(bar(B_SDRAIN), 0, lim)) && R.lane == 0) *abort_flag = 1;
+        } else {
+            for (;; ++ti) {
+                const int t = read_tile(ti);
+                if (t < 0) break;
+                const Tile T = tile_of(t);
+                for (int j = 0; ok && j < T.nit; ++j, ++G) {
+                    if (!(ok = mbar_wait_warp(bar(B_AFULL), G & 1, abort_flag, lim))) break;
+                    // The tile's first products overwrite the accumulators:
+                    // the previous tile's epilogue must have read them.
+                    if (j == 0 && ti > 0 && !(ok = mbar_wait_warp(bar(B_ACCFREE), (ti - 1) & 1, abort_flag, lim)))
+                        break;
+                    tc_fence_after();
+                    issue_acc(G, j == 0);
+                }
+                // DONE completes once every product of the tile has (its
+                // score products completed before its last accumulating
+                // products were issued): the epilogue's signal.
+                if (ok) commit_to(bar(B_DONE));
+            }
+            // Nothing of ours may still run on the tensor cores at teardown.
+            commit_to(bar(B_ADRAIN));
+            if (!__all_sync(0xffffffffu, mbar_wait_drain(bar(B_ADRAIN), 0, lim)) && R.lane == 0) *abort_flag = 1;
+        }
     } else {
         // ------------------------------------------------------------ element-wise + epilogue
         const int wg = R.wg(), r = R.row();
         const uint32_t lo = R.lane_off();
-        const int kj = k0 + r;  // this thread's key
         const float c = p.scale_log2;
-        // The tile's K_1 (warpgroup 0) and K_2 (warpgroup 1) rows into TMEM,
-        // the A operand of every block's score products.
-        bool ok = mbar_wait_warp(bar(B_TILE), 0, abort_flag, lim), big = false;
-        if (ok) {
+        bool ok = true, big = false;
+        // The finished tile's dV and dK from TMEM to global memory (after
+        // its last products): warpgroup 0 writes dV columns [0, 64) and
+        // dK_1, warpgroup 1 dV columns [64, 128) and dK_2; then the
+        // accumulators are released to the next tile's products.
+        auto epilogue = [&](const Tile &T, int ti) -> bool {
+            if (!mbar_wait_warp(bar(B_DONE), ti & 1, abort_flag, lim)) return false;
+            const int b = T.b, h = T.h, hn = T.hn, hv = T.hv, kj = T.k0 + r;
+                // Warpgroup 0 writes dV columns [0, 64) and dK_1; warpgroup 1 dV
+                // columns [64, 128) and dK_2.  Every lane takes part in the TMEM
+                // loads (warp-collective); only rows of keys below N are stored.
+                tc_fence_after();
+                const bool own = kj < p.N;
+                const int krow = own ? kj : 0;
+                float x[64];
+                tmem_row64(tbase + lo + KM_DV + 64 * wg, x);
+                if (own) {
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dv) + (size_t)b * p.dv_s[0] +
+                                         (size_t)krow * p.dv_s[1] + (size_t)hv * p.dv_s[2] + 64 * wg;
+                    float *acc = p.acc_dv ? p.acc_dv + (((size_t)b * p.N + krow) * p.H_V + hv) * HDV + 64 * wg : nullptr;
+                    put_row<64>(x, 1.0f, dst, acc);
+                }
+                tmem_row64(tbase + lo + (wg ? KM_DK2 : KM_DK1), x);
+                if (own) {
+                    if (F16QK) unrotate64(x, krow, p.rope_g);
+                    if (wg == 0) {
+                        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dk1) + (size_t)b * p.dk1_s[0] +
+                                             (size_t)krow * p.dk1_s[1] + (size_t)h * p.dk1_s[2];
+                        put_row<64>(x, p.scale, dst, nullptr);
+                    } else {
+                        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dk2) + (size_t)b * p.dk2_s[0] +
+                                             (size_t)krow * p.dk2_s[1] + (size_t)hn * p.dk2_s[2];
+                        float *acc = p.acc_dk2 ? p.acc_dk2 + (((size_t)b * p.N + krow) * p.H_N + hn) * HD : nullptr;
+                        put_row<64>(x, p.scale, dst, acc);
+                    }
+                }
+            tc_fence_before();
+            __syncwarp();
+            if (R.lane == 0) mbar_arrive(bar(B_ACCFREE));
+            return true;
+        };
+        int G = 0, ti = 0;
+        Tile prev{};
+        for (;; ++ti) {
+            const int t = read_tile(ti);
+            if (t < 0) break;
+            const Tile T = tile_of(t);
+            const int kj = T.k0 + r;  // this thread's key
+            // The tile's K_1 (warpgroup 0) and K_2 (warpgroup 1) rows into
+            // TMEM, the A operand of every block's score products (the
+            // producer loaded them once the previous tile's score products
+            // were done with the old ones).
+            if (!(ok = mbar_wait_warp(bar(B_TILE), ti & 1, abort_flag, lim))) break;
             tile_row_to_tmem(sbase + (wg ? KT_K2 : KT_K1), r, tbase + lo + (wg ? KM_AK2 : KM_AK1));
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (R.lane == 0) mbar_arrive(bar(B_AOP));
-        }
-        for (int j = 0; ok && j < nit; ++j) {
-            if (!(ok = mbar_wait_warp(bar(B_SFULL), j & 1, abort_flag, lim))) break;
-            tc_fence_after();
+            // The previous tile's epilogue, while this tile's first score
+            // products run.
+            if (ti > 0 && !(ok = epilogue(prev, ti - 1))) break;
+            for (int j = 0; ok && j < T.nit; ++j, ++G) {
+                if (!(ok = mbar_wait_warp(bar(B_SFULL), G & 1, abort_flag, lim))) break;
+                tc_fence_after();
             uint32_t s1[32], s2[32], dp[32];
             tmem_ld32(tbase + lo + KM_S1 + 32 * wg, s1);
             tmem_ld32(tbase + lo + KM_S2 + 32 * wg, s2);
@@ -659,9 +815,9 @@ __global__ void __launch_bounds__(NT, 1)
             __syncwarp();
             if (R.lane == 0) mbar_arrive(bar(B_SFREE));
             // This warpgroup's 32 queries of the block, and their statistics.
-            const int qb = (qb0 + j) * BB + 32 * wg;
-            const uint32_t st = sbase + KT_STAGE0 + (j % KSTAGES) * KB_BYTES + KB_ST + 4 * 32 * wg;
-            const bool mask = (p.causal && qb < k0 + BT - 1) || (p.window > 0 && qb + 31 - k0 >= p.window);
+            const int qb = (T.qb0 + j) * BB + 32 * wg;
+            const uint32_t st = sbase + KT_STAGE0 + (G % KSTAGES) * KB_BYTES + KB_ST + 4 * 32 * wg;
+            const bool mask = (p.causal && qb < T.k0 + BT - 1) || (p.window > 0 && qb + 31 - T.k0 >= p.window);
             uint32_t pv[16], d1p[16], d2p[16];
             const float2 c2 = make_float2(c, c);
 #pragma unroll
@@ -713,48 +869,21 @@ __global__ void __launch_bounds__(NT, 1)
                 // point: hoisted all at once they would need 160 registers.
                 asm volatile("" ::: "memory");
             }
-            // The previous block's accumulating products must have read the
-            // A operands before they are overwritten.
-            if (j > 0 && !(ok = mbar_wait_warp(bar(B_AFREE), (j - 1) & 1, abort_flag, lim))) break;
+            // The previous block's accumulating products (of this tile or the
+            // one before) must have read the A operands before they are
+            // overwritten.
+            if (G > 0 && !(ok = mbar_wait_warp(bar(B_AFREE), (G - 1) & 1, abort_flag, lim))) break;
             st_operand_half(sbase + KT_A + KA_PV, r, wg, pv);
             st_operand_half(sbase + KT_A + KA_DS1, r, wg, d1p);
             st_operand_half(sbase + KT_A + KA_DS2, r, wg, d2p);
             fence_proxy_async_smem();
             __syncwarp();
             if (R.lane == 0) mbar_arrive(bar(B_AFULL));
+            }
+            prev = T;
         }
+        if (ok && ti > 0) ok = epilogue(prev, ti - 1);
         if (big) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
-        if (ok) ok = mbar_wait_warp(bar(B_DONE), 0, abort_flag, lim);
-        if (ok) {
-            // Warpgroup 0 writes dV columns [0, 64) and dK_1; warpgroup 1 dV
-            // columns [64, 128) and dK_2.  Every lane takes part in the TMEM
-            // loads (warp-collective); only rows of keys below N are stored.
-            tc_fence_after();
-            const bool own = kj < p.N;
-            const int krow = own ? kj : 0;
-            float x[64];
-            tmem_row64(tbase + lo + KM_DV + 64 * wg, x);
-            if (own) {
-                __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dv) + (size_t)b * p.dv_s[0] +
-                                     (size_t)krow * p.dv_s[1] + (size_t)hv * p.dv_s[2] + 64 * wg;
-                float *acc = p.acc_dv ? p.acc_dv + (((size_t)b * p.N + krow) * p.H_V + hv) * HDV + 64 * wg : nullptr;
-                put_row<64>(x, 1.0f, dst, acc);
-            }
-            tmem_row64(tbase + lo + (wg ? KM_DK2 : KM_DK1), x);
-            if (own) {
-                if (F16QK) unrotate64(x, krow, p.rope_g);
-                if (wg == 0) {
-                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dk1) + (size_t)b * p.dk1_s[0] +
-                                         (size_t)krow * p.dk1_s[1] + (size_t)h * p.dk1_s[2];
-                    put_row<64>(x, p.scale, dst, nullptr);
-                } else {
-                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dk2) + (size_t)b * p.dk2_s[0] +
-                                         (size_t)krow * p.dk2_s[1] + (size_t)hn * p.dk2_s[2];
-                    float *acc = p.acc_dk2 ? p.acc_dk2 + (((size_t)b * p.N + krow) * p.H_N + hn) * HD : nullptr;
-                    put_row<64>(x, p.scale, dst, acc);
-                }
-            }
-        }
     }
     tc_fence_before();
     __syncthreads();
@@ -1077,10 +1206,14 @@ cudaError_t launch_bwd(const BwdKeyMaps &km, const BwdQueryMaps &qm, const BwdPa
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (ev.start) cudaEventRecord(ev.start, stream);
+    // The key-tile kernel is persistent: one CTA per SM (or per tile, when
+    // there are fewer).
+    const int sms = device_sm_count();
+    const int key_grid = tiles < sms ? tiles : sms;
     if (p.qk_f16)
-        bwd_key_kernel<true><<<tiles, NT, KT_SMEM, stream>>>(km, p);
+        bwd_key_kernel<true><<<key_grid, NT, KT_SMEM, stream>>>(km, p);
     else
-        bwd_key_kernel<false><<<tiles, NT, KT_SMEM, stream>>>(km, p);
+        bwd_key_kernel<false><<<key_grid, NT, KT_SMEM, stream>>>(km, p);
     ++*launches;
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
