@@ -80,14 +80,14 @@ enum : int {
     B_SFREE,                        // the element-wise warps loaded them (8 arrivals)
     B_AFULL,                        // the element-wise warps wrote the A operands (8 arrivals)
     B_AFREE,                        // the accumulating products have read the A operands (commit)
-    B_DONE,                         // every product of the CTA has completed (commit)
+    B_DONE,                         // every product of the tile has completed (commit)
     B_SDRAIN,                       // the score issuer's products have completed (commit)
     B_AOP,                          // the tile's A operands are in TMEM (8 arrivals)
     B_TILEFREE,                     // key tiles: the tile's score products are done with its K and V (commit)
-    B_ACCFREE,                      // key tiles: the epilogue has read the accumulators (8 arrivals)
-    B_ADRAIN,                       // key tiles: the accumulating issuer's products have completed (commit)
-    B_ITEM,                         // key tiles: [4] a tile index published (1 arrival)
-    B_ITEMFREE = B_ITEM + 4,        // key tiles: [4] the tile index read by all ten reader warps
+    B_ACCFREE,                      // the epilogue has read the accumulators (8 arrivals)
+    B_ADRAIN,                       // the accumulating issuer's products have completed (commit)
+    B_ITEM,                         // [4] a tile index published (1 arrival)
+    B_ITEMFREE = B_ITEM + 4,        // [4] the tile index read by all ten reader warps
     NBARS = B_ITEMFREE + 4
 };
 
@@ -121,7 +121,7 @@ constexpr uint32_t QB_K1 = 0, QB_K2 = 8192, QB_V = 16384, QB_BYTES = 32768;
 constexpr uint32_t QT_A = QT_STAGE0 + QSTAGES * QB_BYTES;
 constexpr uint32_t QA_DS1 = 0, QA_DS2 = 16384;
 constexpr uint32_t QT_BARS = QT_A + 2 * 16384;
-constexpr uint32_t QT_SMEM = QT_BARS + 8 * NBARS + 16;
+constexpr uint32_t QT_SMEM = QT_BARS + 8 * NBARS + 32;  // + TMEM address, abort flag, 4-slot tile ring
 // TMEM columns: dQ_1, dQ_2 accumulators, then S_1, S_2, dP, then the tile's
 // Q_1, Q_2 and dD (16-bit pairs) as the A operands of the score and dP
 // products, so that every block's products read only K and V from shared
@@ -464,47 +464,17 @@ struct Roles {
     __device__ __forceinline__ uint32_t lane_off() const { return uint32_t((warp & 3) * 32) << 16; }
 };
 
-// The two MMA issuers of a tile kernel, one warp each, so that neither
-// kind of product waits behind the other in one warp's program order:
-//  * the score issuer: block j's score and dP products, once its stage has
-//    landed and the element-wise warps have taken block j-1's products out
-//    of TMEM (early in their step);
-//  * the accumulating issuer: block j's accumulating products, once the
-//    element-wise warps have written their A operands (at the end of their
-//    step).
-// Block j's score products are complete before its accumulating products
-// are issued (the element-wise warps waited for them), so the accumulating
-// issuer's last commit covers every product of the tile.  Every wait is
+// Both tile kernels run two MMA issuers, one warp each, so that neither
+// kind of product waits behind the other in one warp's program order: the
+// score issuer (a block's score and dP products, once its stage has landed
+// and the element-wise warps have taken the previous block's products out
+// of TMEM, early in their step) and the accumulating issuer (a block's
+// accumulating products, once the element-wise warps have written their A
+// operands, at the end of their step).  A block's score products are
+// complete before its accumulating products are issued (the element-wise
+// warps waited for them), so the accumulating issuer's commit after a
+// tile's last block covers every product of the tile.  Every wait is
 // bounded; each issuer drains what it issued before the CTA tears down.
-template <int ST, class IssueS>
-__device__ __forceinline__ void score_issuer(int nit, uint32_t bar_aop, uint32_t bar_full, uint32_t bar_sfree,
-                                             uint32_t bar_drain, volatile int *abort_flag, uint64_t lim,
-                                             IssueS issue_s, int lane)
-{
-    bool ok = mbar_wait_warp(bar_aop, 0, abort_flag, lim);  // the tile's A operands are in TMEM
-    for (int j = 0; ok && j < nit; ++j) {
-        if (!(ok = mbar_wait_warp(bar_full + 8 * (j % ST), (j / ST) & 1, abort_flag, lim))) break;
-        if (j > 0 && !(ok = mbar_wait_warp(bar_sfree, (j - 1) & 1, abort_flag, lim))) break;
-        tc_fence_after();
-        issue_s(j);
-    }
-    commit_to(bar_drain);
-    if (!__all_sync(0xffffffffu, mbar_wait_drain(bar_drain, 0, lim)) && lane == 0) *abort_flag = 1;
-}
-template <class IssueAcc>
-__device__ __forceinline__ void acc_issuer(int nit, uint32_t bar_afull, uint32_t bar_done, volatile int *abort_flag,
-                                           uint64_t lim, IssueAcc issue_acc, int lane)
-{
-    for (int j = 0; j < nit; ++j) {
-        if (!mbar_wait_warp(bar_afull, j & 1, abort_flag, lim)) break;
-        tc_fence_after();
-        issue_acc(j);
-    }
-    // DONE completes once everything issued has: the epilogue's signal,
-    // and the teardown's guarantee that no product still runs.
-    commit_to(bar_done);
-    if (!__all_sync(0xffffffffu, mbar_wait_drain(bar_done, 0, lim)) && lane == 0) *abort_flag = 1;
-}
 
 // ---------------------------------------------------------------- 2. key tiles
 // A persistent kernel: one CTA per SM takes key tiles, heaviest first (under
@@ -647,6 +617,7 @@ __global__ void __launch_bounds__(NT, 1)
                 __syncwarp();
                 ++G;
             }
+            if (!ok) break;
         }
         // No load of ours may land after the CTA has gone.
         bool drained = true;
@@ -709,7 +680,8 @@ __global__ void __launch_bounds__(NT, 1)
                     tc_fence_after();
                     issue_s(G);
                 }
-                if (ok) commit_to(bar(B_TILEFREE));  // the tile's K (TMEM) and V may be replaced once these are done
+                if (!ok) break;
+                commit_to(bar(B_TILEFREE));  // the tile's K (TMEM) and V may be replaced once these are done
             }
             // Nothing of ours may still run on the tensor cores at teardown.
             commit_to(bar(B_SDRAIN));
@@ -728,10 +700,11 @@ __global__ void __launch_bounds__(NT, 1)
                     tc_fence_after();
                     issue_acc(G, j == 0);
                 }
+                if (!ok) break;
                 // DONE completes once every product of the tile has (its
                 // score products completed before its last accumulating
                 // products were issued): the epilogue's signal.
-                if (ok) commit_to(bar(B_DONE));
+                commit_to(bar(B_DONE));
             }
             // Nothing of ours may still run on the tensor cores at teardown.
             commit_to(bar(B_ADRAIN));
@@ -750,34 +723,34 @@ __global__ void __launch_bounds__(NT, 1)
         auto epilogue = [&](const Tile &T, int ti) -> bool {
             if (!mbar_wait_warp(bar(B_DONE), ti & 1, abort_flag, lim)) return false;
             const int b = T.b, h = T.h, hn = T.hn, hv = T.hv, kj = T.k0 + r;
-                // Warpgroup 0 writes dV columns [0, 64) and dK_1; warpgroup 1 dV
-                // columns [64, 128) and dK_2.  Every lane takes part in the TMEM
-                // loads (warp-collective); only rows of keys below N are stored.
-                tc_fence_after();
-                const bool own = kj < p.N;
-                const int krow = own ? kj : 0;
-                float x[64];
-                tmem_row64(tbase + lo + KM_DV + 64 * wg, x);
-                if (own) {
-                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dv) + (size_t)b * p.dv_s[0] +
-                                         (size_t)krow * p.dv_s[1] + (size_t)hv * p.dv_s[2] + 64 * wg;
-                    float *acc = p.acc_dv ? p.acc_dv + (((size_t)b * p.N + krow) * p.H_V + hv) * HDV + 64 * wg : nullptr;
-                    put_row<64>(x, 1.0f, dst, acc);
+            // Warpgroup 0 writes dV columns [0, 64) and dK_1; warpgroup 1 dV
+            // columns [64, 128) and dK_2.  Every lane takes part in the TMEM
+            // loads (warp-collective); only rows of keys below N are stored.
+            tc_fence_after();
+            const bool own = kj < p.N;
+            const int krow = own ? kj : 0;
+            float x[64];
+            tmem_row64(tbase + lo + KM_DV + 64 * wg, x);
+            if (own) {
+                __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dv) + (size_t)b * p.dv_s[0] +
+                                     (size_t)krow * p.dv_s[1] + (size_t)hv * p.dv_s[2] + 64 * wg;
+                float *acc = p.acc_dv ? p.acc_dv + (((size_t)b * p.N + krow) * p.H_V + hv) * HDV + 64 * wg : nullptr;
+                put_row<64>(x, 1.0f, dst, acc);
+            }
+            tmem_row64(tbase + lo + (wg ? KM_DK2 : KM_DK1), x);
+            if (own) {
+                if (F16QK) unrotate64(x, krow, p.rope_g);
+                if (wg == 0) {
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dk1) + (size_t)b * p.dk1_s[0] +
+                                         (size_t)krow * p.dk1_s[1] + (size_t)h * p.dk1_s[2];
+                    put_row<64>(x, p.scale, dst, nullptr);
+                } else {
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dk2) + (size_t)b * p.dk2_s[0] +
+                                         (size_t)krow * p.dk2_s[1] + (size_t)hn * p.dk2_s[2];
+                    float *acc = p.acc_dk2 ? p.acc_dk2 + (((size_t)b * p.N + krow) * p.H_N + hn) * HD : nullptr;
+                    put_row<64>(x, p.scale, dst, acc);
                 }
-                tmem_row64(tbase + lo + (wg ? KM_DK2 : KM_DK1), x);
-                if (own) {
-                    if (F16QK) unrotate64(x, krow, p.rope_g);
-                    if (wg == 0) {
-                        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dk1) + (size_t)b * p.dk1_s[0] +
-                                             (size_t)krow * p.dk1_s[1] + (size_t)h * p.dk1_s[2];
-                        put_row<64>(x, p.scale, dst, nullptr);
-                    } else {
-                        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dk2) + (size_t)b * p.dk2_s[0] +
-                                             (size_t)krow * p.dk2_s[1] + (size_t)hn * p.dk2_s[2];
-                        float *acc = p.acc_dk2 ? p.acc_dk2 + (((size_t)b * p.N + krow) * p.H_N + hn) * HD : nullptr;
-                        put_row<64>(x, p.scale, dst, acc);
-                    }
-                }
+            }
             tc_fence_before();
             __syncwarp();
             if (R.lane == 0) mbar_arrive(bar(B_ACCFREE));
@@ -806,80 +779,81 @@ __global__ void __launch_bounds__(NT, 1)
             for (int j = 0; ok && j < T.nit; ++j, ++G) {
                 if (!(ok = mbar_wait_warp(bar(B_SFULL), G & 1, abort_flag, lim))) break;
                 tc_fence_after();
-            uint32_t s1[32], s2[32], dp[32];
-            tmem_ld32(tbase + lo + KM_S1 + 32 * wg, s1);
-            tmem_ld32(tbase + lo + KM_S2 + 32 * wg, s2);
-            tmem_ld32(tbase + lo + KM_DP + 32 * wg, dp);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (R.lane == 0) mbar_arrive(bar(B_SFREE));
-            // This warpgroup's 32 queries of the block, and their statistics.
-            const int qb = (T.qb0 + j) * BB + 32 * wg;
-            const uint32_t st = sbase + KT_STAGE0 + (G % KSTAGES) * KB_BYTES + KB_ST + 4 * 32 * wg;
-            const bool mask = (p.causal && qb < T.k0 + BT - 1) || (p.window > 0 && qb + 31 - T.k0 >= p.window);
-            uint32_t pv[16], d1p[16], d2p[16];
-            const float2 c2 = make_float2(c, c);
+                uint32_t s1[32], s2[32], dp[32];
+                tmem_ld32(tbase + lo + KM_S1 + 32 * wg, s1);
+                tmem_ld32(tbase + lo + KM_S2 + 32 * wg, s2);
+                tmem_ld32(tbase + lo + KM_DP + 32 * wg, dp);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (R.lane == 0) mbar_arrive(bar(B_SFREE));
+                // This warpgroup's 32 queries of the block, and their statistics.
+                const int qb = (T.qb0 + j) * BB + 32 * wg;
+                const uint32_t st = sbase + KT_STAGE0 + (G % KSTAGES) * KB_BYTES + KB_ST + 4 * 32 * wg;
+                const bool mask = (p.causal && qb < T.k0 + BT - 1) || (p.window > 0 && qb + 31 - T.k0 >= p.window);
+                uint32_t pv[16], d1p[16], d2p[16];
+                const float2 c2 = make_float2(c, c);
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-                // the four queries' statistics, negated: -lse_1, -lse_2,
-                // -Delta_1, -Delta_2, -lambda
-                const uint4 ul1 = ld_shared_v4(st + 4 * i), ul2 = ld_shared_v4(st + 256 + 4 * i);
-                const uint4 ud1 = ld_shared_v4(st + 512 + 4 * i), ud2 = ld_shared_v4(st + 768 + 4 * i);
-                const uint4 ulm = ld_shared_v4(st + 1024 + 4 * i);
-                const uint32_t l1[4] = {ul1.x, ul1.y, ul1.z, ul1.w}, l2[4] = {ul2.x, ul2.y, ul2.z, ul2.w};
-                const uint32_t D1[4] = {ud1.x, ud1.y, ud1.z, ud1.w}, D2[4] = {ud2.x, ud2.y, ud2.z, ud2.w};
-                const uint32_t LM[4] = {ulm.x, ulm.y, ulm.z, ulm.w};
+                for (int i = 0; i < 32; i += 4) {
+                    // the four queries' statistics, negated: -lse_1, -lse_2,
+                    // -Delta_1, -Delta_2, -lambda
+                    const uint4 ul1 = ld_shared_v4(st + 4 * i), ul2 = ld_shared_v4(st + 256 + 4 * i);
+                    const uint4 ud1 = ld_shared_v4(st + 512 + 4 * i), ud2 = ld_shared_v4(st + 768 + 4 * i);
+                    const uint4 ulm = ld_shared_v4(st + 1024 + 4 * i);
+                    const uint32_t l1[4] = {ul1.x, ul1.y, ul1.z, ul1.w}, l2[4] = {ul2.x, ul2.y, ul2.z, ul2.w};
+                    const uint32_t D1[4] = {ud1.x, ud1.y, ud1.z, ud1.w}, D2[4] = {ud2.x, ud2.y, ud2.z, ud2.w};
+                    const uint32_t LM[4] = {ulm.x, ulm.y, ulm.z, ulm.w};
 #pragma unroll
-                for (int e = 0; e < 4; e += 2) {  // two queries at a time, in packed arithmetic
-                    auto f2 = [](const uint32_t *a, int k) { return make_float2(__uint_as_float(a[k]), __uint_as_float(a[k + 1])); };
-                    const float2 x1 = ffma2(f2(s1, i + e), c2, f2(l1, e));
-                    const float2 x2 = ffma2(f2(s2, i + e), c2, f2(l2, e));
-                    float2 p1, p2;
-                    if ((BWD_SOFT_EXP_MASK >> (((i + e) >> 1) & 7)) & 1u) {
-                        p1 = exp2_soft2(x1);
-                        p2 = exp2_soft2(x2);
-                    } else {
-                        p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
-                        p2 = make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
-                    }
-                    if (mask) {
+                    for (int e = 0; e < 4; e += 2) {  // two queries at a time, in packed arithmetic
+                        auto f2 = [](const uint32_t *a, int k) { return make_float2(__uint_as_float(a[k]), __uint_as_float(a[k + 1])); };
+                        const float2 x1 = ffma2(f2(s1, i + e), c2, f2(l1, e));
+                        const float2 x2 = ffma2(f2(s2, i + e), c2, f2(l2, e));
+                        float2 p1, p2;
+                        if ((BWD_SOFT_EXP_MASK >> (((i + e) >> 1) & 7)) & 1u) {
+                            p1 = exp2_soft2(x1);
+                            p2 = exp2_soft2(x2);
+                        } else {
+                            p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+                            p2 = make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
+                        }
+                        if (mask) {
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int q = qb + i + e + u;
-                            const bool vis = (!p.causal || q >= kj) && (p.window <= 0 || q - kj < p.window);
-                            if (!vis) {
-                                if (u) p1.y = p2.y = 0.f;
-                                else p1.x = p2.x = 0.f;
+                            for (int u = 0; u < 2; ++u) {
+                                const int q = qb + i + e + u;
+                                const bool vis = (!p.causal || q >= kj) && (p.window <= 0 || q - kj < p.window);
+                                if (!vis) {
+                                    if (u) p1.y = p2.y = 0.f;
+                                    else p1.x = p2.x = 0.f;
+                                }
                             }
                         }
+                        const float2 g = f2(dp, i + e), nlam = f2(LM, e);
+                        const float2 vp = ffma2(nlam, p2, p1);                     // P_1 - lambda P_2
+                        const float2 v1 = fmul2(p1, fadd2(g, f2(D1, e)));          // P_1 (dP - Delta_1)
+                        const float2 v2 = fmul2(p2, ffma2(nlam, g, f2(D2, e)));    // P_2 (-lambda dP - Delta_2)
+                        if (F16QK)
+                            big |= !(fabsf(v1.x) <= 65504.0f && fabsf(v1.y) <= 65504.0f && fabsf(v2.x) <= 65504.0f &&
+                                     fabsf(v2.y) <= 65504.0f);
+                        pv[(i + e) / 2] = pack_half2(vp.x, vp.y);
+                        d1p[(i + e) / 2] = pack_ds(v1.x, v1.y, F16QK);
+                        d2p[(i + e) / 2] = pack_ds(v2.x, v2.y, F16QK);
                     }
-                    const float2 g = f2(dp, i + e), nlam = f2(LM, e);
-                    const float2 vp = ffma2(nlam, p2, p1);                     // P_1 - lambda P_2
-                    const float2 v1 = fmul2(p1, fadd2(g, f2(D1, e)));          // P_1 (dP - Delta_1)
-                    const float2 v2 = fmul2(p2, ffma2(nlam, g, f2(D2, e)));    // P_2 (-lambda dP - Delta_2)
-                    if (F16QK)
-                        big |= !(fabsf(v1.x) <= 65504.0f && fabsf(v1.y) <= 65504.0f && fabsf(v2.x) <= 65504.0f &&
-                                 fabsf(v2.y) <= 65504.0f);
-                    pv[(i + e) / 2] = pack_half2(vp.x, vp.y);
-                    d1p[(i + e) / 2] = pack_ds(v1.x, v1.y, F16QK);
-                    d2p[(i + e) / 2] = pack_ds(v2.x, v2.y, F16QK);
+                    // Keep the next four queries' statistics loads below this
+                    // point: hoisted all at once they would need 160 registers.
+                    asm volatile("" ::: "memory");
                 }
-                // Keep the next four queries' statistics loads below this
-                // point: hoisted all at once they would need 160 registers.
-                asm volatile("" ::: "memory");
+                // The previous block's accumulating products (of this tile or the
+                // one before) must have read the A operands before they are
+                // overwritten.
+                if (G > 0 && !(ok = mbar_wait_warp(bar(B_AFREE), (G - 1) & 1, abort_flag, lim))) break;
+                st_operand_half(sbase + KT_A + KA_PV, r, wg, pv);
+                st_operand_half(sbase + KT_A + KA_DS1, r, wg, d1p);
+                st_operand_half(sbase + KT_A + KA_DS2, r, wg, d2p);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (R.lane == 0) mbar_arrive(bar(B_AFULL));
             }
-            // The previous block's accumulating products (of this tile or the
-            // one before) must have read the A operands before they are
-            // overwritten.
-            if (G > 0 && !(ok = mbar_wait_warp(bar(B_AFREE), (G - 1) & 1, abort_flag, lim))) break;
-            st_operand_half(sbase + KT_A + KA_PV, r, wg, pv);
-            st_operand_half(sbase + KT_A + KA_DS1, r, wg, d1p);
-            st_operand_half(sbase + KT_A + KA_DS2, r, wg, d2p);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (R.lane == 0) mbar_arrive(bar(B_AFULL));
-            }
+            if (!ok) break;
             prev = T;
         }
         if (ok && ti > 0) ok = epilogue(prev, ti - 1);
@@ -895,6 +869,20 @@ __global__ void __launch_bounds__(NT, 1)
 }
 
 // ---------------------------------------------------------------- 3. query tiles
+// Persistent like the key-tile kernel: one CTA per SM takes query tiles,
+// heaviest first (under the causal mask the last query tile meets every
+// key), from the second workspace counter through a 4-slot ring.  The
+// tile's Q_1, Q_2 and dD rows live in TMEM (the A operands of its score and
+// dP products), so their shared-memory copy may be replaced once they are
+// there.  Per tile:
+//   producer: AOP (previous tile) -> the tile's Q_1, Q_2, dD -> its blocks;
+//   score issuer: AOP (tile) -> the blocks' score and dP products;
+//   accumulating issuer: per block AFULL (block 0 also ACCFREE, previous
+//     tile) -> dQ_1, dQ_2 products -> DONE (tile) after the last block;
+//   element-wise warps: TILE -> Q and dD rows into TMEM (the previous
+//     tile's score products are complete: its last SFULL was seen), AOP ->
+//     the previous tile's epilogue (DONE, TMEM reads, stores), ACCFREE ->
+//     the tile's blocks.
 template <bool F16QK>
 __global__ void __launch_bounds__(NT, 1)
     bwd_query_kernel(const __grid_constant__ BwdQueryMaps m, const BwdParams p)
@@ -906,24 +894,46 @@ __global__ void __launch_bounds__(NT, 1)
         if (threadIdx.x == 0) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
         return;
     }
-    // Heavy tiles first: under the causal mask the last query tile meets every key.
-    const int BH = p.B * p.H;
-    const int qt = p.num_qt - 1 - (int)(blockIdx.x / BH), bh = blockIdx.x % BH, b = bh / p.H, h = bh % p.H;
-    const int hn = h / (p.H / p.H_N), hv = h / (p.H / p.H_V);
-    const int q0 = qt * BT;
-    // Key blocks the tile's queries see: up to the diagonal when causal;
-    // under a window of W keys from the block holding key q0 - W + 1.
+    const int BH = p.B * p.H, n_tiles = p.num_qt * BH;
     const int nkb_all = (p.N + BB - 1) / BB;
-    const int kb0 = p.window > 0 ? max(0, q0 - p.window + 1) / BB : 0;
-    const int kb1 = p.causal ? min(nkb_all, (q0 + BT - 1) / BB + 1) : nkb_all;
-    const int nit = kb1 - kb0;  // >= 1
+    struct Tile {
+        int b, h, hn, hv, q0, kb0, nit;
+    };
+    auto tile_of = [&](int t) {
+        Tile T;
+        const int qt = p.num_qt - 1 - t / BH, bh = t % BH;
+        T.b = bh / p.H;
+        T.h = bh % p.H;
+        T.hn = T.h / (p.H / p.H_N);
+        T.hv = T.h / (p.H / p.H_V);
+        T.q0 = qt * BT;
+        // Key blocks the tile's queries see: up to the diagonal when causal;
+        // under a window of W keys from the block holding key q0 - W + 1.
+        T.kb0 = p.window > 0 ? max(0, T.q0 - p.window + 1) / BB : 0;
+        const int kb1 = p.causal ? min(nkb_all, (T.q0 + BT - 1) / BB + 1) : nkb_all;
+        T.nit = kb1 - T.kb0;  // >= 1
+        return T;
+    };
     auto bar = [&](int i) { return sbase + QT_BARS + 8 * i; };
     uint32_t *tmem_ptr = reinterpret_cast<uint32_t *>(smem + QT_BARS + 8 * NBARS);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + QT_BARS + 8 * NBARS + 4);
+    int *sItem = reinterpret_cast<int *>(smem + QT_BARS + 8 * NBARS + 16);
     const uint64_t lim = p.timeout_ns;
+    auto read_tile = [&](int k) -> int {
+        const int slot = k & 3;
+        if (!mbar_wait_warp(bar(B_ITEM + slot), (k >> 2) & 1, abort_flag, lim)) return -1;
+        const int t = *reinterpret_cast<volatile int *>(&sItem[slot]);
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) mbar_arrive(bar(B_ITEMFREE + slot));
+        return t;
+    };
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_TILE), 1);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(bar(B_ITEM + i), 1);
+            mbar_init(bar(B_ITEMFREE + i), 2 + NEW);
+        }
         for (int s = 0; s < MAXSTAGES; ++s) {
             mbar_init(bar(B_FULL + s), 1);
             mbar_init(bar(B_EMPTY + s), 1);
@@ -935,6 +945,8 @@ __global__ void __launch_bounds__(NT, 1)
         mbar_init(bar(B_DONE), 1);
         mbar_init(bar(B_SDRAIN), 1);
         mbar_init(bar(B_AOP), NEW);
+        mbar_init(bar(B_ACCFREE), NEW);
+        mbar_init(bar(B_ADRAIN), 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -948,37 +960,63 @@ __global__ void __launch_bounds__(NT, 1)
     const uint32_t tbase = *tmem_ptr;
 
     if (R.producer()) {
-        if (elect_one()) {
-            mbar_arrive_expect_tx(bar(B_TILE), QT_STAGE0);
-            tma_load_4d_nohint(sbase + QT_Q1, &m.q1, bar(B_TILE), 0, q0, h, b);
-            tma_load_4d_nohint(sbase + QT_Q2, &m.q2, bar(B_TILE), 0, q0, hn, b);
-            tma_load_4d_nohint(sbase + QT_DD, &m.dd, bar(B_TILE), 0, q0, h, b);
-            tma_load_4d_nohint(sbase + QT_DD + 16384, &m.dd, bar(B_TILE), 64, q0, h, b);
-        }
-        __syncwarp();
-        int loads = 0;
-        for (int j = 0; j < nit; ++j) {
-            const int s = j % QSTAGES;
-            if (j >= QSTAGES && !mbar_wait_warp(bar(B_EMPTY + s), ((j / QSTAGES) - 1) & 1, abort_flag, lim)) break;
+        // ------------------------------------------------------------ TMA producer
+        int G = 0, ti = 0, tile_loads = 0;
+        bool ok = true;
+        for (;; ++ti) {
+            const int slot = ti & 3;
+            if (ti >= 4 && !(ok = mbar_wait_warp(bar(B_ITEMFREE + slot), ((ti >> 2) - 1) & 1, abort_flag, lim)))
+                break;
+            int t = 0;
+            if (R.lane == 0) {
+                t = *abort_flag ? n_tiles : atomicAdd(p.tile_counter + 1, 1);
+                sItem[slot] = t < n_tiles ? t : -1;
+                mbar_arrive(bar(B_ITEM + slot));
+            }
+            t = __shfl_sync(0xffffffffu, t, 0);
+            if (t >= n_tiles) break;
+            const Tile T = tile_of(t);
+            // The previous tile's rows must be in TMEM before its shared-memory
+            // copy is replaced.
+            if (ti > 0 && !(ok = mbar_wait_warp(bar(B_AOP), (ti - 1) & 1, abort_flag, lim))) break;
             if (elect_one()) {
-                const uint32_t st = sbase + QT_STAGE0 + s * QB_BYTES, fb = bar(B_FULL + s);
-                const int k0 = (kb0 + j) * BB;
-                mbar_arrive_expect_tx(fb, QB_BYTES);
-                tma_load_4d_nohint(st + QB_K1, &m.k1, fb, 0, k0, h, b);
-                tma_load_4d_nohint(st + QB_K2, &m.k2, fb, 0, k0, hn, b);
-                tma_load_4d_nohint(st + QB_V, &m.v, fb, 0, k0, hv, b);
-                tma_load_4d_nohint(st + QB_V + 8192, &m.v, fb, 64, k0, hv, b);
+                mbar_arrive_expect_tx(bar(B_TILE), QT_STAGE0);
+                tma_load_4d_nohint(sbase + QT_Q1, &m.q1, bar(B_TILE), 0, T.q0, T.h, T.b);
+                tma_load_4d_nohint(sbase + QT_Q2, &m.q2, bar(B_TILE), 0, T.q0, T.hn, T.b);
+                tma_load_4d_nohint(sbase + QT_DD, &m.dd, bar(B_TILE), 0, T.q0, T.h, T.b);
+                tma_load_4d_nohint(sbase + QT_DD + 16384, &m.dd, bar(B_TILE), 64, T.q0, T.h, T.b);
             }
             __syncwarp();
-            loads = j + 1;
+            ++tile_loads;
+            for (int j = 0; j < T.nit; ++j) {
+                const int s = G % QSTAGES;
+                if (G >= QSTAGES &&
+                    !(ok = mbar_wait_warp(bar(B_EMPTY + s), ((G / QSTAGES) - 1) & 1, abort_flag, lim)))
+                    break;
+                if (elect_one()) {
+                    const uint32_t st = sbase + QT_STAGE0 + s * QB_BYTES, fb = bar(B_FULL + s);
+                    const int k0 = (T.kb0 + j) * BB;
+                    mbar_arrive_expect_tx(fb, QB_BYTES);
+                    tma_load_4d_nohint(st + QB_K1, &m.k1, fb, 0, k0, T.h, T.b);
+                    tma_load_4d_nohint(st + QB_K2, &m.k2, fb, 0, k0, T.hn, T.b);
+                    tma_load_4d_nohint(st + QB_V, &m.v, fb, 0, k0, T.hv, T.b);
+                    tma_load_4d_nohint(st + QB_V + 8192, &m.v, fb, 64, k0, T.hv, T.b);
+                }
+                __syncwarp();
+                ++G;
+            }
+            if (!ok) break;
         }
-        bool drained = mbar_wait_drain(bar(B_TILE), 0, lim);
-        for (int k = (loads > QSTAGES ? loads - QSTAGES : 0); k < loads; ++k)
+        // No load of ours may land after the CTA has gone.
+        bool drained = true;
+        if (tile_loads > 0) drained = mbar_wait_drain(bar(B_TILE), (tile_loads - 1) & 1, lim);
+        for (int k = (G > QSTAGES ? G - QSTAGES : 0); k < G; ++k)
             drained &= mbar_wait_drain(bar(B_FULL + k % QSTAGES), (k / QSTAGES) & 1, lim);
         if (!__all_sync(0xffffffffu, drained) && R.lane == 0) *abort_flag = 1;
     } else if (R.score_issuer() || R.acc_issuer()) {
-        auto issue_s = [&](int j) {
-            const uint32_t st = sbase + QT_STAGE0 + (j % QSTAGES) * QB_BYTES;
+        // ------------------------------------------------------------ MMA issuers
+        auto issue_s = [&](int G) {
+            const uint32_t st = sbase + QT_STAGE0 + (G % QSTAGES) * QB_BYTES;
 #pragma unroll
             for (int kk = 0; kk < HD / 16; ++kk)
                 mma_issue_ts(tbase + QM_S1, tbase + QM_AQ1 + 8 * kk, sw128(st + QB_K1 + 32 * kk), Ids<F16QK>::S,
@@ -995,38 +1033,112 @@ __global__ void __launch_bounds__(NT, 1)
             }
             commit_to(bar(B_SFULL));
         };
-        auto issue_acc = [&](int j) {
-            const uint32_t st = sbase + QT_STAGE0 + (j % QSTAGES) * QB_BYTES;
+        auto issue_acc = [&](int G, bool first) {
+            const uint32_t st = sbase + QT_STAGE0 + (G % QSTAGES) * QB_BYTES;
             // dQ_t += dS_t K_t (B: the K block, MN-major).
 #pragma unroll
             for (int kk = 0; kk < BB / 16; ++kk)
                 mma_issue(tbase + QM_DQ1, sw128(sbase + QT_A + QA_DS1 + 32 * kk), sw128(st + QB_K1 + 2048 * kk, 8192),
-                          Ids<F16QK>::DS, j > 0 || kk > 0);
+                          Ids<F16QK>::DS, !first || kk > 0);
 #pragma unroll
             for (int kk = 0; kk < BB / 16; ++kk)
                 mma_issue(tbase + QM_DQ2, sw128(sbase + QT_A + QA_DS2 + 32 * kk), sw128(st + QB_K2 + 2048 * kk, 8192),
-                          Ids<F16QK>::DS, j > 0 || kk > 0);
+                          Ids<F16QK>::DS, !first || kk > 0);
             commit_to(bar(B_AFREE));
-            commit_to(bar(B_EMPTY + j % QSTAGES));
+            commit_to(bar(B_EMPTY + G % QSTAGES));
         };
-        if (R.score_issuer())
-            score_issuer<QSTAGES>(nit, bar(B_AOP), bar(B_FULL), bar(B_SFREE), bar(B_SDRAIN), abort_flag, lim, issue_s,
-                                  R.lane);
-        else
-            acc_issuer(nit, bar(B_AFULL), bar(B_DONE), abort_flag, lim, issue_acc, R.lane);
+        int G = 0, ti = 0;
+        bool ok = true;
+        if (R.score_issuer()) {
+            for (;; ++ti) {
+                const int t = read_tile(ti);
+                if (t < 0) break;
+                const Tile T = tile_of(t);
+                // the tile's Q and dD rows are in TMEM
+                if (!(ok = mbar_wait_warp(bar(B_AOP), ti & 1, abort_flag, lim))) break;
+                for (int j = 0; ok && j < T.nit; ++j, ++G) {
+                    if (!(ok = mbar_wait_warp(bar(B_FULL + G % QSTAGES), (G / QSTAGES) & 1, abort_flag, lim))) break;
+                    if (G > 0 && !(ok = mbar_wait_warp(bar(B_SFREE), (G - 1) & 1, abort_flag, lim))) break;
+                    tc_fence_after();
+                    issue_s(G);
+                }
+                if (!ok) break;
+            }
+            // Nothing of ours may still run on the tensor cores at teardown.
+            commit_to(bar(B_SDRAIN));
+            if (!__all_sync(0xffffffffu, mbar_wait_drain(bar(B_SDRAIN), 0, lim)) && R.lane == 0) *abort_flag = 1;
+        } else {
+            for (;; ++ti) {
+                const int t = read_tile(ti);
+                if (t < 0) break;
+                const Tile T = tile_of(t);
+                for (int j = 0; ok && j < T.nit; ++j, ++G) {
+                    if (!(ok = mbar_wait_warp(bar(B_AFULL), G & 1, abort_flag, lim))) break;
+                    // The tile's first products overwrite the accumulators:
+                    // the previous tile's epilogue must have read them.
+                    if (j == 0 && ti > 0 && !(ok = mbar_wait_warp(bar(B_ACCFREE), (ti - 1) & 1, abort_flag, lim)))
+                        break;
+                    tc_fence_after();
+                    issue_acc(G, j == 0);
+                }
+                if (!ok) break;
+                // DONE completes once every product of the tile has: the
+                // epilogue's signal.
+                commit_to(bar(B_DONE));
+            }
+            // Nothing of ours may still run on the tensor cores at teardown.
+            commit_to(bar(B_ADRAIN));
+            if (!__all_sync(0xffffffffu, mbar_wait_drain(bar(B_ADRAIN), 0, lim)) && R.lane == 0) *abort_flag = 1;
+        }
     } else {
+        // ------------------------------------------------------------ element-wise + epilogue
         const int wg = R.wg(), r = R.row();
         const uint32_t lo = R.lane_off();
-        const int qrow = q0 + r;  // this thread's query
         const float c = p.scale_log2;
-        const float *strow = p.stats + (size_t)(b * p.H + h) * kBwdStats * p.n_pad + qrow;
-        // (stored negated: -lse_1, -lse_2, -Delta_1, -Delta_2, -lambda)
-        const float nlse1 = strow[0], nlse2 = strow[p.n_pad], ndel1 = strow[2 * p.n_pad], ndel2 = strow[3 * p.n_pad];
-        const float nlam = strow[4 * p.n_pad];
-        // The tile's Q_1, Q_2 (warpgroup 0) and dD (warpgroup 1) rows into
-        // TMEM, the A operands of every block's score and dP products.
-        bool ok = mbar_wait_warp(bar(B_TILE), 0, abort_flag, lim), big = false;
-        if (ok) {
+        bool ok = true, big = false;
+        // The finished tile's dQ from TMEM to global memory (after its last
+        // products): warpgroup 0 writes dQ_1, warpgroup 1 dQ_2, rows below N
+        // only; then the accumulators are released to the next tile.
+        auto epilogue = [&](const Tile &T, int ti) -> bool {
+            if (!mbar_wait_warp(bar(B_DONE), ti & 1, abort_flag, lim)) return false;
+            tc_fence_after();
+            const int qrow = T.q0 + r;
+            const bool own = qrow < p.N;
+            const int qr = own ? qrow : 0;
+            float x[64];
+            tmem_row64(tbase + lo + (wg ? QM_DQ2 : QM_DQ1), x);
+            if (own) {
+                if (F16QK) unrotate64(x, qr, p.rope_g);
+                if (wg == 0) {
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dq1) + (size_t)T.b * p.dq1_s[0] +
+                                         (size_t)qr * p.dq1_s[1] + (size_t)T.h * p.dq1_s[2];
+                    put_row<64>(x, p.scale, dst, nullptr);
+                } else {
+                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dq2) + (size_t)T.b * p.dq2_s[0] +
+                                         (size_t)qr * p.dq2_s[1] + (size_t)T.hn * p.dq2_s[2];
+                    float *acc = p.acc_dq2 ? p.acc_dq2 + (((size_t)T.b * p.N + qr) * p.H_N + T.hn) * HD : nullptr;
+                    put_row<64>(x, p.scale, dst, acc);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (R.lane == 0) mbar_arrive(bar(B_ACCFREE));
+            return true;
+        };
+        int G = 0, ti = 0;
+        Tile prev{};
+        for (;; ++ti) {
+            const int t = read_tile(ti);
+            if (t < 0) break;
+            const Tile T = tile_of(t);
+            const int qrow = T.q0 + r;  // this thread's query
+            const float *strow = p.stats + (size_t)(T.b * p.H + T.h) * kBwdStats * p.n_pad + qrow;
+            // (stored negated: -lse_1, -lse_2, -Delta_1, -Delta_2, -lambda)
+            const float nlse1 = strow[0], nlse2 = strow[p.n_pad], ndel1 = strow[2 * p.n_pad],
+                        ndel2 = strow[3 * p.n_pad], nlam = strow[4 * p.n_pad];
+            // The tile's Q_1, Q_2 (warpgroup 0) and dD (warpgroup 1) rows into
+            // TMEM, the A operands of every block's score and dP products.
+            if (!(ok = mbar_wait_warp(bar(B_TILE), ti & 1, abort_flag, lim))) break;
             if (wg == 0) {
                 tile_row_to_tmem(sbase + QT_Q1, r, tbase + lo + QM_AQ1);
                 tile_row_to_tmem(sbase + QT_Q2, r, tbase + lo + QM_AQ2);
@@ -1038,85 +1150,71 @@ __global__ void __launch_bounds__(NT, 1)
             tc_fence_before();
             __syncwarp();
             if (R.lane == 0) mbar_arrive(bar(B_AOP));
-        }
-        for (int j = 0; ok && j < nit; ++j) {
-            if (!(ok = mbar_wait_warp(bar(B_SFULL), j & 1, abort_flag, lim))) break;
-            tc_fence_after();
-            uint32_t s1[32], s2[32], dp[32];
-            tmem_ld32(tbase + lo + QM_S1 + 32 * wg, s1);
-            tmem_ld32(tbase + lo + QM_S2 + 32 * wg, s2);
-            tmem_ld32(tbase + lo + QM_DP + 32 * wg, dp);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (R.lane == 0) mbar_arrive(bar(B_SFREE));
-            const int kb = (kb0 + j) * BB + 32 * wg;  // this warpgroup's 32 keys of the block
-            const bool mask = (p.causal && kb + 31 > q0) || (p.window > 0 && q0 + BT - 1 - kb >= p.window);
-            uint32_t d1p[16], d2p[16];
+            // The previous tile's epilogue, while this tile's first score
+            // products run.
+            if (ti > 0 && !(ok = epilogue(prev, ti - 1))) break;
             const float2 c2 = make_float2(c, c), nl1 = make_float2(nlse1, nlse1), nl2 = make_float2(nlse2, nlse2);
             const float2 nd1 = make_float2(ndel1, ndel1), nd2 = make_float2(ndel2, ndel2), nlm = make_float2(nlam, nlam);
+            for (int j = 0; ok && j < T.nit; ++j, ++G) {
+                if (!(ok = mbar_wait_warp(bar(B_SFULL), G & 1, abort_flag, lim))) break;
+                tc_fence_after();
+                uint32_t s1[32], s2[32], dp[32];
+                tmem_ld32(tbase + lo + QM_S1 + 32 * wg, s1);
+                tmem_ld32(tbase + lo + QM_S2 + 32 * wg, s2);
+                tmem_ld32(tbase + lo + QM_DP + 32 * wg, dp);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (R.lane == 0) mbar_arrive(bar(B_SFREE));
+                const int kb = (T.kb0 + j) * BB + 32 * wg;  // this warpgroup's 32 keys of the block
+                const bool mask = (p.causal && kb + 31 > T.q0) || (p.window > 0 && T.q0 + BT - 1 - kb >= p.window);
+                uint32_t d1p[16], d2p[16];
 #pragma unroll
-            for (int i = 0; i < 32; i += 2) {  // two keys at a time, in packed arithmetic
-                const float2 x1 = ffma2(make_float2(__uint_as_float(s1[i]), __uint_as_float(s1[i + 1])), c2, nl1);
-                const float2 x2 = ffma2(make_float2(__uint_as_float(s2[i]), __uint_as_float(s2[i + 1])), c2, nl2);
-                float2 p1, p2;
-                if ((BWD_SOFT_EXP_MASK >> ((i >> 1) & 7)) & 1u) {
-                    p1 = exp2_soft2(x1);
-                    p2 = exp2_soft2(x2);
-                } else {
-                    p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
-                    p2 = make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
-                }
-                if (mask) {
+                for (int i = 0; i < 32; i += 2) {  // two keys at a time, in packed arithmetic
+                    const float2 x1 = ffma2(make_float2(__uint_as_float(s1[i]), __uint_as_float(s1[i + 1])), c2, nl1);
+                    const float2 x2 = ffma2(make_float2(__uint_as_float(s2[i]), __uint_as_float(s2[i + 1])), c2, nl2);
+                    float2 p1, p2;
+                    if ((BWD_SOFT_EXP_MASK >> ((i >> 1) & 7)) & 1u) {
+                        p1 = exp2_soft2(x1);
+                        p2 = exp2_soft2(x2);
+                    } else {
+                        p1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+                        p2 = make_float2(ex2_approx(x2.x), ex2_approx(x2.y));
+                    }
+                    if (mask) {
 #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int key = kb + i + u;
-                        const bool vis = (!p.causal || key <= qrow) && (p.window <= 0 || qrow - key < p.window);
-                        if (!vis) {
-                            if (u) p1.y = p2.y = 0.f;
-                            else p1.x = p2.x = 0.f;
+                        for (int u = 0; u < 2; ++u) {
+                            const int key = kb + i + u;
+                            const bool vis = (!p.causal || key <= qrow) && (p.window <= 0 || qrow - key < p.window);
+                            if (!vis) {
+                                if (u) p1.y = p2.y = 0.f;
+                                else p1.x = p2.x = 0.f;
+                            }
                         }
                     }
+                    const float2 g = make_float2(__uint_as_float(dp[i]), __uint_as_float(dp[i + 1]));
+                    const float2 v1 = fmul2(p1, fadd2(g, nd1));        // P_1 (dP - Delta_1)
+                    const float2 v2 = fmul2(p2, ffma2(nlm, g, nd2));   // P_2 (-lambda dP - Delta_2)
+                    if (F16QK)
+                        big |= !(fabsf(v1.x) <= 65504.0f && fabsf(v1.y) <= 65504.0f && fabsf(v2.x) <= 65504.0f &&
+                                 fabsf(v2.y) <= 65504.0f);
+                    d1p[i / 2] = pack_ds(v1.x, v1.y, F16QK);
+                    d2p[i / 2] = pack_ds(v2.x, v2.y, F16QK);
                 }
-                const float2 g = make_float2(__uint_as_float(dp[i]), __uint_as_float(dp[i + 1]));
-                const float2 v1 = fmul2(p1, fadd2(g, nd1));        // P_1 (dP - Delta_1)
-                const float2 v2 = fmul2(p2, ffma2(nlm, g, nd2));   // P_2 (-lambda dP - Delta_2)
-                if (F16QK)
-                    big |= !(fabsf(v1.x) <= 65504.0f && fabsf(v1.y) <= 65504.0f && fabsf(v2.x) <= 65504.0f &&
-                             fabsf(v2.y) <= 65504.0f);
-                d1p[i / 2] = pack_ds(v1.x, v1.y, F16QK);
-                d2p[i / 2] = pack_ds(v2.x, v2.y, F16QK);
+                // The previous block's accumulating products (of this tile or
+                // the one before) must have read the A operands.
+                if (G > 0 && !(ok = mbar_wait_warp(bar(B_AFREE), (G - 1) & 1, abort_flag, lim))) break;
+                st_operand_half(sbase + QT_A + QA_DS1, r, wg, d1p);
+                st_operand_half(sbase + QT_A + QA_DS2, r, wg, d2p);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (R.lane == 0) mbar_arrive(bar(B_AFULL));
             }
-            if (j > 0 && !(ok = mbar_wait_warp(bar(B_AFREE), (j - 1) & 1, abort_flag, lim))) break;
-            st_operand_half(sbase + QT_A + QA_DS1, r, wg, d1p);
-            st_operand_half(sbase + QT_A + QA_DS2, r, wg, d2p);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (R.lane == 0) mbar_arrive(bar(B_AFULL));
+            if (!ok) break;
+            prev = T;
         }
+        if (ok && ti > 0) ok = epilogue(prev, ti - 1);
         if (big) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
-        if (ok) ok = mbar_wait_warp(bar(B_DONE), 0, abort_flag, lim);
-        if (ok) {
-            // Warpgroup 0 writes dQ_1, warpgroup 1 dQ_2; rows below N only.
-            tc_fence_after();
-            const bool own = qrow < p.N;
-            const int qr = own ? qrow : 0;
-            float x[64];
-            tmem_row64(tbase + lo + (wg ? QM_DQ2 : QM_DQ1), x);
-            if (own) {
-                if (F16QK) unrotate64(x, qr, p.rope_g);
-                if (wg == 0) {
-                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dq1) + (size_t)b * p.dq1_s[0] +
-                                         (size_t)qr * p.dq1_s[1] + (size_t)h * p.dq1_s[2];
-                    put_row<64>(x, p.scale, dst, nullptr);
-                } else {
-                    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(p.dq2) + (size_t)b * p.dq2_s[0] +
-                                         (size_t)qr * p.dq2_s[1] + (size_t)hn * p.dq2_s[2];
-                    float *acc = p.acc_dq2 ? p.acc_dq2 + (((size_t)b * p.N + qr) * p.H_N + hn) * HD : nullptr;
-                    put_row<64>(x, p.scale, dst, acc);
-                }
-            }
-        }
     }
     tc_fence_before();
     __syncthreads();
@@ -1206,7 +1304,7 @@ cudaError_t launch_bwd(const BwdKeyMaps &km, const BwdQueryMaps &qm, const BwdPa
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (ev.start) cudaEventRecord(ev.start, stream);
-    // The key-tile kernel is persistent: one CTA per SM (or per tile, when
+    // Both tile kernels are persistent: one CTA per SM (or per tile, when
     // there are fewer).
     const int sms = device_sm_count();
     const int key_grid = tiles < sms ? tiles : sms;
@@ -1218,9 +1316,9 @@ cudaError_t launch_bwd(const BwdKeyMaps &km, const BwdQueryMaps &qm, const BwdPa
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.qk_f16)
-        bwd_query_kernel<true><<<tiles, NT, QT_SMEM, stream>>>(qm, p);
+        bwd_query_kernel<true><<<key_grid, NT, QT_SMEM, stream>>>(qm, p);
     else
-        bwd_query_kernel<false><<<tiles, NT, QT_SMEM, stream>>>(qm, p);
+        bwd_query_kernel<false><<<key_grid, NT, QT_SMEM, stream>>>(qm, p);
     ++*launches;
     if (ev.stop) cudaEventRecord(ev.stop, stream);
     e = cudaGetLastError();

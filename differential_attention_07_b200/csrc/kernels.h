@@ -125,7 +125,7 @@ struct BwdParams {
     int64_t dg_sb, dg_sn, dg_sh;
     int qk_f16;           // Q/K operands are the rotated fp16 copies (rotary embedding)
     double rope_g[32];    // turns per token of pair c: theta^(-2c/64) / (2 pi)
-    int *tile_counter;    // key-tile work counter, zeroed by the staging kernel
+    int *tile_counter;    // two work counters (key tiles, query tiles), zeroed by the staging kernel
     int32_t *dev_status;
     uint64_t timeout_ns;
 };
