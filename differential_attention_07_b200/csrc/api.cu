@@ -405,8 +405,12 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
                  qk_stride[1][0], qk_stride[1][1], qk_stride[1][2], da::kPrefillKeyRows) &&
         make_map(&mk2, qkt, qk[3], 64, a->N, HN, a->B,
                  qk_stride[3][0], qk_stride[3][1], qk_stride[3][2], da::kPrefillKeyRows) &&
-        make_map(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws, 128, a->N, HV, a->B, a->N * HV * 128,
-                 HV * 128, 128, da::kPrefillKeyRows) &&
+        (a->window > 0
+             // the window kernel reads the caller's bf16 V and converts each step itself
+             ? make_map(&mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->v, 128, a->N, HV, a->B, a->v_stride[0],
+                        a->v_stride[1], a->v_stride[2], da::kPrefillKeyRows)
+             : make_map(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, ws, 128, a->N, HV, a->B, a->N * HV * 128,
+                        HV * 128, 128, da::kPrefillKeyRows)) &&
         make_map(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->out, 128, a->N, a->H, a->B,
                  a->out_stride[0], a->out_stride[1], a->out_stride[2], da::kPrefillOutRows);
     if (!ok) {
@@ -425,7 +429,7 @@ diffattn_status run_fwd(const diffattn_fwd_args *a, void *ws, size_t ws_bytes, v
     cudaError_t e = da::launch_v_to_f16(a->v, a->v_stride[0], a->v_stride[1], a->v_stride[2], ws,
                                         (int)a->B, (int)a->N, (int)HV, a->dev_status,
                                         tile_counter, noise_ready, paired ? noise_tiles(a) : 0, rope,
-                                        sms, s, &launches);
+                                        sms, s, &launches, a->window <= 0);
     if (e != cudaSuccess) return cuda_status(e);
 
     da::PrefillParams p{};

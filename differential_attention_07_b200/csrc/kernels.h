@@ -87,10 +87,12 @@ struct RopeStage {
 
 // `zero`/`n_zero`: ints the staging kernel also clears (the grouped pairs'
 // ready counts), or nullptr / 0.  `sm_count`: SMs of the device (grid size).
+// `stage_v` false: no fp16 copy of V (the sliding-window prefill converts
+// each V step itself); the counters, `zero` and RoPE are done as usual.
 cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, void *dst, int B,
                             int N, int H_V, int32_t *dev_status, int *tile_counter,
                             int *zero, int64_t n_zero, const RopeStage &rope, int sm_count,
-                            cudaStream_t stream, int *launches);
+                            cudaStream_t stream, int *launches, bool stage_v = true);
 
 // SM count of the current device, looked up once per device (thread-safe);
 // 148 (a B200) when no device is visible, for host-only size queries.

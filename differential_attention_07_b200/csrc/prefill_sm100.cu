@@ -93,7 +93,8 @@ enum : int {
     B_ITEM = B_STAT + 2,         // [ITEM_SLOTS] work item published (1 arrival)
     B_ITEMFREE = B_ITEM + 4,     // [ITEM_SLOTS] work item read by all 10 reader warps
     B_AN = B_ITEMFREE + 4,       // [4 epilogue warps] the warp's A_N rows landed (bulk-copy bytes)
-    NBARS = B_AN + 4
+    B_VCVT = B_AN + 4,           // [STAGES] window kernels: the step's V converted to fp16 (1 arrival)
+    NBARS = B_VCVT + STAGES
 };
 // S and P barriers come one per S buffer: a softmax may run two steps ahead
 // of its MMA warp's wait, and with one P barrier per map the second arrival
@@ -106,6 +107,7 @@ constexpr uint32_t OFF_TMEM_PTR = OFF_BARS + NBARS * 8;
 constexpr uint32_t OFF_ABORT = OFF_TMEM_PTR + 4;
 constexpr int ITEM_SLOTS = 4;
 constexpr int ITEM_READERS = 14;                         // 2 MMA, 8 softmax and 4 epilogue warps
+                                                         // (and the V converter under a window)
 constexpr uint32_t ITEM_BYTES = 48;                      // one published work item: three int4
 constexpr uint32_t OFF_ITEM = (OFF_ABORT + 4 + 15) & ~15u;  // [ITEM_SLOTS] work-item ring
 // float [2 tile parities][l1, l2][128]: the softmax warps' row sums
@@ -441,9 +443,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_init(bar(B_STAT), 8);    // one arrival per softmax warp
         mbar_init(bar(B_STAT + 1), 8);
         for (int i = 0; i < 4; ++i) mbar_init(bar(B_AN + i), 1);
+        if (WINDOW)
+            for (int s = 0; s < STAGES; ++s) mbar_init(bar(B_VCVT + s), 1);
         for (int i = 0; i < ITEM_SLOTS; ++i) {
             mbar_init(bar(B_ITEM + i), 1);
-            mbar_init(bar(B_ITEMFREE + i), ITEM_READERS);
+            mbar_init(bar(B_ITEMFREE + i), ITEM_READERS + (WINDOW ? 1 : 0));
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -652,6 +656,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (j == 0 && tiles > 0 &&
                     !(ok = mbar_wait_warp(bar(B_OFREE), (tiles - 1) & 1, abort_flag, lim)))
                     break;
+                // Under a window V arrives in bf16 and warp 3 converts it.
+                if (WINDOW && !(ok = mbar_wait_warp(bar(B_VCVT + s), (gg / STAGES) & 1, abort_flag, lim)))
+                    break;
                 tc_fence_after();
                 issue_pv(s, buf, j > 0);
                 commit(bar_pv);
@@ -674,6 +681,47 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         commit(bar(B_PV + t));
         const bool drained = mbar_wait_drain(bar(B_PV + t), g & 1, lim);
         if (!__all_sync(0xffffffffu, drained) && lane == 0) *abort_flag = 1;
+      } else if (WINDOW) {
+        // ------------------------------------------------------------ V converter (window kernels)
+        // A window tile has only a few key steps, so each V step is used by
+        // about two tiles: converting it here, once per use, costs less than
+        // a separate pass over all of V.  Each landed stage's V (bf16, in
+        // the 128-byte swizzle) is rewritten in place as fp16 -- the swizzle
+        // moves 16-byte chunks, so the layout is unchanged -- and released
+        // to the P.V MMAs.
+        int g = 0;
+        bool ok = true, overflow = false;
+        for (int tiles = 0;; ++tiles) {
+            Item it;
+            if (!read_item(tiles, it)) break;
+            for (int j = 0; j < it.nkv; ++j, ++g) {
+                const int s = g % STAGES;
+                if (!(ok = mbar_wait_warp(bar_full(s), (g / STAGES) & 1, abort_flag, lim))) break;
+                const uint32_t va = sbase + OFF_STAGE0 + s * STAGE_BYTES + 2 * K_BYTES;
+                float big = 0.0f;
+#pragma unroll 4
+                for (int k = 0; k < int(V_BYTES / 16 / 32); ++k) {
+                    const uint32_t a = va + 16u * (32u * k + lane);
+                    const uint4 x = ld_shared_v4(a);
+                    const uint32_t in[4] = {x.x, x.y, x.z, x.w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float lo = __uint_as_float(in[e] << 16), hi = __uint_as_float(in[e] & 0xffff0000u);
+                        big = fmaxf(big, fmaxf(fabsf(lo), fabsf(hi)));
+                        o[e] = pack_half2(lo, hi);
+                    }
+                    st_shared_v4(a, o[0], o[1], o[2], o[3]);
+                }
+                overflow |= big > 65504.0f;
+                // the generic-proxy writes, visible to the tensor cores' reads
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_VCVT + s));
+            }
+            if (!ok) break;
+        }
+        if (__any_sync(0xffffffffu, overflow) && lane == 0) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
       }
     } else if (warp < 12) {
         regs_increase<REGS_SOFTMAX>();
@@ -1103,7 +1151,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb, int64_t sn,
                                 int64_t sh, __half *__restrict__ dst, int B, int N, int H_V,
                                 int32_t *dev_status, int *tile_counter, int *zero, int64_t n_zero,
-                                const RopeStage rope)
+                                const RopeStage rope, int stage_v)
 {
     // The prefill launch that follows may become resident and run its
     // prologue now; it waits for this kernel to finish before reading.
@@ -1120,7 +1168,7 @@ __global__ void v_to_f16_kernel(const __nv_bfloat16 *__restrict__ v, int64_t sb,
     // array, so its chunk i needs no index arithmetic, and each thread keeps
     // four loads in flight; otherwise chunk i is decomposed into (b, n, head,
     // column) -- 64-bit divisions that made the pass compute-bound.
-    const int64_t total = (int64_t)B * N * H_V * (HDV / 8);
+    const int64_t total = stage_v ? (int64_t)B * N * H_V * (HDV / 8) : 0;
     const bool dense = sh == HDV && sn == (int64_t)H_V * HDV && sb == (int64_t)N * H_V * HDV;
     bool overflow = false;
     auto to_f16 = [&](const uint4 src) {
@@ -1286,16 +1334,19 @@ cudaError_t launch_prefill(const CUtensorMap &q1, const CUtensorMap &q2, const C
 cudaError_t launch_v_to_f16(const void *v, int64_t sb, int64_t sn, int64_t sh, void *dst, int B,
                             int N, int H_V, int32_t *dev_status, int *tile_counter,
                             int *zero, int64_t n_zero, const RopeStage &rope, int sm_count,
-                            cudaStream_t stream, int *launches)
+                            cudaStream_t stream, int *launches, bool stage_v)
 {
     const int64_t total = (int64_t)B * N * H_V * (HDV / 8);
     if (total == 0) return cudaSuccess;  // nothing to stage; the prefill is skipped too
     const int threads = 256;
-    int blocks = (int)((total + threads - 1) / threads);
+    // Without the V copy (and without RoPE) only the counters are cleared.
+    const int64_t work = stage_v || rope.enabled ? total : (n_zero > 0 ? n_zero : 1);
+    int blocks = (int)((work + threads - 1) / threads);
     if (blocks > sm_count * 8) blocks = sm_count * 8;  // resident at once (2048 threads per SM); grid-stride beyond
     v_to_f16_kernel<<<blocks, threads, 0, stream>>>(static_cast<const __nv_bfloat16 *>(v), sb, sn,
                                                     sh, static_cast<__half *>(dst), B, N, H_V,
-                                                    dev_status, tile_counter, zero, n_zero, rope);
+                                                    dev_status, tile_counter, zero, n_zero, rope,
+                                                    stage_v ? 1 : 0);
     ++*launches;
     return cudaGetLastError();
 }
