@@ -67,18 +67,22 @@ def test_many_one_token_sequences(cuda_ok):
     _check(y, ref)
 
 
-def test_v_beyond_fp16_range_is_reported(cuda_ok):
+@pytest.mark.parametrize("window", [0, 64])
+def test_v_beyond_fp16_range_is_reported(cuda_ok, window):
     """bf16 can hold values the fp16 P.V product cannot: the staging kernel
-    reports DIFFATTN_ERR_UNSUPPORTED (2) in the status word; nothing faults
-    and the next call is fine."""
-    x = {k: v.cuda() for k, v in inputs.prefill_inputs(1, 128, 1, seed=5).items()}
-    x["v"][0, 7, 0, 3] = 70000.0
+    (or, under a sliding window, the kernel's own V conversion) reports
+    DIFFATTN_ERR_UNSUPPORTED (2) in the status word; nothing faults and the
+    next call is fine."""
+    x = {k: v.cuda() for k, v in inputs.prefill_inputs(1, 300, 1, seed=5).items()}
+    x["v"][0, 207, 0, 3] = 70000.0
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    ops.diffattn_fwd(x["q1"], x["q2"], x["k1"], x["k2"], x["v"], x["lam"], x["gain"], dev_status=st)
+    ops.diffattn_fwd(x["q1"], x["q2"], x["k1"], x["k2"], x["v"], x["lam"], x["gain"], dev_status=st,
+                     window=window)
     torch.cuda.synchronize()
     assert st.item() == 2
-    x["v"][0, 7, 0, 3] = 1.0
+    x["v"][0, 207, 0, 3] = 1.0
     st.zero_()
-    ops.diffattn_fwd(x["q1"], x["q2"], x["k1"], x["k2"], x["v"], x["lam"], x["gain"], dev_status=st)
+    ops.diffattn_fwd(x["q1"], x["q2"], x["k1"], x["k2"], x["v"], x["lam"], x["gain"], dev_status=st,
+                     window=window)
     torch.cuda.synchronize()
     assert st.item() == 0
