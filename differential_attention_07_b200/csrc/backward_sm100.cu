@@ -114,23 +114,22 @@ constexpr uint32_t KM_DV = 0, KM_DK1 = 128, KM_DK2 = 192, KM_S1 = 256, KM_S2 = 3
 // ---------------------------------------------------------------- query-tile kernel
 // Shared memory: the tile's Q_1, Q_2 ([128][64]) and dD (fp16 [128][128] as
 // two halves); QSTAGES block stages of K_1, K_2 ([64][64]) and fp16 V
-// ([64][128] as two halves); the A operands dS_1, dS_2 ([128 queries][64
-// keys]).
+// ([64][128] as two halves).
 constexpr uint32_t QT_Q1 = 0, QT_Q2 = 16384, QT_DD = 32768, QT_STAGE0 = 65536;
 constexpr uint32_t QB_K1 = 0, QB_K2 = 8192, QB_V = 16384, QB_BYTES = 32768;
-constexpr uint32_t QT_A = QT_STAGE0 + QSTAGES * QB_BYTES;
-constexpr uint32_t QA_DS1 = 0, QA_DS2 = 16384;
-constexpr uint32_t QT_BARS = QT_A + 2 * 16384;
+constexpr uint32_t QT_BARS = QT_STAGE0 + QSTAGES * QB_BYTES;
 constexpr uint32_t QT_SMEM = QT_BARS + 8 * NBARS + 32;  // + TMEM address, abort flag, 4-slot tile ring
 // TMEM columns: dQ_1, dQ_2 accumulators, then S_1, S_2, dP, then the tile's
 // Q_1, Q_2 and dD (16-bit pairs) as the A operands of the score and dP
 // products, so that every block's products read only K and V from shared
-// memory (the kernel is bound by shared-memory bandwidth).
+// memory (the kernel is bound by shared-memory bandwidth), then the block's
+// dS_1, dS_2 (16-bit pairs) as the A operands of the dQ products, written
+// by the element-wise warps with TMEM stores.
 constexpr uint32_t QM_DQ1 = 0, QM_DQ2 = 64, QM_S1 = 128, QM_S2 = 192, QM_DP = 256, QM_AQ1 = 320,
-                   QM_AQ2 = 352, QM_ADD = 384;
+                   QM_AQ2 = 352, QM_ADD = 384, QM_ADS1 = 448, QM_ADS2 = 480;
 
 static_assert(KT_SMEM <= 232448 && QT_SMEM <= 232448, "shared memory budget");
-static_assert(KT_A % 1024 == 0 && QT_A % 1024 == 0 && KB_BYTES % 1024 == 0, "SW128 tiles are 1 KB aligned");
+static_assert(KT_A % 1024 == 0 && QT_STAGE0 % 1024 == 0 && KB_BYTES % 1024 == 0, "SW128 tiles are 1 KB aligned");
 static_assert(KT_SMEM > 116 * 1024 && QT_SMEM > 116 * 1024, "one CTA per SM owns the 512 TMEM columns");
 
 // Instruction descriptors (fp32 accumulate).  F16QK: Q/K are the rotated
@@ -1035,15 +1034,15 @@ __global__ void __launch_bounds__(NT, 1)
         };
         auto issue_acc = [&](int G, bool first) {
             const uint32_t st = sbase + QT_STAGE0 + (G % QSTAGES) * QB_BYTES;
-            // dQ_t += dS_t K_t (B: the K block, MN-major).
+            // dQ_t += dS_t K_t (A: dS_t in TMEM; B: the K block, MN-major).
 #pragma unroll
             for (int kk = 0; kk < BB / 16; ++kk)
-                mma_issue(tbase + QM_DQ1, sw128(sbase + QT_A + QA_DS1 + 32 * kk), sw128(st + QB_K1 + 2048 * kk, 8192),
-                          Ids<F16QK>::DS, !first || kk > 0);
+                mma_issue_ts(tbase + QM_DQ1, tbase + QM_ADS1 + 8 * kk, sw128(st + QB_K1 + 2048 * kk, 8192),
+                             Ids<F16QK>::DS, !first || kk > 0);
 #pragma unroll
             for (int kk = 0; kk < BB / 16; ++kk)
-                mma_issue(tbase + QM_DQ2, sw128(sbase + QT_A + QA_DS2 + 32 * kk), sw128(st + QB_K2 + 2048 * kk, 8192),
-                          Ids<F16QK>::DS, !first || kk > 0);
+                mma_issue_ts(tbase + QM_DQ2, tbase + QM_ADS2 + 8 * kk, sw128(st + QB_K2 + 2048 * kk, 8192),
+                             Ids<F16QK>::DS, !first || kk > 0);
             commit_to(bar(B_AFREE));
             commit_to(bar(B_EMPTY + G % QSTAGES));
         };
@@ -1204,9 +1203,11 @@ __global__ void __launch_bounds__(NT, 1)
                 // The previous block's accumulating products (of this tile or
                 // the one before) must have read the A operands.
                 if (G > 0 && !(ok = mbar_wait_warp(bar(B_AFREE), (G - 1) & 1, abort_flag, lim))) break;
-                st_operand_half(sbase + QT_A + QA_DS1, r, wg, d1p);
-                st_operand_half(sbase + QT_A + QA_DS2, r, wg, d2p);
-                fence_proxy_async_smem();
+                // this warpgroup's 32 keys: TMEM columns [16 wg, 16 wg + 16) of each operand
+                tmem_st16(tbase + lo + QM_ADS1 + 16 * wg, d1p);
+                tmem_st16(tbase + lo + QM_ADS2 + 16 * wg, d2p);
+                tmem_wait_st();
+                tc_fence_before();
                 __syncwarp();
                 if (R.lane == 0) mbar_arrive(bar(B_AFULL));
             }
