@@ -254,20 +254,26 @@ __device__ __forceinline__ void tmem_row64(uint32_t taddr, float (&x)[64])
 }
 
 // ---------------------------------------------------------------- 1. row preparation
-// One CTA per (batch entry, head, 128-row query tile), one thread per row.
-// Dynamic shared memory [128][129] fp32 holds the per-row dgain terms when
-// dgain is requested (and the norm applied), so that one thread per column
-// sums them.
-__global__ void __launch_bounds__(128)
+// Four threads per row (thread q of a row takes columns [32 q, 32 q + 32):
+// 8 chunks of 4 fp32 of A_1 and of A_2, 32 of dY), 64 rows per CTA: a
+// quarter row of A_1, A_2 fits in registers, so both passes (the norm's
+// sums, then dD) read the saved state once; the row sums combine the four
+// quarters with two shuffles.  In a warp, 8 rows x 4 quarters: each load
+// instruction reads 8 consecutive rows of 4 chunks of the chunk-major
+// state, four full 128-byte lines.  Dynamic shared memory [64][129] fp32
+// holds the per-row dgain terms when dgain is requested (and the norm
+// applied), summed per column by threads 0-127.
+constexpr int PREP_THREADS = 256, PREP_ROWS = PREP_THREADS / 4;
+constexpr int PREP_RED_BYTES = PREP_ROWS * (HDV + 1) * 4;
+__global__ void __launch_bounds__(PREP_THREADS, 2)
     bwd_prep_kernel(const BwdParams p)
 {
-    // dgain reduction: a group of 32 columns of every row ([128][33] floats,
-    // padded against bank conflicts), then per-warp partial column sums.
     extern __shared__ float red[];
-    __shared__ float warp_sum[4];
-    __shared__ float col_part[4][32];
-    const int qt = blockIdx.x % p.num_qt, h = (blockIdx.x / p.num_qt) % p.H, b = blockIdx.x / (p.num_qt * p.H);
-    const int r = threadIdx.x, row = qt * BT + r;
+    __shared__ float warp_sum[PREP_THREADS / 32];
+    const int part = blockIdx.x % (BT / PREP_ROWS), t = blockIdx.x / (BT / PREP_ROWS);
+    const int qt = t % p.num_qt, h = (t / p.num_qt) % p.H, b = t / (p.num_qt * p.H);
+    const int q = threadIdx.x & 3, rr = threadIdx.x >> 2;  // column quarter, row of the CTA
+    const int r = PREP_ROWS * part + rr, row = qt * BT + r;   // row of the tile, of the sequence
     const bool valid = row < p.N;
     const int rowc = valid ? row : 0;
     const float *tile = p.save + ((size_t)(b * p.H + h) * p.num_qt + qt) * kSaveTileFloats;
@@ -277,62 +283,71 @@ __global__ void __launch_bounds__(128)
     const float lam = p.lam_logits ? logistic_fast(ll) : p.lambda[h];
     const float4 *g4p = p.gain ? reinterpret_cast<const float4 *>(p.gain + (size_t)h * HDV) : nullptr;
     const __nv_bfloat16 *dy = static_cast<const __nv_bfloat16 *>(p.dout) + (size_t)b * p.do_sb +
-                              (size_t)rowc * p.do_sn + (size_t)h * p.do_sh;
+                              (size_t)rowc * p.do_sn + (size_t)h * p.do_sh + 32 * q;
     const __nv_bfloat16 *gl = p.gate ? static_cast<const __nv_bfloat16 *>(p.gate) + (size_t)b * p.gate_sb +
-                                           (size_t)rowc * p.gate_sn + (size_t)h * p.gate_sh
+                                           (size_t)rowc * p.gate_sn + (size_t)h * p.gate_sh + 32 * q
                                      : nullptr;
     const bool want_dgain = p.apply_norm && p.dgain;
 
-    // 8 columns (8 c8 .. 8 c8 + 7) of a bf16 row: one 16-byte load.
-    auto load8 = [](const __nv_bfloat16 *src, int c8, float (&y)[8]) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(src + 8 * c8);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    // This thread's quarter row: A_1, A_2 (8 chunks each) and dY, the gate
+    // logits (bf16, packed), all loaded at once.
+    float4 a1[8], a2[8];
+    uint4 dyu[4], glu[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            y[2 * k] = __uint_as_float(w[k] << 16);
-            y[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+    for (int k = 0; k < 8; ++k) a1[k] = a2[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) dyu[k] = glu[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (valid) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            a1[k] = a1p[(8 * q + k) * BT];
+            a2[k] = a2p[(8 * q + k) * BT];
         }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) dyu[k] = *reinterpret_cast<const uint4 *>(dy + 8 * k);
+        if (gl) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) glu[k] = *reinterpret_cast<const uint4 *>(gl + 8 * k);
+        }
+    }
+    // Column i (of the quarter) of a packed bf16 quarter row.
+    auto col = [](const uint4 (&u)[4], int i) {
+        const uint4 x = u[i >> 3];
+        const int e = (i >> 1) & 3;
+        const uint32_t w = e == 0 ? x.x : e == 1 ? x.y : e == 2 ? x.z : x.w;
+        return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
+    };
+    // dYn = dY sigma(G) of column i (the gate is the forward's last step), and sigma(G)
+    auto dyn = [&](int i, float &sgv) {
+        sgv = gl ? logistic_fast(col(glu, i)) : 1.0f;
+        return col(dyu, i) * sgv;
     };
     auto gain4 = [&](int c) { return g4p ? __ldg(g4p + c) : make_float4(1.f, 1.f, 1.f, 1.f); };
-    // dYn = dY sigma(G) (the gate is the forward's last step), and sigma(G)
-    auto dyn8 = [&](int c8, float (&y)[8], float (&sg)[8]) {
-        load8(dy, c8, y);
-        if (gl) {
-            float g[8];
-            load8(gl, c8, g);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                sg[e] = logistic_fast(g[e]);
-                y[e] *= sg[e];
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) sg[e] = 1.0f;
-        }
+    // the row's sum of the four quarters' values (lanes 4 i .. 4 i + 3 of a warp)
+    auto row_sum = [](float x) {
+        x += __shfl_xor_sync(0xffffffffu, x, 1);
+        return x + __shfl_xor_sync(0xffffffffu, x, 2);
     };
 
-    // Pass 1: sum of squares of D and sum_c dYn gain D, 8 columns (two float4
-    // chunks of A_1, A_2) at a time.
+    // Pass 1: sum of squares of D and sum_c dYn gain D.
     float ss = 0.f, tg = 0.f;
-    if (valid && p.apply_norm) {
-#pragma unroll 2
-        for (int c8 = 0; c8 < 16; ++c8) {
-            float y[8], sg[8];
-            dyn8(c8, y, sg);
+    if (p.apply_norm) {
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int c = 2 * c8 + hh;
-                const float4 a1 = a1p[c * BT], a2 = a2p[c * BT], g = gain4(c);
-                const float d[4] = {fmaf(-lam, a2.x, a1.x), fmaf(-lam, a2.y, a1.y), fmaf(-lam, a2.z, a1.z),
-                                    fmaf(-lam, a2.w, a1.w)};
-                const float gg[4] = {g.x, g.y, g.z, g.w};
+        for (int k = 0; k < 8; ++k) {
+            const float4 g = gain4(8 * q + k);
+            const float av1[4] = {a1[k].x, a1[k].y, a1[k].z, a1[k].w}, av2[4] = {a2[k].x, a2[k].y, a2[k].z, a2[k].w};
+            const float gg[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    ss = fmaf(d[e], d[e], ss);
-                    tg = fmaf(gg[e] * y[4 * hh + e], d[e], tg);
-                }
+            for (int e = 0; e < 4; ++e) {
+                const float d = fmaf(-lam, av2[e], av1[e]);
+                float sgv;
+                const float yv = dyn(4 * k + e, sgv);
+                ss = fmaf(d, d, ss);
+                tg = fmaf(gg[e] * yv, d, tg);
             }
         }
+        ss = row_sum(ss);
+        tg = row_sum(tg);
     }
     const float rn = p.apply_norm ? 1.0f / sqrtf(ss * (1.0f / HDV) + p.eps) : 1.0f;
     const float coef = rn * rn * rn * (1.0f / HDV) * tg;
@@ -345,72 +360,49 @@ __global__ void __launch_bounds__(128)
     // in the gradient).  dlambda takes dD itself.
     float delta1 = 0.f, dot2 = 0.f, dot2h = 0.f;
     bool bad = false;
-    __half *ddrow = static_cast<__half *>(p.dd) + (((size_t)b * p.N + rowc) * p.H + h) * HDV;
-    __nv_bfloat16 *dgrow = p.dgate ? static_cast<__nv_bfloat16 *>(p.dgate) + (size_t)b * p.dg_sb +
-                                         (size_t)rowc * p.dg_sn + (size_t)h * p.dg_sh
-                                   : nullptr;
-    float dgc0 = 0.f, dgc1 = 0.f, dgc2 = 0.f, dgc3 = 0.f;  // thread r < 32: columns r, 32 + r, 64 + r, 96 + r
-#pragma unroll 2
-    for (int c8 = 0; c8 < 16; ++c8) {
-        float dd[8], gt[8], dgv[8];
+    uint32_t ddw[16], dgw[16];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) dd[e] = gt[e] = dgv[e] = 0.f;
-        if (valid) {
-            float y[8], sg[8];
-            dyn8(c8, y, sg);
+    for (int k = 0; k < 8; ++k) {
+        const float4 g = gain4(8 * q + k);
+        const float av1[4] = {a1[k].x, a1[k].y, a1[k].z, a1[k].w}, av2[4] = {a2[k].x, a2[k].y, a2[k].z, a2[k].w};
+        const float gg[4] = {g.x, g.y, g.z, g.w};
+        float dd[4], dgv[4];
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int c = 2 * c8 + hh;
-                const float4 a1 = a1p[c * BT], a2 = a2p[c * BT], g = gain4(c);
-                const float av1[4] = {a1.x, a1.y, a1.z, a1.w}, av2[4] = {a2.x, a2.y, a2.z, a2.w};
-                const float gg[4] = {g.x, g.y, g.z, g.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int k = 4 * hh + e;
-                    const float d = fmaf(-lam, av2[e], av1[e]);
-                    dd[k] = p.apply_norm ? fmaf(rn * gg[e], y[k], -coef * d) : y[k];
-                    const float ddh = __half2float(__float2half_rn(dd[k]));
-                    delta1 = fmaf(ddh, av1[e], delta1);
-                    dot2h = fmaf(ddh, av2[e], dot2h);
-                    dot2 = fmaf(dd[k], av2[e], dot2);
-                    gt[k] = y[k] * d * rn;
-                    bad |= !(fabsf(dd[k]) <= 65504.0f);
-                    // dG = dY Yn sigma'(G) = dYn Yn (1 - sigma(G)), Yn = D r gain (or D)
-                    const float yn = p.apply_norm ? d * rn * gg[e] : d;
-                    dgv[k] = y[k] * yn * (1.0f - sg[k]);
-                }
-            }
-            *reinterpret_cast<uint4 *>(ddrow + 8 * c8) =
-                make_uint4(pack_half2(dd[0], dd[1]), pack_half2(dd[2], dd[3]), pack_half2(dd[4], dd[5]),
-                           pack_half2(dd[6], dd[7]));
-            if (dgrow)
-                *reinterpret_cast<uint4 *>(dgrow + 8 * c8) =
-                    make_uint4(pack_bf162(dgv[0], dgv[1]), pack_bf162(dgv[2], dgv[3]), pack_bf162(dgv[4], dgv[5]),
-                               pack_bf162(dgv[6], dgv[7]));
+        for (int e = 0; e < 4; ++e) {
+            const int i = 4 * k + e;
+            const float d = fmaf(-lam, av2[e], av1[e]);
+            float sgv;
+            const float yv = dyn(i, sgv);
+            dd[e] = p.apply_norm ? fmaf(rn * gg[e], yv, -coef * d) : yv;
+            const float ddh = __half2float(__float2half_rn(dd[e]));
+            delta1 = fmaf(ddh, av1[e], delta1);
+            dot2h = fmaf(ddh, av2[e], dot2h);
+            dot2 = fmaf(dd[e], av2[e], dot2);
+            if (want_dgain) red[rr * (HDV + 1) + 32 * q + i] = yv * d * rn;
+            bad |= !(fabsf(dd[e]) <= 65504.0f);
+            // dG = dY Yn sigma'(G) = dYn Yn (1 - sigma(G)), Yn = D r gain (or D)
+            const float yn = p.apply_norm ? d * rn * gg[e] : d;
+            dgv[e] = yv * yn * (1.0f - sgv);
         }
-        if (want_dgain) {
-            // This row's terms of columns 8 c8 .. 8 c8 + 7; after every fourth
-            // step the CTA sums the group's 32 columns over its 128 rows (a
-            // quarter of the rows per warp, then the four partials).
+        ddw[2 * k] = pack_half2(dd[0], dd[1]);
+        ddw[2 * k + 1] = pack_half2(dd[2], dd[3]);
+        dgw[2 * k] = pack_bf162(dgv[0], dgv[1]);
+        dgw[2 * k + 1] = pack_bf162(dgv[2], dgv[3]);
+    }
+    delta1 = row_sum(delta1);
+    dot2h = row_sum(dot2h);
+    dot2 = row_sum(dot2);
+    if (valid) {
+        uint4 *ddrow = reinterpret_cast<uint4 *>(static_cast<__half *>(p.dd) +
+                                                 (((size_t)b * p.N + row) * p.H + h) * HDV + 32 * q);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) red[r * 33 + 8 * (c8 & 3) + e] = gt[e];
-            if ((c8 & 3) == 3) {
-                __syncthreads();
-                const int col = r & 31, r0 = (r >> 5) * 32;
-                float v = 0.f;
-#pragma unroll 8
-                for (int i = 0; i < 32; ++i) v += red[(r0 + i) * 33 + col];
-                col_part[r >> 5][col] = v;
-                __syncthreads();
-                if (r < 32) {
-                    const float t = col_part[0][r] + col_part[1][r] + col_part[2][r] + col_part[3][r];
-                    const int grp = c8 >> 2;
-                    dgc0 = grp == 0 ? t : dgc0;
-                    dgc1 = grp == 1 ? t : dgc1;
-                    dgc2 = grp == 2 ? t : dgc2;
-                    dgc3 = grp == 3 ? t : dgc3;
-                }
-            }
+        for (int k = 0; k < 4; ++k) ddrow[k] = make_uint4(ddw[4 * k], ddw[4 * k + 1], ddw[4 * k + 2], ddw[4 * k + 3]);
+        if (p.dgate) {
+            uint4 *dgrow = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.dgate) + (size_t)b * p.dg_sb +
+                                                     (size_t)row * p.dg_sn + (size_t)h * p.dg_sh + 32 * q);
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                dgrow[k] = make_uint4(dgw[4 * k], dgw[4 * k + 1], dgw[4 * k + 2], dgw[4 * k + 3]);
         }
     }
     if (bad) report_error(p.dev_status, DIFFATTN_ERR_UNSUPPORTED);
@@ -418,35 +410,40 @@ __global__ void __launch_bounds__(128)
     // Row statistics, negated (-lse_1, -lse_2, -Delta_1, -Delta_2, -lambda:
     // the tile kernels add them in packed fused multiply-adds); rows past N
     // get zeros (the tile kernels' products see zero operands there).
-    float *st = p.stats + (size_t)(b * p.H + h) * kBwdStats * p.n_pad + row;
-    const float *lse = tile + 2 * BT * HDV;
-    st[0] = valid ? -lse[r] : 0.f;
-    st[p.n_pad] = valid ? -lse[BT + r] : 0.f;
-    st[2 * p.n_pad] = -delta1;
-    st[3 * p.n_pad] = lam * dot2h;
-    st[4 * p.n_pad] = valid ? -lam : 0.f;
+    if (q == 0) {
+        float *st = p.stats + (size_t)(b * p.H + h) * kBwdStats * p.n_pad + qt * BT + r;
+        const float *lse = tile + 2 * BT * HDV;
+        st[0] = valid ? -lse[r] : 0.f;
+        st[p.n_pad] = valid ? -lse[BT + r] : 0.f;
+        st[2 * p.n_pad] = -delta1;
+        st[3 * p.n_pad] = lam * dot2h;
+        st[4 * p.n_pad] = valid ? -lam : 0.f;
+    }
 
     // dlambda_i = -dD . A_2: per token through sigma' with lambda logits,
-    // else summed over the tile's rows into the head's dlambda.
+    // else summed over the CTA's rows into the head's dlambda.
     if (p.lam_logits) {
-        if (p.dlam_logits && valid)
+        if (p.dlam_logits && valid && q == 0)
             p.dlam_logits[b * p.dll_sb + (int64_t)row * p.dll_sn + h * p.dll_sh] = -dot2 * lam * (1.0f - lam);
     } else if (p.dlambda) {
-        float v = -dot2;
+        float v = q == 0 ? -dot2 : 0.f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if ((r & 31) == 0) warp_sum[r >> 5] = v;
+        if ((threadIdx.x & 31) == 0) warp_sum[threadIdx.x >> 5] = v;
     }
     __syncthreads();
-    if (!p.lam_logits && p.dlambda && r == 0)
-        atomicAdd(p.dlambda + h, warp_sum[0] + warp_sum[1] + warp_sum[2] + warp_sum[3]);
-    // dgain[h][c] += the tile's column sums.
-    if (want_dgain && r < 32) {
-        float *dg = p.dgain + (size_t)h * HDV + r;
-        atomicAdd(dg, dgc0);
-        atomicAdd(dg + 32, dgc1);
-        atomicAdd(dg + 64, dgc2);
-        atomicAdd(dg + 96, dgc3);
+    if (!p.lam_logits && p.dlambda && threadIdx.x == 0) {
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < PREP_THREADS / 32; ++w) v += warp_sum[w];
+        atomicAdd(p.dlambda + h, v);
+    }
+    // dgain[h][c] += the CTA's column sums (rows past N hold zeros).
+    if (want_dgain && threadIdx.x < HDV) {
+        float v = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < PREP_ROWS; ++i) v += red[i * (HDV + 1) + threadIdx.x];
+        atomicAdd(p.dgain + (size_t)h * HDV + threadIdx.x, v);
     }
 }
 
@@ -1280,11 +1277,10 @@ cudaError_t launch_bwd(const BwdKeyMaps &km, const BwdQueryMaps &qm, const BwdPa
         set_internal_error("device ordinal beyond the library's table");
         return cudaErrorInvalidDevice;
     }
-    const int red_bytes = BT * 33 * (int)sizeof(float);  // one group of 32 columns
     if (!attr_set[dev].load(std::memory_order_acquire)) {
         std::lock_guard<std::mutex> lock(attr_mutex);  // first calls from several host threads
         if (!attr_set[dev].load(std::memory_order_relaxed)) {
-            e = cudaFuncSetAttribute(bwd_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, red_bytes);
+            e = cudaFuncSetAttribute(bwd_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_RED_BYTES);
             if (e != cudaSuccess) return e;
             for (const void *k : {(const void *)bwd_key_kernel<false>, (const void *)bwd_key_kernel<true>}) {
                 e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)KT_SMEM);
@@ -1300,7 +1296,7 @@ cudaError_t launch_bwd(const BwdKeyMaps &km, const BwdQueryMaps &qm, const BwdPa
     if ((int64_t)p.B * p.H * p.num_qt == 0) return cudaSuccess;
     const bool want_dgain = p.apply_norm && p.dgain;
     const int tiles = p.B * p.H * p.num_qt;  // query tiles, and key tiles alike: ceil(N / 128)
-    bwd_prep_kernel<<<tiles, 128, want_dgain ? red_bytes : 0, stream>>>(p);
+    bwd_prep_kernel<<<tiles * (BT / PREP_ROWS), PREP_THREADS, want_dgain ? PREP_RED_BYTES : 0, stream>>>(p);
     ++*launches;
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
