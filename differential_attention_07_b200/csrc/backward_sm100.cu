@@ -255,17 +255,18 @@ __device__ __forceinline__ void tmem_row64(uint32_t taddr, float (&x)[64])
 
 // ---------------------------------------------------------------- 1. row preparation
 // Four threads per row (thread q of a row takes columns [32 q, 32 q + 32):
-// 8 chunks of 4 fp32 of A_1 and of A_2, 32 of dY), 64 rows per CTA: a
+// 8 chunks of 4 fp32 of A_1 and of A_2, 32 of dY), 16 rows per CTA: a
 // quarter row of A_1, A_2 fits in registers, so both passes (the norm's
 // sums, then dD) read the saved state once; the row sums combine the four
 // quarters with two shuffles.  In a warp, 8 rows x 4 quarters: each load
 // instruction reads 8 consecutive rows of 4 chunks of the chunk-major
-// state, four full 128-byte lines.  Dynamic shared memory [64][129] fp32
+// state, four full 128-byte lines.  Small CTAs (eight per SM) keep loads
+// of some in flight while others reduce.  Dynamic shared memory [16][129] fp32
 // holds the per-row dgain terms when dgain is requested (and the norm
-// applied), summed per column by threads 0-127.
-constexpr int PREP_THREADS = 256, PREP_ROWS = PREP_THREADS / 4;
+// applied), summed per column.
+constexpr int PREP_THREADS = 64, PREP_ROWS = PREP_THREADS / 4;
 constexpr int PREP_RED_BYTES = PREP_ROWS * (HDV + 1) * 4;
-__global__ void __launch_bounds__(PREP_THREADS, 2)
+__global__ void __launch_bounds__(PREP_THREADS, 8)
     bwd_prep_kernel(const BwdParams p)
 {
     extern __shared__ float red[];
@@ -439,11 +440,13 @@ __global__ void __launch_bounds__(PREP_THREADS, 2)
         atomicAdd(p.dlambda + h, v);
     }
     // dgain[h][c] += the CTA's column sums (rows past N hold zeros).
-    if (want_dgain && threadIdx.x < HDV) {
-        float v = 0.f;
+    if (want_dgain) {
+        for (int c = threadIdx.x; c < HDV; c += PREP_THREADS) {
+            float v = 0.f;
 #pragma unroll 8
-        for (int i = 0; i < PREP_ROWS; ++i) v += red[i * (HDV + 1) + threadIdx.x];
-        atomicAdd(p.dgain + (size_t)h * HDV + threadIdx.x, v);
+            for (int i = 0; i < PREP_ROWS; ++i) v += red[i * (HDV + 1) + c];
+            atomicAdd(p.dgain + (size_t)h * HDV + c, v);
+        }
     }
 }
 
