@@ -429,7 +429,7 @@ def run_prefill_workload(w, steps, warmup, device, ops, rank=0, clocks=None, pla
     f = ops.diffattn_grouped_fwd if grouped else ops.diffattn_fwd
     out_full = torch.zeros(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=device)
     out = out_full[plan["b0"]:plan["b1"], :, plan["h0"]:plan["h1"]]
-    ws = torch.empty(max(1, ops.fwd_workspace_size(sw.B, sw.N, sw.H, sw.H_V, sw.H_N, sw.rope_theta)
+    ws = torch.empty(max(1, ops.fwd_workspace_size(sw.B, sw.N, sw.H, sw.H_V, sw.H_N, sw.rope_theta, sw.window)
                          if not empty else 1), dtype=torch.uint8, device=device)
     status = torch.zeros(1, dtype=torch.int32, device=device)
 
@@ -488,7 +488,7 @@ def e2e_prefill(w, steps, warmup, device, ops, x):
     dev = {k: torch.empty_like(v, device=device) for k, v in host.items()}
     out = torch.empty(w.B, w.N, w.H, w.dv, dtype=torch.bfloat16, device=device)
     out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    ws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H, w.H_V, w.H_N, w.rope_theta), dtype=torch.uint8, device=device)
+    ws = torch.empty(ops.fwd_workspace_size(w.B, w.N, w.H, w.H_V, w.H_N, w.rope_theta, w.window), dtype=torch.uint8, device=device)
     f = ops.diffattn_grouped_fwd if w.kind == "grouped" else ops.diffattn_fwd
     s_in, s_c, s_out = (torch.cuda.Stream(device) for _ in range(3))
     per_batch = [k for k in dev if dev[k].dim() == 4]          # [B, N, heads, dim] tensors

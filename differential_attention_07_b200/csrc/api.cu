@@ -123,7 +123,7 @@ bool grouped_pairs(const diffattn_fwd_args *a)
     return g >= 3 && g % 2 == 1;
 }
 
-// Prefill workspace: [fp16 V][256 B work counters][paired grouped heads
+// Prefill workspace: [fp16 V, except under a window][256 B work counters][paired grouped heads
 // only: noise outputs, one fp32 128 x 128 block per (b, noise head, query
 // tile), then one ready count per such tile][rotated Q1, K1, Q2, K2 when
 // rope_theta > 0: contiguous [B, N, heads, 64] fp16 each].
@@ -143,9 +143,12 @@ size_t rope_bytes(const diffattn_fwd_args *a)
     return n;
 }
 
-// Bytes of the fp16 V copy at the start of the prefill workspace.
+// Bytes of the fp16 V copy at the start of the prefill workspace (none
+// under a sliding window, whose kernel reads the caller's V and converts
+// each step itself).
 size_t v16_bytes(const diffattn_fwd_args *a)
 {
+    if (a->window > 0) return 0;
     const int64_t HV = a->H_V ? a->H_V : a->H;
     return align256((size_t)a->B * a->N * HV * 128 * 2);
 }

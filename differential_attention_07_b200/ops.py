@@ -335,11 +335,12 @@ def diffattn_grouped_fwd(q1, q2, k1, k2, v, lam, gain=None, *, scale=0.125, eps=
                     save=save, test_withhold_load=test_withhold_load)
 
 
-def fwd_workspace_size(B, N, H, H_V=None, H_N=None, rope_theta=0.0):
+def fwd_workspace_size(B, N, H, H_V=None, H_N=None, rope_theta=0.0, window=0):
     """Workspace bytes of a prefill call with these sizes."""
     a = FwdArgs()
     a.B, a.N, a.H, a.H_N, a.H_V, a.d, a.dv = B, N, H, H_N or H, H_V or H, 64, 128
     a.rope_theta = float(rope_theta)
+    a.window = int(window)
     return int(lib().diffattn_fwd_workspace_size(ctypes.byref(a)))
 
 

@@ -141,8 +141,9 @@ diffattn_status diffattn_grouped_fwd(const diffattn_fwd_args *args, void *worksp
                                      size_t ws_bytes, void *stream);
 
 /* Bytes of workspace diffattn_fwd / diffattn_grouped_fwd need for `args`
- * (an fp16 copy of V for the tensor-core P.V product, the work counters, and
- * depending on the arguments the grouped heads' noise outputs and the
+ * (an fp16 copy of V for the tensor-core P.V product -- not under a sliding
+ * window, whose kernel converts each V step itself --, the work counters,
+ * and depending on the arguments the grouped heads' noise outputs and the
  * rotated copies of Q1, K1, Q2, K2).                                        */
 size_t diffattn_fwd_workspace_size(const diffattn_fwd_args *args);
 

@@ -132,6 +132,11 @@ def test_fwd_rejects_before_launch(L):
                                                              + 2 * 8 * 3 * 128 * 128 * 4 + 256)
     g = _fake_fwd_args(H=24, H_N=8, H_V=24)
     assert L.diffattn_fwd_workspace_size(ctypes.byref(g)) == 2 * 300 * 24 * 128 * 2 + 256
+    # under a sliding window the kernel reads V itself: no fp16 copy
+    w = _fake_fwd_args()
+    w.window = 128
+    assert L.diffattn_fwd_workspace_size(ctypes.byref(w)) == 256
+    assert ops.fwd_workspace_size(2, 300, 4, window=128) == 256
 
 
 def _fake_decode_args(B=3, H=2, L=1000, base=1 << 20):
