@@ -110,7 +110,7 @@ def decode_bytes(w):
 # prefill_kernel launch on the 4 x 4096 x 16-head workload, from one ncu
 # capture, keyed by a hash of the kernel sources it was taken on.  A kernel
 # whose sources no longer hash to this value reports null traffic.
-PREFILL_TRAFFIC = {"source_sha256_16": "dce10853aab3f22e", "bytes": 268_173_312 + 47_439_872}
+PREFILL_TRAFFIC = {"source_sha256_16": "e4427aace67f1a28", "bytes": 268_173_312 + 47_439_872}
 
 
 def prefill_traffic():

@@ -284,9 +284,6 @@ __device__ __forceinline__ bool wait_flag_geq(const int *flag, int target, volat
 // 790 / 931, 3 of 8 810 / 893, 2 of 8 860 / 909, 1 of 8 861 / 959, none
 // 843 / 996: with the pipeline overlapped, issue slots matter more than
 // MUFU time, so only one pair in eight goes to the FMA pipe.
-// Not under a sliding window, where the V converter shares an SM
-// sub-partition with two softmax warps and the polynomial's extra
-// instructions cost more than the MUFU work they save (measured).
 constexpr uint32_t SOFT_EXP_MASK = 0x20u;  // pair 5 of every 8
 
 // Softmax of one map for one 64-key step, for the query row this thread owns;
@@ -374,7 +371,7 @@ __device__ __forceinline__ bool softmax_step(uint32_t tS, uint32_t tO, bool firs
     for (int i = 0; i < 32; ++i) {
         const int c = i >> 4, e = (2 * i) & 31;
         const float2 x = ffma2(make_float2(__uint_as_float(v[c][e]), __uint_as_float(v[c][e + 1])), sc, nm);
-        const float2 pp = (!WINDOW && ((SOFT_EXP_MASK >> (i & 7)) & 1u))
+        const float2 pp = ((SOFT_EXP_MASK >> (i & 7)) & 1u)
                               ? exp2_soft2(x)
                               : make_float2(ex2_approx(x.x), ex2_approx(x.y));
         acc[i & 3] = fadd2(acc[i & 3], pp);
