@@ -224,8 +224,9 @@ diffattn_status diffattn_bwd(const diffattn_bwd_args *args, void *workspace, siz
                              void *stream);
 
 /* Workspace bytes of diffattn_bwd (fp16 copies of V and of dD, per-row
- * statistics, and depending on the arguments the rotated copies of Q1, K1,
- * Q2, K2 and fp32 sums of the gradients of shared noise and V heads).      */
+ * statistics, the two tile kernels' work counters, and depending on the
+ * arguments the rotated copies of Q1, K1, Q2, K2 and fp32 sums of the
+ * gradients of shared noise and V heads).                                   */
 size_t diffattn_bwd_workspace_size(const diffattn_bwd_args *args);
 
 /* Host-only argument check of a prefill call: the status diffattn_fwd (or,
